@@ -1,0 +1,298 @@
+"""Pins for the float64 oracle: checks against what the pages and the mathematics
+fix, not against the oracle itself.
+
+Each ``pin_*`` takes an implementation namespace ``impl`` exposing
+``rotate``, ``inverse_rotate``, ``awq_pack``, ``awq_unpack``, ``dequant`` and
+``w4_linear_from_codes`` with the oracle's signatures, and raises
+AssertionError when the implementation disagrees.  ``test_oracle_pins.py``
+runs them on the oracle; ``test_oracle_mutations.py`` runs them on copies of
+the oracle with planted mistakes and checks that each mistake is caught.
+
+Sources (GPTQModel wiki page "ParoQuant"):
+  * "Pairwise Givens rotations": a' = a cos t + b sin t, b' = -a sin t + b cos t;
+    stages in order; inverse = reversed order with negated angles; pair
+    indices local to each group.
+  * "Activation and weight transforms": R orthogonal; X_r = X D^-1 R,
+    W_r = W D R, X_r W_r^T = X W^T without quantisation; the equivalent
+    original-domain weight is Q(W_r) R^T D^-1.
+  * "Stored tensors": identity state = zero angles and unit channel scales.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rand_tables(rng, K, G, krot, active=None):
+    pairs = np.empty((krot, K), np.int16)
+    theta = np.zeros((krot, K // 2), np.float64)
+    half = G // 2
+    for s in range(krot):
+        for g in range(K // G):
+            pairs[s, g * G:(g + 1) * G] = rng.permutation(G)
+            n = half if active is None else active
+            sel = rng.choice(half, n, replace=False)
+            theta[s, g * half + sel] = rng.uniform(-np.pi, np.pi, n)
+    return pairs, theta
+
+
+def _givens_matrix_of_stage(pairs_s, theta_s, K, G):
+    """Dense K x K matrix M of one stage in the row-vector convention
+    (x' = x M), written entry by entry from the pair formula:
+        x'_i = c x_i + s x_j   ->  M[i, i] = c,  M[j, i] = s
+        x'_j = -s x_i + c x_j  ->  M[i, j] = -s, M[j, j] = c
+    Built with explicit Python loops over groups and pairs."""
+    M = np.zeros((K, K))
+    for g in range(K // G):
+        for p in range(G // 2):
+            i = g * G + int(pairs_s[g * G + 2 * p])
+            j = g * G + int(pairs_s[g * G + 2 * p + 1])
+            t = float(theta_s[g * (G // 2) + p])
+            c, s = math.cos(t), math.sin(t)
+            M[i, i] = c
+            M[j, i] = s
+            M[i, j] = -s
+            M[j, j] = c
+    return M
+
+
+def dense_R(pairs, theta, K, G):
+    R = np.eye(K)
+    for s in range(pairs.shape[0]):
+        R = R @ _givens_matrix_of_stage(pairs[s], theta[s], K, G)
+    return R
+
+
+# ---------------------------------------------------------------- rotation pins
+
+def pin_single_pair_closed_forms(impl):
+    """t = pi/2: (a,b) -> (b,-a); t = pi: (a,b) -> (-a,-b); t = 0: identity."""
+    K = G = 8
+    pairs = np.array([[3, 5, 0, 1, 2, 4, 6, 7]], np.int16)   # pair 0 = (3, 5)
+    x = np.array([[0.1, -0.2, 0.3, 1.25, 0.5, -0.75, 0.7, 0.9]])
+    for t, (ea, eb) in [(math.pi / 2, (-0.75, -1.25)), (math.pi, (-1.25, 0.75)),
+                        (0.0, (1.25, -0.75))]:
+        theta = np.zeros((1, K // 2))
+        theta[0, 0] = t
+        y = impl.rotate(x, None, pairs, theta, G)
+        assert abs(y[0, 3] - ea) <= 1e-15 and abs(y[0, 5] - eb) <= 1e-15, (t, y[0, 3], y[0, 5])
+        others = [0, 1, 2, 4, 6, 7]
+        assert np.array_equal(y[0, others], x[0, others])
+
+
+def pin_stage_composition(impl):
+    """Two stages with the same pairs and angles t1, t2 equal one stage t1 + t2."""
+    rng = np.random.default_rng(11)
+    K, G = 256, 128
+    p1, t1 = _rand_tables(rng, K, G, 1)
+    t2 = rng.uniform(-np.pi, np.pi, t1.shape)
+    x = rng.standard_normal((5, K))
+    two = impl.rotate(x, None, np.concatenate([p1, p1]), np.concatenate([t1, t2]), G)
+    one = impl.rotate(x, None, p1, t1 + t2, G)
+    assert np.max(np.abs(two - one)) <= 1e-13
+
+
+def pin_inverse_restores(impl):
+    """Reversed stage order with negated angles restores the input (<= 1e-12)."""
+    rng = np.random.default_rng(12)
+    K, G = 512, 128
+    pairs, theta = _rand_tables(rng, K, G, 8)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))
+    x = rng.standard_normal((7, K)) * 3
+    xr = impl.rotate(x, cs, pairs, theta, G)
+    back = impl.inverse_rotate(xr, cs, pairs, theta, G)
+    assert np.max(np.abs(back - x)) <= 1e-12 * max(1.0, np.max(np.abs(x)))
+
+
+def pin_group_norms_preserved(impl):
+    """R is orthogonal and group-local: each group's L2 norm of x*cs is kept."""
+    rng = np.random.default_rng(13)
+    K, G = 384, 128
+    pairs, theta = _rand_tables(rng, K, G, 8)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))
+    x = rng.standard_normal((6, K))
+    xr = impl.rotate(x, cs, pairs, theta, G)
+    n0 = np.linalg.norm((x * cs).reshape(6, K // G, G), axis=2)
+    n1 = np.linalg.norm(xr.reshape(6, K // G, G), axis=2)
+    assert np.max(np.abs(n1 - n0) / n0) <= 1e-12
+
+
+def pin_dense_R_brute_force(impl):
+    """Small K: the stage-by-stage result equals (x * cs) @ R with R the product
+    of dense per-stage Givens matrices built entry by entry."""
+    rng = np.random.default_rng(14)
+    for K, G, krot in [(128, 128, 1), (128, 128, 3), (256, 128, 2), (256, 128, 8), (64, 16, 4)]:
+        pairs, theta = _rand_tables(rng, K, G, krot)
+        cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))
+        x = rng.standard_normal((3, K))
+        ref = (x * cs) @ dense_R(pairs, theta, K, G)
+        got = impl.rotate(x, cs, pairs, theta, G)
+        assert np.max(np.abs(got - ref)) <= 1e-12, (K, G, krot)
+
+
+def pin_golden_g4(impl):
+    g = json.load(open(os.path.join(GOLDEN, "rotation_g4_krot2.json")))
+    theta = np.array([[math.pi / 2, 0.0], [math.pi / 3, math.pi]])
+    got = impl.rotate(np.array(g["x"]), np.array(g["channel_scales"]),
+                      np.array(g["pairs"], np.int16), theta, g["group_size"])
+    assert np.max(np.abs(got - np.array(g["expected"]))) <= 1e-14, got
+
+
+def pin_group_size_minus_one(impl):
+    """group_size=-1 is the whole input width."""
+    rng = np.random.default_rng(15)
+    K = 64
+    pairs, theta = _rand_tables(rng, K, K, 2)
+    x = rng.standard_normal((2, K))
+    a = impl.rotate(x, None, pairs, theta, -1)
+    b = x @ dense_R(pairs, theta, K, K)
+    assert np.max(np.abs(a - b)) <= 1e-12
+
+
+def pin_unquantized_identity(impl):
+    """X_r W_r^T = X W^T with W_r = W D R (rows of W rotated like activations
+    but scaled by D = 1/channel_scales)."""
+    rng = np.random.default_rng(16)
+    K, G, N, M = 512, 128, 48, 9
+    pairs, theta = _rand_tables(rng, K, G, 8)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))      # D^-1
+    x = rng.standard_normal((M, K))
+    W = rng.standard_normal((N, K))
+    xr = impl.rotate(x, cs, pairs, theta, G)
+    wr = impl.rotate(W, 1.0 / cs, pairs, theta, G)
+    lhs = xr @ wr.T
+    rhs = x @ W.T
+    assert np.max(np.abs(lhs - rhs)) <= 1e-10 * np.max(np.abs(rhs))
+
+
+# ------------------------------------------------------------- packing pins
+
+def pin_awq_golden_word(impl):
+    g = json.load(open(os.path.join(GOLDEN, "awq_word.json")))
+    codes = np.zeros((8, 128), np.uint8)
+    codes[:, 0] = g["codes_of_columns_0_to_7"]
+    qw, _ = impl.awq_pack(codes, np.zeros((8, 1), np.uint8), 128)
+    assert int(np.uint32(qw.view(np.uint32)[0, 0])) == int(g["word_hex"], 16), hex(int(qw.view(np.uint32)[0, 0]))
+
+
+def pin_awq_one_hot(impl):
+    """A single code 15 at (n, k) lands in word (k, n//8) at nibble position
+    pos[n % 8], pos = [0,4,1,5,2,6,3,7]; every other nibble is 0."""
+    g = json.load(open(os.path.join(GOLDEN, "awq_word.json")))
+    pos = g["nibble_position_of_column"]
+    N, K, G = 24, 256, 128
+    for n in range(N):
+        for k in (0, 1, 127, 128, 255):
+            codes = np.zeros((N, K), np.uint8)
+            codes[n, k] = 15
+            zeros = np.zeros((N, K // G), np.uint8)
+            zeros[n, k // G] = 9
+            qw, qz = impl.awq_pack(codes, zeros, G)
+            u = qw.view(np.uint32)
+            assert u[k, n // 8] == np.uint32(15 << (4 * pos[n % 8]))
+            assert np.count_nonzero(u) == 1
+            uz = qz.view(np.uint32)
+            assert uz[k // G, n // 8] == np.uint32(9 << (4 * pos[n % 8]))
+            assert np.count_nonzero(uz) == 1
+
+
+def pin_awq_round_trip(impl):
+    rng = np.random.default_rng(17)
+    N, K, G = 64, 512, 128
+    codes = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    zeros = rng.integers(0, 16, (N, K // G), dtype=np.uint8)
+    qw, qz = impl.awq_pack(codes, zeros, G)
+    assert qw.dtype == np.int32 and qw.shape == (K, N // 8) and qz.shape == (K // G, N // 8)
+    c2, z2 = impl.awq_unpack(qw, qz, N, K, G)
+    assert np.array_equal(c2, codes) and np.array_equal(z2, zeros)
+
+
+# ---------------------------------------------------------- dequant + linear pins
+
+def _brute_linear(x, codes, zeros, scales, bias, G):
+    """Y[m, n] = sum_k x[m, k] * (codes[n, k] - zeros[n, k//G]) * scales[k//G, n] + bias[n],
+    one output at a time."""
+    M, K = x.shape
+    N = codes.shape[0]
+    Y = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += float(x[m, k]) * (int(codes[n, k]) - int(zeros[n, k // G])) * float(scales[k // G, n])
+            Y[m, n] = acc + (0.0 if bias is None else float(bias[n]))
+    return Y
+
+
+def pin_identity_state_is_plain_w4(impl):
+    """Zero angles and unit channel scales reduce the layer to a plain W4
+    dequant-matmul, checked one output at a time."""
+    rng = np.random.default_rng(18)
+    M, K, N, G = 2, 256, 16, 128
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    codes = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    zeros = rng.integers(0, 16, (N, K // G), dtype=np.uint8)
+    scales = rng.uniform(0.005, 0.02, (K // G, N)).astype(np.float16)
+    bias = rng.standard_normal(N).astype(np.float16)
+    pairs, _ = _rand_tables(rng, K, G, 8)
+    theta = np.zeros((8, K // 2))
+    ref = _brute_linear(x, codes, zeros, scales, bias, G)
+    got = impl.w4_linear_from_codes(x, codes, zeros, scales, bias, np.ones(K), pairs, theta, G, 8)
+    assert np.max(np.abs(got - ref)) <= 1e-10 * np.max(np.abs(ref))
+    got0 = impl.w4_linear_from_codes(x, codes, zeros, scales, bias, None, None, None, G, 0)
+    assert np.max(np.abs(got0 - ref)) <= 1e-10 * np.max(np.abs(ref))
+
+
+def pin_equivalent_weight_route(impl):
+    """Y = X_r Q(W_r)^T + b equals X (Q(W_r) R^T D^-1)^T + b (equivalent
+    original-domain weight)."""
+    rng = np.random.default_rng(19)
+    M, K, N, G = 3, 256, 24, 128
+    x = rng.standard_normal((M, K))
+    pairs, theta = _rand_tables(rng, K, G, 8)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))       # D^-1
+    codes = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    zeros = rng.integers(0, 16, (N, K // G), dtype=np.uint8)
+    scales = rng.uniform(0.005, 0.02, (K // G, N))
+    bias = rng.standard_normal(N)
+    Wq = np.empty((N, K))                                       # Q(W_r), out x in
+    for n in range(N):
+        for k in range(K):
+            Wq[n, k] = (int(codes[n, k]) - int(zeros[n, k // G])) * scales[k // G, n]
+    R = dense_R(pairs, theta, K, G)
+    W_eq = Wq @ R.T @ np.diag(cs)
+    ref = x @ W_eq.T + bias
+    got = impl.w4_linear_from_codes(x, codes, zeros, scales, bias, cs, pairs, theta, G, 8)
+    assert np.max(np.abs(got - ref)) <= 1e-10 * np.max(np.abs(ref))
+
+
+def pin_dequant_formula(impl):
+    """(q - z) * s on single elements, one group boundary crossed."""
+    N, K, G = 8, 256, 128
+    codes = np.zeros((N, K), np.uint8)
+    zeros = np.full((N, K // G), 8, np.uint8)
+    scales = np.ones((K // G, N))
+    codes[3, 5] = 15
+    codes[6, 200] = 0
+    zeros[6, 1] = 3
+    scales[1, 6] = 0.5
+    W = impl.dequant(codes, zeros, scales, G)
+    assert W.shape == (K, N)
+    assert W[5, 3] == 7.0
+    assert W[200, 6] == -1.5
+    assert W[0, 0] == -8.0
+    assert W[130, 6] == -1.5
+
+
+ALL_PINS = [
+    pin_single_pair_closed_forms, pin_stage_composition, pin_inverse_restores,
+    pin_group_norms_preserved, pin_dense_R_brute_force, pin_golden_g4,
+    pin_group_size_minus_one, pin_unquantized_identity, pin_awq_golden_word,
+    pin_awq_one_hot, pin_awq_round_trip, pin_identity_state_is_plain_w4,
+    pin_equivalent_weight_route, pin_dequant_formula,
+]

@@ -1,0 +1,125 @@
+"""Planted mistakes: copies of the oracle with one plausible bug each must fail
+at least one pin.  This shows the pins can tell a right oracle from a wrong one.
+(All on the CPU; nothing here touches a GPU.)"""
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+ORDER_OK = (0, 2, 4, 6, 1, 3, 5, 7)
+
+
+def make_impl(sign_flip=False, reverse_stages=False, swap_roles=False, no_scale=False,
+              theta_global=False, order=ORDER_OK, no_zero=False, group0_scale=False,
+              inverse_forward_order=False, shared_group_base=False):
+    def stage_idx(pairs_s, G):
+        K = pairs_s.shape[0]
+        local = pairs_s.astype(np.int64)
+        base = 0 if shared_group_base else (np.arange(K // 2) // (G // 2)) * G
+        i, j = local[0::2] + base, local[1::2] + base
+        return (j, i) if swap_roles else (i, j)
+
+    def apply_stage(X, pairs_s, theta_s, G, sgn=1.0):
+        i, j = stage_idx(pairs_s, G)
+        t = sgn * np.asarray(theta_s, np.float64)
+        if theta_global:
+            t = t[::-1]
+        c, s = np.cos(t), np.sin(t)
+        a, b = X[:, i].copy(), X[:, j].copy()
+        X[:, i] = a * c + b * s
+        X[:, j] = (a * s if sign_flip else -a * s) + b * c
+
+    def rotate(x, cs, pairs, theta, group_size, krot=None):
+        X = np.array(x, np.float64)
+        G = oracle.normalize_group_size(group_size, X.shape[1])
+        if cs is not None and not no_scale:
+            X *= np.asarray(cs, np.float64)
+        if krot is None:
+            krot = 0 if pairs is None else pairs.shape[0]
+        order = reversed(range(krot)) if reverse_stages else range(krot)
+        for s in order:
+            apply_stage(X, pairs[s], theta[s], G)
+        return X
+
+    def inverse_rotate(xr, cs, pairs, theta, group_size):
+        X = np.array(xr, np.float64)
+        G = oracle.normalize_group_size(group_size, X.shape[1])
+        order = range(pairs.shape[0]) if inverse_forward_order else reversed(range(pairs.shape[0]))
+        for s in order:
+            apply_stage(X, pairs[s], theta[s], G, sgn=-1.0)
+        if cs is not None and not no_scale:
+            X /= np.asarray(cs, np.float64)
+        return X
+
+    def awq_pack(codes, zeros, G):
+        N = codes.shape[0]
+
+        def pk(c):
+            w = np.zeros((c.shape[1], N // 8), np.uint64)
+            for t in range(8):
+                w |= c.T.astype(np.uint64)[:, order[t]::8] << np.uint64(4 * t)
+            return w.astype(np.uint32).view(np.int32)
+        return pk(codes), pk(zeros)
+
+    def awq_unpack(qw, qz, N, K, G):
+        def up(words):
+            w = np.asarray(words).view(np.uint32).astype(np.uint64)
+            out = np.zeros((w.shape[0], N), np.uint8)
+            for t in range(8):
+                out[:, order[t]::8] = ((w >> np.uint64(4 * t)) & np.uint64(15)).astype(np.uint8)
+            return out.T.copy()
+        return up(qw), up(qz)
+
+    def dequant(codes, zeros, scales, G):
+        q = codes.T.astype(np.float64)
+        z = np.repeat(zeros.T.astype(np.float64), G, axis=0)
+        s = np.repeat(np.asarray(scales, np.float64), G, axis=0)
+        if group0_scale:
+            s = np.repeat(np.asarray(scales, np.float64)[:1], q.shape[0], axis=0)
+        return (q if no_zero else q - z) * s
+
+    def w4_linear_from_codes(x, codes, zeros, scales, bias, cs, pairs, theta, G, krot):
+        Y = rotate(x, cs, pairs, theta, G, krot=krot) @ dequant(codes, zeros, scales, G)
+        if bias is not None:
+            Y += np.asarray(bias, np.float64)
+        return Y
+
+    return types.SimpleNamespace(rotate=rotate, inverse_rotate=inverse_rotate, awq_pack=awq_pack,
+                                 awq_unpack=awq_unpack, dequant=dequant,
+                                 w4_linear_from_codes=w4_linear_from_codes)
+
+
+def failing_pins(impl):
+    bad = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(impl)
+        except (AssertionError, IndexError, ValueError):
+            bad.append(pin.__name__)
+    return bad
+
+
+def test_unmutated_copy_passes_all_pins():
+    assert failing_pins(make_impl()) == []
+
+
+MUTATIONS = {
+    "sign_flip": dict(sign_flip=True),
+    "reverse_stages": dict(reverse_stages=True),
+    "swap_pair_roles": dict(swap_roles=True),
+    "dropped_channel_scale": dict(no_scale=True),
+    "theta_misindexed": dict(theta_global=True),
+    "identity_nibble_order": dict(order=tuple(range(8))),
+    "dropped_zero_point": dict(no_zero=True),
+    "scale_group_misindexed": dict(group0_scale=True),
+    "inverse_not_reversed": dict(inverse_forward_order=True),
+    "pairs_not_group_local": dict(shared_group_base=True),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTATIONS))
+def test_planted_mistake_is_caught(name):
+    assert failing_pins(make_impl(**MUTATIONS[name])), name
