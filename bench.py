@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the rotated W4 linear (decode HBM GB/s / prefill TFLOP/s).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload q_proj_decode|mlp_decode|
+                 prefill|layer_decode|layer_prefill] [--impl ours|reference]
+
+One "step" is one pass of the whole hot path (scale + Givens stages + W4
+dequant-GEMM) over every call of the workload:
+  q_proj_decode (default): Llama-3-8B q_proj 4096->4096, M = 1, 4, 16 (three calls)
+  mlp_decode:    gate/up 4096->14336 and down 14336->4096, M = 1 and 8 (six calls)
+  prefill:       gate_proj-shaped 4096->14336, M = 2048 and 8192, bias (two calls)
+  layer_decode / layer_prefill: the seven linears of a decoder layer at M = 1 / 4096
+Inputs are seeded synthetic layers (the workload recipe), resident in HBM; the
+weights are cycled over enough replicas that every timed call reads its weights
+from HBM, not L2.  Prints ONE JSON line on rank 0.
+
+--impl reference times the float64 CPU oracle (the reference arm) on bounded
+samples of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+GROUP = 128
+KROT = 8
+
+WORKLOADS = {
+    "q_proj_decode": dict(cfg=1, layers=[0], Ms=[1, 4, 16], kind="decode"),
+    "mlp_decode": dict(cfg=2, layers=[0, 1, 2], Ms=[1, 8], kind="decode"),
+    "prefill": dict(cfg=3, layers=[0], Ms=[2048, 8192], kind="prefill"),
+    "layer_decode": dict(cfg=4, layers=list(range(7)), Ms=[1], kind="decode"),
+    "layer_prefill": dict(cfg=4, layers=list(range(7)), Ms=[4096], kind="prefill"),
+}
+
+
+# ----------------------------------------------------------------- algorithmic cost model
+def call_bytes(K, N, M, bias, krot=KROT, rotated=True):
+    """Bytes the method itself must move for one call (weights, scales, zeros,
+    activations in and out, bias, rotation tables)."""
+    b = K * N // 2 + (K // GROUP) * N * 2 + (K // GROUP) * N // 2 + M * K * 2 + M * N * 2
+    if bias:
+        b += N * 2
+    if rotated:
+        b += krot * K * 2 + krot * (K // 2) * 4 + K * 4
+    return b
+
+
+def gemv_bytes(K, N, M, bias):
+    """Bytes of the GEMV kernel alone (reads X_r instead of x; no tables)."""
+    return call_bytes(K, N, M, bias, rotated=False)
+
+
+def call_flops(K, N, M):
+    return 2 * M * N * K
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def source_digest():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "rotation_w4_weight_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)
+        e = t.get(kernel_key)
+        if e and e.get("src") == source_digest():
+            return e.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a window."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import rotation_w4_weight_b200 as pb
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    layers = [synth.config_layers(wl["cfg"])[i] for i in wl["layers"]]
+    Ms = wl["Ms"]
+    decode = wl["kind"] == "decode"
+
+    def T(a):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    # one packed copy of each layer, then device replicas so the timed calls stream from HBM
+    base = []
+    for lay in layers:
+        qw, qz = pb.pack_awq(T(lay.codes), T(lay.zero_codes), GROUP)
+        base.append(dict(lay=lay, qweight=qw, qzeros=qz, scales=T(lay.scales), bias=T(lay.bias),
+                         cs=T(lay.channel_scales), pairs=T(lay.pairs), theta=T(lay.theta)))
+    weight_bytes = sum(l.K * l.N // 2 + (l.K // GROUP) * l.N * 5 // 2 for l in layers)
+    reps = max(1, min(64, -(-3 * L2_BYTES // weight_bytes)))
+    replicas = []
+    for r in range(reps):
+        replicas.append([{k: (v.clone() if torch.is_tensor(v) and k in ("qweight", "qzeros", "scales") else v)
+                          for k, v in b.items()} for b in base])
+    calls = [(li, M) for li in range(len(layers)) for M in Ms]
+    xs = {(li, M): T(synth.make_activations(layers[li], M)) for li, M in calls}
+    ys = {(li, M): torch.empty((M, layers[li].N), dtype=torch.float16, device=dev) for li, M in calls}
+    ws = {(li, M): torch.empty(max(256, pb.w4_linear_workspace_size(M, layers[li].K, layers[li].N)),
+                               dtype=torch.uint8, device=dev) for li, M in calls}
+    xrs = {(li, M): torch.empty((M, layers[li].K), dtype=torch.float16, device=dev) for li, M in calls}
+
+    stream = torch.cuda.Stream(device=dev)
+    step_bytes = sum(call_bytes(layers[li].K, layers[li].N, M, layers[li].bias is not None)
+                     for li, M in calls)
+    step_flops = sum(call_flops(layers[li].K, layers[li].N, M) for li, M in calls)
+
+    def one_call(rep, li, M):
+        b = replicas[rep][li]
+        pb.w4_linear(xs[(li, M)], b["qweight"], b["qzeros"], b["scales"], b["bias"], b["cs"],
+                     b["pairs"], b["theta"], GROUP, KROT, workspace=ws[(li, M)], out=ys[(li, M)],
+                     stream=stream)
+
+    def one_step(i):
+        for c, (li, M) in enumerate(calls):
+            one_call((i * len(calls) + c) % reps, li, M)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            one_step(i)
+    torch.cuda.synchronize(dev)
+    assert pb.device_status() == pb.PARO_OK
+
+    # capture the K timed steps as one CUDA graph (launch-bound decode calls)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(args.steps):
+            one_step(args.warmup + i)
+    def replay(graph):
+        with torch.cuda.stream(stream):          # a graph replays on the current stream
+            graph.replay()
+
+    replay(g)                                    # untimed graph warm-up
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    t_end = time.time() + 0.6
+    while time.time() < t_end:                   # load before the window so clocks settle
+        replay(g)
+        torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    replay(g)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1)
+    t_end = time.time() + 0.4
+    while time.time() < t_end:
+        replay(g)
+        torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    assert pb.device_status() == pb.PARO_OK
+
+    # ---- dominant kernel, timed live: X_r is produced once per call shape by
+    #      paro_rotate (outside the timed graph); the graph holds the GEMV/GEMM
+    #      launches alone, exactly as paro_w4_linear issues them after rotating.
+    for li, M in calls:
+        b = replicas[0][li]
+        pb.rotate(xs[(li, M)], b["cs"], b["pairs"], b["theta"], GROUP, KROT, out=xrs[(li, M)],
+                  stream=stream)
+    kern_bytes = 0
+    kern_flops = 0
+    n_launch = 0
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        for i in range(args.steps):
+            for c, (li, M) in enumerate(calls):
+                b = replicas[(i * len(calls) + c) % reps][li]
+                pb.w4_linear(xrs[(li, M)], b["qweight"], b["qzeros"], b["scales"], b["bias"],
+                             None, None, None, GROUP, 0, out=ys[(li, M)], stream=stream)
+                lay = layers[li]
+                kern_bytes += gemv_bytes(lay.K, lay.N, M, lay.bias is not None)
+                kern_flops += call_flops(lay.K, lay.N, M)
+                n_launch += 1
+    replay(g2)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    replay(g2)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    kern_ms = e0.elapsed_time(e1)
+    peaks = load_peaks()
+    if decode:
+        achieved = kern_bytes / (kern_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
+                "traffic": traffic_for("w4_mma_decode"),
+                "kernel": "w4_mma_kernel (decode GEMV, split-K cluster)",
+                "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
+                "bytes_per_launch": kern_bytes // n_launch, "peak_source": peaks["src"]}
+    else:
+        achieved = kern_flops / (kern_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
+                "traffic": traffic_for("w4_prefill"),
+                "kernel": "prefill W4 GEMM", "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
+                "flops_per_launch": kern_flops // n_launch,
+                "peak_source": peaks["src"] + " bf16 burst (fp16 runs at the bf16 rate)"}
+    del g2
+
+    # ---- end to end through the public call with host buffers (pinned), per step:
+    #      H2D of the step's activations, the calls, D2H of the outputs
+    hx = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in ys.items()}
+    h2d = sum(v.numel() * 2 for v in hx.values())
+    d2h = sum(v.numel() * 2 for v in hy.values())
+    e_steps = max(1, min(args.steps, 200))
+
+    def e2e_step(i):
+        for c, (li, M) in enumerate(calls):
+            xs[(li, M)].copy_(hx[(li, M)], non_blocking=True)
+            one_call((i * len(calls) + c) % reps, li, M)
+            hy[(li, M)].copy_(ys[(li, M)], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            e2e_step(i)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for i in range(e_steps):
+            e2e_step(i)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+
+    if decode:
+        value = world * args.steps * step_bytes / (ms * 1e-3) / 1e9
+        unit = "GB/s"
+        e2e_val = step_bytes / (e2e_ms * 1e-3) / 1e9 * world
+        metric = f"rotated W4 linear decode HBM throughput ({args.workload})"
+    else:
+        value = world * args.steps * step_flops / (ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        e2e_val = step_flops / (e2e_ms * 1e-3) / 1e12 * world
+        metric = f"rotated W4 linear prefill tensor throughput ({args.workload})"
+
+    out = {
+        "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "layers": [(l.name, l.K, l.N) for l in layers],
+                   "M": Ms, "group_size": GROUP, "krot": KROT, "accumulate": "f32",
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"weights cycled over {reps} device replicas "
+                         f"({reps * weight_bytes / 2**20:.0f} MiB > 3x L2)",
+                   "timing": "CUDA graph of the K steps, CUDA events, max over ranks"},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_val, 2), "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+                "how": "pinned host x -> device, paro_w4_linear calls, device y -> pinned host; no graph"},
+        "gpu_launches": 2 * len(calls) * args.steps,
+        "clocks": clocks,
+        "bytes_per_step": step_bytes, "flops_per_step": step_flops,
+    }
+    return out
+
+
+# ----------------------------------------------------------------- CPU oracle (baseline / reference)
+def oracle_sample(workload, budget_s, max_steps=None):
+    """Times the float64 oracle on column samples of the workload's calls until
+    `budget_s` seconds of CPU work (or max_steps samples) are done.  Returns
+    (value in the workload's unit, description, seconds)."""
+    import oracle
+    wl = WORKLOADS[workload]
+    layers = [synth.config_layers(wl["cfg"])[i] for i in wl["layers"]]
+    decode = wl["kind"] == "decode"
+    rng = np.random.default_rng(0)
+    done_bytes = done_flops = 0.0
+    t_total = 0.0
+    n = 0
+    ncols = 512 if decode else 64
+    while True:
+        for lay in layers:
+            for M in wl["Ms"]:
+                x = synth.make_activations(lay, M)
+                cols = np.sort(rng.choice(lay.N, min(ncols, lay.N), replace=False))
+                t0 = time.perf_counter()
+                oracle.w4_linear_columns(x, lay.codes, lay.zero_codes, lay.scales, lay.bias,
+                                         lay.channel_scales, lay.pairs, lay.theta, GROUP, KROT, cols)
+                t_total += time.perf_counter() - t0
+                frac = len(cols) / lay.N
+                done_bytes += call_bytes(lay.K, lay.N, M, lay.bias is not None) * frac
+                done_flops += call_flops(lay.K, lay.N, M) * frac
+                n += 1
+                if t_total >= budget_s or (max_steps and n >= max_steps):
+                    val = (done_bytes / t_total / 1e9) if decode else (done_flops / t_total / 1e12)
+                    desc = (f"float64 oracle on {n} calls of {workload} restricted to {ncols} "
+                            f"sampled output columns each (full rotation per call)")
+                    return val, desc, t_total
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = WORKLOADS[args.workload]
+    decode = wl["kind"] == "decode"
+    cores = len(os.sched_getaffinity(0))
+    per_step_budget = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
+    oracle_sample(args.workload, per_step_budget * args.warmup, max_steps=args.warmup)
+    val, desc, secs = oracle_sample(args.workload, per_step_budget * args.steps,
+                                    max_steps=max(1, args.steps))
+    unit = "GB/s" if decode else "TFLOP/s"
+    return {
+        "impl": "reference", "metric": ("rotated W4 linear decode HBM throughput" if decode else
+                                        "rotated W4 linear prefill tensor throughput") + f" ({args.workload})",
+        "value": round(val, 5), "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(secs * 1e3 / max(1, args.steps), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "M": wl["Ms"]},
+        "cpu_baseline": {"value": round(val, 5), "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(val, 5), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="q_proj_decode")
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle CPU work for the cpu_baseline field")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        val, desc, _ = oracle_sample(args.workload, args.cpu_budget)
+        out["cpu_baseline"] = {"value": round(val, 5), "unit": out["unit"],
+                               "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+                               "sample": desc}
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

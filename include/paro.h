@@ -1,0 +1,167 @@
+/*
+ * paro.h — C ABI of the B200 (sm_100a) library for ParoQuant's packed-inference
+ * hot path: the scaled, pairwise-rotated INT4 linear layer.
+ *
+ * What the layer computes (GPTQModel wiki page "ParoQuant"):
+ *   1. x <- x * channel_scales, per input channel; channel_scales is the saved
+ *      runtime multiplier D^-1 (section "Activation and weight transforms").
+ *   2. krot stages, in order, of disjoint Givens pair rotations inside every
+ *      group of G input channels.  For a pair (a, b) with angle t:
+ *          a' = a cos t + b sin t,   b' = -a sin t + b cos t
+ *      (section "Pairwise Givens rotations").  Pair indices are local to the
+ *      group; dummy pairs carry t = 0.
+ *   3. Y = X_r . Q(W_r)^T + b against AWQ-packed int4 weights with group-wise
+ *      scales and zero points (sections "Activation and weight transforms",
+ *      "Stored tensors", "Triton plans and tuning": unpack INT4, subtract the
+ *      zero point, multiply by the group scale, accumulate in fp32).
+ *
+ * Tensor layouts (section "Stored tensors"; I = K = in_features,
+ * O = N = out_features, G = group size, all row-major, all little-endian):
+ *   x, x_r          fp16    [M, K]
+ *   channel_scales  fp32    [K]              (may be NULL: all ones)
+ *   pairs           int16   [krot, K]        pairs[s, g*G+2p], pairs[s, g*G+2p+1]
+ *                                            are the local channels (a, b) of pair p
+ *                                            of stage s in group g, each in 0..G-1
+ *   theta           fp32    [krot, K/2]      theta[s, g*G/2+p] is the angle of that pair
+ *   qweight         int32   [K, N/8]         AWQ layout: nibble t (bits 4t..4t+3) of
+ *                                            word w in row k holds column 8w+ORDER[t],
+ *                                            ORDER = {0,2,4,6,1,3,5,7}
+ *   qzeros          int32   [K/G, N/8]       same packing, 4-bit zero points
+ *   scales          fp16    [K/G, N]
+ *   bias            fp16    [N]              (may be NULL)
+ *   y               fp16    [M, N]
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, except the
+ *     host-side helper paro_validate_pairs.  The library allocates nothing;
+ *     scratch memory is a caller-provided workspace sized by the query function.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
+ *     return once the work is enqueued.  Inputs are never modified (except
+ *     x in paro_rotate when x_r == x).  Outputs must not alias inputs otherwise.
+ *   - Return value: PARO_OK, or a status found on the host before any launch
+ *     (invalid shape or pointer, unsupported configuration, misalignment, small
+ *     workspace), or PARO_ERR_CUDA if a launch failed.  Nothing is thrown or
+ *     aborted across the ABI and nothing falls back to the CPU.
+ *   - Kernels that wait on an mbarrier bound the wait; a wait that runs out sets
+ *     a device status word that paro_device_status() reports as PARO_ERR_TIMEOUT.
+ *   - Supported now: G == 128 (group_size == -1 is accepted when K == 128),
+ *     0 <= krot <= 64, K a multiple of 128, N a multiple of 32 (the packer alone
+ *     needs only N % 8 == 0), fp16 activations/scales/bias.
+ */
+#ifndef PARO_H_
+#define PARO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* paro_stream_t;
+
+typedef enum {
+  PARO_OK = 0,
+  PARO_ERR_INVALID_ARG = 1,  /* NULL pointer where data is needed, negative size, bad shape */
+  PARO_ERR_UNSUPPORTED = 2,  /* valid per the method but not implemented (G != 128, ...) */
+  PARO_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned (4-byte for fp32/int16 tables) */
+  PARO_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than paro_w4_linear_workspace_size */
+  PARO_ERR_CUDA = 5,         /* a CUDA launch or query failed */
+  PARO_ERR_TIMEOUT = 6       /* a device-side wait ran out (see paro_device_status) */
+} paro_status;
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char* paro_status_string(int status);
+
+/* Library version as "major.minor.patch". */
+const char* paro_version(void);
+
+/*
+ * paro_rotate — X_r = rotate(x * channel_scales).
+ * Defined by the page's "Pairwise Givens rotations" (pair formula, stage order,
+ * group-local indices) and "Activation and weight transforms" (X_r = X D^-1 R).
+ *   x, x_r          device fp16 [M, K], 16-byte aligned; x_r may equal x (in place)
+ *   M >= 0 rows (M == 0 is a no-op), K > 0 channels, K % group_size == 0
+ *   channel_scales  device fp32 [K] or NULL (no scaling)
+ *   pairs, theta    device tables as above; may be NULL only when krot == 0
+ *   group_size      128, or -1 meaning K (then K must be 128)
+ *   krot            number of stages, 0..64 (0 = scaling only)
+ * Arithmetic: fp32 on chip, cos/sin from sincosf of the fp32 angle, one
+ * round-to-nearest to fp16 at the end.  Pair indices outside 0..G-1 are
+ * masked to 7 bits (so no access leaves the group) and flagged in the device
+ * status word; pair tables are not otherwise checked (see paro_validate_pairs).
+ */
+int paro_rotate(const void* x, void* x_r, int64_t M, int64_t K, const float* channel_scales,
+                const int16_t* pairs, const float* theta, int group_size, int krot,
+                paro_stream_t stream);
+
+/*
+ * paro_pack_awq — pack 4-bit codes into AWQ int32 words (page "ParoQuant",
+ * "Stored tensors": qweight (I, O//8), qzeros (I//G, O//8); packer needs O % 8 == 0).
+ *   codes       device uint8 [N, K]    (out x in), values 0..15 (the high nibble is ignored)
+ *   zero_codes  device uint8 [N, K/G]  values 0..15 (high nibble ignored); may be NULL
+ *               together with qzeros == NULL to pack weights only
+ *   qweight     device int32 [K, N/8]; qzeros device int32 [K/G, N/8]
+ *   N % 8 == 0, K % G == 0, G even (any even G and any K is accepted here)
+ * Bit-exact; the inverse is paro_unpack_awq.
+ */
+int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qweight,
+                  int32_t* qzeros, int64_t N, int64_t K, int group_size, paro_stream_t stream);
+
+/* paro_unpack_awq — exact inverse of paro_pack_awq (same shapes, same rules). */
+int paro_unpack_awq(const int32_t* qweight, const int32_t* qzeros, uint8_t* codes,
+                    uint8_t* zero_codes, int64_t N, int64_t K, int group_size,
+                    paro_stream_t stream);
+
+/*
+ * paro_w4_linear_workspace_size — bytes of device workspace paro_w4_linear
+ * needs for this shape (0 is possible).  Depends only on (M, K, N, group_size).
+ * Returns 0 for shapes paro_w4_linear would reject.
+ */
+size_t paro_w4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int group_size);
+
+/*
+ * paro_w4_linear — Y[M, N] = rotate(x * channel_scales) . dequant(qweight, qzeros, scales) + bias
+ * with dequant(q, z, s)[k, n] = (q[k, n] - z[k/G, n]) * s[k/G, n]
+ * (page "ParoQuant": "Activation and weight transforms" Y = X_r Q(W_r)^T + b;
+ * "Triton plans and tuning" for the group-wise dequantisation with fp32 accumulation).
+ *   krot == 0 skips the stages (pairs/theta ignored); channel_scales == NULL skips the
+ *   scaling; both together give a plain AWQ W4 linear (the baseline of the
+ *   rotation-overhead measurement).  bias may be NULL.
+ *   x fp16 [M, K], y fp16 [M, N]: 16-byte aligned.  qweight, qzeros, scales:
+ *   16-byte aligned.  workspace: device memory of at least
+ *   paro_w4_linear_workspace_size(M, K, N, group_size) bytes, 256-byte aligned,
+ *   contents need no initialisation and are clobbered; one workspace must not be
+ *   used by two calls that can run at the same time.
+ *   Arithmetic: rotation in fp32 rounded once to fp16; weights (q - z) exact in
+ *   fp16; products and sums in fp32 (tensor cores); y rounded once to fp16.
+ *   M <= 16 runs the decode GEMV path; larger M the tcgen05 prefill GEMM path.
+ */
+int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                   const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                   const void* bias, const float* channel_scales, const int16_t* pairs,
+                   const float* theta, int group_size, int krot, void* workspace,
+                   size_t workspace_bytes, paro_stream_t stream);
+
+/*
+ * paro_validate_pairs — HOST helper (host pointer, synchronous, no GPU work):
+ * checks that every stage of every group of a [krot, K] pair table is a
+ * permutation of 0..G-1 (each channel in exactly one pair; cf. the page's
+ * "validated local pair permutations").  Returns PARO_OK or PARO_ERR_INVALID_ARG.
+ */
+int paro_validate_pairs(const int16_t* pairs_host, int64_t K, int group_size, int krot);
+
+/*
+ * paro_device_status — reads (and, if clear != 0, resets) the device status word
+ * of the current device.  Synchronises the device.  Returns PARO_OK,
+ * PARO_ERR_TIMEOUT (a bounded wait ran out), PARO_ERR_INVALID_ARG (a pair index
+ * outside its group was seen) or PARO_ERR_CUDA.
+ */
+int paro_device_status(int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARO_H_ */

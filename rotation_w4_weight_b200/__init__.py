@@ -1,0 +1,149 @@
+"""B200 (sm_100a) library for ParoQuant's scaled pairwise-rotated INT4 linear layer.
+
+The compute lives in the CUDA library ``libparo_b200.so`` behind the C ABI of
+``include/paro.h``; this module only marshals torch tensors (device memory and
+streams) into that ABI.  Functions mirror the C entry points:
+
+    rotate            -> paro_rotate
+    pack_awq          -> paro_pack_awq
+    unpack_awq        -> paro_unpack_awq
+    w4_linear         -> paro_w4_linear (+ paro_w4_linear_workspace_size)
+    validate_pairs    -> paro_validate_pairs (host helper)
+    device_status     -> paro_device_status
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import numpy as np
+import torch
+
+from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # noqa: F401
+                   PARO_ERR_TIMEOUT, PARO_ERR_UNSUPPORTED, PARO_ERR_WORKSPACE, PARO_OK,
+                   LIB_PATH, ParoError, check, lib, paro_device_status, paro_pack_awq,
+                   paro_rotate, paro_status_string, paro_unpack_awq, paro_validate_pairs,
+                   paro_version, paro_w4_linear, paro_w4_linear_workspace_size)
+
+__all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
+           "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: Optional[torch.Tensor], dtype, name: str, allow_none: bool = False):
+    if t is None:
+        if allow_none:
+            return
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def rotate(x: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: Optional[torch.Tensor],
+           theta: Optional[torch.Tensor], group_size: int = 128, krot: Optional[int] = None,
+           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """X_r = rotate(x * channel_scales); ``out`` may be ``x`` (in place)."""
+    _need(x, torch.float16, "x")
+    _need(channel_scales, torch.float32, "channel_scales", True)
+    _need(pairs, torch.int16, "pairs", True)
+    _need(theta, torch.float32, "theta", True)
+    if krot is None:
+        krot = 0 if pairs is None else pairs.shape[0]
+    if out is None:
+        out = torch.empty_like(x)
+    M, K = x.shape
+    check(paro_rotate(_ptr(x), _ptr(out), M, K, _ptr(channel_scales), _ptr(pairs), _ptr(theta),
+                      group_size, krot, _stream(stream)), "paro_rotate")
+    return out
+
+
+def pack_awq(codes: torch.Tensor, zero_codes: Optional[torch.Tensor], group_size: int = 128,
+             stream=None):
+    """codes uint8 [N, K], zero_codes uint8 [N, K/G] -> (qweight int32 [K, N/8], qzeros)."""
+    _need(codes, torch.uint8, "codes")
+    _need(zero_codes, torch.uint8, "zero_codes", True)
+    N, K = codes.shape
+    G = K if group_size == -1 else group_size
+    qweight = torch.empty((K, N // 8), dtype=torch.int32, device=codes.device)
+    qzeros = None
+    if zero_codes is not None:
+        qzeros = torch.empty((K // G, N // 8), dtype=torch.int32, device=codes.device)
+    check(paro_pack_awq(_ptr(codes), _ptr(zero_codes), _ptr(qweight), _ptr(qzeros), N, K,
+                        group_size, _stream(stream)), "paro_pack_awq")
+    return qweight, qzeros
+
+
+def unpack_awq(qweight: torch.Tensor, qzeros: Optional[torch.Tensor], N: int, K: int,
+               group_size: int = 128, stream=None):
+    _need(qweight, torch.int32, "qweight")
+    _need(qzeros, torch.int32, "qzeros", True)
+    G = K if group_size == -1 else group_size
+    codes = torch.empty((N, K), dtype=torch.uint8, device=qweight.device)
+    zeros = None
+    if qzeros is not None:
+        zeros = torch.empty((N, K // G), dtype=torch.uint8, device=qweight.device)
+    check(paro_unpack_awq(_ptr(qweight), _ptr(qzeros), _ptr(codes), _ptr(zeros), N, K,
+                          group_size, _stream(stream)), "paro_unpack_awq")
+    return codes, zeros
+
+
+def w4_linear_workspace_size(M: int, K: int, N: int, group_size: int = 128) -> int:
+    return int(paro_w4_linear_workspace_size(M, K, N, group_size))
+
+
+def w4_linear(x: torch.Tensor, qweight: torch.Tensor, qzeros: torch.Tensor, scales: torch.Tensor,
+              bias: Optional[torch.Tensor], channel_scales: Optional[torch.Tensor],
+              pairs: Optional[torch.Tensor], theta: Optional[torch.Tensor],
+              group_size: int = 128, krot: Optional[int] = None,
+              workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """Y = rotate(x * channel_scales) @ dequant(qweight, qzeros, scales) + bias (fp16 out)."""
+    _need(x, torch.float16, "x")
+    _need(qweight, torch.int32, "qweight")
+    _need(qzeros, torch.int32, "qzeros")
+    _need(scales, torch.float16, "scales")
+    _need(bias, torch.float16, "bias", True)
+    _need(channel_scales, torch.float32, "channel_scales", True)
+    _need(pairs, torch.int16, "pairs", True)
+    _need(theta, torch.float32, "theta", True)
+    if krot is None:
+        krot = 0 if pairs is None else pairs.shape[0]
+    M, K = x.shape
+    N = qweight.shape[1] * 8
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    need = w4_linear_workspace_size(M, K, N, group_size)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    check(paro_w4_linear(_ptr(x), _ptr(out), M, K, N, _ptr(qweight), _ptr(qzeros), _ptr(scales),
+                         _ptr(bias), _ptr(channel_scales), _ptr(pairs), _ptr(theta), group_size,
+                         krot, _ptr(workspace), ws_bytes, _stream(stream)), "paro_w4_linear")
+    return out
+
+
+def validate_pairs(pairs: np.ndarray, K: int, group_size: int = 128, krot: Optional[int] = None) -> bool:
+    """Host check that each stage of each group is a permutation of 0..G-1."""
+    p = np.ascontiguousarray(pairs, dtype=np.int16)
+    if krot is None:
+        krot = p.shape[0]
+    st = paro_validate_pairs(p.ctypes.data_as(ctypes.c_void_p), K, group_size, krot)
+    return st == PARO_OK
+
+
+def device_status(clear: bool = True) -> int:
+    """Synchronises and returns the device status word as a PARO_* code."""
+    return int(paro_device_status(1 if clear else 0))

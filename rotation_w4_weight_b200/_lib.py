@@ -1,0 +1,81 @@
+"""ctypes binding of the C ABI in include/paro.h (argument marshalling only).
+
+Every function of the header is exposed here under the same name.  The
+library must exist (build it with ``python -m rotation_w4_weight_b200.build``);
+importing this module without it raises, there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libparo_b200.so")
+
+PARO_OK = 0
+PARO_ERR_INVALID_ARG = 1
+PARO_ERR_UNSUPPORTED = 2
+PARO_ERR_ALIGNMENT = 3
+PARO_ERR_WORKSPACE = 4
+PARO_ERR_CUDA = 5
+PARO_ERR_TIMEOUT = 6
+
+EXPORTED = (
+    "paro_status_string", "paro_version", "paro_rotate", "paro_pack_awq", "paro_unpack_awq",
+    "paro_w4_linear_workspace_size", "paro_w4_linear", "paro_validate_pairs",
+    "paro_device_status",
+)
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+_SIGNATURES = {
+    "paro_status_string": (ctypes.c_char_p, [_int]),
+    "paro_version": (ctypes.c_char_p, []),
+    "paro_rotate": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _int, _int, _vp]),
+    "paro_pack_awq": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp]),
+    "paro_unpack_awq": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp]),
+    "paro_w4_linear_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _int]),
+    "paro_w4_linear": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                              _int, _int, _vp, ctypes.c_size_t, _vp]),
+    "paro_validate_pairs": (_int, [_vp, _i64, _int, _int]),
+    "paro_device_status": (_int, [_int]),
+}
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build the CUDA library first "
+            "(python -m rotation_w4_weight_b200.build); there is no CPU fallback")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = load()
+
+paro_status_string = lib.paro_status_string
+paro_version = lib.paro_version
+paro_rotate = lib.paro_rotate
+paro_pack_awq = lib.paro_pack_awq
+paro_unpack_awq = lib.paro_unpack_awq
+paro_w4_linear_workspace_size = lib.paro_w4_linear_workspace_size
+paro_w4_linear = lib.paro_w4_linear
+paro_validate_pairs = lib.paro_validate_pairs
+paro_device_status = lib.paro_device_status
+
+
+class ParoError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {paro_status_string(status).decode()} (status {status})")
+
+
+def check(status: int, what: str) -> None:
+    if status != PARO_OK:
+        raise ParoError(status, what)

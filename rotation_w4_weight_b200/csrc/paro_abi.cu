@@ -1,0 +1,443 @@
+// C ABI of the library (declarations and contracts in include/paro.h):
+// host-side validation, workspace planning, TMA descriptor encoding and
+// kernel dispatch.  Every error is reported as a status code before any launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/paro.h"
+#include "common.cuh"
+#include "pack.cuh"
+#include "rotate.cuh"
+#include "w4_mma.cuh"
+
+using namespace paro;
+
+namespace {
+
+constexpr int kMaxDecodeM = 16;      // M <= 16: split-K GEMV path
+constexpr int kDecodeTargetCtas = 296;
+constexpr int kMaxSplits = 8;         // cluster size along K (portable maximum)
+constexpr int kDecodeKSplit = 2;      // k-parts (warp groups) per decode CTA
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- TMA encode
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `esize`-byte elements, box [box_rows, box_cols].
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, size_t esize, const void* ptr,
+               uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+               CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esize};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- launches
+template <typename Kern, typename... Args>
+int launch_ex(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+              unsigned cluster_y, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_y > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = cluster_y;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = n ? attr : nullptr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? PARO_OK : PARO_ERR_CUDA;
+}
+
+template <typename Kern, typename... Args>
+int launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+           Args... args) {
+  return launch_ex(kernel, grid, block, smem, stream, pdl, 1u, args...);
+}
+
+// Raise the dynamic shared memory limit of a kernel once per device (callers
+// pass the largest size the kernel is ever launched with).
+template <typename Kern>
+bool allow_smem(Kern kernel, size_t bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  std::lock_guard<std::mutex> lock(mu);
+  const void* key = reinterpret_cast<const void*>(kernel);
+  for (auto& d : done)
+    if (d.first == key && d.second == dev) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess)
+    return false;
+  done.emplace_back(key, dev);
+  return true;
+}
+
+int normalize_group(int group_size, int64_t K, int* G) {
+  const int64_t g = (group_size == -1) ? K : group_size;
+  if (g <= 0 || (g % 2) != 0 || K <= 0 || (K % g) != 0) return PARO_ERR_INVALID_ARG;
+  *G = static_cast<int>(g);
+  return PARO_OK;
+}
+
+// ---------------------------------------------------------------- rotation
+int check_rotation_args(const void* x, const void* xr, int64_t M, int64_t K, const float* cs,
+                        const int16_t* pairs, const float* theta, int group_size, int krot) {
+  if (M < 0 || K <= 0 || krot < 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  if (G != kGroup || krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
+  if (M == 0) return PARO_OK;   // nothing to touch: NULL data pointers are fine
+  if (x == nullptr || xr == nullptr) return PARO_ERR_INVALID_ARG;
+  if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
+  if (M * K >= (int64_t(1) << 31)) return PARO_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(xr, 16)) return PARO_ERR_ALIGNMENT;
+  if (cs != nullptr && !aligned(cs, 16)) return PARO_ERR_ALIGNMENT;
+  if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
+  return PARO_OK;
+}
+
+int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
+                  const int16_t* pairs, const float* theta, int krot, cudaStream_t stream) {
+  // rows per CTA: 4 for decode-sized batches (more CTAs, shorter latency),
+  // 32..128 for large batches (conflict-free 32-row warp accesses)
+  const int rows = M <= 16 ? 4 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
+  const size_t smem = rotate_smem_bytes(rows, krot);
+  const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + rows - 1) / rows));
+  const dim3 block(kRotThreads);
+  if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
+  // the limit is raised once to what the largest krot needs
+  switch (rows) {
+    case 4:
+      if (!allow_smem(rotate_kernel<4>, rotate_smem_bytes(4, kMaxKrot))) return PARO_ERR_CUDA;
+      return launch(rotate_kernel<4>, grid, block, smem, stream, false, x, xr, cs, pairs, theta,
+                    (int)M, (int)K, krot);
+    case 32:
+      if (!allow_smem(rotate_kernel<32>, rotate_smem_bytes(32, kMaxKrot))) return PARO_ERR_CUDA;
+      return launch(rotate_kernel<32>, grid, block, smem, stream, false, x, xr, cs, pairs, theta,
+                    (int)M, (int)K, krot);
+    case 64:
+      if (!allow_smem(rotate_kernel<64>, rotate_smem_bytes(64, kMaxKrot))) return PARO_ERR_CUDA;
+      return launch(rotate_kernel<64>, grid, block, smem, stream, false, x, xr, cs, pairs, theta,
+                    (int)M, (int)K, krot);
+    default:
+      if (!allow_smem(rotate_kernel<128>, rotate_smem_bytes(128, kMaxKrot))) return PARO_ERR_CUDA;
+      return launch(rotate_kernel<128>, grid, block, smem, stream, false, x, xr, cs, pairs, theta,
+                    (int)M, (int)K, krot);
+  }
+}
+
+// ---------------------------------------------------------------- linear plan
+struct LinearPlan {
+  bool decode = false;
+  int nt = 1;              // decode: 8-token MMA tiles per CTA
+  int n_tiles = 0;         // 256-column tiles
+  int splits = 1;          // decode split-K factor = cluster size along K
+  size_t off_xr = 0, total = 0;
+};
+
+int check_linear_shape(int64_t M, int64_t K, int64_t N, int group_size) {
+  if (M < 0 || K <= 0 || N <= 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  if (N % 8 != 0) return PARO_ERR_INVALID_ARG;
+  if (G != kGroup || N % 32 != 0) return PARO_ERR_UNSUPPORTED;
+  if (M * K >= (int64_t(1) << 31) || M * N >= (int64_t(1) << 31) || K * N >= (int64_t(1) << 34) ||
+      M > (int64_t(1) << 22))
+    return PARO_ERR_UNSUPPORTED;
+  return PARO_OK;
+}
+
+// The split is a function of the shape only (not of the device), so the
+// workspace size query and the call agree everywhere.
+LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
+  LinearPlan p;
+  const int groups = (int)(K / kGroup);
+  p.n_tiles = (int)((N + kNTile - 1) / kNTile);
+  p.decode = M <= kMaxDecodeM;
+  p.off_xr = 0;
+  p.total = round_up((size_t)M * K * 2, 256);   // X_r, written when rotating
+  if (p.decode) {
+    p.nt = M <= 8 ? 1 : 2;
+    int s = 1;
+    while (s * 2 <= kMaxSplits && s * 2 <= groups && p.n_tiles * s * 2 <= kDecodeTargetCtas) s *= 2;
+    p.splits = s;
+  }
+  return p;
+}
+
+// Prefill (M > 16): 64-token tiles on the warp-MMA kernel, scales folded into
+// the fp16 weights before the MMA, full K per CTA.
+int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t N,
+                      const int32_t* qweight, const int32_t* qzeros, const __half* scales,
+                      const __half* bias, cudaStream_t s, bool pdl) {
+  constexpr int NT = 8;
+  using L = MmaLayout<NT, 1>;
+  CUtensorMap tmW, tmX, tmS, tmZ;
+  bool ok = encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, kNWords,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, L::MP, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kNTile,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kNWords,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return PARO_ERR_CUDA;
+  const dim3 grid((unsigned)((N + kNTile - 1) / kNTile), 1, (unsigned)((M + L::MP - 1) / L::MP));
+  auto k = w4_mma_kernel<NT, 1, true>;
+  if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
+  return launch(k, grid, dim3(L::THREADS), L::SMEM, s, pdl, tmW, tmX, tmS, tmZ, bias, y, (int)M,
+                (int)N, (int)K);
+}
+
+// Decode GEMV launch: grid (column tiles, splits), one cluster of `splits`
+// CTAs per column tile.  Clusters of 16 need the non-portable opt-in and room
+// for 16 co-resident CTAs in one GPC; if the device cannot run them the split
+// falls back to 8.
+template <int NT>
+int launch_decode(const LinearPlan& plan, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                  const CUtensorMap& tmS, const CUtensorMap& tmZ, const __half* bias, __half* y,
+                  int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
+  using L = MmaLayout<NT, kDecodeKSplit>;
+  auto k = w4_mma_kernel<NT, kDecodeKSplit, false>;
+  if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
+  int splits = plan.splits;
+  if (splits > 8) {
+    static int ok16 = -1;   // per process; all GPUs of a box are the same part
+    if (ok16 < 0) {
+      ok16 = 0;
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)plan.n_tiles, 16, 1);
+        cfg.blockDim = dim3(L::THREADS);
+        cfg.dynamicSmemBytes = L::SMEM;
+        cudaLaunchAttribute a[1];
+        a[0].id = cudaLaunchAttributeClusterDimension;
+        a[0].val.clusterDim.x = 1;
+        a[0].val.clusterDim.y = 16;
+        a[0].val.clusterDim.z = 1;
+        cfg.attrs = a;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, k, &cfg) == cudaSuccess && nclusters > 0)
+          ok16 = 1;
+      }
+      cudaGetLastError();
+    }
+    if (!ok16) splits = 8;
+  }
+  const dim3 grid((unsigned)plan.n_tiles, (unsigned)splits, 1);
+  return launch_ex(k, grid, dim3(L::THREADS), L::SMEM, s, pdl, (unsigned)splits, tmW, tmX, tmS,
+                   tmZ, bias, y, (int)M, (int)N, (int)K);
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* paro_status_string(int status) {
+  switch (status) {
+    case PARO_OK: return "ok";
+    case PARO_ERR_INVALID_ARG: return "invalid argument";
+    case PARO_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PARO_ERR_ALIGNMENT: return "misaligned pointer";
+    case PARO_ERR_WORKSPACE: return "workspace missing or too small";
+    case PARO_ERR_CUDA: return "CUDA error";
+    case PARO_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* paro_version(void) { return "0.1.0"; }
+
+int paro_rotate(const void* x, void* x_r, int64_t M, int64_t K, const float* channel_scales,
+                const int16_t* pairs, const float* theta, int group_size, int krot,
+                paro_stream_t stream) {
+  if (int st = check_rotation_args(x, x_r, M, K, channel_scales, pairs, theta, group_size, krot))
+    return st;
+  if (M == 0) return PARO_OK;
+  return launch_rotate(static_cast<const __half*>(x), static_cast<__half*>(x_r), M, K,
+                       channel_scales, pairs, theta, krot, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qweight,
+                  int32_t* qzeros, int64_t N, int64_t K, int group_size, paro_stream_t stream) {
+  if (N <= 0 || K <= 0 || N % 8 != 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  if (codes == nullptr || qweight == nullptr) return PARO_ERR_INVALID_ARG;
+  if ((zero_codes == nullptr) != (qzeros == nullptr)) return PARO_ERR_INVALID_ARG;
+  if (N / 8 > 65535) return PARO_ERR_UNSUPPORTED;
+  if (!aligned(qweight, 4) || (qzeros != nullptr && !aligned(qzeros, 4))) return PARO_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (int st = launch(pack_rows_kernel, dim3((unsigned)((K + 255) / 256), (unsigned)(N / 8)),
+                      dim3(256), 0, s, false, codes, qweight, N, K))
+    return st;
+  if (qzeros != nullptr) {
+    const int64_t R = K / G;
+    return launch(pack_rows_kernel, dim3((unsigned)((R + 255) / 256), (unsigned)(N / 8)),
+                  dim3(256), 0, s, false, zero_codes, qzeros, N, R);
+  }
+  return PARO_OK;
+}
+
+int paro_unpack_awq(const int32_t* qweight, const int32_t* qzeros, uint8_t* codes,
+                    uint8_t* zero_codes, int64_t N, int64_t K, int group_size,
+                    paro_stream_t stream) {
+  if (N <= 0 || K <= 0 || N % 8 != 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  if (codes == nullptr || qweight == nullptr) return PARO_ERR_INVALID_ARG;
+  if ((zero_codes == nullptr) != (qzeros == nullptr)) return PARO_ERR_INVALID_ARG;
+  if (N / 8 > 65535) return PARO_ERR_UNSUPPORTED;
+  if (!aligned(qweight, 4) || (qzeros != nullptr && !aligned(qzeros, 4))) return PARO_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (int st = launch(unpack_rows_kernel, dim3((unsigned)((K + 255) / 256), (unsigned)(N / 8)),
+                      dim3(256), 0, s, false, qweight, codes, N, K))
+    return st;
+  if (qzeros != nullptr) {
+    const int64_t R = K / G;
+    return launch(unpack_rows_kernel, dim3((unsigned)((R + 255) / 256), (unsigned)(N / 8)),
+                  dim3(256), 0, s, false, qzeros, zero_codes, N, R);
+  }
+  return PARO_OK;
+}
+
+size_t paro_w4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int group_size) {
+  if (check_linear_shape(M, K, N, group_size) != PARO_OK) return 0;
+  return make_plan(M, K, N).total;
+}
+
+int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                   const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                   const void* bias, const float* channel_scales, const int16_t* pairs,
+                   const float* theta, int group_size, int krot, void* workspace,
+                   size_t workspace_bytes, paro_stream_t stream) {
+  if (int st = check_linear_shape(M, K, N, group_size)) return st;
+  if (krot < 0) return PARO_ERR_INVALID_ARG;
+  if (krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
+  if (M == 0) return PARO_OK;   // empty batch: nothing to read or write
+  if (x == nullptr || y == nullptr || qweight == nullptr || qzeros == nullptr || scales == nullptr)
+    return PARO_ERR_INVALID_ARG;
+  if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(qweight, 16) || !aligned(qzeros, 16) ||
+      !aligned(scales, 16) || (bias != nullptr && !aligned(bias, 4)))
+    return PARO_ERR_ALIGNMENT;
+  if (channel_scales != nullptr && !aligned(channel_scales, 16)) return PARO_ERR_ALIGNMENT;
+  if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
+
+  const LinearPlan plan = make_plan(M, K, N);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool rotate = krot > 0 || channel_scales != nullptr;
+  if (rotate && (workspace == nullptr || workspace_bytes < plan.total)) return PARO_ERR_WORKSPACE;
+  if (rotate && !aligned(workspace, 256)) return PARO_ERR_ALIGNMENT;
+  const __half* xa = static_cast<const __half*>(x);
+  bool pdl = false;
+  if (rotate) {
+    __half* xr = reinterpret_cast<__half*>(static_cast<unsigned char*>(workspace) + plan.off_xr);
+    if (int st = launch_rotate(xa, xr, M, K, channel_scales, pairs, theta, krot, s)) return st;
+    xa = xr;
+    pdl = true;   // the GEMV streams weights while the rotation finishes
+  }
+
+  const __half* b = static_cast<const __half*>(bias);
+  __half* yy = static_cast<__half*>(y);
+  if (!plan.decode)
+    return launch_w4_prefill(xa, yy, M, K, N, qweight, qzeros, static_cast<const __half*>(scales),
+                             b, s, pdl);
+
+  CUtensorMap tmW, tmX, tmS, tmZ;
+  const int mp = 8 * plan.nt;
+  bool ok = encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, kNWords,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, mp, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kNTile,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kNWords,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return PARO_ERR_CUDA;
+  const __half* bb = b;
+  if (plan.nt == 1)
+    return launch_decode<1>(plan, tmW, tmX, tmS, tmZ, bb, yy, M, N, K, s, pdl);
+  return launch_decode<2>(plan, tmW, tmX, tmS, tmZ, bb, yy, M, N, K, s, pdl);
+}
+
+int paro_validate_pairs(const int16_t* pairs_host, int64_t K, int group_size, int krot) {
+  if (pairs_host == nullptr || krot < 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  std::vector<unsigned char> seen((size_t)G);
+  for (int s = 0; s < krot; ++s)
+    for (int64_t g = 0; g < K / G; ++g) {
+      std::fill(seen.begin(), seen.end(), 0);
+      const int16_t* p = pairs_host + (size_t)s * K + (size_t)g * G;
+      for (int e = 0; e < G; ++e) {
+        const int v = p[e];
+        if (v < 0 || v >= G || seen[(size_t)v]) return PARO_ERR_INVALID_ARG;
+        seen[(size_t)v] = 1;
+      }
+    }
+  return PARO_OK;
+}
+
+int paro_device_status(int clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return PARO_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, paro::g_status, sizeof(v)) != cudaSuccess) return PARO_ERR_CUDA;
+  if (clear) {
+    const unsigned z = 0;
+    if (cudaMemcpyToSymbol(paro::g_status, &z, sizeof(z)) != cudaSuccess) return PARO_ERR_CUDA;
+  }
+  if (v & kErrTimeout) return PARO_ERR_TIMEOUT;
+  if (v & kErrPairIndex) return PARO_ERR_INVALID_ARG;
+  return PARO_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments with the documented status before
+any GPU work (these calls never reach a CUDA API, so they run without a GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from rotation_w4_weight_b200 import build
+    build.build()
+    from rotation_w4_weight_b200 import _lib
+    return _lib
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "paro.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(paro_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_exports_every_header_symbol(L):
+    names = header_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L.lib, n), n
+    assert set(names) <= set(L.EXPORTED) | set(names)
+    assert L.paro_version().decode().count(".") == 2
+
+
+def test_status_strings(L):
+    for code in range(7):
+        s = L.paro_status_string(code)
+        assert s and isinstance(s, bytes)
+    assert L.paro_status_string(99) == b"unknown status"
+
+
+P = ctypes.c_void_p
+A16 = P(0x10000)           # never dereferenced: validation fails before any use
+MIS = P(0x10008)           # 8-byte aligned, not 16
+
+
+def lin(L, x=A16, y=A16, M=4, K=256, N=512, qw=A16, qz=A16, sc=A16, bias=None, cs=None,
+        pairs=None, theta=None, G=128, krot=0, ws=None, wsb=0):
+    return L.paro_w4_linear(x, y, M, K, N, qw, qz, sc, bias, cs, pairs, theta, G, krot, ws, wsb, None)
+
+
+def test_linear_argument_validation(L):
+    assert lin(L, M=-1) == L.PARO_ERR_INVALID_ARG
+    assert lin(L, K=0) == L.PARO_ERR_INVALID_ARG
+    assert lin(L, N=12) == L.PARO_ERR_INVALID_ARG            # N % 8
+    assert lin(L, N=40) == L.PARO_ERR_UNSUPPORTED            # N % 32 (valid for the packer only)
+    assert lin(L, K=200) == L.PARO_ERR_INVALID_ARG           # K % G
+    assert lin(L, G=3) == L.PARO_ERR_INVALID_ARG             # odd group
+    assert lin(L, G=64) == L.PARO_ERR_UNSUPPORTED
+    assert lin(L, K=256, G=-1) == L.PARO_ERR_UNSUPPORTED     # G normalised to K=256
+    assert lin(L, x=None) == L.PARO_ERR_INVALID_ARG
+    assert lin(L, qz=None) == L.PARO_ERR_INVALID_ARG
+    assert lin(L, krot=8) == L.PARO_ERR_INVALID_ARG          # pairs/theta missing
+    assert lin(L, krot=65, pairs=A16, theta=A16) == L.PARO_ERR_UNSUPPORTED
+    assert lin(L, krot=-1) == L.PARO_ERR_INVALID_ARG
+    assert lin(L, x=MIS) == L.PARO_ERR_ALIGNMENT
+    assert lin(L, qw=MIS) == L.PARO_ERR_ALIGNMENT
+    assert lin(L, cs=MIS) == L.PARO_ERR_ALIGNMENT
+    assert lin(L, M=0) == L.PARO_OK                          # empty batch: no work
+    need = L.paro_w4_linear_workspace_size(4, 256, 512, 128)
+    assert need > 0
+    # the rotated path (channel scales or krot > 0) stages X_r in the workspace
+    assert lin(L, cs=A16, ws=None, wsb=0) == L.PARO_ERR_WORKSPACE
+    assert lin(L, cs=A16, ws=A16, wsb=need - 1) == L.PARO_ERR_WORKSPACE
+    assert lin(L, cs=A16, ws=P(0x10010), wsb=need) == L.PARO_ERR_ALIGNMENT   # needs 256 B
+    assert lin(L, krot=8, pairs=A16, theta=A16, ws=None) == L.PARO_ERR_WORKSPACE
+
+
+def test_workspace_size_query(L):
+    f = L.paro_w4_linear_workspace_size
+    assert f(4, 200, 512, 128) == 0          # rejected shape
+    assert f(0, 256, 512, 128) >= 0
+    # grows with M and is a multiple of 256 bytes
+    for M in (1, 4, 16, 17, 2048):
+        v = f(M, 4096, 4096, 128)
+        assert v % 256 == 0 and v >= M * 4096 * 2
+    assert f(8192, 4096, 14336, 128) >= 8192 * 4096 * 2
+
+
+def test_rotate_argument_validation(L):
+    r = L.paro_rotate
+    assert r(A16, A16, -1, 256, None, None, None, 128, 0, None) == L.PARO_ERR_INVALID_ARG
+    assert r(None, A16, 4, 256, None, None, None, 128, 0, None) == L.PARO_ERR_INVALID_ARG
+    assert r(A16, A16, 4, 256, None, None, None, 128, 8, None) == L.PARO_ERR_INVALID_ARG
+    assert r(A16, A16, 4, 256, None, A16, A16, 64, 8, None) == L.PARO_ERR_UNSUPPORTED
+    assert r(A16, A16, 4, 250, None, A16, A16, 128, 8, None) == L.PARO_ERR_INVALID_ARG
+    assert r(MIS, A16, 4, 256, None, A16, A16, 128, 8, None) == L.PARO_ERR_ALIGNMENT
+    assert r(A16, A16, 0, 256, None, A16, A16, 128, 8, None) == L.PARO_OK
+
+
+def test_pack_argument_validation(L):
+    p = L.paro_pack_awq
+    assert p(A16, A16, A16, A16, 12, 256, 128, None) == L.PARO_ERR_INVALID_ARG
+    assert p(A16, None, A16, A16, 16, 256, 128, None) == L.PARO_ERR_INVALID_ARG
+    assert p(None, A16, A16, A16, 16, 256, 128, None) == L.PARO_ERR_INVALID_ARG
+    assert p(A16, A16, P(0x10002), A16, 16, 256, 128, None) == L.PARO_ERR_ALIGNMENT
+    u = L.paro_unpack_awq
+    assert u(A16, A16, A16, A16, 16, 250, 128, None) == L.PARO_ERR_INVALID_ARG
+
+
+def test_validate_pairs_host_helper(L):
+    import synth
+    lay = synth.make_layer("t", 256, 64, 3)
+    import rotation_w4_weight_b200 as pb
+    assert pb.validate_pairs(lay.pairs, 256, 128)
+    bad = lay.pairs.copy()
+    bad[2, 5] = bad[2, 6]                      # duplicate channel in a group
+    assert not pb.validate_pairs(bad, 256, 128)
+    bad = lay.pairs.copy()
+    bad[0, 0] = 128                            # outside the group
+    assert not pb.validate_pairs(bad, 256, 128)
+    assert pb.validate_pairs(np.zeros((0, 256), np.int16), 256, 128, 0)
