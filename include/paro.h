@@ -145,6 +145,40 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
                    size_t workspace_bytes, paro_stream_t stream);
 
 /*
+ * paro_w4_linear_noalloc — paro_w4_linear for callers that cannot allocate
+ * device memory.  The paper has no counterpart; this entry point exists for
+ * library users, not for the method.
+ *
+ * Some callers cannot hand this library a workspace: code that records CUDA
+ * graphs in the global capture mode (cudaMalloc is not allowed there),
+ * latency-critical loops that must not pay cudaMalloc's implicit device
+ * synchronisation, and plugin hosts that own all device memory and forbid a
+ * library from allocating outside their pool.  This variant takes the same
+ * arguments as paro_w4_linear minus the workspace and stages X_r in a
+ * file-scope device array of PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES bytes that
+ * every GPU which loads the library holds until the process exits.  It calls
+ * no cudaMalloc, cudaFree or allocating library routine.
+ *   - Limit: paro_w4_linear_workspace_size(M, K, N, group_size) must not exceed
+ *     PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES (8 MiB: M*K <= 4 Mi fp16 elements);
+ *     larger shapes return PARO_ERR_WORKSPACE before any GPU work.
+ *   - The first call on a device looks up the array's device address for that
+ *     device (cudaGetSymbolAddress) and caches it; make that first call before
+ *     any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents (it
+ *     needs no clearing: each call overwrites what it reads).  Calls whose work
+ *     can overlap on the GPU (different streams, or different host threads on
+ *     one device) race on the array; serialise them, or use paro_w4_linear with
+ *     separate workspaces.
+ * Results are those of paro_w4_linear for the same arguments.
+ */
+#define PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+int paro_w4_linear_noalloc(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                           const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                           const void* bias, const float* channel_scales, const int16_t* pairs,
+                           const float* theta, int group_size, int krot, paro_stream_t stream);
+
+/*
  * paro_validate_pairs — HOST helper (host pointer, synchronous, no GPU work):
  * checks that every stage of every group of a [krot, K] pair table is a
  * permutation of 0..G-1 (each channel in exactly one pair; cf. the page's

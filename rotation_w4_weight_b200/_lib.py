@@ -22,8 +22,8 @@ PARO_ERR_TIMEOUT = 6
 
 EXPORTED = (
     "paro_status_string", "paro_version", "paro_rotate", "paro_pack_awq", "paro_unpack_awq",
-    "paro_w4_linear_workspace_size", "paro_w4_linear", "paro_validate_pairs",
-    "paro_device_status",
+    "paro_w4_linear_workspace_size", "paro_w4_linear", "paro_w4_linear_noalloc",
+    "paro_validate_pairs", "paro_device_status",
 )
 
 _vp = ctypes.c_void_p
@@ -39,6 +39,8 @@ _SIGNATURES = {
     "paro_w4_linear_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _int]),
     "paro_w4_linear": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                               _int, _int, _vp, ctypes.c_size_t, _vp]),
+    "paro_w4_linear_noalloc": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _vp, _int, _int, _vp]),
     "paro_validate_pairs": (_int, [_vp, _i64, _int, _int]),
     "paro_device_status": (_int, [_int]),
 }
@@ -66,6 +68,8 @@ paro_pack_awq = lib.paro_pack_awq
 paro_unpack_awq = lib.paro_unpack_awq
 paro_w4_linear_workspace_size = lib.paro_w4_linear_workspace_size
 paro_w4_linear = lib.paro_w4_linear
+paro_w4_linear_noalloc = lib.paro_w4_linear_noalloc
+PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES = 8 << 20
 paro_validate_pairs = lib.paro_validate_pairs
 paro_device_status = lib.paro_device_status
 

@@ -409,6 +409,53 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
   return launch_decode<2>(plan, tmW, tmX, tmS, tmZ, bb, yy, M, N, K, s, pdl);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------ no-allocation variant
+// Scratch for paro_w4_linear_noalloc: a file-scope device array (every GPU that
+// loads the library holds it until exit).  Host code must not pass the symbol
+// itself to a kernel — on the host it is only a stand-in; the device address
+// comes from cudaGetSymbolAddress, looked up once per device and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_scratch on the current device (nullptr on failure).
+void* noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+}  // namespace
+
+extern "C" {
+
+int paro_w4_linear_noalloc(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                           const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                           const void* bias, const float* channel_scales, const int16_t* pairs,
+                           const float* theta, int group_size, int krot, paro_stream_t stream) {
+  // An invalid shape yields 0 here and the full validation below reports it.
+  const size_t need = paro_w4_linear_workspace_size(M, K, N, group_size);
+  if (need > (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES) return PARO_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (need > 0 && M > 0) {
+    scratch = noalloc_scratch_address();
+    if (scratch == nullptr) return PARO_ERR_CUDA;
+  }
+  return paro_w4_linear(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
+                        group_size, krot, scratch,
+                        scratch ? (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES : 0, stream);
+}
+
 int paro_validate_pairs(const int16_t* pairs_host, int64_t K, int group_size, int krot) {
   if (pairs_host == nullptr || krot < 0) return PARO_ERR_INVALID_ARG;
   int G = 0;
