@@ -14,16 +14,16 @@
 #include "common.cuh"
 #include "pack.cuh"
 #include "rotate.cuh"
-#include "w4_mma.cuh"
+#include "w4_gemv.cuh"
+#include "w4_tc.cuh"
 
 using namespace paro;
 
 namespace {
 
 constexpr int kMaxDecodeM = 16;      // M <= 16: split-K GEMV path
-constexpr int kDecodeTargetCtas = 296;
+constexpr int kDecodeTargetCtas = 148;   // one decode CTA per SM
 constexpr int kMaxSplits = 8;         // cluster size along K (portable maximum)
-constexpr int kDecodeKSplit = 2;      // k-parts (warp groups) per decode CTA
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -154,19 +154,19 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
   switch (rows) {
     case 4:
       if (!allow_smem(rotate_kernel<4>, rotate_smem_bytes(4, kMaxKrot))) return PARO_ERR_CUDA;
-      return launch(rotate_kernel<4>, grid, block, smem, stream, false, x, xr, cs, pairs, theta,
+      return launch(rotate_kernel<4>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
                     (int)M, (int)K, krot);
     case 32:
       if (!allow_smem(rotate_kernel<32>, rotate_smem_bytes(32, kMaxKrot))) return PARO_ERR_CUDA;
-      return launch(rotate_kernel<32>, grid, block, smem, stream, false, x, xr, cs, pairs, theta,
+      return launch(rotate_kernel<32>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
                     (int)M, (int)K, krot);
     case 64:
       if (!allow_smem(rotate_kernel<64>, rotate_smem_bytes(64, kMaxKrot))) return PARO_ERR_CUDA;
-      return launch(rotate_kernel<64>, grid, block, smem, stream, false, x, xr, cs, pairs, theta,
+      return launch(rotate_kernel<64>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
                     (int)M, (int)K, krot);
     default:
       if (!allow_smem(rotate_kernel<128>, rotate_smem_bytes(128, kMaxKrot))) return PARO_ERR_CUDA;
-      return launch(rotate_kernel<128>, grid, block, smem, stream, false, x, xr, cs, pairs, theta,
+      return launch(rotate_kernel<128>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
                     (int)M, (int)K, krot);
   }
 }
@@ -177,6 +177,7 @@ struct LinearPlan {
   int nt = 1;              // decode: 8-token MMA tiles per CTA
   int n_tiles = 0;         // 256-column tiles
   int splits = 1;          // decode split-K factor = cluster size along K
+  int kparts = 2;          // decode consumer warp sets per CTA
   size_t off_xr = 0, total = 0;
 };
 
@@ -197,7 +198,7 @@ int check_linear_shape(int64_t M, int64_t K, int64_t N, int group_size) {
 LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
   LinearPlan p;
   const int groups = (int)(K / kGroup);
-  p.n_tiles = (int)((N + kNTile - 1) / kNTile);
+  p.n_tiles = (int)((N + kGvTile - 1) / kGvTile);
   p.decode = M <= kMaxDecodeM;
   p.off_xr = 0;
   p.total = round_up((size_t)M * K * 2, 256);   // X_r, written when rotating
@@ -206,73 +207,45 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
     int s = 1;
     while (s * 2 <= kMaxSplits && s * 2 <= groups && p.n_tiles * s * 2 <= kDecodeTargetCtas) s *= 2;
     p.splits = s;
+    const int per_cta = (groups + s - 1) / s;
+    p.kparts = (per_cta <= 4 && p.nt == 1) ? 4 : 2;   // more warps when each has few groups
   }
   return p;
 }
 
-// Prefill (M > 16): 64-token tiles on the warp-MMA kernel, scales folded into
-// the fp16 weights before the MMA, full K per CTA.
+// Prefill (M > 16): tcgen05 GEMM, 128 token rows x 256 output columns per CTA.
 int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t N,
                       const int32_t* qweight, const int32_t* qzeros, const __half* scales,
                       const __half* bias, cudaStream_t s, bool pdl) {
-  constexpr int NT = 8;
-  using L = MmaLayout<NT, 1>;
-  CUtensorMap tmW, tmX, tmS, tmZ;
-  bool ok = encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, kNWords,
+  CUtensorMap tmA, tmW, tmS, tmZ;
+  bool ok = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, kTcBM, kTcBK,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, L::MP, 64,
+            encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, kTcBK, kTcBN / 8,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kNTile,
+            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kTcBN,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
-            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kNWords,
+            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kTcBN / 8,
                       CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return PARO_ERR_CUDA;
-  const dim3 grid((unsigned)((N + kNTile - 1) / kNTile), 1, (unsigned)((M + L::MP - 1) / L::MP));
-  auto k = w4_mma_kernel<NT, 1, true>;
-  if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
-  return launch(k, grid, dim3(L::THREADS), L::SMEM, s, pdl, tmW, tmX, tmS, tmZ, bias, y, (int)M,
-                (int)N, (int)K);
+  const dim3 grid((unsigned)((N + kTcBN - 1) / kTcBN), (unsigned)((M + kTcBM - 1) / kTcBM), 1);
+  if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
+  if (!allow_smem(w4_tc_gemm_kernel, TcLayout::SMEM)) return PARO_ERR_CUDA;
+  return launch(w4_tc_gemm_kernel, grid, dim3(kTcThreads), TcLayout::SMEM, s, pdl, tmA, tmW, tmS,
+                tmZ, bias, y, (int)M, (int)N, (int)K);
 }
 
 // Decode GEMV launch: grid (column tiles, splits), one cluster of `splits`
-// CTAs per column tile.  Clusters of 16 need the non-portable opt-in and room
-// for 16 co-resident CTAs in one GPC; if the device cannot run them the split
-// falls back to 8.
-template <int NT>
-int launch_decode(const LinearPlan& plan, const CUtensorMap& tmW, const CUtensorMap& tmX,
-                  const CUtensorMap& tmS, const CUtensorMap& tmZ, const __half* bias, __half* y,
-                  int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
-  using L = MmaLayout<NT, kDecodeKSplit>;
-  auto k = w4_mma_kernel<NT, kDecodeKSplit, false>;
+// CTAs along K per column tile, one CTA per SM.
+template <int NT, int KP>
+int launch_gemv(const LinearPlan& plan, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                const CUtensorMap& tmS, const CUtensorMap& tmZ, const __half* bias, __half* y,
+                int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
+  using L = GemvLayout<NT, KP>;
+  auto k = w4_gemv_kernel<NT, KP>;
   if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
-  int splits = plan.splits;
-  if (splits > 8) {
-    static int ok16 = -1;   // per process; all GPUs of a box are the same part
-    if (ok16 < 0) {
-      ok16 = 0;
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)plan.n_tiles, 16, 1);
-        cfg.blockDim = dim3(L::THREADS);
-        cfg.dynamicSmemBytes = L::SMEM;
-        cudaLaunchAttribute a[1];
-        a[0].id = cudaLaunchAttributeClusterDimension;
-        a[0].val.clusterDim.x = 1;
-        a[0].val.clusterDim.y = 16;
-        a[0].val.clusterDim.z = 1;
-        cfg.attrs = a;
-        cfg.numAttrs = 1;
-        int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, k, &cfg) == cudaSuccess && nclusters > 0)
-          ok16 = 1;
-      }
-      cudaGetLastError();
-    }
-    if (!ok16) splits = 8;
-  }
-  const dim3 grid((unsigned)plan.n_tiles, (unsigned)splits, 1);
-  return launch_ex(k, grid, dim3(L::THREADS), L::SMEM, s, pdl, (unsigned)splits, tmW, tmX, tmS,
-                   tmZ, bias, y, (int)M, (int)N, (int)K);
+  const dim3 grid((unsigned)plan.n_tiles, (unsigned)plan.splits, 1);
+  return launch_ex(k, grid, dim3(L::THREADS), L::SMEM, s, pdl, (unsigned)plan.splits, tmW, tmX,
+                   tmS, tmZ, bias, y, (int)M, (int)N, (int)K);
 }
 
 }  // namespace
@@ -394,19 +367,20 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
 
   CUtensorMap tmW, tmX, tmS, tmZ;
   const int mp = 8 * plan.nt;
-  bool ok = encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, kNWords,
+  bool ok = encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, kGvWords,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, mp, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kNTile,
+            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kGvTile,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
-            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kNWords,
+            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kGvWords,
                       CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return PARO_ERR_CUDA;
-  const __half* bb = b;
-  if (plan.nt == 1)
-    return launch_decode<1>(plan, tmW, tmX, tmS, tmZ, bb, yy, M, N, K, s, pdl);
-  return launch_decode<2>(plan, tmW, tmX, tmS, tmZ, bb, yy, M, N, K, s, pdl);
+  if (plan.nt == 1) {
+    if (plan.kparts == 4) return launch_gemv<1, 4>(plan, tmW, tmX, tmS, tmZ, b, yy, M, N, K, s, pdl);
+    return launch_gemv<1, 2>(plan, tmW, tmX, tmS, tmZ, b, yy, M, N, K, s, pdl);
+  }
+  return launch_gemv<2, 2>(plan, tmW, tmX, tmS, tmZ, b, yy, M, N, K, s, pdl);
 }
 
 }  // extern "C"

@@ -63,7 +63,12 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
     const __half* x, __half* xr, const float* __restrict__ cs,
     const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot) {
   using T = RotTile<ROWS>;
-  // Let a PDL-launched consumer start its own independent prologue now.
+  // Programmatic dependent launch: wait until the previous kernel in the stream
+  // has completed (no input is read before that), then let the GEMV that
+  // follows launch and start streaming its weights while this kernel works.
+  // Triggering only after the wait keeps everything before this kernel complete
+  // by the time the GEMV runs its independent prologue.
+  pdl_wait_primary();
   pdl_launch_dependents();
 
   extern __shared__ __align__(16) unsigned char smem_raw[];

@@ -1,0 +1,288 @@
+// Prefill W4 GEMM on the sm_100a tensor cores (tcgen05 / TMEM), M > 16 token rows.
+//
+// What it computes (GPTQModel wiki page "ParoQuant", "Activation and weight
+// transforms" and "Triton plans and tuning"):
+//   Y[m, n] = sum_k X_r[m, k] * (q[k, n] - z[k/128, n]) * s[k/128, n] + b[n]
+//
+// CTA tile: 128 token rows x 256 output columns, K in blocks of 64.
+//   A = X_r tile [128 tokens][64 k] fp16, K-major, brought by TMA with the
+//       128-byte swizzle (the UMMA canonical K-major SW128 layout).
+//   B = W^T tile [256 columns][64 k] fp16, K-major, written by the dequant warps
+//       from the AWQ words in the canonical no-swizzle layout: 8x8 core matrices
+//       of 128 contiguous bytes, k-chunks 128 B apart (LBO), 8-row groups
+//       1040 B apart (SBO: one extra 16 bytes per group so the dequant stores
+//       of eight neighbouring groups hit eight different bank groups).
+//   D = fp32 accumulator [128 lanes = tokens][256 columns] in tensor memory.
+// Warp roles (10 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
+// single-thread MMA issuer, warps 2..9 = dequant (k-chunk = warp - 2, word column
+// = lane) and then epilogue.  Per pipeline stage: A, the packed qweight tile
+// [64 rows][32 words] (TMA, 128-byte swizzle), the group's scales and zero
+// words, and the dequantised B tile.  Barriers per stage: tma_full (TMA bytes),
+// b_full (8 dequant warps), empty (tcgen05.commit after the stage's MMAs).
+//
+// Dequantisation of one packed word column w for k-chunk c (8 rows): a byte
+// permute of rows (k, k+1) puts both k's of one column in one register;
+// (v & 0x000F000F) | 0x64006400 and (v & 0x00F000F0) | 0x64006400 give the fp16
+// pairs 1024 + q and 1024 + 16 q exactly; subtracting (1024 + z) or (1024 + 16 z)
+// leaves q - z or 16 (q - z) exactly, and multiplying by s or s/16 rounds
+// (q - z) s to fp16 once.  One 16-byte store per column writes its 8 k's.
+#pragma once
+
+#include "common.cuh"
+
+namespace paro {
+
+constexpr int kTcBM = 128;               // token rows per CTA
+constexpr int kTcBN = 256;               // output columns per CTA
+constexpr int kTcBK = 64;                // k per stage (128-byte rows)
+constexpr int kTcStages = 3;
+constexpr int kTcThreads = 320;          // 10 warps
+constexpr int kTcDequantWarps = 8;
+constexpr int kTcBSbo = 1040;            // B: bytes between 8-row groups
+constexpr int kTcBLbo = 128;             // B: bytes between k-chunks
+
+struct TcLayout {
+  static constexpr int A_OFF = 0;                          // 16384 B, 1024-aligned
+  static constexpr int A_BYTES = kTcBM * kTcBK * 2;
+  static constexpr int WQ_OFF = A_OFF + A_BYTES;           // 8192 B, 1024-aligned
+  static constexpr int WQ_BYTES = kTcBK * (kTcBN / 8) * 4;
+  static constexpr int B_OFF = WQ_OFF + WQ_BYTES;          // 33280 B
+  static constexpr int B_BYTES = (kTcBN / 8) * kTcBSbo;
+  static constexpr int S_OFF = B_OFF + B_BYTES;            // 512 B
+  static constexpr int S_BYTES = kTcBN * 2;
+  static constexpr int Z_OFF = S_OFF + S_BYTES;            // 128 B
+  static constexpr int Z_BYTES = (kTcBN / 8) * 4;
+  static constexpr int STAGE = ((Z_OFF + Z_BYTES + 1023) / 1024) * 1024;
+  static constexpr int TX_BYTES = A_BYTES + WQ_BYTES + S_BYTES + Z_BYTES;
+  static constexpr int BAR_OFF = kTcStages * STAGE;        // 3 x 3 mbarriers + 1
+  static constexpr int MISC_OFF = BAR_OFF + 8 * (3 * kTcStages + 1);
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;
+};
+
+// instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M=128, N=256
+constexpr uint32_t kTcIdesc = (1u << 4) | ((uint32_t)(kTcBN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
+
+// Bounded wait that also gives up as soon as another role of the CTA has given up.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      flag_error(kErrTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
+    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
+    const __half* __restrict__ bias, __half* __restrict__ Y, int M, int N, int K) {
+  using L = TcLayout;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t base = smem_u32(sbase);
+  const uint32_t tma_full0 = base + L::BAR_OFF;
+  const uint32_t b_full0 = tma_full0 + 8 * kTcStages;
+  const uint32_t empty0 = b_full0 + 8 * kTcStages;
+  const uint32_t accum_full = empty0 + 8 * kTcStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::MISC_OFF);
+  volatile int* abort = reinterpret_cast<volatile int*>(sbase + L::MISC_OFF + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * kTcBN;
+  const int tok0 = blockIdx.y * kTcBM;
+  const int nk = K / kTcBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(tma_full0 + 8 * s, 1);
+      mbar_init(b_full0 + 8 * s, kTcDequantWarps);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accum_full, 1);
+    *abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmS);
+    tma_prefetch_desc(&tmZ);
+  }
+  if (warp == 1) {                      // the whole warp allocates 256 TMEM columns
+    tmem_alloc(smem_u32(tmem_slot), kTcBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const int pre = min(kTcStages, nk);
+      // weights, scales and zeros do not depend on the previous kernel
+      for (int kb = 0; kb < pre; ++kb) {
+        const uint32_t st = base + kb * L::STAGE, bar = tma_full0 + 8 * kb;
+        mbar_arrive_expect_tx(bar, L::TX_BYTES);
+        tma_load_2d(st + L::WQ_OFF, &tmW, bar, n0 / 8, kb * kTcBK);
+        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, (kb * kTcBK) / 128);
+        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, (kb * kTcBK) / 128);
+      }
+      pdl_wait_primary();               // X_r is written by the rotation kernel
+      for (int kb = 0; kb < pre; ++kb)
+        tma_load_2d(base + kb * L::STAGE + L::A_OFF, &tmA, tma_full0 + 8 * kb, kb * kTcBK, tok0);
+      for (int kb = pre; kb < nk; ++kb) {
+        const int s = kb % kTcStages;
+        if (!tc_wait(empty0 + 8 * s, ((kb / kTcStages) - 1) & 1, abort)) break;
+        const uint32_t st = base + s * L::STAGE, bar = tma_full0 + 8 * s;
+        mbar_arrive_expect_tx(bar, L::TX_BYTES);
+        tma_load_2d(st + L::WQ_OFF, &tmW, bar, n0 / 8, kb * kTcBK);
+        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, (kb * kTcBK) / 128);
+        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, (kb * kTcBK) / 128);
+        tma_load_2d(st + L::A_OFF, &tmA, bar, kb * kTcBK, tok0);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kTcStages;
+        const uint32_t ph = (kb / kTcStages) & 1;
+        if (!tc_wait(tma_full0 + 8 * s, ph, abort)) break;
+        if (!tc_wait(b_full0 + 8 * s, ph, abort)) break;
+        tc_fence_after();
+        const uint32_t a0 = base + s * L::STAGE + L::A_OFF;
+        const uint32_t b0 = base + s * L::STAGE + L::B_OFF;
+#pragma unroll
+        for (int ks = 0; ks < kTcBK / 16; ++ks) {
+          // A: 128-byte swizzled rows, 8-row groups 1024 B apart; +32 B per 16 k
+          const uint64_t ad = umma_desc(a0 + ks * 32, 16, 1024, 2);
+          // B: no swizzle, k-chunks LBO apart, 8-row groups SBO apart; 2 chunks per 16 k
+          const uint64_t bd = umma_desc(b0 + ks * 2 * kTcBLbo, kTcBLbo, kTcBSbo, 0);
+          umma_f16(tmem_d, ad, bd, kTcIdesc, (kb > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(empty0 + 8 * s);    // frees the stage when these MMAs are done
+      }
+      umma_commit(accum_full);          // all MMAs of the tile are done
+    }
+  } else {
+    // ------------------------------------------------------------ dequant warps
+    const int c = warp - 2;             // k-chunk: rows 8c .. 8c+7 of the stage
+    const int w = lane;                 // packed word column: output columns 8w .. 8w+7
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kTcStages;
+      const uint32_t ph = (kb / kTcStages) & 1;
+      if (!tc_wait(tma_full0 + 8 * s, ph, abort)) break;
+      if (kb >= kTcStages && !tc_wait(empty0 + 8 * s, ph ^ 1, abort)) break;
+      unsigned char* stp = sbase + s * L::STAGE;
+      // 8 words of rows 8c..8c+7, word column w (128-byte swizzled rows)
+      uint32_t wv[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int row = 8 * c + r;
+        wv[r] = *reinterpret_cast<const uint32_t*>(stp + L::WQ_OFF + row * 128 +
+                                                   ((((w >> 2) ^ (row & 7))) << 4) + (w & 3) * 4);
+      }
+      // group zero points and scales of the 8 columns (column j at nibble j/2 + 4 (j & 1))
+      const uint32_t zw = *reinterpret_cast<const uint32_t*>(stp + L::Z_OFF + w * 4);
+      const uint4 s8 = *reinterpret_cast<const uint4*>(stp + L::S_OFF + w * 16);
+      const uint32_t sw[4] = {s8.x, s8.y, s8.z, s8.w};
+      uint32_t outv[8][4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        uint32_t elo[4], ehi[4];
+        const uint32_t mlo = prmt(wv[2 * p], wv[2 * p + 1], 0x5410);
+        const uint32_t mhi = prmt(wv[2 * p], wv[2 * p + 1], 0x7632);
+        const uint32_t mlo8 = mlo >> 8, mhi8 = mhi >> 8;
+        elo[0] = and_or(mlo, 0x000F000Fu, 0x64006400u);
+        elo[1] = and_or(mlo, 0x00F000F0u, 0x64006400u);
+        elo[2] = and_or(mlo8, 0x000F000Fu, 0x64006400u);
+        elo[3] = and_or(mlo8, 0x00F000F0u, 0x64006400u);
+        ehi[0] = and_or(mhi, 0x000F000Fu, 0x64006400u);
+        ehi[1] = and_or(mhi, 0x00F000F0u, 0x64006400u);
+        ehi[2] = and_or(mhi8, 0x000F000Fu, 0x64006400u);
+        ehi[3] = and_or(mhi8, 0x00F000F0u, 0x64006400u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          outv[2 * j][p] = elo[j];        // column 2j   (nibble j)
+          outv[2 * j + 1][p] = ehi[j];    // column 2j+1 (nibble j + 4)
+        }
+      }
+#pragma unroll
+      for (int col = 0; col < 8; ++col) {
+        const int j = col >> 1;
+        const int nib = j + 4 * (col & 1);
+        const uint32_t sh = (j & 1) ? 4u : 0u;
+        const uint32_t z = ((zw >> (4 * nib)) & 0xFu) << sh;
+        const uint32_t zz = (z | (z << 16)) | 0x64006400u;
+        uint32_t sc = prmt(sw[j], sw[j], (col & 1) ? 0x3232 : 0x1010);   // (s, s)
+        if (j & 1) sc = hmul2_u32(sc, 0x2C002C00u);                      // s / 16
+        uint4 o;
+        o.x = hmul2_u32(hsub2_u32(outv[col][0], zz), sc);
+        o.y = hmul2_u32(hsub2_u32(outv[col][1], zz), sc);
+        o.z = hmul2_u32(hsub2_u32(outv[col][2], zz), sc);
+        o.w = hmul2_u32(hsub2_u32(outv[col][3], zz), sc);
+        *reinterpret_cast<uint4*>(stp + L::B_OFF + w * kTcBSbo + c * kTcBLbo + col * 16) = o;
+      }
+      fence_proxy_async_smem();         // make the B tile visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_full0 + 8 * s);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    // warp w reads TMEM lanes 32*(w%4) .. +31 (its token rows); warps 2..5 take
+    // columns 0..127, warps 6..9 columns 128..255.
+    pdl_wait_primary();                 // previous kernels are complete before Y is written
+    const bool ok = tc_wait(accum_full, 0, abort);
+    tc_fence_after();
+    const int quarter = warp & 3;
+    const int chalf = (warp - 2) >> 2;
+    const int tok = tok0 + 32 * quarter + lane;
+    if (ok) {
+#pragma unroll 1
+      for (int cb = 0; cb < 4; ++cb) {
+        const int col0 = chalf * 128 + cb * 32;
+        uint32_t r[32];
+        tmem_ld32(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)col0, r);
+        tmem_ld_wait();
+        const int n = n0 + col0;
+        if (tok < M && n < N) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]);
+            if (bias != nullptr) {      // bias is only 4-byte aligned: half2 loads
+              const __half2* bh = reinterpret_cast<const __half2*>(bias + n + 8 * q);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(bh[e]);
+                v[2 * e] += f.x;
+                v[2 * e + 1] += f.y;
+              }
+            }
+            uint4 o;
+            __half2* oh = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) oh[e] = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+            *reinterpret_cast<uint4*>(Y + (size_t)tok * N + n + 8 * q) = o;
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, kTcBN);
+  }
+}
+
+}  // namespace paro
