@@ -22,7 +22,7 @@ using namespace paro;
 namespace {
 
 constexpr int kMaxDecodeM = 16;      // M <= 16: split-K GEMV path
-constexpr int kDecodeTargetCtas = 148;   // one decode CTA per SM
+constexpr int kDecodeTargetCtas = 296;   // two decode CTAs per SM
 constexpr int kMaxSplits = 8;         // cluster size along K (portable maximum)
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -175,9 +175,9 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
 struct LinearPlan {
   bool decode = false;
   int nt = 1;              // decode: 8-token MMA tiles per CTA
-  int n_tiles = 0;         // 256-column tiles
+  int n_tiles = 0;         // decode column tiles
   int splits = 1;          // decode split-K factor = cluster size along K
-  int kparts = 2;          // decode consumer warp sets per CTA
+  int variant = 0;         // decode kernel configuration (tile, k-parts, stages)
   size_t off_xr = 0, total = 0;
 };
 
@@ -198,17 +198,28 @@ int check_linear_shape(int64_t M, int64_t K, int64_t N, int group_size) {
 LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
   LinearPlan p;
   const int groups = (int)(K / kGroup);
-  p.n_tiles = (int)((N + kGvTile - 1) / kGvTile);
   p.decode = M <= kMaxDecodeM;
   p.off_xr = 0;
   p.total = round_up((size_t)M * K * 2, 256);   // X_r, written when rotating
   if (p.decode) {
     p.nt = M <= 8 ? 1 : 2;
+    // Configuration by shape class, from a sweep on B200 over the Llama-3-8B
+    // decode shapes (column tile, k-parts, stages, split along K):
+    //   wide (N > 4096, e.g. gate/up):      256 columns, 2 k-parts, 4-stage ring, split 2
+    //   deep (N <= 4096, K > 4096, down):   128 columns, 2 k-parts, 4-stage ring, split 8
+    //   square/narrow (q, o, k, v):         128 columns, 4 k-parts, 8 stages, split 4 (8 if N <= 2048)
+    int tile, want;
+    if (N > 4096) {
+      tile = 256; p.variant = 0; want = 2;
+    } else if (K > 4096) {
+      tile = 128; p.variant = 3; want = 8;
+    } else {
+      tile = 128; p.variant = 2; want = N <= 2048 ? 8 : 4;
+    }
+    p.n_tiles = (int)((N + tile - 1) / tile);
     int s = 1;
-    while (s * 2 <= kMaxSplits && s * 2 <= groups && p.n_tiles * s * 2 <= kDecodeTargetCtas) s *= 2;
+    while (s * 2 <= want && s * 2 <= kMaxSplits && s * 2 <= groups && p.n_tiles * s * 2 <= kDecodeTargetCtas) s *= 2;
     p.splits = s;
-    const int per_cta = (groups + s - 1) / s;
-    p.kparts = (per_cta <= 4 && p.nt == 1) ? 4 : 2;   // more warps when each has few groups
   }
   return p;
 }
@@ -235,17 +246,38 @@ int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t
 }
 
 // Decode GEMV launch: grid (column tiles, splits), one cluster of `splits`
-// CTAs along K per column tile, one CTA per SM.
-template <int NT, int KP>
-int launch_gemv(const LinearPlan& plan, const CUtensorMap& tmW, const CUtensorMap& tmX,
-                const CUtensorMap& tmS, const CUtensorMap& tmZ, const __half* bias, __half* y,
+// CTAs along K per column tile.
+template <int NT, int KP, int NTILE, int STAGES>
+int launch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
+                const void* scales, const CUtensorMap& tmX, const __half* bias, __half* y,
                 int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
-  using L = GemvLayout<NT, KP>;
-  auto k = w4_gemv_kernel<NT, KP>;
+  using L = GemvLayout<NT, KP, NTILE, STAGES>;
+  CUtensorMap tmW, tmS, tmZ;
+  const bool ok =
+      encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, L::WORDS,
+                L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) &&
+      encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, NTILE,
+                CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, L::WORDS,
+                CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return PARO_ERR_CUDA;
+  auto k = w4_gemv_kernel<NT, KP, NTILE, STAGES>;
   if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
-  const dim3 grid((unsigned)plan.n_tiles, (unsigned)plan.splits, 1);
+  const dim3 grid((unsigned)((N + NTILE - 1) / NTILE), (unsigned)plan.splits, 1);
   return launch_ex(k, grid, dim3(L::THREADS), L::SMEM, s, pdl, (unsigned)plan.splits, tmW, tmX,
                    tmS, tmZ, bias, y, (int)M, (int)N, (int)K);
+}
+
+template <int NT>
+int dispatch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
+                  const void* scales, const CUtensorMap& tmX, const __half* bias, __half* y,
+                  int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
+  switch (plan.variant) {
+    case 0: return launch_gemv<NT, 2, 256, 4>(plan, qweight, qzeros, scales, tmX, bias, y, M, N, K, s, pdl);
+    case 1: return launch_gemv<NT, 2, 256, 8>(plan, qweight, qzeros, scales, tmX, bias, y, M, N, K, s, pdl);
+    case 2: return launch_gemv<NT, 4, 128, 8>(plan, qweight, qzeros, scales, tmX, bias, y, M, N, K, s, pdl);
+    default: return launch_gemv<NT, 2, 128, 4>(plan, qweight, qzeros, scales, tmX, bias, y, M, N, K, s, pdl);
+  }
 }
 
 }  // namespace
@@ -365,22 +397,13 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
     return launch_w4_prefill(xa, yy, M, K, N, qweight, qzeros, static_cast<const __half*>(scales),
                              b, s, pdl);
 
-  CUtensorMap tmW, tmX, tmS, tmZ;
+  CUtensorMap tmX;
   const int mp = 8 * plan.nt;
-  bool ok = encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, kGvWords,
-                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, mp, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kGvTile,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
-            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kGvWords,
-                      CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (!ok) return PARO_ERR_CUDA;
-  if (plan.nt == 1) {
-    if (plan.kparts == 4) return launch_gemv<1, 4>(plan, tmW, tmX, tmS, tmZ, b, yy, M, N, K, s, pdl);
-    return launch_gemv<1, 2>(plan, tmW, tmX, tmS, tmZ, b, yy, M, N, K, s, pdl);
-  }
-  return launch_gemv<2, 2>(plan, tmW, tmX, tmS, tmZ, b, yy, M, N, K, s, pdl);
+  if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, mp, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return PARO_ERR_CUDA;
+  if (plan.nt == 1) return dispatch_gemv<1>(plan, qweight, qzeros, scales, tmX, b, yy, M, N, K, s, pdl);
+  return dispatch_gemv<2>(plan, qweight, qzeros, scales, tmX, b, yy, M, N, K, s, pdl);
 }
 
 }  // extern "C"

@@ -32,40 +32,47 @@
 // in fp32, then times the group scale (s / 16 for odd j, an exact power of two).
 //
 // Split-K: the S CTAs that share an output tile form a thread-block cluster
-// along K; each leaves its fp32 partial tile in shared memory and CTA r sums
-// columns [r*256/S, (r+1)*256/S) over the S partials through distributed shared
-// memory, in split order, adds the bias and writes fp16 Y.  No global scratch,
-// no atomics, deterministic.
+// along K.  CTA r owns columns [r*NTILE/S, (r+1)*NTILE/S): every CTA pushes its
+// fp32 partial of each slice into the owner's inbox (a dedicated shared-memory
+// area, one slot per sender) with distributed-shared-memory stores; after one
+// cluster barrier each owner sums its inbox in sender order, adds the bias and
+// writes fp16 Y.  No global scratch, no atomics, deterministic.
 #pragma once
 
 #include "common.cuh"
 
 namespace paro {
 
-constexpr int kGvTile = 256;           // output columns per CTA
-constexpr int kGvWords = kGvTile / 8;  // packed words per qweight row segment
-constexpr int kGvStages = 6;
+constexpr int kGvMaxStages = 8;
 constexpr uint32_t kGvMagic = 0x64006400u;  // fp16 pair (1024, 1024)
 constexpr uint32_t kGvOnes = 0x3C003C00u;   // fp16 pair (1, 1)
 
-template <int NT, int KP>
+// NTILE output columns per CTA (64 per column-slice warp), KP k-parts, STAGES
+// groups in flight.
+template <int NT, int KP, int NTILE, int STAGES>
 struct GemvLayout {
-  static constexpr int THREADS = 32 * (1 + 4 * KP);
+  static constexpr int CSL = NTILE / 64;                  // column-slice warps per k-part
+  static constexpr int WORDS = NTILE / 8;                 // packed words per row segment
+  static constexpr int THREADS = 32 * (1 + CSL * KP);
   static constexpr int MP = 8 * NT;                       // token rows per CTA
-  static constexpr int W_BYTES = 128 * kGvWords * 4;      // 16 KB
+  static constexpr int W_BYTES = 128 * WORDS * 4;         // one group of qweight
   static constexpr int X_BYTES = 2 * MP * 128;            // two 64-column boxes
-  static constexpr int S_BYTES = kGvTile * 2;
-  static constexpr int Z_BYTES = kGvWords * 4;
+  static constexpr int S_BYTES = NTILE * 2;
+  static constexpr int Z_BYTES = WORDS * 4;
   static constexpr int X_OFF = W_BYTES;
   static constexpr int S_OFF = X_OFF + ((X_BYTES + 1023) / 1024) * 1024;
   static constexpr int Z_OFF = S_OFF + S_BYTES;
   static constexpr int STAGE = ((Z_OFF + Z_BYTES + 1023) / 1024) * 1024;
-  static constexpr int WSZ_BYTES = W_BYTES + S_BYTES + Z_BYTES;
-  static constexpr int TX_BYTES = WSZ_BYTES + X_BYTES;
-  static constexpr int RED_BYTES = KP * MP * kGvTile * 4;   // k-part partial tiles
-  static constexpr int BAR_OFF = kGvStages * STAGE;         // full[], empty[] mbarriers
-  static constexpr int SMEM = BAR_OFF + 16 * kGvStages + 1024;
-  static_assert(RED_BYTES <= kGvStages * STAGE, "reduction tiles must fit in stage memory");
+  static constexpr int TX_BYTES = W_BYTES + S_BYTES + Z_BYTES + X_BYTES;
+  static constexpr int RED_BYTES = KP * MP * NTILE * 4;     // k-part partial tiles
+  static constexpr int INBOX_OFF = STAGES * STAGE;          // split-K inbox [S][MP][NTILE/S]
+  static constexpr int INBOX_BYTES = MP * NTILE * 4;
+  static constexpr int BAR_OFF = INBOX_OFF + INBOX_BYTES;   // full[], empty[] mbarriers
+  static constexpr int SMEM = BAR_OFF + 16 * STAGES + 1024;
+  static_assert(RED_BYTES <= STAGES * STAGE, "reduction tiles must fit in stage memory");
+  static_assert(STAGES <= kGvMaxStages, "too many stages");
+  // 128-byte swizzle needs 128-byte rows; 64-byte rows use the 64-byte swizzle
+  static constexpr int ROW_BYTES = WORDS * 4;
 };
 
 __device__ __forceinline__ void gv_unpack4(uint32_t m, uint32_t (&e)[4]) {
@@ -76,12 +83,14 @@ __device__ __forceinline__ void gv_unpack4(uint32_t m, uint32_t (&e)[4]) {
   e[3] = and_or(m8, 0x00F000F0u, kGvMagic);
 }
 
-template <int NT, int KP>
-__global__ void __launch_bounds__(32 * (1 + 4 * KP), 1) w4_gemv_kernel(
+template <int NT, int KP, int NTILE, int STAGES>
+__global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP)) w4_gemv_kernel(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
     const __half* __restrict__ bias, __half* __restrict__ Y, int M, int N, int K) {
-  using L = GemvLayout<NT, KP>;
+  using L = GemvLayout<NT, KP, NTILE, STAGES>;
+  constexpr int kGvStages = STAGES;
+  constexpr int kGvTile = NTILE;
   // The next kernel in the stream may launch now; it waits for our completion
   // before it touches anything we read or write.
   pdl_launch_dependents();
@@ -104,7 +113,7 @@ __global__ void __launch_bounds__(32 * (1 + 4 * KP), 1) w4_gemv_kernel(
   if (tid == 0) {
     for (int s = 0; s < kGvStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 4);       // the 4 column-slice warps of one k-part
+      mbar_init(empty0 + 8 * s, L::CSL);  // the column-slice warps of one k-part
     }
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
@@ -122,7 +131,7 @@ __global__ void __launch_bounds__(32 * (1 + 4 * KP), 1) w4_gemv_kernel(
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][nt][e] = 0.f;
   const int cw = warp - 1;                 // consumer index (warp 0 produces)
-  const int cslice = cw & 3, kpart = cw >> 2;
+  const int cslice = cw % L::CSL, kpart = cw / L::CSL;
   const int g = lane >> 2, t = lane & 3;
   const int wcol = 8 * cslice + g;
 
@@ -164,8 +173,11 @@ __global__ void __launch_bounds__(32 * (1 + 4 * KP), 1) w4_gemv_kernel(
     // Swizzled offsets that do not change from group to group.  qweight rows
     // 16 ks + 2t + {0, 1, 8, 9} have (row & 7) = 2t + {0, 1, 0, 1}.
     const int wchunk = wcol >> 2, wword = (wcol & 3) * 4;
-    const uint32_t wo0 = (uint32_t)((2 * t) * 128 + ((wchunk ^ (2 * t)) << 4) + wword);
-    const uint32_t wo1 = (uint32_t)((2 * t + 1) * 128 + ((wchunk ^ (2 * t + 1)) << 4) + wword);
+    constexpr int RB = L::ROW_BYTES;
+    // 128-byte rows: chunk ^ (row & 7); 64-byte rows (64-byte swizzle): chunk ^ ((row >> 1) & 3)
+    auto swz = [&](int row) -> int { return RB == 128 ? (row & 7) : ((row >> 1) & 3); };
+    const uint32_t wo0 = (uint32_t)((2 * t) * RB + ((wchunk ^ swz(2 * t)) << 4) + wword);
+    const uint32_t wo1 = (uint32_t)((2 * t + 1) * RB + ((wchunk ^ swz(2 * t + 1)) << 4) + wword);
     // X_r tile: token rows of 128 B per 64-column box; columns 16 ks + 2t (+8)
     // sit in 16-byte chunk 2 (ks & 3) (+1), swizzled with (token & 7).
     uint32_t xo[4][NT][2];
@@ -192,11 +204,11 @@ __global__ void __launch_bounds__(32 * (1 + 4 * KP), 1) w4_gemv_kernel(
         float rs[NT][4];
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const unsigned char* wrow = stp + ks * 2048;
+          const unsigned char* wrow = stp + ks * 16 * RB;
           const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wrow + wo0);
           const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wrow + wo1);
-          const uint32_t w8 = *reinterpret_cast<const uint32_t*>(wrow + 1024 + wo0);
-          const uint32_t w9 = *reinterpret_cast<const uint32_t*>(wrow + 1024 + wo1);
+          const uint32_t w8 = *reinterpret_cast<const uint32_t*>(wrow + 8 * RB + wo0);
+          const uint32_t w9 = *reinterpret_cast<const uint32_t*>(wrow + 8 * RB + wo1);
           uint32_t b0[NT], b1[NT];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
@@ -273,42 +285,52 @@ __global__ void __launch_bounds__(32 * (1 + 4 * KP), 1) w4_gemv_kernel(
   }
   __syncthreads();
   const int mrows = min(L::MP, M);
-  if (KP > 1) {
-    for (int idx = tid; idx < mrows * kGvTile / 4; idx += L::THREADS) {
-      float4 v = reinterpret_cast<float4*>(red)[idx];
-#pragma unroll
-      for (int kp = 1; kp < KP; ++kp) {
-        const float4 u = reinterpret_cast<const float4*>(red + (size_t)kp * L::MP * kGvTile)[idx];
-        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
-      }
-      reinterpret_cast<float4*>(red)[idx] = v;
-    }
-  }
-
   const int S = gridDim.y;
-  int c_begin = 0, cols = kGvTile;
-  if (S > 1) {
-    cluster_sync();        // every CTA's partial tile is complete and visible
-    cols = kGvTile / S;
-    c_begin = (int)cluster_ctarank() * cols;
-  } else {
-    __syncthreads();
-  }
-  for (int idx = tid; idx < mrows * (cols / 4); idx += L::THREADS) {
-    const int tl = idx / (cols / 4);
-    const int col = c_begin + 4 * (idx % (cols / 4));
+  const int cols = kGvTile / S;                    // columns owned by each CTA of the cluster
+  const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
+  const uint32_t inbox = base + L::INBOX_OFF;
+  // fold the k-parts (fixed order); write Y directly or push to the slice owner
+  for (int idx = tid; idx < mrows * kGvTile / 4; idx += L::THREADS) {
+    float4 v = reinterpret_cast<const float4*>(red)[idx];
+#pragma unroll
+    for (int kp = 1; kp < KP; ++kp) {
+      const float4 u = reinterpret_cast<const float4*>(red + (size_t)kp * L::MP * kGvTile)[idx];
+      v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+    }
+    const int tl = idx / (kGvTile / 4);
+    const int col = 4 * (idx % (kGvTile / 4));
+    if (S > 1) {
+      const int owner = col / cols;
+      const uint32_t off = inbox + (uint32_t)(((int)rank * L::MP + tl) * cols + (col - owner * cols)) * 4u;
+      st_cluster_f4(mapa_shared(off, (uint32_t)owner), v);
+      continue;
+    }
     const int n = n0 + col;
     if (n >= N) continue;
-    float4 sum;
-    if (S > 1) {
-      sum = make_float4(0.f, 0.f, 0.f, 0.f);
-      const uint32_t off = base + (uint32_t)(tl * kGvTile + col) * 4u;
-      for (int q = 0; q < S; ++q) {
-        const float4 v = ld_cluster_f4(mapa_shared(off, (uint32_t)q));
-        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-      }
-    } else {
-      sum = *reinterpret_cast<const float4*>(red + tl * kGvTile + col);
+    if (bias != nullptr) {
+      v.x += __half2float(bias[n]); v.y += __half2float(bias[n + 1]);
+      v.z += __half2float(bias[n + 2]); v.w += __half2float(bias[n + 3]);
+    }
+    const __half2 h0 = __floats2half2_rn(v.x, v.y), h1 = __floats2half2_rn(v.z, v.w);
+    uint2 out;
+    out.x = *reinterpret_cast<const uint32_t*>(&h0);
+    out.y = *reinterpret_cast<const uint32_t*>(&h1);
+    *reinterpret_cast<uint2*>(Y + (size_t)tl * N + n) = out;
+  }
+  if (S == 1) return;
+
+  // every partial pushed into this CTA's inbox is complete and visible after this
+  cluster_sync();
+  const float* box = reinterpret_cast<const float*>(sbase + L::INBOX_OFF);
+  for (int idx = tid; idx < mrows * (cols / 4); idx += L::THREADS) {
+    const int tl = idx / (cols / 4);
+    const int c = 4 * (idx % (cols / 4));
+    const int n = n0 + (int)rank * cols + c;
+    if (n >= N) continue;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < S; ++q) {
+      const float4 v = *reinterpret_cast<const float4*>(box + ((size_t)q * L::MP + tl) * cols + c);
+      sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
     }
     if (bias != nullptr) {
       sum.x += __half2float(bias[n]); sum.y += __half2float(bias[n + 1]);
@@ -320,8 +342,6 @@ __global__ void __launch_bounds__(32 * (1 + 4 * KP), 1) w4_gemv_kernel(
     out.y = *reinterpret_cast<const uint32_t*>(&h1);
     *reinterpret_cast<uint2*>(Y + (size_t)tl * N + n) = out;
   }
-  // keep this CTA's partial tile alive until every CTA of the cluster has read it
-  if (S > 1) cluster_sync();
 }
 
 }  // namespace paro
