@@ -15,10 +15,12 @@
 //   D = fp32 accumulator [128 lanes = tokens][256 columns] in tensor memory.
 // Warp roles (10 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
 // single-thread MMA issuer, warps 2..9 = dequant (k-chunk = warp - 2, word column
-// = lane) and then epilogue.  Per pipeline stage: A, the packed qweight tile
-// [64 rows][32 words] (TMA, 128-byte swizzle), the group's scales and zero
-// words, and the dequantised B tile.  Barriers per stage: tma_full (TMA bytes),
-// b_full (8 dequant warps), empty (tcgen05.commit after the stage's MMAs).
+// = lane) and then epilogue.  Two rings: a 6-deep TMA ring (A, the packed
+// qweight tile [64 rows][32 words] with 128-byte swizzle, the group's scales
+// and zero words) — deep enough to cover the TMA round trip — and a 2-deep ring
+// of dequantised B tiles.  Barriers: tma_full / tma_empty per TMA stage (bytes
+// landed / MMAs done), b_full / b_empty per B buffer (8 dequant warps / MMAs
+// done); tcgen05.commit signals the "empty" ones when the MMAs complete.
 //
 // Dequantisation of one packed word column w for k-chunk c (8 rows): a byte
 // permute of rows (k, k+1) puts both k's of one column in one register;
@@ -35,27 +37,33 @@ namespace paro {
 constexpr int kTcBM = 128;               // token rows per CTA
 constexpr int kTcBN = 256;               // output columns per CTA
 constexpr int kTcBK = 64;                // k per stage (128-byte rows)
-constexpr int kTcStages = 3;
+constexpr int kTcStages = 6;             // TMA ring: A, packed weights, scales, zeros
+constexpr int kTcBBufs = 2;              // dequantised B ring
 constexpr int kTcThreads = 320;          // 10 warps
 constexpr int kTcDequantWarps = 8;
 constexpr int kTcBSbo = 1040;            // B: bytes between 8-row groups
 constexpr int kTcBLbo = 128;             // B: bytes between k-chunks
 
 struct TcLayout {
-  static constexpr int A_OFF = 0;                          // 16384 B, 1024-aligned
+  // TMA stage (1024-aligned): A | packed weights | scales | zeros
+  static constexpr int A_OFF = 0;                          // 16384 B
   static constexpr int A_BYTES = kTcBM * kTcBK * 2;
   static constexpr int WQ_OFF = A_OFF + A_BYTES;           // 8192 B, 1024-aligned
   static constexpr int WQ_BYTES = kTcBK * (kTcBN / 8) * 4;
-  static constexpr int B_OFF = WQ_OFF + WQ_BYTES;          // 33280 B
-  static constexpr int B_BYTES = (kTcBN / 8) * kTcBSbo;
-  static constexpr int S_OFF = B_OFF + B_BYTES;            // 512 B
+  static constexpr int S_OFF = WQ_OFF + WQ_BYTES;          // 512 B
   static constexpr int S_BYTES = kTcBN * 2;
   static constexpr int Z_OFF = S_OFF + S_BYTES;            // 128 B
   static constexpr int Z_BYTES = (kTcBN / 8) * 4;
   static constexpr int STAGE = ((Z_OFF + Z_BYTES + 1023) / 1024) * 1024;
   static constexpr int TX_BYTES = A_BYTES + WQ_BYTES + S_BYTES + Z_BYTES;
-  static constexpr int BAR_OFF = kTcStages * STAGE;        // 3 x 3 mbarriers + 1
-  static constexpr int MISC_OFF = BAR_OFF + 8 * (3 * kTcStages + 1);
+  // dequantised B buffers after the TMA ring
+  static constexpr int B_RING = kTcStages * STAGE;
+  static constexpr int B_BYTES = (kTcBN / 8) * kTcBSbo;   // 33280 B
+  static constexpr int B_STRIDE = ((B_BYTES + 127) / 128) * 128;
+  static constexpr int BAR_OFF = B_RING + kTcBBufs * B_STRIDE;
+  // barriers: tma_full[S], tma_empty[S], b_full[B], b_empty[B], accum_full
+  static constexpr int NBARS = 2 * kTcStages + 2 * kTcBBufs + 1;
+  static constexpr int MISC_OFF = BAR_OFF + 8 * NBARS;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
 };
 
@@ -86,9 +94,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t base = smem_u32(sbase);
   const uint32_t tma_full0 = base + L::BAR_OFF;
-  const uint32_t b_full0 = tma_full0 + 8 * kTcStages;
-  const uint32_t empty0 = b_full0 + 8 * kTcStages;
-  const uint32_t accum_full = empty0 + 8 * kTcStages;
+  const uint32_t tma_empty0 = tma_full0 + 8 * kTcStages;
+  const uint32_t b_full0 = tma_empty0 + 8 * kTcStages;
+  const uint32_t b_empty0 = b_full0 + 8 * kTcBBufs;
+  const uint32_t accum_full = b_empty0 + 8 * kTcBBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::MISC_OFF);
   volatile int* abort = reinterpret_cast<volatile int*>(sbase + L::MISC_OFF + 4);
 
@@ -100,8 +109,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
   if (tid == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       mbar_init(tma_full0 + 8 * s, 1);
-      mbar_init(b_full0 + 8 * s, kTcDequantWarps);
-      mbar_init(empty0 + 8 * s, 1);
+      mbar_init(tma_empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < kTcBBufs; ++b) {
+      mbar_init(b_full0 + 8 * b, kTcDequantWarps);
+      mbar_init(b_empty0 + 8 * b, 1);
     }
     mbar_init(accum_full, 1);
     *abort = 0;
@@ -137,7 +149,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         tma_load_2d(base + kb * L::STAGE + L::A_OFF, &tmA, tma_full0 + 8 * kb, kb * kTcBK, tok0);
       for (int kb = pre; kb < nk; ++kb) {
         const int s = kb % kTcStages;
-        if (!tc_wait(empty0 + 8 * s, ((kb / kTcStages) - 1) & 1, abort)) break;
+        if (!tc_wait(tma_empty0 + 8 * s, ((kb / kTcStages) - 1) & 1, abort)) break;
         const uint32_t st = base + s * L::STAGE, bar = tma_full0 + 8 * s;
         mbar_arrive_expect_tx(bar, L::TX_BYTES);
         tma_load_2d(st + L::WQ_OFF, &tmW, bar, n0 / 8, kb * kTcBK);
@@ -150,13 +162,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % kTcStages;
-        const uint32_t ph = (kb / kTcStages) & 1;
-        if (!tc_wait(tma_full0 + 8 * s, ph, abort)) break;
-        if (!tc_wait(b_full0 + 8 * s, ph, abort)) break;
+        const int s = kb % kTcStages, b = kb % kTcBBufs;
+        if (!tc_wait(tma_full0 + 8 * s, (kb / kTcStages) & 1, abort)) break;
+        if (!tc_wait(b_full0 + 8 * b, (kb / kTcBBufs) & 1, abort)) break;
         tc_fence_after();
         const uint32_t a0 = base + s * L::STAGE + L::A_OFF;
-        const uint32_t b0 = base + s * L::STAGE + L::B_OFF;
+        const uint32_t b0 = base + L::B_RING + b * L::B_STRIDE;
 #pragma unroll
         for (int ks = 0; ks < kTcBK / 16; ++ks) {
           // A: 128-byte swizzled rows, 8-row groups 1024 B apart; +32 B per 16 k
@@ -165,7 +176,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
           const uint64_t bd = umma_desc(b0 + ks * 2 * kTcBLbo, kTcBLbo, kTcBSbo, 0);
           umma_f16(tmem_d, ad, bd, kTcIdesc, (kb > 0 || ks > 0) ? 1u : 0u);
         }
-        umma_commit(empty0 + 8 * s);    // frees the stage when these MMAs are done
+        umma_commit(tma_empty0 + 8 * s);   // the TMA stage and ...
+        umma_commit(b_empty0 + 8 * b);     // ... the B buffer are free once these MMAs finish
       }
       umma_commit(accum_full);          // all MMAs of the tile are done
     }
@@ -174,11 +186,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     const int c = warp - 2;             // k-chunk: rows 8c .. 8c+7 of the stage
     const int w = lane;                 // packed word column: output columns 8w .. 8w+7
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kTcStages;
-      const uint32_t ph = (kb / kTcStages) & 1;
-      if (!tc_wait(tma_full0 + 8 * s, ph, abort)) break;
-      if (kb >= kTcStages && !tc_wait(empty0 + 8 * s, ph ^ 1, abort)) break;
+      const int s = kb % kTcStages, bb = kb % kTcBBufs;
+      if (!tc_wait(tma_full0 + 8 * s, (kb / kTcStages) & 1, abort)) break;
+      if (kb >= kTcBBufs && !tc_wait(b_empty0 + 8 * bb, ((kb / kTcBBufs) - 1) & 1, abort)) break;
       unsigned char* stp = sbase + s * L::STAGE;
+      unsigned char* btile = sbase + L::B_RING + bb * L::B_STRIDE;
       // 8 words of rows 8c..8c+7, word column w (128-byte swizzled rows)
       uint32_t wv[8];
 #pragma unroll
@@ -226,11 +238,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         o.y = hmul2_u32(hsub2_u32(outv[col][1], zz), sc);
         o.z = hmul2_u32(hsub2_u32(outv[col][2], zz), sc);
         o.w = hmul2_u32(hsub2_u32(outv[col][3], zz), sc);
-        *reinterpret_cast<uint4*>(stp + L::B_OFF + w * kTcBSbo + c * kTcBLbo + col * 16) = o;
+        *reinterpret_cast<uint4*>(btile + w * kTcBSbo + c * kTcBLbo + col * 16) = o;
       }
       fence_proxy_async_smem();         // make the B tile visible to the tensor core
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_full0 + 8 * s);
+      if (lane == 0) mbar_arrive(b_full0 + 8 * bb);
     }
 
     // ------------------------------------------------------------ epilogue
