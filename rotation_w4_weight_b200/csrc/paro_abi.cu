@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "pack.cuh"
 #include "rotate.cuh"
+#include "rotate_tmem.cuh"
 #include "w4_gemv.cuh"
 #include "w4_tc.cuh"
 
@@ -143,8 +144,16 @@ int check_rotation_args(const void* x, const void* xr, int64_t M, int64_t K, con
 
 int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
                   const int16_t* pairs, const float* theta, int krot, cudaStream_t stream) {
+  // Large batches: tensor memory as the permutation network, 128 rows per CTA.
+  if (M > 64) {
+    const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + kRtRows - 1) / kRtRows));
+    if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
+    if (!allow_smem(rotate_tmem_kernel, RtLayout::bytes(kMaxKrot))) return PARO_ERR_CUDA;
+    return launch(rotate_tmem_kernel, grid, dim3(kRtThreads), RtLayout::bytes(krot), stream, true,
+                  x, xr, cs, pairs, theta, (int)M, (int)K, krot);
+  }
   // rows per CTA: 4 for decode-sized batches (more CTAs, shorter latency),
-  // 32..128 for large batches (conflict-free 32-row warp accesses)
+  // 32..64 otherwise (conflict-free 32-row warp accesses)
   const int rows = M <= 16 ? 4 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
   const size_t smem = rotate_smem_bytes(rows, krot);
   const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + rows - 1) / rows));

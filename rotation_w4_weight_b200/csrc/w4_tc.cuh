@@ -13,21 +13,21 @@
 //       1040 B apart (SBO: one extra 16 bytes per group so the dequant stores
 //       of eight neighbouring groups hit eight different bank groups).
 //   D = fp32 accumulator [128 lanes = tokens][256 columns] in tensor memory.
-// Warp roles (10 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
-// single-thread MMA issuer, warps 2..9 = dequant (k-chunk = warp - 2, word column
-// = lane) and then epilogue.  Two rings: a 6-deep TMA ring (A, the packed
-// qweight tile [64 rows][32 words] with 128-byte swizzle, the group's scales
-// and zero words) — deep enough to cover the TMA round trip — and a 2-deep ring
-// of dequantised B tiles.  Barriers: tma_full / tma_empty per TMA stage (bytes
+// Warp roles (18 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
+// single-thread MMA issuer, warps 2..17 = dequant (k-chunk (warp-2)/2, 16 word
+// columns, 4 rows per lane) and then epilogue (the first 8 of them).  Two rings: a 4-deep TMA ring (A, the packed qweight tile
+// [64 rows][32 words] with 128-byte swizzle, the group's scales and zero words),
+// deep enough to cover the TMA round trip, and a 3-deep ring of dequantised B
+// tiles so the dequant warps run ahead of the tensor core.  Barriers: tma_full / tma_empty per TMA stage (bytes
 // landed / MMAs done), b_full / b_empty per B buffer (8 dequant warps / MMAs
 // done); tcgen05.commit signals the "empty" ones when the MMAs complete.
 //
-// Dequantisation of one packed word column w for k-chunk c (8 rows): a byte
+// Dequantisation of one packed word column w for 4 rows of k-chunk c: a byte
 // permute of rows (k, k+1) puts both k's of one column in one register;
 // (v & 0x000F000F) | 0x64006400 and (v & 0x00F000F0) | 0x64006400 give the fp16
 // pairs 1024 + q and 1024 + 16 q exactly; subtracting (1024 + z) or (1024 + 16 z)
 // leaves q - z or 16 (q - z) exactly, and multiplying by s or s/16 rounds
-// (q - z) s to fp16 once.  One 16-byte store per column writes its 8 k's.
+// (q - z) s to fp16 once.  One 8-byte store per column writes its 4 k's.
 #pragma once
 
 #include "common.cuh"
@@ -37,10 +37,10 @@ namespace paro {
 constexpr int kTcBM = 128;               // token rows per CTA
 constexpr int kTcBN = 256;               // output columns per CTA
 constexpr int kTcBK = 64;                // k per stage (128-byte rows)
-constexpr int kTcStages = 6;             // TMA ring: A, packed weights, scales, zeros
-constexpr int kTcBBufs = 2;              // dequantised B ring
-constexpr int kTcThreads = 320;          // 10 warps
-constexpr int kTcDequantWarps = 8;
+constexpr int kTcStages = 4;             // TMA ring: A, packed weights, scales, zeros
+constexpr int kTcBBufs = 3;              // dequantised B ring
+constexpr int kTcDequantWarps = 16;      // (k-chunk, half of its 8 rows) per warp
+constexpr int kTcThreads = 32 * (2 + kTcDequantWarps);
 constexpr int kTcBSbo = 1040;            // B: bytes between 8-row groups
 constexpr int kTcBLbo = 128;             // B: bytes between k-chunks
 
@@ -183,19 +183,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     }
   } else {
     // ------------------------------------------------------------ dequant warps
-    const int c = warp - 2;             // k-chunk: rows 8c .. 8c+7 of the stage
-    const int w = lane;                 // packed word column: output columns 8w .. 8w+7
+    // warp (c, wh): k-chunk c (rows 8c .. 8c+7), word columns 16 wh .. 16 wh + 15;
+    // lane (w, h): word column w, rows 8c + 4h .. +3.  Neighbouring lanes differ in
+    // h, so the 8-byte stores of a half-warp land in 16 different 8-byte slots.
+    const int dw = warp - 2;
+    const int c = dw >> 1;
+    const int w = 16 * (dw & 1) + (lane >> 1);   // packed word column: output columns 8w .. 8w+7
+    const int h = lane & 1;
     for (int kb = 0; kb < nk; ++kb) {
       const int s = kb % kTcStages, bb = kb % kTcBBufs;
       if (!tc_wait(tma_full0 + 8 * s, (kb / kTcStages) & 1, abort)) break;
       if (kb >= kTcBBufs && !tc_wait(b_empty0 + 8 * bb, ((kb / kTcBBufs) - 1) & 1, abort)) break;
       unsigned char* stp = sbase + s * L::STAGE;
       unsigned char* btile = sbase + L::B_RING + bb * L::B_STRIDE;
-      // 8 words of rows 8c..8c+7, word column w (128-byte swizzled rows)
-      uint32_t wv[8];
+      // 4 words of rows 8c+4h .. +3, word column w (128-byte swizzled rows)
+      uint32_t wv[4];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int row = 8 * c + r;
+      for (int r = 0; r < 4; ++r) {
+        const int row = 8 * c + 4 * h + r;
         wv[r] = *reinterpret_cast<const uint32_t*>(stp + L::WQ_OFF + row * 128 +
                                                    ((((w >> 2) ^ (row & 7))) << 4) + (w & 3) * 4);
       }
@@ -203,9 +208,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
       const uint32_t zw = *reinterpret_cast<const uint32_t*>(stp + L::Z_OFF + w * 4);
       const uint4 s8 = *reinterpret_cast<const uint4*>(stp + L::S_OFF + w * 16);
       const uint32_t sw[4] = {s8.x, s8.y, s8.z, s8.w};
-      uint32_t outv[8][4];
+      uint32_t outv[8][2];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
+      for (int p = 0; p < 2; ++p) {
         uint32_t elo[4], ehi[4];
         const uint32_t mlo = prmt(wv[2 * p], wv[2 * p + 1], 0x5410);
         const uint32_t mhi = prmt(wv[2 * p], wv[2 * p + 1], 0x7632);
@@ -233,12 +238,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         const uint32_t zz = (z | (z << 16)) | 0x64006400u;
         uint32_t sc = prmt(sw[j], sw[j], (col & 1) ? 0x3232 : 0x1010);   // (s, s)
         if (j & 1) sc = hmul2_u32(sc, 0x2C002C00u);                      // s / 16
-        uint4 o;
+        uint2 o;
         o.x = hmul2_u32(hsub2_u32(outv[col][0], zz), sc);
         o.y = hmul2_u32(hsub2_u32(outv[col][1], zz), sc);
-        o.z = hmul2_u32(hsub2_u32(outv[col][2], zz), sc);
-        o.w = hmul2_u32(hsub2_u32(outv[col][3], zz), sc);
-        *reinterpret_cast<uint4*>(btile + w * kTcBSbo + c * kTcBLbo + col * 16) = o;
+        *reinterpret_cast<uint2*>(btile + w * kTcBSbo + c * kTcBLbo + col * 16 + h * 8) = o;
       }
       fence_proxy_async_smem();         // make the B tile visible to the tensor core
       __syncwarp();
@@ -247,9 +250,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
 
     // ------------------------------------------------------------ epilogue
     // warp w reads TMEM lanes 32*(w%4) .. +31 (its token rows); warps 2..5 take
-    // columns 0..127, warps 6..9 columns 128..255.
+    // columns 0..127, warps 6..9 columns 128..255; warps 10..17 are done.
     pdl_wait_primary();                 // previous kernels are complete before Y is written
-    const bool ok = tc_wait(accum_full, 0, abort);
+    const bool ok = warp < 10 && tc_wait(accum_full, 0, abort);
     tc_fence_after();
     const int quarter = warp & 3;
     const int chalf = (warp - 2) >> 2;
@@ -260,7 +263,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         const int col0 = chalf * 128 + cb * 32;
         uint32_t r[32];
         tmem_ld32(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)col0, r);
-        tmem_ld_wait();
+        tmem_ld_wait_tie(r);
         const int n = n0 + col0;
         if (tok < M && n < N) {
 #pragma unroll

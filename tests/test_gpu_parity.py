@@ -64,6 +64,8 @@ ROT_CASES = [
     (5, 384, 1, True, None),          # krot = 1
     (9, 256, 0, True, None),          # scaling only
     (33, 256, 64, True, None),        # krot at the supported maximum
+    (129, 256, 64, True, None),       # krot maximum on the tensor-memory kernel
+    (65, 384, 1, False, None),        # tensor-memory kernel, krot = 1, ragged tile
     (3, 14336, 8, True, None),        # down_proj width
 ]
 
@@ -81,9 +83,10 @@ def test_rotate_vs_oracle(M, K, krot, use_cs, active):
     assert rot_err(got, ref) <= ROT_TOL
 
 
-def test_rotate_in_place_and_identity_state():
+@pytest.mark.parametrize("M", [40, 200])   # shared-memory and tensor-memory kernels
+def test_rotate_in_place_and_identity_state(M):
     lay = synth.config_layers(0)[0]
-    x = synth.make_activations(lay, 40)
+    x = synth.make_activations(lay, M)
     xt = dev(x)
     pb.rotate(xt, dev(lay.channel_scales), dev(lay.pairs), dev(lay.theta), 128, out=xt)
     ref = oracle.rotate(x, lay.channel_scales, lay.pairs, lay.theta, 128)
@@ -92,6 +95,17 @@ def test_rotate_in_place_and_identity_state():
     got = pb.rotate(dev(x), dev(np.ones(256, np.float32)), dev(lay.pairs),
                     dev(np.zeros_like(lay.theta)), 128)
     assert np.array_equal(got.cpu().numpy(), x)
+
+
+def test_rotate_krot_zero_large_batch_is_scaling_only():
+    lay = synth.config_layers(0)[0]
+    x = synth.make_activations(lay, 300)
+    got = pb.rotate(dev(x), dev(lay.channel_scales), None, None, 128, 0).cpu().numpy()
+    # the kernel's documented arithmetic: fp32 product, one round-to-nearest to fp16
+    ref32 = (x.astype(np.float32) * lay.channel_scales.astype(np.float32)).astype(np.float16)
+    assert np.array_equal(got, ref32)
+    exact = oracle.rotate(x, lay.channel_scales, None, None, 128, krot=0)
+    assert rot_err(got.astype(np.float64), exact) <= ROT_TOL
 
 
 def test_rotate_empty_batch():
