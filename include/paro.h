@@ -190,7 +190,9 @@ int paro_validate_pairs(const int16_t* pairs_host, int64_t K, int group_size, in
  * paro_device_status — reads (and, if clear != 0, resets) the device status word
  * of the current device.  Synchronises the device.  Returns PARO_OK,
  * PARO_ERR_TIMEOUT (a bounded wait ran out), PARO_ERR_INVALID_ARG (a pair index
- * outside its group was seen) or PARO_ERR_CUDA.
+ * outside its group was seen) or PARO_ERR_CUDA (the CUDA query failed, or a
+ * kernel found a device resource laid out other than it requires and skipped
+ * its work).
  */
 int paro_device_status(int clear);
 

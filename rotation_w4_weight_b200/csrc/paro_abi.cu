@@ -65,6 +65,35 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, size_t esize, const voi
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// ---------------------------------------------------------------- device facts
+struct DeviceInfo {
+  int sms = 0;
+  size_t smem_per_sm = 0, smem_reserved_per_block = 0;
+};
+
+// SM count and shared-memory capacity of the current device, queried once per
+// device (entries are never moved, so returned references stay valid).
+const DeviceInfo& device_info() {
+  constexpr int kDevs = 64;
+  static std::mutex mu;
+  static DeviceInfo table[kDevs];
+  static const DeviceInfo none;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) return none;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceInfo& d = table[dev];
+  if (d.sms != 0) return d;
+  int sms = 0, per_sm = 0, reserved = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+    return none;
+  d.smem_per_sm = (size_t)per_sm;
+  d.smem_reserved_per_block = (size_t)reserved;
+  d.sms = sms;
+  return d;
+}
+
 // ---------------------------------------------------------------- launches
 template <typename Kern, typename... Args>
 int launch_ex(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
@@ -100,7 +129,8 @@ int launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
 }
 
 // Raise the dynamic shared memory limit of a kernel once per device (callers
-// pass the largest size the kernel is ever launched with).
+// pass the largest size the kernel is ever launched with) and ask for the
+// largest shared-memory carveout.
 template <typename Kern>
 bool allow_smem(Kern kernel, size_t bytes) {
   int dev = 0;
@@ -113,6 +143,11 @@ bool allow_smem(Kern kernel, size_t bytes) {
     if (d.first == key && d.second == dev) return true;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
       cudaSuccess)
+    return false;
+  // every kernel here stages its operands in shared memory: prefer the largest carveout
+  // (occupancy queries then see the configuration the launches get)
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
     return false;
   done.emplace_back(key, dev);
   return true;
@@ -144,13 +179,39 @@ int check_rotation_args(const void* x, const void* xr, int64_t M, int64_t K, con
 
 int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
                   const int16_t* pairs, const float* theta, int krot, cudaStream_t stream) {
-  // Large batches: tensor memory as the permutation network, 128 rows per CTA.
+  // Large batches: tensor memory as the permutation network; CTAs stay resident
+  // over several 128-row tiles of one group (one wave of at most 2 CTAs per SM:
+  // the shared-memory floor of the kernel guarantees no more fit).
   if (M > 64) {
-    const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + kRtRows - 1) / kRtRows));
-    if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
-    if (!allow_smem(rotate_tmem_kernel, RtLayout::bytes(kMaxKrot))) return PARO_ERR_CUDA;
-    return launch(rotate_tmem_kernel, grid, dim3(kRtThreads), RtLayout::bytes(krot), stream, true,
-                  x, xr, cs, pairs, theta, (int)M, (int)K, krot);
+    const size_t smem = RtLayout::bytes(krot);
+    const DeviceInfo& di = device_info();
+    if (di.sms == 0) return PARO_ERR_CUDA;
+    const bool abs_tables = krot <= kRtAbsMaxKrot;
+    if (abs_tables ? !allow_smem(rotate_tmem_kernel<true>, RtLayout::bytes(kRtAbsMaxKrot))
+                   : !allow_smem(rotate_tmem_kernel<false>, RtLayout::bytes(kMaxKrot)))
+      return PARO_ERR_CUDA;
+    const size_t per_block = smem + di.smem_reserved_per_block;
+    int per_sm = (int)(di.smem_per_sm / per_block);
+    per_sm = per_sm < 1 ? 1 : (per_sm > kRtMaxCtasPerSm ? kRtMaxCtasPerSm : per_sm);
+    // one wave: gridDim.y row-tile slots per group, then as few tiles per CTA
+    // as that allows, spread evenly
+    const int64_t groups = K / kGroup, ntiles = (M + kRtRows - 1) / kRtRows;
+    const int64_t slots = (int64_t)di.sms * per_sm;
+    int64_t gy = slots / groups;
+    gy = gy < 1 ? 1 : (gy > ntiles ? ntiles : gy);
+    const int64_t per_cta = (ntiles + gy - 1) / gy;
+    gy = (ntiles + per_cta - 1) / per_cta;
+    if (gy > 65535) gy = 65535;
+    CUtensorMap tmX;
+    if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, kRtRows, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return PARO_ERR_CUDA;
+    const dim3 grid((unsigned)groups, (unsigned)gy);
+    if (abs_tables)
+      return launch(rotate_tmem_kernel<true>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
+                    pairs, theta, (int)M, (int)K, krot);
+    return launch(rotate_tmem_kernel<false>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
+                  pairs, theta, (int)M, (int)K, krot);
   }
   // rows per CTA: 4 for decode-sized batches (more CTAs, shorter latency),
   // 32..64 otherwise (conflict-free 32-row warp accesses)
@@ -490,6 +551,7 @@ int paro_device_status(int clear) {
   }
   if (v & kErrTimeout) return PARO_ERR_TIMEOUT;
   if (v & kErrPairIndex) return PARO_ERR_INVALID_ARG;
+  if (v & kErrInternal) return PARO_ERR_CUDA;
   return PARO_OK;
 }
 

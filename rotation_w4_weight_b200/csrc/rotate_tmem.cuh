@@ -7,19 +7,32 @@
 // order, pair indices local to the 128-channel group, fp32 on chip, one
 // round-to-nearest to fp16 at the end.
 //
-// A CTA of 4 warps owns one group of 128 token rows: thread t holds row t, i.e.
-// TMEM lane t, 128 fp32 columns.  A stage needs, in every row, the two channels
-// of each pair side by side; registers cannot be indexed by a runtime pair
-// table, but a tcgen05.ld of one column per lane takes a warp-uniform column
-// address.  So each stage gathers its 128 operands in pair order (128 one-column
-// loads), rotates them in registers with compile-time register indices, and
-// writes the 128 results back in that pair order with bulk stores; the next
-// stage's gather addresses are composed with that order once per CTA, in a
-// shared-memory table.  The last stage scatters to
-// the natural channel order instead, and a bulk load brings the row back.
-// Tensor memory is split between the four SM sub-partitions, so the data
-// movement of a stage no longer funnels through the single shared-memory pipe
-// that bounds rotate_kernel.
+// A CTA owns one 128-channel group and walks over 128-row tiles (blockIdx.y,
+// blockIdx.y + gridDim.y, ...), so its stage tables are built once.  Row t of a
+// tile lives in TMEM lane t; the 8 warps are (lane quadrant, half of the pairs).
+// A stage needs, in every row, the two channels of each pair side by side;
+// registers cannot be indexed by a runtime pair table, but a tcgen05.ld of one
+// column per lane takes a warp-uniform column address.  So a warp gathers the
+// 64 operands of its 32 pairs (one-column loads), rotates them in registers at
+// compile-time register indices, and writes the results with bulk stores in
+// that "slot" order into the other of two 128-column buffers; the next stage's
+// gather table is composed with that order.  The two warps of a lane quadrant
+// meet at a named barrier once per stage.  The last stage scatters to the
+// natural channel order and bulk loads bring each warp's half row back.
+// Tensor memory is split between the SM sub-partitions, so a stage's data
+// movement does not funnel through the one shared-memory pipe that bounds
+// rotate_kernel.
+//
+// Slot order of a stage: pairs 2u and 2u+1 form unit u, whose four slots hold
+// (a_2u, a_2u+1, b_2u, b_2u+1), so a unit is rotated with packed fp32x2
+// multiplies and fmas: A' = A*C + B*S, B' = A*(-S) + B*C, A = (a_2u, a_2u+1).
+//
+// With ABS the gather tables hold absolute TMEM addresses, one copy per lane
+// quadrant, so a gather is a quarter of a table read and one load; without it
+// (many stages) one table of columns is offset by the quadrant's lane base.
+// Input tiles arrive by TMA (two 64-channel boxes, 128-byte swizzle, so the
+// row-per-thread reads are conflict-free) into two buffers, two tiles ahead of
+// use.
 #pragma once
 
 #include "rotate.cuh"
@@ -27,194 +40,305 @@
 namespace paro {
 
 constexpr int kRtRows = 128;
-constexpr int kRtThreads = 128;
-constexpr int kRtCols = 128;             // TMEM columns per CTA (one fp32 per channel)
-constexpr int kRtMinSmem = 48 * 1024;    // at most 4 CTAs (4 x 128 TMEM columns) per SM
+constexpr int kRtThreads = 256;          // 8 warps: (lane quadrant, pair half)
+constexpr int kRtCols = 256;             // two 128-column buffers
+constexpr int kRtMaxCtasPerSm = 2;       // 2 x 256 TMEM columns
+constexpr int kRtAbsMaxKrot = 16;        // per-quadrant address tables up to this many stages
+constexpr size_t kRtMinSmem = 80 * 1024; // above a third of an SM's shared memory: <= 2 CTAs/SM
 
 struct RtLayout {
-  // float2 (cos, sin)[krot][64] | uint32 gather column[krot][128] | int pos[2][128] |
-  // uint32 final scatter column[128] | tmem slot
-  __host__ __device__ static size_t cs_off() { return 0; }
-  __host__ __device__ static size_t gather_off(int krot) { return (size_t)krot * 64 * 8; }
-  __host__ __device__ static size_t pos_off(int krot) { return gather_off(krot) + (size_t)krot * 128 * 4; }
-  __host__ __device__ static size_t fin_off(int krot) { return pos_off(krot) + 2 * 128 * 4; }
-  __host__ __device__ static size_t slot_off(int krot) { return fin_off(krot) + 128 * 4; }
-  __host__ __device__ static size_t bytes(int krot) {
-    const size_t b = slot_off(krot) + 16;
-    return b < (size_t)kRtMinSmem ? (size_t)kRtMinSmem : b;
+  // IN tiles[2] | scale[128] | per stage (c0,c1,s0,s1)[32 units] |
+  // gather addresses[Q][krot][128] | scatter addresses[Q][128] | raw pairs[krot][64] |
+  // pos[128] | mbarriers[2] | tmem slot, abort flag
+  // (Q = 4 lane quadrants for up to kRtAbsMaxKrot stages, else 1 table of columns)
+  static constexpr size_t TILE = (size_t)kRtRows * 128 * 2;      // two 64-channel boxes
+  static constexpr size_t BOX = TILE / 2;
+  static constexpr size_t CS_STAGE = 32 * 16;
+  __host__ __device__ static constexpr int copies(int krot) { return krot <= kRtAbsMaxKrot ? 4 : 1; }
+  __host__ __device__ static constexpr size_t scale_off() { return 2 * TILE; }
+  __host__ __device__ static constexpr size_t cs_off() { return scale_off() + 128 * 4; }
+  __host__ __device__ static constexpr size_t g_off(int krot) { return cs_off() + (size_t)krot * CS_STAGE; }
+  __host__ __device__ static constexpr size_t f_off(int krot) {
+    return g_off(krot) + (size_t)copies(krot) * krot * 128 * 4;
+  }
+  __host__ __device__ static constexpr size_t praw_off(int krot) { return f_off(krot) + (size_t)copies(krot) * 128 * 4; }
+  __host__ __device__ static constexpr size_t pos_off(int krot) { return praw_off(krot) + (size_t)krot * 64 * 4; }
+  __host__ __device__ static constexpr size_t bar_off(int krot) { return pos_off(krot) + 128 * 4; }
+  __host__ __device__ static constexpr size_t slot_off(int krot) { return bar_off(krot) + 16; }
+  // + 1 KB so the tiles can be aligned to the 1024 bytes the swizzle pattern needs
+  __host__ __device__ static constexpr size_t bytes(int krot) {
+    return slot_off(krot) + 16 + 1024 < kRtMinSmem ? kRtMinSmem : slot_off(krot) + 16 + 1024;
   }
 };
 
-__global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
-    const __half* x, __half* xr, const float* __restrict__ cs, const int16_t* __restrict__ pairs,
-    const float* __restrict__ theta, int M, int K, int krot) {
-  // Wait for the previous kernel before reading any input, then let the GEMM
-  // that follows start streaming its weights (see rotate_kernel).
-  pdl_wait_primary();
-  pdl_launch_dependents();
+// The two warps of lane quadrant qd: their TMEM accesses so far are complete
+// and visible to each other.  Barrier ids are immediates (5 hardware barriers).
+__device__ __forceinline__ void rt_quadrant_sync(int qd) {
+  tmem_st_wait();
+  tc_fence_before();
+  switch (qd) {
+    case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+    case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+    case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+    default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+  }
+  tc_fence_after();
+}
 
+// grid: (K/128, row-tile slots), block 256.  tmX is x as [M, K] fp16 with box
+// {64 channels, 128 rows}, 128-byte swizzle (rows past M read as zeros).
+template <bool ABS>
+__global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
+    const __grid_constant__ CUtensorMap tmX, __half* xr, const float* __restrict__ cs,
+    const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot) {
+  using L = RtLayout;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float2* cstab = reinterpret_cast<float2*>(smem_raw + RtLayout::cs_off());
-  uint32_t* gather = reinterpret_cast<uint32_t*>(smem_raw + RtLayout::gather_off(krot));
-  int* pos = reinterpret_cast<int*>(smem_raw + RtLayout::pos_off(krot));
-  uint32_t* fin = reinterpret_cast<uint32_t*>(smem_raw + RtLayout::fin_off(krot));
-  uint32_t* slot = reinterpret_cast<uint32_t*>(smem_raw + RtLayout::slot_off(krot));
+  unsigned char* const sb = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t in_base = smem_u32(sb);
+  float* scale = reinterpret_cast<float*>(sb + L::scale_off());
+  unsigned char* cstab = sb + L::cs_off();
+  uint32_t* gtab = reinterpret_cast<uint32_t*>(sb + L::g_off(krot));
+  uint32_t* ftab = reinterpret_cast<uint32_t*>(sb + L::f_off(krot));
+  uint32_t* praw = reinterpret_cast<uint32_t*>(sb + L::praw_off(krot));
+  int* pos = reinterpret_cast<int*>(sb + L::pos_off(krot));
+  const uint32_t bar0 = smem_u32(sb + L::bar_off(krot));
+  uint32_t* slot = reinterpret_cast<uint32_t*>(sb + L::slot_off(krot));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(slot + 1);
 
   const int grp = blockIdx.x;
-  const int row0 = blockIdx.y * kRtRows;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, h = warp >> 2;            // lane quadrant, pair half
+  const int ntiles = (M + kRtRows - 1) / kRtRows;
+  const int gy = (int)gridDim.y;
 
+  // Wait for the previous kernel before reading any input.  Tensor memory is
+  // taken before dependents may launch: a dependent GEMM that allocates TMEM
+  // early can then never hold what this kernel still needs.
+  pdl_wait_primary();
   if (warp == 0) {
     tmem_alloc(smem_u32(slot), kRtCols);
     tmem_relinquish();
   }
+  int issued = 0;                                    // tiles whose load thread 0 has issued
+  if (tid == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmX);
+    // the first two tiles are in flight while the tables are built
+    for (int b = 0; b < 2; ++b) {
+      const int t = (int)blockIdx.y + b * gy;
+      if (t >= ntiles) break;
+      ++issued;
+      mbar_arrive_expect_tx(bar0 + 8 * b, (uint32_t)L::TILE);
+      tma_load_2d(in_base + b * (uint32_t)L::TILE, &tmX, bar0 + 8 * b, grp * kGroup, t * kRtRows);
+      tma_load_2d(in_base + b * (uint32_t)L::TILE + (uint32_t)L::BOX, &tmX, bar0 + 8 * b,
+                  grp * kGroup + 64, t * kRtRows);
+    }
+  }
 
-  // ---- tables: (cos, sin) per pair; gather columns per stage.  Stage s reads
-  // channel ch from column ch (s = 0) or from its position in stage s-1's pair
-  // order (2p for the pair's a, 2p+1 for its b).  Indices outside the group are
-  // masked to 7 bits (every column stays inside this CTA's allocation) and flagged.
+  // ---- tables, 1: every stage's pairs and angles, loads issued together.
+  // Indices outside the group are masked to 7 bits (every address stays inside
+  // this CTA's allocation) and flagged.
+  if (tid < 128) scale[tid] = cs != nullptr ? cs[grp * kGroup + tid] : 1.0f;
   for (int idx = tid; idx < krot * 64; idx += kRtThreads) {
-    const int s = idx >> 6, p = idx & 63;
+    const int s = idx >> 6, p = idx & 63, u = p >> 1, w = p & 1;
+    const uint32_t pr =
+        *reinterpret_cast<const uint32_t*>(pairs + (size_t)s * K + (size_t)grp * kGroup + 2 * p);
+    int i = (int)(int16_t)(pr & 0xFFFFu), j = (int)(int16_t)(pr >> 16);
+    if ((unsigned)i >= 128u || (unsigned)j >= 128u) {
+      flag_error(kErrPairIndex);
+      i &= 127;
+      j &= 127;
+    }
+    praw[idx] = (uint32_t)i | ((uint32_t)j << 16);
     float sn, c;
     sincosf(theta[(size_t)s * (K / 2) + (size_t)grp * 64 + p], &sn, &c);
-    cstab[idx] = make_float2(c, sn);
-  }
-  for (int s = 0; s < krot; ++s) {
-    int* cur = pos + (s & 1) * 128;          // positions in stage s's pair order
-    const int* prev = pos + ((s + 1) & 1) * 128;
-    if (s > 0) __syncthreads();              // prev written, cur free to overwrite
-    for (int e = tid; e < 128; e += kRtThreads) cur[e] = e;   // defined even for bad tables
-    __syncthreads();
-    for (int p = tid; p < 64; p += kRtThreads) {
-      const int16_t* ps = pairs + (size_t)s * K + (size_t)grp * kGroup + 2 * p;
-      int i = ps[0], j = ps[1];
-      if ((unsigned)i >= 128u || (unsigned)j >= 128u) {
-        flag_error(kErrPairIndex);
-        i &= 127;
-        j &= 127;
-      }
-      gather[s * 128 + 2 * p] = (uint32_t)(s == 0 ? i : prev[i]);
-      gather[s * 128 + 2 * p + 1] = (uint32_t)(s == 0 ? j : prev[j]);
-      if (s == krot - 1) {                    // the last stage scatters to channel order
-        fin[2 * p] = (uint32_t)i;
-        fin[2 * p + 1] = (uint32_t)j;
-      }
-      cur[i] = 2 * p;
-      cur[j] = 2 * p + 1;
-    }
+    float* csu = reinterpret_cast<float*>(cstab + s * L::CS_STAGE) + 4 * u;
+    csu[w] = c;
+    csu[2 + w] = sn;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tbase = *slot + ((uint32_t)(32 * warp) << 16);   // this warp's 32 lanes
+  pdl_launch_dependents();
+  const uint32_t tmem0 = *slot;
 
-  // ---- load the row, scale, store to TMEM in natural channel order
-  const int row = row0 + tid;
-  uint32_t v[128];
-  {
-    const __half* src = x + (size_t)row * K + (size_t)grp * kGroup;
+  // ---- tables, 2 (warp 0): stage s reads buffer (s & 1) and writes buffer
+  // ((s + 1) & 1); a slot's gather entry is where its channel sits in that
+  // buffer: the channel index (s = 0) or its slot in stage s-1.  With ABS an
+  // entry is the full TMEM address for each lane quadrant, else the column.
+  constexpr int Q = ABS ? 4 : 1;
+  if (warp == 0) {
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      uint4 raw = make_uint4(0, 0, 0, 0);
-      if (row < M) raw = *reinterpret_cast<const uint4*>(src + 8 * q);
-      const __half2* h = reinterpret_cast<const __half2*>(&raw);
-      float sc[8];
-      if (cs != nullptr) {
-        const float4 a = *reinterpret_cast<const float4*>(cs + grp * kGroup + 8 * q);
-        const float4 b = *reinterpret_cast<const float4*>(cs + grp * kGroup + 8 * q + 4);
-        sc[0] = a.x; sc[1] = a.y; sc[2] = a.z; sc[3] = a.w;
-        sc[4] = b.x; sc[5] = b.y; sc[6] = b.z; sc[7] = b.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sc[e] = 1.0f;
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h[e]);
-        v[8 * q + 2 * e] = __float_as_uint(f.x * sc[2 * e]);
-        v[8 * q + 2 * e + 1] = __float_as_uint(f.y * sc[2 * e + 1]);
-      }
-    }
-  }
-  if (krot > 0) {
-#pragma unroll
-    for (int b = 0; b < 4; ++b) tmem_st32(tbase + 32 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
-    tmem_st_wait();
-
+    for (int c = 0; c < 4; ++c) pos[lane + 32 * c] = lane + 32 * c;
+    __syncwarp();
     for (int s = 0; s < krot; ++s) {
-      // gather the stage's operands in pair order
-      const uint4* gs = reinterpret_cast<const uint4*>(gather + s * 128);
+      int si[2], sj[2], ii[2], jj[2];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const uint4 g4 = gs[q];
-        v[4 * q] = tmem_ld1(tbase + g4.x);
-        v[4 * q + 1] = tmem_ld1(tbase + g4.y);
-        v[4 * q + 2] = tmem_ld1(tbase + g4.z);
-        v[4 * q + 3] = tmem_ld1(tbase + g4.w);
-      }
-      tmem_ld_wait_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[64]));
-      tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[96]));
-      // rotate every pair (registers 2p, 2p+1)
-      const float4* cs4 = reinterpret_cast<const float4*>(cstab + s * 64);
+      for (int e = 0; e < 2; ++e) {
+        const int p = lane + 32 * e, u = p >> 1, w = p & 1;
+        const uint32_t pr = praw[s * 64 + p];
+        ii[e] = (int)(pr & 0xFFFFu);
+        jj[e] = (int)(pr >> 16);
+        si[e] = 4 * u + w;
+        sj[e] = 4 * u + 2 + w;
+        const uint32_t ci = (uint32_t)((s & 1) * 128 + pos[ii[e]]);
+        const uint32_t cj = (uint32_t)((s & 1) * 128 + pos[jj[e]]);
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const float4 t = cs4[q];             // (cos, sin) of pairs 2q and 2q+1
-        float a = __uint_as_float(v[4 * q]), b = __uint_as_float(v[4 * q + 1]);
-        v[4 * q] = __float_as_uint(fmaf(a, t.x, b * t.y));
-        v[4 * q + 1] = __float_as_uint(fmaf(b, t.x, -(a * t.y)));
-        a = __uint_as_float(v[4 * q + 2]);
-        b = __uint_as_float(v[4 * q + 3]);
-        v[4 * q + 2] = __float_as_uint(fmaf(a, t.z, b * t.w));
-        v[4 * q + 3] = __float_as_uint(fmaf(b, t.z, -(a * t.w)));
-      }
-      if (s + 1 < krot) {
-        // write back in this stage's pair order (the next gather composes with it)
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          tmem_st32(tbase + 32 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
-      } else {
-        // last stage: scatter to the natural channel order
-        const uint4* f4 = reinterpret_cast<const uint4*>(fin);
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const uint4 f = f4[q];
-          tmem_st1(tbase + f.x, v[4 * q]);
-          tmem_st1(tbase + f.y, v[4 * q + 1]);
-          tmem_st1(tbase + f.z, v[4 * q + 2]);
-          tmem_st1(tbase + f.w, v[4 * q + 3]);
+        for (int q = 0; q < Q; ++q) {
+          const uint32_t lb = ABS ? tmem0 + ((uint32_t)(32 * q) << 16) : 0u;
+          gtab[((size_t)q * krot + s) * 128 + si[e]] = lb + ci;
+          gtab[((size_t)q * krot + s) * 128 + sj[e]] = lb + cj;
+          if (s == krot - 1) {                       // the last stage scatters to channel order
+            ftab[q * 128 + si[e]] = lb + (uint32_t)((krot & 1) * 128 + ii[e]);
+            ftab[q * 128 + sj[e]] = lb + (uint32_t)((krot & 1) * 128 + jj[e]);
+          }
         }
       }
-      tmem_st_wait();
-    }
+      __syncwarp();
 #pragma unroll
-    for (int b = 0; b < 4; ++b) tmem_ld32(tbase + 32 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
-    tmem_ld_wait_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-    tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-    tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[64]));
-    tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+      for (int e = 0; e < 2; ++e) {
+        pos[ii[e]] = si[e];
+        pos[jj[e]] = sj[e];
+      }
+      __syncwarp();
+    }
   }
+  __syncthreads();
 
-  // ---- fp16 (round to nearest) row out
-  if (row < M) {
-    __half* dst = xr + (size_t)row * K + (size_t)grp * kGroup;
+  const int r = 32 * qd + lane;                      // row within the tile = TMEM lane
+  const uint32_t lbase = tmem0 + ((uint32_t)(32 * qd) << 16);
+  const uint32_t goff = ABS ? 0u : lbase;            // added to a table entry
+  // this warp's 64 slots of stage 0 and of the final scatter
+  const uint32_t g_half = smem_u32(gtab + (ABS ? (size_t)qd * krot * 128 : 0) + 64 * h);
+  const uint32_t f_half = smem_u32(ftab + (ABS ? qd * 128 : 0) + 64 * h);
+  const uint32_t cs_half = smem_u32(cstab) + 256u * h;              // units 16h .. 16h+15
+  const float4* scale4 = reinterpret_cast<const float4*>(scale + 64 * h);
+  const uint32_t rsw = (uint32_t)(r & 7);            // swizzle phase of row r
+
+  int it = 0;
+  for (int tile = blockIdx.y; tile < ntiles; tile += gy, ++it) {
+    const int buf = it & 1;
+    // ---- row r, channels 64h .. 64h+63: 8 swizzled 16-byte chunks of box h, scaled
+    if (!mbar_wait_bounded(bar0 + 8 * buf, (uint32_t)((it >> 1) & 1))) *abort_flag = 1;
+    uint32_t v[64];
+    const unsigned char* rowp = sb + buf * L::TILE + h * L::BOX + r * 128;
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      uint4 out;
-      __half2* h = reinterpret_cast<__half2*>(&out);
+    for (int q = 0; q < 8; ++q) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(rowp + ((((uint32_t)q) ^ rsw) << 4));
+      const __half2* hv = reinterpret_cast<const __half2*>(&raw);
+      const float4 sa = scale4[2 * q], sc = scale4[2 * q + 1];
+      const float2 s2[4] = {make_float2(sa.x, sa.y), make_float2(sa.z, sa.w), make_float2(sc.x, sc.y),
+                            make_float2(sc.z, sc.w)};
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        h[e] = __floats2half2_rn(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
-      *reinterpret_cast<uint4*>(dst + 8 * q) = out;
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __fmul2_rn(__half22float2(hv[e]), s2[e]);
+        v[8 * q + 2 * e] = __float_as_uint(f.x);
+        v[8 * q + 2 * e + 1] = __float_as_uint(f.y);
+      }
     }
+    __syncthreads();                                 // every row read: this buffer is free
+    if (*abort_flag) break;                          // uniform: set only before the barrier
+    if (tid == 0 && tile + 2 * gy < ntiles) {
+      ++issued;
+      const int nrow = (tile + 2 * gy) * kRtRows;
+      const uint32_t dstb = in_base + buf * (uint32_t)L::TILE;
+      mbar_arrive_expect_tx(bar0 + 8 * buf, (uint32_t)L::TILE);
+      tma_load_2d(dstb, &tmX, bar0 + 8 * buf, grp * kGroup, nrow);
+      tma_load_2d(dstb + (uint32_t)L::BOX, &tmX, bar0 + 8 * buf, grp * kGroup + 64, nrow);
+    }
+
+    if (krot > 0) {
+      tmem_st32(lbase + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_st32(lbase + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      rt_quadrant_sync(qd);
+      for (int s = 0; s < krot; ++s) {
+        // gather this warp's 64 slots; table reads run four 16-byte loads ahead
+        const uint32_t gs = g_half + (uint32_t)s * 512u;
+        uint4 g[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) g[k] = lds128(gs + 16 * k);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint4 a = g[k & 3];
+          v[4 * k] = tmem_ld1(a.x + goff);
+          v[4 * k + 1] = tmem_ld1(a.y + goff);
+          v[4 * k + 2] = tmem_ld1(a.z + goff);
+          v[4 * k + 3] = tmem_ld1(a.w + goff);
+          if (k + 4 < 16) g[k & 3] = lds128(gs + 16 * (k + 4));
+        }
+        tmem_ld_wait_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        // rotate the 16 units (A = slots 0,1; B = slots 2,3)
+        const uint32_t cst = cs_half + (uint32_t)s * (uint32_t)L::CS_STAGE;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint4 t = lds128(cst + 16 * k);      // (c0, c1, s0, s1)
+          const float2 C = make_float2(__uint_as_float(t.x), __uint_as_float(t.y));
+          const float2 S = make_float2(__uint_as_float(t.z), __uint_as_float(t.w));
+          const float2 NS = make_float2(-S.x, -S.y);
+          const float2 A = make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]));
+          const float2 B = make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+          const float2 A2 = __ffma2_rn(A, C, __fmul2_rn(B, S));
+          const float2 B2 = __ffma2_rn(A, NS, __fmul2_rn(B, C));
+          v[4 * k] = __float_as_uint(A2.x);
+          v[4 * k + 1] = __float_as_uint(A2.y);
+          v[4 * k + 2] = __float_as_uint(B2.x);
+          v[4 * k + 3] = __float_as_uint(B2.y);
+        }
+        if (s + 1 < krot) {
+          const uint32_t d = lbase + (uint32_t)((s + 1) & 1) * 128u + 64u * h;
+          tmem_st32(d, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_st32(d + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        } else {
+          // last stage: scatter to the natural channel order
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint4 f = lds128(f_half + 16 * k);
+            tmem_st1(f.x + goff, v[4 * k]);
+            tmem_st1(f.y + goff, v[4 * k + 1]);
+            tmem_st1(f.z + goff, v[4 * k + 2]);
+            tmem_st1(f.w + goff, v[4 * k + 3]);
+          }
+        }
+        rt_quadrant_sync(qd);
+      }
+      const uint32_t fb = lbase + (uint32_t)(krot & 1) * 128u + 64u * h;
+      tmem_ld32(fb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(fb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_ld_wait_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+    }
+
+    // ---- fp16 (round to nearest), row r, channels 64h .. 64h+63
+    const int row = tile * kRtRows + r;
+    if (row < M) {
+      __half* dstp = xr + (size_t)row * K + (size_t)grp * kGroup + 64 * h;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint4 out;
+        __half2* hv = reinterpret_cast<__half2*>(&out);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          hv[e] = __floats2half2_rn(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
+        *reinterpret_cast<uint4*>(dstp + 8 * q) = out;
+      }
+    }
+  }
+  if (tid == 0 && *abort_flag) {
+    // a wait gave up: let the loads still in flight land (bounded) before the
+    // shared memory is released
+    for (int t = it; t < issued; ++t)
+      if (!mbar_wait_bounded(bar0 + 8 * (t & 1), (uint32_t)((t >> 1) & 1))) break;
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(*slot, kRtCols);
+    tmem_dealloc(tmem0, kRtCols);
   }
 }
 

@@ -67,6 +67,9 @@ ROT_CASES = [
     (129, 256, 64, True, None),       # krot maximum on the tensor-memory kernel
     (65, 384, 1, False, None),        # tensor-memory kernel, krot = 1, ragged tile
     (3, 14336, 8, True, None),        # down_proj width
+    (300, 512, 16, True, None),       # tensor-memory kernel, per-warp address tables at their limit
+    (300, 512, 17, True, None),       # tensor-memory kernel, one shared column table
+    (20000, 1024, 8, True, None),     # CTAs walk several row tiles; ragged last tile
 ]
 
 
