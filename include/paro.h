@@ -44,6 +44,16 @@
  *     aborted across the ABI and nothing falls back to the CPU.
  *   - Kernels that wait on an mbarrier bound the wait; a wait that runs out sets
  *     a device status word that paro_device_status() reports as PARO_ERR_TIMEOUT.
+ *   - Launch overlap.  paro_rotate and paro_w4_linear launch with programmatic
+ *     dependent launch: a call's kernels may start while the kernel ahead of them
+ *     in the stream is still running, and they read the layer constants
+ *     (qweight, qzeros, scales, channel_scales, pairs, theta) before waiting for
+ *     it; activations are read, and outputs and the workspace written, only
+ *     after it has completed.  So the layer constants must not be written by the
+ *     kernel immediately ahead of the call if that kernel releases its dependents
+ *     early (griddepcontrol.launch_dependents).  No kernel of this library that
+ *     releases early writes layer constants (paro_pack_awq does not release
+ *     early), and kernels that never release early are always safe.
  *   - Supported now: G == 128 (group_size == -1 is accepted when K == 128),
  *     0 <= krot <= 64, K a multiple of 128, N a multiple of 32 (the packer alone
  *     needs only N % 8 == 0), fp16 activations/scales/bias.

@@ -65,6 +65,22 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, size_t esize, const voi
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// X as [K/64 chunks][rows][64] (chunk stride 128 bytes, row stride K*2 bytes):
+// box {64 columns, box_rows rows, box_chunks chunks}, 128-byte swizzle.  One
+// copy brings several groups' activation columns in the layout the GEMV reads.
+bool encode_x_chunks(CUtensorMap* map, const void* x, uint64_t rows, uint64_t K, uint32_t box_rows,
+                     uint32_t box_chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {64, rows, K / 64};
+  cuuint64_t strides[2] = {K * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_chunks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- device facts
 struct DeviceInfo {
   int sms = 0;
@@ -289,7 +305,11 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
     p.n_tiles = (int)((N + tile - 1) / tile);
     int s = 1;
     while (s * 2 <= want && s * 2 <= kMaxSplits && s * 2 <= groups && p.n_tiles * s * 2 <= kDecodeTargetCtas) s *= 2;
+    // a CTA holds at most kGvMaxGroups groups of activations and constants
+    while ((groups + s - 1) / s > kGvMaxGroups && s < kMaxSplits) s *= 2;
     p.splits = s;
+    // deeper than the GEMV's reach (K > 16384): the tensor-core GEMM serves it
+    if ((groups + s - 1) / s > kGvMaxGroups) p.decode = false;
   }
   return p;
 }
@@ -319,34 +339,37 @@ int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t
 // CTAs along K per column tile.
 template <int NT, int KP, int NTILE, int STAGES>
 int launch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
-                const void* scales, const CUtensorMap& tmX, const __half* bias, __half* y,
+                const void* scales, const __half* x, const __half* bias, __half* y,
                 int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
-  CUtensorMap tmW, tmS, tmZ;
+  const int groups = (int)(K / kGroup);
+  const int gmax = (groups + plan.splits - 1) / plan.splits;   // largest group range of a CTA
+  if (gmax > kGvMaxGroups) return PARO_ERR_UNSUPPORTED;
+  CUtensorMap tmW, tmS, tmZ, tmX;
   const bool ok =
       encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, L::WORDS,
                 L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) &&
-      encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, NTILE,
-                CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, L::WORDS,
-                CU_TENSOR_MAP_SWIZZLE_NONE);
+      encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, (uint32_t)gmax,
+                NTILE, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, (uint32_t)gmax,
+                L::WORDS, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      encode_x_chunks(&tmX, x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP, (uint32_t)(2 * gmax));
   if (!ok) return PARO_ERR_CUDA;
   auto k = w4_gemv_kernel<NT, KP, NTILE, STAGES>;
   if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
   const dim3 grid((unsigned)((N + NTILE - 1) / NTILE), (unsigned)plan.splits, 1);
   return launch_ex(k, grid, dim3(L::THREADS), L::SMEM, s, pdl, (unsigned)plan.splits, tmW, tmX,
-                   tmS, tmZ, bias, y, (int)M, (int)N, (int)K);
+                   tmS, tmZ, bias, y, (int)M, (int)N, (int)K, gmax);
 }
 
 template <int NT>
 int dispatch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
-                  const void* scales, const CUtensorMap& tmX, const __half* bias, __half* y,
+                  const void* scales, const __half* x, const __half* bias, __half* y,
                   int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
   switch (plan.variant) {
-    case 0: return launch_gemv<NT, 2, 256, 4>(plan, qweight, qzeros, scales, tmX, bias, y, M, N, K, s, pdl);
-    case 1: return launch_gemv<NT, 2, 256, 8>(plan, qweight, qzeros, scales, tmX, bias, y, M, N, K, s, pdl);
-    case 2: return launch_gemv<NT, 4, 128, 8>(plan, qweight, qzeros, scales, tmX, bias, y, M, N, K, s, pdl);
-    default: return launch_gemv<NT, 2, 128, 4>(plan, qweight, qzeros, scales, tmX, bias, y, M, N, K, s, pdl);
+    case 0: return launch_gemv<NT, 2, 256, 4>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
+    case 2: return launch_gemv<NT, 4, 128, 8>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
+    default: return launch_gemv<NT, 2, 128, 4>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
   }
 }
 
@@ -453,12 +476,14 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
   if (rotate && (workspace == nullptr || workspace_bytes < plan.total)) return PARO_ERR_WORKSPACE;
   if (rotate && !aligned(workspace, 256)) return PARO_ERR_ALIGNMENT;
   const __half* xa = static_cast<const __half*>(x);
-  bool pdl = false;
+  // Programmatic dependent launch throughout: the GEMV/GEMM requests weights,
+  // scales and zero points before it waits for the kernel ahead of it (the
+  // rotation, or whatever preceded the call), and reads activations after.
+  const bool pdl = true;
   if (rotate) {
     __half* xr = reinterpret_cast<__half*>(static_cast<unsigned char*>(workspace) + plan.off_xr);
     if (int st = launch_rotate(xa, xr, M, K, channel_scales, pairs, theta, krot, s)) return st;
     xa = xr;
-    pdl = true;   // the GEMV streams weights while the rotation finishes
   }
 
   const __half* b = static_cast<const __half*>(bias);
@@ -467,13 +492,8 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
     return launch_w4_prefill(xa, yy, M, K, N, qweight, qzeros, static_cast<const __half*>(scales),
                              b, s, pdl);
 
-  CUtensorMap tmX;
-  const int mp = 8 * plan.nt;
-  if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, mp, 64,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
-    return PARO_ERR_CUDA;
-  if (plan.nt == 1) return dispatch_gemv<1>(plan, qweight, qzeros, scales, tmX, b, yy, M, N, K, s, pdl);
-  return dispatch_gemv<2>(plan, qweight, qzeros, scales, tmX, b, yy, M, N, K, s, pdl);
+  if (plan.nt == 1) return dispatch_gemv<1>(plan, qweight, qzeros, scales, xa, b, yy, M, N, K, s, pdl);
+  return dispatch_gemv<2>(plan, qweight, qzeros, scales, xa, b, yy, M, N, K, s, pdl);
 }
 
 }  // extern "C"

@@ -63,12 +63,10 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
     const __half* x, __half* xr, const float* __restrict__ cs,
     const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot) {
   using T = RotTile<ROWS>;
-  // Programmatic dependent launch: wait until the previous kernel in the stream
-  // has completed (no input is read before that), then let the GEMV that
-  // follows launch and start streaming its weights while this kernel works.
-  // Triggering only after the wait keeps everything before this kernel complete
-  // by the time the GEMV runs its independent prologue.
-  pdl_wait_primary();
+  // Programmatic dependent launch: the GEMV that follows may launch at once and
+  // stream its weights while this kernel works.  The stage tables are layer
+  // constants (read-only for the call, not written by the previous kernel), so
+  // they are read before waiting for the previous kernel; x is read after.
   pdl_launch_dependents();
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -79,6 +77,9 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
   const int row0 = blockIdx.y * ROWS;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+
+  load_rot_params(prm, pairs, theta, K, krot, grp, tid, kRotThreads);
+  pdl_wait_primary();
 
   // ---- load + scale: item = (8-channel chunk v, row r), rows fastest
   for (int idx = tid; idx < 16 * ROWS; idx += kRotThreads) {
@@ -105,7 +106,6 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
       xs[(8 * v + 2 * e + 1) * T::PITCH + r] = f.y * sc[2 * e + 1];
     }
   }
-  load_rot_params(prm, pairs, theta, K, krot, grp, tid, kRotThreads);
   __syncthreads();
 
   // ---- stages: warp w applies pairs 8w..8w+7; lane = (pair sub-index, row)

@@ -5,15 +5,17 @@
 // transforms" and "Triton plans and tuning"):
 //   Y[m, n] = sum_g s[g, n] * sum_{k in g} X_r[m, k] * (q[k, n] - z[g, n]) + b[n]
 //
-// Work layout.  A CTA owns 256 output columns (32 packed words = one 128-byte
-// line of every qweight row) and a contiguous range of 128-row groups of K.
-// Warp 0 is the producer: one lane streams each group through a ring of STAGES
-// shared-memory stages with TMA (qweight 128 rows x 128 B, 128-byte swizzle;
-// the group's 256 scales and 32 zero words; the matching 128 columns of X_r),
-// signalling "full" mbarriers; consumers release a stage on its "empty"
-// mbarrier.  Weights, scales and zeros do not depend on the previous kernel, so
-// the producer streams them before griddepcontrol.wait (programmatic dependent
-// launch) and only the X_r loads wait for the rotation kernel.
+// Work layout.  A CTA owns NTILE output columns (NTILE/8 packed words of every
+// qweight row) and a contiguous range of at most kGvMaxGroups 128-row groups of
+// K.  Warp 0 is the producer.  One lane streams each group's qweight block
+// (128 rows, 64- or 128-byte swizzle) through a ring of STAGES shared-memory
+// stages with TMA, signalling "full" mbarriers; consumers release a stage on its
+// "empty" mbarrier.  The CTA's scales, zero words and X_r columns are each one
+// TMA copy for the whole range (a TMA instruction costs tens of cycles to issue
+// whatever its size, so few large copies start the stream sooner), resident
+// for the whole kernel.  Weights, scales and zeros do not depend on the
+// previous kernel, so they are requested before griddepcontrol.wait
+// (programmatic dependent launch); only the X_r copy waits for the rotation.
 // Consumer warps are 4 column slices (64 columns each) x KP k-parts; k-part p
 // takes the CTA's groups p, p+KP, ... so every warp works on whole groups.
 //
@@ -32,11 +34,12 @@
 // in fp32, then times the group scale (s / 16 for odd j, an exact power of two).
 //
 // Split-K: the S CTAs that share an output tile form a thread-block cluster
-// along K.  CTA r owns columns [r*NTILE/S, (r+1)*NTILE/S): every CTA pushes its
-// fp32 partial of each slice into the owner's inbox (a dedicated shared-memory
-// area, one slot per sender) with distributed-shared-memory stores; after one
-// cluster barrier each owner sums its inbox in sender order, adds the bias and
-// writes fp16 Y.  No global scratch, no atomics, deterministic.
+// along K.  CTA r owns columns [r*NTILE/S, (r+1)*NTILE/S): every consumer warp
+// pushes its fp32 partials of each slice straight from registers into the
+// owner's inbox (a dedicated shared-memory area, one slot per sender CTA and
+// k-part) with distributed-shared-memory stores; after one cluster barrier
+// each owner sums its inbox in a fixed order, adds the bias and writes fp16 Y.
+// No global scratch, no atomics, deterministic.
 #pragma once
 
 #include "common.cuh"
@@ -44,6 +47,7 @@
 namespace paro {
 
 constexpr int kGvMaxStages = 8;
+constexpr int kGvMaxGroups = 16;            // 128-row groups of K per CTA
 constexpr uint32_t kGvMagic = 0x64006400u;  // fp16 pair (1024, 1024)
 constexpr uint32_t kGvOnes = 0x3C003C00u;   // fp16 pair (1, 1)
 
@@ -56,20 +60,18 @@ struct GemvLayout {
   static constexpr int THREADS = 32 * (1 + CSL * KP);
   static constexpr int MP = 8 * NT;                       // token rows per CTA
   static constexpr int W_BYTES = 128 * WORDS * 4;         // one group of qweight
-  static constexpr int X_BYTES = 2 * MP * 128;            // two 64-column boxes
-  static constexpr int S_BYTES = NTILE * 2;
-  static constexpr int Z_BYTES = WORDS * 4;
-  static constexpr int X_OFF = W_BYTES;
-  static constexpr int S_OFF = X_OFF + ((X_BYTES + 1023) / 1024) * 1024;
-  static constexpr int Z_OFF = S_OFF + S_BYTES;
-  static constexpr int STAGE = ((Z_OFF + Z_BYTES + 1023) / 1024) * 1024;
-  static constexpr int TX_BYTES = W_BYTES + S_BYTES + Z_BYTES + X_BYTES;
-  static constexpr int RED_BYTES = KP * MP * NTILE * 4;     // k-part partial tiles
-  static constexpr int INBOX_OFF = STAGES * STAGE;          // split-K inbox [S][MP][NTILE/S]
-  static constexpr int INBOX_BYTES = MP * NTILE * 4;
-  static constexpr int BAR_OFF = INBOX_OFF + INBOX_BYTES;   // full[], empty[] mbarriers
-  static constexpr int SMEM = BAR_OFF + 16 * STAGES + 1024;
-  static_assert(RED_BYTES <= STAGES * STAGE, "reduction tiles must fit in stage memory");
+  static constexpr int STAGE = ((W_BYTES + 1023) / 1024) * 1024;
+  // resident for the whole kernel: X_r as [64-column chunk][token][64] (two
+  // chunks per group), scales [group][NTILE], zero words [group][WORDS]
+  static constexpr int XG_BYTES = 2 * MP * 128;           // X_r of one group
+  static constexpr int X_OFF = STAGES * STAGE;
+  static constexpr int S_OFF = X_OFF + kGvMaxGroups * XG_BYTES;
+  static constexpr int Z_OFF = S_OFF + kGvMaxGroups * NTILE * 2;
+  static constexpr int INBOX_OFF = ((Z_OFF + kGvMaxGroups * WORDS * 4 + 1023) / 1024) * 1024;
+  static constexpr int INBOX_BYTES = KP * MP * NTILE * 4;   // partials [S][KP][MP][NTILE/S]
+  static constexpr int BAR_OFF = INBOX_OFF + INBOX_BYTES;   // full[], empty[], consts, X_r
+  static constexpr int SMEM = BAR_OFF + 16 * STAGES + 16 + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   static_assert(STAGES <= kGvMaxStages, "too many stages");
   // 128-byte swizzle needs 128-byte rows; 64-byte rows use the 64-byte swizzle
   static constexpr int ROW_BYTES = WORDS * 4;
@@ -84,10 +86,10 @@ __device__ __forceinline__ void gv_unpack4(uint32_t m, uint32_t (&e)[4]) {
 }
 
 template <int NT, int KP, int NTILE, int STAGES>
-__global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP)) w4_gemv_kernel(
+__global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kernel(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
-    const __half* __restrict__ bias, __half* __restrict__ Y, int M, int N, int K) {
+    const __half* __restrict__ bias, __half* __restrict__ Y, int M, int N, int K, int gmax) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
   constexpr int kGvStages = STAGES;
   constexpr int kGvTile = NTILE;
@@ -101,12 +103,15 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP)) w4_gemv_kernel(
   const uint32_t base = smem_u32(sbase);
   const uint32_t full0 = base + L::BAR_OFF;
   const uint32_t empty0 = full0 + 8 * kGvStages;
+  const uint32_t cbar = empty0 + 8 * kGvStages;   // scales + zero words
+  const uint32_t xbar = cbar + 8;                  // X_r
 
   const int ntile = blockIdx.x, split = blockIdx.y;
   const int n0 = ntile * kGvTile;
   const int groups = K / 128;
-  const int g_begin = (int)(((long long)split * groups) / gridDim.y);
-  const int g_end = (int)(((long long)(split + 1) * groups) / gridDim.y);
+  // 32-bit arithmetic (groups <= 2^16, splits <= 8): no 64-bit division routine
+  const int g_begin = (int)(((unsigned)split * (unsigned)groups) / gridDim.y);
+  const int g_end = (int)(((unsigned)(split + 1) * (unsigned)groups) / gridDim.y);
   const int ng = g_end - g_begin;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -115,6 +120,8 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP)) w4_gemv_kernel(
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, L::CSL);  // the column-slice warps of one k-part
     }
+    mbar_init(cbar, 1);
+    mbar_init(xbar, 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
@@ -140,32 +147,25 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP)) w4_gemv_kernel(
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const int pre = min(kGvStages, ng);
+      // the tensor maps' boxes hold gmax groups (the largest range of any CTA;
+      // rows past this CTA's range are loaded and not used)
+      mbar_arrive_expect_tx(cbar, (uint32_t)(gmax * (NTILE * 2 + L::WORDS * 4)));
+      tma_load_2d(base + L::S_OFF, &tmS, cbar, n0, g_begin);
+      tma_load_2d(base + L::Z_OFF, &tmZ, cbar, n0 / 8, g_begin);
       for (int i = 0; i < pre; ++i) {
-        const uint32_t st = base + i * L::STAGE, bar = full0 + 8 * i;
-        const int kg = g_begin + i;
-        mbar_arrive_expect_tx(bar, L::TX_BYTES);
-        tma_load_2d_hint(st, &tmW, bar, n0 / 8, kg * 128, pol);
-        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, kg);
-        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, kg);
+        const uint32_t bar = full0 + 8 * i;
+        mbar_arrive_expect_tx(bar, L::W_BYTES);
+        tma_load_2d_hint(base + i * L::STAGE, &tmW, bar, n0 / 8, (g_begin + i) * 128, pol);
       }
       pdl_wait_primary();                  // X_r comes from the rotation kernel
-      for (int i = 0; i < pre; ++i) {
-        const uint32_t st = base + i * L::STAGE, bar = full0 + 8 * i;
-        const int kg = g_begin + i;
-        tma_load_2d(st + L::X_OFF, &tmX, bar, kg * 128, 0);
-        tma_load_2d(st + L::X_OFF + L::MP * 128, &tmX, bar, kg * 128 + 64, 0);
-      }
+      mbar_arrive_expect_tx(xbar, (uint32_t)(gmax * L::XG_BYTES));
+      tma_load_3d(base + L::X_OFF, &tmX, xbar, 0, 0, 2 * g_begin);
       for (int i = pre; i < ng; ++i) {
         const int s = i % kGvStages;
         if (!mbar_wait_bounded(empty0 + 8 * s, ((i / kGvStages) - 1) & 1)) break;
-        const uint32_t st = base + s * L::STAGE, bar = full0 + 8 * s;
-        const int kg = g_begin + i;
-        mbar_arrive_expect_tx(bar, L::TX_BYTES);
-        tma_load_2d_hint(st, &tmW, bar, n0 / 8, kg * 128, pol);
-        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, kg);
-        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, kg);
-        tma_load_2d(st + L::X_OFF, &tmX, bar, kg * 128, 0);
-        tma_load_2d(st + L::X_OFF + L::MP * 128, &tmX, bar, kg * 128 + 64, 0);
+        const uint32_t bar = full0 + 8 * s;
+        mbar_arrive_expect_tx(bar, L::W_BYTES);
+        tma_load_2d_hint(base + s * L::STAGE, &tmW, bar, n0 / 8, (g_begin + i) * 128, pol);
       }
     }
   } else {
@@ -187,19 +187,22 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP)) w4_gemv_kernel(
       for (int nt = 0; nt < NT; ++nt) {
         const int tok = 8 * nt + g;
         const int c0 = 2 * q;
-        xo[q][nt][0] = (uint32_t)(L::X_OFF + tok * 128 + (((c0) ^ (tok & 7)) << 4) + 4 * t);
-        xo[q][nt][1] = (uint32_t)(L::X_OFF + tok * 128 + (((c0 + 1) ^ (tok & 7)) << 4) + 4 * t);
+        xo[q][nt][0] = (uint32_t)(tok * 128 + (((c0) ^ (tok & 7)) << 4) + 4 * t);
+        xo[q][nt][1] = (uint32_t)(tok * 128 + (((c0 + 1) ^ (tok & 7)) << 4) + 4 * t);
       }
     const uint32_t ones[4] = {kGvOnes, kGvOnes, kGvOnes, kGvOnes};
 
+    // scales, zero words and X_r of every group of the range (once)
+    bool consts_ready = mbar_wait_bounded(cbar, 0);
+    consts_ready = mbar_wait_bounded(xbar, 0) && consts_ready;
     for (int i = kpart; i < ng; i += KP) {
       const int s = i % kGvStages;
       const unsigned char* stp = sbase + s * L::STAGE;
-      const bool ready = mbar_wait_bounded(full0 + 8 * s, (i / kGvStages) & 1);
+      const bool ready = mbar_wait_bounded(full0 + 8 * s, (i / kGvStages) & 1) && consts_ready;
       if (ready) {
         // group constants for this thread's 8 columns
-        const uint32_t zw = *reinterpret_cast<const uint32_t*>(stp + L::Z_OFF + wcol * 4);
-        const uint4 s8 = *reinterpret_cast<const uint4*>(stp + L::S_OFF + wcol * 16);
+        const uint32_t zw = *reinterpret_cast<const uint32_t*>(sbase + L::Z_OFF + (i * L::WORDS + wcol) * 4);
+        const uint4 s8 = *reinterpret_cast<const uint4*>(sbase + L::S_OFF + i * NTILE * 2 + wcol * 16);
         float cg[4][NT][4];
         float rs[NT][4];
 #pragma unroll
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP)) w4_gemv_kernel(
           uint32_t b0[NT], b1[NT];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const unsigned char* xb = stp + (ks >> 2) * (L::MP * 128);
+            const unsigned char* xb = sbase + L::X_OFF + i * L::XG_BYTES + (ks >> 2) * (L::MP * 128);
             b0[nt] = *reinterpret_cast<const uint32_t*>(xb + xo[ks & 3][nt][0]);
             b1[nt] = *reinterpret_cast<const uint32_t*>(xb + xo[ks & 3][nt][1]);
           }
@@ -266,75 +269,72 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP)) w4_gemv_kernel(
 
   // Everything before us in the stream is complete before anyone writes Y.
   pdl_wait_primary();
-  __syncthreads();
 
-  // ---------------- reduction over k-parts (shared memory, fixed order)
-  float* red = reinterpret_cast<float*>(sbase);
+  // ---------------- reduction over k-parts and the split along K.  Every
+  // consumer thread holds 8 consecutive columns for each of its tokens; it
+  // writes them straight into the inbox of the CTA that owns those columns
+  // (slot [sender rank][k-part]); after one barrier each owner folds its
+  // inbox in a fixed order (deterministic), adds the bias and writes fp16 Y.
+  const int mrows = min(L::MP, M);
+  const int S = gridDim.y;
+  const int cols = kGvTile / S;                    // columns owned by each CTA of the cluster
+  const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
+  const uint32_t inbox = base + L::INBOX_OFF;      // fp32 [S][KP][MP][cols]
   if (warp != 0) {
+    const int owner = (8 * wcol) / cols;
+    const int c0 = 8 * wcol - owner * cols;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int tt = 0; tt < 2; ++tt) {
         const int tl = 8 * nt + 2 * t + tt;
-        float* p = red + ((size_t)kpart * L::MP + tl) * kGvTile + 8 * wcol;
-        *reinterpret_cast<float4*>(p) =
+        if (tl >= mrows) continue;
+        const uint32_t off = inbox + (uint32_t)(((((int)rank * KP + kpart) * L::MP + tl) * cols + c0) * 4);
+        const float4 v0 =
             make_float4(acc[0][nt][tt], acc[0][nt][2 + tt], acc[1][nt][tt], acc[1][nt][2 + tt]);
-        *reinterpret_cast<float4*>(p + 4) =
+        const float4 v1 =
             make_float4(acc[2][nt][tt], acc[2][nt][2 + tt], acc[3][nt][tt], acc[3][nt][2 + tt]);
+        if (S > 1) {
+          st_cluster_f4(mapa_shared(off, (uint32_t)owner), v0);
+          st_cluster_f4(mapa_shared(off + 16, (uint32_t)owner), v1);
+        } else {
+          sts128(off, v0);
+          sts128(off + 16, v1);
+        }
       }
   }
-  __syncthreads();
-  const int mrows = min(L::MP, M);
-  const int S = gridDim.y;
-  const int cols = kGvTile / S;                    // columns owned by each CTA of the cluster
-  const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
-  const uint32_t inbox = base + L::INBOX_OFF;
-  // fold the k-parts (fixed order); write Y directly or push to the slice owner
-  for (int idx = tid; idx < mrows * kGvTile / 4; idx += L::THREADS) {
-    float4 v = reinterpret_cast<const float4*>(red)[idx];
-#pragma unroll
-    for (int kp = 1; kp < KP; ++kp) {
-      const float4 u = reinterpret_cast<const float4*>(red + (size_t)kp * L::MP * kGvTile)[idx];
-      v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+  // this thread's first output (the bias load overlaps the barrier)
+  const int nq = mrows * (cols / 4);
+  float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (bias != nullptr && tid < nq) {
+    const int n = n0 + (int)rank * cols + 4 * (tid % (cols / 4));
+    if (n < N) {
+      const __half2 b0 = *reinterpret_cast<const __half2*>(bias + n);
+      const __half2 b1 = *reinterpret_cast<const __half2*>(bias + n + 2);
+      bv = make_float4(__low2float(b0), __high2float(b0), __low2float(b1), __high2float(b1));
     }
-    const int tl = idx / (kGvTile / 4);
-    const int col = 4 * (idx % (kGvTile / 4));
-    if (S > 1) {
-      const int owner = col / cols;
-      const uint32_t off = inbox + (uint32_t)(((int)rank * L::MP + tl) * cols + (col - owner * cols)) * 4u;
-      st_cluster_f4(mapa_shared(off, (uint32_t)owner), v);
-      continue;
-    }
-    const int n = n0 + col;
-    if (n >= N) continue;
-    if (bias != nullptr) {
-      v.x += __half2float(bias[n]); v.y += __half2float(bias[n + 1]);
-      v.z += __half2float(bias[n + 2]); v.w += __half2float(bias[n + 3]);
-    }
-    const __half2 h0 = __floats2half2_rn(v.x, v.y), h1 = __floats2half2_rn(v.z, v.w);
-    uint2 out;
-    out.x = *reinterpret_cast<const uint32_t*>(&h0);
-    out.y = *reinterpret_cast<const uint32_t*>(&h1);
-    *reinterpret_cast<uint2*>(Y + (size_t)tl * N + n) = out;
   }
-  if (S == 1) return;
-
   // every partial pushed into this CTA's inbox is complete and visible after this
-  cluster_sync();
+  if (S > 1) cluster_sync();
+  else __syncthreads();
   const float* box = reinterpret_cast<const float*>(sbase + L::INBOX_OFF);
-  for (int idx = tid; idx < mrows * (cols / 4); idx += L::THREADS) {
+  for (int idx = tid; idx < nq; idx += L::THREADS) {
     const int tl = idx / (cols / 4);
     const int c = 4 * (idx % (cols / 4));
     const int n = n0 + (int)rank * cols + c;
     if (n >= N) continue;
     float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int q = 0; q < S; ++q) {
+    for (int q = 0; q < S * KP; ++q) {
       const float4 v = *reinterpret_cast<const float4*>(box + ((size_t)q * L::MP + tl) * cols + c);
       sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
     }
     if (bias != nullptr) {
-      sum.x += __half2float(bias[n]); sum.y += __half2float(bias[n + 1]);
-      sum.z += __half2float(bias[n + 2]); sum.w += __half2float(bias[n + 3]);
+      if (idx != tid) {
+        const __half2 b0 = *reinterpret_cast<const __half2*>(bias + n);
+        const __half2 b1 = *reinterpret_cast<const __half2*>(bias + n + 2);
+        bv = make_float4(__low2float(b0), __high2float(b0), __low2float(b1), __high2float(b1));
+      }
+      sum.x += bv.x; sum.y += bv.y; sum.z += bv.z; sum.w += bv.w;
     }
     const __half2 h0 = __floats2half2_rn(sum.x, sum.y), h1 = __floats2half2_rn(sum.z, sum.w);
     uint2 out;
