@@ -290,16 +290,16 @@ def run_ours(args, rank, world, local_rank):
         achieved = kern_bytes / (kern_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                "traffic": traffic_for("w4_mma_decode"),
-                "kernel": "w4_mma_kernel (decode GEMV, split-K cluster)",
+                "traffic": traffic_for("w4_gemv_decode"),
+                "kernel": "w4_gemv_kernel (decode GEMV, split-K cluster)",
                 "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
                 "bytes_per_launch": kern_bytes // n_launch, "peak_source": peaks["src"]}
     else:
         achieved = kern_flops / (kern_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
-                "traffic": traffic_for("w4_prefill"),
-                "kernel": "prefill W4 GEMM", "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
+                "traffic": traffic_for("w4_tc_prefill"),
+                "kernel": "w4_tc_gemm_kernel (prefill tcgen05 GEMM)", "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
                 "flops_per_launch": kern_flops // n_launch,
                 "peak_source": peaks["src"] + " bf16 burst (fp16 runs at the bf16 rate)"}
     del g2
