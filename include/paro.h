@@ -97,8 +97,9 @@ const char* paro_version(void);
  *   pairs, theta    device tables as above; may be NULL only when krot == 0
  *   group_size      128, or -1 meaning K (then K must be 128)
  *   krot            number of stages, 0..64 (0 = scaling only)
- * Arithmetic: fp32 on chip, cos/sin from sincosf of the fp32 angle, one
- * round-to-nearest to fp16 at the end.  Pair indices outside 0..G-1 are
+ * Arithmetic: fp32 on chip; cos/sin of the fp32 angle by the hardware
+ * approximation after one reduction into [-pi, pi] (absolute error about
+ * 2^-21); one round-to-nearest to fp16 at the end.  Pair indices outside 0..G-1 are
  * masked to 7 bits (so no access leaves the group) and flagged in the device
  * status word; pair tables are not otherwise checked (see paro_validate_pairs).
  */

@@ -180,6 +180,18 @@ __device__ __forceinline__ void sts128(uint32_t addr, float4 v) {
                : "memory");
 }
 
+// ---------------------------------------------------------------- rotation angles
+// (sin, cos) of a Givens angle.  One Cody-Waite step with 2*pi split into an
+// fp32 head and tail brings the angle into [-pi, pi]; there the hardware
+// approximation's absolute error is about 2^-21.4 (CUDA C programming guide,
+// intrinsic functions), four orders below the 1e-3 relative bound on X_r.
+__device__ __forceinline__ void rot_sincos(float t, float* s, float* c) {
+  const float k = rintf(t * 0.159154943f);                 // t / (2 pi), nearest integer
+  t = fmaf(-k, 6.28318548f, t);                            // 2 pi, fp32 head
+  t = fmaf(-k, -1.74845553e-7f, t);                        // 2 pi - head
+  __sincosf(t, s, c);
+}
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;

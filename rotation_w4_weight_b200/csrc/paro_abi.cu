@@ -289,18 +289,21 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
   p.total = round_up((size_t)M * K * 2, 256);   // X_r, written when rotating
   if (p.decode) {
     p.nt = M <= 8 ? 1 : 2;
-    // Configuration by shape class, from a sweep on B200 over the Llama-3-8B
+    // Configuration by shape class, from sweeps on B200 over the Llama-3-8B
     // decode shapes (column tile, k-parts, stages, split along K):
     //   wide (N > 4096, e.g. gate/up):      256 columns, 2 k-parts, 4-stage ring, split 2
     //   deep (N <= 4096, K > 4096, down):   128 columns, 2 k-parts, 4-stage ring, split 8
-    //   square/narrow (q, o, k, v):         128 columns, 4 k-parts, 8 stages, split 4 (8 if N <= 2048)
+    //   square/narrow (q, o, k, v), M <= 8: 128 columns, 4 k-parts, 8 stages, split 4 (8 if N <= 2048)
+    //   square/narrow, 8 < M <= 16:         64 columns, 4 k-parts, 8 stages, split 2 (8 if N <= 2048)
     int tile, want;
     if (N > 4096) {
       tile = 256; p.variant = 0; want = 2;
     } else if (K > 4096) {
       tile = 128; p.variant = 3; want = 8;
-    } else {
+    } else if (M <= 8) {
       tile = 128; p.variant = 2; want = N <= 2048 ? 8 : 4;
+    } else {
+      tile = 64; p.variant = 5; want = N <= 2048 ? 8 : 2;
     }
     p.n_tiles = (int)((N + tile - 1) / tile);
     int s = 1;
@@ -348,7 +351,8 @@ int launch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
   CUtensorMap tmW, tmS, tmZ, tmX;
   const bool ok =
       encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, L::WORDS,
-                L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) &&
+                L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                    : (L::ROW_BYTES == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE)) &&
       encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, (uint32_t)gmax,
                 NTILE, CU_TENSOR_MAP_SWIZZLE_NONE) &&
       encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, (uint32_t)gmax,
@@ -356,9 +360,11 @@ int launch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
       encode_x_chunks(&tmX, x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP, (uint32_t)(2 * gmax));
   if (!ok) return PARO_ERR_CUDA;
   auto k = w4_gemv_kernel<NT, KP, NTILE, STAGES>;
-  if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
+  if (!allow_smem(k, L::smem(kGvMaxGroups))) return PARO_ERR_CUDA;
   const dim3 grid((unsigned)((N + NTILE - 1) / NTILE), (unsigned)plan.splits, 1);
-  return launch_ex(k, grid, dim3(L::THREADS), L::SMEM, s, pdl, (unsigned)plan.splits, tmW, tmX,
+  // launched with the largest footprint (one CTA per SM): two CTAs of one
+  // grid packed onto an SM stream slower than the same CTAs spread out
+  return launch_ex(k, grid, dim3(L::THREADS), (size_t)L::smem(kGvMaxGroups), s, pdl, (unsigned)plan.splits, tmW, tmX,
                    tmS, tmZ, bias, y, (int)M, (int)N, (int)K, gmax);
 }
 
@@ -369,6 +375,7 @@ int dispatch_gemv(const LinearPlan& plan, const void* qweight, const void* qzero
   switch (plan.variant) {
     case 0: return launch_gemv<NT, 2, 256, 4>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
     case 2: return launch_gemv<NT, 4, 128, 8>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
+    case 5: return launch_gemv<NT, 4, 64, 8>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
     default: return launch_gemv<NT, 2, 128, 4>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
   }
 }

@@ -43,7 +43,7 @@ __device__ __forceinline__ void load_rot_params(RotParam* prm, const int16_t* __
       j &= kGroup - 1;
     }
     float sn, cs;
-    sincosf(theta[(size_t)s * (K / 2) + (size_t)grp * (kGroup / 2) + p], &sn, &cs);
+    rot_sincos(theta[(size_t)s * (K / 2) + (size_t)grp * (kGroup / 2) + p], &sn, &cs);
     prm[idx] = RotParam{cs, sn, i, j};
   }
 }

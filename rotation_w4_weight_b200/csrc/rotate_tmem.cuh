@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
     }
     praw[idx] = (uint32_t)i | ((uint32_t)j << 16);
     float sn, c;
-    sincosf(theta[(size_t)s * (K / 2) + (size_t)grp * 64 + p], &sn, &c);
+    rot_sincos(theta[(size_t)s * (K / 2) + (size_t)grp * 64 + p], &sn, &c);
     float* csu = reinterpret_cast<float*>(cstab + s * L::CS_STAGE) + 4 * u;
     csu[w] = c;
     csu[2 + w] = sn;

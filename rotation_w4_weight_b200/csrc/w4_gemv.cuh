@@ -61,17 +61,22 @@ struct GemvLayout {
   static constexpr int MP = 8 * NT;                       // token rows per CTA
   static constexpr int W_BYTES = 128 * WORDS * 4;         // one group of qweight
   static constexpr int STAGE = ((W_BYTES + 1023) / 1024) * 1024;
-  // resident for the whole kernel: X_r as [64-column chunk][token][64] (two
-  // chunks per group), scales [group][NTILE], zero words [group][WORDS]
+  // resident for the whole kernel, laid out for the launch's largest group
+  // range gmax: X_r as [64-column chunk][token][64] (two chunks per group),
+  // scales [group][NTILE], zero words [group][WORDS]; then the split-K inbox
+  // and the barriers.
   static constexpr int XG_BYTES = 2 * MP * 128;           // X_r of one group
   static constexpr int X_OFF = STAGES * STAGE;
-  static constexpr int S_OFF = X_OFF + kGvMaxGroups * XG_BYTES;
-  static constexpr int Z_OFF = S_OFF + kGvMaxGroups * NTILE * 2;
-  static constexpr int INBOX_OFF = ((Z_OFF + kGvMaxGroups * WORDS * 4 + 1023) / 1024) * 1024;
   static constexpr int INBOX_BYTES = KP * MP * NTILE * 4;   // partials [S][KP][MP][NTILE/S]
-  static constexpr int BAR_OFF = INBOX_OFF + INBOX_BYTES;   // full[], empty[], consts, X_r
-  static constexpr int SMEM = BAR_OFF + 16 * STAGES + 16 + 1024;
-  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  __host__ __device__ static constexpr int s_off(int gmax) { return X_OFF + gmax * XG_BYTES; }
+  __host__ __device__ static constexpr int z_off(int gmax) { return s_off(gmax) + gmax * NTILE * 2; }
+  __host__ __device__ static constexpr int inbox_off(int gmax) {
+    return ((z_off(gmax) + gmax * WORDS * 4 + 1023) / 1024) * 1024;
+  }
+  // barriers: full[STAGES], empty[STAGES], consts, X_r
+  __host__ __device__ static constexpr int bar_off(int gmax) { return inbox_off(gmax) + INBOX_BYTES; }
+  __host__ __device__ static constexpr int smem(int gmax) { return bar_off(gmax) + 8 * (2 * STAGES + 2) + 1024; }
+  static_assert(smem(kGvMaxGroups) <= 227 * 1024, "shared memory per CTA");
   static_assert(STAGES <= kGvMaxStages, "too many stages");
   // 128-byte swizzle needs 128-byte rows; 64-byte rows use the 64-byte swizzle
   static constexpr int ROW_BYTES = WORDS * 4;
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // 1024-byte aligned base, derived on the shared array so every access stays LDS/STS
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t base = smem_u32(sbase);
-  const uint32_t full0 = base + L::BAR_OFF;
+  const uint32_t full0 = base + L::bar_off(gmax);
   const uint32_t empty0 = full0 + 8 * kGvStages;
   const uint32_t cbar = empty0 + 8 * kGvStages;   // scales + zero words
   const uint32_t xbar = cbar + 8;                  // X_r
@@ -150,8 +155,8 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       // the tensor maps' boxes hold gmax groups (the largest range of any CTA;
       // rows past this CTA's range are loaded and not used)
       mbar_arrive_expect_tx(cbar, (uint32_t)(gmax * (NTILE * 2 + L::WORDS * 4)));
-      tma_load_2d(base + L::S_OFF, &tmS, cbar, n0, g_begin);
-      tma_load_2d(base + L::Z_OFF, &tmZ, cbar, n0 / 8, g_begin);
+      tma_load_2d(base + L::s_off(gmax), &tmS, cbar, n0, g_begin);
+      tma_load_2d(base + L::z_off(gmax), &tmZ, cbar, n0 / 8, g_begin);
       for (int i = 0; i < pre; ++i) {
         const uint32_t bar = full0 + 8 * i;
         mbar_arrive_expect_tx(bar, L::W_BYTES);
@@ -174,8 +179,9 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     // 16 ks + 2t + {0, 1, 8, 9} have (row & 7) = 2t + {0, 1, 0, 1}.
     const int wchunk = wcol >> 2, wword = (wcol & 3) * 4;
     constexpr int RB = L::ROW_BYTES;
-    // 128-byte rows: chunk ^ (row & 7); 64-byte rows (64-byte swizzle): chunk ^ ((row >> 1) & 3)
-    auto swz = [&](int row) -> int { return RB == 128 ? (row & 7) : ((row >> 1) & 3); };
+    // 128-byte rows: chunk ^ (row & 7); 64-byte rows (64-byte swizzle): chunk ^ ((row >> 1) & 3);
+    // 32-byte rows are not swizzled (four rows of a warp's load already span all banks)
+    auto swz = [&](int row) -> int { return RB == 128 ? (row & 7) : (RB == 64 ? ((row >> 1) & 3) : 0); };
     const uint32_t wo0 = (uint32_t)((2 * t) * RB + ((wchunk ^ swz(2 * t)) << 4) + wword);
     const uint32_t wo1 = (uint32_t)((2 * t + 1) * RB + ((wchunk ^ swz(2 * t + 1)) << 4) + wword);
     // X_r tile: token rows of 128 B per 64-column box; columns 16 ks + 2t (+8)
@@ -191,6 +197,8 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
         xo[q][nt][1] = (uint32_t)(tok * 128 + (((c0 + 1) ^ (tok & 7)) << 4) + 4 * t);
       }
     const uint32_t ones[4] = {kGvOnes, kGvOnes, kGvOnes, kGvOnes};
+    const unsigned char* const sbase_s = sbase + L::s_off(gmax);
+    const unsigned char* const zbase = sbase + L::z_off(gmax);
 
     // scales, zero words and X_r of every group of the range (once)
     bool consts_ready = mbar_wait_bounded(cbar, 0);
@@ -201,8 +209,8 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       const bool ready = mbar_wait_bounded(full0 + 8 * s, (i / kGvStages) & 1) && consts_ready;
       if (ready) {
         // group constants for this thread's 8 columns
-        const uint32_t zw = *reinterpret_cast<const uint32_t*>(sbase + L::Z_OFF + (i * L::WORDS + wcol) * 4);
-        const uint4 s8 = *reinterpret_cast<const uint4*>(sbase + L::S_OFF + i * NTILE * 2 + wcol * 16);
+        const uint32_t zw = *reinterpret_cast<const uint32_t*>(zbase + (i * L::WORDS + wcol) * 4);
+        const uint4 s8 = *reinterpret_cast<const uint4*>(sbase_s + i * NTILE * 2 + wcol * 16);
         float cg[4][NT][4];
         float rs[NT][4];
 #pragma unroll
@@ -279,7 +287,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const int S = gridDim.y;
   const int cols = kGvTile / S;                    // columns owned by each CTA of the cluster
   const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
-  const uint32_t inbox = base + L::INBOX_OFF;      // fp32 [S][KP][MP][cols]
+  const uint32_t inbox = base + L::inbox_off(gmax);  // fp32 [S][KP][MP][cols]
   if (warp != 0) {
     const int owner = (8 * wcol) / cols;
     const int c0 = 8 * wcol - owner * cols;
@@ -317,7 +325,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // every partial pushed into this CTA's inbox is complete and visible after this
   if (S > 1) cluster_sync();
   else __syncthreads();
-  const float* box = reinterpret_cast<const float*>(sbase + L::INBOX_OFF);
+  const float* box = reinterpret_cast<const float*>(sbase + L::inbox_off(gmax));
   for (int idx = tid; idx < nq; idx += L::THREADS) {
     const int tl = idx / (cols / 4);
     const int c = 4 * (idx % (cols / 4));

@@ -170,6 +170,27 @@ def test_linear_vs_oracle(M, K, N):
     assert lin_err(got, ref) <= LIN_TOL
 
 
+@pytest.mark.parametrize("krot", [1, 8, 12])   # decode rotation inside the GEMV up to 8 stages
+@pytest.mark.parametrize("M", [1, 9, 16])
+def test_linear_decode_rotation_paths(M, krot):
+    lay = synth.make_layer("k", 1024, 512, seed=90 + krot, krot=krot, bias_std=0.01, n_outliers=4)
+    d = layer_to_device(lay)
+    x = synth.make_activations(lay, M)
+    got = run_linear(lay, d, x).cpu().numpy().astype(np.float64)
+    ref = oracle_linear(lay, x)
+    assert lin_err(got, ref) <= LIN_TOL
+
+
+def test_linear_decode_scales_only():
+    """krot = 0 with channel scales: the decode GEMV scales x itself."""
+    lay = synth.make_layer("c", 512, 1024, seed=91)
+    d = layer_to_device(lay)
+    x = synth.make_activations(lay, 5)
+    got = run_linear(lay, d, x, krot=0).cpu().numpy().astype(np.float64)
+    ref = oracle_linear(lay, x, krot=0)
+    assert lin_err(got, ref) <= LIN_TOL
+
+
 @pytest.mark.parametrize("M", [1, 16, 100])
 def test_linear_plain_awq_baseline(M):
     """krot = 0 and no channel scales: a plain AWQ W4 linear."""
