@@ -73,9 +73,9 @@ struct GemvLayout {
   __host__ __device__ static constexpr int inbox_off(int gmax) {
     return ((z_off(gmax) + gmax * WORDS * 4 + 1023) / 1024) * 1024;
   }
-  // barriers: full[STAGES], empty[STAGES], consts, X_r
+  // barriers: full[STAGES], empty[STAGES], consts, X_r, inbox
   __host__ __device__ static constexpr int bar_off(int gmax) { return inbox_off(gmax) + INBOX_BYTES; }
-  __host__ __device__ static constexpr int smem(int gmax) { return bar_off(gmax) + 8 * (2 * STAGES + 2) + 1024; }
+  __host__ __device__ static constexpr int smem(int gmax) { return bar_off(gmax) + 8 * (2 * STAGES + 3) + 1024; }
   static_assert(smem(kGvMaxGroups) <= 227 * 1024, "shared memory per CTA");
   static_assert(STAGES <= kGvMaxStages, "too many stages");
   // 128-byte swizzle needs 128-byte rows; 64-byte rows use the 64-byte swizzle
@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const uint32_t empty0 = full0 + 8 * kGvStages;
   const uint32_t cbar = empty0 + 8 * kGvStages;   // scales + zero words
   const uint32_t xbar = cbar + 8;                  // X_r
+  const uint32_t inbar = xbar + 8;                 // peers' split-K partials landed
 
   const int ntile = blockIdx.x, split = blockIdx.y;
   const int n0 = ntile * kGvTile;
@@ -119,6 +120,8 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const int g_end = (int)(((unsigned)(split + 1) * (unsigned)groups) / gridDim.y);
   const int ng = g_end - g_begin;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = gridDim.y;                          // CTAs of the cluster along K
+  const int mrows = min(L::MP, M);
 
   if (tid == 0) {
     for (int s = 0; s < kGvStages; ++s) {
@@ -127,13 +130,18 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     }
     mbar_init(cbar, 1);
     mbar_init(xbar, 1);
+    mbar_init(inbar, 1);
     fence_barrier_init();
+    // every peer's k-part partials of this CTA's columns, counted in bytes
+    if (S > 1) mbar_arrive_expect_tx(inbar, (uint32_t)((S - 1) * KP * mrows * (kGvTile / S) * 4));
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmS);
     tma_prefetch_desc(&tmZ);
   }
   __syncthreads();
+  // the peers may address this CTA's inbox barrier once every CTA has set its own up
+  if (S > 1) cluster_arrive_release();
 
   float acc[4][NT][4];
 #pragma unroll
@@ -281,13 +289,16 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // ---------------- reduction over k-parts and the split along K.  Every
   // consumer thread holds 8 consecutive columns for each of its tokens; it
   // writes them straight into the inbox of the CTA that owns those columns
-  // (slot [sender rank][k-part]); after one barrier each owner folds its
-  // inbox in a fixed order (deterministic), adds the bias and writes fp16 Y.
-  const int mrows = min(L::MP, M);
-  const int S = gridDim.y;
+  // (slot [sender rank][k-part]): its own with plain stores, a peer's with
+  // st.async counted on the peer's inbox barrier.  Each owner waits for its
+  // own stores (CTA barrier) and the peers' bytes (its mbarrier), then folds
+  // the inbox in a fixed order (deterministic), adds the bias and writes Y.
+  // No cluster-wide barrier at the end; a CTA leaves only once every byte
+  // addressed to it has landed.
   const int cols = kGvTile / S;                    // columns owned by each CTA of the cluster
   const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
   const uint32_t inbox = base + L::inbox_off(gmax);  // fp32 [S][KP][MP][cols]
+  if (S > 1) cluster_wait_acquire();               // every peer's inbox barrier is set up
   if (warp != 0) {
     const int owner = (8 * wcol) / cols;
     const int c0 = 8 * wcol - owner * cols;
@@ -302,9 +313,10 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
             make_float4(acc[0][nt][tt], acc[0][nt][2 + tt], acc[1][nt][tt], acc[1][nt][2 + tt]);
         const float4 v1 =
             make_float4(acc[2][nt][tt], acc[2][nt][2 + tt], acc[3][nt][tt], acc[3][nt][2 + tt]);
-        if (S > 1) {
-          st_cluster_f4(mapa_shared(off, (uint32_t)owner), v0);
-          st_cluster_f4(mapa_shared(off + 16, (uint32_t)owner), v1);
+        if (owner != (int)rank) {
+          const uint32_t rbar = mapa_shared(inbar, (uint32_t)owner);
+          st_async_f4(mapa_shared(off, (uint32_t)owner), v0, rbar);
+          st_async_f4(mapa_shared(off + 16, (uint32_t)owner), v1, rbar);
         } else {
           sts128(off, v0);
           sts128(off + 16, v1);
@@ -322,9 +334,9 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       bv = make_float4(__low2float(b0), __high2float(b0), __low2float(b1), __high2float(b1));
     }
   }
-  // every partial pushed into this CTA's inbox is complete and visible after this
-  if (S > 1) cluster_sync();
-  else __syncthreads();
+  // this CTA's own partials (CTA barrier) and every peer's (the inbox barrier)
+  __syncthreads();
+  if (S > 1 && !mbar_wait_bounded(inbar, 0)) flag_error(kErrTimeout);
   const float* box = reinterpret_cast<const float*>(sbase + L::inbox_off(gmax));
   for (int idx = tid; idx < nq; idx += L::THREADS) {
     const int tl = idx / (cols / 4);
