@@ -322,7 +322,7 @@ int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t
                       const int32_t* qweight, const int32_t* qzeros, const __half* scales,
                       const __half* bias, cudaStream_t s, bool pdl) {
   CUtensorMap tmA, tmW, tmS, tmZ;
-  bool ok = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, kTcBM, kTcBK,
+  bool ok = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, kTcMB * kTcBM, kTcBK,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, kTcBK, kTcBN / 8,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -331,7 +331,7 @@ int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t
             encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kTcBN / 8,
                       CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return PARO_ERR_CUDA;
-  const dim3 grid((unsigned)((N + kTcBN - 1) / kTcBN), (unsigned)((M + kTcBM - 1) / kTcBM), 1);
+  const dim3 grid((unsigned)((N + kTcBN - 1) / kTcBN), (unsigned)((M + kTcMB * kTcBM - 1) / (kTcMB * kTcBM)), 1);
   if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
   if (!allow_smem(w4_tc_gemm_kernel, TcLayout::SMEM)) return PARO_ERR_CUDA;
   return launch(w4_tc_gemm_kernel, grid, dim3(kTcThreads), TcLayout::SMEM, s, pdl, tmA, tmW, tmS,

@@ -4,18 +4,22 @@
 // transforms" and "Triton plans and tuning"):
 //   Y[m, n] = sum_k X_r[m, k] * (q[k, n] - z[k/128, n]) * s[k/128, n] + b[n]
 //
-// CTA tile: 128 token rows x 256 output columns, K in blocks of 64.
-//   A = X_r tile [128 tokens][64 k] fp16, K-major, brought by TMA with the
-//       128-byte swizzle (the UMMA canonical K-major SW128 layout).
+// CTA tile: 256 token rows x 256 output columns, K in blocks of 64, as two
+// 128-token accumulators that share every dequantised weight tile (the int4
+// -> fp16 work per tensor-core FLOP is half that of a 128-token tile).
+//   A = X_r tile [256 tokens][64 k] fp16, K-major, brought by TMA with the
+//       128-byte swizzle (the UMMA canonical K-major SW128 layout); token block
+//       b starts 16 KB in.
 //   B = W^T tile [256 columns][64 k] fp16, K-major, written by the dequant warps
 //       from the AWQ words in the canonical no-swizzle layout: 8x8 core matrices
 //       of 128 contiguous bytes, k-chunks 128 B apart (LBO), 8-row groups
 //       1040 B apart (SBO: one extra 16 bytes per group so the dequant stores
 //       of eight neighbouring groups hit eight different bank groups).
-//   D = fp32 accumulator [128 lanes = tokens][256 columns] in tensor memory.
+//   D = two fp32 accumulators [128 lanes = tokens][256 columns] in tensor
+//       memory (all 512 columns; one CTA per SM).
 // Warp roles (18 warps): warp 0 = TMA producer, warp 1 = TMEM allocator and
 // single-thread MMA issuer, warps 2..17 = dequant (k-chunk (warp-2)/2, 16 word
-// columns, 4 rows per lane) and then epilogue (the first 8 of them).  Two rings: a 4-deep TMA ring (A, the packed qweight tile
+// columns, 4 rows per lane) and then epilogue.  Two rings: a 3-deep TMA ring (A, the packed qweight tile
 // [64 rows][32 words] with 128-byte swizzle, the group's scales and zero words),
 // deep enough to cover the TMA round trip, and a 3-deep ring of dequantised B
 // tiles so the dequant warps run ahead of the tensor core.  Barriers: tma_full / tma_empty per TMA stage (bytes
@@ -34,10 +38,11 @@
 
 namespace paro {
 
-constexpr int kTcBM = 128;               // token rows per CTA
+constexpr int kTcBM = 128;               // token rows per accumulator (UMMA M)
+constexpr int kTcMB = 2;                 // accumulators (token blocks) per CTA
 constexpr int kTcBN = 256;               // output columns per CTA
 constexpr int kTcBK = 64;                // k per stage (128-byte rows)
-constexpr int kTcStages = 4;             // TMA ring: A, packed weights, scales, zeros
+constexpr int kTcStages = 3;             // TMA ring: A, packed weights, scales, zeros
 constexpr int kTcBBufs = 3;              // dequantised B ring
 constexpr int kTcDequantWarps = 16;      // (k-chunk, half of its 8 rows) per warp
 constexpr int kTcThreads = 32 * (2 + kTcDequantWarps);
@@ -46,8 +51,9 @@ constexpr int kTcBLbo = 128;             // B: bytes between k-chunks
 
 struct TcLayout {
   // TMA stage (1024-aligned): A | packed weights | scales | zeros
-  static constexpr int A_OFF = 0;                          // 16384 B
-  static constexpr int A_BYTES = kTcBM * kTcBK * 2;
+  static constexpr int A_OFF = 0;                          // 32768 B
+  static constexpr int A_BLOCK = kTcBM * kTcBK * 2;         // one token block
+  static constexpr int A_BYTES = kTcMB * A_BLOCK;
   static constexpr int WQ_OFF = A_OFF + A_BYTES;           // 8192 B, 1024-aligned
   static constexpr int WQ_BYTES = kTcBK * (kTcBN / 8) * 4;
   static constexpr int S_OFF = WQ_OFF + WQ_BYTES;          // 512 B
@@ -65,6 +71,7 @@ struct TcLayout {
   static constexpr int NBARS = 2 * kTcStages + 2 * kTcBBufs + 1;
   static constexpr int MISC_OFF = BAR_OFF + 8 * NBARS;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 // instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M=128, N=256
@@ -103,7 +110,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = blockIdx.x * kTcBN;
-  const int tok0 = blockIdx.y * kTcBM;
+  const int tok0 = blockIdx.y * (kTcMB * kTcBM);
   const int nk = K / kTcBK;
 
   if (tid == 0) {
@@ -123,8 +130,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     tma_prefetch_desc(&tmS);
     tma_prefetch_desc(&tmZ);
   }
-  if (warp == 1) {                      // the whole warp allocates 256 TMEM columns
-    tmem_alloc(smem_u32(tmem_slot), kTcBN);
+  if (warp == 1) {                      // the whole warp allocates 2 x 256 TMEM columns
+    tmem_alloc(smem_u32(tmem_slot), kTcMB * kTcBN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -170,11 +177,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         const uint32_t b0 = base + L::B_RING + b * L::B_STRIDE;
 #pragma unroll
         for (int ks = 0; ks < kTcBK / 16; ++ks) {
-          // A: 128-byte swizzled rows, 8-row groups 1024 B apart; +32 B per 16 k
-          const uint64_t ad = umma_desc(a0 + ks * 32, 16, 1024, 2);
           // B: no swizzle, k-chunks LBO apart, 8-row groups SBO apart; 2 chunks per 16 k
           const uint64_t bd = umma_desc(b0 + ks * 2 * kTcBLbo, kTcBLbo, kTcBSbo, 0);
-          umma_f16(tmem_d, ad, bd, kTcIdesc, (kb > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+          for (int mb = 0; mb < kTcMB; ++mb) {
+            // A: 128-byte swizzled rows, 8-row groups 1024 B apart; +32 B per 16 k
+            const uint64_t ad = umma_desc(a0 + mb * L::A_BLOCK + ks * 32, 16, 1024, 2);
+            umma_f16(tmem_d + (uint32_t)(mb * kTcBN), ad, bd, kTcIdesc, (kb > 0 || ks > 0) ? 1u : 0u);
+          }
         }
         umma_commit(tma_empty0 + 8 * s);   // the TMA stage and ...
         umma_commit(b_empty0 + 8 * b);     // ... the B buffer are free once these MMAs finish
@@ -194,19 +204,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
       const int s = kb % kTcStages, bb = kb % kTcBBufs;
       if (!tc_wait(tma_full0 + 8 * s, (kb / kTcStages) & 1, abort)) break;
       if (kb >= kTcBBufs && !tc_wait(b_empty0 + 8 * bb, ((kb / kTcBBufs) - 1) & 1, abort)) break;
-      unsigned char* stp = sbase + s * L::STAGE;
-      unsigned char* btile = sbase + L::B_RING + bb * L::B_STRIDE;
+      // shared-memory addresses (explicit ld/st.shared: no generic-address path)
+      const uint32_t stp = base + (uint32_t)(s * L::STAGE);
+      const uint32_t btile = base + (uint32_t)(L::B_RING + bb * L::B_STRIDE);
       // 4 words of rows 8c+4h .. +3, word column w (128-byte swizzled rows)
       uint32_t wv[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int row = 8 * c + 4 * h + r;
-        wv[r] = *reinterpret_cast<const uint32_t*>(stp + L::WQ_OFF + row * 128 +
-                                                   ((((w >> 2) ^ (row & 7))) << 4) + (w & 3) * 4);
+        wv[r] = lds32(stp + (uint32_t)(L::WQ_OFF + row * 128 + ((((w >> 2) ^ (row & 7))) << 4) + (w & 3) * 4));
       }
       // group zero points and scales of the 8 columns (column j at nibble j/2 + 4 (j & 1))
-      const uint32_t zw = *reinterpret_cast<const uint32_t*>(stp + L::Z_OFF + w * 4);
-      const uint4 s8 = *reinterpret_cast<const uint4*>(stp + L::S_OFF + w * 16);
+      const uint32_t zw = lds32(stp + (uint32_t)(L::Z_OFF + w * 4));
+      const uint4 s8 = lds128(stp + (uint32_t)(L::S_OFF + w * 16));
       const uint32_t sw[4] = {s8.x, s8.y, s8.z, s8.w};
       uint32_t outv[8][2];
 #pragma unroll
@@ -241,7 +251,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         uint2 o;
         o.x = hmul2_u32(hsub2_u32(outv[col][0], zz), sc);
         o.y = hmul2_u32(hsub2_u32(outv[col][1], zz), sc);
-        *reinterpret_cast<uint2*>(btile + w * kTcBSbo + c * kTcBLbo + col * 16 + h * 8) = o;
+        sts64(btile + (uint32_t)(w * kTcBSbo + c * kTcBLbo + col * 16 + h * 8), o);
       }
       fence_proxy_async_smem();         // make the B tile visible to the tensor core
       __syncwarp();
@@ -249,20 +259,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     }
 
     // ------------------------------------------------------------ epilogue
-    // warp w reads TMEM lanes 32*(w%4) .. +31 (its token rows); warps 2..5 take
-    // columns 0..127, warps 6..9 columns 128..255; warps 10..17 are done.
+    // warp w reads TMEM lanes 32*(w%4) .. +31 (its token rows of a block);
+    // warps 2..5 take block 0 columns 0..127, 6..9 block 0 columns 128..255,
+    // 10..13 and 14..17 the same halves of block 1.
     pdl_wait_primary();                 // previous kernels are complete before Y is written
-    const bool ok = warp < 10 && tc_wait(accum_full, 0, abort);
+    const bool ok = tc_wait(accum_full, 0, abort);
     tc_fence_after();
     const int quarter = warp & 3;
-    const int chalf = (warp - 2) >> 2;
-    const int tok = tok0 + 32 * quarter + lane;
+    const int cq = (warp - 2) >> 2;                 // 0..3
+    const int mb = cq >> 1, chalf = cq & 1;
+    const int tok = tok0 + mb * kTcBM + 32 * quarter + lane;
     if (ok) {
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         const int col0 = chalf * 128 + cb * 32;
         uint32_t r[32];
-        tmem_ld32(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)col0, r);
+        tmem_ld32(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(mb * kTcBN + col0), r);
         tmem_ld_wait_tie(r);
         const int n = n0 + col0;
         if (tok < M && n < N) {
@@ -296,7 +308,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_d, kTcBN);
+    tmem_dealloc(tmem_d, kTcMB * kTcBN);
   }
 }
 
