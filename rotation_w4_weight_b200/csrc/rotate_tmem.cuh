@@ -17,7 +17,8 @@
 // compile-time register indices, and writes the results with bulk stores in
 // that "slot" order into the other of two 128-column buffers; the next stage's
 // gather table is composed with that order.  The two warps of a lane quadrant
-// meet at a named barrier once per stage.  The last stage scatters to the
+// meet at a named barrier once per stage (four warps per quadrant measured
+// slower: more barrier traffic, no better latency hiding).  The last stage scatters to the
 // natural channel order and bulk loads bring each warp's half row back.
 // Tensor memory is split between the SM sub-partitions, so a stage's data
 // movement does not funnel through the one shared-memory pipe that bounds
@@ -40,7 +41,8 @@
 namespace paro {
 
 constexpr int kRtRows = 128;
-constexpr int kRtThreads = 256;          // 8 warps: (lane quadrant, pair half)
+constexpr int kRtWpq = 2;                // warps per TMEM lane quadrant (each takes 128/kRtWpq slots)
+constexpr int kRtThreads = 128 * kRtWpq; // warps: (lane quadrant, slot range)
 constexpr int kRtCols = 256;             // two 128-column buffers
 constexpr int kRtMaxCtasPerSm = 2;       // 2 x 256 TMEM columns
 constexpr int kRtAbsMaxKrot = 16;        // per-quadrant address tables up to this many stages
@@ -71,16 +73,16 @@ struct RtLayout {
   }
 };
 
-// The two warps of lane quadrant qd: their TMEM accesses so far are complete
+// The warps of lane quadrant qd: their TMEM accesses so far are complete
 // and visible to each other.  Barrier ids are immediates (5 hardware barriers).
 __device__ __forceinline__ void rt_quadrant_sync(int qd) {
   tmem_st_wait();
   tc_fence_before();
   switch (qd) {
-    case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
-    case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
-    case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
-    default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+    case 0: asm volatile("bar.sync 1, %0;" ::"n"(32 * kRtWpq) : "memory"); break;
+    case 1: asm volatile("bar.sync 2, %0;" ::"n"(32 * kRtWpq) : "memory"); break;
+    case 2: asm volatile("bar.sync 3, %0;" ::"n"(32 * kRtWpq) : "memory"); break;
+    default: asm volatile("bar.sync 4, %0;" ::"n"(32 * kRtWpq) : "memory"); break;
   }
   tc_fence_after();
 }
@@ -88,7 +90,7 @@ __device__ __forceinline__ void rt_quadrant_sync(int qd) {
 // grid: (K/128, row-tile slots), block 256.  tmX is x as [M, K] fp16 with box
 // {64 channels, 128 rows}, 128-byte swizzle (rows past M read as zeros).
 template <bool ABS>
-__global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
+__global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kernel(
     const __grid_constant__ CUtensorMap tmX, __half* xr, const float* __restrict__ cs,
     const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot) {
   using L = RtLayout;
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
 
   const int grp = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, h = warp >> 2;            // lane quadrant, pair half
+  const int qd = warp & 3, h = warp >> 2;            // lane quadrant, slot range
   const int ntiles = (M + kRtRows - 1) / kRtRows;
   const int gy = (int)gridDim.y;
 
@@ -208,26 +210,28 @@ __global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
   }
   __syncthreads();
 
+  constexpr int SW = 128 / kRtWpq;                   // slots (channels) per warp
   const int r = 32 * qd + lane;                      // row within the tile = TMEM lane
   const uint32_t lbase = tmem0 + ((uint32_t)(32 * qd) << 16);
   const uint32_t goff = ABS ? 0u : lbase;            // added to a table entry
-  // this warp's 64 slots of stage 0 and of the final scatter
-  const uint32_t g_half = smem_u32(gtab + (ABS ? (size_t)qd * krot * 128 : 0) + 64 * h);
-  const uint32_t f_half = smem_u32(ftab + (ABS ? qd * 128 : 0) + 64 * h);
-  const uint32_t cs_half = smem_u32(cstab) + 256u * h;              // units 16h .. 16h+15
-  const float4* scale4 = reinterpret_cast<const float4*>(scale + 64 * h);
+  // this warp's SW slots of stage 0 and of the final scatter
+  const uint32_t g_part = smem_u32(gtab + (ABS ? (size_t)qd * krot * 128 : 0) + SW * h);
+  const uint32_t f_part = smem_u32(ftab + (ABS ? qd * 128 : 0) + SW * h);
+  const uint32_t cs_part = smem_u32(cstab) + 4u * SW * h;            // units SW/4 * h ..
+  const float4* scale4 = reinterpret_cast<const float4*>(scale + SW * h);
   const uint32_t rsw = (uint32_t)(r & 7);            // swizzle phase of row r
 
   int it = 0;
   for (int tile = blockIdx.y; tile < ntiles; tile += gy, ++it) {
     const int buf = it & 1;
-    // ---- row r, channels 64h .. 64h+63: 8 swizzled 16-byte chunks of box h, scaled
+    // ---- row r, channels SW*h .. SW*h+SW-1: swizzled 16-byte chunks, scaled
     if (!mbar_wait_bounded(bar0 + 8 * buf, (uint32_t)((it >> 1) & 1))) *abort_flag = 1;
-    uint32_t v[64];
-    const unsigned char* rowp = sb + buf * L::TILE + h * L::BOX + r * 128;
+    uint32_t v[SW];
+    const unsigned char* rowp = sb + buf * L::TILE + ((SW * h) >> 6) * L::BOX + r * 128;
+    const int q0 = ((SW * h) & 63) >> 3;             // first 16-byte chunk in the box row
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(rowp + ((((uint32_t)q) ^ rsw) << 4));
+    for (int q = 0; q < SW / 8; ++q) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(rowp + ((((uint32_t)(q0 + q)) ^ rsw) << 4));
       const __half2* hv = reinterpret_cast<const __half2*>(&raw);
       const float4 sa = scale4[2 * q], sc = scale4[2 * q + 1];
       const float2 s2[4] = {make_float2(sa.x, sa.y), make_float2(sa.z, sa.w), make_float2(sc.x, sc.y),
@@ -251,30 +255,32 @@ __global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
     }
 
     if (krot > 0) {
-      tmem_st32(lbase + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_st32(lbase + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+#pragma unroll
+      for (int b = 0; b < SW / 32; ++b)
+        tmem_st32(lbase + SW * h + 32 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
       rt_quadrant_sync(qd);
       for (int s = 0; s < krot; ++s) {
-        // gather this warp's 64 slots; table reads run four 16-byte loads ahead
-        const uint32_t gs = g_half + (uint32_t)s * 512u;
+        // gather this warp's SW slots; table reads run four 16-byte loads ahead
+        const uint32_t gs = g_part + (uint32_t)s * 512u;
         uint4 g[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) g[k] = lds128(gs + 16 * k);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
+        for (int k = 0; k < SW / 4; ++k) {
           const uint4 a = g[k & 3];
           v[4 * k] = tmem_ld1(a.x + goff);
           v[4 * k + 1] = tmem_ld1(a.y + goff);
           v[4 * k + 2] = tmem_ld1(a.z + goff);
           v[4 * k + 3] = tmem_ld1(a.w + goff);
-          if (k + 4 < 16) g[k & 3] = lds128(gs + 16 * (k + 4));
+          if (k + 4 < SW / 4) g[k & 3] = lds128(gs + 16 * (k + 4));
         }
         tmem_ld_wait_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        // rotate the 16 units (A = slots 0,1; B = slots 2,3)
-        const uint32_t cst = cs_half + (uint32_t)s * (uint32_t)L::CS_STAGE;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
+        for (int b = 1; b < SW / 32; ++b) tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
+        // rotate the SW/4 units (A = slots 0,1; B = slots 2,3)
+        const uint32_t cst = cs_part + (uint32_t)s * (uint32_t)L::CS_STAGE;
+#pragma unroll
+        for (int k = 0; k < SW / 4; ++k) {
           const uint4 t = lds128(cst + 16 * k);      // (c0, c1, s0, s1)
           const float2 C = make_float2(__uint_as_float(t.x), __uint_as_float(t.y));
           const float2 S = make_float2(__uint_as_float(t.z), __uint_as_float(t.w));
@@ -289,14 +295,14 @@ __global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
           v[4 * k + 3] = __float_as_uint(B2.y);
         }
         if (s + 1 < krot) {
-          const uint32_t d = lbase + (uint32_t)((s + 1) & 1) * 128u + 64u * h;
-          tmem_st32(d, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-          tmem_st32(d + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          const uint32_t d = lbase + (uint32_t)((s + 1) & 1) * 128u + (uint32_t)(SW * h);
+#pragma unroll
+          for (int b = 0; b < SW / 32; ++b) tmem_st32(d + 32 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
         } else {
           // last stage: scatter to the natural channel order
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const uint4 f = lds128(f_half + 16 * k);
+          for (int k = 0; k < SW / 4; ++k) {
+            const uint4 f = lds128(f_part + 16 * k);
             tmem_st1(f.x + goff, v[4 * k]);
             tmem_st1(f.y + goff, v[4 * k + 1]);
             tmem_st1(f.z + goff, v[4 * k + 2]);
@@ -305,19 +311,20 @@ __global__ void __launch_bounds__(kRtThreads) rotate_tmem_kernel(
         }
         rt_quadrant_sync(qd);
       }
-      const uint32_t fb = lbase + (uint32_t)(krot & 1) * 128u + 64u * h;
-      tmem_ld32(fb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(fb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      const uint32_t fb = lbase + (uint32_t)(krot & 1) * 128u + (uint32_t)(SW * h);
+#pragma unroll
+      for (int b = 0; b < SW / 32; ++b) tmem_ld32(fb + 32 * b, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
       tmem_ld_wait_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+#pragma unroll
+      for (int b = 1; b < SW / 32; ++b) tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
     }
 
-    // ---- fp16 (round to nearest), row r, channels 64h .. 64h+63
+    // ---- fp16 (round to nearest), row r, channels SW*h .. SW*h+SW-1
     const int row = tile * kRtRows + r;
     if (row < M) {
-      __half* dstp = xr + (size_t)row * K + (size_t)grp * kGroup + 64 * h;
+      __half* dstp = xr + (size_t)row * K + (size_t)grp * kGroup + SW * h;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < SW / 8; ++q) {
         uint4 out;
         __half2* hv = reinterpret_cast<__half2*>(&out);
 #pragma unroll
