@@ -229,6 +229,14 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
     return launch(rotate_tmem_kernel<false>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
                   pairs, theta, (int)M, (int)K, krot);
   }
+  // Decode batches with few stages: one warp per row, no block barrier per stage.
+  if (M <= 16 && krot <= kRrMaxKrot) {
+    const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + kRrWarps - 1) / kRrWarps));
+    const int warps = M < kRrWarps ? (int)M : kRrWarps;
+    if (!allow_smem(rotate_rows_kernel, RrLayout::bytes(kRrMaxKrot))) return PARO_ERR_CUDA;
+    return launch(rotate_rows_kernel, grid, dim3(32 * warps), RrLayout::bytes(krot), stream, true, x, xr,
+                  cs, pairs, theta, (int)M, (int)K, krot);
+  }
   // rows per CTA: 4 for decode-sized batches (more CTAs, shorter latency),
   // 32..64 otherwise (conflict-free 32-row warp accesses)
   const int rows = M <= 16 ? 4 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));

@@ -144,6 +144,108 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Decode batches (M <= 16, krot <= 8): one warp per token row of a group, so
+// no block-wide barrier sits between stages.  The CTA first turns the stage
+// tables into per-channel form (partner channel, cos, signed sin: channel i of
+// pair (i, j) gets +sin, channel j gets -sin, so both updates read
+// x' = x cos + x_partner sin_signed, the same fma order as rotate_kernel); a
+// lane keeps its four channels' entries for every stage in registers.  Per
+// stage a warp publishes its row (128 fp32) in its own shared buffer, reads the
+// four partner values and updates its channels.  Tables are layer constants,
+// built before waiting for the previous kernel; x is read after.
+constexpr int kRrWarps = 8;                // token rows per CTA
+constexpr int kRrMaxKrot = 8;              // stages kept in registers
+
+struct RrLayout {
+  // partner[krot][128] u8 | cos[krot][128] f32 | signed sin[krot][128] f32 | row buffers[kRrWarps][128] f32
+  __host__ __device__ static constexpr size_t cos_off(int krot) { return ((size_t)krot * 128 + 15) / 16 * 16; }
+  __host__ __device__ static constexpr size_t sin_off(int krot) { return cos_off(krot) + (size_t)krot * 512; }
+  __host__ __device__ static constexpr size_t row_off(int krot) { return sin_off(krot) + (size_t)krot * 512; }
+  __host__ __device__ static constexpr size_t bytes(int krot) { return row_off(krot) + kRrWarps * 512; }
+};
+
+__global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(
+    const __half* x, __half* xr, const float* __restrict__ cs, const int16_t* __restrict__ pairs,
+    const float* __restrict__ theta, int M, int K, int krot) {
+  pdl_launch_dependents();                         // the GEMV may start streaming weights
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint8_t* partner = smem_raw;
+  float* cosv = reinterpret_cast<float*>(smem_raw + RrLayout::cos_off(krot));
+  float* sinv = reinterpret_cast<float*>(smem_raw + RrLayout::sin_off(krot));
+  const int grp = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.y * kRrWarps + warp;
+
+  // ---- per-channel tables (identity first, so every entry is defined)
+  for (int idx = tid; idx < krot * 128; idx += blockDim.x) {
+    partner[idx] = (uint8_t)(idx & 127);
+    cosv[idx] = 1.f;
+    sinv[idx] = 0.f;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < krot * 64; idx += blockDim.x) {
+    const int st = idx >> 6, p = idx & 63;
+    const uint32_t pr = *reinterpret_cast<const uint32_t*>(pairs + (size_t)st * K + (size_t)grp * kGroup + 2 * p);
+    uint32_t i = pr & 0xFFFFu, j = pr >> 16;
+    if ((i | j) >= 128u) {                         // masked to the group, flagged
+      flag_error(kErrPairIndex);
+      i &= 127u;
+      j &= 127u;
+    }
+    float sn, c;
+    rot_sincos(theta[(size_t)st * (K / 2) + (size_t)grp * 64 + p], &sn, &c);
+    partner[st * 128 + i] = (uint8_t)j;
+    cosv[st * 128 + i] = c;
+    sinv[st * 128 + i] = sn;
+    partner[st * 128 + j] = (uint8_t)i;
+    cosv[st * 128 + j] = c;
+    sinv[st * 128 + j] = -sn;
+  }
+  __syncthreads();
+  const int ch = 4 * lane;                         // this lane's channels ch .. ch+3
+  uint32_t pw[kRrMaxKrot];
+  float4 cf[kRrMaxKrot], sf[kRrMaxKrot];
+#pragma unroll
+  for (int st = 0; st < kRrMaxKrot; ++st) {
+    if (st < krot) {
+      pw[st] = *reinterpret_cast<const uint32_t*>(partner + st * 128 + ch);
+      cf[st] = *reinterpret_cast<const float4*>(cosv + st * 128 + ch);
+      sf[st] = *reinterpret_cast<const float4*>(sinv + st * 128 + ch);
+    }
+  }
+  float4 csv = make_float4(1.f, 1.f, 1.f, 1.f);
+  if (cs != nullptr) csv = *reinterpret_cast<const float4*>(cs + (size_t)grp * kGroup + ch);
+
+  pdl_wait_primary();                              // x may come from the previous kernel
+  if (row >= M) return;
+  const uint2 raw = *reinterpret_cast<const uint2*>(x + (size_t)row * K + (size_t)grp * kGroup + ch);
+  const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+  const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+  float v[4] = {lo.x * csv.x, lo.y * csv.y, hi.x * csv.z, hi.y * csv.w};
+  const uint32_t rb = smem_u32(smem_raw + RrLayout::row_off(krot) + warp * 512);
+#pragma unroll
+  for (int st = 0; st < kRrMaxKrot; ++st) {
+    if (st < krot) {
+      sts128(rb + 4u * ch, make_float4(v[0], v[1], v[2], v[3]));
+      __syncwarp();
+      float xp[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) xp[k] = __uint_as_float(lds32(rb + 4u * ((pw[st] >> (8 * k)) & 0xFFu)));
+      __syncwarp();                                // every lane has read before the next publish
+      const float c4[4] = {cf[st].x, cf[st].y, cf[st].z, cf[st].w};
+      const float s4[4] = {sf[st].x, sf[st].y, sf[st].z, sf[st].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = fmaf(v[k], c4[k], xp[k] * s4[k]);
+    }
+  }
+  const __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
+  uint2 out;
+  out.x = *reinterpret_cast<const uint32_t*>(&h0);
+  out.y = *reinterpret_cast<const uint32_t*>(&h1);
+  *reinterpret_cast<uint2*>(xr + (size_t)row * K + (size_t)grp * kGroup + ch) = out;
+}
+
 inline size_t rotate_smem_bytes(int rows, int krot) {
   const size_t tile = rows < 32 ? (size_t)kGroup * (rows + 1) * 4 : (size_t)kGroup * rows * 4;
   return (size_t)krot * (kGroup / 2) * sizeof(RotParam) + tile;
