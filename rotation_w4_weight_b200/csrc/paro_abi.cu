@@ -231,10 +231,10 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
   }
   // Decode batches with few stages: one warp per row, no block barrier per stage.
   if (M <= 16 && krot <= kRrMaxKrot) {
+    // always 8 warps: all of them build the tables, warps past the batch then leave
     const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + kRrWarps - 1) / kRrWarps));
-    const int warps = M < kRrWarps ? (int)M : kRrWarps;
     if (!allow_smem(rotate_rows_kernel, RrLayout::bytes(kRrMaxKrot))) return PARO_ERR_CUDA;
-    return launch(rotate_rows_kernel, grid, dim3(32 * warps), RrLayout::bytes(krot), stream, true, x, xr,
+    return launch(rotate_rows_kernel, grid, dim3(32 * kRrWarps), RrLayout::bytes(krot), stream, true, x, xr,
                   cs, pairs, theta, (int)M, (int)K, krot);
   }
   // rows per CTA: 4 for decode-sized batches (more CTAs, shorter latency),
