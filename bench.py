@@ -160,6 +160,32 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ----------------------------------------------------------------- multi-rank helpers
+def max_over_ranks(value, world, device):
+    """The largest `value` over all ranks (identity for one rank): every timed
+    number of a multi-GPU run is the slowest rank's."""
+    if world <= 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, steps, per_step, ms):
+    """Whole-job throughput: every rank runs `steps` steps of `per_step` units
+    (bytes or flops) in `ms` milliseconds (the slowest rank's time)."""
+    return world * steps * per_step / (ms * 1e-3)
+
+
+def workload_config(workload, world):
+    """The workload description shared by both arms' JSON lines."""
+    wl = WORKLOADS[workload]
+    layers = [synth.config_layers(wl["cfg"])[i] for i in wl["layers"]]
+    return {"workload": workload, "layers": [(l.name, l.K, l.N) for l in layers], "M": wl["Ms"],
+            "group_size": GROUP, "krot": KROT, "accumulate": "f32", "parallelism": f"replicas x{world}"}
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -251,10 +277,7 @@ def run_ours(args, rank, world, local_rank):
         replay(g)
         torch.cuda.synchronize(dev)
     clocks = sampler.stop()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     assert pb.device_status() == pb.PARO_OK
 
     # ---- dominant kernel, timed live: X_r is produced once per call shape by
@@ -329,28 +352,26 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e_steps
 
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     if decode:
-        value = world * args.steps * step_bytes / (ms * 1e-3) / 1e9
+        value = job_throughput(world, args.steps, step_bytes, ms) / 1e9
         unit = "GB/s"
-        e2e_val = step_bytes / (e2e_ms * 1e-3) / 1e9 * world
-        metric = f"rotated W4 linear decode HBM throughput ({args.workload})"
+        e2e_val = job_throughput(world, 1, step_bytes, e2e_ms) / 1e9
     else:
-        value = world * args.steps * step_flops / (ms * 1e-3) / 1e12
+        value = job_throughput(world, args.steps, step_flops, ms) / 1e12
         unit = "TFLOP/s"
-        e2e_val = step_flops / (e2e_ms * 1e-3) / 1e12 * world
-        metric = f"rotated W4 linear prefill tensor throughput ({args.workload})"
+        e2e_val = job_throughput(world, 1, step_flops, e2e_ms) / 1e12
+    metric = metric_name(args.workload)
 
     out = {
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
-        "config": {"workload": args.workload, "layers": [(l.name, l.K, l.N) for l in layers],
-                   "M": Ms, "group_size": GROUP, "krot": KROT, "accumulate": "f32",
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"weights cycled over {reps} device replicas "
-                         f"({reps * weight_bytes / 2**20:.0f} MiB > 3x L2)",
-                   "timing": "CUDA graph of the K steps, CUDA events, max over ranks"},
+        "config": dict(workload_config(args.workload, world),
+                       l2=f"weights cycled over {reps} device replicas "
+                          f"({reps * weight_bytes / 2**20:.0f} MiB > 3x L2)",
+                       timing="CUDA graph of the K steps, CUDA events, max over ranks"),
         "roofline": roof,
         "e2e": {"value": round(e2e_val, 2), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
@@ -396,7 +417,15 @@ def oracle_sample(workload, budget_s, max_steps=None):
                     return val, desc, t_total
 
 
+def metric_name(workload):
+    decode = WORKLOADS[workload]["kind"] == "decode"
+    return ("rotated W4 linear decode HBM throughput" if decode else
+            "rotated W4 linear prefill tensor throughput") + f" ({workload})"
+
+
 def run_reference(args, rank, world):
+    """The reference arm: the float64 oracle, on rank 0 only (other ranks return
+    None and exit without work)."""
     if rank != 0:
         return None
     wl = WORKLOADS[args.workload]
@@ -408,12 +437,12 @@ def run_reference(args, rank, world):
                                     max_steps=max(1, args.steps))
     unit = "GB/s" if decode else "TFLOP/s"
     return {
-        "impl": "reference", "metric": ("rotated W4 linear decode HBM throughput" if decode else
-                                        "rotated W4 linear prefill tensor throughput") + f" ({args.workload})",
+        "impl": "reference", "metric": metric_name(args.workload),
         "value": round(val, 5), "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(secs * 1e3 / max(1, args.steps), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": args.workload, "M": wl["Ms"]},
+        "data": "synthetic",
+        "config": dict(workload_config(args.workload, world), timing="host wall clock of the oracle"),
         "cpu_baseline": {"value": round(val, 5), "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": round(val, 5), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
