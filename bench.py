@@ -318,13 +318,16 @@ def run_ours(args, rank, world, local_rank):
                 "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
                 "bytes_per_launch": kern_bytes // n_launch, "peak_source": peaks["src"]}
     else:
+        # the GEMM graph runs for many milliseconds under the power cap: the
+        # sustained dense peak is its denominator (the burst one is for a kernel timed alone)
         achieved = kern_flops / (kern_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16"],
-                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16"], 4),
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_sus"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_sus"], 4),
                 "traffic": traffic_for("w4_tc_prefill"),
                 "kernel": "w4_tc_gemm_kernel (prefill tcgen05 GEMM)", "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
                 "flops_per_launch": kern_flops // n_launch,
-                "peak_source": peaks["src"] + " bf16 burst (fp16 runs at the bf16 rate)"}
+                "peak_source": peaks["src"] + " bf16 sustained (fp16 runs at the bf16 rate)",
+                "peak_burst": peaks["bf16"], "frac_of_burst": round(achieved / peaks["bf16"], 4)}
     del g2
 
     # ---- end to end through the public call with host buffers (pinned), per step:
