@@ -205,35 +205,36 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
         xo[q][nt][1] = (uint32_t)(tok * 128 + (((c0 + 1) ^ (tok & 7)) << 4) + 4 * t);
       }
     const uint32_t ones[4] = {kGvOnes, kGvOnes, kGvOnes, kGvOnes};
-    const unsigned char* const sbase_s = sbase + L::s_off(gmax);
-    const unsigned char* const zbase = sbase + L::z_off(gmax);
+    const uint32_t sq = base + (uint32_t)L::s_off(gmax);   // scales of the range
+    const uint32_t zq = base + (uint32_t)L::z_off(gmax);   // zero words of the range
 
     // scales, zero words and X_r of every group of the range (once)
     bool consts_ready = mbar_wait_bounded(cbar, 0);
     consts_ready = mbar_wait_bounded(xbar, 0) && consts_ready;
     for (int i = kpart; i < ng; i += KP) {
       const int s = i % kGvStages;
-      const unsigned char* stp = sbase + s * L::STAGE;
+      // explicit ld.shared: generic loads of shared memory take the long-latency path
+      const uint32_t stq = base + (uint32_t)(s * L::STAGE);
       const bool ready = mbar_wait_bounded(full0 + 8 * s, (i / kGvStages) & 1) && consts_ready;
       if (ready) {
         // group constants for this thread's 8 columns
-        const uint32_t zw = *reinterpret_cast<const uint32_t*>(zbase + (i * L::WORDS + wcol) * 4);
-        const uint4 s8 = *reinterpret_cast<const uint4*>(sbase_s + i * NTILE * 2 + wcol * 16);
+        const uint32_t zw = lds32(zq + (uint32_t)((i * L::WORDS + wcol) * 4));
+        const uint4 s8 = lds128(sq + (uint32_t)(i * NTILE * 2 + wcol * 16));
         float cg[4][NT][4];
         float rs[NT][4];
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const unsigned char* wrow = stp + ks * 16 * RB;
-          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wrow + wo0);
-          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wrow + wo1);
-          const uint32_t w8 = *reinterpret_cast<const uint32_t*>(wrow + 8 * RB + wo0);
-          const uint32_t w9 = *reinterpret_cast<const uint32_t*>(wrow + 8 * RB + wo1);
+          const uint32_t wrow = stq + (uint32_t)(ks * 16 * RB);
+          const uint32_t w0 = lds32(wrow + wo0);
+          const uint32_t w1 = lds32(wrow + wo1);
+          const uint32_t w8 = lds32(wrow + 8 * RB + wo0);
+          const uint32_t w9 = lds32(wrow + 8 * RB + wo1);
           uint32_t b0[NT], b1[NT];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const unsigned char* xb = sbase + L::X_OFF + i * L::XG_BYTES + (ks >> 2) * (L::MP * 128);
-            b0[nt] = *reinterpret_cast<const uint32_t*>(xb + xo[ks & 3][nt][0]);
-            b1[nt] = *reinterpret_cast<const uint32_t*>(xb + xo[ks & 3][nt][1]);
+            const uint32_t xb = base + (uint32_t)(L::X_OFF + i * L::XG_BYTES + (ks >> 2) * (L::MP * 128));
+            b0[nt] = lds32(xb + xo[ks & 3][nt][0]);
+            b1[nt] = lds32(xb + xo[ks & 3][nt][1]);
           }
           uint32_t elo01[4], ehi01[4], elo89[4], ehi89[4];
           gv_unpack4(prmt(w0, w1, 0x5410), elo01);
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // this CTA's own partials (CTA barrier) and every peer's (the inbox barrier)
   __syncthreads();
   if (S > 1 && !mbar_wait_bounded(inbar, 0)) flag_error(kErrTimeout);
-  const float* box = reinterpret_cast<const float*>(sbase + L::inbox_off(gmax));
+  const uint32_t box = base + (uint32_t)L::inbox_off(gmax);
   for (int idx = tid; idx < nq; idx += L::THREADS) {
     const int tl = idx / (cols / 4);
     const int c = 4 * (idx % (cols / 4));
@@ -345,8 +346,9 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     if (n >= N) continue;
     float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int q = 0; q < S * KP; ++q) {
-      const float4 v = *reinterpret_cast<const float4*>(box + ((size_t)q * L::MP + tl) * cols + c);
-      sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+      const uint4 v = lds128(box + (uint32_t)(((q * L::MP + tl) * cols + c) * 4));
+      sum.x += __uint_as_float(v.x); sum.y += __uint_as_float(v.y);
+      sum.z += __uint_as_float(v.z); sum.w += __uint_as_float(v.w);
     }
     if (bias != nullptr) {
       if (idx != tid) {
