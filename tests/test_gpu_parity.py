@@ -170,8 +170,10 @@ def test_linear_vs_oracle(M, K, N):
     assert lin_err(got, ref) <= LIN_TOL
 
 
-@pytest.mark.parametrize("krot", [1, 8, 12])   # decode rotation inside the GEMV up to 8 stages
-@pytest.mark.parametrize("M", [1, 9, 16])
+# rotation kernel choice at decode sizes: one warp per (group, row) up to 8
+# stages and 16 rows, the shared-memory kernel beyond
+@pytest.mark.parametrize("krot", [1, 8, 9, 12])
+@pytest.mark.parametrize("M", [1, 3, 4, 5, 9, 16])
 def test_linear_decode_rotation_paths(M, krot):
     lay = synth.make_layer("k", 1024, 512, seed=90 + krot, krot=krot, bias_std=0.01, n_outliers=4)
     d = layer_to_device(lay)
@@ -181,11 +183,12 @@ def test_linear_decode_rotation_paths(M, krot):
     assert lin_err(got, ref) <= LIN_TOL
 
 
-def test_linear_decode_scales_only():
-    """krot = 0 with channel scales: the decode GEMV scales x itself."""
+@pytest.mark.parametrize("M", [2, 5])
+def test_linear_decode_scales_only(M):
+    """krot = 0 with channel scales: a scaling-only pass ahead of the GEMV."""
     lay = synth.make_layer("c", 512, 1024, seed=91)
     d = layer_to_device(lay)
-    x = synth.make_activations(lay, 5)
+    x = synth.make_activations(lay, M)
     got = run_linear(lay, d, x, krot=0).cpu().numpy().astype(np.float64)
     ref = oracle_linear(lay, x, krot=0)
     assert lin_err(got, ref) <= LIN_TOL
