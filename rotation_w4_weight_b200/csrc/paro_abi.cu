@@ -84,7 +84,7 @@ bool encode_x_chunks(CUtensorMap* map, const void* x, uint64_t rows, uint64_t K,
 // ---------------------------------------------------------------- device facts
 struct DeviceInfo {
   int sms = 0;
-  size_t smem_per_sm = 0, smem_reserved_per_block = 0;
+  size_t smem_per_sm = 0, smem_reserved_per_block = 0, smem_optin = 0;
 };
 
 // SM count and shared-memory capacity of the current device, queried once per
@@ -99,13 +99,15 @@ const DeviceInfo& device_info() {
   std::lock_guard<std::mutex> lock(mu);
   DeviceInfo& d = table[dev];
   if (d.sms != 0) return d;
-  int sms = 0, per_sm = 0, reserved = 0;
+  int sms = 0, per_sm = 0, reserved = 0, optin = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
     return none;
   d.smem_per_sm = (size_t)per_sm;
   d.smem_reserved_per_block = (size_t)reserved;
+  d.smem_optin = (size_t)optin;
   d.sms = sms;
   return d;
 }
@@ -113,13 +115,13 @@ const DeviceInfo& device_info() {
 // ---------------------------------------------------------------- launches
 template <typename Kern, typename... Args>
 int launch_ex(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
-              unsigned cluster_y, Args... args) {
+              unsigned cluster_y, bool balance, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   unsigned n = 0;
   if (pdl) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -133,6 +135,12 @@ int launch_ex(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stre
     attr[n].val.clusterDim.z = 1;
     ++n;
   }
+  if (cluster_y > 1 && balance) {
+    // let the hardware place a cluster's CTAs by load rather than packing them
+    attr[n].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    attr[n].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
+    ++n;
+  }
   cfg.attrs = n ? attr : nullptr;
   cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? PARO_OK : PARO_ERR_CUDA;
@@ -141,7 +149,7 @@ int launch_ex(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stre
 template <typename Kern, typename... Args>
 int launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
            Args... args) {
-  return launch_ex(kernel, grid, block, smem, stream, pdl, 1u, args...);
+  return launch_ex(kernel, grid, block, smem, stream, pdl, 1u, false, args...);
 }
 
 // Raise the dynamic shared memory limit of a kernel once per device (callers
@@ -302,7 +310,8 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
     //   wide (N > 4096, e.g. gate/up):      256 columns, 2 k-parts, 4-stage ring, split 2
     //   deep (N <= 4096, K > 4096, down):   128 columns, 2 k-parts, 4-stage ring, split 8
     //   square/narrow (q, o, k, v), M <= 8: 128 columns, 4 k-parts, 8 stages, split 4 (8 if N <= 2048)
-    //   square/narrow, 8 < M <= 16:         64 columns, 4 k-parts, 8 stages, split 2 (8 if N <= 2048)
+    //   square, 8 < M <= 16:                64 columns, 4 k-parts, 8 stages, split 2
+    //   narrow (N <= 2048), 8 < M <= 16:    128 columns, 2 k-parts, 4 stages, split 8
     int tile, want;
     if (N > 4096) {
       tile = 256; p.variant = 0; want = 2;
@@ -310,8 +319,10 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
       tile = 128; p.variant = 3; want = 8;
     } else if (M <= 8) {
       tile = 128; p.variant = 2; want = N <= 2048 ? 8 : 4;
+    } else if (N <= 2048) {
+      tile = 128; p.variant = 3; want = 8;
     } else {
-      tile = 64; p.variant = 5; want = N <= 2048 ? 8 : 2;
+      tile = 64; p.variant = 5; want = 2;
     }
     p.n_tiles = (int)((N + tile - 1) / tile);
     int s = 1;
@@ -346,6 +357,20 @@ int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t
                 tmZ, bias, y, (int)M, (int)N, (int)K);
 }
 
+// Shared memory a GEMV CTA is launched with: at least what its group range
+// needs, padded so that no more than ceil(ctas / SMs) CTAs of the grid fit on
+// one SM.  CTAs of one grid packed onto an SM stream slower than the same CTAs
+// spread out, while a grid larger than the SM count must still fit in one wave.
+// Returns 0 when the device's limits are unknown.
+size_t gemv_footprint(size_t need, int64_t ctas) {
+  const DeviceInfo& dev = device_info();
+  if (dev.sms <= 0 || dev.smem_per_sm == 0 || dev.smem_optin < need) return 0;
+  const int64_t per_sm = (ctas + dev.sms - 1) / dev.sms;      // CTAs each SM must hold
+  const size_t pad = dev.smem_per_sm / (size_t)(per_sm + 1) + 1;  // one more no longer fits
+  const size_t want = pad > dev.smem_reserved_per_block ? pad - dev.smem_reserved_per_block : 0;
+  return std::min(dev.smem_optin, std::max(need, want));
+}
+
 // Decode GEMV launch: grid (column tiles, splits), one cluster of `splits`
 // CTAs along K per column tile.
 template <int NT, int KP, int NTILE, int STAGES>
@@ -368,11 +393,13 @@ int launch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
       encode_x_chunks(&tmX, x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP, (uint32_t)(2 * gmax));
   if (!ok) return PARO_ERR_CUDA;
   auto k = w4_gemv_kernel<NT, KP, NTILE, STAGES>;
-  if (!allow_smem(k, L::smem(kGvMaxGroups))) return PARO_ERR_CUDA;
   const dim3 grid((unsigned)((N + NTILE - 1) / NTILE), (unsigned)plan.splits, 1);
-  // launched with the largest footprint (one CTA per SM): two CTAs of one
-  // grid packed onto an SM stream slower than the same CTAs spread out
-  return launch_ex(k, grid, dim3(L::THREADS), (size_t)L::smem(kGvMaxGroups), s, pdl, (unsigned)plan.splits, tmW, tmX,
+  const size_t smem = gemv_footprint((size_t)L::smem(gmax), (int64_t)grid.x * grid.y);
+  if (smem == 0 || !allow_smem(k, device_info().smem_optin)) return PARO_ERR_CUDA;
+  // a grid larger than the SM count places its clusters by load (measured:
+  // 256-CTA grids of 8-CTA clusters ran 1-10 % faster; one-per-SM grids did not gain)
+  const bool balance = (int64_t)grid.x * grid.y > device_info().sms;
+  return launch_ex(k, grid, dim3(L::THREADS), smem, s, pdl, (unsigned)plan.splits, balance, tmW, tmX,
                    tmS, tmZ, bias, y, (int)M, (int)N, (int)K, gmax);
 }
 
