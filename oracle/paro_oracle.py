@@ -30,6 +30,17 @@ notes and pinned by a test where something can pin it):
   checkpoints is parity unpinned (no checkpoint is available).
 * Dequantisation is (q - z) * s with q, z unpacked codes 0..15.
 * theta and channel_scales are float32 at the boundary and are widened exactly.
+
+Weight side (the step before packing): W_r = W D R with D = 1 / channel_scales
+(section "Activation and weight transforms": the saved channel_scales are
+D^-1), the rows of W (out x in) taking the activations' stages; then the
+four-bit symmetric quantiser of section "Activation and weight transforms"
+(signed codes -8..7 exported unsigned with zero point 8, quantiser scales
+bounded to [1e-5, 1e5]).  The pages give the code range and the bounds but
+not the rounding of the quotient: round to nearest with ties to even is the
+reading taken (the rounding the pages name for the pseudo-quantisation
+kernels in section "STE acceleration kernels").  The quantiser scales are an
+input (learned during calibration).
 """
 from __future__ import annotations
 
@@ -39,6 +50,11 @@ import numpy as np
 
 # nibble t of a packed word holds column 8*w + AWQ_ORDER[t]
 AWQ_ORDER = (0, 2, 4, 6, 1, 3, 5, 7)
+
+# four-bit symmetric quantiser: signed levels, exported zero point, scale bounds
+SYM_QMIN, SYM_QMAX = -8, 7
+SYM_ZERO_CODE = 8
+QSCALE_MIN, QSCALE_MAX = 1e-5, 1e5
 
 
 def normalize_group_size(group_size: int, K: int) -> int:
@@ -209,3 +225,47 @@ def w4_linear_columns(x, codes, zero_codes, scales, bias, channel_scales, pairs,
     if bias is not None:
         Y += np.asarray(bias, dtype=np.float64)[cols].reshape(1, -1)
     return Y
+
+
+def transform_weight(W: np.ndarray, channel_scales: Optional[np.ndarray], pairs: Optional[np.ndarray],
+                     theta: Optional[np.ndarray], group_size: int, krot: Optional[int] = None) -> np.ndarray:
+    """W_r = W D R in float64: row n of W [N, K] (out x in) is multiplied by
+    D = 1 / channel_scales per input channel and then takes the same krot
+    stages as an activation row, so that X_r W_r^T = X W^T."""
+    W = np.asarray(W)
+    if W.ndim != 2:
+        raise ValueError("W must be 2-D [N, K]")
+    D = None
+    if channel_scales is not None:
+        D = 1.0 / np.asarray(channel_scales, dtype=np.float64)
+    return rotate(W, D, pairs, theta, group_size, krot=krot)
+
+
+def quantize_sym4(W_r: np.ndarray, scales: np.ndarray, group_size: int):
+    """Four-bit symmetric quantisation of W_r [N, K] with group scales [K//G, N].
+
+    s = scales[k // G, n] bounded to [QSCALE_MIN, QSCALE_MAX];
+    q = clamp(round_half_even(W_r / s), -8, 7); code = q + 8 (uint8 0..15).
+    Returns codes [N, K] and zero codes [N, K//G] (all 8), the ``awq_pack`` inputs.
+    """
+    W_r = np.asarray(W_r, dtype=np.float64)
+    N, K = W_r.shape
+    G = normalize_group_size(group_size, K)
+    s = np.clip(np.asarray(scales, dtype=np.float64), QSCALE_MIN, QSCALE_MAX)
+    if s.shape != (K // G, N):
+        raise ValueError(f"scales must be [{K // G}, {N}]")
+    s_nk = np.repeat(s.T, G, axis=1)                       # [N, K]
+    q = np.clip(np.rint(W_r / s_nk), SYM_QMIN, SYM_QMAX)   # np.rint: ties to even
+    codes = (q + SYM_ZERO_CODE).astype(np.uint8)
+    zeros = np.full((N, K // G), SYM_ZERO_CODE, dtype=np.uint8)
+    return codes, zeros
+
+
+def quantize_weight(W, channel_scales, pairs, theta, scales, group_size, krot=None):
+    """Packed runtime weights from float weights: AWQ-packed Q(W_r).
+    Returns qweight [K, N//8] int32 and qzeros [K//G, N//8] int32."""
+    K = np.asarray(W).shape[1]
+    G = normalize_group_size(group_size, K)
+    W_r = transform_weight(W, channel_scales, pairs, theta, G, krot=krot)
+    codes, zeros = quantize_sym4(W_r, scales, G)
+    return awq_pack(codes, zeros, G)

@@ -30,6 +30,8 @@ Value distributions (the workload recipe):
   * theta: U(-pi, pi) -> fp32 for active pairs, exactly 0 for dummy pairs
     (same page: "unused channels are filled with dummy pairs whose angles stay
     zero").
+  * weight-side quantiser inputs (``make_float_weight``): W N(0, 0.02^2) with
+    two rows x 8 -> fp16; quantiser scales U[0.006, 0.012] -> fp16.
   * codes: U{0..15}; zero codes all 8 (the unsigned export of the symmetric
     4-bit quantiser uses zero point 8, same page, "Straight-through
     estimation"); scales U[0.005, 0.02] -> fp16; bias 0 or N(0, 0.01) -> fp16.
@@ -109,6 +111,27 @@ def make_activations(layer: Layer, M: int, seed: Optional[int] = None) -> np.nda
     if layer.outlier_channels.size:
         x[:, layer.outlier_channels] *= 20.0
     return x.astype(np.float16)
+
+
+def make_float_weight(layer: Layer, seed: Optional[int] = None, std: float = 0.02,
+                      outlier_rows: int = 2):
+    """Float inputs of the weight-side quantiser for ``layer``'s shape:
+
+    * W [N, K] fp16 (out x in): N(0, std^2), with ``outlier_rows`` whole rows
+      x 8 so that some groups clamp at the code range;
+    * quantiser scales [K//G, N] fp16: U[0.3, 0.6] * std, about a third to a
+      sixth of the largest |W_r| of a group of 128, so that a few per cent of
+      the codes sit at -8 or 7.
+
+    The rotation tables and channel scales are the layer's own."""
+    rng = np.random.default_rng((layer.seed if seed is None else seed, 11))
+    W = rng.standard_normal((layer.N, layer.K)) * std
+    if outlier_rows:
+        rows = rng.choice(layer.N, size=min(outlier_rows, layer.N), replace=False)
+        W[rows] *= 8.0
+    G = layer.group_size
+    qscales = rng.uniform(0.3 * std, 0.6 * std, size=(layer.K // G, layer.N))
+    return W.astype(np.float16), qscales.astype(np.float16)
 
 
 def one_percent(K: int) -> int:

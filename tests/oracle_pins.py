@@ -2,8 +2,9 @@
 fix, not against the oracle itself.
 
 Each ``pin_*`` takes an implementation namespace ``impl`` exposing
-``rotate``, ``inverse_rotate``, ``awq_pack``, ``awq_unpack``, ``dequant`` and
-``w4_linear_from_codes`` with the oracle's signatures, and raises
+``rotate``, ``inverse_rotate``, ``awq_pack``, ``awq_unpack``, ``dequant``,
+``w4_linear_from_codes``, ``transform_weight`` and ``quantize_sym4`` with the
+oracle's signatures, and raises
 AssertionError when the implementation disagrees.  ``test_oracle_pins.py``
 runs them on the oracle; ``test_oracle_mutations.py`` runs them on copies of
 the oracle with planted mistakes and checks that each mistake is caught.
@@ -16,6 +17,10 @@ Sources (GPTQModel wiki page "ParoQuant"):
     W_r = W D R, X_r W_r^T = X W^T without quantisation; the equivalent
     original-domain weight is Q(W_r) R^T D^-1.
   * "Stored tensors": identity state = zero angles and unit channel scales.
+  * "Activation and weight transforms" (quantiser paragraph): four-bit
+    symmetric codes -8..7, exported unsigned with zero point 8, quantiser
+    scales bounded to [1e-5, 1e5]; nearest level with ties to even (the
+    rounding named in "STE acceleration kernels").
 """
 from __future__ import annotations
 
@@ -289,10 +294,114 @@ def pin_dequant_formula(impl):
     assert W[130, 6] == -1.5
 
 
+# ------------------------------------------------------- weight-side pins
+
+def pin_weight_transform_identity(impl):
+    """transform_weight gives W_r = W D R: with the activations' X_r = X D^-1 R,
+    X_r W_r^T = X W^T (no quantisation), and zero angles with unit scales
+    leave W unchanged."""
+    rng = np.random.default_rng(21)
+    K, G, N, M = 384, 128, 40, 5
+    pairs, theta = _rand_tables(rng, K, G, 8)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))      # D^-1
+    x = rng.standard_normal((M, K))
+    W = rng.standard_normal((N, K))
+    lhs = impl.rotate(x, cs, pairs, theta, G) @ impl.transform_weight(W, cs, pairs, theta, G).T
+    rhs = x @ W.T
+    assert np.max(np.abs(lhs - rhs)) <= 1e-10 * np.max(np.abs(rhs))
+    same = impl.transform_weight(W, np.ones(K), pairs, np.zeros_like(theta), G)
+    assert np.max(np.abs(same - W)) <= 1e-15 * np.max(np.abs(W))
+    # one channel, one pair at a right angle: (a, b) -> (b, -a) after the 1/cs scaling
+    p1 = np.tile(np.arange(G, dtype=np.int16), (1, K // G))
+    t1 = np.zeros((1, K // 2))
+    t1[0, 0] = np.pi / 2
+    w1 = np.zeros((1, K))
+    w1[0, 0], w1[0, 1] = 3.0, 5.0
+    c1 = np.ones(K)
+    c1[0], c1[1] = 2.0, 0.5
+    got = impl.transform_weight(w1, c1, p1, t1, G)
+    assert abs(got[0, 0] - 10.0) <= 1e-12 and abs(got[0, 1] + 1.5) <= 1e-12
+
+
+def pin_sym4_closed_forms(impl):
+    """Code of chosen quotients (exact in binary): nearest level, ties to even,
+    clamping to -8..7, zero point 8, scale bounds."""
+    K, G = 128, 128
+    t = np.array([0.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.25, 6.5, 7.4, 7.5, 100.0,
+                  -7.5, -8.4, -8.5, -100.0, 1.0, -1.0])
+    want_q = np.array([0, 0, 2, 2, 0, -2, -2, 3, 6, 7, 7, 7, -8, -8, -8, -8, 1, -1])
+    s = 0.25                                                  # power of two: W_r / s is exact
+    W = np.zeros((8, K))
+    W[0, :t.size] = t * s
+    scales = np.full((K // G, 8), s)
+    codes, zeros = impl.quantize_sym4(W, scales, G)
+    assert codes.dtype == np.uint8 and codes.shape == (8, K) and zeros.shape == (8, K // G)
+    assert np.array_equal(codes[0, :t.size].astype(int), want_q + 8), codes[0, :t.size]
+    assert np.all(codes[1:] == 8) and np.all(zeros == 8)
+    # bounds: a zero scale acts as 1e-5, a huge one as 1e5
+    W2 = np.zeros((8, K))
+    W2[0, 0] = 3e-5
+    W2[1, 0] = 2.5e5
+    W2[2, 0] = -7e5
+    sc2 = np.ones((K // G, 8))
+    sc2[0, 0] = 0.0
+    sc2[0, 1] = 1e6
+    sc2[0, 2] = 1e9
+    c2, _ = impl.quantize_sym4(W2, sc2, G)
+    assert int(c2[0, 0]) == 11 and int(c2[1, 0]) == 10 and int(c2[2, 0]) == 1, c2[:3, 0]
+
+
+def pin_sym4_nearest_level_brute_force(impl):
+    """Every code's level (code - 8) * s is a nearest one of the 16 levels
+    -8 s .. 7 s to the value, found by trying them all; groups and columns
+    each use their own scale."""
+    rng = np.random.default_rng(22)
+    N, K, G = 16, 256, 128
+    scales = rng.uniform(0.05, 0.3, (K // G, N))
+    W = rng.standard_normal((N, K)) * 0.8
+    codes, zeros = impl.quantize_sym4(W, scales, G)
+    levels = np.arange(-8, 8)
+    for n in range(N):
+        for k in range(K):
+            sc = scales[k // G, n]
+            d = np.abs(levels * sc - W[n, k])
+            got = (int(codes[n, k]) - int(zeros[n, k // G])) * sc
+            assert abs(got - W[n, k]) <= d.min() + 1e-12, (n, k)
+
+
+def pin_quantized_replay(impl):
+    """The packed layer replays Y = X_r Q(W_r)^T + b: the codes from
+    quantize_sym4(transform_weight(W)) through w4_linear_from_codes equal a
+    one-output-at-a-time sum over the nearest levels of W_r."""
+    rng = np.random.default_rng(23)
+    M, K, N, G = 2, 256, 16, 128
+    pairs, theta = _rand_tables(rng, K, G, 8)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))
+    W = rng.standard_normal((N, K))
+    x = rng.standard_normal((M, K))
+    bias = rng.standard_normal(N)
+    W_r = impl.transform_weight(W, cs, pairs, theta, G)
+    scales = np.max(np.abs(W_r).reshape(N, K // G, G), axis=2).T / 6.0
+    codes, zeros = impl.quantize_sym4(W_r, scales, G)
+    got = impl.w4_linear_from_codes(x, codes, zeros, scales, bias, cs, pairs, theta, G, 8)
+    xr = impl.rotate(x, cs, pairs, theta, G)
+    levels = np.arange(-8, 8)
+    ref = np.zeros((M, N))
+    for n in range(N):
+        for k in range(K):
+            sc = scales[k // G, n]
+            lv = levels[np.argmin(np.abs(levels * sc - W_r[n, k]))] * sc
+            ref[:, n] += xr[:, k] * lv
+    ref += bias
+    assert np.max(np.abs(got - ref)) <= 1e-10 * np.max(np.abs(ref))
+
+
 ALL_PINS = [
     pin_single_pair_closed_forms, pin_stage_composition, pin_inverse_restores,
     pin_group_norms_preserved, pin_dense_R_brute_force, pin_golden_g4,
     pin_group_size_minus_one, pin_unquantized_identity, pin_awq_golden_word,
     pin_awq_one_hot, pin_awq_round_trip, pin_identity_state_is_plain_w4,
     pin_equivalent_weight_route, pin_dequant_formula,
+    pin_weight_transform_identity, pin_sym4_closed_forms, pin_sym4_nearest_level_brute_force,
+    pin_quantized_replay,
 ]

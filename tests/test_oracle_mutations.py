@@ -14,7 +14,9 @@ ORDER_OK = (0, 2, 4, 6, 1, 3, 5, 7)
 
 def make_impl(sign_flip=False, reverse_stages=False, swap_roles=False, no_scale=False,
               theta_global=False, order=ORDER_OK, no_zero=False, group0_scale=False,
-              inverse_forward_order=False, shared_group_base=False):
+              inverse_forward_order=False, shared_group_base=False, q_half_away=False,
+              q_clamp7=False, q_no_offset=False, w_scale_multiplied=False, q_group0_scale=False,
+              q_no_bound=False, w_no_stages=False):
     def stage_idx(pairs_s, G):
         K = pairs_s.shape[0]
         local = pairs_s.astype(np.int64)
@@ -87,9 +89,33 @@ def make_impl(sign_flip=False, reverse_stages=False, swap_roles=False, no_scale=
             Y += np.asarray(bias, np.float64)
         return Y
 
+    def transform_weight(W, cs, pairs, theta, group_size, krot=None):
+        D = None if cs is None else (np.asarray(cs, np.float64) if w_scale_multiplied
+                                     else 1.0 / np.asarray(cs, np.float64))
+        if w_no_stages:
+            krot = 0
+        return rotate(W, D, pairs, theta, group_size, krot=krot)
+
+    def quantize_sym4(W_r, scales, G):
+        W_r = np.asarray(W_r, np.float64)
+        N, K = W_r.shape
+        sc = np.asarray(scales, np.float64)
+        if not q_no_bound:
+            sc = np.clip(sc, 1e-5, 1e5)
+        if q_group0_scale:
+            sc = np.repeat(sc[:1], sc.shape[0], axis=0)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            t = W_r / np.repeat(sc.T, G, axis=1)
+        q = np.sign(t) * np.floor(np.abs(t) + 0.5) if q_half_away else np.rint(t)
+        q = np.nan_to_num(q, nan=0.0, posinf=99.0, neginf=-99.0)
+        q = np.clip(q, -7 if q_clamp7 else -8, 7)
+        codes = (q.astype(np.int64) & 15).astype(np.uint8) if q_no_offset else (q + 8).astype(np.uint8)
+        return codes, np.full((N, K // G), 0 if q_no_offset else 8, np.uint8)
+
     return types.SimpleNamespace(rotate=rotate, inverse_rotate=inverse_rotate, awq_pack=awq_pack,
                                  awq_unpack=awq_unpack, dequant=dequant,
-                                 w4_linear_from_codes=w4_linear_from_codes)
+                                 w4_linear_from_codes=w4_linear_from_codes,
+                                 transform_weight=transform_weight, quantize_sym4=quantize_sym4)
 
 
 def failing_pins(impl):
@@ -117,6 +143,13 @@ MUTATIONS = {
     "scale_group_misindexed": dict(group0_scale=True),
     "inverse_not_reversed": dict(inverse_forward_order=True),
     "pairs_not_group_local": dict(shared_group_base=True),
+    "quant_ties_away_from_zero": dict(q_half_away=True),
+    "quant_clamped_to_plus_minus_7": dict(q_clamp7=True),
+    "quant_twos_complement_codes": dict(q_no_offset=True),
+    "weight_scaled_by_cs_not_its_inverse": dict(w_scale_multiplied=True),
+    "quant_scale_group_misindexed": dict(q_group0_scale=True),
+    "quant_scale_unbounded": dict(q_no_bound=True),
+    "weight_stages_skipped": dict(w_no_stages=True),
 }
 
 

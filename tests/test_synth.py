@@ -59,3 +59,13 @@ def test_config_shapes_listing():
         (4096, 4096), (4096, 1024), (4096, 1024), (4096, 4096),
         (4096, 14336), (4096, 14336), (14336, 4096)]
     assert synth.CONFIG_M[1] == [1, 4, 16]
+
+
+def test_float_weight_inputs_are_seeded_and_typed():
+    lay = synth.make_layer("w", 256, 64, 5)
+    W1, s1 = synth.make_float_weight(lay)
+    W2, s2 = synth.make_float_weight(lay)
+    assert W1.dtype == np.float16 and W1.shape == (64, 256)
+    assert s1.dtype == np.float16 and s1.shape == (2, 64)
+    assert np.array_equal(W1, W2) and np.array_equal(s1, s2)
+    assert np.all(s1 > 0)
