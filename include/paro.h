@@ -53,7 +53,8 @@
  *     kernel immediately ahead of the call if that kernel releases its dependents
  *     early (griddepcontrol.launch_dependents).  No kernel of this library that
  *     releases early writes layer constants (paro_pack_awq does not release
- *     early), and kernels that never release early are always safe.
+ *     early; paro_quantize_w4 does not release early), and kernels that never
+ *     release early are always safe.
  *   - Supported now: G == 128 (group_size == -1 is accepted when K == 128),
  *     0 <= krot <= 64, K a multiple of 128, N a multiple of 32 (the packer alone
  *     needs only N % 8 == 0), fp16 activations/scales/bias.
@@ -119,6 +120,32 @@ int paro_rotate(const void* x, void* x_r, int64_t M, int64_t K, const float* cha
  */
 int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qweight,
                   int32_t* qzeros, int64_t N, int64_t K, int group_size, paro_stream_t stream);
+
+/*
+ * paro_quantize_w4 — packed runtime weights from float weights: the weight-side
+ * transform W_r = W D R (page "ParoQuant", "Activation and weight transforms":
+ * D = 1 / channel_scales, the rows of W taking the activations' stages) followed
+ * by the four-bit symmetric quantiser of the same section (signed codes -8..7,
+ * exported unsigned with zero point 8, quantiser scales bounded to [1e-5, 1e5])
+ * and AWQ packing, in one pass.
+ *   w               device fp16 [N, K] (out x in), 16-byte aligned
+ *   channel_scales  device fp32 [K] (the runtime D^-1) or NULL (D = 1)
+ *   pairs, theta    the layer's rotation tables (as for paro_rotate); NULL only when krot == 0
+ *   scales          device fp16 [K/G, N] quantiser (= dequantisation) scales
+ *   qweight         device int32 [K, N/8]; qzeros device int32 [K/G, N/8] (all 0x88888888)
+ *   N >= 0, N % 8 == 0 (N == 0 is a no-op); K % 128 == 0; group_size 128 (or -1 with K == 128);
+ *   krot 0..64; N * K < 2^31
+ * Arithmetic: W * D with D = 1/channel_scales in fp32, the stages as in
+ * paro_rotate (fp32, no fp16 rounding of W_r), q = rint(W_r * (1/s)) with ties
+ * to even, s bounded first, then clamped to -8..7 and offset by 8.  A code can
+ * differ from the exactly computed one only where W_r / s lies within the fp32
+ * rounding of the transform of a half-integer.  Pair indices outside the group
+ * are masked and flagged as in paro_rotate.  The kernel does not release its
+ * dependents early, so a paro_w4_linear right after it may use its outputs.
+ */
+int paro_quantize_w4(const void* w, const float* channel_scales, const int16_t* pairs,
+                     const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
+                     int64_t N, int64_t K, int group_size, int krot, paro_stream_t stream);
 
 /* paro_unpack_awq — exact inverse of paro_pack_awq (same shapes, same rules). */
 int paro_unpack_awq(const int32_t* qweight, const int32_t* qzeros, uint8_t* codes,

@@ -8,6 +8,7 @@ streams) into that ABI.  Functions mirror the C entry points:
     pack_awq          -> paro_pack_awq
     unpack_awq        -> paro_unpack_awq
     w4_linear         -> paro_w4_linear (+ paro_w4_linear_workspace_size)
+    quantize_w4       -> paro_quantize_w4
     validate_pairs    -> paro_validate_pairs (host helper)
     device_status     -> paro_device_status
 """
@@ -22,11 +23,11 @@ import torch
 from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # noqa: F401
                    PARO_ERR_TIMEOUT, PARO_ERR_UNSUPPORTED, PARO_ERR_WORKSPACE, PARO_OK,
                    LIB_PATH, ParoError, check, lib, paro_device_status, paro_pack_awq,
-                   paro_rotate, paro_status_string, paro_unpack_awq, paro_validate_pairs,
-                   paro_version, paro_w4_linear, paro_w4_linear_workspace_size)
+                   paro_quantize_w4, paro_rotate, paro_status_string, paro_unpack_awq,
+                   paro_validate_pairs, paro_version, paro_w4_linear, paro_w4_linear_workspace_size)
 
 __all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
-           "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
+           "quantize_w4", "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -83,6 +84,30 @@ def pack_awq(codes: torch.Tensor, zero_codes: Optional[torch.Tensor], group_size
         qzeros = torch.empty((K // G, N // 8), dtype=torch.int32, device=codes.device)
     check(paro_pack_awq(_ptr(codes), _ptr(zero_codes), _ptr(qweight), _ptr(qzeros), N, K,
                         group_size, _stream(stream)), "paro_pack_awq")
+    return qweight, qzeros
+
+
+def quantize_w4(w: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: Optional[torch.Tensor],
+                theta: Optional[torch.Tensor], scales: torch.Tensor, group_size: int = 128,
+                krot: Optional[int] = None, out=None, stream=None):
+    """Float weights w fp16 [N, K] (out x in) -> (qweight int32 [K, N/8], qzeros int32 [K/G, N/8]):
+    W_r = W D R, four-bit symmetric codes with the fp16 quantiser scales [K/G, N], AWQ-packed."""
+    _need(w, torch.float16, "w")
+    _need(channel_scales, torch.float32, "channel_scales", True)
+    _need(pairs, torch.int16, "pairs", True)
+    _need(theta, torch.float32, "theta", True)
+    _need(scales, torch.float16, "scales")
+    if krot is None:
+        krot = 0 if pairs is None else pairs.shape[0]
+    N, K = w.shape
+    G = K if group_size == -1 else group_size
+    if out is None:
+        out = (torch.empty((K, N // 8), dtype=torch.int32, device=w.device),
+               torch.empty((K // G, N // 8), dtype=torch.int32, device=w.device))
+    qweight, qzeros = out
+    check(paro_quantize_w4(_ptr(w), _ptr(channel_scales), _ptr(pairs), _ptr(theta), _ptr(scales),
+                           _ptr(qweight), _ptr(qzeros), N, K, group_size, krot, _stream(stream)),
+          "paro_quantize_w4")
     return qweight, qzeros
 
 

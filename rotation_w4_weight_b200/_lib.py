@@ -23,7 +23,7 @@ PARO_ERR_TIMEOUT = 6
 EXPORTED = (
     "paro_status_string", "paro_version", "paro_rotate", "paro_pack_awq", "paro_unpack_awq",
     "paro_w4_linear_workspace_size", "paro_w4_linear", "paro_w4_linear_noalloc",
-    "paro_validate_pairs", "paro_device_status",
+    "paro_validate_pairs", "paro_device_status", "paro_quantize_w4",
 )
 
 _vp = ctypes.c_void_p
@@ -43,6 +43,7 @@ _SIGNATURES = {
                                       _vp, _int, _int, _vp]),
     "paro_validate_pairs": (_int, [_vp, _i64, _int, _int]),
     "paro_device_status": (_int, [_int]),
+    "paro_quantize_w4": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp]),
 }
 
 
@@ -72,6 +73,7 @@ paro_w4_linear_noalloc = lib.paro_w4_linear_noalloc
 PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES = 8 << 20
 paro_validate_pairs = lib.paro_validate_pairs
 paro_device_status = lib.paro_device_status
+paro_quantize_w4 = lib.paro_quantize_w4
 
 
 class ParoError(RuntimeError):

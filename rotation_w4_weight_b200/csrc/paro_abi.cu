@@ -201,42 +201,48 @@ int check_rotation_args(const void* x, const void* xr, int64_t M, int64_t K, con
   return PARO_OK;
 }
 
+// Tensor-memory rotation kernel (and, with QUANT, the weight quantiser): CTAs
+// stay resident over several 128-row tiles of one group (one wave of at most
+// 2 CTAs per SM: the shared-memory floor of the kernel guarantees no more fit).
+template <bool QUANT>
+int launch_rotate_tmem(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
+                       const int16_t* pairs, const float* theta, int krot, const RtQuant& qo,
+                       cudaStream_t stream) {
+  const size_t smem = RtLayout::bytes(krot, QUANT);
+  const DeviceInfo& di = device_info();
+  if (di.sms == 0) return PARO_ERR_CUDA;
+  const bool abs_tables = krot <= kRtAbsMaxKrot;
+  if (abs_tables ? !allow_smem(rotate_tmem_kernel<true, QUANT>, RtLayout::bytes(kRtAbsMaxKrot, QUANT))
+                 : !allow_smem(rotate_tmem_kernel<false, QUANT>, RtLayout::bytes(kMaxKrot, QUANT)))
+    return PARO_ERR_CUDA;
+  const size_t per_block = smem + di.smem_reserved_per_block;
+  int per_sm = (int)(di.smem_per_sm / per_block);
+  per_sm = per_sm < 1 ? 1 : (per_sm > kRtMaxCtasPerSm ? kRtMaxCtasPerSm : per_sm);
+  // one wave: gridDim.y row-tile slots per group, then as few tiles per CTA
+  // as that allows, spread evenly
+  const int64_t groups = K / kGroup, ntiles = (M + kRtRows - 1) / kRtRows;
+  const int64_t slots = (int64_t)di.sms * per_sm;
+  int64_t gy = slots / groups;
+  gy = gy < 1 ? 1 : (gy > ntiles ? ntiles : gy);
+  const int64_t per_cta = (ntiles + gy - 1) / gy;
+  gy = (ntiles + per_cta - 1) / per_cta;
+  if (gy > 65535) gy = 65535;
+  CUtensorMap tmX;
+  if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, kRtRows, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return PARO_ERR_CUDA;
+  const dim3 grid((unsigned)groups, (unsigned)gy);
+  if (abs_tables)
+    return launch(rotate_tmem_kernel<true, QUANT>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
+                  pairs, theta, (int)M, (int)K, krot, qo);
+  return launch(rotate_tmem_kernel<false, QUANT>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
+                pairs, theta, (int)M, (int)K, krot, qo);
+}
+
 int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
                   const int16_t* pairs, const float* theta, int krot, cudaStream_t stream) {
-  // Large batches: tensor memory as the permutation network; CTAs stay resident
-  // over several 128-row tiles of one group (one wave of at most 2 CTAs per SM:
-  // the shared-memory floor of the kernel guarantees no more fit).
-  if (M > 64) {
-    const size_t smem = RtLayout::bytes(krot);
-    const DeviceInfo& di = device_info();
-    if (di.sms == 0) return PARO_ERR_CUDA;
-    const bool abs_tables = krot <= kRtAbsMaxKrot;
-    if (abs_tables ? !allow_smem(rotate_tmem_kernel<true>, RtLayout::bytes(kRtAbsMaxKrot))
-                   : !allow_smem(rotate_tmem_kernel<false>, RtLayout::bytes(kMaxKrot)))
-      return PARO_ERR_CUDA;
-    const size_t per_block = smem + di.smem_reserved_per_block;
-    int per_sm = (int)(di.smem_per_sm / per_block);
-    per_sm = per_sm < 1 ? 1 : (per_sm > kRtMaxCtasPerSm ? kRtMaxCtasPerSm : per_sm);
-    // one wave: gridDim.y row-tile slots per group, then as few tiles per CTA
-    // as that allows, spread evenly
-    const int64_t groups = K / kGroup, ntiles = (M + kRtRows - 1) / kRtRows;
-    const int64_t slots = (int64_t)di.sms * per_sm;
-    int64_t gy = slots / groups;
-    gy = gy < 1 ? 1 : (gy > ntiles ? ntiles : gy);
-    const int64_t per_cta = (ntiles + gy - 1) / gy;
-    gy = (ntiles + per_cta - 1) / per_cta;
-    if (gy > 65535) gy = 65535;
-    CUtensorMap tmX;
-    if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, kRtRows, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
-      return PARO_ERR_CUDA;
-    const dim3 grid((unsigned)groups, (unsigned)gy);
-    if (abs_tables)
-      return launch(rotate_tmem_kernel<true>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
-                    pairs, theta, (int)M, (int)K, krot);
-    return launch(rotate_tmem_kernel<false>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
-                  pairs, theta, (int)M, (int)K, krot);
-  }
+  // Large batches: tensor memory as the permutation network.
+  if (M > 64) return launch_rotate_tmem<false>(x, xr, M, K, cs, pairs, theta, krot, RtQuant{}, stream);
   // Decode batches with few stages: one warp per row, no block barrier per stage.
   if (M <= 16 && krot <= kRrMaxKrot) {
     // always 8 warps: all of them build the tables, warps past the batch then leave
@@ -443,6 +449,26 @@ int paro_rotate(const void* x, void* x_r, int64_t M, int64_t K, const float* cha
   if (M == 0) return PARO_OK;
   return launch_rotate(static_cast<const __half*>(x), static_cast<__half*>(x_r), M, K,
                        channel_scales, pairs, theta, krot, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int paro_quantize_w4(const void* w, const float* channel_scales, const int16_t* pairs,
+                     const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
+                     int64_t N, int64_t K, int group_size, int krot, paro_stream_t stream) {
+  if (N < 0 || K <= 0 || krot < 0 || N % 8 != 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  if (G != kGroup || krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
+  if (N == 0) return PARO_OK;   // nothing to touch: NULL data pointers are fine
+  if (w == nullptr || scales == nullptr || qweight == nullptr || qzeros == nullptr) return PARO_ERR_INVALID_ARG;
+  if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
+  if (N * K >= (int64_t(1) << 31)) return PARO_ERR_UNSUPPORTED;
+  if (!aligned(w, 16) || !aligned(scales, 2) || !aligned(qweight, 4) || !aligned(qzeros, 4))
+    return PARO_ERR_ALIGNMENT;
+  if (channel_scales != nullptr && !aligned(channel_scales, 4)) return PARO_ERR_ALIGNMENT;
+  if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
+  const RtQuant qo{static_cast<const __half*>(scales), qweight, qzeros};
+  return launch_rotate_tmem<true>(static_cast<const __half*>(w), nullptr, N, K, channel_scales, pairs, theta,
+                                  krot, qo, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qweight,

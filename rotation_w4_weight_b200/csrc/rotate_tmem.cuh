@@ -34,6 +34,17 @@
 // Input tiles arrive by TMA (two 64-channel boxes, 128-byte swizzle, so the
 // row-per-thread reads are conflict-free) into two buffers, two tiles ahead of
 // use.
+//
+// With QUANT the rows are weight rows (out x in) and the kernel is the
+// weight-side quantiser of the same page, section "Activation and weight
+// transforms": W_r = W D R with D = 1 / channel_scales (the scaling step
+// multiplies by D evaluated once per channel in fp32), then four-bit symmetric
+// codes q = clamp(rint(W_r / s), -8, 7) + 8 with s the group scale bounded to
+// [1e-5, 1e5] (the quotient as W_r times the fp32 reciprocal of s, rounded to
+// nearest even), written straight into the AWQ layout: the codes of a tile go
+// to shared memory transposed (channel-major bytes), and each packed word
+// collects eight output rows' codes of one channel in the nibble order
+// (0, 2, 4, 6, 1, 3, 5, 7).  qzeros gets the constant zero code 8.
 #pragma once
 
 #include "rotate.cuh"
@@ -47,6 +58,13 @@ constexpr int kRtCols = 256;             // two 128-column buffers
 constexpr int kRtMaxCtasPerSm = 2;       // 2 x 256 TMEM columns
 constexpr int kRtAbsMaxKrot = 16;        // per-quadrant address tables up to this many stages
 constexpr size_t kRtMinSmem = 80 * 1024; // above a third of an SM's shared memory: <= 2 CTAs/SM
+
+// Output of the quantising instantiation (rows = N output channels).
+struct RtQuant {
+  const __half* scales;   // [K/128, N] quantiser scales
+  int32_t* qweight;       // [K, N/8] AWQ words
+  int32_t* qzeros;        // [K/128, N/8] AWQ words (all 8)
+};
 
 struct RtLayout {
   // IN tiles[2] | scale[128] | per stage (c0,c1,s0,s1)[32 units] |
@@ -67,9 +85,14 @@ struct RtLayout {
   __host__ __device__ static constexpr size_t pos_off(int krot) { return praw_off(krot) + (size_t)krot * 64 * 4; }
   __host__ __device__ static constexpr size_t bar_off(int krot) { return pos_off(krot) + 128 * 4; }
   __host__ __device__ static constexpr size_t slot_off(int krot) { return bar_off(krot) + 16; }
+  // quantiser only: the tile's codes, channel-major bytes [128 channels][128 rows]
+  __host__ __device__ static constexpr size_t codes_off(int krot) { return slot_off(krot) + 16; }
+  static constexpr size_t CODES = 128 * 128;
   // + 1 KB so the tiles can be aligned to the 1024 bytes the swizzle pattern needs
-  __host__ __device__ static constexpr size_t bytes(int krot) {
-    return slot_off(krot) + 16 + 1024 < kRtMinSmem ? kRtMinSmem : slot_off(krot) + 16 + 1024;
+  __host__ __device__ static constexpr size_t bytes(int krot, bool quant = false) {
+    return codes_off(krot) + (quant ? CODES : 0) + 1024 < kRtMinSmem
+               ? kRtMinSmem
+               : codes_off(krot) + (quant ? CODES : 0) + 1024;
   }
 };
 
@@ -87,12 +110,24 @@ __device__ __forceinline__ void rt_quadrant_sync(int qd) {
   tc_fence_after();
 }
 
+// Four-bit AWQ word of eight codes (bytes c0..c7 of output rows 8w .. 8w+7):
+// nibble t holds the code of row 8w + (0, 2, 4, 6, 1, 3, 5, 7)[t].
+__device__ __forceinline__ uint32_t rt_awq_word(uint32_t lo, uint32_t hi) {
+  const uint32_t e = __byte_perm(lo, hi, 0x6420);   // c0 c2 c4 c6
+  const uint32_t o = __byte_perm(lo, hi, 0x7531);   // c1 c3 c5 c7
+  const uint32_t e4 = (e & 0xFu) | ((e >> 4) & 0xF0u) | ((e >> 8) & 0xF00u) | ((e >> 12) & 0xF000u);
+  const uint32_t o4 = (o & 0xFu) | ((o >> 4) & 0xF0u) | ((o >> 8) & 0xF00u) | ((o >> 12) & 0xF000u);
+  return e4 | (o4 << 16);
+}
+
 // grid: (K/128, row-tile slots), block 256.  tmX is x as [M, K] fp16 with box
 // {64 channels, 128 rows}, 128-byte swizzle (rows past M read as zeros).
-template <bool ABS>
+// QUANT: x is W [N = M, K], xr is unused and qo receives the packed codes.
+template <bool ABS, bool QUANT>
 __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kernel(
     const __grid_constant__ CUtensorMap tmX, __half* xr, const float* __restrict__ cs,
-    const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot) {
+    const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot,
+    const RtQuant qo) {
   using L = RtLayout;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   unsigned char* const sb = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -143,7 +178,10 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
   // ---- tables, 1: every stage's pairs and angles, loads issued together.
   // Indices outside the group are masked to 7 bits (every address stays inside
   // this CTA's allocation) and flagged.
-  if (tid < 128) scale[tid] = cs != nullptr ? cs[grp * kGroup + tid] : 1.0f;
+  if (tid < 128) {
+    const float c = cs != nullptr ? cs[grp * kGroup + tid] : 1.0f;
+    scale[tid] = QUANT ? 1.0f / c : c;               // weights take D = 1 / channel_scales
+  }
   for (int idx = tid; idx < krot * 64; idx += kRtThreads) {
     const int s = idx >> 6, p = idx & 63, u = p >> 1, w = p & 1;
     const uint32_t pr =
@@ -164,7 +202,9 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_launch_dependents();
+  // the quantiser writes layer constants (qweight, qzeros): it never releases
+  // its dependents early, so a following call may read them before its wait
+  if constexpr (!QUANT) pdl_launch_dependents();
   const uint32_t tmem0 = *slot;
 
   // ---- tables, 2 (warp 0): stage s reads buffer (s & 1) and writes buffer
@@ -319,9 +359,35 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
       for (int b = 1; b < SW / 32; ++b) tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
     }
 
-    // ---- fp16 (round to nearest), row r, channels SW*h .. SW*h+SW-1
     const int row = tile * kRtRows + r;
-    if (row < M) {
+    if constexpr (QUANT) {
+      // ---- codes of row r (an output channel), channels SW*h .. SW*h+SW-1,
+      // transposed into shared memory; then 8 AWQ words per thread
+      float sc = row < M ? __half2float(qo.scales[(size_t)grp * M + row]) : 1.0f;
+      sc = fminf(fmaxf(sc, 1e-5f), 1e5f);
+      const float inv = 1.0f / sc;
+      const uint32_t cb = smem_u32(sb + L::codes_off(krot)) + (uint32_t)(SW * h) * 128u + (uint32_t)r;
+#pragma unroll
+      for (int i = 0; i < SW; ++i) {
+        int q = __float2int_rn(__uint_as_float(v[i]) * inv);
+        q = min(max(q, -8), 7) + 8;
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(cb + (uint32_t)i * 128u), "r"(q) : "memory");
+      }
+      __syncthreads();
+      const uint32_t c0 = smem_u32(sb + L::codes_off(krot));
+      const int nw = M / 8;                           // words per channel row of qweight
+#pragma unroll
+      for (int j = 0; j < (128 * 16) / kRtThreads; ++j) {
+        const int idx = tid + kRtThreads * j, k = idx >> 4, w = idx & 15;
+        const int wcol = tile * 16 + w;               // word column: rows 8 wcol .. 8 wcol + 7
+        uint32_t lo, hi;
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi) : "r"(c0 + (uint32_t)k * 128u + 8u * w)
+                     : "memory");
+        if (wcol < nw) qo.qweight[(size_t)(grp * kGroup + k) * nw + wcol] = (int32_t)rt_awq_word(lo, hi);
+      }
+      if (tid < 16 && tile * 16 + tid < nw) qo.qzeros[(size_t)grp * nw + tile * 16 + tid] = (int32_t)0x88888888u;
+    } else if (row < M) {
+      // ---- fp16 (round to nearest), row r, channels SW*h .. SW*h+SW-1
       __half* dstp = xr + (size_t)row * K + (size_t)grp * kGroup + SW * h;
 #pragma unroll
       for (int q = 0; q < SW / 8; ++q) {

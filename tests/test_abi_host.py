@@ -122,3 +122,20 @@ def test_validate_pairs_host_helper(L):
     bad[0, 0] = 128                            # outside the group
     assert not pb.validate_pairs(bad, 256, 128)
     assert pb.validate_pairs(np.zeros((0, 256), np.int16), 256, 128, 0)
+
+
+def test_quantize_argument_validation(L):
+    q = L.paro_quantize_w4
+    # (w, cs, pairs, theta, scales, qweight, qzeros, N, K, G, krot, stream)
+    assert q(A16, None, A16, A16, A16, A16, A16, 12, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG   # N % 8
+    assert q(A16, None, A16, A16, A16, A16, A16, -8, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG
+    assert q(A16, None, None, None, A16, A16, A16, 16, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG
+    assert q(None, None, A16, A16, A16, A16, A16, 16, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG
+    assert q(A16, None, A16, A16, None, A16, A16, 16, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG
+    assert q(A16, None, A16, A16, A16, A16, None, 16, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG
+    assert q(A16, None, A16, A16, A16, A16, A16, 16, 256, 64, 8, None) == L.PARO_ERR_UNSUPPORTED
+    assert q(A16, None, A16, A16, A16, A16, A16, 16, 250, 128, 8, None) == L.PARO_ERR_INVALID_ARG
+    assert q(A16, None, A16, A16, A16, A16, A16, 16, 256, 128, 65, None) == L.PARO_ERR_UNSUPPORTED
+    assert q(MIS, None, A16, A16, A16, A16, A16, 16, 256, 128, 8, None) == L.PARO_ERR_ALIGNMENT
+    assert q(A16, None, A16, A16, A16, P(0x10002), A16, 16, 256, 128, 8, None) == L.PARO_ERR_ALIGNMENT
+    assert q(A16, None, A16, A16, A16, A16, A16, 0, 256, 128, 8, None) == L.PARO_OK   # empty: no-op
