@@ -2,7 +2,7 @@
 """Benchmark of the rotated W4 linear (decode HBM GB/s / prefill TFLOP/s).
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload q_proj_decode|mlp_decode|
-                 prefill|layer_decode|layer_prefill] [--impl ours|reference]
+                 prefill|layer_decode|layer_prefill|quantize_gate_proj] [--impl ours|reference]
 
 One "step" is one pass of the whole hot path (scale + Givens stages + W4
 dequant-GEMM) over every call of the workload:
@@ -10,6 +10,9 @@ dequant-GEMM) over every call of the workload:
   mlp_decode:    gate/up 4096->14336 and down 14336->4096, M = 1 and 8 (six calls)
   prefill:       gate_proj-shaped 4096->14336, M = 2048 and 8192, bias (two calls)
   layer_decode / layer_prefill: the seven linears of a decoder layer at M = 1 / 4096
+  quantize_gate_proj: the weight-side step before packing (W_r = W D R,
+                 four-bit symmetric codes, AWQ words) on a float gate_proj
+                 14336 x 4096, in HBM GB/s (one call per step)
 Inputs are seeded synthetic layers (the workload recipe), resident in HBM; the
 weights are cycled over enough replicas that every timed call reads its weights
 from HBM, not L2.  Prints ONE JSON line on rank 0.
@@ -46,6 +49,7 @@ WORKLOADS = {
     "prefill": dict(cfg=3, layers=[0], Ms=[2048, 8192], kind="prefill"),
     "layer_decode": dict(cfg=4, layers=list(range(7)), Ms=[1], kind="decode"),
     "layer_prefill": dict(cfg=4, layers=list(range(7)), Ms=[4096], kind="prefill"),
+    "quantize_gate_proj": dict(cfg=2, layers=[0], Ms=[], kind="quantize"),
 }
 
 
@@ -59,6 +63,13 @@ def call_bytes(K, N, M, bias, krot=KROT, rotated=True):
     if rotated:
         b += krot * K * 2 + krot * (K // 2) * 4 + K * 4
     return b
+
+
+def quantize_bytes(K, N, krot=KROT):
+    """Bytes of one weight-quantiser call: float W in, quantiser scales in,
+    packed weights and zeros out, rotation tables."""
+    return (N * K * 2 + (K // GROUP) * N * 2 + K * N // 2 + (K // GROUP) * N // 2
+            + krot * K * 2 + krot * (K // 2) * 4 + K * 4)
 
 
 def gemv_bytes(K, N, M, bias):
@@ -182,6 +193,10 @@ def workload_config(workload, world):
     """The workload description shared by both arms' JSON lines."""
     wl = WORKLOADS[workload]
     layers = [synth.config_layers(wl["cfg"])[i] for i in wl["layers"]]
+    if wl["kind"] == "quantize":
+        return {"workload": workload, "weights": [(l.name, l.N, l.K) for l in layers],
+                "input": "float W fp16 [N, K] and quantiser scales fp16 [K/128, N]",
+                "group_size": GROUP, "krot": KROT, "parallelism": f"replicas x{world}"}
     return {"workload": workload, "layers": [(l.name, l.K, l.N) for l in layers], "M": wl["Ms"],
             "group_size": GROUP, "krot": KROT, "accumulate": "f32", "parallelism": f"replicas x{world}"}
 
@@ -386,6 +401,156 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+# ----------------------------------------------------------------- weight quantiser
+def run_quantize(args, rank, world, local_rank):
+    """paro_quantize_w4 on a float gate_proj: one call per step, inputs resident
+    in HBM and cycled over replicas larger than L2 together."""
+    import torch
+    import rotation_w4_weight_b200 as pb
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    lay = synth.config_layers(wl["cfg"])[wl["layers"][0]]
+    W, qs = synth.make_float_weight(lay)
+
+    def T(a):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    Wd, qsd = T(W), T(qs)
+    cs, pairs, theta = T(lay.channel_scales), T(lay.pairs), T(lay.theta)
+    reps = max(2, -(-3 * L2_BYTES // (W.nbytes + qs.nbytes)))
+    Ws = [Wd] + [Wd.clone() for _ in range(reps - 1)]
+    outs = [(torch.empty((lay.K, lay.N // 8), dtype=torch.int32, device=dev),
+             torch.empty((lay.K // GROUP, lay.N // 8), dtype=torch.int32, device=dev)) for _ in range(2)]
+    per_call = quantize_bytes(lay.K, lay.N)
+    stream = torch.cuda.Stream(device=dev)
+
+    def one_step(i):
+        pb.quantize_w4(Ws[i % reps], cs, pairs, theta, qsd, GROUP, KROT, out=outs[i % 2], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            one_step(i)
+    torch.cuda.synchronize(dev)
+    assert pb.device_status() == pb.PARO_OK
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(args.steps):
+            one_step(args.warmup + i)
+
+    def replay():
+        with torch.cuda.stream(stream):
+            g.replay()
+
+    replay()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    t_end = time.time() + 0.6
+    while time.time() < t_end:
+        replay()
+        torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1)
+    t_end = time.time() + 0.4
+    while time.time() < t_end:
+        replay()
+        torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = max_over_ranks(ms, world, dev)
+    assert pb.device_status() == pb.PARO_OK
+    del g
+
+    # one kernel per call: the step time is the kernel's launch time
+    peaks = load_peaks()
+    achieved = per_call * args.steps / (ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm"], 4), "traffic": traffic_for("quantize_gate_proj"),
+            "kernel": "rotate_tmem_kernel<true, true> (weight quantiser)",
+            "avg_launch_us": round(ms * 1e3 / args.steps, 3), "bytes_per_launch": per_call,
+            "peak_source": peaks["src"]}
+
+    # end to end through the public call with host buffers: pinned W in, packed words out
+    hW = Ws[0].cpu().pin_memory()
+    hq = (torch.empty(outs[0][0].shape, dtype=torch.int32).pin_memory(),
+          torch.empty(outs[0][1].shape, dtype=torch.int32).pin_memory())
+    e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        Ws[0].copy_(hW, non_blocking=True)
+        pb.quantize_w4(Ws[0], cs, pairs, theta, qsd, GROUP, KROT, out=outs[0], stream=stream)
+        hq[0].copy_(outs[0][0], non_blocking=True)
+        hq[1].copy_(outs[0][1], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
+
+    return {
+        "metric": metric_name(args.workload),
+        "value": round(job_throughput(world, args.steps, per_call, ms) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(args.workload, world),
+                       l2=f"float weights cycled over {reps} device replicas "
+                          f"({reps * (W.nbytes + qs.nbytes) / 2**20:.0f} MiB > 3x L2)",
+                       timing="CUDA graph of the K steps, CUDA events, max over ranks"),
+        "roofline": roof,
+        "e2e": {"value": round(job_throughput(world, 1, per_call, e2e_ms) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": int(hW.numel() * 2),
+                "d2h_bytes_per_step": int((hq[0].numel() + hq[1].numel()) * 4),
+                "ms_per_step": round(e2e_ms, 4),
+                "how": "pinned host W -> device, paro_quantize_w4, packed words -> pinned host; no graph"},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "bytes_per_step": per_call,
+    }
+
+
+def quantize_oracle_sample(workload, budget_s, max_steps=None):
+    """The float64 oracle's weight quantiser on row samples of the workload's
+    weight (256 rows per sample), until `budget_s` seconds or max_steps samples."""
+    import oracle
+    wl = WORKLOADS[workload]
+    lay = synth.config_layers(wl["cfg"])[wl["layers"][0]]
+    W, qs = synth.make_float_weight(lay)
+    rng = np.random.default_rng(0)
+    done = 0.0
+    t_total = 0.0
+    n = 0
+    rows_per = 256
+    while True:
+        rows = np.sort(rng.choice(lay.N, rows_per, replace=False))
+        t0 = time.perf_counter()
+        oracle.quantize_weight(W[rows], lay.channel_scales, lay.pairs, lay.theta, qs[:, rows], GROUP, KROT)
+        t_total += time.perf_counter() - t0
+        done += quantize_bytes(lay.K, lay.N) * rows_per / lay.N
+        n += 1
+        if t_total >= budget_s or (max_steps and n >= max_steps):
+            desc = (f"float64 oracle weight quantiser on {n} samples of {rows_per} rows of "
+                    f"{lay.name} {lay.N}x{lay.K} (transform, quantise, pack)")
+            return done / t_total / 1e9, desc, t_total
+
+
 # ----------------------------------------------------------------- CPU oracle (baseline / reference)
 def oracle_sample(workload, budget_s, max_steps=None):
     """Times the float64 oracle on column samples of the workload's calls until
@@ -393,6 +558,8 @@ def oracle_sample(workload, budget_s, max_steps=None):
     (value in the workload's unit, description, seconds)."""
     import oracle
     wl = WORKLOADS[workload]
+    if wl["kind"] == "quantize":
+        return quantize_oracle_sample(workload, budget_s, max_steps)
     layers = [synth.config_layers(wl["cfg"])[i] for i in wl["layers"]]
     decode = wl["kind"] == "decode"
     rng = np.random.default_rng(0)
@@ -421,6 +588,8 @@ def oracle_sample(workload, budget_s, max_steps=None):
 
 
 def metric_name(workload):
+    if WORKLOADS[workload]["kind"] == "quantize":
+        return f"weight quantiser HBM throughput ({workload})"
     decode = WORKLOADS[workload]["kind"] == "decode"
     return ("rotated W4 linear decode HBM throughput" if decode else
             "rotated W4 linear prefill tensor throughput") + f" ({workload})"
@@ -432,7 +601,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     wl = WORKLOADS[args.workload]
-    decode = wl["kind"] == "decode"
+    decode = wl["kind"] in ("decode", "quantize")
     cores = len(os.sched_getaffinity(0))
     per_step_budget = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
     oracle_sample(args.workload, per_step_budget * args.warmup, max_steps=args.warmup)
@@ -482,7 +651,10 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    out = run_ours(args, rank, world, local_rank)
+    if WORKLOADS[args.workload]["kind"] == "quantize":
+        out = run_quantize(args, rank, world, local_rank)
+    else:
+        out = run_ours(args, rank, world, local_rank)
     if rank == 0:
         val, desc, _ = oracle_sample(args.workload, args.cpu_budget)
         out["cpu_baseline"] = {"value": round(val, 5), "unit": out["unit"],
