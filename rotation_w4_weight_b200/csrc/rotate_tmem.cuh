@@ -25,8 +25,21 @@
 // rotate_kernel.
 //
 // Slot order of a stage: pairs 2u and 2u+1 form unit u, whose four slots hold
-// (a_2u, a_2u+1, b_2u, b_2u+1), so a unit is rotated with packed fp32x2
-// multiplies and fmas: A' = A*C + B*S, B' = A*(-S) + B*C, A = (a_2u, a_2u+1).
+// (a_2u, a_2u+1, b_2u, b_2u+1), so a unit is rotated with packed fp32x2 fmas.
+//
+// Factored rotations (the square-root-free Givens form of Gentleman, 1973):
+// the value kept for a channel is its true value divided by a per-channel
+// factor f that depends only on the tables, so it is known when they are
+// built.  A pair (a, b) with factors (fa, fb) then takes two fmas,
+// a' = a + kA b and b' = b + kB a.  If |cos| >= |sin|: kA = tan * fb / fa,
+// kB = -tan * fa / fb and both factors take a cos.  Otherwise the two
+// channels trade slots: the slot of a receives b's new value and the slot of
+// b a's, with kA = -cot * fb / fa, kB = cot * fa / fb and factors (-sin fa)
+// for b and (sin fb) for a (tan, cot here mean sin/cos, cos/sin).  Choosing
+// the larger of |cos|, |sin| keeps |tan|, |cot| <= 1 and each factor within
+// [2^(-s/2), 1] of its start after s stages.  The starting factor is the
+// channel scale, so the input is not scaled; the final factors multiply the
+// output once.
 //
 // With ABS the gather tables hold absolute TMEM addresses, one copy per lane
 // quadrant, so a gather is a quarter of a table read and one load; without it
@@ -211,6 +224,8 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
   // ((s + 1) & 1); a slot's gather entry is where its channel sits in that
   // buffer: the channel index (s = 0) or its slot in stage s-1.  With ABS an
   // entry is the full TMEM address for each lane quadrant, else the column.
+  // The unit table's (cos, sin) become the factored form's (kA, kB), and
+  // scale[] follows every channel's factor (the final factors at the end).
   constexpr int Q = ABS ? 4 : 1;
   if (warp == 0) {
 #pragma unroll
@@ -218,6 +233,7 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
     __syncwarp();
     for (int s = 0; s < krot; ++s) {
       int si[2], sj[2], ii[2], jj[2];
+      bool tr[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int p = lane + 32 * e, u = p >> 1, w = p & 1;
@@ -228,22 +244,47 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
         sj[e] = 4 * u + 2 + w;
         const uint32_t ci = (uint32_t)((s & 1) * 128 + pos[ii[e]]);
         const uint32_t cj = (uint32_t)((s & 1) * 128 + pos[jj[e]]);
+        // factored form of this pair (each channel belongs to one pair of the
+        // stage, so its factor is read and written by this lane only)
+        float* csu = reinterpret_cast<float*>(cstab + s * L::CS_STAGE) + 4 * u;
+        const float c = csu[w], sn = csu[2 + w];
+        const float fa = scale[ii[e]], fb = scale[jj[e]];
+        const bool trade = fabsf(sn) > fabsf(c);
+        float ka, kb, nfa, nfb;
+        if (!trade) {
+          const float t = sn / c;
+          ka = t * (fb / fa);
+          kb = -t * (fa / fb);
+          nfa = c * fa;
+          nfb = c * fb;
+        } else {
+          const float t = c / sn;
+          ka = -t * (fb / fa);
+          kb = t * (fa / fb);
+          nfa = sn * fb;                             // a's new value, now in b's slot
+          nfb = -sn * fa;                            // b's new value, now in a's slot
+        }
+        csu[w] = ka;
+        csu[2 + w] = kb;
+        scale[ii[e]] = nfa;
+        scale[jj[e]] = nfb;
+        tr[e] = trade;
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
           const uint32_t lb = ABS ? tmem0 + ((uint32_t)(32 * q) << 16) : 0u;
           gtab[((size_t)q * krot + s) * 128 + si[e]] = lb + ci;
           gtab[((size_t)q * krot + s) * 128 + sj[e]] = lb + cj;
           if (s == krot - 1) {                       // the last stage scatters to channel order
-            ftab[q * 128 + si[e]] = lb + (uint32_t)((krot & 1) * 128 + ii[e]);
-            ftab[q * 128 + sj[e]] = lb + (uint32_t)((krot & 1) * 128 + jj[e]);
+            ftab[q * 128 + si[e]] = lb + (uint32_t)((krot & 1) * 128 + (trade ? jj[e] : ii[e]));
+            ftab[q * 128 + sj[e]] = lb + (uint32_t)((krot & 1) * 128 + (trade ? ii[e] : jj[e]));
           }
         }
       }
       __syncwarp();
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        pos[ii[e]] = si[e];
-        pos[jj[e]] = sj[e];
+        pos[ii[e]] = tr[e] ? sj[e] : si[e];
+        pos[jj[e]] = tr[e] ? si[e] : sj[e];
       }
       __syncwarp();
     }
@@ -273,12 +314,9 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
     for (int q = 0; q < SW / 8; ++q) {
       const uint4 raw = *reinterpret_cast<const uint4*>(rowp + ((((uint32_t)(q0 + q)) ^ rsw) << 4));
       const __half2* hv = reinterpret_cast<const __half2*>(&raw);
-      const float4 sa = scale4[2 * q], sc = scale4[2 * q + 1];
-      const float2 s2[4] = {make_float2(sa.x, sa.y), make_float2(sa.z, sa.w), make_float2(sc.x, sc.y),
-                            make_float2(sc.z, sc.w)};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __fmul2_rn(__half22float2(hv[e]), s2[e]);
+      for (int e = 0; e < 4; ++e) {                  // the channel scale is the starting factor
+        const float2 f = __half22float2(hv[e]);
         v[8 * q + 2 * e] = __float_as_uint(f.x);
         v[8 * q + 2 * e + 1] = __float_as_uint(f.y);
       }
@@ -317,18 +355,17 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
         tmem_ld_wait_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[0]));
 #pragma unroll
         for (int b = 1; b < SW / 32; ++b) tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
-        // rotate the SW/4 units (A = slots 0,1; B = slots 2,3)
+        // rotate the SW/4 units (A = slots 0,1; B = slots 2,3), factored form
         const uint32_t cst = cs_part + (uint32_t)s * (uint32_t)L::CS_STAGE;
 #pragma unroll
         for (int k = 0; k < SW / 4; ++k) {
-          const uint4 t = lds128(cst + 16 * k);      // (c0, c1, s0, s1)
-          const float2 C = make_float2(__uint_as_float(t.x), __uint_as_float(t.y));
-          const float2 S = make_float2(__uint_as_float(t.z), __uint_as_float(t.w));
-          const float2 NS = make_float2(-S.x, -S.y);
+          const uint4 t = lds128(cst + 16 * k);      // (kA0, kA1, kB0, kB1)
+          const float2 KA = make_float2(__uint_as_float(t.x), __uint_as_float(t.y));
+          const float2 KB = make_float2(__uint_as_float(t.z), __uint_as_float(t.w));
           const float2 A = make_float2(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]));
           const float2 B = make_float2(__uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
-          const float2 A2 = __ffma2_rn(A, C, __fmul2_rn(B, S));
-          const float2 B2 = __ffma2_rn(A, NS, __fmul2_rn(B, C));
+          const float2 A2 = __ffma2_rn(B, KA, A);
+          const float2 B2 = __ffma2_rn(A, KB, B);
           v[4 * k] = __float_as_uint(A2.x);
           v[4 * k + 1] = __float_as_uint(A2.y);
           v[4 * k + 2] = __float_as_uint(B2.x);
@@ -359,6 +396,19 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
       for (int b = 1; b < SW / 32; ++b) tmem_tie(*reinterpret_cast<uint32_t(*)[32]>(&v[32 * b]));
     }
 
+    // ---- true values of channels SW*h .. SW*h+SW-1: times their final factors
+#pragma unroll
+    for (int q = 0; q < SW / 4; ++q) {
+      const float4 f = scale4[q];
+      const float2 lo = __fmul2_rn(make_float2(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1])),
+                                   make_float2(f.x, f.y));
+      const float2 hi = __fmul2_rn(make_float2(__uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])),
+                                   make_float2(f.z, f.w));
+      v[4 * q] = __float_as_uint(lo.x);
+      v[4 * q + 1] = __float_as_uint(lo.y);
+      v[4 * q + 2] = __float_as_uint(hi.x);
+      v[4 * q + 3] = __float_as_uint(hi.y);
+    }
     const int row = tile * kRtRows + r;
     if constexpr (QUANT) {
       // ---- codes of row r (an output channel), channels SW*h .. SW*h+SW-1,
