@@ -183,6 +183,41 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
                    size_t workspace_bytes, paro_stream_t stream);
 
 /*
+ * Grouped decoder-layer calls — several linears that read the same x (a
+ * decoder layer's q/k/v, or gate/up), each with its own weights, rotation
+ * tables and output: y_i = rotate_i(x * cs_i) W_i + b_i for every member,
+ * exactly as that many paro_w4_linear calls would compute it (page
+ * "ParoQuant", "Activation and weight transforms": Y = X_r Q(W_r)^T + b per
+ * member).  At decode sizes the members share one rotation launch and one
+ * GEMV launch when the combined grid fits the GPU at once; otherwise (and for
+ * M > 16) the members run one after another.  Results may differ from the
+ * separate calls in fp32 summation order only.
+ *   linears         HOST array of `count` (1..PARO_MAX_GROUP) member descriptors;
+ *                   each member's fields follow paro_w4_linear's rules
+ *   x               device fp16 [M, K] shared by all members
+ *   workspace       >= paro_w4_linear_group_workspace_size(...) bytes, 256-byte
+ *                   aligned (may be NULL when no member rotates)
+ */
+#define PARO_MAX_GROUP 4
+typedef struct paro_linear {
+  int64_t N;                       /* output features of this member */
+  const int32_t* qweight;          /* [K, N/8] */
+  const int32_t* qzeros;           /* [K/G, N/8] */
+  const void* scales;              /* fp16 [K/G, N] */
+  const void* bias;                /* fp16 [N] or NULL */
+  const float* channel_scales;     /* [K] or NULL */
+  const int16_t* pairs;            /* [krot, K]; NULL only when krot == 0 */
+  const float* theta;              /* [krot, K/2]; NULL only when krot == 0 */
+  int krot;
+  void* y;                         /* fp16 [M, N] output */
+} paro_linear;
+
+size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, const paro_linear* linears,
+                                           int group_size);
+int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
+                         int group_size, void* workspace, size_t workspace_bytes, paro_stream_t stream);
+
+/*
  * paro_w4_linear_noalloc — paro_w4_linear for callers that cannot allocate
  * device memory.  The paper has no counterpart; this entry point exists for
  * library users, not for the method.

@@ -8,6 +8,7 @@ streams) into that ABI.  Functions mirror the C entry points:
     pack_awq          -> paro_pack_awq
     unpack_awq        -> paro_unpack_awq
     w4_linear         -> paro_w4_linear (+ paro_w4_linear_workspace_size)
+    w4_linear_group   -> paro_w4_linear_group (+ paro_w4_linear_group_workspace_size)
     quantize_w4       -> paro_quantize_w4
     validate_pairs    -> paro_validate_pairs (host helper)
     device_status     -> paro_device_status
@@ -24,10 +25,11 @@ from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # n
                    PARO_ERR_TIMEOUT, PARO_ERR_UNSUPPORTED, PARO_ERR_WORKSPACE, PARO_OK,
                    LIB_PATH, ParoError, check, lib, paro_device_status, paro_pack_awq,
                    paro_quantize_w4, paro_rotate, paro_status_string, paro_unpack_awq,
-                   paro_validate_pairs, paro_version, paro_w4_linear, paro_w4_linear_workspace_size)
+                   paro_validate_pairs, paro_version, paro_w4_linear, paro_w4_linear_workspace_size,
+                   PARO_MAX_GROUP, ParoLinear, paro_w4_linear_group, paro_w4_linear_group_workspace_size)
 
 __all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
-           "quantize_w4", "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
+           "w4_linear_group", "quantize_w4", "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -172,3 +174,45 @@ def validate_pairs(pairs: np.ndarray, K: int, group_size: int = 128, krot: Optio
 def device_status(clear: bool = True) -> int:
     """Synchronises and returns the device status word as a PARO_* code."""
     return int(paro_device_status(1 if clear else 0))
+
+
+def _members(x: torch.Tensor, members, outs):
+    arr = (ParoLinear * len(members))()
+    for i, m in enumerate(members):
+        _need(m["qweight"], torch.int32, "qweight")
+        _need(m["qzeros"], torch.int32, "qzeros")
+        _need(m["scales"], torch.float16, "scales")
+        _need(m.get("bias"), torch.float16, "bias", True)
+        _need(m.get("channel_scales"), torch.float32, "channel_scales", True)
+        _need(m.get("pairs"), torch.int16, "pairs", True)
+        _need(m.get("theta"), torch.float32, "theta", True)
+        krot = m.get("krot")
+        if krot is None:
+            krot = 0 if m.get("pairs") is None else m["pairs"].shape[0]
+        N = m["qweight"].shape[1] * 8
+        arr[i] = ParoLinear(N, m["qweight"].data_ptr(), m["qzeros"].data_ptr(), m["scales"].data_ptr(),
+                            None if m.get("bias") is None else m["bias"].data_ptr(),
+                            None if m.get("channel_scales") is None else m["channel_scales"].data_ptr(),
+                            None if m.get("pairs") is None else m["pairs"].data_ptr(),
+                            None if m.get("theta") is None else m["theta"].data_ptr(), krot,
+                            outs[i].data_ptr())
+    return arr
+
+
+def w4_linear_group(x: torch.Tensor, members, group_size: int = 128, workspace: Optional[torch.Tensor] = None,
+                    out=None, stream=None):
+    """Several linears over the same x (q/k/v, gate/up): ``members`` is a list of
+    dicts with keys qweight, qzeros, scales and optionally bias, channel_scales,
+    pairs, theta, krot.  Returns the list of fp16 outputs [M, N_i]."""
+    _need(x, torch.float16, "x")
+    M, K = x.shape
+    if out is None:
+        out = [torch.empty((M, m["qweight"].shape[1] * 8), dtype=torch.float16, device=x.device)
+               for m in members]
+    arr = _members(x, members, out)
+    need = int(paro_w4_linear_group_workspace_size(M, K, len(members), arr, group_size))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    check(paro_w4_linear_group(_ptr(x), M, K, len(members), arr, group_size, _ptr(workspace),
+                               workspace.numel(), _stream(stream)), "paro_w4_linear_group")
+    return out

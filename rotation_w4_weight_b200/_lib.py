@@ -24,7 +24,18 @@ EXPORTED = (
     "paro_status_string", "paro_version", "paro_rotate", "paro_pack_awq", "paro_unpack_awq",
     "paro_w4_linear_workspace_size", "paro_w4_linear", "paro_w4_linear_noalloc",
     "paro_validate_pairs", "paro_device_status", "paro_quantize_w4",
+    "paro_w4_linear_group_workspace_size", "paro_w4_linear_group",
 )
+
+PARO_MAX_GROUP = 4
+
+
+class ParoLinear(ctypes.Structure):
+    """struct paro_linear of the header (one member of a grouped call)."""
+    _fields_ = [("N", ctypes.c_int64), ("qweight", ctypes.c_void_p), ("qzeros", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("channel_scales", ctypes.c_void_p),
+                ("pairs", ctypes.c_void_p), ("theta", ctypes.c_void_p), ("krot", ctypes.c_int),
+                ("y", ctypes.c_void_p)]
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -44,6 +55,8 @@ _SIGNATURES = {
     "paro_validate_pairs": (_int, [_vp, _i64, _int, _int]),
     "paro_device_status": (_int, [_int]),
     "paro_quantize_w4": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp]),
+    "paro_w4_linear_group_workspace_size": (ctypes.c_size_t, [_i64, _i64, _int, _vp, _int]),
+    "paro_w4_linear_group": (_int, [_vp, _i64, _i64, _int, _vp, _int, _vp, ctypes.c_size_t, _vp]),
 }
 
 
@@ -74,6 +87,8 @@ PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES = 8 << 20
 paro_validate_pairs = lib.paro_validate_pairs
 paro_device_status = lib.paro_device_status
 paro_quantize_w4 = lib.paro_quantize_w4
+paro_w4_linear_group_workspace_size = lib.paro_w4_linear_group_workspace_size
+paro_w4_linear_group = lib.paro_w4_linear_group
 
 
 class ParoError(RuntimeError):

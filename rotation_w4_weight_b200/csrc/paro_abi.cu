@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
+#include <cstring>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -201,6 +203,17 @@ int check_rotation_args(const void* x, const void* xr, int64_t M, int64_t K, con
   return PARO_OK;
 }
 
+// Warp-per-row rotation of one x for `count` linears (blockIdx.z), decode sizes
+// (M <= 16, every krot <= kRrMaxKrot; max_krot sizes the tables).
+int launch_rotate_rows(const __half* x, const RrBatch& b, int count, int64_t M, int64_t K, int max_krot,
+                       cudaStream_t stream) {
+  // always 8 warps: all of them build the tables, warps past the batch then leave
+  const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + kRrWarps - 1) / kRrWarps), (unsigned)count);
+  if (!allow_smem(rotate_rows_kernel, RrLayout::bytes(kRrMaxKrot))) return PARO_ERR_CUDA;
+  return launch(rotate_rows_kernel, grid, dim3(32 * kRrWarps), RrLayout::bytes(max_krot), stream, true, b, x,
+                (int)M, (int)K);
+}
+
 // Tensor-memory rotation kernel (and, with QUANT, the weight quantiser): CTAs
 // stay resident over several 128-row tiles of one group (one wave of at most
 // 2 CTAs per SM: the shared-memory floor of the kernel guarantees no more fit).
@@ -245,11 +258,10 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
   if (M > 64) return launch_rotate_tmem<false>(x, xr, M, K, cs, pairs, theta, krot, RtQuant{}, stream);
   // Decode batches with few stages: one warp per row, no block barrier per stage.
   if (M <= 16 && krot <= kRrMaxKrot) {
-    // always 8 warps: all of them build the tables, warps past the batch then leave
-    const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + kRrWarps - 1) / kRrWarps));
-    if (!allow_smem(rotate_rows_kernel, RrLayout::bytes(kRrMaxKrot))) return PARO_ERR_CUDA;
-    return launch(rotate_rows_kernel, grid, dim3(32 * kRrWarps), RrLayout::bytes(krot), stream, true, x, xr,
-                  cs, pairs, theta, (int)M, (int)K, krot);
+    RrBatch b;
+    std::memset(&b, 0, sizeof(b));
+    b.op[0] = RrOperand{xr, cs, pairs, theta, krot};
+    return launch_rotate_rows(x, b, 1, M, K, krot, stream);
   }
   // rows per CTA: 4 for decode-sized batches (more CTAs, shorter latency),
   // 32..64 otherwise (conflict-free 32-row warp accesses)
@@ -377,48 +389,83 @@ size_t gemv_footprint(size_t need, int64_t ctas) {
   return std::min(dev.smem_optin, std::max(need, want));
 }
 
-// Decode GEMV launch: grid (column tiles, splits), one cluster of `splits`
-// CTAs along K per column tile.
-template <int NT, int KP, int NTILE, int STAGES>
-int launch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
-                const void* scales, const __half* x, const __half* bias, __half* y,
-                int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
+// One linear of a decode GEMV launch.
+struct GemvLinearArgs {
+  const void* qweight;
+  const void* qzeros;
+  const void* scales;
+  const __half* x;        // the activations the GEMV reads (X_r, or x itself)
+  const __half* bias;
+  __half* y;
+  int64_t N;
+};
+
+// Decode GEMV launch over `count` (<= NL) linears sharing M and K: grid
+// (column tiles of every linear, splits), one cluster of `splits` CTAs along K
+// per column tile.
+template <int NT, int KP, int NTILE, int STAGES, int NL>
+int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, int64_t M, int64_t K,
+                cudaStream_t s, bool pdl) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
   const int groups = (int)(K / kGroup);
   const int gmax = (groups + plan.splits - 1) / plan.splits;   // largest group range of a CTA
-  if (gmax > kGvMaxGroups) return PARO_ERR_UNSUPPORTED;
-  CUtensorMap tmW, tmS, tmZ, tmX;
-  const bool ok =
-      encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 128, L::WORDS,
-                L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                    : (L::ROW_BYTES == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE)) &&
-      encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, (uint32_t)gmax,
-                NTILE, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, (uint32_t)gmax,
-                L::WORDS, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      encode_x_chunks(&tmX, x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP, (uint32_t)(2 * gmax));
-  if (!ok) return PARO_ERR_CUDA;
-  auto k = w4_gemv_kernel<NT, KP, NTILE, STAGES>;
-  const dim3 grid((unsigned)((N + NTILE - 1) / NTILE), (unsigned)plan.splits, 1);
+  if (gmax > kGvMaxGroups || count < 1 || count > NL) return PARO_ERR_UNSUPPORTED;
+  GemvBatch<NL> b;
+  std::memset(&b, 0, sizeof(b));
+  int64_t tiles = 0;
+  for (int i = 0; i < NL; ++i) {
+    GemvOperand& o = b.op[i];
+    if (i >= count) {
+      o.tile_begin = INT_MAX;                   // never selected
+      continue;
+    }
+    const int64_t N = lin[i].N;
+    const bool ok =
+        encode_2d(&o.w, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qweight, K, N / 8, 128, L::WORDS,
+                  L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                      : (L::ROW_BYTES == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE)) &&
+        encode_2d(&o.s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, lin[i].scales, K / kGroup, N, (uint32_t)gmax,
+                  NTILE, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, K / kGroup, N / 8, (uint32_t)gmax,
+                  L::WORDS, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        encode_x_chunks(&o.x, lin[i].x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP, (uint32_t)(2 * gmax));
+    if (!ok) return PARO_ERR_CUDA;
+    o.bias = lin[i].bias;
+    o.y = lin[i].y;
+    o.n = (int)N;
+    o.tile_begin = (int)tiles;
+    tiles += (N + NTILE - 1) / NTILE;
+  }
+  if (tiles > INT_MAX / 2) return PARO_ERR_UNSUPPORTED;
+  auto k = w4_gemv_kernel<NT, KP, NTILE, STAGES, NL>;
+  const dim3 grid((unsigned)tiles, (unsigned)plan.splits, 1);
   const size_t smem = gemv_footprint((size_t)L::smem(gmax), (int64_t)grid.x * grid.y);
   if (smem == 0 || !allow_smem(k, device_info().smem_optin)) return PARO_ERR_CUDA;
   // a grid larger than the SM count places its clusters by load (measured:
   // 256-CTA grids of 8-CTA clusters ran 1-10 % faster; one-per-SM grids did not gain)
   const bool balance = (int64_t)grid.x * grid.y > device_info().sms;
-  return launch_ex(k, grid, dim3(L::THREADS), smem, s, pdl, (unsigned)plan.splits, balance, tmW, tmX,
-                   tmS, tmZ, bias, y, (int)M, (int)N, (int)K, gmax);
+  return launch_ex(k, grid, dim3(L::THREADS), smem, s, pdl, (unsigned)plan.splits, balance, b, (int)M,
+                   (int)K, gmax);
 }
 
-template <int NT>
-int dispatch_gemv(const LinearPlan& plan, const void* qweight, const void* qzeros,
-                  const void* scales, const __half* x, const __half* bias, __half* y,
-                  int64_t M, int64_t N, int64_t K, cudaStream_t s, bool pdl) {
+template <int NT, int NL>
+int dispatch_gemv_nl(const LinearPlan& plan, const GemvLinearArgs* lin, int count, int64_t M, int64_t K,
+                     cudaStream_t s, bool pdl) {
   switch (plan.variant) {
-    case 0: return launch_gemv<NT, 2, 256, 4>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
-    case 2: return launch_gemv<NT, 4, 128, 8>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
-    case 5: return launch_gemv<NT, 4, 64, 8>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
-    default: return launch_gemv<NT, 2, 128, 4>(plan, qweight, qzeros, scales, x, bias, y, M, N, K, s, pdl);
+    case 0: return launch_gemv<NT, 2, 256, 4, NL>(plan, lin, count, M, K, s, pdl);
+    case 2: return launch_gemv<NT, 4, 128, 8, NL>(plan, lin, count, M, K, s, pdl);
+    case 5: return launch_gemv<NT, 4, 64, 8, NL>(plan, lin, count, M, K, s, pdl);
+    default: return launch_gemv<NT, 2, 128, 4, NL>(plan, lin, count, M, K, s, pdl);
   }
+}
+
+int dispatch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, int64_t M, int64_t K,
+                  cudaStream_t s, bool pdl) {
+  if (count == 1)
+    return plan.nt == 1 ? dispatch_gemv_nl<1, 1>(plan, lin, count, M, K, s, pdl)
+                        : dispatch_gemv_nl<2, 1>(plan, lin, count, M, K, s, pdl);
+  return plan.nt == 1 ? dispatch_gemv_nl<1, kGvMaxLinears>(plan, lin, count, M, K, s, pdl)
+                      : dispatch_gemv_nl<2, kGvMaxLinears>(plan, lin, count, M, K, s, pdl);
 }
 
 }  // namespace
@@ -519,11 +566,13 @@ size_t paro_w4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int group_
   return make_plan(M, K, N).total;
 }
 
-int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
-                   const int32_t* qweight, const int32_t* qzeros, const void* scales,
-                   const void* bias, const float* channel_scales, const int16_t* pairs,
-                   const float* theta, int group_size, int krot, void* workspace,
-                   size_t workspace_bytes, paro_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// Every check of paro_w4_linear that does not involve the workspace.
+int check_linear_args(const void* x, const void* y, int64_t M, int64_t K, int64_t N, const int32_t* qweight,
+                      const int32_t* qzeros, const void* scales, const void* bias, const float* channel_scales,
+                      const int16_t* pairs, const float* theta, int group_size, int krot) {
   if (int st = check_linear_shape(M, K, N, group_size)) return st;
   if (krot < 0) return PARO_ERR_INVALID_ARG;
   if (krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
@@ -536,6 +585,59 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
     return PARO_ERR_ALIGNMENT;
   if (channel_scales != nullptr && !aligned(channel_scales, 16)) return PARO_ERR_ALIGNMENT;
   if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
+  return PARO_OK;
+}
+
+// Shared memory of the GEMV layout of a plan, for `gmax` groups per CTA.
+size_t gemv_smem(const LinearPlan& p, int gmax) {
+  const bool one = p.nt == 1;
+  switch (p.variant) {
+    case 0: return one ? GemvLayout<1, 2, 256, 4>::smem(gmax) : GemvLayout<2, 2, 256, 4>::smem(gmax);
+    case 2: return one ? GemvLayout<1, 4, 128, 8>::smem(gmax) : GemvLayout<2, 4, 128, 8>::smem(gmax);
+    case 5: return one ? GemvLayout<1, 4, 64, 8>::smem(gmax) : GemvLayout<2, 4, 64, 8>::smem(gmax);
+    default: return one ? GemvLayout<1, 2, 128, 4>::smem(gmax) : GemvLayout<2, 2, 128, 4>::smem(gmax);
+  }
+}
+
+int plan_tile(const LinearPlan& p) { return p.variant == 0 ? 256 : (p.variant == 5 ? 64 : 128); }
+
+// One GEMV launch for a group of decode linears sharing x: the plan of the
+// widest member for all of them, taken only when the whole grid is resident
+// at once with that plan's footprint (larger groups gain nothing from sharing
+// a launch: each member already fills the GPU).
+bool group_plan(int64_t M, int64_t K, const paro_linear* lin, int count, LinearPlan* out) {
+  int64_t widest = 0;
+  for (int i = 0; i < count; ++i) widest = std::max(widest, lin[i].N);
+  LinearPlan p = make_plan(M, K, widest);
+  if (!p.decode) return false;
+  const int tile = plan_tile(p);
+  int64_t tiles = 0;
+  for (int i = 0; i < count; ++i) tiles += (lin[i].N + tile - 1) / tile;
+  const int64_t ctas = tiles * p.splits;
+  const int groups = (int)(K / kGroup);
+  const int gmax = (groups + p.splits - 1) / p.splits;
+  const size_t fp = gemv_footprint(gemv_smem(p, gmax), ctas);
+  const DeviceInfo& dev = device_info();
+  if (fp == 0 || dev.sms <= 0) return false;
+  const int64_t per_sm = (int64_t)(dev.smem_per_sm / (fp + dev.smem_reserved_per_block));
+  if (ctas > per_sm * dev.sms) return false;
+  p.n_tiles = (int)tiles;
+  *out = p;
+  return true;
+}
+}  // namespace
+
+extern "C" {
+
+int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                   const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                   const void* bias, const float* channel_scales, const int16_t* pairs,
+                   const float* theta, int group_size, int krot, void* workspace,
+                   size_t workspace_bytes, paro_stream_t stream) {
+  if (int st = check_linear_args(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
+                                 group_size, krot))
+    return st;
+  if (M == 0) return PARO_OK;   // empty batch: nothing to read or write
 
   const LinearPlan plan = make_plan(M, K, N);
 
@@ -560,8 +662,88 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
     return launch_w4_prefill(xa, yy, M, K, N, qweight, qzeros, static_cast<const __half*>(scales),
                              b, s, pdl);
 
-  if (plan.nt == 1) return dispatch_gemv<1>(plan, qweight, qzeros, scales, xa, b, yy, M, N, K, s, pdl);
-  return dispatch_gemv<2>(plan, qweight, qzeros, scales, xa, b, yy, M, N, K, s, pdl);
+  const GemvLinearArgs one{qweight, qzeros, scales, xa, b, yy, N};
+  return dispatch_gemv(plan, &one, 1, M, K, s, pdl);
+}
+
+static_assert(PARO_MAX_GROUP == kGvMaxLinears && PARO_MAX_GROUP == kRrMaxLinears,
+              "one launch holds every member of a group");
+
+size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, const paro_linear* linears,
+                                           int group_size) {
+  if (count < 1 || count > PARO_MAX_GROUP || linears == nullptr) return 0;
+  size_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    if (check_linear_shape(M, K, linears[i].N, group_size) != PARO_OK) return 0;
+    total += make_plan(M, K, linears[i].N).total;
+  }
+  return total;
+}
+
+int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
+                         int group_size, void* workspace, size_t workspace_bytes, paro_stream_t stream) {
+  if (count < 1 || linears == nullptr) return PARO_ERR_INVALID_ARG;
+  if (count > PARO_MAX_GROUP) return PARO_ERR_UNSUPPORTED;
+  bool any_rotate = false;
+  for (int i = 0; i < count; ++i) {
+    const paro_linear& l = linears[i];
+    if (int st = check_linear_args(x, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, l.channel_scales,
+                                   l.pairs, l.theta, group_size, l.krot))
+      return st;
+    any_rotate = any_rotate || l.krot > 0 || l.channel_scales != nullptr;
+  }
+  if (M == 0) return PARO_OK;
+  const size_t need = paro_w4_linear_group_workspace_size(M, K, count, linears, group_size);
+  if (any_rotate && (workspace == nullptr || workspace_bytes < need)) return PARO_ERR_WORKSPACE;
+  if (any_rotate && !aligned(workspace, 256)) return PARO_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // member i's X_r lives at workspace + i * per (all members share M and K)
+  const size_t per = make_plan(M, K, linears[0].N).total;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+
+  LinearPlan gp;
+  if (count == 1 || !group_plan(M, K, linears, count, &gp)) {
+    // one call per member, each with its own slice of the workspace
+    for (int i = 0; i < count; ++i) {
+      const paro_linear& l = linears[i];
+      if (int st = paro_w4_linear(x, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, l.channel_scales,
+                                  l.pairs, l.theta, group_size, l.krot, ws ? ws + i * per : nullptr,
+                                  ws ? per : 0, stream))
+        return st;
+    }
+    return PARO_OK;
+  }
+
+  // every member's rotation of x: one warp-per-row launch when all fit it
+  const __half* xa = static_cast<const __half*>(x);
+  GemvLinearArgs lin[PARO_MAX_GROUP];
+  RrBatch rb;
+  std::memset(&rb, 0, sizeof(rb));
+  int nrot = 0, max_krot = 0;
+  bool rows_ok = M <= 16;
+  for (int i = 0; i < count; ++i) {
+    const paro_linear& l = linears[i];
+    const bool rot = l.krot > 0 || l.channel_scales != nullptr;
+    __half* xr = rot ? reinterpret_cast<__half*>(ws + i * per) : nullptr;
+    if (rot) {
+      rb.op[nrot++] = RrOperand{xr, l.channel_scales, l.pairs, l.theta, l.krot};
+      max_krot = std::max(max_krot, l.krot);
+      rows_ok = rows_ok && l.krot <= kRrMaxKrot;
+    }
+    lin[i] = GemvLinearArgs{l.qweight, l.qzeros, l.scales, rot ? xr : xa, static_cast<const __half*>(l.bias),
+                            static_cast<__half*>(l.y), l.N};
+  }
+  if (nrot > 0) {
+    if (rows_ok) {
+      if (int st = launch_rotate_rows(xa, rb, nrot, M, K, max_krot, s)) return st;
+    } else {
+      for (int r = 0; r < nrot; ++r)
+        if (int st = launch_rotate(xa, rb.op[r].xr, M, K, rb.op[r].cs, rb.op[r].pairs, rb.op[r].theta,
+                                   rb.op[r].krot, s))
+          return st;
+    }
+  }
+  return dispatch_gemv(gp, lin, count, M, K, s, true);
 }
 
 }  // extern "C"

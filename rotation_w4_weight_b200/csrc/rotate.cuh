@@ -165,10 +165,32 @@ struct RrLayout {
   __host__ __device__ static constexpr size_t bytes(int krot) { return row_off(krot) + kRrWarps * 512; }
 };
 
-__global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(
-    const __half* x, __half* xr, const float* __restrict__ cs, const int16_t* __restrict__ pairs,
-    const float* __restrict__ theta, int M, int K, int krot) {
+// Rotation tables and output of one linear; a launch rotates the same x for up
+// to kRrMaxLinears linears (blockIdx.z), each with its own tables.
+constexpr int kRrMaxLinears = 4;
+struct RrOperand {
+  __half* xr;
+  const float* cs;
+  const int16_t* pairs;
+  const float* theta;
+  int krot;
+};
+struct RrBatch {
+  RrOperand op[kRrMaxLinears];
+};
+
+__global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(const RrBatch batch, const __half* x,
+                                                                    int M, int K) {
   pdl_launch_dependents();                         // the GEMV may start streaming weights
+  RrOperand o = batch.op[0];
+#pragma unroll
+  for (int i = 1; i < kRrMaxLinears; ++i)
+    if ((int)blockIdx.z == i) o = batch.op[i];
+  __half* const xr = o.xr;
+  const float* __restrict__ const cs = o.cs;
+  const int16_t* __restrict__ const pairs = o.pairs;
+  const float* __restrict__ const theta = o.theta;
+  const int krot = o.krot;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint8_t* partner = smem_raw;
   float* cosv = reinterpret_cast<float*>(smem_raw + RrLayout::cos_off(krot));

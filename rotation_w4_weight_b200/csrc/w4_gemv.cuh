@@ -82,6 +82,25 @@ struct GemvLayout {
   static constexpr int ROW_BYTES = WORDS * 4;
 };
 
+// Operands of one linear of a launch.  A launch covers NL linears that share
+// the token count and K (a decoder layer's q/k/v, say): the column tiles of
+// linear l are blockIdx.x = tile_begin .. tile_begin + ceil(n / NTILE) - 1.
+struct alignas(64) GemvOperand {
+  CUtensorMap w;          // qweight [K, N/8] int32, box {NTILE/8 words, 128 rows}
+  CUtensorMap x;          // X_r [M, K] fp16 as [K/64][M][64], box {64, MP, 2 gmax}
+  CUtensorMap s;          // scales [K/128, N] fp16, box {NTILE, gmax}
+  CUtensorMap z;          // qzeros [K/128, N/8] int32, box {NTILE/8, gmax}
+  const __half* bias;     // [N] or nullptr
+  __half* y;              // [M, N]
+  int n;                  // output columns
+  int tile_begin;         // first column tile of this linear in the grid
+};
+template <int NL>
+struct GemvBatch {
+  GemvOperand op[NL];
+};
+constexpr int kGvMaxLinears = 4;
+
 __device__ __forceinline__ void gv_unpack4(uint32_t m, uint32_t (&e)[4]) {
   const uint32_t m8 = m >> 8;
   e[0] = and_or(m, 0x000F000Fu, kGvMagic);
@@ -90,12 +109,22 @@ __device__ __forceinline__ void gv_unpack4(uint32_t m, uint32_t (&e)[4]) {
   e[3] = and_or(m8, 0x00F000F0u, kGvMagic);
 }
 
-template <int NT, int KP, int NTILE, int STAGES>
+template <int NT, int KP, int NTILE, int STAGES, int NL>
 __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kernel(
-    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
-    const __half* __restrict__ bias, __half* __restrict__ Y, int M, int N, int K, int gmax) {
+    const __grid_constant__ GemvBatch<NL> ops, int M, int K, int gmax) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
+  // this CTA's linear (selected by constant offsets into the parameter block)
+  const GemvOperand* op = &ops.op[0];
+#pragma unroll
+  for (int i = 1; i < NL; ++i)
+    if ((int)blockIdx.x >= ops.op[i].tile_begin) op = &ops.op[i];
+  const CUtensorMap* const tmW = &op->w;
+  const CUtensorMap* const tmX = &op->x;
+  const CUtensorMap* const tmS = &op->s;
+  const CUtensorMap* const tmZ = &op->z;
+  const __half* const bias = op->bias;
+  __half* const Y = op->y;
+  const int N = op->n;
   constexpr int kGvStages = STAGES;
   constexpr int kGvTile = NTILE;
   // The next kernel in the stream may launch now; it waits for our completion
@@ -112,7 +141,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const uint32_t xbar = cbar + 8;                  // X_r
   const uint32_t inbar = xbar + 8;                 // peers' split-K partials landed
 
-  const int ntile = blockIdx.x, split = blockIdx.y;
+  const int ntile = (int)blockIdx.x - op->tile_begin, split = blockIdx.y;
   const int n0 = ntile * kGvTile;
   const int groups = K / 128;
   // 32-bit arithmetic (groups <= 2^16, splits <= 8): no 64-bit division routine
@@ -134,10 +163,10 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     fence_barrier_init();
     // every peer's k-part partials of this CTA's columns, counted in bytes
     if (S > 1) mbar_arrive_expect_tx(inbar, (uint32_t)((S - 1) * KP * mrows * (kGvTile / S) * 4));
-    tma_prefetch_desc(&tmW);
-    tma_prefetch_desc(&tmX);
-    tma_prefetch_desc(&tmS);
-    tma_prefetch_desc(&tmZ);
+    tma_prefetch_desc(tmW);
+    tma_prefetch_desc(tmX);
+    tma_prefetch_desc(tmS);
+    tma_prefetch_desc(tmZ);
   }
   __syncthreads();
   // the peers may address this CTA's inbox barrier once every CTA has set its own up
@@ -163,22 +192,22 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       // the tensor maps' boxes hold gmax groups (the largest range of any CTA;
       // rows past this CTA's range are loaded and not used)
       mbar_arrive_expect_tx(cbar, (uint32_t)(gmax * (NTILE * 2 + L::WORDS * 4)));
-      tma_load_2d(base + L::s_off(gmax), &tmS, cbar, n0, g_begin);
-      tma_load_2d(base + L::z_off(gmax), &tmZ, cbar, n0 / 8, g_begin);
+      tma_load_2d(base + L::s_off(gmax), tmS, cbar, n0, g_begin);
+      tma_load_2d(base + L::z_off(gmax), tmZ, cbar, n0 / 8, g_begin);
       for (int i = 0; i < pre; ++i) {
         const uint32_t bar = full0 + 8 * i;
         mbar_arrive_expect_tx(bar, L::W_BYTES);
-        tma_load_2d_hint(base + i * L::STAGE, &tmW, bar, n0 / 8, (g_begin + i) * 128, pol);
+        tma_load_2d_hint(base + i * L::STAGE, tmW, bar, n0 / 8, (g_begin + i) * 128, pol);
       }
       pdl_wait_primary();                  // X_r comes from the rotation kernel
       mbar_arrive_expect_tx(xbar, (uint32_t)(gmax * L::XG_BYTES));
-      tma_load_3d(base + L::X_OFF, &tmX, xbar, 0, 0, 2 * g_begin);
+      tma_load_3d(base + L::X_OFF, tmX, xbar, 0, 0, 2 * g_begin);
       for (int i = pre; i < ng; ++i) {
         const int s = i % kGvStages;
         if (!mbar_wait_bounded(empty0 + 8 * s, ((i / kGvStages) - 1) & 1)) break;
         const uint32_t bar = full0 + 8 * s;
         mbar_arrive_expect_tx(bar, L::W_BYTES);
-        tma_load_2d_hint(base + s * L::STAGE, &tmW, bar, n0 / 8, (g_begin + i) * 128, pol);
+        tma_load_2d_hint(base + s * L::STAGE, tmW, bar, n0 / 8, (g_begin + i) * 128, pol);
       }
     }
   } else {

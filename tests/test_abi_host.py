@@ -139,3 +139,31 @@ def test_quantize_argument_validation(L):
     assert q(MIS, None, A16, A16, A16, A16, A16, 16, 256, 128, 8, None) == L.PARO_ERR_ALIGNMENT
     assert q(A16, None, A16, A16, A16, P(0x10002), A16, 16, 256, 128, 8, None) == L.PARO_ERR_ALIGNMENT
     assert q(A16, None, A16, A16, A16, A16, A16, 0, 256, 128, 8, None) == L.PARO_OK   # empty: no-op
+
+
+def test_group_argument_validation_and_workspace(L):
+    def member(N=512, krot=8, y=A16, pairs=A16, qweight=A16):
+        return L.ParoLinear(N, qweight.value, A16.value, A16.value, None, A16.value, pairs and pairs.value,
+                            A16.value, krot, y and y.value)
+    arr = (L.ParoLinear * 3)(member(4096), member(1024), member(1024))
+    f = L.paro_w4_linear_group_workspace_size
+    per = L.paro_w4_linear_workspace_size(4, 4096, 4096, 128)
+    assert per > 0 and f(4, 4096, 3, arr, 128) == 3 * per
+    assert f(4, 4096, 0, arr, 128) == 0 and f(4, 4096, 5, arr, 128) == 0
+    g = L.paro_w4_linear_group
+    assert g(A16, 4, 4096, 0, arr, 128, A16, 1 << 30, None) == L.PARO_ERR_INVALID_ARG
+    assert g(A16, 4, 4096, 5, arr, 128, A16, 1 << 30, None) == L.PARO_ERR_UNSUPPORTED
+    assert g(A16, 4, 4096, 3, None, 128, A16, 1 << 30, None) == L.PARO_ERR_INVALID_ARG
+    bad = (L.ParoLinear * 2)(member(4096), member(1004))          # N % 8
+    assert g(A16, 4, 4096, 2, bad, 128, A16, 1 << 30, None) == L.PARO_ERR_INVALID_ARG
+    bad = (L.ParoLinear * 2)(member(4096), member(1024, y=None))  # no output
+    assert g(A16, 4, 4096, 2, bad, 128, A16, 1 << 30, None) == L.PARO_ERR_INVALID_ARG
+    bad = (L.ParoLinear * 2)(member(4096), member(1024, pairs=None))
+    assert g(A16, 4, 4096, 2, bad, 128, A16, 1 << 30, None) == L.PARO_ERR_INVALID_ARG
+    bad = (L.ParoLinear * 2)(member(4096), member(1024, qweight=MIS))
+    assert g(A16, 4, 4096, 2, bad, 128, A16, 1 << 30, None) == L.PARO_ERR_ALIGNMENT
+    assert g(MIS, 4, 4096, 3, arr, 128, A16, 1 << 30, None) == L.PARO_ERR_ALIGNMENT
+    assert g(A16, 4, 4096, 3, arr, 128, None, 0, None) == L.PARO_ERR_WORKSPACE
+    assert g(A16, 4, 4096, 3, arr, 128, A16, 3 * per - 1, None) == L.PARO_ERR_WORKSPACE
+    assert g(A16, 4, 4096, 3, arr, 128, P(0x10010), 1 << 30, None) == L.PARO_ERR_ALIGNMENT
+    assert g(A16, 0, 4096, 3, arr, 128, None, 0, None) == L.PARO_OK      # empty batch
