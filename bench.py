@@ -43,12 +43,16 @@ L2_BYTES = 126 * 1024 * 1024
 GROUP = 128
 KROT = 8
 
+# "groups": linears that read the same x go through one grouped call
+# (paro_w4_linear_group: q/k/v and gate/up of a decoder layer)
 WORKLOADS = {
-    "q_proj_decode": dict(cfg=1, layers=[0], Ms=[1, 4, 16], kind="decode"),
-    "mlp_decode": dict(cfg=2, layers=[0, 1, 2], Ms=[1, 8], kind="decode"),
-    "prefill": dict(cfg=3, layers=[0], Ms=[2048, 8192], kind="prefill"),
-    "layer_decode": dict(cfg=4, layers=list(range(7)), Ms=[1], kind="decode"),
-    "layer_prefill": dict(cfg=4, layers=list(range(7)), Ms=[4096], kind="prefill"),
+    "q_proj_decode": dict(cfg=1, layers=[0], Ms=[1, 4, 16], kind="decode", groups=[[0]]),
+    "mlp_decode": dict(cfg=2, layers=[0, 1, 2], Ms=[1, 8], kind="decode", groups=[[0, 1], [2]]),
+    "prefill": dict(cfg=3, layers=[0], Ms=[2048, 8192], kind="prefill", groups=[[0]]),
+    "layer_decode": dict(cfg=4, layers=list(range(7)), Ms=[1], kind="decode",
+                         groups=[[0, 1, 2], [3], [4, 5], [6]]),
+    "layer_prefill": dict(cfg=4, layers=list(range(7)), Ms=[4096], kind="prefill",
+                          groups=[[0, 1, 2], [3], [4, 5], [6]]),
     "quantize_gate_proj": dict(cfg=2, layers=[0], Ms=[], kind="quantize"),
 }
 
@@ -198,6 +202,7 @@ def workload_config(workload, world):
                 "input": "float W fp16 [N, K] and quantiser scales fp16 [K/128, N]",
                 "group_size": GROUP, "krot": KROT, "parallelism": f"replicas x{world}"}
     return {"workload": workload, "layers": [(l.name, l.K, l.N) for l in layers], "M": wl["Ms"],
+            "calls": [[layers[i].name for i in g] for g in wl["groups"]],
             "group_size": GROUP, "krot": KROT, "accumulate": "f32", "parallelism": f"replicas x{world}"}
 
 
@@ -229,26 +234,51 @@ def run_ours(args, rank, world, local_rank):
         replicas.append([{k: (v.clone() if torch.is_tensor(v) and k in ("qweight", "qzeros", "scales") else v)
                           for k, v in b.items()} for b in base])
     calls = [(li, M) for li in range(len(layers)) for M in Ms]
-    xs = {(li, M): T(synth.make_activations(layers[li], M)) for li, M in calls}
+    groups = wl["groups"]
+    gcalls = [(gi, M) for gi in range(len(groups)) for M in Ms]
+    # members of a group share their first layer's activations
+    xs = {}
+    for gi, M in gcalls:
+        xg = T(synth.make_activations(layers[groups[gi][0]], M))
+        for li in groups[gi]:
+            xs[(li, M)] = xg
     ys = {(li, M): torch.empty((M, layers[li].N), dtype=torch.float16, device=dev) for li, M in calls}
-    ws = {(li, M): torch.empty(max(256, pb.w4_linear_workspace_size(M, layers[li].K, layers[li].N)),
-                               dtype=torch.uint8, device=dev) for li, M in calls}
+    ws = {(gi, M): torch.empty(max(256, sum(pb.w4_linear_workspace_size(M, layers[li].K, layers[li].N)
+                                            for li in groups[gi])), dtype=torch.uint8, device=dev)
+          for gi, M in gcalls}
     xrs = {(li, M): torch.empty((M, layers[li].K), dtype=torch.float16, device=dev) for li, M in calls}
+
+    def launches(gi, M, rotate=True):
+        grp = groups[gi]
+        return pb.w4_linear_group_launches(
+            M, layers[grp[0]].K, [dict(N=layers[li].N, krot=KROT if rotate else 0, channel_scales=rotate)
+                                  for li in grp], GROUP)
 
     stream = torch.cuda.Stream(device=dev)
     step_bytes = sum(call_bytes(layers[li].K, layers[li].N, M, layers[li].bias is not None)
                      for li, M in calls)
     step_flops = sum(call_flops(layers[li].K, layers[li].N, M) for li, M in calls)
 
-    def one_call(rep, li, M):
-        b = replicas[rep][li]
-        pb.w4_linear(xs[(li, M)], b["qweight"], b["qzeros"], b["scales"], b["bias"], b["cs"],
-                     b["pairs"], b["theta"], GROUP, KROT, workspace=ws[(li, M)], out=ys[(li, M)],
-                     stream=stream)
+    def member(b, rotate=True):
+        return dict(qweight=b["qweight"], qzeros=b["qzeros"], scales=b["scales"], bias=b["bias"],
+                    channel_scales=b["cs"] if rotate else None, pairs=b["pairs"] if rotate else None,
+                    theta=b["theta"] if rotate else None, krot=KROT if rotate else 0)
+
+    def one_call(rep, gi, M):
+        grp = groups[gi]
+        if len(grp) == 1:
+            li = grp[0]
+            b = replicas[rep][li]
+            pb.w4_linear(xs[(li, M)], b["qweight"], b["qzeros"], b["scales"], b["bias"], b["cs"],
+                         b["pairs"], b["theta"], GROUP, KROT, workspace=ws[(gi, M)], out=ys[(li, M)],
+                         stream=stream)
+        else:
+            pb.w4_linear_group(xs[(grp[0], M)], [member(replicas[rep][li]) for li in grp], GROUP,
+                               workspace=ws[(gi, M)], out=[ys[(li, M)] for li in grp], stream=stream)
 
     def one_step(i):
-        for c, (li, M) in enumerate(calls):
-            one_call((i * len(calls) + c) % reps, li, M)
+        for c, (gi, M) in enumerate(gcalls):
+            one_call((i * len(gcalls) + c) % reps, gi, M)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -305,17 +335,26 @@ def run_ours(args, rank, world, local_rank):
     kern_bytes = 0
     kern_flops = 0
     n_launch = 0
+    # (a group's GEMV reads the first member's X_r for every member: the same
+    # bytes and work as the members' own X_r)
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g2, stream=stream):
         for i in range(args.steps):
-            for c, (li, M) in enumerate(calls):
-                b = replicas[(i * len(calls) + c) % reps][li]
-                pb.w4_linear(xrs[(li, M)], b["qweight"], b["qzeros"], b["scales"], b["bias"],
-                             None, None, None, GROUP, 0, out=ys[(li, M)], stream=stream)
-                lay = layers[li]
-                kern_bytes += gemv_bytes(lay.K, lay.N, M, lay.bias is not None)
-                kern_flops += call_flops(lay.K, lay.N, M)
-                n_launch += 1
+            for c, (gi, M) in enumerate(gcalls):
+                rep = (i * len(gcalls) + c) % reps
+                grp = groups[gi]
+                if len(grp) == 1:
+                    b = replicas[rep][grp[0]]
+                    pb.w4_linear(xrs[(grp[0], M)], b["qweight"], b["qzeros"], b["scales"], b["bias"],
+                                 None, None, None, GROUP, 0, out=ys[(grp[0], M)], stream=stream)
+                else:
+                    pb.w4_linear_group(xrs[(grp[0], M)], [member(replicas[rep][li], False) for li in grp],
+                                       GROUP, out=[ys[(li, M)] for li in grp], stream=stream)
+                for li in grp:
+                    lay = layers[li]
+                    kern_bytes += gemv_bytes(lay.K, lay.N, M, lay.bias is not None)
+                    kern_flops += call_flops(lay.K, lay.N, M)
+                n_launch += launches(gi, M, rotate=False)
     replay(g2)
     torch.cuda.synchronize(dev)
     e0.record(stream)
@@ -347,17 +386,19 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end through the public call with host buffers (pinned), per step:
     #      H2D of the step's activations, the calls, D2H of the outputs
-    hx = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    hx = {(groups[gi][0], M): xs[(groups[gi][0], M)].cpu().pin_memory() for gi, M in gcalls}
     hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in ys.items()}
     h2d = sum(v.numel() * 2 for v in hx.values())
     d2h = sum(v.numel() * 2 for v in hy.values())
     e_steps = max(1, min(args.steps, 200))
 
     def e2e_step(i):
-        for c, (li, M) in enumerate(calls):
-            xs[(li, M)].copy_(hx[(li, M)], non_blocking=True)
-            one_call((i * len(calls) + c) % reps, li, M)
-            hy[(li, M)].copy_(ys[(li, M)], non_blocking=True)
+        for c, (gi, M) in enumerate(gcalls):
+            grp = groups[gi]
+            xs[(grp[0], M)].copy_(hx[(grp[0], M)], non_blocking=True)
+            one_call((i * len(gcalls) + c) % reps, gi, M)
+            for li in grp:
+                hy[(li, M)].copy_(ys[(li, M)], non_blocking=True)
 
     with torch.cuda.stream(stream):
         for i in range(2):
@@ -394,7 +435,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_val, 2), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                 "how": "pinned host x -> device, paro_w4_linear calls, device y -> pinned host; no graph"},
-        "gpu_launches": 2 * len(calls) * args.steps,
+        "gpu_launches": sum(launches(gi, M) for gi, M in gcalls) * args.steps,
         "clocks": clocks,
         "bytes_per_step": step_bytes, "flops_per_step": step_flops,
     }

@@ -216,6 +216,10 @@ size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, cons
                                            int group_size);
 int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
                          int group_size, void* workspace, size_t workspace_bytes, paro_stream_t stream);
+/* Kernel launches paro_w4_linear_group issues for this group (rotations plus
+ * GEMV/GEMM launches; 0 for an invalid shape or M == 0).  Host-only query. */
+int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_linear* linears,
+                                  int group_size);
 
 /*
  * paro_w4_linear_noalloc — paro_w4_linear for callers that cannot allocate

@@ -26,10 +26,11 @@ from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # n
                    LIB_PATH, ParoError, check, lib, paro_device_status, paro_pack_awq,
                    paro_quantize_w4, paro_rotate, paro_status_string, paro_unpack_awq,
                    paro_validate_pairs, paro_version, paro_w4_linear, paro_w4_linear_workspace_size,
-                   PARO_MAX_GROUP, ParoLinear, paro_w4_linear_group, paro_w4_linear_group_workspace_size)
+                   PARO_MAX_GROUP, ParoLinear, paro_w4_linear_group, paro_w4_linear_group_launches,
+                   paro_w4_linear_group_workspace_size)
 
 __all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
-           "w4_linear_group", "quantize_w4", "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
+           "w4_linear_group", "w4_linear_group_launches", "quantize_w4", "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -216,3 +217,12 @@ def w4_linear_group(x: torch.Tensor, members, group_size: int = 128, workspace: 
     check(paro_w4_linear_group(_ptr(x), M, K, len(members), arr, group_size, _ptr(workspace),
                                workspace.numel(), _stream(stream)), "paro_w4_linear_group")
     return out
+
+
+def w4_linear_group_launches(M: int, K: int, members, group_size: int = 128) -> int:
+    """Kernel launches one ``w4_linear_group`` call of this shape issues."""
+    arr = (ParoLinear * len(members))()
+    for i, m in enumerate(members):
+        arr[i] = ParoLinear(m["N"], None, None, None, None,
+                            1 if m.get("channel_scales", True) else None, None, None, m.get("krot", 8), None)
+    return int(paro_w4_linear_group_launches(M, K, len(members), arr, group_size))

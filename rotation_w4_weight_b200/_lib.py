@@ -24,7 +24,7 @@ EXPORTED = (
     "paro_status_string", "paro_version", "paro_rotate", "paro_pack_awq", "paro_unpack_awq",
     "paro_w4_linear_workspace_size", "paro_w4_linear", "paro_w4_linear_noalloc",
     "paro_validate_pairs", "paro_device_status", "paro_quantize_w4",
-    "paro_w4_linear_group_workspace_size", "paro_w4_linear_group",
+    "paro_w4_linear_group_workspace_size", "paro_w4_linear_group", "paro_w4_linear_group_launches",
 )
 
 PARO_MAX_GROUP = 4
@@ -57,6 +57,7 @@ _SIGNATURES = {
     "paro_quantize_w4": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp]),
     "paro_w4_linear_group_workspace_size": (ctypes.c_size_t, [_i64, _i64, _int, _vp, _int]),
     "paro_w4_linear_group": (_int, [_vp, _i64, _i64, _int, _vp, _int, _vp, ctypes.c_size_t, _vp]),
+    "paro_w4_linear_group_launches": (_int, [_i64, _i64, _int, _vp, _int]),
 }
 
 
@@ -89,6 +90,7 @@ paro_device_status = lib.paro_device_status
 paro_quantize_w4 = lib.paro_quantize_w4
 paro_w4_linear_group_workspace_size = lib.paro_w4_linear_group_workspace_size
 paro_w4_linear_group = lib.paro_w4_linear_group
+paro_w4_linear_group_launches = lib.paro_w4_linear_group_launches
 
 
 class ParoError(RuntimeError):

@@ -680,6 +680,26 @@ size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, cons
   return total;
 }
 
+int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_linear* linears,
+                                  int group_size) {
+  if (count < 1 || count > PARO_MAX_GROUP || linears == nullptr) return 0;
+  int rot = 0;
+  bool rows_ok = M <= 16;
+  for (int i = 0; i < count; ++i) {
+    if (check_linear_shape(M, K, linears[i].N, group_size) != PARO_OK || linears[i].krot < 0 ||
+        linears[i].krot > kMaxKrot)
+      return 0;
+    if (linears[i].krot > 0 || linears[i].channel_scales != nullptr) {
+      ++rot;
+      rows_ok = rows_ok && linears[i].krot <= kRrMaxKrot;
+    }
+  }
+  if (M == 0) return 0;
+  LinearPlan gp;
+  if (count == 1 || !group_plan(M, K, linears, count, &gp)) return rot + count;
+  return (rot > 0 ? (rows_ok ? 1 : rot) : 0) + 1;
+}
+
 int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
                          int group_size, void* workspace, size_t workspace_bytes, paro_stream_t stream) {
   if (count < 1 || linears == nullptr) return PARO_ERR_INVALID_ARG;

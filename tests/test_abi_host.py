@@ -167,3 +167,14 @@ def test_group_argument_validation_and_workspace(L):
     assert g(A16, 4, 4096, 3, arr, 128, A16, 3 * per - 1, None) == L.PARO_ERR_WORKSPACE
     assert g(A16, 4, 4096, 3, arr, 128, P(0x10010), 1 << 30, None) == L.PARO_ERR_ALIGNMENT
     assert g(A16, 0, 4096, 3, arr, 128, None, 0, None) == L.PARO_OK      # empty batch
+
+
+def test_group_launch_count_query(L):
+    import rotation_w4_weight_b200 as pb
+    qkv = [dict(N=4096), dict(N=1024), dict(N=1024)]
+    n = pb.w4_linear_group_launches(1, 4096, qkv)
+    assert n in (2, 6)                        # shared launches, or one rotation + one GEMV each
+    assert pb.w4_linear_group_launches(4096, 4096, qkv) == 6            # prefill: one after another
+    assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096)]) == 2
+    assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096, krot=0, channel_scales=False)]) == 1
+    assert pb.w4_linear_group_launches(1, 4000, qkv) == 0               # invalid K
