@@ -435,6 +435,13 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_val, 2), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                 "how": "pinned host x -> device, paro_w4_linear calls, device y -> pinned host; no graph"},
+        # the same calls with krot = 0 and no channel scales are the GEMV/GEMM
+        # graph timed for the roofline: the fused path's cost over it
+        "rotation_overhead": {"frac": round(ms / kern_ms - 1.0, 4),
+                              "ms_per_step_rotated": round(ms / args.steps, 5),
+                              "ms_per_step_unrotated": round(kern_ms / args.steps, 5),
+                              "how": "same K steps as CUDA graphs; unrotated = krot 0, no channel "
+                                     "scales, same kernels on X_r"},
         "gpu_launches": sum(launches(gi, M) for gi, M in gcalls) * args.steps,
         "clocks": clocks,
         "bytes_per_step": step_bytes, "flops_per_step": step_flops,

@@ -17,6 +17,7 @@
 #include "pack.cuh"
 #include "rotate.cuh"
 #include "rotate_tmem.cuh"
+#include "rotate_tc.cuh"
 #include "w4_gemv.cuh"
 #include "w4_tc.cuh"
 
@@ -27,6 +28,9 @@ namespace {
 constexpr int kMaxDecodeM = 16;      // M <= 16: split-K GEMV path
 constexpr int kDecodeTargetCtas = 296;   // two decode CTAs per SM
 constexpr int kMaxSplits = 8;         // cluster size along K (portable maximum)
+// M >= this: paro_w4_linear rotates on the tensor cores (R' built per call into
+// the workspace); below it the tensor-memory / shared-memory / warp-per-row kernels
+constexpr int64_t kRotTcMinM = 256;
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -291,6 +295,29 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
   }
 }
 
+// Rotation as X R' on the tensor cores: one launch builds R' (fp16 parts,
+// transposed) into `rt`, a second computes X_r = X R'.
+int launch_rotate_tc(const __half* x, __half* xr, __half* rt, int64_t M, int64_t K, const float* cs,
+                     const int16_t* pairs, const float* theta, int krot, cudaStream_t stream) {
+  const DeviceInfo& di = device_info();
+  if (di.sms == 0) return PARO_ERR_CUDA;
+  const int64_t groups = K / kGroup, tiles = (M + 127) / 128;
+  if (!allow_smem(rmat_build_kernel, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
+  if (int st = launch(rmat_build_kernel, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows)), dim3(kRbThreads),
+                      rb_smem_bytes(krot), stream, true, cs, pairs, theta, rt, (int)K, krot))
+    return st;
+  CUtensorMap tmX, tmR;
+  if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tmR, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rt, 2 * K, kGroup, 128, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return PARO_ERR_CUDA;
+  if (!allow_smem(rotate_tc_kernel, RcLayout::SMEM)) return PARO_ERR_CUDA;
+  const int64_t jobs = groups * tiles;
+  const int64_t ctas = jobs < di.sms ? jobs : di.sms;
+  return launch(rotate_tc_kernel, dim3((unsigned)ctas), dim3(kRcThreads), RcLayout::SMEM, stream, true, tmX,
+                tmR, xr, (int)M, (int)K, (int)tiles, (long long)jobs);
+}
+
 // ---------------------------------------------------------------- linear plan
 struct LinearPlan {
   bool decode = false;
@@ -298,7 +325,8 @@ struct LinearPlan {
   int n_tiles = 0;         // decode column tiles
   int splits = 1;          // decode split-K factor = cluster size along K
   int variant = 0;         // decode kernel configuration (tile, k-parts, stages)
-  size_t off_xr = 0, total = 0;
+  bool rot_tc = false;     // the rotation runs on the tensor cores (R' in the workspace)
+  size_t off_xr = 0, off_rt = 0, total = 0;
 };
 
 int check_linear_shape(int64_t M, int64_t K, int64_t N, int group_size) {
@@ -321,6 +349,11 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
   p.decode = M <= kMaxDecodeM;
   p.off_xr = 0;
   p.total = round_up((size_t)M * K * 2, 256);   // X_r, written when rotating
+  if (M >= kRotTcMinM) {                          // R' parts: fp16 [2][K][128]
+    p.rot_tc = true;
+    p.off_rt = p.total;
+    p.total += (size_t)K * kGroup * 2 * 2;
+  }
   if (p.decode) {
     p.nt = M <= 8 ? 1 : 2;
     // Configuration by shape class, from sweeps on B200 over the Llama-3-8B
@@ -651,8 +684,14 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
   // rotation, or whatever preceded the call), and reads activations after.
   const bool pdl = true;
   if (rotate) {
-    __half* xr = reinterpret_cast<__half*>(static_cast<unsigned char*>(workspace) + plan.off_xr);
-    if (int st = launch_rotate(xa, xr, M, K, channel_scales, pairs, theta, krot, s)) return st;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    __half* xr = reinterpret_cast<__half*>(ws + plan.off_xr);
+    if (plan.rot_tc) {
+      __half* rt = reinterpret_cast<__half*>(ws + plan.off_rt);
+      if (int st = launch_rotate_tc(xa, xr, rt, M, K, channel_scales, pairs, theta, krot, s)) return st;
+    } else if (int st = launch_rotate(xa, xr, M, K, channel_scales, pairs, theta, krot, s)) {
+      return st;
+    }
     xa = xr;
   }
 
@@ -696,7 +735,10 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
   }
   if (M == 0) return 0;
   LinearPlan gp;
-  if (count == 1 || !group_plan(M, K, linears, count, &gp)) return rot + count;
+  // one after another: each rotating member launches its rotation (two
+  // kernels on the tensor-core path) and its GEMV / GEMM
+  if (count == 1 || !group_plan(M, K, linears, count, &gp))
+    return rot * (make_plan(M, K, linears[0].N).rot_tc ? 2 : 1) + count;
   return (rot > 0 ? (rows_ok ? 1 : rot) : 0) + 1;
 }
 

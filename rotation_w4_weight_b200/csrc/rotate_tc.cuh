@@ -1,0 +1,337 @@
+// Channel scaling + krot Givens stages on the tensor cores (sm_100a), for
+// large token counts.
+//
+// The stages of one 128-channel group are a fixed linear map of the group's
+// channels (GPTQModel wiki page "ParoQuant", "Activation and weight
+// transforms": X_r = X D^-1 R; "Pairwise Givens rotations": a' = a cos t +
+// b sin t, b' = -a sin t + b cos t, stages in order, pair indices local to the
+// group).  With the channel scale folded in, every token row x of group g
+// becomes x R'_g with
+//     R'_g = diag(cs_g) G_0 G_1 ... G_{krot-1}      (128 x 128, fp32),
+// and row k of R'_g is the basis vector e_k, scaled by cs[k] and taken through
+// the stages exactly as a token row would be.  So:
+//   1. rmat_build_kernel rotates the 128 scaled basis rows of every group in
+//      fp32 (the same per-pair arithmetic as the other rotation kernels) and
+//      stores R'_g transposed, split into two fp16 parts
+//      R'_g = Rhi + Rlo, Rlo = fp16(R'_g - Rhi);
+//   2. rotate_tc_kernel computes the block-diagonal product X R' on the
+//      tensor cores, X Rhi + X Rlo accumulated in fp32 in tensor memory, and
+//      rounds X_r to fp16 once.
+// X is fp16 and exact as an MMA operand, and Rhi + Rlo carries R' to about
+// 2^-22 relative, so the result is the fp32 rotation up to summation order.
+// The cost no longer grows with krot: 2 * 2 * M * 128 * K flops (two fp16
+// products) against 4 * M * K bytes of HBM traffic, about 4.4 GFLOP per
+// 16 MB of activations moved -- under the time the bytes take at HBM speed.
+//
+// Layout of the transposed parts in global memory: fp16 [2][K][128]; part 0 is
+// Rhi, part 1 is Rlo; row g*128 + n, column k holds R'_g[k][n], i.e. each
+// 128-row block is the K-major B operand (N = output channel, K = input
+// channel) of one group.
+#pragma once
+
+#include "rotate.cuh"
+
+namespace paro {
+
+// ------------------------------------------------------------------ R' build
+constexpr int kRbRows = 32;               // basis rows per CTA (4 CTAs per group)
+constexpr int kRbThreads = 256;           // (row, one eighth of the pairs) per thread
+constexpr int kRbPitch = 129;             // fp32 words per row in shared memory
+
+__host__ __device__ constexpr size_t rb_smem_bytes(int krot) {
+  return (size_t)krot * (kGroup / 2) * sizeof(RotParam) + (size_t)kRbRows * kRbPitch * 4;
+}
+
+// grid (K/128, 128/kRbRows), block kRbThreads.  rt: fp16 [2][K][128] (above).
+__global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(
+    const float* __restrict__ cs, const int16_t* __restrict__ pairs,
+    const float* __restrict__ theta, __half* __restrict__ rt, int K, int krot) {
+  // The rotation that follows waits for this kernel's completion; let it
+  // launch and set itself up meanwhile.
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  RotParam* prm = reinterpret_cast<RotParam*>(smem_raw);
+  float* v = reinterpret_cast<float*>(smem_raw + (size_t)krot * (kGroup / 2) * sizeof(RotParam));
+  const int grp = blockIdx.x, r0 = blockIdx.y * kRbRows, tid = threadIdx.x;
+
+  // stage tables of the group (layer constants: read before waiting for the
+  // kernel ahead); indices outside the group are masked and flagged
+  load_rot_params(prm, pairs, theta, K, krot, grp, tid, kRbThreads);
+  // basis rows r0 .. r0+31, scaled: row r has cs[r0 + r] at channel r0 + r
+  for (int idx = tid; idx < kRbRows * kGroup; idx += kRbThreads) {
+    const int r = idx >> 7, c = idx & (kGroup - 1);
+    float val = 0.0f;
+    if (c == r0 + r) val = cs != nullptr ? cs[(size_t)grp * kGroup + c] : 1.0f;
+    v[r * kRbPitch + c] = val;
+  }
+  __syncthreads();
+
+  // stages: thread (row r, part) applies pairs 8 part .. 8 part + 7 of every
+  // stage to its row; a stage's pairs are disjoint, so the parts of a row
+  // never touch the same channel within a stage
+  {
+    const int r = tid >> 3, part = tid & 7;
+    float* row = v + r * kRbPitch;
+    for (int s = 0; s < krot; ++s) {
+      const RotParam* ps = prm + s * (kGroup / 2) + part * 8;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const RotParam p = ps[q];
+        const float a = row[p.i];
+        const float b = row[p.j];
+        row[p.i] = fmaf(a, p.c, b * p.s);
+        row[p.j] = fmaf(b, p.c, -(a * p.s));
+      }
+      __syncthreads();
+    }
+  }
+
+  // The parts go into the caller's workspace, which the kernel ahead may
+  // still be using.
+  pdl_wait_primary();
+  // thread (n, h): output channel n, basis rows r0 + 16h .. r0 + 16h + 15
+  // (32 contiguous bytes of row g*128 + n of each part)
+  const int n = tid & (kGroup - 1), h = tid >> 7;
+  uint32_t hi[8], lo[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float a = v[(16 * h + 2 * e) * kRbPitch + n];
+    const float b = v[(16 * h + 2 * e + 1) * kRbPitch + n];
+    const __half ah = __float2half_rn(a), bh = __float2half_rn(b);
+    const __half al = __float2half_rn(a - __half2float(ah));
+    const __half bl = __float2half_rn(b - __half2float(bh));
+    const __half2 ph = __halves2half2(ah, bh), pl = __halves2half2(al, bl);
+    hi[e] = *reinterpret_cast<const uint32_t*>(&ph);
+    lo[e] = *reinterpret_cast<const uint32_t*>(&pl);
+  }
+  __half* dst = rt + ((size_t)grp * kGroup + n) * kGroup + r0 + 16 * h;
+  uint4* dh = reinterpret_cast<uint4*>(dst);
+  uint4* dl = reinterpret_cast<uint4*>(dst + (size_t)K * kGroup);
+  dh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  dh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+  dl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  dl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+}
+
+// ------------------------------------------------------------------ X R'
+// Work: jobs (group g, 128-row tile t), group-major; CTA c of P (one per SM)
+// takes the contiguous range [c J / P, (c+1) J / P), so every CTA moves the
+// same number of tiles and holds one group's R' at a time (a range crosses a
+// group boundary at most a few times; R' is reloaded there).
+//
+// Warp roles: warp 0 = TMA producer (R' parts, x tiles through a
+// kRcStages-deep ring), warp 1 = TMEM allocator and single-thread MMA issuer,
+// warps 2..5 = epilogue (warp w reads TMEM lane quadrant w % 4: rows
+// 32 (w % 4) .. +31 of the tile).
+//   A = x tile [128 rows][128 channels] fp16: two {64 channels, 128 rows}
+//       boxes with the 128-byte swizzle (canonical K-major SW128 layout).
+//   B = Rhi, Rlo of the group [128 n][128 k]: two boxes each, same layout.
+//   D = fp32 [128 lanes = rows][128 columns = output channels], two buffers
+//       (256 TMEM columns) so the epilogue of one tile overlaps the MMAs of
+//       the next.
+// Per tile: 8 k-steps of 16 channels, each one MMA with Rhi and one with Rlo
+// into the same accumulator (M = 128, N = 128, K = 16, kind::f16).
+constexpr int kRcStages = 4;
+constexpr int kRcEpiWarps = 4;
+constexpr int kRcThreads = 32 * (2 + kRcEpiWarps);
+constexpr int kRcCols = 256;
+
+struct RcLayout {
+  static constexpr int BOX = 128 * 64 * 2;                 // 16 KB
+  static constexpr int R_OFF = 0;                          // Rhi 0, Rhi 1, Rlo 0, Rlo 1
+  static constexpr int X_OFF = 4 * BOX;
+  static constexpr int X_STAGE = 2 * BOX;
+  static constexpr int BAR_OFF = X_OFF + kRcStages * X_STAGE;
+  // x_full[S], x_empty[S], acc_full[2], acc_empty[2], r_full, r_free, mma_done
+  static constexpr int NBARS = 2 * kRcStages + 7;
+  static constexpr int MISC_OFF = BAR_OFF + 8 * NBARS;     // TMEM address, abort flag
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;        // + slack for 1024-byte alignment
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+// instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M = 128, N = 128
+constexpr uint32_t kRcIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+// 32 fp32 accumulator columns of one row -> 32 fp16 (round to nearest) at dst.
+__device__ __forceinline__ void rc_store32(uint4* dst, const uint32_t (&r)[32]) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    uint4 o;
+    __half2* oh = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      oh[e] = __floats2half2_rn(__uint_as_float(r[8 * v + 2 * e]), __uint_as_float(r[8 * v + 2 * e + 1]));
+    dst[v] = o;
+  }
+}
+
+// grid P <= number of SMs, block kRcThreads.  tmX: x [M, K] fp16, box {64, 128},
+// 128-byte swizzle.  tmR: the parts as [2K, 128] fp16, same box and swizzle.
+__global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR,
+    __half* __restrict__ xr, int M, int K, int tiles, long long jobs) {
+  using L = RcLayout;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t base = smem_u32(sbase);
+  const uint32_t x_full0 = base + L::BAR_OFF;
+  const uint32_t x_empty0 = x_full0 + 8 * kRcStages;
+  const uint32_t acc_full0 = x_empty0 + 8 * kRcStages;
+  const uint32_t acc_empty0 = acc_full0 + 16;
+  const uint32_t r_full = acc_empty0 + 16;
+  const uint32_t r_free = r_full + 8;
+  const uint32_t mma_done = r_free + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::MISC_OFF);
+  volatile int* abort = reinterpret_cast<volatile int*>(sbase + L::MISC_OFF + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long P = gridDim.x, c = blockIdx.x;
+  const long long j0 = c * jobs / P, j1 = (c + 1) * jobs / P;
+  const int nj = (int)(j1 - j0);
+
+  if (tid == 0) {
+    for (int s = 0; s < kRcStages; ++s) {
+      mbar_init(x_full0 + 8 * s, 1);
+      mbar_init(x_empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(acc_full0 + 8 * a, 1);
+      mbar_init(acc_empty0 + 8 * a, kRcEpiWarps);
+    }
+    mbar_init(r_full, 1);
+    mbar_init(r_free, 1);
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmR);
+  }
+  if (warp == 1) {                         // the whole warp allocates the two accumulators
+    tmem_alloc(smem_u32(tmem_slot), kRcCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // tensor memory is held: a dependent kernel may launch now without ever
+  // taking columns this one still needs
+  pdl_launch_dependents();
+  const uint32_t tmem0 = *tmem_slot;
+  // R' comes from the build kernel, x from the kernel before it (the build
+  // kernel completes only after that one has)
+  pdl_wait_primary();
+
+  int issued = 0, r_loads = 0;             // producer's count of x tiles and R' loads
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int cur_g = -1;
+      for (int i = 0; i < nj; ++i) {
+        const long long j = j0 + i;
+        const int g = (int)(j / tiles), t = (int)(j % tiles);
+        if (g != cur_g) {
+          // every MMA that reads the previous group's R' has completed
+          if (r_loads > 0 && !tc_wait(r_free, (uint32_t)((r_loads - 1) & 1), abort)) break;
+          mbar_arrive_expect_tx(r_full, 4 * L::BOX);
+          tma_load_2d(base + L::R_OFF + 0 * L::BOX, &tmR, r_full, 0, g * 128);
+          tma_load_2d(base + L::R_OFF + 1 * L::BOX, &tmR, r_full, 64, g * 128);
+          tma_load_2d(base + L::R_OFF + 2 * L::BOX, &tmR, r_full, 0, K + g * 128);
+          tma_load_2d(base + L::R_OFF + 3 * L::BOX, &tmR, r_full, 64, K + g * 128);
+          ++r_loads;
+          cur_g = g;
+        }
+        const int s = i % kRcStages;
+        if (i >= kRcStages && !tc_wait(x_empty0 + 8 * s, (uint32_t)(((i / kRcStages) - 1) & 1), abort)) break;
+        const uint32_t dst = base + L::X_OFF + s * L::X_STAGE;
+        mbar_arrive_expect_tx(x_full0 + 8 * s, L::X_STAGE);
+        tma_load_2d(dst, &tmX, x_full0 + 8 * s, g * 128, t * 128);
+        tma_load_2d(dst + L::BOX, &tmX, x_full0 + 8 * s, g * 128 + 64, t * 128);
+        ++issued;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int cur_g = -1, gi = -1;
+      for (int i = 0; i < nj; ++i) {
+        const long long j = j0 + i;
+        const int g = (int)(j / tiles);
+        if (g != cur_g) {
+          ++gi;
+          cur_g = g;
+          if (!tc_wait(r_full, (uint32_t)(gi & 1), abort)) break;
+        }
+        const int s = i % kRcStages, a = i & 1;
+        if (!tc_wait(x_full0 + 8 * s, (uint32_t)((i / kRcStages) & 1), abort)) break;
+        if (i >= 2 && !tc_wait(acc_empty0 + 8 * a, (uint32_t)(((i >> 1) - 1) & 1), abort)) break;
+        tc_fence_after();
+        const uint32_t d = tmem0 + (uint32_t)(a * 128);
+        const uint32_t xs = base + L::X_OFF + s * L::X_STAGE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          // 128-byte swizzled rows, 8-row groups 1024 B apart; +32 B per 16 channels
+          const uint32_t box = (uint32_t)(ks >> 2) * L::BOX, off = (uint32_t)(ks & 3) * 32;
+          const uint64_t ad = umma_desc(xs + box + off, 16, 1024, 2);
+          const uint64_t bh = umma_desc(base + L::R_OFF + box + off, 16, 1024, 2);
+          const uint64_t bl = umma_desc(base + L::R_OFF + 2 * L::BOX + box + off, 16, 1024, 2);
+          umma_f16(d, ad, bh, kRcIdesc, ks > 0 ? 1u : 0u);
+          umma_f16(d, ad, bl, kRcIdesc, 1u);
+        }
+        umma_commit(x_empty0 + 8 * s);    // the x stage and ...
+        umma_commit(acc_full0 + 8 * a);   // ... the accumulator, once these MMAs finish
+        if (i + 1 == nj || (j + 1) / tiles != g) umma_commit(r_free);   // last tile of the group
+      }
+      // every MMA issued here has completed before tensor memory is released
+      umma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                // TMEM lane quadrant of this warp
+    for (int i = 0; i < nj; ++i) {
+      const long long j = j0 + i;
+      const int g = (int)(j / tiles), t = (int)(j % tiles);
+      const int a = i & 1;
+      if (!tc_wait(acc_full0 + 8 * a, (uint32_t)((i >> 1) & 1), abort)) break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      const uint32_t ta = tmem0 + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128);
+      tmem_ld32(ta, r0);
+      tmem_ld32(ta + 32, r1);
+      tmem_ld32(ta + 64, r2);
+      tmem_ld32(ta + 96, r3);
+      tmem_ld_wait_tie(r0);
+      tmem_tie(r1);
+      tmem_tie(r2);
+      tmem_tie(r3);
+      // the accumulator may be overwritten once every warp has read it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty0 + 8 * a);
+      const int row = t * 128 + 32 * q + lane;
+      if (row < M) {
+        uint4* dst = reinterpret_cast<uint4*>(xr + (size_t)row * K + (size_t)g * 128);
+        rc_store32(dst, r0);
+        rc_store32(dst + 4, r1);
+        rc_store32(dst + 8, r2);
+        rc_store32(dst + 12, r3);
+      }
+    }
+  }
+
+  if (warp == 0 && lane == 0 && *abort) {
+    // a wait gave up: let this thread's copies still in flight land (bounded)
+    // before the shared memory is released
+    for (int i = issued > kRcStages ? issued - kRcStages : 0; i < issued; ++i)
+      if (!mbar_wait_bounded(x_full0 + 8 * (i % kRcStages), (uint32_t)((i / kRcStages) & 1))) break;
+    if (r_loads > 0) mbar_wait_bounded(r_full, (uint32_t)((r_loads - 1) & 1));
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem0, kRcCols);
+  }
+}
+
+}  // namespace paro

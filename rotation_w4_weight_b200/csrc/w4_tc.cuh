@@ -77,21 +77,6 @@ struct TcLayout {
 // instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M=128, N=256
 constexpr uint32_t kTcIdesc = (1u << 4) | ((uint32_t)(kTcBN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
 
-// Bounded wait that also gives up as soon as another role of the CTA has given up.
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      flag_error(kErrTimeout);
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
 __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
