@@ -306,16 +306,17 @@ int launch_rotate_tc(const __half* x, __half* xr, __half* rt, int64_t M, int64_t
   if (int st = launch(rmat_build_kernel, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows)), dim3(kRbThreads),
                       rb_smem_bytes(krot), stream, true, cs, pairs, theta, rt, (int)K, krot))
     return st;
-  CUtensorMap tmX, tmR;
+  CUtensorMap tmX, tmR, tmY;
   if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&tmR, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rt, 2 * K, kGroup, 128, 64,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xr, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return PARO_ERR_CUDA;
   if (!allow_smem(rotate_tc_kernel, RcLayout::SMEM)) return PARO_ERR_CUDA;
   const int64_t jobs = groups * tiles;
   const int64_t ctas = jobs < di.sms ? jobs : di.sms;
   return launch(rotate_tc_kernel, dim3((unsigned)ctas), dim3(kRcThreads), RcLayout::SMEM, stream, true, tmX,
-                tmR, xr, (int)M, (int)K, (int)tiles, (long long)jobs);
+                tmR, tmY, (int)K, (int)tiles, (long long)jobs);
 }
 
 // ---------------------------------------------------------------- linear plan

@@ -34,9 +34,9 @@
 namespace paro {
 
 // ------------------------------------------------------------------ R' build
-constexpr int kRbRows = 32;               // basis rows per CTA (4 CTAs per group)
-constexpr int kRbThreads = 256;           // (row, one eighth of the pairs) per thread
-constexpr int kRbPitch = 129;             // fp32 words per row in shared memory
+constexpr int kRbRows = 32;               // basis rows per CTA (4 CTAs per group), one per lane
+constexpr int kRbThreads = 256;           // warp w applies pairs 8w .. 8w+7 of every stage
+constexpr int kRbPitch = 129;             // fp32 words per row: lanes (rows) hit distinct banks
 
 __host__ __device__ constexpr size_t rb_smem_bytes(int krot) {
   return (size_t)krot * (kGroup / 2) * sizeof(RotParam) + (size_t)kRbRows * kRbPitch * 4;
@@ -51,8 +51,9 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(
   pdl_launch_dependents();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RotParam* prm = reinterpret_cast<RotParam*>(smem_raw);
-  float* v = reinterpret_cast<float*>(smem_raw + (size_t)krot * (kGroup / 2) * sizeof(RotParam));
+  const uint32_t vbase = smem_u32(smem_raw + (size_t)krot * (kGroup / 2) * sizeof(RotParam));
   const int grp = blockIdx.x, r0 = blockIdx.y * kRbRows, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
 
   // stage tables of the group (layer constants: read before waiting for the
   // kernel ahead); indices outside the group are masked and flagged
@@ -62,28 +63,31 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(
     const int r = idx >> 7, c = idx & (kGroup - 1);
     float val = 0.0f;
     if (c == r0 + r) val = cs != nullptr ? cs[(size_t)grp * kGroup + c] : 1.0f;
-    v[r * kRbPitch + c] = val;
+    sts_f32(vbase + (uint32_t)(r * kRbPitch + c) * 4u, val);
   }
   __syncthreads();
 
-  // stages: thread (row r, part) applies pairs 8 part .. 8 part + 7 of every
-  // stage to its row; a stage's pairs are disjoint, so the parts of a row
-  // never touch the same channel within a stage
-  {
-    const int r = tid >> 3, part = tid & 7;
-    float* row = v + r * kRbPitch;
-    for (int s = 0; s < krot; ++s) {
-      const RotParam* ps = prm + s * (kGroup / 2) + part * 8;
+  // stages: lane = basis row, warp = its eight pairs of the stage.  The pairs
+  // of a stage are disjoint, so all sixteen operands are loaded before any
+  // result is stored, and the warps of a stage never touch the same channel.
+  const uint32_t row = vbase + (uint32_t)(lane * kRbPitch) * 4u;
+  for (int s = 0; s < krot; ++s) {
+    const RotParam* ps = prm + s * (kGroup / 2) + warp * 8;
+    RotParam p[8];
+    float a[8], b[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const RotParam p = ps[q];
-        const float a = row[p.i];
-        const float b = row[p.j];
-        row[p.i] = fmaf(a, p.c, b * p.s);
-        row[p.j] = fmaf(b, p.c, -(a * p.s));
-      }
-      __syncthreads();
+    for (int q = 0; q < 8; ++q) p[q] = ps[q];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      a[q] = lds_f32(row + (uint32_t)p[q].i * 4u);
+      b[q] = lds_f32(row + (uint32_t)p[q].j * 4u);
     }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      sts_f32(row + (uint32_t)p[q].i * 4u, fmaf(a[q], p[q].c, b[q] * p[q].s));
+      sts_f32(row + (uint32_t)p[q].j * 4u, fmaf(b[q], p[q].c, -(a[q] * p[q].s)));
+    }
+    __syncthreads();
   }
 
   // The parts go into the caller's workspace, which the kernel ahead may
@@ -95,11 +99,11 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(
   uint32_t hi[8], lo[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    const float a = v[(16 * h + 2 * e) * kRbPitch + n];
-    const float b = v[(16 * h + 2 * e + 1) * kRbPitch + n];
-    const __half ah = __float2half_rn(a), bh = __float2half_rn(b);
-    const __half al = __float2half_rn(a - __half2float(ah));
-    const __half bl = __float2half_rn(b - __half2float(bh));
+    const float va = lds_f32(vbase + (uint32_t)((16 * h + 2 * e) * kRbPitch + n) * 4u);
+    const float vb = lds_f32(vbase + (uint32_t)((16 * h + 2 * e + 1) * kRbPitch + n) * 4u);
+    const __half ah = __float2half_rn(va), bh = __float2half_rn(vb);
+    const __half al = __float2half_rn(va - __half2float(ah));
+    const __half bl = __float2half_rn(vb - __half2float(bh));
     const __half2 ph = __halves2half2(ah, bh), pl = __halves2half2(al, bl);
     hi[e] = *reinterpret_cast<const uint32_t*>(&ph);
     lo[e] = *reinterpret_cast<const uint32_t*>(&pl);
@@ -122,7 +126,10 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(
 // Warp roles: warp 0 = TMA producer (R' parts, x tiles through a
 // kRcStages-deep ring), warp 1 = TMEM allocator and single-thread MMA issuer,
 // warps 2..5 = epilogue (warp w reads TMEM lane quadrant w % 4: rows
-// 32 (w % 4) .. +31 of the tile).
+// 32 (w % 4) .. +31 of the tile).  The epilogue rounds its rows to fp16 into a
+// staging tile in shared memory (two boxes, 128-byte swizzle) and one thread
+// writes the tile to X_r with two TMA stores (clipped at row M), so every
+// global write is a full line; two staging tiles alternate.
 //   A = x tile [128 rows][128 channels] fp16: two {64 channels, 128 rows}
 //       boxes with the 128-byte swizzle (canonical K-major SW128 layout).
 //   B = Rhi, Rlo of the group [128 n][128 k]: two boxes each, same layout.
@@ -131,7 +138,7 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(
 //       the next.
 // Per tile: 8 k-steps of 16 channels, each one MMA with Rhi and one with Rlo
 // into the same accumulator (M = 128, N = 128, K = 16, kind::f16).
-constexpr int kRcStages = 4;
+constexpr int kRcStages = 3;
 constexpr int kRcEpiWarps = 4;
 constexpr int kRcThreads = 32 * (2 + kRcEpiWarps);
 constexpr int kRcCols = 256;
@@ -141,7 +148,9 @@ struct RcLayout {
   static constexpr int R_OFF = 0;                          // Rhi 0, Rhi 1, Rlo 0, Rlo 1
   static constexpr int X_OFF = 4 * BOX;
   static constexpr int X_STAGE = 2 * BOX;
-  static constexpr int BAR_OFF = X_OFF + kRcStages * X_STAGE;
+  static constexpr int O_OFF = X_OFF + kRcStages * X_STAGE;  // staging tiles [2]
+  static constexpr int O_STAGE = 2 * BOX;
+  static constexpr int BAR_OFF = O_OFF + 2 * O_STAGE;
   // x_full[S], x_empty[S], acc_full[2], acc_empty[2], r_full, r_free, mma_done
   static constexpr int NBARS = 2 * kRcStages + 7;
   static constexpr int MISC_OFF = BAR_OFF + 8 * NBARS;     // TMEM address, abort flag
@@ -152,24 +161,30 @@ struct RcLayout {
 // instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M = 128, N = 128
 constexpr uint32_t kRcIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
-// 32 fp32 accumulator columns of one row -> 32 fp16 (round to nearest) at dst.
-__device__ __forceinline__ void rc_store32(uint4* dst, const uint32_t (&r)[32]) {
+// 32 fp32 accumulator columns (chunk cb of 4) of tile row r -> fp16 (round to
+// nearest) in the staging tile: 64-channel box cb / 2, 16-byte chunks
+// 4 (cb % 2) .. +3 of the row, XOR-swizzled by (r & 7) as the 128-byte TMA
+// swizzle expects.
+__device__ __forceinline__ void rc_stage32(uint32_t tile, int r, int cb, const uint32_t (&v)[32]) {
+  const uint32_t rowp = tile + (uint32_t)(cb >> 1) * RcLayout::BOX + (uint32_t)r * 128u;
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
+  for (int c = 0; c < 4; ++c) {
     uint4 o;
     __half2* oh = reinterpret_cast<__half2*>(&o);
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      oh[e] = __floats2half2_rn(__uint_as_float(r[8 * v + 2 * e]), __uint_as_float(r[8 * v + 2 * e + 1]));
-    dst[v] = o;
+      oh[e] = __floats2half2_rn(__uint_as_float(v[8 * c + 2 * e]), __uint_as_float(v[8 * c + 2 * e + 1]));
+    const uint32_t chunk = (uint32_t)(4 * (cb & 1) + c);
+    sts128u(rowp + ((chunk ^ (uint32_t)(r & 7)) << 4), o);
   }
 }
 
 // grid P <= number of SMs, block kRcThreads.  tmX: x [M, K] fp16, box {64, 128},
-// 128-byte swizzle.  tmR: the parts as [2K, 128] fp16, same box and swizzle.
+// 128-byte swizzle; tmY: X_r, same shape, box and swizzle (stores).  tmR: the
+// parts as [2K, 128] fp16, same box and swizzle.
 __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR,
-    __half* __restrict__ xr, int M, int K, int tiles, long long jobs) {
+    const __grid_constant__ CUtensorMap tmY, int K, int tiles, long long jobs) {
   using L = RcLayout;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -205,6 +220,7 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
     fence_barrier_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmR);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {                         // the whole warp allocates the two accumulators
     tmem_alloc(smem_u32(tmem_slot), kRcCols);
@@ -288,35 +304,54 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                // TMEM lane quadrant of this warp
+    const int r = 32 * q + lane;           // tile row of this thread
+    const bool leader = warp == 2 && lane == 0;   // issues the TMA stores
+    // All four warps take part in both named barriers of every tile, even
+    // after a wait has given up (the work is skipped, the barriers are not),
+    // so no warp can be left at a barrier; a given-up wait returns at once.
     for (int i = 0; i < nj; ++i) {
       const long long j = j0 + i;
       const int g = (int)(j / tiles), t = (int)(j % tiles);
       const int a = i & 1;
-      if (!tc_wait(acc_full0 + 8 * a, (uint32_t)((i >> 1) & 1), abort)) break;
-      tc_fence_after();
-      uint32_t r0[32], r1[32], r2[32], r3[32];
-      const uint32_t ta = tmem0 + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128);
-      tmem_ld32(ta, r0);
-      tmem_ld32(ta + 32, r1);
-      tmem_ld32(ta + 64, r2);
-      tmem_ld32(ta + 96, r3);
-      tmem_ld_wait_tie(r0);
-      tmem_tie(r1);
-      tmem_tie(r2);
-      tmem_tie(r3);
+      // warp-uniform (tcgen05.ld is a warp-wide instruction)
+      const bool ok = __all_sync(0xffffffffu, tc_wait(acc_full0 + 8 * a, (uint32_t)((i >> 1) & 1), abort));
+      uint32_t v0[32], v1[32], v2[32], v3[32];
+      if (ok) {
+        tc_fence_after();
+        const uint32_t ta = tmem0 + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128);
+        tmem_ld32(ta, v0);
+        tmem_ld32(ta + 32, v1);
+        tmem_ld32(ta + 64, v2);
+        tmem_ld32(ta + 96, v3);
+        tmem_ld_wait_tie(v0);
+        tmem_tie(v1);
+        tmem_tie(v2);
+        tmem_tie(v3);
+      }
       // the accumulator may be overwritten once every warp has read it
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty0 + 8 * a);
-      const int row = t * 128 + 32 * q + lane;
-      if (row < M) {
-        uint4* dst = reinterpret_cast<uint4*>(xr + (size_t)row * K + (size_t)g * 128);
-        rc_store32(dst, r0);
-        rc_store32(dst + 4, r1);
-        rc_store32(dst + 8, r2);
-        rc_store32(dst + 12, r3);
+      if (lane == 0 && ok) mbar_arrive(acc_empty0 + 8 * a);
+      // staging tile i & 1 is free once the stores of tile i - 2 have read it
+      if (leader) bulk_wait_group_read<1>();
+      named_bar_sync(1, 32 * kRcEpiWarps);
+      const uint32_t tile = base + L::O_OFF + (uint32_t)(i & 1) * L::O_STAGE;
+      if (ok) {
+        rc_stage32(tile, r, 0, v0);
+        rc_stage32(tile, r, 1, v1);
+        rc_stage32(tile, r, 2, v2);
+        rc_stage32(tile, r, 3, v3);
+      }
+      fence_proxy_async_smem();            // the tile is read by the TMA (async proxy)
+      named_bar_sync(2, 32 * kRcEpiWarps);
+      if (leader && !*abort) {
+        tma_store_2d(&tmY, tile, g * 128, t * 128);
+        tma_store_2d(&tmY, tile + L::BOX, g * 128 + 64, t * 128);
+        bulk_commit_group();
       }
     }
+    // the stores have written X_r before the kernel completes
+    if (leader) bulk_wait_group_all();
   }
 
   if (warp == 0 && lane == 0 && *abort) {
