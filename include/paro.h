@@ -174,12 +174,12 @@ size_t paro_w4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int group_
  *   used by two calls that can run at the same time.  After a call that rotates
  *   (krot > 0 or channel_scales != NULL) has completed, the first M*K*2 bytes of
  *   the workspace hold X_r (fp16 [M, K], row-major) until the workspace is used
- *   again; from M >= 256 the next 2*K*128*2 bytes hold the rotation matrices
+ *   again; from M >= 65 the next 2*K*128*2 bytes hold the rotation matrices
  *   (below), the rest is scratch.
  *   Arithmetic: rotation in fp32 rounded once to fp16; weights (q - z) exact in
  *   fp16; products and sums in fp32 (tensor cores); y rounded once to fp16.
  *   M <= 16 runs the decode GEMV path; larger M the tcgen05 prefill GEMM path.
- *   From M >= 256 the rotation itself runs on the tensor cores: each group's
+ *   From M >= 65 the rotation itself runs on the tensor cores: each group's
  *   stages with its channel scales are the 128 x 128 matrix
  *   R' = diag(cs) G_0 ... G_{krot-1}, built per call in fp32 (its 128 basis rows
  *   taken through the stages) and stored as two fp16 parts R' = Rhi + Rlo;
@@ -248,7 +248,7 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
  * no cudaMalloc, cudaFree or allocating library routine.
  *   - Limit: paro_w4_linear_workspace_size(M, K, N, group_size) must not exceed
  *     PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES (8 MiB: M*K <= 4 Mi fp16 elements
- *     below 256 rows; from 256 rows up M*K*2 + 512*K bytes, e.g. M <= 768 at
+ *     up to 64 rows; above 64 rows M*K*2 + 512*K bytes, e.g. M <= 768 at
  *     K = 4096); larger shapes return PARO_ERR_WORKSPACE before any GPU work.
  *   - The first call on a device looks up the array's device address for that
  *     device (cudaGetSymbolAddress) and caches it; make that first call before

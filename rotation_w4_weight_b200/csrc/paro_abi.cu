@@ -29,8 +29,9 @@ constexpr int kMaxDecodeM = 16;      // M <= 16: split-K GEMV path
 constexpr int kDecodeTargetCtas = 296;   // two decode CTAs per SM
 constexpr int kMaxSplits = 8;         // cluster size along K (portable maximum)
 // M >= this: paro_w4_linear rotates on the tensor cores (R' built per call into
-// the workspace); below it the tensor-memory / shared-memory / warp-per-row kernels
-constexpr int64_t kRotTcMinM = 256;
+// the workspace; measured faster than the pair-by-pair tensor-memory kernel from
+// one 128-row tile up); below it the shared-memory / warp-per-row kernels
+constexpr int64_t kRotTcMinM = 65;
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

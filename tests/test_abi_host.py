@@ -87,9 +87,9 @@ def test_workspace_size_query(L):
         v = f(M, 4096, 4096, 128)
         assert v % 256 == 0 and v >= M * 4096 * 2
     assert f(8192, 4096, 14336, 128) >= 8192 * 4096 * 2
-    # from 256 rows up the rotation's R' parts (fp16 [2][K][128]) follow X_r
-    assert f(256, 4096, 4096, 128) == 256 * 4096 * 2 + 2 * 4096 * 128 * 2
-    assert f(255, 4096, 4096, 128) == 255 * 4096 * 2
+    # above 64 rows the rotation's R' parts (fp16 [2][K][128]) follow X_r
+    assert f(65, 4096, 4096, 128) == 65 * 4096 * 2 + 2 * 4096 * 128 * 2
+    assert f(64, 4096, 4096, 128) == 64 * 4096 * 2
 
 
 def test_rotate_argument_validation(L):
@@ -178,9 +178,10 @@ def test_group_launch_count_query(L):
     n = pb.w4_linear_group_launches(1, 4096, qkv)
     assert n in (2, 6)                        # shared launches, or one rotation + one GEMV each
     # prefill, one member after another: the tensor-core rotation is two launches
-    # (R' build, X R') from 256 rows up, one below; then the GEMM
+    # (R' build, X R') above 64 rows, one below; then the GEMM
     assert pb.w4_linear_group_launches(4096, 4096, qkv) == 9
-    assert pb.w4_linear_group_launches(200, 4096, qkv) == 6
+    assert pb.w4_linear_group_launches(65, 4096, qkv) == 9
+    assert pb.w4_linear_group_launches(64, 4096, qkv) == 6
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096)]) == 2
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096, krot=0, channel_scales=False)]) == 1
     assert pb.w4_linear_group_launches(1, 4000, qkv) == 0               # invalid K

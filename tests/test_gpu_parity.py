@@ -271,3 +271,16 @@ def test_config4_layer_set_decode_and_prefill():
     for lay in synth.config_layers(4):
         for M in synth.CONFIG_M[4]:
             sampled_check(lay, M, ncols=32)
+
+
+# Prefill GEMM grids of more 256 x 256 tiles than SMs (several waves), full
+# outputs against the oracle; K = 128 gives two k-blocks per tile (fewer than
+# the dequantised-weight ring holds).
+@pytest.mark.parametrize("M,K,N", [(600, 256, 14336), (1024, 128, 14336), (1300, 256, 14336)])
+def test_linear_prefill_several_tiles_per_cta(M, K, N):
+    lay = synth.make_layer("s", K, N, seed=M + K, bias_std=0.01, zero_point=None, n_outliers=2)
+    d = layer_to_device(lay)
+    x = synth.make_activations(lay, M)
+    got = run_linear(lay, d, x).cpu().numpy().astype(np.float64)
+    ref = oracle_linear(lay, x)
+    assert lin_err(got, ref) <= LIN_TOL

@@ -1,5 +1,5 @@
-"""GPU parity of the tensor-core rotation that paro_w4_linear uses from 256
-token rows up: R' = diag(cs) G_0 ... G_{krot-1} built per group, then
+"""GPU parity of the tensor-core rotation that paro_w4_linear uses above 64
+token rows: R' = diag(cs) G_0 ... G_{krot-1} built per group, then
 X_r = X R' on the tensor cores.  X_r is read back from the first M*K*2 bytes
 of the workspace (the header guarantees it holds X_r after a rotating call)
 and compared with the float64 oracle's rotation, element by element; Y is
@@ -29,7 +29,10 @@ def _status_clean():
 
 TC_CASES = [
     # (M, K, N, krot, use_cs, active pairs)
-    (256, 256, 512, 8, True, None),        # smallest batch on this path; 4 tiles, fewer CTAs than SMs
+    (65, 256, 512, 8, True, None),         # smallest batch on this path: one 128-row tile, 63 rows clipped
+    (128, 512, 256, 8, True, None),        # exactly one full tile per group
+    (200, 1024, 256, 17, True, None),      # krot 17
+    (256, 256, 512, 8, True, None),        # 4 tiles, fewer CTAs than SMs
     (300, 1024, 256, 8, True, None),       # ragged last row tile
     (512, 128, 256, 8, True, None),        # one group: every CTA shares it
     (1000, 384, 256, 1, False, None),      # krot = 1, no channel scales
