@@ -393,7 +393,7 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
 int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t N,
                       const int32_t* qweight, const int32_t* qzeros, const __half* scales,
                       const __half* bias, cudaStream_t s, bool pdl) {
-  CUtensorMap tmA, tmW, tmS, tmZ;
+  CUtensorMap tmA, tmW, tmS, tmZ, tmY;
   bool ok = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, kTcMB * kTcBM, kTcBK,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, kTcBK, kTcBN / 8,
@@ -401,13 +401,15 @@ int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t
             encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kTcBN,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kTcBN / 8,
-                      CU_TENSOR_MAP_SWIZZLE_NONE);
+                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            encode_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, y, M, N, kTcMB * kTcBM, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return PARO_ERR_CUDA;
   const dim3 grid((unsigned)((N + kTcBN - 1) / kTcBN), (unsigned)((M + kTcMB * kTcBM - 1) / (kTcMB * kTcBM)), 1);
   if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
   if (!allow_smem(w4_tc_gemm_kernel, TcLayout::SMEM)) return PARO_ERR_CUDA;
   return launch(w4_tc_gemm_kernel, grid, dim3(kTcThreads), TcLayout::SMEM, s, pdl, tmA, tmW, tmS,
-                tmZ, bias, y, (int)M, (int)N, (int)K);
+                tmZ, tmY, bias, (int)M, (int)N, (int)K);
 }
 
 // Shared memory a GEMV CTA is launched with: at least what its group range

@@ -72,6 +72,10 @@ struct TcLayout {
   static constexpr int MISC_OFF = BAR_OFF + 8 * NBARS;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  // epilogue staging of the fp16 output tile, over the (then idle) TMA ring
+  // and the start of the B ring: four {64 columns, 256 rows} boxes
+  static constexpr int O_BOX = kTcMB * kTcBM * 64 * 2;     // 32 KB
+  static_assert((kTcBN / 64) * O_BOX <= BAR_OFF, "output staging fits before the barriers");
 };
 
 // instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M=128, N=256
@@ -80,7 +84,7 @@ constexpr uint32_t kTcIdesc = (1u << 4) | ((uint32_t)(kTcBN >> 3) << 17) | ((uin
 __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
-    const __half* __restrict__ bias, __half* __restrict__ Y, int M, int N, int K) {
+    const __grid_constant__ CUtensorMap tmY, const __half* __restrict__ bias, int M, int N, int K) {
   using L = TcLayout;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -114,6 +118,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmS);
     tma_prefetch_desc(&tmZ);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {                      // the whole warp allocates 2 x 256 TMEM columns
     tmem_alloc(smem_u32(tmem_slot), kTcMB * kTcBN);
@@ -246,14 +251,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     // ------------------------------------------------------------ epilogue
     // warp w reads TMEM lanes 32*(w%4) .. +31 (its token rows of a block);
     // warps 2..5 take block 0 columns 0..127, 6..9 block 0 columns 128..255,
-    // 10..13 and 14..17 the same halves of block 1.
+    // 10..13 and 14..17 the same halves of block 1.  The fp16 tile (+ bias) is
+    // staged in shared memory — the TMA ring, idle once every MMA is done — as
+    // four {64 columns, 256 rows} boxes with the 128-byte swizzle, and one
+    // thread writes it with four TMA stores (clipped at row M and column N),
+    // so every global write is a full line.
     pdl_wait_primary();                 // previous kernels are complete before Y is written
-    const bool ok = tc_wait(accum_full, 0, abort);
+    const bool ok = __all_sync(0xffffffffu, tc_wait(accum_full, 0, abort));   // warp-uniform
     tc_fence_after();
     const int quarter = warp & 3;
     const int cq = (warp - 2) >> 2;                 // 0..3
     const int mb = cq >> 1, chalf = cq & 1;
-    const int tok = tok0 + mb * kTcBM + 32 * quarter + lane;
+    const int row = mb * kTcBM + 32 * quarter + lane;   // token row within the tile
     if (ok) {
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
@@ -262,29 +271,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         tmem_ld32(tmem_d + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(mb * kTcBN + col0), r);
         tmem_ld_wait_tie(r);
         const int n = n0 + col0;
-        if (tok < M && n < N) {
+        // box col0 / 64, 16-byte chunks (col0 % 64) / 8 .. +3 of this row
+        const uint32_t rowp = base + (uint32_t)(col0 >> 6) * L::O_BOX + (uint32_t)row * 128u;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float v[8];
+        for (int q = 0; q < 4; ++q) {
+          float v[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]);
-            if (bias != nullptr) {      // bias is only 4-byte aligned: half2 loads
-              const __half2* bh = reinterpret_cast<const __half2*>(bias + n + 8 * q);
+          for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]);
+          if (bias != nullptr && n < N) {   // bias is only 4-byte aligned: half2 loads
+            const __half2* bh = reinterpret_cast<const __half2*>(bias + n + 8 * q);
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(bh[e]);
-                v[2 * e] += f.x;
-                v[2 * e + 1] += f.y;
-              }
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(bh[e]);
+              v[2 * e] += f.x;
+              v[2 * e + 1] += f.y;
             }
-            uint4 o;
-            __half2* oh = reinterpret_cast<__half2*>(&o);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) oh[e] = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
-            *reinterpret_cast<uint4*>(Y + (size_t)tok * N + n + 8 * q) = o;
           }
+          uint4 o;
+          __half2* oh = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) oh[e] = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+          const uint32_t chunk = (uint32_t)(((col0 & 63) >> 3) + q);
+          sts128u(rowp + ((chunk ^ (uint32_t)(row & 7)) << 4), o);
         }
       }
+    }
+    fence_proxy_async_smem();           // the staged tile is read by the TMA (async proxy)
+    named_bar_sync(1, 32 * kTcDequantWarps);
+    if (warp == 2 && lane == 0 && !*abort) {
+#pragma unroll
+      for (int b = 0; b < kTcBN / 64; ++b)
+        if (n0 + 64 * b < N) tma_store_2d(&tmY, base + (uint32_t)b * L::O_BOX, n0 + 64 * b, tok0);
+      bulk_commit_group();
+      bulk_wait_group_all();            // written before the kernel completes
     }
   }
 
