@@ -200,8 +200,9 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
  * exactly as that many paro_w4_linear calls would compute it (page
  * "ParoQuant", "Activation and weight transforms": Y = X_r Q(W_r)^T + b per
  * member).  At decode sizes the members share one rotation launch and one
- * GEMV launch when the combined grid fits the GPU at once; otherwise (and for
- * M > 16) the members run one after another.  Results may differ from the
+ * GEMV launch when the combined grid fits the GPU at once; above 64 rows the
+ * rotating members share one R' build and one X R' launch, then each runs its
+ * GEMM; otherwise the members run one after another.  Results may differ from the
  * separate calls in fp32 summation order only.
  *   linears         HOST array of `count` (1..PARO_MAX_GROUP) member descriptors;
  *                   each member's fields follow paro_w4_linear's rules

@@ -296,28 +296,50 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
   }
 }
 
-// Rotation as X R' on the tensor cores: one launch builds R' (fp16 parts,
-// transposed) into `rt`, a second computes X_r = X R'.
-int launch_rotate_tc(const __half* x, __half* xr, __half* rt, int64_t M, int64_t K, const float* cs,
-                     const int16_t* pairs, const float* theta, int krot, cudaStream_t stream) {
+// Rotation as X R' on the tensor cores for `count` linears that read the same
+// x: one launch builds every member's R' (fp16 parts, transposed) into its `rt`,
+// a second computes every member's X_r = X R'.
+struct RotTcMember {
+  const float* cs;
+  const int16_t* pairs;
+  const float* theta;
+  int krot;
+  __half* xr;       // X_r [M, K]
+  __half* rt;       // R' parts [2][K][128]
+};
+
+int launch_rotate_tc(const __half* x, const RotTcMember* mem, int count, int64_t M, int64_t K,
+                     cudaStream_t stream) {
   const DeviceInfo& di = device_info();
   if (di.sms == 0) return PARO_ERR_CUDA;
+  if (count < 1 || count > kRcMaxMembers) return PARO_ERR_UNSUPPORTED;
   const int64_t groups = K / kGroup, tiles = (M + 127) / 128;
+  RbBatch rb;
+  std::memset(&rb, 0, sizeof(rb));
+  RcBatch rc;
+  std::memset(&rc, 0, sizeof(rc));
+  int max_krot = 0;
+  for (int i = 0; i < count; ++i) {
+    rb.op[i] = RbOperand{mem[i].cs, mem[i].pairs, mem[i].theta, mem[i].rt, mem[i].krot};
+    max_krot = std::max(max_krot, mem[i].krot);
+    if (!encode_2d(&rc.t[i].r, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, mem[i].rt, 2 * K, kGroup, 128, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&rc.t[i].y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, mem[i].xr, M, K, 128, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return PARO_ERR_CUDA;
+  }
   if (!allow_smem(rmat_build_kernel, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
-  if (int st = launch(rmat_build_kernel, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows)), dim3(kRbThreads),
-                      rb_smem_bytes(krot), stream, true, cs, pairs, theta, rt, (int)K, krot))
+  if (int st = launch(rmat_build_kernel, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows), (unsigned)count),
+                      dim3(kRbThreads), rb_smem_bytes(max_krot), stream, true, rb, (int)K))
     return st;
-  CUtensorMap tmX, tmR, tmY;
-  if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&tmR, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rt, 2 * K, kGroup, 128, 64,
-                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xr, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+  CUtensorMap tmX;
+  if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return PARO_ERR_CUDA;
   if (!allow_smem(rotate_tc_kernel, RcLayout::SMEM)) return PARO_ERR_CUDA;
-  const int64_t jobs = groups * tiles;
+  const int64_t jobs = (int64_t)count * groups * tiles;
   const int64_t ctas = jobs < di.sms ? jobs : di.sms;
   return launch(rotate_tc_kernel, dim3((unsigned)ctas), dim3(kRcThreads), RcLayout::SMEM, stream, true, tmX,
-                tmR, tmY, (int)K, (int)tiles, (long long)jobs);
+                rc, count, (int)K, (int)groups, (int)tiles, (long long)jobs);
 }
 
 // ---------------------------------------------------------------- linear plan
@@ -691,8 +713,8 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     __half* xr = reinterpret_cast<__half*>(ws + plan.off_xr);
     if (plan.rot_tc) {
-      __half* rt = reinterpret_cast<__half*>(ws + plan.off_rt);
-      if (int st = launch_rotate_tc(xa, xr, rt, M, K, channel_scales, pairs, theta, krot, s)) return st;
+      const RotTcMember one{channel_scales, pairs, theta, krot, xr, reinterpret_cast<__half*>(ws + plan.off_rt)};
+      if (int st = launch_rotate_tc(xa, &one, 1, M, K, s)) return st;
     } else if (int st = launch_rotate(xa, xr, M, K, channel_scales, pairs, theta, krot, s)) {
       return st;
     }
@@ -709,7 +731,7 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
   return dispatch_gemv(plan, &one, 1, M, K, s, pdl);
 }
 
-static_assert(PARO_MAX_GROUP == kGvMaxLinears && PARO_MAX_GROUP == kRrMaxLinears,
+static_assert(PARO_MAX_GROUP == kGvMaxLinears && PARO_MAX_GROUP == kRrMaxLinears && PARO_MAX_GROUP == kRcMaxMembers,
               "one launch holds every member of a group");
 
 size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, const paro_linear* linears,
@@ -738,11 +760,12 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
     }
   }
   if (M == 0) return 0;
+  // prefill batches rotating on the tensor cores: one R' build and one X R'
+  // launch for all rotating members, then one GEMM each
+  if (make_plan(M, K, linears[0].N).rot_tc) return (rot > 0 ? 2 : 0) + count;
   LinearPlan gp;
-  // one after another: each rotating member launches its rotation (two
-  // kernels on the tensor-core path) and its GEMV / GEMM
-  if (count == 1 || !group_plan(M, K, linears, count, &gp))
-    return rot * (make_plan(M, K, linears[0].N).rot_tc ? 2 : 1) + count;
+  // one after another: each rotating member launches its rotation and its GEMV / GEMM
+  if (count == 1 || !group_plan(M, K, linears, count, &gp)) return rot + count;
   return (rot > 0 ? (rows_ok ? 1 : rot) : 0) + 1;
 }
 
@@ -766,6 +789,35 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
   // member i's X_r lives at workspace + i * per (all members share M and K)
   const size_t per = make_plan(M, K, linears[0].N).total;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
+
+  const LinearPlan first = make_plan(M, K, linears[0].N);
+  if (count > 1 && first.rot_tc) {
+    // prefill: every rotating member's X_r in one R' build + one X R' launch
+    // (x is read once per tile for all of them), then one GEMM per member
+    RotTcMember rm[PARO_MAX_GROUP];
+    int nrot = 0;
+    const __half* xs[PARO_MAX_GROUP];
+    for (int i = 0; i < count; ++i) {
+      const paro_linear& l = linears[i];
+      xs[i] = static_cast<const __half*>(x);
+      if (l.krot > 0 || l.channel_scales != nullptr) {
+        __half* xr = reinterpret_cast<__half*>(ws + i * per + first.off_xr);
+        rm[nrot++] = RotTcMember{l.channel_scales, l.pairs, l.theta, l.krot, xr,
+                                 reinterpret_cast<__half*>(ws + i * per + first.off_rt)};
+        xs[i] = xr;
+      }
+    }
+    if (nrot > 0)
+      if (int st = launch_rotate_tc(static_cast<const __half*>(x), rm, nrot, M, K, s)) return st;
+    for (int i = 0; i < count; ++i) {
+      const paro_linear& l = linears[i];
+      if (int st = launch_w4_prefill(xs[i], static_cast<__half*>(l.y), M, K, l.N, l.qweight, l.qzeros,
+                                     static_cast<const __half*>(l.scales), static_cast<const __half*>(l.bias), s,
+                                     true))
+        return st;
+    }
+    return PARO_OK;
+  }
 
   LinearPlan gp;
   if (count == 1 || !group_plan(M, K, linears, count, &gp)) {

@@ -42,13 +42,33 @@ __host__ __device__ constexpr size_t rb_smem_bytes(int krot) {
   return (size_t)krot * (kGroup / 2) * sizeof(RotParam) + (size_t)kRbRows * kRbPitch * 4;
 }
 
-// grid (K/128, 128/kRbRows), block kRbThreads.  rt: fp16 [2][K][128] (above).
-__global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(
-    const float* __restrict__ cs, const int16_t* __restrict__ pairs,
-    const float* __restrict__ theta, __half* __restrict__ rt, int K, int krot) {
+// Linears that rotate the same x (a decoder layer's q/k/v, or gate/up) are
+// handled by one launch of each kernel: member i has its own tables, R' parts
+// and X_r.
+constexpr int kRcMaxMembers = 4;
+struct RbOperand {
+  const float* cs;         // [K] or nullptr
+  const int16_t* pairs;    // [krot, K]
+  const float* theta;      // [krot, K/2]
+  __half* rt;              // R' parts, fp16 [2][K][128]
+  int krot;
+};
+struct RbBatch {
+  RbOperand op[kRcMaxMembers];
+};
+
+// grid (K/128, 128/kRbRows, members), block kRbThreads; dynamic shared memory
+// for the largest krot of the batch.
+__global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_constant__ RbBatch batch, int K) {
   // The rotation that follows waits for this kernel's completion; let it
   // launch and set itself up meanwhile.
   pdl_launch_dependents();
+  const RbOperand& op = batch.op[blockIdx.z];
+  const float* __restrict__ cs = op.cs;
+  const int16_t* __restrict__ pairs = op.pairs;
+  const float* __restrict__ theta = op.theta;
+  __half* __restrict__ rt = op.rt;
+  const int krot = op.krot;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RotParam* prm = reinterpret_cast<RotParam*>(smem_raw);
   const uint32_t vbase = smem_u32(smem_raw + (size_t)krot * (kGroup / 2) * sizeof(RotParam));
@@ -118,10 +138,11 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(
 }
 
 // ------------------------------------------------------------------ X R'
-// Work: jobs (group g, 128-row tile t), group-major; CTA c of P (one per SM)
-// takes the contiguous range [c J / P, (c+1) J / P), so every CTA moves the
-// same number of tiles and holds one group's R' at a time (a range crosses a
-// group boundary at most a few times; R' is reloaded there).
+// Work: jobs (member m, group g, 128-row tile t), member-major then
+// group-major; CTA c of P (one per SM) takes the contiguous range
+// [c J / P, (c+1) J / P), so every CTA moves the same number of tiles and
+// holds one (member, group) R' at a time (a range crosses such a boundary at
+// most a few times; R' is reloaded there).  All members read the same x.
 //
 // Warp roles: warp 0 = TMA producer (R' parts, x tiles through a
 // kRcStages-deep ring), warp 1 = TMEM allocator and single-thread MMA issuer,
@@ -179,12 +200,21 @@ __device__ __forceinline__ void rc_stage32(uint32_t tile, int r, int cb, const u
   }
 }
 
+// Per member: r = its R' parts as [2K, 128] fp16, y = its X_r [M, K] fp16
+// (stores), both box {64, 128} with the 128-byte swizzle.
+struct alignas(64) RcTarget {
+  CUtensorMap r;
+  CUtensorMap y;
+};
+struct RcBatch {
+  RcTarget t[kRcMaxMembers];
+};
+
 // grid P <= number of SMs, block kRcThreads.  tmX: x [M, K] fp16, box {64, 128},
-// 128-byte swizzle; tmY: X_r, same shape, box and swizzle (stores).  tmR: the
-// parts as [2K, 128] fp16, same box and swizzle.
+// 128-byte swizzle.  jobs = members * groups * tiles.
 __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
-    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR,
-    const __grid_constant__ CUtensorMap tmY, int K, int tiles, long long jobs) {
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ RcBatch batch, int members, int K,
+    int groups, int tiles, long long jobs) {
   using L = RcLayout;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -219,8 +249,10 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
     *abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmX);
-    tma_prefetch_desc(&tmR);
-    tma_prefetch_desc(&tmY);
+    for (int m = 0; m < members; ++m) {
+      tma_prefetch_desc(&batch.t[m].r);
+      tma_prefetch_desc(&batch.t[m].y);
+    }
   }
   if (warp == 1) {                         // the whole warp allocates the two accumulators
     tmem_alloc(smem_u32(tmem_slot), kRcCols);
@@ -241,20 +273,22 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int cur_g = -1;
+      long long cur_u = -1;
       for (int i = 0; i < nj; ++i) {
         const long long j = j0 + i;
-        const int g = (int)(j / tiles), t = (int)(j % tiles);
-        if (g != cur_g) {
-          // every MMA that reads the previous group's R' has completed
+        const long long u = j / tiles;                 // (member, group) unit
+        const int m = (int)(u / groups), g = (int)(u % groups), t = (int)(j % tiles);
+        if (u != cur_u) {
+          // every MMA that reads the previous unit's R' has completed
           if (r_loads > 0 && !tc_wait(r_free, (uint32_t)((r_loads - 1) & 1), abort)) break;
+          const CUtensorMap* tmR = &batch.t[m].r;
           mbar_arrive_expect_tx(r_full, 4 * L::BOX);
-          tma_load_2d(base + L::R_OFF + 0 * L::BOX, &tmR, r_full, 0, g * 128);
-          tma_load_2d(base + L::R_OFF + 1 * L::BOX, &tmR, r_full, 64, g * 128);
-          tma_load_2d(base + L::R_OFF + 2 * L::BOX, &tmR, r_full, 0, K + g * 128);
-          tma_load_2d(base + L::R_OFF + 3 * L::BOX, &tmR, r_full, 64, K + g * 128);
+          tma_load_2d(base + L::R_OFF + 0 * L::BOX, tmR, r_full, 0, g * 128);
+          tma_load_2d(base + L::R_OFF + 1 * L::BOX, tmR, r_full, 64, g * 128);
+          tma_load_2d(base + L::R_OFF + 2 * L::BOX, tmR, r_full, 0, K + g * 128);
+          tma_load_2d(base + L::R_OFF + 3 * L::BOX, tmR, r_full, 64, K + g * 128);
           ++r_loads;
-          cur_g = g;
+          cur_u = u;
         }
         const int s = i % kRcStages;
         if (i >= kRcStages && !tc_wait(x_empty0 + 8 * s, (uint32_t)(((i / kRcStages) - 1) & 1), abort)) break;
@@ -268,13 +302,14 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int cur_g = -1, gi = -1;
+      long long cur_u = -1;
+      int gi = -1;
       for (int i = 0; i < nj; ++i) {
         const long long j = j0 + i;
-        const int g = (int)(j / tiles);
-        if (g != cur_g) {
+        const long long u = j / tiles;                 // (member, group) unit
+        if (u != cur_u) {
           ++gi;
-          cur_g = g;
+          cur_u = u;
           if (!tc_wait(r_full, (uint32_t)(gi & 1), abort)) break;
         }
         const int s = i % kRcStages, a = i & 1;
@@ -295,7 +330,7 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
         }
         umma_commit(x_empty0 + 8 * s);    // the x stage and ...
         umma_commit(acc_full0 + 8 * a);   // ... the accumulator, once these MMAs finish
-        if (i + 1 == nj || (j + 1) / tiles != g) umma_commit(r_free);   // last tile of the group
+        if (i + 1 == nj || (j + 1) / tiles != u) umma_commit(r_free);   // last tile of the unit
       }
       // every MMA issued here has completed before tensor memory is released
       umma_commit(mma_done);
@@ -311,7 +346,8 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
     // so no warp can be left at a barrier; a given-up wait returns at once.
     for (int i = 0; i < nj; ++i) {
       const long long j = j0 + i;
-      const int g = (int)(j / tiles), t = (int)(j % tiles);
+      const long long u = j / tiles;
+      const int m = (int)(u / groups), g = (int)(u % groups), t = (int)(j % tiles);
       const int a = i & 1;
       // warp-uniform (tcgen05.ld is a warp-wide instruction)
       const bool ok = __all_sync(0xffffffffu, tc_wait(acc_full0 + 8 * a, (uint32_t)((i >> 1) & 1), abort));
@@ -345,8 +381,8 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
       fence_proxy_async_smem();            // the tile is read by the TMA (async proxy)
       named_bar_sync(2, 32 * kRcEpiWarps);
       if (leader && !*abort) {
-        tma_store_2d(&tmY, tile, g * 128, t * 128);
-        tma_store_2d(&tmY, tile + L::BOX, g * 128 + 64, t * 128);
+        tma_store_2d(&batch.t[m].y, tile, g * 128, t * 128);
+        tma_store_2d(&batch.t[m].y, tile + L::BOX, g * 128 + 64, t * 128);
         bulk_commit_group();
       }
     }

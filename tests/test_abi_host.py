@@ -177,11 +177,12 @@ def test_group_launch_count_query(L):
     qkv = [dict(N=4096), dict(N=1024), dict(N=1024)]
     n = pb.w4_linear_group_launches(1, 4096, qkv)
     assert n in (2, 6)                        # shared launches, or one rotation + one GEMV each
-    # prefill, one member after another: the tensor-core rotation is two launches
-    # (R' build, X R') above 64 rows, one below; then the GEMM
-    assert pb.w4_linear_group_launches(4096, 4096, qkv) == 9
-    assert pb.w4_linear_group_launches(65, 4096, qkv) == 9
+    # prefill above 64 rows: one R' build and one X R' launch for all rotating
+    # members, then one GEMM each; up to 64 rows one rotation + one GEMM per member
+    assert pb.w4_linear_group_launches(4096, 4096, qkv) == 5
+    assert pb.w4_linear_group_launches(65, 4096, qkv) == 5
     assert pb.w4_linear_group_launches(64, 4096, qkv) == 6
+    assert pb.w4_linear_group_launches(4096, 4096, [dict(N=4096, krot=0, channel_scales=False)] * 2) == 2
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096)]) == 2
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096, krot=0, channel_scales=False)]) == 1
     assert pb.w4_linear_group_launches(1, 4000, qkv) == 0               # invalid K

@@ -111,3 +111,13 @@ def test_group_deterministic_and_empty():
         assert torch.equal(u, v)
     e = pb.w4_linear_group(dev(synth.make_activations(lays[0], 1))[:0], mem)
     assert all(t.shape[0] == 0 for t in e)
+
+
+@pytest.mark.parametrize("M", [65, 300, 1000])
+def test_group_prefill_batched_rotation(M):
+    """Above 64 rows the rotating members share one R' build and one X R'
+    launch (x read once per tile for all of them): a plain member, krot 8,
+    krot 17 and scales only, each against the oracle and the separate call."""
+    lays = [synth.make_layer("p%d" % i, 1024, N, 60 + i, krot=k, bias_std=0.01, n_outliers=10)
+            for i, (N, k) in enumerate([(512, 8), (256, 8), (768, 17), (1024, 8)])]
+    check_group(lays, [(0, False), (None, True), (None, True), (0, True)], M)
