@@ -202,7 +202,10 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
  * member).  At decode sizes the members share one rotation launch and one
  * GEMV launch when the combined grid fits the GPU at once; above 64 rows the
  * rotating members share one R' build and one X R' launch, then each runs its
- * GEMM; otherwise the members run one after another.  Results may differ from the
+ * GEMM; otherwise the members run one after another.  Members whose rotation
+ * is the same — equal krot and the same channel_scales, pairs and theta
+ * pointers (experts that share one rotation) — rotate x once: the first of
+ * them computes X_r and the others read it.  Results may differ from the
  * separate calls in fp32 summation order only.
  *   linears         HOST array of `count` (1..PARO_MAX_GROUP) member descriptors;
  *                   each member's fields follow paro_w4_linear's rules

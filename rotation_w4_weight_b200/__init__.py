@@ -220,9 +220,17 @@ def w4_linear_group(x: torch.Tensor, members, group_size: int = 128, workspace: 
 
 
 def w4_linear_group_launches(M: int, K: int, members, group_size: int = 128) -> int:
-    """Kernel launches one ``w4_linear_group`` call of this shape issues."""
+    """Kernel launches one ``w4_linear_group`` call of this shape issues.
+
+    ``members``: dicts with N and optionally krot (default 8), channel_scales
+    (bool, default True) and same_rotation_as (index of an earlier member whose
+    rotation tables this member shares).  Only shapes and table identity
+    matter: the descriptors carry placeholder addresses, never dereferenced."""
     arr = (ParoLinear * len(members))()
     for i, m in enumerate(members):
-        arr[i] = ParoLinear(m["N"], None, None, None, None,
-                            1 if m.get("channel_scales", True) else None, None, None, m.get("krot", 8), None)
+        owner = m.get("same_rotation_as", i)
+        tag = 16 * (owner + 1)                   # distinct per rotation, shared by its members
+        krot = m.get("krot", 8)
+        arr[i] = ParoLinear(m["N"], None, None, None, None, tag if m.get("channel_scales", True) else None,
+                            tag if krot > 0 else None, tag if krot > 0 else None, krot, None)
     return int(paro_w4_linear_group_launches(M, K, len(members), arr, group_size))

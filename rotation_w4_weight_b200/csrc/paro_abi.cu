@@ -734,6 +734,26 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
 static_assert(PARO_MAX_GROUP == kGvMaxLinears && PARO_MAX_GROUP == kRrMaxLinears && PARO_MAX_GROUP == kRcMaxMembers,
               "one launch holds every member of a group");
 
+}  // extern "C"
+
+namespace {
+bool rotates(const paro_linear& l) { return l.krot > 0 || l.channel_scales != nullptr; }
+
+// The member whose X_r member i reads: the first member with the same rotation
+// (same krot and the same channel_scales, pairs and theta tensors — experts
+// that share one rotation rotate x once), or -1 when member i does not rotate.
+int rotation_owner(const paro_linear* l, int i) {
+  if (!rotates(l[i])) return -1;
+  for (int j = 0; j < i; ++j)
+    if (rotates(l[j]) && l[j].krot == l[i].krot && l[j].channel_scales == l[i].channel_scales &&
+        (l[i].krot == 0 || (l[j].pairs == l[i].pairs && l[j].theta == l[i].theta)))
+      return j;
+  return i;
+}
+}  // namespace
+
+extern "C" {
+
 size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, const paro_linear* linears,
                                            int group_size) {
   if (count < 1 || count > PARO_MAX_GROUP || linears == nullptr) return 0;
@@ -754,7 +774,7 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
     if (check_linear_shape(M, K, linears[i].N, group_size) != PARO_OK || linears[i].krot < 0 ||
         linears[i].krot > kMaxKrot)
       return 0;
-    if (linears[i].krot > 0 || linears[i].channel_scales != nullptr) {
+    if (rotation_owner(linears, i) == i) {       // one rotation per distinct set of tables
       ++rot;
       rows_ok = rows_ok && linears[i].krot <= kRrMaxKrot;
     }
@@ -799,13 +819,14 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
     const __half* xs[PARO_MAX_GROUP];
     for (int i = 0; i < count; ++i) {
       const paro_linear& l = linears[i];
+      const int o = rotation_owner(linears, i);
       xs[i] = static_cast<const __half*>(x);
-      if (l.krot > 0 || l.channel_scales != nullptr) {
-        __half* xr = reinterpret_cast<__half*>(ws + i * per + first.off_xr);
+      if (o < 0) continue;
+      __half* xr = reinterpret_cast<__half*>(ws + o * per + first.off_xr);
+      if (o == i)
         rm[nrot++] = RotTcMember{l.channel_scales, l.pairs, l.theta, l.krot, xr,
                                  reinterpret_cast<__half*>(ws + i * per + first.off_rt)};
-        xs[i] = xr;
-      }
+      xs[i] = xr;
     }
     if (nrot > 0)
       if (int st = launch_rotate_tc(static_cast<const __half*>(x), rm, nrot, M, K, s)) return st;
@@ -821,13 +842,19 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
 
   LinearPlan gp;
   if (count == 1 || !group_plan(M, K, linears, count, &gp)) {
-    // one call per member, each with its own slice of the workspace
+    // one call per member, each with its own slice of the workspace; a member
+    // that shares an earlier member's rotation reads that member's X_r
     for (int i = 0; i < count; ++i) {
       const paro_linear& l = linears[i];
-      if (int st = paro_w4_linear(x, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, l.channel_scales,
-                                  l.pairs, l.theta, group_size, l.krot, ws ? ws + i * per : nullptr,
-                                  ws ? per : 0, stream))
-        return st;
+      const int o = rotation_owner(linears, i);
+      int st;
+      if (o >= 0 && o != i)
+        st = paro_w4_linear(ws + o * per + first.off_xr, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias,
+                            nullptr, nullptr, nullptr, group_size, 0, nullptr, 0, stream);
+      else
+        st = paro_w4_linear(x, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, l.channel_scales, l.pairs,
+                            l.theta, group_size, l.krot, ws ? ws + i * per : nullptr, ws ? per : 0, stream);
+      if (st) return st;
     }
     return PARO_OK;
   }
@@ -841,14 +868,14 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
   bool rows_ok = M <= 16;
   for (int i = 0; i < count; ++i) {
     const paro_linear& l = linears[i];
-    const bool rot = l.krot > 0 || l.channel_scales != nullptr;
-    __half* xr = rot ? reinterpret_cast<__half*>(ws + i * per) : nullptr;
-    if (rot) {
+    const int o = rotation_owner(linears, i);
+    __half* xr = o >= 0 ? reinterpret_cast<__half*>(ws + o * per) : nullptr;
+    if (o == i) {
       rb.op[nrot++] = RrOperand{xr, l.channel_scales, l.pairs, l.theta, l.krot};
       max_krot = std::max(max_krot, l.krot);
       rows_ok = rows_ok && l.krot <= kRrMaxKrot;
     }
-    lin[i] = GemvLinearArgs{l.qweight, l.qzeros, l.scales, rot ? xr : xa, static_cast<const __half*>(l.bias),
+    lin[i] = GemvLinearArgs{l.qweight, l.qzeros, l.scales, o >= 0 ? xr : xa, static_cast<const __half*>(l.bias),
                             static_cast<__half*>(l.y), l.N};
   }
   if (nrot > 0) {

@@ -183,6 +183,12 @@ def test_group_launch_count_query(L):
     assert pb.w4_linear_group_launches(65, 4096, qkv) == 5
     assert pb.w4_linear_group_launches(64, 4096, qkv) == 6
     assert pb.w4_linear_group_launches(4096, 4096, [dict(N=4096, krot=0, channel_scales=False)] * 2) == 2
+    # experts sharing one rotation rotate x once: one rotation (not three) up to
+    # 64 rows, and the single-rotation count on the other paths
+    shared = [dict(N=1024), dict(N=1024, same_rotation_as=0), dict(N=1024, same_rotation_as=0)]
+    assert pb.w4_linear_group_launches(64, 4096, shared) == 1 + 3
+    assert pb.w4_linear_group_launches(4096, 4096, shared) == 2 + 3
+    assert pb.w4_linear_group_launches(1, 4096, shared) in (2, 4)
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096)]) == 2
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096, krot=0, channel_scales=False)]) == 1
     assert pb.w4_linear_group_launches(1, 4000, qkv) == 0               # invalid K

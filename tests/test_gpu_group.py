@@ -121,3 +121,33 @@ def test_group_prefill_batched_rotation(M):
     lays = [synth.make_layer("p%d" % i, 1024, N, 60 + i, krot=k, bias_std=0.01, n_outliers=10)
             for i, (N, k) in enumerate([(512, 8), (256, 8), (768, 17), (1024, 8)])]
     check_group(lays, [(0, False), (None, True), (None, True), (0, True)], M)
+
+
+@pytest.mark.parametrize("M", [1, 40, 300])
+def test_group_experts_sharing_one_rotation(M):
+    """Experts with their own weights and one shared rotation (the same
+    channel-scale, pair and angle tensors): x is rotated once and every expert
+    reads that X_r; each output against the oracle and the separate call."""
+    lays = [synth.make_layer("e%d" % i, 1024, 512, 70 + i, bias_std=0.01, n_outliers=10) for i in range(3)]
+    for lay in lays[1:]:
+        lay.pairs, lay.theta, lay.channel_scales = lays[0].pairs, lays[0].theta, lays[0].channel_scales
+    ds = [layer_to_device(l) for l in lays]
+    for d in ds[1:]:
+        d["pairs"], d["theta"], d["cs"] = ds[0]["pairs"], ds[0]["theta"], ds[0]["cs"]
+    x = synth.make_activations(lays[0], M)
+    mem = [member(l, d) for l, d in zip(lays, ds)]
+    outs = pb.w4_linear_group(dev(x), mem)
+    torch.cuda.synchronize()
+    specs = [dict(N=512), dict(N=512, same_rotation_as=0), dict(N=512, same_rotation_as=0)]
+    # never more launches than three separate rotations (the batched prefill
+    # rotation is two launches either way)
+    assert pb.w4_linear_group_launches(M, 1024, specs) <= pb.w4_linear_group_launches(M, 1024, [dict(N=512)] * 3)
+    rng = np.random.default_rng(M)
+    for lay, y, m in zip(lays, outs, mem):
+        cols = np.sort(rng.choice(lay.N, 128, replace=False))
+        got = y.cpu().numpy().astype(np.float64)[:, cols]
+        assert lin_err(got, oracle_cols(lay, x, cols)) <= LIN_TOL, lay.name
+        single = pb.w4_linear(dev(x), m["qweight"], m["qzeros"], m["scales"], m["bias"], m["channel_scales"],
+                              m["pairs"], m["theta"], 128, m["krot"])
+        a, b = y.float(), single.float()
+        assert float((a - b).abs().max()) <= 1e-2 * float(b.pow(2).mean().sqrt()), lay.name
