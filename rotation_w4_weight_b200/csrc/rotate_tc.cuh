@@ -20,8 +20,9 @@
 // X is fp16 and exact as an MMA operand, and Rhi + Rlo carries R' to about
 // 2^-22 relative, so the result is the fp32 rotation up to summation order.
 // The cost no longer grows with krot: 2 * 2 * M * 128 * K flops (two fp16
-// products) against 4 * M * K bytes of HBM traffic, about 4.4 GFLOP per
-// 16 MB of activations moved -- under the time the bytes take at HBM speed.
+// products) against 4 * M * K bytes of HBM traffic, i.e. 512 flops per 4 bytes
+// moved (about 2.1 GFLOP per 16 MB) -- less tensor-core time than the bytes
+// take at HBM speed.
 //
 // Layout of the transposed parts in global memory: fp16 [2][K][128]; part 0 is
 // Rhi, part 1 is Rlo; row g*128 + n, column k holds R'_g[k][n], i.e. each
