@@ -3,8 +3,8 @@ fix, not against the oracle itself.
 
 Each ``pin_*`` takes an implementation namespace ``impl`` exposing
 ``rotate``, ``inverse_rotate``, ``awq_pack``, ``awq_unpack``, ``dequant``,
-``w4_linear_from_codes``, ``transform_weight`` and ``quantize_sym4`` with the
-oracle's signatures, and raises
+``w4_linear_from_codes``, ``transform_weight``, ``quantize_sym4`` and
+``quantize_weight`` with the oracle's signatures, and raises
 AssertionError when the implementation disagrees.  ``test_oracle_pins.py``
 runs them on the oracle; ``test_oracle_mutations.py`` runs them on copies of
 the oracle with planted mistakes and checks that each mistake is caught.
@@ -396,6 +396,51 @@ def pin_quantized_replay(impl):
     assert np.max(np.abs(got - ref)) <= 1e-10 * np.max(np.abs(ref))
 
 
+def _nibble_codes(qw, N, K):
+    """Codes [N, K] read out of AWQ words bit by bit, with the nibble position
+    of each column taken from the golden word fixture (not from any packer)."""
+    g = json.load(open(os.path.join(GOLDEN, "awq_word.json")))
+    pos = g["nibble_position_of_column"]
+    u = np.asarray(qw).view(np.uint32)
+    codes = np.empty((N, K), np.int64)
+    for n in range(N):
+        for k in range(K):
+            codes[n, k] = (int(u[k, n // 8]) >> (4 * pos[n % 8])) & 0xF
+    return codes
+
+
+def pin_quantize_weight_packed(impl):
+    """quantize_weight (transform, quantise, pack in one call) against a route
+    that shares none of its steps: W_r = (W / cs) @ R with R the dense product
+    of per-stage Givens matrices built entry by entry, every word read back
+    nibble by nibble from the golden positions, and each code's level a
+    nearest of the 16 levels -8 s .. 7 s of W_r (found by trying them all).
+    Zero words are all 0x88888888 (zero point 8 in every nibble)."""
+    rng = np.random.default_rng(24)
+    N, K, G, krot = 16, 256, 128, 5
+    pairs, theta = _rand_tables(rng, K, G, krot)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))
+    W = rng.standard_normal((N, K)) * 0.7
+    W_r = (W / cs) @ dense_R(pairs, theta, K, G)
+    scales = rng.uniform(0.6, 1.2, (K // G, N)) * np.max(np.abs(W_r)) / 7.0
+    qw, qz = impl.quantize_weight(W, cs, pairs, theta, scales, G, krot)
+    qw, qz = np.asarray(qw), np.asarray(qz)
+    assert qw.dtype == np.int32 and qw.shape == (K, N // 8), (qw.dtype, qw.shape)
+    assert qz.dtype == np.int32 and qz.shape == (K // G, N // 8), (qz.dtype, qz.shape)
+    assert np.all(qz.view(np.uint32) == np.uint32(0x88888888))
+    codes = _nibble_codes(qw, N, K)
+    levels = np.arange(-8, 8)
+    for n in range(N):
+        for k in range(K):
+            sc = scales[k // G, n]
+            best = np.min(np.abs(levels * sc - W_r[n, k]))
+            got = abs((codes[n, k] - 8) * sc - W_r[n, k])
+            assert got <= best + 1e-12, (n, k, codes[n, k])
+    # krot=None takes every stage of the table
+    qw2, _ = impl.quantize_weight(W, cs, pairs, theta, scales, G)
+    assert np.array_equal(np.asarray(qw2), qw)
+
+
 ALL_PINS = [
     pin_single_pair_closed_forms, pin_stage_composition, pin_inverse_restores,
     pin_group_norms_preserved, pin_dense_R_brute_force, pin_golden_g4,
@@ -403,5 +448,5 @@ ALL_PINS = [
     pin_awq_one_hot, pin_awq_round_trip, pin_identity_state_is_plain_w4,
     pin_equivalent_weight_route, pin_dequant_formula,
     pin_weight_transform_identity, pin_sym4_closed_forms, pin_sym4_nearest_level_brute_force,
-    pin_quantized_replay,
+    pin_quantized_replay, pin_quantize_weight_packed,
 ]

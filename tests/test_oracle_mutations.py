@@ -16,7 +16,7 @@ def make_impl(sign_flip=False, reverse_stages=False, swap_roles=False, no_scale=
               theta_global=False, order=ORDER_OK, no_zero=False, group0_scale=False,
               inverse_forward_order=False, shared_group_base=False, q_half_away=False,
               q_clamp7=False, q_no_offset=False, w_scale_multiplied=False, q_group0_scale=False,
-              q_no_bound=False, w_no_stages=False):
+              q_no_bound=False, w_no_stages=False, qw_no_stages=False, qw_untransposed=False):
     def stage_idx(pairs_s, G):
         K = pairs_s.shape[0]
         local = pairs_s.astype(np.int64)
@@ -112,10 +112,18 @@ def make_impl(sign_flip=False, reverse_stages=False, swap_roles=False, no_scale=
         codes = (q.astype(np.int64) & 15).astype(np.uint8) if q_no_offset else (q + 8).astype(np.uint8)
         return codes, np.full((N, K // G), 0 if q_no_offset else 8, np.uint8)
 
+    def quantize_weight(W, cs, pairs, theta, scales, G, krot=None):
+        W_r = transform_weight(W, cs, pairs, theta, G, krot=0 if qw_no_stages else krot)
+        codes, zeros = quantize_sym4(W_r, scales, G)
+        if qw_untransposed:                   # words built along the wrong axis
+            return awq_pack(np.ascontiguousarray(codes.reshape(codes.shape[1], codes.shape[0])), zeros, G)
+        return awq_pack(codes, zeros, G)
+
     return types.SimpleNamespace(rotate=rotate, inverse_rotate=inverse_rotate, awq_pack=awq_pack,
                                  awq_unpack=awq_unpack, dequant=dequant,
                                  w4_linear_from_codes=w4_linear_from_codes,
-                                 transform_weight=transform_weight, quantize_sym4=quantize_sym4)
+                                 transform_weight=transform_weight, quantize_sym4=quantize_sym4,
+                                 quantize_weight=quantize_weight)
 
 
 def failing_pins(impl):
@@ -150,6 +158,8 @@ MUTATIONS = {
     "quant_scale_group_misindexed": dict(q_group0_scale=True),
     "quant_scale_unbounded": dict(q_no_bound=True),
     "weight_stages_skipped": dict(w_no_stages=True),
+    "quantize_weight_drops_the_stages": dict(qw_no_stages=True),
+    "quantize_weight_packs_untransposed_codes": dict(qw_untransposed=True),
 }
 
 
