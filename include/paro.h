@@ -250,10 +250,14 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
  * file-scope device array of PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES bytes that
  * every GPU which loads the library holds until the process exits.  It calls
  * no cudaMalloc, cudaFree or allocating library routine.
- *   - Limit: paro_w4_linear_workspace_size(M, K, N, group_size) must not exceed
+ *   - Limit: a call that rotates (krot > 0 or channel_scales != NULL) needs
+ *     paro_w4_linear_workspace_size(M, K, N, group_size) <=
  *     PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES (8 MiB: M*K <= 4 Mi fp16 elements
  *     up to 64 rows; above 64 rows M*K*2 + 512*K bytes, e.g. M <= 768 at
  *     K = 4096); larger shapes return PARO_ERR_WORKSPACE before any GPU work.
+ *     A call that does not rotate stages nothing and has no limit.  Arguments
+ *     are checked first, exactly as paro_w4_linear checks them, so a bad
+ *     argument gets the same status from both entry points.
  *   - The first call on a device looks up the array's device address for that
  *     device (cudaGetSymbolAddress) and caches it; make that first call before
  *     any stream capture.

@@ -925,17 +925,22 @@ int paro_w4_linear_noalloc(const void* x, void* y, int64_t M, int64_t K, int64_t
                            const int32_t* qweight, const int32_t* qzeros, const void* scales,
                            const void* bias, const float* channel_scales, const int16_t* pairs,
                            const float* theta, int group_size, int krot, paro_stream_t stream) {
-  // An invalid shape yields 0 here and the full validation below reports it.
-  const size_t need = paro_w4_linear_workspace_size(M, K, N, group_size);
-  if (need > (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES) return PARO_ERR_WORKSPACE;
-  void* scratch = nullptr;
-  if (need > 0 && M > 0) {
-    scratch = noalloc_scratch_address();
-    if (scratch == nullptr) return PARO_ERR_CUDA;
-  }
+  // the same argument checks, in the same order, as paro_w4_linear
+  if (int st = check_linear_args(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
+                                 group_size, krot))
+    return st;
+  if (M == 0) return PARO_OK;
+  // only a call that rotates (krot > 0 or channel scales) stages anything
+  const bool rotate = krot > 0 || channel_scales != nullptr;
+  if (!rotate)
+    return paro_w4_linear(x, y, M, K, N, qweight, qzeros, scales, bias, nullptr, pairs, theta, group_size, 0,
+                          nullptr, 0, stream);
+  if (paro_w4_linear_workspace_size(M, K, N, group_size) > (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES)
+    return PARO_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_address();
+  if (scratch == nullptr) return PARO_ERR_CUDA;
   return paro_w4_linear(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
-                        group_size, krot, scratch,
-                        scratch ? (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES : 0, stream);
+                        group_size, krot, scratch, (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int paro_validate_pairs(const int16_t* pairs_host, int64_t K, int group_size, int krot) {
