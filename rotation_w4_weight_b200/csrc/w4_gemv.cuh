@@ -39,7 +39,9 @@
 // owner's inbox (a dedicated shared-memory area, one slot per sender CTA and
 // k-part) with distributed-shared-memory stores; after one cluster barrier
 // each owner sums its inbox in a fixed order, adds the bias and writes fp16 Y.
-// No global scratch, no atomics, deterministic.
+// No global scratch, no atomics, deterministic.  A second cluster-barrier phase
+// (arrive after the pushes, wait at exit) keeps every CTA resident until all
+// its peers have issued their pushes, even when an inbox wait runs out.
 #pragma once
 
 #include "common.cuh"
@@ -353,6 +355,9 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
         }
       }
   }
+  // second cluster-barrier phase: arriving says "my pushes are issued".  A CTA
+  // waits on it before it exits, so no peer can still address its inbox then.
+  if (S > 1) cluster_arrive_release();
   // this thread's first output (the bias load overlaps the barrier)
   const int nq = mrows * (cols / 4);
   float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -366,7 +371,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   }
   // this CTA's own partials (CTA barrier) and every peer's (the inbox barrier)
   __syncthreads();
-  if (S > 1 && !mbar_wait_bounded(inbar, 0)) flag_error(kErrTimeout);
+  const bool landed = S == 1 || mbar_wait_bounded(inbar, 0);   // a timeout is flagged inside
   const uint32_t box = base + (uint32_t)L::inbox_off(gmax);
   for (int idx = tid; idx < nq; idx += L::THREADS) {
     const int tl = idx / (cols / 4);
@@ -392,6 +397,13 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     out.x = *reinterpret_cast<const uint32_t*>(&h0);
     out.y = *reinterpret_cast<const uint32_t*>(&h1);
     *reinterpret_cast<uint2*>(Y + (size_t)tl * N + n) = out;
+  }
+  if (S > 1) {
+    // every peer has issued its pushes once this returns (each peer arrives
+    // after finitely many bounded waits); if the bytes had not all landed, give
+    // the late ones one more bounded wait before this CTA's shared memory goes away
+    cluster_wait_acquire();
+    if (!landed) mbar_wait_bounded(inbar, 0);
   }
 }
 
