@@ -1,12 +1,17 @@
 #!/usr/bin/env python
 """Benchmark of the rotated W4 linear (decode HBM GB/s / prefill TFLOP/s).
 
-python bench.py [--gpus N] [--steps K] [--warmup W] [--workload q_proj_decode|mlp_decode|
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload layer|q_proj_decode|mlp_decode|
                  prefill|layer_decode|layer_prefill|quantize_gate_proj] [--impl ours|reference]
 
 One "step" is one pass of the whole hot path (scale + Givens stages + W4
 dequant-GEMM) over every call of the workload:
-  q_proj_decode (default): Llama-3-8B q_proj 4096->4096, M = 1, 4, 16 (three calls)
+  layer (default): the full Llama-3-8B decoder-layer linear set (q, k, v, o,
+                 gate, up, down) at M = 1 (decode, the line's value in HBM GB/s)
+                 and at M = 4096 (prefill, TFLOP/s, in the line's "prefill"
+                 object); each half is timed, roofline-checked and baselined
+                 on its own
+  q_proj_decode: Llama-3-8B q_proj 4096->4096, M = 1, 4, 16 (three calls)
   mlp_decode:    gate/up 4096->14336 and down 14336->4096, M = 1 and 8 (six calls)
   prefill:       gate_proj-shaped 4096->14336, M = 2048 and 8192, bias (two calls)
   layer_decode / layer_prefill: the seven linears of a decoder layer at M = 1 / 4096
@@ -54,7 +59,21 @@ WORKLOADS = {
     "layer_prefill": dict(cfg=4, layers=list(range(7)), Ms=[4096], kind="prefill",
                           groups=[[0, 1, 2], [3], [4, 5], [6]]),
     "quantize_gate_proj": dict(cfg=2, layers=[0], Ms=[], kind="quantize"),
+    # both halves of the decoder-layer set in one line
+    "layer": dict(cfg=4, kind="pair", halves=["layer_decode", "layer_prefill"]),
 }
+REPLAYS = 7          # timed replays of the K-step graph; the median is reported
+
+
+_LAYERS = {}
+
+
+def cfg_layers(cfg):
+    """The seeded layers of a workload config, drawn once per process (the
+    arrays are read, never written)."""
+    if cfg not in _LAYERS:
+        _LAYERS[cfg] = synth.config_layers(cfg)
+    return _LAYERS[cfg]
 
 
 # ----------------------------------------------------------------- algorithmic cost model
@@ -193,28 +212,63 @@ def job_throughput(world, steps, per_step, ms):
     return world * steps * per_step / (ms * 1e-3)
 
 
+def timed_replays(replay, stream, world, device, replays=REPLAYS):
+    """Times `replays` runs of `replay()` (one CUDA graph of exactly K steps)
+    with CUDA events on `stream`, each bracketed by a barrier and device syncs.
+    Returns the per-replay milliseconds, each the max over ranks."""
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    out = []
+    for _ in range(replays):
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(device)
+        e0.record(stream)
+        replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            torch.distributed.barrier()
+        out.append(max_over_ranks(e0.elapsed_time(e1), world, device))
+    return out
+
+
+def spread(ms_list, steps):
+    """Median, fastest and slowest replay, per step (ms)."""
+    return {"replays": len(ms_list), "median_ms_per_step": round(statistics.median(ms_list) / steps, 5),
+            "min_ms_per_step": round(min(ms_list) / steps, 5),
+            "max_ms_per_step": round(max(ms_list) / steps, 5)}
+
+
 def workload_config(workload, world):
     """The workload description shared by both arms' JSON lines."""
     wl = WORKLOADS[workload]
-    layers = [synth.config_layers(wl["cfg"])[i] for i in wl["layers"]]
+    if wl["kind"] == "pair":
+        dec, pre = (workload_config(h, world) for h in wl["halves"])
+        return {"workload": workload, "layers": dec["layers"], "calls": dec["calls"],
+                "M": {"decode": dec["M"], "prefill": pre["M"]}, "group_size": GROUP, "krot": KROT,
+                "accumulate": "f32", "parallelism": f"replicas x{world}"}
+    layers = [synth.config_layer_shapes(wl["cfg"])[i] for i in wl["layers"]]
     if wl["kind"] == "quantize":
-        return {"workload": workload, "weights": [(l.name, l.N, l.K) for l in layers],
+        return {"workload": workload, "weights": [(n, N, K) for n, K, N in layers],
                 "input": "float W fp16 [N, K] and quantiser scales fp16 [K/128, N]",
                 "group_size": GROUP, "krot": KROT, "parallelism": f"replicas x{world}"}
-    return {"workload": workload, "layers": [(l.name, l.K, l.N) for l in layers], "M": wl["Ms"],
-            "calls": [[layers[i].name for i in g] for g in wl["groups"]],
+    return {"workload": workload, "layers": [(n, K, N) for n, K, N in layers], "M": wl["Ms"],
+            "calls": [[layers[i][0] for i in g] for g in wl["groups"]],
             "group_size": GROUP, "krot": KROT, "accumulate": "f32", "parallelism": f"replicas x{world}"}
 
 
 # ----------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
+def run_ours(args, rank, world, local_rank, workload=None):
     import torch
     import rotation_w4_weight_b200 as pb
 
+    workload = workload or args.workload
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = WORKLOADS[args.workload]
-    layers = [synth.config_layers(wl["cfg"])[i] for i in wl["layers"]]
+    wl = WORKLOADS[workload]
+    layers = [cfg_layers(wl["cfg"])[i] for i in wl["layers"]]
     Ms = wl["Ms"]
     decode = wl["kind"] == "decode"
 
@@ -305,25 +359,16 @@ def run_ours(args, rank, world, local_rank):
     while time.time() < t_end:                   # load before the window so clocks settle
         replay(g)
         torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    replay(g)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    ms = e0.elapsed_time(e1)
+    step_ms = timed_replays(lambda: replay(g), stream, world, dev)
+    ms = statistics.median(step_ms)
     t_end = time.time() + 0.4
     while time.time() < t_end:
         replay(g)
         torch.cuda.synchronize(dev)
     clocks = sampler.stop()
-    ms = max_over_ranks(ms, world, dev)
     assert pb.device_status() == pb.PARO_OK
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
 
     # ---- dominant kernel, timed live: X_r is produced once per call shape by
     #      paro_rotate (outside the timed graph); the graph holds the GEMV/GEMM
@@ -357,17 +402,14 @@ def run_ours(args, rank, world, local_rank):
                 n_launch += launches(gi, M, rotate=False)
     replay(g2)
     torch.cuda.synchronize(dev)
-    e0.record(stream)
-    replay(g2)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    kern_ms = e0.elapsed_time(e1)
+    kern_list = timed_replays(lambda: replay(g2), stream, world, dev)
+    kern_ms = statistics.median(kern_list)
     peaks = load_peaks()
     if decode:
         achieved = kern_bytes / (kern_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                "traffic": traffic_for("w4_gemv_decode"),
+                "traffic": traffic_for(workload),
                 "kernel": "w4_gemv_kernel (decode GEMV, split-K cluster)",
                 "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
                 "bytes_per_launch": kern_bytes // n_launch, "peak_source": peaks["src"]}
@@ -377,7 +419,7 @@ def run_ours(args, rank, world, local_rank):
         achieved = kern_flops / (kern_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_sus"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_sus"], 4),
-                "traffic": traffic_for("w4_tc_prefill"),
+                "traffic": traffic_for(workload),
                 "kernel": "w4_tc_gemm_kernel (prefill tcgen05 GEMM)", "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
                 "flops_per_launch": kern_flops // n_launch,
                 "peak_source": peaks["src"] + " bf16 sustained (fp16 runs at the bf16 rate)",
@@ -390,7 +432,7 @@ def run_ours(args, rank, world, local_rank):
     hy = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in ys.items()}
     h2d = sum(v.numel() * 2 for v in hx.values())
     d2h = sum(v.numel() * 2 for v in hy.values())
-    e_steps = max(1, min(args.steps, 200))
+    e_steps = max(1, min(args.steps, 200 if decode else 20))
 
     def e2e_step(i):
         for c, (gi, M) in enumerate(gcalls):
@@ -420,17 +462,19 @@ def run_ours(args, rank, world, local_rank):
         value = job_throughput(world, args.steps, step_flops, ms) / 1e12
         unit = "TFLOP/s"
         e2e_val = job_throughput(world, 1, step_flops, e2e_ms) / 1e12
-    metric = metric_name(args.workload)
+    metric = metric_name(workload)
 
     out = {
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
-        "config": dict(workload_config(args.workload, world),
+        "config": dict(workload_config(workload, world),
                        l2=f"weights cycled over {reps} device replicas "
                           f"({reps * weight_bytes / 2**20:.0f} MiB > 3x L2)",
-                       timing="CUDA graph of the K steps, CUDA events, max over ranks"),
+                       timing=f"median of {len(step_ms)} replays of a CUDA graph of the K steps, "
+                              "CUDA events, max over ranks"),
+        "timing": spread(step_ms, args.steps),
         "roofline": roof,
         "e2e": {"value": round(e2e_val, 2), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
@@ -440,12 +484,36 @@ def run_ours(args, rank, world, local_rank):
         "rotation_overhead": {"frac": round(ms / kern_ms - 1.0, 4),
                               "ms_per_step_rotated": round(ms / args.steps, 5),
                               "ms_per_step_unrotated": round(kern_ms / args.steps, 5),
+                              "unrotated_timing": spread(kern_list, args.steps),
                               "how": "same K steps as CUDA graphs; unrotated = krot 0, no channel "
                                      "scales, same kernels on X_r"},
         "gpu_launches": sum(launches(gi, M) for gi, M in gcalls) * args.steps,
         "clocks": clocks,
         "bytes_per_step": step_bytes, "flops_per_step": step_flops,
     }
+    return out
+
+
+def run_pair(args, rank, world, local_rank):
+    """Both halves of a paired workload (decode at the line's top level, prefill
+    in its "prefill" object), one after the other on the same GPU."""
+    import torch
+    wl = WORKLOADS[args.workload]
+    dec_name, pre_name = wl["halves"]
+    dec = run_ours(args, rank, world, local_rank, dec_name)
+    torch.cuda.empty_cache()
+    pre = run_ours(args, rank, world, local_rank, pre_name)
+    torch.cuda.empty_cache()
+    out = dict(dec)
+    out["metric"] = metric_name(args.workload)
+    out["config"] = dict(workload_config(args.workload, world), l2=dec["config"]["l2"],
+                         timing=dec["config"]["timing"])
+    out["decode_workload"] = dec_name
+    out["prefill"] = {k: pre[k] for k in ("metric", "value", "unit", "ms_per_step", "timing", "roofline",
+                                          "e2e", "rotation_overhead", "gpu_launches", "clocks",
+                                          "bytes_per_step", "flops_per_step")}
+    out["prefill"]["workload"] = pre_name
+    out["prefill"]["steps"] = args.steps
     return out
 
 
@@ -459,7 +527,7 @@ def run_quantize(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = WORKLOADS[args.workload]
-    lay = synth.config_layers(wl["cfg"])[wl["layers"][0]]
+    lay = cfg_layers(wl["cfg"])[wl["layers"][0]]
     W, qs = synth.make_float_weight(lay)
 
     def T(a):
@@ -579,7 +647,7 @@ def quantize_oracle_sample(workload, budget_s, max_steps=None):
     weight (256 rows per sample), until `budget_s` seconds or max_steps samples."""
     import oracle
     wl = WORKLOADS[workload]
-    lay = synth.config_layers(wl["cfg"])[wl["layers"][0]]
+    lay = cfg_layers(wl["cfg"])[wl["layers"][0]]
     W, qs = synth.make_float_weight(lay)
     rng = np.random.default_rng(0)
     done = 0.0
@@ -608,7 +676,7 @@ def oracle_sample(workload, budget_s, max_steps=None):
     wl = WORKLOADS[workload]
     if wl["kind"] == "quantize":
         return quantize_oracle_sample(workload, budget_s, max_steps)
-    layers = [synth.config_layers(wl["cfg"])[i] for i in wl["layers"]]
+    layers = [cfg_layers(wl["cfg"])[i] for i in wl["layers"]]
     decode = wl["kind"] == "decode"
     rng = np.random.default_rng(0)
     done_bytes = done_flops = 0.0
@@ -636,11 +704,36 @@ def oracle_sample(workload, budget_s, max_steps=None):
 
 
 def metric_name(workload):
+    if WORKLOADS[workload]["kind"] == "pair":
+        return ("rotated W4 linear, Llama-3-8B decoder-layer linear set: decode HBM GB/s at M=1 "
+                "(value) and prefill TFLOP/s at M=4096 (prefill.value), % of roofline")
     if WORKLOADS[workload]["kind"] == "quantize":
         return f"weight quantiser HBM throughput ({workload})"
     decode = WORKLOADS[workload]["kind"] == "decode"
     return ("rotated W4 linear decode HBM throughput" if decode else
             "rotated W4 linear prefill tensor throughput") + f" ({workload})"
+
+
+def reference_half(workload, steps, warmup, world):
+    """One workload of the reference arm: the oracle on bounded samples."""
+    wl = WORKLOADS[workload]
+    decode = wl["kind"] in ("decode", "quantize")
+    cores = len(os.sched_getaffinity(0))
+    per_step_budget = max(0.2, min(2.0, 150.0 / max(1, steps + warmup)))
+    oracle_sample(workload, per_step_budget * warmup, max_steps=warmup)
+    val, desc, secs = oracle_sample(workload, per_step_budget * steps, max_steps=max(1, steps))
+    unit = "GB/s" if decode else "TFLOP/s"
+    return {
+        "impl": "reference", "metric": metric_name(workload),
+        "value": round(val, 5), "unit": unit, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(secs * 1e3 / max(1, steps), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": dict(workload_config(workload, world), timing="host wall clock of the oracle"),
+        "cpu_baseline": {"value": round(val, 5), "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(val, 5), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
 
 
 def run_reference(args, rank, world):
@@ -649,24 +742,17 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     wl = WORKLOADS[args.workload]
-    decode = wl["kind"] in ("decode", "quantize")
-    cores = len(os.sched_getaffinity(0))
-    per_step_budget = max(0.2, min(2.0, 150.0 / max(1, args.steps + args.warmup)))
-    oracle_sample(args.workload, per_step_budget * args.warmup, max_steps=args.warmup)
-    val, desc, secs = oracle_sample(args.workload, per_step_budget * args.steps,
-                                    max_steps=max(1, args.steps))
-    unit = "GB/s" if decode else "TFLOP/s"
-    return {
-        "impl": "reference", "metric": metric_name(args.workload),
-        "value": round(val, 5), "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(secs * 1e3 / max(1, args.steps), 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
-        "config": dict(workload_config(args.workload, world), timing="host wall clock of the oracle"),
-        "cpu_baseline": {"value": round(val, 5), "unit": unit, "cores": cores, "kind": "oracle",
-                         "sample": desc},
-        "e2e": {"value": round(val, 5), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
+    if wl["kind"] != "pair":
+        return reference_half(args.workload, args.steps, args.warmup, world)
+    dec_name, pre_name = wl["halves"]
+    # both halves share the few minutes the arm may take
+    dec = reference_half(dec_name, max(1, args.steps // 2), args.warmup, world)
+    pre = reference_half(pre_name, max(1, args.steps // 2), args.warmup, world)
+    dec["metric"] = metric_name(args.workload)
+    dec["steps"] = args.steps
+    dec["config"] = dict(workload_config(args.workload, world), timing="host wall clock of the oracle")
+    dec["prefill"] = {k: pre[k] for k in ("metric", "value", "unit", "ms_per_step", "cpu_baseline", "e2e")}
+    return dec
 
 
 # ----------------------------------------------------------------- main
@@ -676,7 +762,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default="q_proj_decode")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="layer")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle CPU work for the cpu_baseline field")
     args = ap.parse_args()
@@ -699,15 +785,25 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    if WORKLOADS[args.workload]["kind"] == "quantize":
+    wl = WORKLOADS[args.workload]
+    if wl["kind"] == "quantize":
         out = run_quantize(args, rank, world, local_rank)
+    elif wl["kind"] == "pair":
+        out = run_pair(args, rank, world, local_rank)
     else:
         out = run_ours(args, rank, world, local_rank)
     if rank == 0:
-        val, desc, _ = oracle_sample(args.workload, args.cpu_budget)
-        out["cpu_baseline"] = {"value": round(val, 5), "unit": out["unit"],
-                               "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-                               "sample": desc}
+        if wl["kind"] == "pair":
+            for half, obj in zip(wl["halves"], (out, out["prefill"])):
+                val, desc, _ = oracle_sample(half, args.cpu_budget / 2)
+                obj["cpu_baseline"] = {"value": round(val, 5), "unit": obj["unit"],
+                                       "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+                                       "sample": desc}
+        else:
+            val, desc, _ = oracle_sample(args.workload, args.cpu_budget)
+            out["cpu_baseline"] = {"value": round(val, 5), "unit": out["unit"],
+                                   "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+                                   "sample": desc}
         print(json.dumps(out), flush=True)
     if world > 1:
         torch.distributed.barrier()
