@@ -287,11 +287,25 @@ int paro_validate_pairs(const int16_t* pairs_host, int64_t K, int group_size, in
  * paro_device_status — reads (and, if clear != 0, resets) the device status word
  * of the current device.  Synchronises the device.  Returns PARO_OK,
  * PARO_ERR_TIMEOUT (a bounded wait ran out), PARO_ERR_INVALID_ARG (a pair index
- * outside its group was seen) or PARO_ERR_CUDA (the CUDA query failed, or a
- * kernel found a device resource laid out other than it requires and skipped
- * its work).
+ * outside its group was seen) or PARO_ERR_CUDA (the CUDA query failed).
  */
 int paro_device_status(int clear);
+
+/*
+ * paro_selftest_wait_timeout — failure-detection self-test (the pages have no
+ * counterpart; it checks this library's own error path).  Runs one kernel whose
+ * single thread waits, with the bounded wait every kernel of this library uses
+ * but a limit of `limit_ns` nanoseconds, on an mbarrier that nothing arrives
+ * at.  The wait runs out, sets the timeout bit of the device status word (so
+ * paro_device_status then reports PARO_ERR_TIMEOUT) and the kernel returns
+ * normally; no copy or other work is in flight, and the context stays usable.
+ *   limit_ns    1 .. 100 000 000 (100 ms), else PARO_ERR_INVALID_ARG
+ *   elapsed_ns  HOST pointer or NULL: nanoseconds the wait took before giving up
+ *               (device %globaltimer), 0 if it had completed instead
+ * Synchronises `stream`.  Returns PARO_OK once the kernel has run, or
+ * PARO_ERR_CUDA if the launch or the read-back failed.
+ */
+int paro_selftest_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns, paro_stream_t stream);
 
 #ifdef __cplusplus
 }

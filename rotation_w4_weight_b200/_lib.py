@@ -1,7 +1,7 @@
 """ctypes binding of the C ABI in include/paro.h (argument marshalling only).
 
 Every function of the header is exposed here under the same name.  The
-library must exist (build it with ``python -m rotation_w4_weight_b200.build``);
+library must exist (build it with ``python rotation_w4_weight_b200/build.py``);
 importing this module without it raises, there is no fallback.
 """
 from __future__ import annotations
@@ -25,6 +25,7 @@ EXPORTED = (
     "paro_w4_linear_workspace_size", "paro_w4_linear", "paro_w4_linear_noalloc",
     "paro_validate_pairs", "paro_device_status", "paro_quantize_w4",
     "paro_w4_linear_group_workspace_size", "paro_w4_linear_group", "paro_w4_linear_group_launches",
+    "paro_selftest_wait_timeout",
 )
 
 PARO_MAX_GROUP = 4
@@ -58,6 +59,7 @@ _SIGNATURES = {
     "paro_w4_linear_group_workspace_size": (ctypes.c_size_t, [_i64, _i64, _int, _vp, _int]),
     "paro_w4_linear_group": (_int, [_vp, _i64, _i64, _int, _vp, _int, _vp, ctypes.c_size_t, _vp]),
     "paro_w4_linear_group_launches": (_int, [_i64, _i64, _int, _vp, _int]),
+    "paro_selftest_wait_timeout": (_int, [ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64), _vp]),
 }
 
 
@@ -65,7 +67,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(
             f"{path} is missing: build the CUDA library first "
-            "(python -m rotation_w4_weight_b200.build); there is no CPU fallback")
+            "(python rotation_w4_weight_b200/build.py); there is no CPU fallback")
     lib = ctypes.CDLL(path)
     for name, (res, args) in _SIGNATURES.items():
         fn = getattr(lib, name)
@@ -91,6 +93,7 @@ paro_quantize_w4 = lib.paro_quantize_w4
 paro_w4_linear_group_workspace_size = lib.paro_w4_linear_group_workspace_size
 paro_w4_linear_group = lib.paro_w4_linear_group
 paro_w4_linear_group_launches = lib.paro_w4_linear_group_launches
+paro_selftest_wait_timeout = lib.paro_selftest_wait_timeout
 
 
 class ParoError(RuntimeError):

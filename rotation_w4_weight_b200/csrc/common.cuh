@@ -14,7 +14,6 @@ namespace paro {
 // Device status word bits (read by paro_device_status).
 constexpr unsigned kErrTimeout = 1u;
 constexpr unsigned kErrPairIndex = 2u;
-constexpr unsigned kErrInternal = 4u;     // a device-side layout assumption failed
 
 // The library is one translation unit (no relocatable device code), so the
 // status word is defined here, once.
@@ -66,17 +65,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false (and
-// sets the timeout bit) if it did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// sets the timeout bit) if it did not complete within `limit_ns` nanoseconds.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       flag_error(kErrTimeout);
       return false;
     }
   }
+}
+
+// The wait every kernel uses: bounded by kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  return mbar_wait_limit(bar, parity, kWaitLimitNs);
 }
 
 // Bounded wait that also gives up as soon as another role of the CTA has given up
@@ -394,6 +398,24 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
                                               uint32_t layout) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+
+// ---------------------------------------------------------------- self-test
+// Elapsed nanoseconds of the last wait_selftest_kernel (read by the host).
+__device__ unsigned long long g_selftest_elapsed_ns = 0ull;
+
+// One bounded wait on an mbarrier that nothing arrives at: the wait runs out
+// after `limit_ns`, sets the timeout bit of the status word, and the kernel
+// returns.  No copy or other thread is involved, so nothing is left in flight.
+__global__ void __launch_bounds__(32) wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  const unsigned long long t0 = globaltimer();
+  const bool done = mbar_wait_limit(b, 0, limit_ns);
+  g_selftest_elapsed_ns = done ? 0ull : globaltimer() - t0;
 }
 
 // Named barrier over `count` threads (a subset of the CTA, whole warps).

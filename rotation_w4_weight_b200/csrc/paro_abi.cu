@@ -32,6 +32,8 @@ constexpr int kMaxSplits = 8;         // cluster size along K (portable maximum)
 // the workspace; measured faster than the pair-by-pair tensor-memory kernel from
 // one 128-row tile up); below it the shared-memory / warp-per-row kernels
 constexpr int64_t kRotTcMinM = 65;
+// longest wait paro_selftest_wait_timeout accepts (it holds the stream that long)
+constexpr uint64_t kSelftestMaxLimitNs = 100000000ull;   // 100 ms
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -971,7 +973,19 @@ int paro_device_status(int clear) {
   }
   if (v & kErrTimeout) return PARO_ERR_TIMEOUT;
   if (v & kErrPairIndex) return PARO_ERR_INVALID_ARG;
-  if (v & kErrInternal) return PARO_ERR_CUDA;
+  return PARO_OK;
+}
+
+int paro_selftest_wait_timeout(uint64_t limit_ns, uint64_t* elapsed_ns, paro_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > kSelftestMaxLimitNs) return PARO_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  wait_selftest_kernel<<<1, 32, 0, s>>>((unsigned long long)limit_ns);
+  if (cudaGetLastError() != cudaSuccess) return PARO_ERR_CUDA;
+  unsigned long long e = 0;
+  if (cudaMemcpyFromSymbolAsync(&e, g_selftest_elapsed_ns, sizeof(e), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return PARO_ERR_CUDA;
+  if (elapsed_ns != nullptr) *elapsed_ns = (uint64_t)e;
   return PARO_OK;
 }
 

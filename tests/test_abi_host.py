@@ -13,8 +13,12 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def L():
-    from rotation_w4_weight_b200 import build
-    build.build()
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_paro_build", os.path.join(ROOT, "rotation_w4_weight_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    b.build()                       # rebuild if a source is newer, before the library loads
     from rotation_w4_weight_b200 import _lib
     return _lib
 
@@ -192,3 +196,11 @@ def test_group_launch_count_query(L):
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096)]) == 2
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096, krot=0, channel_scales=False)]) == 1
     assert pb.w4_linear_group_launches(1, 4000, qkv) == 0               # invalid K
+
+
+def test_selftest_wait_limit_is_checked_on_the_host(L):
+    # a zero or over-long limit is refused before any launch
+    e = ctypes.c_uint64(7)
+    assert L.paro_selftest_wait_timeout(0, ctypes.byref(e), None) == L.PARO_ERR_INVALID_ARG
+    assert L.paro_selftest_wait_timeout(100_000_001, ctypes.byref(e), None) == L.PARO_ERR_INVALID_ARG
+    assert e.value == 7
