@@ -40,8 +40,9 @@
 // k-part) with distributed-shared-memory stores; after one cluster barrier
 // each owner sums its inbox in a fixed order, adds the bias and writes fp16 Y.
 // No global scratch, no atomics, deterministic.  A second cluster-barrier phase
-// (arrive after the pushes, wait at exit) keeps every CTA resident until all
-// its peers have issued their pushes, even when an inbox wait runs out.
+// (each CTA arrives once all bytes addressed to it have landed, and waits at
+// exit) keeps every CTA resident until every push of the cluster has landed, so
+// no st.async is ever in flight from or to a CTA that has left.
 #pragma once
 
 #include "common.cuh"
@@ -330,6 +331,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const int cols = kGvTile / S;                    // columns owned by each CTA of the cluster
   const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
   const uint32_t inbox = base + L::inbox_off(gmax);  // fp32 [S][KP][MP][cols]
+  __syncwarp();
   if (S > 1) cluster_wait_acquire();               // every peer's inbox barrier is set up
   if (warp != 0) {
     const int owner = (8 * wcol) / cols;
@@ -355,9 +357,6 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
         }
       }
   }
-  // second cluster-barrier phase: arriving says "my pushes are issued".  A CTA
-  // waits on it before it exits, so no peer can still address its inbox then.
-  if (S > 1) cluster_arrive_release();
   // this thread's first output (the bias load overlaps the barrier)
   const int nq = mrows * (cols / 4);
   float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -372,6 +371,12 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // this CTA's own partials (CTA barrier) and every peer's (the inbox barrier)
   __syncthreads();
   const bool landed = S == 1 || mbar_wait_bounded(inbar, 0);   // a timeout is flagged inside
+  // second cluster-barrier phase: a CTA arrives once every byte addressed to it
+  // has landed, and waits on the phase before it exits; so when any CTA leaves,
+  // every push of the cluster has landed and no st.async is still in flight
+  // (from it or to it)
+  __syncwarp();
+  if (S > 1) cluster_arrive_release();
   const uint32_t box = base + (uint32_t)L::inbox_off(gmax);
   for (int idx = tid; idx < nq; idx += L::THREADS) {
     const int tl = idx / (cols / 4);
@@ -399,9 +404,11 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     *reinterpret_cast<uint2*>(Y + (size_t)tl * N + n) = out;
   }
   if (S > 1) {
-    // every peer has issued its pushes once this returns (each peer arrives
-    // after finitely many bounded waits); if the bytes had not all landed, give
-    // the late ones one more bounded wait before this CTA's shared memory goes away
+    // returns once every CTA of the cluster has received all its bytes (each
+    // arrives after finitely many bounded waits); if this CTA's own bytes had
+    // not all landed, give the late ones one more bounded wait before its
+    // shared memory goes away
+    __syncwarp();
     cluster_wait_acquire();
     if (!landed) mbar_wait_bounded(inbar, 0);
   }
