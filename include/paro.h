@@ -55,9 +55,13 @@
  *     releases early writes layer constants (paro_pack_awq does not release
  *     early; paro_quantize_w4 does not release early), and kernels that never
  *     release early are always safe.
- *   - Supported now: G == 128 (group_size == -1 is accepted when K == 128),
- *     0 <= krot <= 64, K a multiple of 128, N a multiple of 32 (the packer alone
- *     needs only N % 8 == 0), fp16 activations/scales/bias.
+ *   - Supported now: G in {16, 32, 64, 128} (the page's "Backend reference"
+ *     lists groups 16/32/64/128 and -1; group_size == -1 is accepted when it
+ *     normalises to one of these, i.e. K == 128, since K must be a multiple of
+ *     128: the kernels work on 128-channel tiles holding 128 / G groups), the
+ *     rotation groups and the quantisation groups share G; 0 <= krot <= 64;
+ *     N a multiple of 32 (the packer alone needs only N % 8 == 0 and any even
+ *     G); fp16 activations/scales/bias.
  */
 #ifndef PARO_H_
 #define PARO_H_
@@ -96,7 +100,7 @@ const char* paro_version(void);
  *   M >= 0 rows (M == 0 is a no-op), K > 0 channels, K % group_size == 0
  *   channel_scales  device fp32 [K] or NULL (no scaling)
  *   pairs, theta    device tables as above; may be NULL only when krot == 0
- *   group_size      128, or -1 meaning K (then K must be 128)
+ *   group_size      16, 32, 64 or 128, or -1 meaning K (then K must be 128)
  *   krot            number of stages, 0..64 (0 = scaling only)
  * Arithmetic: fp32 on chip; cos/sin of the fp32 angle by the hardware
  * approximation after one reduction into [-pi, pi] (absolute error about

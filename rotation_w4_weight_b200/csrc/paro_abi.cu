@@ -186,6 +186,16 @@ bool allow_smem(Kern kernel, size_t bytes) {
   return true;
 }
 
+// Group sizes the kernels implement: every power of two that divides their
+// 128-channel tiles down to 16 (the rotation groups and the quantisation
+// groups share G; K must be a multiple of 128).
+inline bool supported_group(int G, int64_t K) {
+  return (G == 16 || G == 32 || G == 64 || G == 128) && K % kGroup == 0;
+}
+
+// The group size of a call whose arguments passed the checks (-1 is K).
+inline int group_of(int group_size, int64_t K) { return group_size == -1 ? (int)K : group_size; }
+
 int normalize_group(int group_size, int64_t K, int* G) {
   const int64_t g = (group_size == -1) ? K : group_size;
   if (g <= 0 || (g % 2) != 0 || K <= 0 || (K % g) != 0) return PARO_ERR_INVALID_ARG;
@@ -199,7 +209,7 @@ int check_rotation_args(const void* x, const void* xr, int64_t M, int64_t K, con
   if (M < 0 || K <= 0 || krot < 0) return PARO_ERR_INVALID_ARG;
   int G = 0;
   if (int st = normalize_group(group_size, K, &G)) return st;
-  if (G != kGroup || krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
+  if (!supported_group(G, K) || krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
   if (M == 0) return PARO_OK;   // nothing to touch: NULL data pointers are fine
   if (x == nullptr || xr == nullptr) return PARO_ERR_INVALID_ARG;
   if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
@@ -213,12 +223,12 @@ int check_rotation_args(const void* x, const void* xr, int64_t M, int64_t K, con
 // Warp-per-row rotation of one x for `count` linears (blockIdx.z), decode sizes
 // (M <= 16, every krot <= kRrMaxKrot; max_krot sizes the tables).
 int launch_rotate_rows(const __half* x, const RrBatch& b, int count, int64_t M, int64_t K, int max_krot,
-                       cudaStream_t stream) {
+                       int gsz, cudaStream_t stream) {
   // always 8 warps: all of them build the tables, warps past the batch then leave
   const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + kRrWarps - 1) / kRrWarps), (unsigned)count);
   if (!allow_smem(rotate_rows_kernel, RrLayout::bytes(kRrMaxKrot))) return PARO_ERR_CUDA;
   return launch(rotate_rows_kernel, grid, dim3(32 * kRrWarps), RrLayout::bytes(max_krot), stream, true, b, x,
-                (int)M, (int)K);
+                (int)M, (int)K, gsz);
 }
 
 // Tensor-memory rotation kernel (and, with QUANT, the weight quantiser): CTAs
@@ -226,7 +236,7 @@ int launch_rotate_rows(const __half* x, const RrBatch& b, int count, int64_t M, 
 // 2 CTAs per SM: the shared-memory floor of the kernel guarantees no more fit).
 template <bool QUANT>
 int launch_rotate_tmem(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
-                       const int16_t* pairs, const float* theta, int krot, const RtQuant& qo,
+                       const int16_t* pairs, const float* theta, int krot, int gsz, const RtQuant& qo,
                        cudaStream_t stream) {
   const size_t smem = RtLayout::bytes(krot, QUANT);
   const DeviceInfo& di = device_info();
@@ -254,21 +264,21 @@ int launch_rotate_tmem(const __half* x, __half* xr, int64_t M, int64_t K, const 
   const dim3 grid((unsigned)groups, (unsigned)gy);
   if (abs_tables)
     return launch(rotate_tmem_kernel<true, QUANT>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
-                  pairs, theta, (int)M, (int)K, krot, qo);
+                  pairs, theta, (int)M, (int)K, krot, gsz, qo);
   return launch(rotate_tmem_kernel<false, QUANT>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
-                pairs, theta, (int)M, (int)K, krot, qo);
+                pairs, theta, (int)M, (int)K, krot, gsz, qo);
 }
 
 int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
-                  const int16_t* pairs, const float* theta, int krot, cudaStream_t stream) {
+                  const int16_t* pairs, const float* theta, int krot, int gsz, cudaStream_t stream) {
   // Large batches: tensor memory as the permutation network.
-  if (M > 64) return launch_rotate_tmem<false>(x, xr, M, K, cs, pairs, theta, krot, RtQuant{}, stream);
+  if (M > 64) return launch_rotate_tmem<false>(x, xr, M, K, cs, pairs, theta, krot, gsz, RtQuant{}, stream);
   // Decode batches with few stages: one warp per row, no block barrier per stage.
   if (M <= 16 && krot <= kRrMaxKrot) {
     RrBatch b;
     std::memset(&b, 0, sizeof(b));
     b.op[0] = RrOperand{xr, cs, pairs, theta, krot};
-    return launch_rotate_rows(x, b, 1, M, K, krot, stream);
+    return launch_rotate_rows(x, b, 1, M, K, krot, gsz, stream);
   }
   // rows per CTA: 4 for decode-sized batches (more CTAs, shorter latency),
   // 32..64 otherwise (conflict-free 32-row warp accesses)
@@ -282,19 +292,19 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
     case 4:
       if (!allow_smem(rotate_kernel<4>, rotate_smem_bytes(4, kMaxKrot))) return PARO_ERR_CUDA;
       return launch(rotate_kernel<4>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
-                    (int)M, (int)K, krot);
+                    (int)M, (int)K, krot, gsz);
     case 32:
       if (!allow_smem(rotate_kernel<32>, rotate_smem_bytes(32, kMaxKrot))) return PARO_ERR_CUDA;
       return launch(rotate_kernel<32>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
-                    (int)M, (int)K, krot);
+                    (int)M, (int)K, krot, gsz);
     case 64:
       if (!allow_smem(rotate_kernel<64>, rotate_smem_bytes(64, kMaxKrot))) return PARO_ERR_CUDA;
       return launch(rotate_kernel<64>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
-                    (int)M, (int)K, krot);
+                    (int)M, (int)K, krot, gsz);
     default:
       if (!allow_smem(rotate_kernel<128>, rotate_smem_bytes(128, kMaxKrot))) return PARO_ERR_CUDA;
       return launch(rotate_kernel<128>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
-                    (int)M, (int)K, krot);
+                    (int)M, (int)K, krot, gsz);
   }
 }
 
@@ -310,7 +320,7 @@ struct RotTcMember {
   __half* rt;       // R' parts [2][K][128]
 };
 
-int launch_rotate_tc(const __half* x, const RotTcMember* mem, int count, int64_t M, int64_t K,
+int launch_rotate_tc(const __half* x, const RotTcMember* mem, int count, int64_t M, int64_t K, int gsz,
                      cudaStream_t stream) {
   const DeviceInfo& di = device_info();
   if (di.sms == 0) return PARO_ERR_CUDA;
@@ -332,7 +342,7 @@ int launch_rotate_tc(const __half* x, const RotTcMember* mem, int count, int64_t
   }
   if (!allow_smem(rmat_build_kernel, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
   if (int st = launch(rmat_build_kernel, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows), (unsigned)count),
-                      dim3(kRbThreads), rb_smem_bytes(max_krot), stream, true, rb, (int)K))
+                      dim3(kRbThreads), rb_smem_bytes(max_krot), stream, true, rb, (int)K, gsz))
     return st;
   CUtensorMap tmX;
   if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -352,6 +362,7 @@ struct LinearPlan {
   int splits = 1;          // decode split-K factor = cluster size along K
   int variant = 0;         // decode kernel configuration (tile, k-parts, stages)
   bool rot_tc = false;     // the rotation runs on the tensor cores (R' in the workspace)
+  int gsz = kGroup;        // group size (rotation and quantisation)
   size_t off_xr = 0, off_rt = 0, total = 0;
 };
 
@@ -360,17 +371,31 @@ int check_linear_shape(int64_t M, int64_t K, int64_t N, int group_size) {
   int G = 0;
   if (int st = normalize_group(group_size, K, &G)) return st;
   if (N % 8 != 0) return PARO_ERR_INVALID_ARG;
-  if (G != kGroup || N % 32 != 0) return PARO_ERR_UNSUPPORTED;
+  if (!supported_group(G, K) || N % 32 != 0) return PARO_ERR_UNSUPPORTED;
   if (M * K >= (int64_t(1) << 31) || M * N >= (int64_t(1) << 31) || K * N >= (int64_t(1) << 34) ||
       M > (int64_t(1) << 22))
     return PARO_ERR_UNSUPPORTED;
   return PARO_OK;
 }
 
+// Shared memory of a decode GEMV configuration (variant, token tiles) for
+// `gmax` 128-row groups and `gr` quantisation-group rows per CTA.
+size_t gemv_layout_bytes(int variant, int nt, int gmax, int gr) {
+  const bool one = nt == 1;
+  switch (variant) {
+    case 0: return one ? GemvLayout<1, 2, 256, 4>::smem(gmax, gr) : GemvLayout<2, 2, 256, 4>::smem(gmax, gr);
+    case 2: return one ? GemvLayout<1, 4, 128, 8>::smem(gmax, gr) : GemvLayout<2, 4, 128, 8>::smem(gmax, gr);
+    case 5: return one ? GemvLayout<1, 4, 64, 8>::smem(gmax, gr) : GemvLayout<2, 4, 64, 8>::smem(gmax, gr);
+    default: return one ? GemvLayout<1, 2, 128, 4>::smem(gmax, gr) : GemvLayout<2, 2, 128, 4>::smem(gmax, gr);
+  }
+}
+constexpr size_t kSmemPerCta = 227 * 1024;   // dynamic shared memory a CTA may use (sm_100)
+
 // The split is a function of the shape only (not of the device), so the
 // workspace size query and the call agree everywhere.
-LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
+LinearPlan make_plan(int64_t M, int64_t K, int64_t N, int gsz) {
   LinearPlan p;
+  p.gsz = gsz;
   const int groups = (int)(K / kGroup);
   p.decode = M <= kMaxDecodeM;
   p.off_xr = 0;
@@ -404,36 +429,57 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N) {
     p.n_tiles = (int)((N + tile - 1) / tile);
     int s = 1;
     while (s * 2 <= want && s * 2 <= kMaxSplits && s * 2 <= groups && p.n_tiles * s * 2 <= kDecodeTargetCtas) s *= 2;
-    // a CTA holds at most kGvMaxGroups groups of activations and constants
-    while ((groups + s - 1) / s > kGvMaxGroups && s < kMaxSplits) s *= 2;
+    // a CTA holds at most kGvMaxGroups groups of activations and constants,
+    // and its layout (with 128 / G rows of scales and zero words per group)
+    // must fit the shared memory of one CTA
+    const int gq = kGroup / gsz;
+    auto bytes = [&](int sp) {
+      const int gm = (groups + sp - 1) / sp;
+      return gemv_layout_bytes(p.variant, p.nt, gm, gm * gq);
+    };
+    while (((groups + s - 1) / s > kGvMaxGroups || bytes(s) > kSmemPerCta) && s < kMaxSplits) s *= 2;
     p.splits = s;
-    // deeper than the GEMV's reach (K > 16384): the tensor-core GEMM serves it
-    if ((groups + s - 1) / s > kGvMaxGroups) p.decode = false;
+    // deeper than the GEMV's reach (K > 16384, or small groups of a very deep
+    // K): the tensor-core GEMM serves it
+    if ((groups + s - 1) / s > kGvMaxGroups || bytes(s) > kSmemPerCta) p.decode = false;
   }
   return p;
 }
 
-// Prefill (M > 16): tcgen05 GEMM, 128 token rows x 256 output columns per CTA.
-int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t N,
-                      const int32_t* qweight, const int32_t* qzeros, const __half* scales,
-                      const __half* bias, cudaStream_t s, bool pdl) {
+// Prefill (M > 16): tcgen05 GEMM, 256 token rows x 256 output columns per CTA.
+template <int SR>
+int launch_w4_prefill_sr(const __half* xa, __half* y, int64_t M, int64_t K, int64_t N,
+                         const int32_t* qweight, const int32_t* qzeros, const __half* scales,
+                         const __half* bias, int gsz, cudaStream_t s, bool pdl) {
   CUtensorMap tmA, tmW, tmS, tmZ, tmY;
   bool ok = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, kTcMB * kTcBM, kTcBK,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, kTcBK, kTcBN / 8,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / kGroup, N, 1, kTcBN,
+            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / gsz, N, SR, kTcBN,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
-            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / kGroup, N / 8, 1, kTcBN / 8,
+            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / gsz, N / 8, SR, kTcBN / 8,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, y, M, N, kTcMB * kTcBM, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return PARO_ERR_CUDA;
   const dim3 grid((unsigned)((N + kTcBN - 1) / kTcBN), (unsigned)((M + kTcMB * kTcBM - 1) / (kTcMB * kTcBM)), 1);
   if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
-  if (!allow_smem(w4_tc_gemm_kernel, TcLayout::SMEM)) return PARO_ERR_CUDA;
-  return launch(w4_tc_gemm_kernel, grid, dim3(kTcThreads), TcLayout::SMEM, s, pdl, tmA, tmW, tmS,
-                tmZ, tmY, bias, (int)M, (int)N, (int)K);
+  using L = TcLayoutT<SR>;
+  if (!allow_smem(w4_tc_gemm_kernel<SR>, L::SMEM)) return PARO_ERR_CUDA;
+  return launch(w4_tc_gemm_kernel<SR>, grid, dim3(kTcThreads), L::SMEM, s, pdl, tmA, tmW, tmS,
+                tmZ, tmY, bias, (int)M, (int)N, (int)K, gsz);
+}
+
+int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t N,
+                      const int32_t* qweight, const int32_t* qzeros, const __half* scales,
+                      const __half* bias, int gsz, cudaStream_t s, bool pdl) {
+  // scale rows per 64-row k-block: 64 / G groups below G = 64
+  switch (gsz) {
+    case 32: return launch_w4_prefill_sr<2>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
+    case 16: return launch_w4_prefill_sr<4>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
+    default: return launch_w4_prefill_sr<1>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
+  }
 }
 
 // Shared memory a GEMV CTA is launched with: at least what its group range
@@ -470,6 +516,7 @@ int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, in
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
   const int groups = (int)(K / kGroup);
   const int gmax = (groups + plan.splits - 1) / plan.splits;   // largest group range of a CTA
+  const int gq = kGroup / plan.gsz;                             // quantisation groups per 128 rows
   if (gmax > kGvMaxGroups || count < 1 || count > NL) return PARO_ERR_UNSUPPORTED;
   GemvBatch<NL> b;
   std::memset(&b, 0, sizeof(b));
@@ -485,10 +532,10 @@ int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, in
         encode_2d(&o.w, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qweight, K, N / 8, 128, L::WORDS,
                   L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                       : (L::ROW_BYTES == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE)) &&
-        encode_2d(&o.s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, lin[i].scales, K / kGroup, N, (uint32_t)gmax,
-                  NTILE, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, K / kGroup, N / 8, (uint32_t)gmax,
-                  L::WORDS, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        encode_2d(&o.s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, lin[i].scales, K / plan.gsz, N,
+                  (uint32_t)(gmax * gq), NTILE, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, K / plan.gsz, N / 8,
+                  (uint32_t)(gmax * gq), L::WORDS, CU_TENSOR_MAP_SWIZZLE_NONE) &&
         encode_x_chunks(&o.x, lin[i].x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP, (uint32_t)(2 * gmax));
     if (!ok) return PARO_ERR_CUDA;
     o.bias = lin[i].bias;
@@ -500,13 +547,13 @@ int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, in
   if (tiles > INT_MAX / 2) return PARO_ERR_UNSUPPORTED;
   auto k = w4_gemv_kernel<NT, KP, NTILE, STAGES, NL>;
   const dim3 grid((unsigned)tiles, (unsigned)plan.splits, 1);
-  const size_t smem = gemv_footprint((size_t)L::smem(gmax), (int64_t)grid.x * grid.y);
+  const size_t smem = gemv_footprint((size_t)L::smem(gmax, gmax * gq), (int64_t)grid.x * grid.y);
   if (smem == 0 || !allow_smem(k, device_info().smem_optin)) return PARO_ERR_CUDA;
   // a grid larger than the SM count places its clusters by load (measured:
   // 256-CTA grids of 8-CTA clusters ran 1-10 % faster; one-per-SM grids did not gain)
   const bool balance = (int64_t)grid.x * grid.y > device_info().sms;
   return launch_ex(k, grid, dim3(L::THREADS), smem, s, pdl, (unsigned)plan.splits, balance, b, (int)M,
-                   (int)K, gmax);
+                   (int)K, gmax, gq);
 }
 
 template <int NT, int NL>
@@ -556,7 +603,8 @@ int paro_rotate(const void* x, void* x_r, int64_t M, int64_t K, const float* cha
     return st;
   if (M == 0) return PARO_OK;
   return launch_rotate(static_cast<const __half*>(x), static_cast<__half*>(x_r), M, K,
-                       channel_scales, pairs, theta, krot, reinterpret_cast<cudaStream_t>(stream));
+                       channel_scales, pairs, theta, krot, group_of(group_size, K),
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 int paro_quantize_w4(const void* w, const float* channel_scales, const int16_t* pairs,
@@ -565,7 +613,7 @@ int paro_quantize_w4(const void* w, const float* channel_scales, const int16_t* 
   if (N < 0 || K <= 0 || krot < 0 || N % 8 != 0) return PARO_ERR_INVALID_ARG;
   int G = 0;
   if (int st = normalize_group(group_size, K, &G)) return st;
-  if (G != kGroup || krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
+  if (!supported_group(G, K) || krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
   if (N == 0) return PARO_OK;   // nothing to touch: NULL data pointers are fine
   if (w == nullptr || scales == nullptr || qweight == nullptr || qzeros == nullptr) return PARO_ERR_INVALID_ARG;
   if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
@@ -576,7 +624,7 @@ int paro_quantize_w4(const void* w, const float* channel_scales, const int16_t* 
   if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
   const RtQuant qo{static_cast<const __half*>(scales), qweight, qzeros};
   return launch_rotate_tmem<true>(static_cast<const __half*>(w), nullptr, N, K, channel_scales, pairs, theta,
-                                  krot, qo, reinterpret_cast<cudaStream_t>(stream));
+                                  krot, G, qo, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qweight,
@@ -624,7 +672,7 @@ int paro_unpack_awq(const int32_t* qweight, const int32_t* qzeros, uint8_t* code
 
 size_t paro_w4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int group_size) {
   if (check_linear_shape(M, K, N, group_size) != PARO_OK) return 0;
-  return make_plan(M, K, N).total;
+  return make_plan(M, K, N, group_of(group_size, K)).total;
 }
 
 }  // extern "C"
@@ -651,13 +699,7 @@ int check_linear_args(const void* x, const void* y, int64_t M, int64_t K, int64_
 
 // Shared memory of the GEMV layout of a plan, for `gmax` groups per CTA.
 size_t gemv_smem(const LinearPlan& p, int gmax) {
-  const bool one = p.nt == 1;
-  switch (p.variant) {
-    case 0: return one ? GemvLayout<1, 2, 256, 4>::smem(gmax) : GemvLayout<2, 2, 256, 4>::smem(gmax);
-    case 2: return one ? GemvLayout<1, 4, 128, 8>::smem(gmax) : GemvLayout<2, 4, 128, 8>::smem(gmax);
-    case 5: return one ? GemvLayout<1, 4, 64, 8>::smem(gmax) : GemvLayout<2, 4, 64, 8>::smem(gmax);
-    default: return one ? GemvLayout<1, 2, 128, 4>::smem(gmax) : GemvLayout<2, 2, 128, 4>::smem(gmax);
-  }
+  return gemv_layout_bytes(p.variant, p.nt, gmax, gmax * (kGroup / p.gsz));
 }
 
 int plan_tile(const LinearPlan& p) { return p.variant == 0 ? 256 : (p.variant == 5 ? 64 : 128); }
@@ -666,10 +708,10 @@ int plan_tile(const LinearPlan& p) { return p.variant == 0 ? 256 : (p.variant ==
 // widest member for all of them, taken only when the whole grid is resident
 // at once with that plan's footprint (larger groups gain nothing from sharing
 // a launch: each member already fills the GPU).
-bool group_plan(int64_t M, int64_t K, const paro_linear* lin, int count, LinearPlan* out) {
+bool group_plan(int64_t M, int64_t K, const paro_linear* lin, int count, int gsz, LinearPlan* out) {
   int64_t widest = 0;
   for (int i = 0; i < count; ++i) widest = std::max(widest, lin[i].N);
-  LinearPlan p = make_plan(M, K, widest);
+  LinearPlan p = make_plan(M, K, widest, gsz);
   if (!p.decode) return false;
   const int tile = plan_tile(p);
   int64_t tiles = 0;
@@ -700,7 +742,8 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
     return st;
   if (M == 0) return PARO_OK;   // empty batch: nothing to read or write
 
-  const LinearPlan plan = make_plan(M, K, N);
+  const int G = group_of(group_size, K);
+  const LinearPlan plan = make_plan(M, K, N, G);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool rotate = krot > 0 || channel_scales != nullptr;
@@ -716,8 +759,8 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
     __half* xr = reinterpret_cast<__half*>(ws + plan.off_xr);
     if (plan.rot_tc) {
       const RotTcMember one{channel_scales, pairs, theta, krot, xr, reinterpret_cast<__half*>(ws + plan.off_rt)};
-      if (int st = launch_rotate_tc(xa, &one, 1, M, K, s)) return st;
-    } else if (int st = launch_rotate(xa, xr, M, K, channel_scales, pairs, theta, krot, s)) {
+      if (int st = launch_rotate_tc(xa, &one, 1, M, K, G, s)) return st;
+    } else if (int st = launch_rotate(xa, xr, M, K, channel_scales, pairs, theta, krot, G, s)) {
       return st;
     }
     xa = xr;
@@ -727,7 +770,7 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
   __half* yy = static_cast<__half*>(y);
   if (!plan.decode)
     return launch_w4_prefill(xa, yy, M, K, N, qweight, qzeros, static_cast<const __half*>(scales),
-                             b, s, pdl);
+                             b, G, s, pdl);
 
   const GemvLinearArgs one{qweight, qzeros, scales, xa, b, yy, N};
   return dispatch_gemv(plan, &one, 1, M, K, s, pdl);
@@ -762,7 +805,7 @@ size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, cons
   size_t total = 0;
   for (int i = 0; i < count; ++i) {
     if (check_linear_shape(M, K, linears[i].N, group_size) != PARO_OK) return 0;
-    total += make_plan(M, K, linears[i].N).total;
+    total += make_plan(M, K, linears[i].N, group_of(group_size, K)).total;
   }
   return total;
 }
@@ -784,10 +827,11 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
   if (M == 0) return 0;
   // prefill batches rotating on the tensor cores: one R' build and one X R'
   // launch for all rotating members, then one GEMM each
-  if (make_plan(M, K, linears[0].N).rot_tc) return (rot > 0 ? 2 : 0) + count;
+  const int G = group_of(group_size, K);
+  if (make_plan(M, K, linears[0].N, G).rot_tc) return (rot > 0 ? 2 : 0) + count;
   LinearPlan gp;
   // one after another: each rotating member launches its rotation and its GEMV / GEMM
-  if (count == 1 || !group_plan(M, K, linears, count, &gp)) return rot + count;
+  if (count == 1 || !group_plan(M, K, linears, count, G, &gp)) return rot + count;
   return (rot > 0 ? (rows_ok ? 1 : rot) : 0) + 1;
 }
 
@@ -809,10 +853,11 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
   if (any_rotate && !aligned(workspace, 256)) return PARO_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // member i's X_r lives at workspace + i * per (all members share M and K)
-  const size_t per = make_plan(M, K, linears[0].N).total;
+  const int G = group_of(group_size, K);
+  const size_t per = make_plan(M, K, linears[0].N, G).total;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
-  const LinearPlan first = make_plan(M, K, linears[0].N);
+  const LinearPlan first = make_plan(M, K, linears[0].N, G);
   if (count > 1 && first.rot_tc) {
     // prefill: every rotating member's X_r in one R' build + one X R' launch
     // (x is read once per tile for all of them), then one GEMM per member
@@ -831,11 +876,11 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
       xs[i] = xr;
     }
     if (nrot > 0)
-      if (int st = launch_rotate_tc(static_cast<const __half*>(x), rm, nrot, M, K, s)) return st;
+      if (int st = launch_rotate_tc(static_cast<const __half*>(x), rm, nrot, M, K, G, s)) return st;
     for (int i = 0; i < count; ++i) {
       const paro_linear& l = linears[i];
       if (int st = launch_w4_prefill(xs[i], static_cast<__half*>(l.y), M, K, l.N, l.qweight, l.qzeros,
-                                     static_cast<const __half*>(l.scales), static_cast<const __half*>(l.bias), s,
+                                     static_cast<const __half*>(l.scales), static_cast<const __half*>(l.bias), G, s,
                                      true))
         return st;
     }
@@ -843,7 +888,7 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
   }
 
   LinearPlan gp;
-  if (count == 1 || !group_plan(M, K, linears, count, &gp)) {
+  if (count == 1 || !group_plan(M, K, linears, count, G, &gp)) {
     // one call per member, each with its own slice of the workspace; a member
     // that shares an earlier member's rotation reads that member's X_r
     for (int i = 0; i < count; ++i) {
@@ -882,11 +927,11 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
   }
   if (nrot > 0) {
     if (rows_ok) {
-      if (int st = launch_rotate_rows(xa, rb, nrot, M, K, max_krot, s)) return st;
+      if (int st = launch_rotate_rows(xa, rb, nrot, M, K, max_krot, G, s)) return st;
     } else {
       for (int r = 0; r < nrot; ++r)
         if (int st = launch_rotate(xa, rb.op[r].xr, M, K, rb.op[r].cs, rb.op[r].pairs, rb.op[r].theta,
-                                   rb.op[r].krot, s))
+                                   rb.op[r].krot, G, s))
           return st;
     }
   }

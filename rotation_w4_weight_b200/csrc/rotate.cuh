@@ -27,21 +27,35 @@ struct RotParam {
   int i, j;
 };
 
-// Stage tables of group `grp` -> shared memory.  Indices outside 0..127 are
-// masked (so no access can leave the tile) and flagged in the status word.
+// The kernels work on 128-channel tiles; a tile holds 128 / G rotation groups
+// (G = 16, 32, 64 or 128).  Pair p of a tile's stage (entries 2p, 2p+1 of the
+// tile's slice of the pair table, angle p of its slice of theta) belongs to
+// the tile's group 2p / G, and its group-local indices become tile channels
+// by that group's offset.  An index outside 0..G-1 is masked to the group (so
+// no access can leave it) and flagged in the status word.
+__device__ __forceinline__ void tile_pair(uint32_t raw, int p, int gsz, int* i, int* j) {
+  uint32_t a = raw & 0xFFFFu, b = raw >> 16;
+  if ((a | b) >= (uint32_t)gsz) {
+    flag_error(kErrPairIndex);
+    a &= (uint32_t)(gsz - 1);
+    b &= (uint32_t)(gsz - 1);
+  }
+  const int off = (2 * p) & ~(gsz - 1);           // first channel of the pair's group in the tile
+  *i = (int)a + off;
+  *j = (int)b + off;
+}
+
+// Stage tables of tile `grp` -> shared memory.
 __device__ __forceinline__ void load_rot_params(RotParam* prm, const int16_t* __restrict__ pairs,
                                                 const float* __restrict__ theta, int K, int krot,
-                                                int grp, int tid, int nthreads) {
+                                                int grp, int gsz, int tid, int nthreads) {
   for (int idx = tid; idx < krot * (kGroup / 2); idx += nthreads) {
     const int s = idx / (kGroup / 2);
     const int p = idx % (kGroup / 2);
-    const int16_t* ps = pairs + (size_t)s * K + (size_t)grp * kGroup + 2 * p;
-    int i = ps[0], j = ps[1];
-    if ((unsigned)i >= (unsigned)kGroup || (unsigned)j >= (unsigned)kGroup) {
-      flag_error(kErrPairIndex);
-      i &= kGroup - 1;
-      j &= kGroup - 1;
-    }
+    const uint32_t raw =
+        *reinterpret_cast<const uint32_t*>(pairs + (size_t)s * K + (size_t)grp * kGroup + 2 * p);
+    int i, j;
+    tile_pair(raw, p, gsz, &i, &j);
     float sn, cs;
     rot_sincos(theta[(size_t)s * (K / 2) + (size_t)grp * (kGroup / 2) + p], &sn, &cs);
     prm[idx] = RotParam{cs, sn, i, j};
@@ -61,7 +75,7 @@ struct RotTile {
 template <int ROWS>
 __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
     const __half* x, __half* xr, const float* __restrict__ cs,
-    const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot) {
+    const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot, int gsz) {
   using T = RotTile<ROWS>;
   // Programmatic dependent launch: the GEMV that follows may launch at once and
   // stream its weights while this kernel works.  The stage tables are layer
@@ -78,7 +92,7 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
-  load_rot_params(prm, pairs, theta, K, krot, grp, tid, kRotThreads);
+  load_rot_params(prm, pairs, theta, K, krot, grp, gsz, tid, kRotThreads);
   pdl_wait_primary();
 
   // ---- load + scale: item = (8-channel chunk v, row r), rows fastest
@@ -180,7 +194,7 @@ struct RrBatch {
 };
 
 __global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(const RrBatch batch, const __half* x,
-                                                                    int M, int K) {
+                                                                    int M, int K, int gsz) {
   pdl_launch_dependents();                         // the GEMV may start streaming weights
   RrOperand o = batch.op[0];
 #pragma unroll
@@ -209,12 +223,8 @@ __global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(const RrBatc
   for (int idx = tid; idx < krot * 64; idx += blockDim.x) {
     const int st = idx >> 6, p = idx & 63;
     const uint32_t pr = *reinterpret_cast<const uint32_t*>(pairs + (size_t)st * K + (size_t)grp * kGroup + 2 * p);
-    uint32_t i = pr & 0xFFFFu, j = pr >> 16;
-    if ((i | j) >= 128u) {                         // masked to the group, flagged
-      flag_error(kErrPairIndex);
-      i &= 127u;
-      j &= 127u;
-    }
+    int i, j;
+    tile_pair(pr, p, gsz, &i, &j);                 // masked to the group, flagged
     float sn, c;
     rot_sincos(theta[(size_t)st * (K / 2) + (size_t)grp * 64 + p], &sn, &c);
     partner[st * 128 + i] = (uint8_t)j;

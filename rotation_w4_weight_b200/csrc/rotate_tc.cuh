@@ -60,7 +60,8 @@ struct RbBatch {
 
 // grid (K/128, 128/kRbRows, members), block kRbThreads; dynamic shared memory
 // for the largest krot of the batch.
-__global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_constant__ RbBatch batch, int K) {
+__global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_constant__ RbBatch batch, int K,
+                                                                int gsz) {
   // The rotation that follows waits for this kernel's completion; let it
   // launch and set itself up meanwhile.
   pdl_launch_dependents();
@@ -78,7 +79,7 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_con
 
   // stage tables of the group (layer constants: read before waiting for the
   // kernel ahead); indices outside the group are masked and flagged
-  load_rot_params(prm, pairs, theta, K, krot, grp, tid, kRbThreads);
+  load_rot_params(prm, pairs, theta, K, krot, grp, gsz, tid, kRbThreads);
   // basis rows r0 .. r0+31, scaled: row r has cs[r0 + r] at channel r0 + r
   for (int idx = tid; idx < kRbRows * kGroup; idx += kRbThreads) {
     const int r = idx >> 7, c = idx & (kGroup - 1);

@@ -74,9 +74,9 @@ constexpr size_t kRtMinSmem = 80 * 1024; // above a third of an SM's shared memo
 
 // Output of the quantising instantiation (rows = N output channels).
 struct RtQuant {
-  const __half* scales;   // [K/128, N] quantiser scales
+  const __half* scales;   // [K/G, N] quantiser scales
   int32_t* qweight;       // [K, N/8] AWQ words
-  int32_t* qzeros;        // [K/128, N/8] AWQ words (all 8)
+  int32_t* qzeros;        // [K/G, N/8] AWQ words (all 8)
 };
 
 struct RtLayout {
@@ -139,7 +139,7 @@ __device__ __forceinline__ uint32_t rt_awq_word(uint32_t lo, uint32_t hi) {
 template <bool ABS, bool QUANT>
 __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kernel(
     const __grid_constant__ CUtensorMap tmX, __half* xr, const float* __restrict__ cs,
-    const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot,
+    const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot, int gsz,
     const RtQuant qo) {
   using L = RtLayout;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -199,12 +199,8 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
     const int s = idx >> 6, p = idx & 63, u = p >> 1, w = p & 1;
     const uint32_t pr =
         *reinterpret_cast<const uint32_t*>(pairs + (size_t)s * K + (size_t)grp * kGroup + 2 * p);
-    int i = (int)(int16_t)(pr & 0xFFFFu), j = (int)(int16_t)(pr >> 16);
-    if ((unsigned)i >= 128u || (unsigned)j >= 128u) {
-      flag_error(kErrPairIndex);
-      i &= 127;
-      j &= 127;
-    }
+    int i, j;
+    tile_pair(pr, p, gsz, &i, &j);                   // tile channels of the pair's group
     praw[idx] = (uint32_t)i | ((uint32_t)j << 16);
     float sn, c;
     rot_sincos(theta[(size_t)s * (K / 2) + (size_t)grp * 64 + p], &sn, &c);
@@ -413,13 +409,20 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
     if constexpr (QUANT) {
       // ---- codes of row r (an output channel), channels SW*h .. SW*h+SW-1,
       // transposed into shared memory; then 8 AWQ words per thread
-      float sc = row < M ? __half2float(qo.scales[(size_t)grp * M + row]) : 1.0f;
-      sc = fminf(fmaxf(sc, 1e-5f), 1e5f);
-      const float inv = 1.0f / sc;
+      // quantiser scale of each 16-channel chunk (a chunk lies in one group of
+      // G >= 16 channels): scales row tile * 128 / G + channel / G
+      float inv[SW / 16];
+#pragma unroll
+      for (int k = 0; k < SW / 16; ++k) {
+        const int qg = (grp * kGroup + SW * h + 16 * k) / gsz;
+        float sc = row < M ? __half2float(qo.scales[(size_t)qg * M + row]) : 1.0f;
+        sc = fminf(fmaxf(sc, 1e-5f), 1e5f);
+        inv[k] = 1.0f / sc;
+      }
       const uint32_t cb = smem_u32(sb + L::codes_off(krot)) + (uint32_t)(SW * h) * 128u + (uint32_t)r;
 #pragma unroll
       for (int i = 0; i < SW; ++i) {
-        int q = __float2int_rn(__uint_as_float(v[i]) * inv);
+        int q = __float2int_rn(__uint_as_float(v[i]) * inv[i / 16]);
         q = min(max(q, -8), 7) + 8;
         asm volatile("st.shared.u8 [%0], %1;" ::"r"(cb + (uint32_t)i * 128u), "r"(q) : "memory");
       }
@@ -435,7 +438,11 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
                      : "memory");
         if (wcol < nw) qo.qweight[(size_t)(grp * kGroup + k) * nw + wcol] = (int32_t)rt_awq_word(lo, hi);
       }
-      if (tid < 16 && tile * 16 + tid < nw) qo.qzeros[(size_t)grp * nw + tile * 16 + tid] = (int32_t)0x88888888u;
+      // zero words of the tile's 128 / G quantisation groups: all code 8
+      for (int z = tid; z < 16 * (kGroup / gsz); z += kRtThreads) {
+        const int zr = z >> 4, zc = tile * 16 + (z & 15);
+        if (zc < nw) qo.qzeros[(size_t)(grp * (kGroup / gsz) + zr) * nw + zc] = (int32_t)0x88888888u;
+      }
     } else if (row < M) {
       // ---- fp16 (round to nearest), row r, channels SW*h .. SW*h+SW-1
       __half* dstp = xr + (size_t)row * K + (size_t)grp * kGroup + SW * h;

@@ -19,6 +19,9 @@
 // Consumer warps are 4 column slices (64 columns each) x KP k-parts; k-part p
 // takes the CTA's groups p, p+KP, ... so every warp works on whole groups.
 //
+// Quantisation groups of G = 128, 64, 32 or 16 rows: the fold below runs at
+// the end of every G / 16 k-steps with that group's scales and zero words.
+//
 // MMA mapping (Y^T = W^T X_r^T: weights are the 16-row A operand, tokens the
 // 8-wide B operand).  Thread (g = lane/4, t = lane%4) of column slice c owns
 // word column wcol = 8c + g, i.e. columns 8*wcol .. 8*wcol+7; m-tile j's rows g
@@ -71,15 +74,17 @@ struct GemvLayout {
   static constexpr int XG_BYTES = 2 * MP * 128;           // X_r of one group
   static constexpr int X_OFF = STAGES * STAGE;
   static constexpr int INBOX_BYTES = KP * MP * NTILE * 4;   // partials [S][KP][MP][NTILE/S]
+  // scales and zero words hold gr = gmax * 128 / G quantisation-group rows
   __host__ __device__ static constexpr int s_off(int gmax) { return X_OFF + gmax * XG_BYTES; }
-  __host__ __device__ static constexpr int z_off(int gmax) { return s_off(gmax) + gmax * NTILE * 2; }
-  __host__ __device__ static constexpr int inbox_off(int gmax) {
-    return ((z_off(gmax) + gmax * WORDS * 4 + 1023) / 1024) * 1024;
+  __host__ __device__ static constexpr int z_off(int gmax, int gr) { return s_off(gmax) + gr * NTILE * 2; }
+  __host__ __device__ static constexpr int inbox_off(int gmax, int gr) {
+    return ((z_off(gmax, gr) + gr * WORDS * 4 + 1023) / 1024) * 1024;
   }
   // barriers: full[STAGES], empty[STAGES], consts, X_r, inbox
-  __host__ __device__ static constexpr int bar_off(int gmax) { return inbox_off(gmax) + INBOX_BYTES; }
-  __host__ __device__ static constexpr int smem(int gmax) { return bar_off(gmax) + 8 * (2 * STAGES + 3) + 1024; }
-  static_assert(smem(kGvMaxGroups) <= 227 * 1024, "shared memory per CTA");
+  __host__ __device__ static constexpr int bar_off(int gmax, int gr) { return inbox_off(gmax, gr) + INBOX_BYTES; }
+  __host__ __device__ static constexpr int smem(int gmax, int gr) {
+    return bar_off(gmax, gr) + 8 * (2 * STAGES + 3) + 1024;
+  }
   static_assert(STAGES <= kGvMaxStages, "too many stages");
   // 128-byte swizzle needs 128-byte rows; 64-byte rows use the 64-byte swizzle
   static constexpr int ROW_BYTES = WORDS * 4;
@@ -91,8 +96,8 @@ struct GemvLayout {
 struct alignas(64) GemvOperand {
   CUtensorMap w;          // qweight [K, N/8] int32, box {NTILE/8 words, 128 rows}
   CUtensorMap x;          // X_r [M, K] fp16 as [K/64][M][64], box {64, MP, 2 gmax}
-  CUtensorMap s;          // scales [K/128, N] fp16, box {NTILE, gmax}
-  CUtensorMap z;          // qzeros [K/128, N/8] int32, box {NTILE/8, gmax}
+  CUtensorMap s;          // scales [K/G, N] fp16, box {NTILE, gmax * 128 / G}
+  CUtensorMap z;          // qzeros [K/G, N/8] int32, box {NTILE/8, gmax * 128 / G}
   const __half* bias;     // [N] or nullptr
   __half* y;              // [M, N]
   int n;                  // output columns
@@ -114,7 +119,7 @@ __device__ __forceinline__ void gv_unpack4(uint32_t m, uint32_t (&e)[4]) {
 
 template <int NT, int KP, int NTILE, int STAGES, int NL>
 __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kernel(
-    const __grid_constant__ GemvBatch<NL> ops, int M, int K, int gmax) {
+    const __grid_constant__ GemvBatch<NL> ops, int M, int K, int gmax, int gq) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
   // this CTA's linear (selected by constant offsets into the parameter block)
   const GemvOperand* op = &ops.op[0];
@@ -138,7 +143,10 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // 1024-byte aligned base, derived on the shared array so every access stays LDS/STS
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t base = smem_u32(sbase);
-  const uint32_t full0 = base + L::bar_off(gmax);
+  // gq = 128 / G quantisation groups per 128-row group (G = 128, 64, 32, 16);
+  // spq = G / 16 k-steps of 16 rows each
+  const int gr = gmax * gq, spq = 8 / gq;
+  const uint32_t full0 = base + L::bar_off(gmax, gr);
   const uint32_t empty0 = full0 + 8 * kGvStages;
   const uint32_t cbar = empty0 + 8 * kGvStages;   // scales + zero words
   const uint32_t xbar = cbar + 8;                  // X_r
@@ -194,9 +202,9 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       const int pre = min(kGvStages, ng);
       // the tensor maps' boxes hold gmax groups (the largest range of any CTA;
       // rows past this CTA's range are loaded and not used)
-      mbar_arrive_expect_tx(cbar, (uint32_t)(gmax * (NTILE * 2 + L::WORDS * 4)));
-      tma_load_2d(base + L::s_off(gmax), tmS, cbar, n0, g_begin);
-      tma_load_2d(base + L::z_off(gmax), tmZ, cbar, n0 / 8, g_begin);
+      mbar_arrive_expect_tx(cbar, (uint32_t)(gr * (NTILE * 2 + L::WORDS * 4)));
+      tma_load_2d(base + L::s_off(gmax), tmS, cbar, n0, g_begin * gq);
+      tma_load_2d(base + L::z_off(gmax, gr), tmZ, cbar, n0 / 8, g_begin * gq);
       for (int i = 0; i < pre; ++i) {
         const uint32_t bar = full0 + 8 * i;
         mbar_arrive_expect_tx(bar, L::W_BYTES);
@@ -238,7 +246,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       }
     const uint32_t ones[4] = {kGvOnes, kGvOnes, kGvOnes, kGvOnes};
     const uint32_t sq = base + (uint32_t)L::s_off(gmax);   // scales of the range
-    const uint32_t zq = base + (uint32_t)L::z_off(gmax);   // zero words of the range
+    const uint32_t zq = base + (uint32_t)L::z_off(gmax, gr);   // zero words of the range
 
     // scales, zero words and X_r of every group of the range (once)
     bool consts_ready = mbar_wait_bounded(cbar, 0);
@@ -249,9 +257,6 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       const uint32_t stq = base + (uint32_t)(s * L::STAGE);
       const bool ready = mbar_wait_bounded(full0 + 8 * s, (i / kGvStages) & 1) && consts_ready;
       if (ready) {
-        // group constants for this thread's 8 columns
-        const uint32_t zw = lds32(zq + (uint32_t)((i * L::WORDS + wcol) * 4));
-        const uint4 s8 = lds128(sq + (uint32_t)(i * NTILE * 2 + wcol * 16));
         float cg[4][NT][4];
         float rs[NT][4];
 #pragma unroll
@@ -273,42 +278,50 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
           gv_unpack4(prmt(w0, w1, 0x7632), ehi01);
           gv_unpack4(prmt(w8, w9, 0x5410), elo89);
           gv_unpack4(prmt(w8, w9, 0x7632), ehi89);
+          // the first k-step of a quantisation group starts its sums at zero
+          const bool first = (ks & (spq - 1)) == 0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint32_t a[4] = {elo01[j], ehi01[j], elo89[j], ehi89[j]};
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              if (ks == 0) mma_16816_zc(cg[j][nt], a, b0[nt], b1[nt]);
+              if (first) mma_16816_zc(cg[j][nt], a, b0[nt], b1[nt]);
               else mma_16816(cg[j][nt], a, b0[nt], b1[nt]);
             }
           }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            if (ks == 0) mma_16816_zc(rs[nt], ones, b0[nt], b1[nt]);
+            if (first) mma_16816_zc(rs[nt], ones, b0[nt], b1[nt]);
             else mma_16816(rs[nt], ones, b0[nt], b1[nt]);
+          }
+          if ((ks & (spq - 1)) == spq - 1) {
+            // end of a quantisation group: zero-point correction and group
+            // scale, in fp32, with this thread's 8 columns' constants
+            const int qrow = i * gq + ks / spq;
+            const uint32_t zw = lds32(zq + (uint32_t)((qrow * L::WORDS + wcol) * 4));
+            const uint4 s8 = lds128(sq + (uint32_t)(qrow * NTILE * 2 + wcol * 16));
+            const uint32_t sw[4] = {s8.x, s8.y, s8.z, s8.w};   // (s[2j], s[2j+1])
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int sh = (j & 1) ? 4 : 0;
+              const float zl = 1024.f + (float)(((zw >> (4 * j)) & 0xFu) << sh);
+              const float zh = 1024.f + (float)(((zw >> (16 + 4 * j)) & 0xFu) << sh);
+              float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sw[j]));
+              if (j & 1) sf.x *= 0.0625f, sf.y *= 0.0625f;
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                const float r0 = rs[nt][0], r1 = rs[nt][1];   // row sums of tokens 2t, 2t+1
+                acc[j][nt][0] = fmaf(sf.x, fmaf(-zl, r0, cg[j][nt][0]), acc[j][nt][0]);
+                acc[j][nt][1] = fmaf(sf.x, fmaf(-zl, r1, cg[j][nt][1]), acc[j][nt][1]);
+                acc[j][nt][2] = fmaf(sf.y, fmaf(-zh, r0, cg[j][nt][2]), acc[j][nt][2]);
+                acc[j][nt][3] = fmaf(sf.y, fmaf(-zh, r1, cg[j][nt][3]), acc[j][nt][3]);
+              }
+            }
           }
         }
         // this warp is done reading the stage
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
-        // zero-point correction and group scale, in fp32
-        const uint32_t sw[4] = {s8.x, s8.y, s8.z, s8.w};   // (s[2j], s[2j+1])
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int sh = (j & 1) ? 4 : 0;
-          const float zl = 1024.f + (float)(((zw >> (4 * j)) & 0xFu) << sh);
-          const float zh = 1024.f + (float)(((zw >> (16 + 4 * j)) & 0xFu) << sh);
-          float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sw[j]));
-          if (j & 1) sf.x *= 0.0625f, sf.y *= 0.0625f;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const float r0 = rs[nt][0], r1 = rs[nt][1];   // row sums of tokens 2t, 2t+1
-            acc[j][nt][0] = fmaf(sf.x, fmaf(-zl, r0, cg[j][nt][0]), acc[j][nt][0]);
-            acc[j][nt][1] = fmaf(sf.x, fmaf(-zl, r1, cg[j][nt][1]), acc[j][nt][1]);
-            acc[j][nt][2] = fmaf(sf.y, fmaf(-zh, r0, cg[j][nt][2]), acc[j][nt][2]);
-            acc[j][nt][3] = fmaf(sf.y, fmaf(-zh, r1, cg[j][nt][3]), acc[j][nt][3]);
-          }
-        }
       } else {
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);   // keep the producer moving
@@ -330,7 +343,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // addressed to it has landed.
   const int cols = kGvTile / S;                    // columns owned by each CTA of the cluster
   const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
-  const uint32_t inbox = base + L::inbox_off(gmax);  // fp32 [S][KP][MP][cols]
+  const uint32_t inbox = base + L::inbox_off(gmax, gr);  // fp32 [S][KP][MP][cols]
   __syncwarp();
   if (S > 1) cluster_wait_acquire();               // every peer's inbox barrier is set up
   if (warp != 0) {
@@ -377,7 +390,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // (from it or to it)
   __syncwarp();
   if (S > 1) cluster_arrive_release();
-  const uint32_t box = base + (uint32_t)L::inbox_off(gmax);
+  const uint32_t box = base + (uint32_t)L::inbox_off(gmax, gr);
   for (int idx = tid; idx < nq; idx += L::THREADS) {
     const int tl = idx / (cols / 4);
     const int c = 4 * (idx % (cols / 4));

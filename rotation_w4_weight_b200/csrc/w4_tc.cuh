@@ -1,8 +1,10 @@
 // Prefill W4 GEMM on the sm_100a tensor cores (tcgen05 / TMEM), M > 16 token rows.
+// Quantisation groups of G = 128, 64, 32 or 16 rows (scales and zero words of
+// the 64-row k-block's max(1, 64 / G) groups come with each TMA stage).
 //
 // What it computes (GPTQModel wiki page "ParoQuant", "Activation and weight
 // transforms" and "Triton plans and tuning"):
-//   Y[m, n] = sum_k X_r[m, k] * (q[k, n] - z[k/128, n]) * s[k/128, n] + b[n]
+//   Y[m, n] = sum_k X_r[m, k] * (q[k, n] - z[k/G, n]) * s[k/G, n] + b[n]
 //
 // CTA tile: 256 token rows x 256 output columns, K in blocks of 64, as two
 // 128-token accumulators that share every dequantised weight tile (the int4
@@ -49,26 +51,32 @@ constexpr int kTcThreads = 32 * (2 + kTcDequantWarps);
 constexpr int kTcBSbo = 1040;            // B: bytes between 8-row groups
 constexpr int kTcBLbo = 128;             // B: bytes between k-chunks
 
-struct TcLayout {
+// SR = scale / zero rows per 64-row k-block: 1 for G >= 64, 64 / G below
+// (G = 32: 2, G = 16: 4, which leaves room for only 2 dequantised B buffers).
+template <int SR>
+struct TcLayoutT {
+  static constexpr int BBUFS = SR >= 4 ? 2 : kTcBBufs;
   // TMA stage (1024-aligned): A | packed weights | scales | zeros
   static constexpr int A_OFF = 0;                          // 32768 B
   static constexpr int A_BLOCK = kTcBM * kTcBK * 2;         // one token block
   static constexpr int A_BYTES = kTcMB * A_BLOCK;
   static constexpr int WQ_OFF = A_OFF + A_BYTES;           // 8192 B, 1024-aligned
   static constexpr int WQ_BYTES = kTcBK * (kTcBN / 8) * 4;
-  static constexpr int S_OFF = WQ_OFF + WQ_BYTES;          // 512 B
-  static constexpr int S_BYTES = kTcBN * 2;
-  static constexpr int Z_OFF = S_OFF + S_BYTES;            // 128 B
-  static constexpr int Z_BYTES = (kTcBN / 8) * 4;
+  static constexpr int S_OFF = WQ_OFF + WQ_BYTES;          // SR x 512 B
+  static constexpr int S_ROW = kTcBN * 2;
+  static constexpr int S_BYTES = SR * S_ROW;
+  static constexpr int Z_OFF = S_OFF + S_BYTES;            // SR x 128 B
+  static constexpr int Z_ROW = (kTcBN / 8) * 4;
+  static constexpr int Z_BYTES = SR * Z_ROW;
   static constexpr int STAGE = ((Z_OFF + Z_BYTES + 1023) / 1024) * 1024;
   static constexpr int TX_BYTES = A_BYTES + WQ_BYTES + S_BYTES + Z_BYTES;
   // dequantised B buffers after the TMA ring
   static constexpr int B_RING = kTcStages * STAGE;
   static constexpr int B_BYTES = (kTcBN / 8) * kTcBSbo;   // 33280 B
   static constexpr int B_STRIDE = ((B_BYTES + 127) / 128) * 128;
-  static constexpr int BAR_OFF = B_RING + kTcBBufs * B_STRIDE;
+  static constexpr int BAR_OFF = B_RING + BBUFS * B_STRIDE;
   // barriers: tma_full[S], tma_empty[S], b_full[B], b_empty[B], accum_full
-  static constexpr int NBARS = 2 * kTcStages + 2 * kTcBBufs + 1;
+  static constexpr int NBARS = 2 * kTcStages + 2 * BBUFS + 1;
   static constexpr int MISC_OFF = BAR_OFF + 8 * NBARS;
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
@@ -81,11 +89,13 @@ struct TcLayout {
 // instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M=128, N=256
 constexpr uint32_t kTcIdesc = (1u << 4) | ((uint32_t)(kTcBN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
 
+template <int SR>
 __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
-    const __grid_constant__ CUtensorMap tmY, const __half* __restrict__ bias, int M, int N, int K) {
-  using L = TcLayout;
+    const __grid_constant__ CUtensorMap tmY, const __half* __restrict__ bias, int M, int N, int K, int gsz) {
+  using L = TcLayoutT<SR>;
+  constexpr int kTcBBufs = L::BBUFS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t base = smem_u32(sbase);
@@ -138,8 +148,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         const uint32_t st = base + kb * L::STAGE, bar = tma_full0 + 8 * kb;
         mbar_arrive_expect_tx(bar, L::TX_BYTES);
         tma_load_2d(st + L::WQ_OFF, &tmW, bar, n0 / 8, kb * kTcBK);
-        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, (kb * kTcBK) / 128);
-        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, (kb * kTcBK) / 128);
+        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, (kb * kTcBK) / gsz);
       }
       pdl_wait_primary();               // X_r is written by the rotation kernel
       for (int kb = 0; kb < pre; ++kb)
@@ -150,8 +160,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         const uint32_t st = base + s * L::STAGE, bar = tma_full0 + 8 * s;
         mbar_arrive_expect_tx(bar, L::TX_BYTES);
         tma_load_2d(st + L::WQ_OFF, &tmW, bar, n0 / 8, kb * kTcBK);
-        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, (kb * kTcBK) / 128);
-        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, (kb * kTcBK) / 128);
+        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, (kb * kTcBK) / gsz);
         tma_load_2d(st + L::A_OFF, &tmA, bar, kb * kTcBK, tok0);
       }
     }
@@ -204,9 +214,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         const int row = 8 * c + 4 * h + r;
         wv[r] = lds32(stp + (uint32_t)(L::WQ_OFF + row * 128 + ((((w >> 2) ^ (row & 7))) << 4) + (w & 3) * 4));
       }
-      // group zero points and scales of the 8 columns (column j at nibble j/2 + 4 (j & 1))
-      const uint32_t zw = lds32(stp + (uint32_t)(L::Z_OFF + w * 4));
-      const uint4 s8 = lds128(stp + (uint32_t)(L::S_OFF + w * 16));
+      // group zero points and scales of the 8 columns (column j at nibble j/2 + 4 (j & 1));
+      // rows 8c .. 8c+7 of the block lie in quantisation group (8 c) / G of its SR
+      const int sr = SR > 1 ? (8 * c) / gsz : 0;
+      const uint32_t zw = lds32(stp + (uint32_t)(L::Z_OFF + sr * L::Z_ROW + w * 4));
+      const uint4 s8 = lds128(stp + (uint32_t)(L::S_OFF + sr * L::S_ROW + w * 16));
       const uint32_t sw[4] = {s8.x, s8.y, s8.z, s8.w};
       uint32_t outv[8][2];
 #pragma unroll

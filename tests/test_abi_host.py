@@ -62,8 +62,13 @@ def test_linear_argument_validation(L):
     assert lin(L, N=40) == L.PARO_ERR_UNSUPPORTED            # N % 32 (valid for the packer only)
     assert lin(L, K=200) == L.PARO_ERR_INVALID_ARG           # K % G
     assert lin(L, G=3) == L.PARO_ERR_INVALID_ARG             # odd group
-    assert lin(L, G=64) == L.PARO_ERR_UNSUPPORTED
+    # group sizes: 16, 32, 64 and 128 are implemented (checked on the GPU);
+    # other valid ones are refused before any work
+    assert lin(L, G=8) == L.PARO_ERR_UNSUPPORTED
+    assert lin(L, K=384, G=48) == L.PARO_ERR_UNSUPPORTED
+    assert lin(L, G=256) == L.PARO_ERR_UNSUPPORTED
     assert lin(L, K=256, G=-1) == L.PARO_ERR_UNSUPPORTED     # G normalised to K=256
+    assert lin(L, K=64, G=-1) == L.PARO_ERR_UNSUPPORTED      # G = 64, but K must be a multiple of 128
     assert lin(L, x=None) == L.PARO_ERR_INVALID_ARG
     assert lin(L, qz=None) == L.PARO_ERR_INVALID_ARG
     assert lin(L, krot=8) == L.PARO_ERR_INVALID_ARG          # pairs/theta missing
@@ -101,7 +106,8 @@ def test_rotate_argument_validation(L):
     assert r(A16, A16, -1, 256, None, None, None, 128, 0, None) == L.PARO_ERR_INVALID_ARG
     assert r(None, A16, 4, 256, None, None, None, 128, 0, None) == L.PARO_ERR_INVALID_ARG
     assert r(A16, A16, 4, 256, None, None, None, 128, 8, None) == L.PARO_ERR_INVALID_ARG
-    assert r(A16, A16, 4, 256, None, A16, A16, 64, 8, None) == L.PARO_ERR_UNSUPPORTED
+    assert r(A16, A16, 4, 256, None, A16, A16, 8, 8, None) == L.PARO_ERR_UNSUPPORTED
+    assert r(A16, A16, 4, 256, None, A16, A16, 256, 8, None) == L.PARO_ERR_UNSUPPORTED
     assert r(A16, A16, 4, 250, None, A16, A16, 128, 8, None) == L.PARO_ERR_INVALID_ARG
     assert r(MIS, A16, 4, 256, None, A16, A16, 128, 8, None) == L.PARO_ERR_ALIGNMENT
     assert r(A16, A16, 0, 256, None, A16, A16, 128, 8, None) == L.PARO_OK
@@ -140,7 +146,7 @@ def test_quantize_argument_validation(L):
     assert q(None, None, A16, A16, A16, A16, A16, 16, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG
     assert q(A16, None, A16, A16, None, A16, A16, 16, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG
     assert q(A16, None, A16, A16, A16, A16, None, 16, 256, 128, 8, None) == L.PARO_ERR_INVALID_ARG
-    assert q(A16, None, A16, A16, A16, A16, A16, 16, 256, 64, 8, None) == L.PARO_ERR_UNSUPPORTED
+    assert q(A16, None, A16, A16, A16, A16, A16, 16, 256, 8, 8, None) == L.PARO_ERR_UNSUPPORTED
     assert q(A16, None, A16, A16, A16, A16, A16, 16, 250, 128, 8, None) == L.PARO_ERR_INVALID_ARG
     assert q(A16, None, A16, A16, A16, A16, A16, 16, 256, 128, 65, None) == L.PARO_ERR_UNSUPPORTED
     assert q(MIS, None, A16, A16, A16, A16, A16, 16, 256, 128, 8, None) == L.PARO_ERR_ALIGNMENT
