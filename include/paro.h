@@ -79,7 +79,7 @@ typedef struct CUstream_st* paro_stream_t;
 typedef enum {
   PARO_OK = 0,
   PARO_ERR_INVALID_ARG = 1,  /* NULL pointer where data is needed, negative size, bad shape */
-  PARO_ERR_UNSUPPORTED = 2,  /* valid per the method but not implemented (G != 128, ...) */
+  PARO_ERR_UNSUPPORTED = 2,  /* valid per the method but not implemented (G not in {16,32,64,128}, ...) */
   PARO_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned (4-byte for fp32/int16 tables) */
   PARO_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than paro_w4_linear_workspace_size */
   PARO_ERR_CUDA = 5,         /* a CUDA launch or query failed */
@@ -137,7 +137,7 @@ int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qwei
  *   pairs, theta    the layer's rotation tables (as for paro_rotate); NULL only when krot == 0
  *   scales          device fp16 [K/G, N] quantiser (= dequantisation) scales
  *   qweight         device int32 [K, N/8]; qzeros device int32 [K/G, N/8] (all 0x88888888)
- *   N >= 0, N % 8 == 0 (N == 0 is a no-op); K % 128 == 0; group_size 128 (or -1 with K == 128);
+ *   N >= 0, N % 8 == 0 (N == 0 is a no-op); K % 128 == 0; group_size 16, 32, 64 or 128 (or -1 with K == 128);
  *   krot 0..64; N * K < 2^31
  * Arithmetic: W * D with D = 1/channel_scales in fp32, the stages as in
  * paro_rotate (fp32, no fp16 rounding of W_r), q = rint(W_r * (1/s)) with ties
