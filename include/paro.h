@@ -17,7 +17,7 @@
  *
  * Tensor layouts (section "Stored tensors"; I = K = in_features,
  * O = N = out_features, G = group size, all row-major, all little-endian):
- *   x, x_r          fp16    [M, K]
+ *   x, x_r          fp16    [M, K]   (bf16 through the *_dt entry points)
  *   channel_scales  fp32    [K]              (may be NULL: all ones)
  *   pairs           int16   [krot, K]        pairs[s, g*G+2p], pairs[s, g*G+2p+1]
  *                                            are the local channels (a, b) of pair p
@@ -27,9 +27,9 @@
  *                                            word w in row k holds column 8w+ORDER[t],
  *                                            ORDER = {0,2,4,6,1,3,5,7}
  *   qzeros          int32   [K/G, N/8]       same packing, 4-bit zero points
- *   scales          fp16    [K/G, N]
- *   bias            fp16    [N]              (may be NULL)
- *   y               fp16    [M, N]
+ *   scales          fp16    [K/G, N]         (same type as x)
+ *   bias            fp16    [N]              (may be NULL; same type as x)
+ *   y               fp16    [M, N]           (same type as x)
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, except the
@@ -61,7 +61,15 @@
  *     128: the kernels work on 128-channel tiles holding 128 / G groups), the
  *     rotation groups and the quantisation groups share G; 0 <= krot <= 64;
  *     N a multiple of 32 (the packer alone needs only N % 8 == 0 and any even
- *     G); fp16 activations/scales/bias.
+ *     G); fp16 or bf16 activations/scales/bias/outputs (one type per call).
+ *   - Activation type.  The plain entry points take fp16.  Each has a *_dt twin
+ *     with one more argument, `dtype` (a paro_dtype), that selects fp16 or bf16
+ *     for every 16-bit floating-point tensor of the call (x, x_r, w, scales,
+ *     bias, y); any other value returns PARO_ERR_INVALID_ARG.  The page's
+ *     "Stored tensors" section fixes no activation type (fp16 is the common
+ *     serving type); the arithmetic is the same for both, only the final
+ *     roundings and the tensor-core operand type change: in bf16 the weights
+ *     (q - z) are still exact and products are still summed in fp32.
  */
 #ifndef PARO_H_
 #define PARO_H_
@@ -86,6 +94,12 @@ typedef enum {
   PARO_ERR_TIMEOUT = 6       /* a device-side wait ran out (see paro_device_status) */
 } paro_status;
 
+/* Type of the 16-bit floating-point tensors of a *_dt call. */
+typedef enum {
+  PARO_DTYPE_F16 = 0,   /* IEEE binary16 */
+  PARO_DTYPE_BF16 = 1   /* bfloat16 */
+} paro_dtype;
+
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char* paro_status_string(int status);
 
@@ -104,13 +118,17 @@ const char* paro_version(void);
  *   krot            number of stages, 0..64 (0 = scaling only)
  * Arithmetic: fp32 on chip; cos/sin of the fp32 angle by the hardware
  * approximation after one reduction into [-pi, pi] (absolute error about
- * 2^-21); one round-to-nearest to fp16 at the end.  Pair indices outside 0..G-1 are
- * masked to 7 bits (so no access leaves the group) and flagged in the device
- * status word; pair tables are not otherwise checked (see paro_validate_pairs).
+ * 2^-21); one round-to-nearest to fp16 (bf16) at the end.  Pair indices outside
+ * 0..G-1 are masked into 0..G-1 (so no access leaves the group) and flagged in
+ * the device status word; pair tables are not otherwise checked (see
+ * paro_validate_pairs).
  */
 int paro_rotate(const void* x, void* x_r, int64_t M, int64_t K, const float* channel_scales,
                 const int16_t* pairs, const float* theta, int group_size, int krot,
                 paro_stream_t stream);
+int paro_rotate_dt(const void* x, void* x_r, int64_t M, int64_t K, const float* channel_scales,
+                   const int16_t* pairs, const float* theta, int group_size, int krot, int dtype,
+                   paro_stream_t stream);
 
 /*
  * paro_pack_awq — pack 4-bit codes into AWQ int32 words (page "ParoQuant",
@@ -150,6 +168,11 @@ int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qwei
 int paro_quantize_w4(const void* w, const float* channel_scales, const int16_t* pairs,
                      const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
                      int64_t N, int64_t K, int group_size, int krot, paro_stream_t stream);
+/* The same with w and scales of type `dtype` (the codes depend only on the
+ * values of w and scales, read exactly in either type). */
+int paro_quantize_w4_dt(const void* w, const float* channel_scales, const int16_t* pairs,
+                        const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
+                        int64_t N, int64_t K, int group_size, int krot, int dtype, paro_stream_t stream);
 
 /* paro_unpack_awq — exact inverse of paro_pack_awq (same shapes, same rules). */
 int paro_unpack_awq(const int32_t* qweight, const int32_t* qzeros, uint8_t* codes,
@@ -180,14 +203,17 @@ size_t paro_w4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int group_
  *   the workspace hold X_r (fp16 [M, K], row-major) until the workspace is used
  *   again; from M >= 65 the next 2*K*128*2 bytes hold the rotation matrices
  *   (below), the rest is scratch.
- *   Arithmetic: rotation in fp32 rounded once to fp16; weights (q - z) exact in
- *   fp16; products and sums in fp32 (tensor cores); y rounded once to fp16.
+ *   Arithmetic: rotation in fp32 rounded once to fp16 (bf16); weights (q - z)
+ *   exact in fp16 (bf16), times the group scale rounded to the activation type
+ *   on the prefill path; products and sums in fp32 (tensor cores); y rounded
+ *   once to fp16 (bf16).
  *   M <= 16 runs the decode GEMV path; larger M the tcgen05 prefill GEMM path.
  *   From M >= 65 the rotation itself runs on the tensor cores: each group's
  *   stages with its channel scales are the 128 x 128 matrix
  *   R' = diag(cs) G_0 ... G_{krot-1}, built per call in fp32 (its 128 basis rows
- *   taken through the stages) and stored as two fp16 parts R' = Rhi + Rlo;
- *   X_r = X Rhi + X Rlo accumulated in fp32 (R' kept to about 2^-22 relative).
+ *   taken through the stages) and stored as two parts of the activation type,
+ *   R' = Rhi + Rlo; X_r = X Rhi + X Rlo accumulated in fp32 (R' kept to about
+ *   2^-22 relative in fp16, about 2^-16 in bf16).
  *   Smaller batches apply the stages pair by pair.  paro_rotate always applies
  *   them pair by pair (it has no workspace for R').
  */
@@ -196,6 +222,13 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
                    const void* bias, const float* channel_scales, const int16_t* pairs,
                    const float* theta, int group_size, int krot, void* workspace,
                    size_t workspace_bytes, paro_stream_t stream);
+/* The same with x, scales, bias and y of type `dtype`; the workspace size does
+ * not depend on the type. */
+int paro_w4_linear_dt(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                      const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                      const void* bias, const float* channel_scales, const int16_t* pairs,
+                      const float* theta, int group_size, int krot, int dtype, void* workspace,
+                      size_t workspace_bytes, paro_stream_t stream);
 
 /*
  * Grouped decoder-layer calls — several linears that read the same x (a
@@ -213,7 +246,7 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
  * separate calls in fp32 summation order only.
  *   linears         HOST array of `count` (1..PARO_MAX_GROUP) member descriptors;
  *                   each member's fields follow paro_w4_linear's rules
- *   x               device fp16 [M, K] shared by all members
+ *   x               device fp16 (or `dtype`) [M, K] shared by all members
  *   workspace       >= paro_w4_linear_group_workspace_size(...) bytes, 256-byte
  *                   aligned (may be NULL when no member rotates)
  */
@@ -222,19 +255,22 @@ typedef struct paro_linear {
   int64_t N;                       /* output features of this member */
   const int32_t* qweight;          /* [K, N/8] */
   const int32_t* qzeros;           /* [K/G, N/8] */
-  const void* scales;              /* fp16 [K/G, N] */
-  const void* bias;                /* fp16 [N] or NULL */
+  const void* scales;              /* fp16 (or dtype) [K/G, N] */
+  const void* bias;                /* fp16 (or dtype) [N] or NULL */
   const float* channel_scales;     /* [K] or NULL */
   const int16_t* pairs;            /* [krot, K]; NULL only when krot == 0 */
   const float* theta;              /* [krot, K/2]; NULL only when krot == 0 */
   int krot;
-  void* y;                         /* fp16 [M, N] output */
+  void* y;                         /* fp16 (or dtype) [M, N] output */
 } paro_linear;
 
 size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, const paro_linear* linears,
                                            int group_size);
 int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
                          int group_size, void* workspace, size_t workspace_bytes, paro_stream_t stream);
+int paro_w4_linear_group_dt(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
+                            int group_size, int dtype, void* workspace, size_t workspace_bytes,
+                            paro_stream_t stream);
 /* Kernel launches paro_w4_linear_group issues for this group (rotations plus
  * GEMV/GEMM launches; 0 for an invalid shape or M == 0).  Host-only query. */
 int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_linear* linears,
@@ -278,6 +314,10 @@ int paro_w4_linear_noalloc(const void* x, void* y, int64_t M, int64_t K, int64_t
                            const int32_t* qweight, const int32_t* qzeros, const void* scales,
                            const void* bias, const float* channel_scales, const int16_t* pairs,
                            const float* theta, int group_size, int krot, paro_stream_t stream);
+int paro_w4_linear_noalloc_dt(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                              const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                              const void* bias, const float* channel_scales, const int16_t* pairs,
+                              const float* theta, int group_size, int krot, int dtype, paro_stream_t stream);
 
 /*
  * paro_validate_pairs — HOST helper (host pointer, synchronous, no GPU work):

@@ -4,14 +4,18 @@ The compute lives in the CUDA library ``libparo_b200.so`` behind the C ABI of
 ``include/paro.h``; this module only marshals torch tensors (device memory and
 streams) into that ABI.  Functions mirror the C entry points:
 
-    rotate            -> paro_rotate
+    rotate            -> paro_rotate / paro_rotate_dt
     pack_awq          -> paro_pack_awq
     unpack_awq        -> paro_unpack_awq
-    w4_linear         -> paro_w4_linear (+ paro_w4_linear_workspace_size)
-    w4_linear_group   -> paro_w4_linear_group (+ paro_w4_linear_group_workspace_size)
-    quantize_w4       -> paro_quantize_w4
+    w4_linear         -> paro_w4_linear / paro_w4_linear_dt (+ paro_w4_linear_workspace_size)
+    w4_linear_group   -> paro_w4_linear_group / paro_w4_linear_group_dt (+ ..._workspace_size)
+    quantize_w4       -> paro_quantize_w4 / paro_quantize_w4_dt
     validate_pairs    -> paro_validate_pairs (host helper)
     device_status     -> paro_device_status
+
+Activations, scales, bias and outputs are fp16 or bf16 (one type per call,
+taken from x): fp16 calls go to the plain entry points, bf16 calls to the
+``*_dt`` twins with ``PARO_DTYPE_BF16``.
 """
 from __future__ import annotations
 
@@ -27,7 +31,8 @@ from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # n
                    paro_quantize_w4, paro_rotate, paro_status_string, paro_unpack_awq,
                    paro_validate_pairs, paro_version, paro_w4_linear, paro_w4_linear_workspace_size,
                    PARO_MAX_GROUP, ParoLinear, paro_w4_linear_group, paro_w4_linear_group_launches,
-                   paro_w4_linear_group_workspace_size)
+                   paro_w4_linear_group_workspace_size, PARO_DTYPE_BF16, paro_rotate_dt, paro_quantize_w4_dt,
+                   paro_w4_linear_dt, paro_w4_linear_group_dt)
 
 __all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
            "w4_linear_group", "w4_linear_group_launches", "quantize_w4", "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
@@ -41,6 +46,16 @@ def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+_ACT_TYPES = (torch.float16, torch.bfloat16)
+
+
+def _act(t: torch.Tensor, name: str):
+    """The activation type of a call (fp16 or bf16), taken from its input."""
+    if t.dtype not in _ACT_TYPES:
+        raise TypeError(f"{name} must be float16 or bfloat16, got {t.dtype}")
+    return t.dtype
 
 
 def _need(t: Optional[torch.Tensor], dtype, name: str, allow_none: bool = False):
@@ -60,7 +75,8 @@ def rotate(x: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: Optio
            theta: Optional[torch.Tensor], group_size: int = 128, krot: Optional[int] = None,
            out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """X_r = rotate(x * channel_scales); ``out`` may be ``x`` (in place)."""
-    _need(x, torch.float16, "x")
+    dt = _act(x, "x")
+    _need(x, dt, "x")
     _need(channel_scales, torch.float32, "channel_scales", True)
     _need(pairs, torch.int16, "pairs", True)
     _need(theta, torch.float32, "theta", True)
@@ -68,9 +84,13 @@ def rotate(x: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: Optio
         krot = 0 if pairs is None else pairs.shape[0]
     if out is None:
         out = torch.empty_like(x)
+    _need(out, dt, "out")
     M, K = x.shape
-    check(paro_rotate(_ptr(x), _ptr(out), M, K, _ptr(channel_scales), _ptr(pairs), _ptr(theta),
-                      group_size, krot, _stream(stream)), "paro_rotate")
+    args = (_ptr(x), _ptr(out), M, K, _ptr(channel_scales), _ptr(pairs), _ptr(theta), group_size, krot)
+    if dt == torch.float16:
+        check(paro_rotate(*args, _stream(stream)), "paro_rotate")
+    else:
+        check(paro_rotate_dt(*args, PARO_DTYPE_BF16, _stream(stream)), "paro_rotate_dt")
     return out
 
 
@@ -93,13 +113,14 @@ def pack_awq(codes: torch.Tensor, zero_codes: Optional[torch.Tensor], group_size
 def quantize_w4(w: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: Optional[torch.Tensor],
                 theta: Optional[torch.Tensor], scales: torch.Tensor, group_size: int = 128,
                 krot: Optional[int] = None, out=None, stream=None):
-    """Float weights w fp16 [N, K] (out x in) -> (qweight int32 [K, N/8], qzeros int32 [K/G, N/8]):
-    W_r = W D R, four-bit symmetric codes with the fp16 quantiser scales [K/G, N], AWQ-packed."""
-    _need(w, torch.float16, "w")
+    """Float weights w fp16/bf16 [N, K] (out x in) -> (qweight int32 [K, N/8], qzeros int32 [K/G, N/8]):
+    W_r = W D R, four-bit symmetric codes with the quantiser scales [K/G, N] (w's type), AWQ-packed."""
+    dt = _act(w, "w")
+    _need(w, dt, "w")
     _need(channel_scales, torch.float32, "channel_scales", True)
     _need(pairs, torch.int16, "pairs", True)
     _need(theta, torch.float32, "theta", True)
-    _need(scales, torch.float16, "scales")
+    _need(scales, dt, "scales")
     if krot is None:
         krot = 0 if pairs is None else pairs.shape[0]
     N, K = w.shape
@@ -108,9 +129,12 @@ def quantize_w4(w: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: 
         out = (torch.empty((K, N // 8), dtype=torch.int32, device=w.device),
                torch.empty((K // G, N // 8), dtype=torch.int32, device=w.device))
     qweight, qzeros = out
-    check(paro_quantize_w4(_ptr(w), _ptr(channel_scales), _ptr(pairs), _ptr(theta), _ptr(scales),
-                           _ptr(qweight), _ptr(qzeros), N, K, group_size, krot, _stream(stream)),
-          "paro_quantize_w4")
+    args = (_ptr(w), _ptr(channel_scales), _ptr(pairs), _ptr(theta), _ptr(scales), _ptr(qweight), _ptr(qzeros),
+            N, K, group_size, krot)
+    if dt == torch.float16:
+        check(paro_quantize_w4(*args, _stream(stream)), "paro_quantize_w4")
+    else:
+        check(paro_quantize_w4_dt(*args, PARO_DTYPE_BF16, _stream(stream)), "paro_quantize_w4_dt")
     return qweight, qzeros
 
 
@@ -138,12 +162,13 @@ def w4_linear(x: torch.Tensor, qweight: torch.Tensor, qzeros: torch.Tensor, scal
               group_size: int = 128, krot: Optional[int] = None,
               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
               stream=None) -> torch.Tensor:
-    """Y = rotate(x * channel_scales) @ dequant(qweight, qzeros, scales) + bias (fp16 out)."""
-    _need(x, torch.float16, "x")
+    """Y = rotate(x * channel_scales) @ dequant(qweight, qzeros, scales) + bias (out in x's type)."""
+    dt = _act(x, "x")
+    _need(x, dt, "x")
     _need(qweight, torch.int32, "qweight")
     _need(qzeros, torch.int32, "qzeros")
-    _need(scales, torch.float16, "scales")
-    _need(bias, torch.float16, "bias", True)
+    _need(scales, dt, "scales")
+    _need(bias, dt, "bias", True)
     _need(channel_scales, torch.float32, "channel_scales", True)
     _need(pairs, torch.int16, "pairs", True)
     _need(theta, torch.float32, "theta", True)
@@ -152,14 +177,19 @@ def w4_linear(x: torch.Tensor, qweight: torch.Tensor, qzeros: torch.Tensor, scal
     M, K = x.shape
     N = qweight.shape[1] * 8
     if out is None:
-        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+        out = torch.empty((M, N), dtype=dt, device=x.device)
+    _need(out, dt, "out")
     need = w4_linear_workspace_size(M, K, N, group_size)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    check(paro_w4_linear(_ptr(x), _ptr(out), M, K, N, _ptr(qweight), _ptr(qzeros), _ptr(scales),
-                         _ptr(bias), _ptr(channel_scales), _ptr(pairs), _ptr(theta), group_size,
-                         krot, _ptr(workspace), ws_bytes, _stream(stream)), "paro_w4_linear")
+    args = (_ptr(x), _ptr(out), M, K, N, _ptr(qweight), _ptr(qzeros), _ptr(scales), _ptr(bias),
+            _ptr(channel_scales), _ptr(pairs), _ptr(theta), group_size, krot)
+    if dt == torch.float16:
+        check(paro_w4_linear(*args, _ptr(workspace), ws_bytes, _stream(stream)), "paro_w4_linear")
+    else:
+        check(paro_w4_linear_dt(*args, PARO_DTYPE_BF16, _ptr(workspace), ws_bytes, _stream(stream)),
+              "paro_w4_linear_dt")
     return out
 
 
@@ -182,8 +212,9 @@ def _members(x: torch.Tensor, members, outs):
     for i, m in enumerate(members):
         _need(m["qweight"], torch.int32, "qweight")
         _need(m["qzeros"], torch.int32, "qzeros")
-        _need(m["scales"], torch.float16, "scales")
-        _need(m.get("bias"), torch.float16, "bias", True)
+        _need(m["scales"], x.dtype, "scales")
+        _need(m.get("bias"), x.dtype, "bias", True)
+        _need(outs[i], x.dtype, "out")
         _need(m.get("channel_scales"), torch.float32, "channel_scales", True)
         _need(m.get("pairs"), torch.int16, "pairs", True)
         _need(m.get("theta"), torch.float32, "theta", True)
@@ -204,18 +235,23 @@ def w4_linear_group(x: torch.Tensor, members, group_size: int = 128, workspace: 
                     out=None, stream=None):
     """Several linears over the same x (q/k/v, gate/up): ``members`` is a list of
     dicts with keys qweight, qzeros, scales and optionally bias, channel_scales,
-    pairs, theta, krot.  Returns the list of fp16 outputs [M, N_i]."""
-    _need(x, torch.float16, "x")
+    pairs, theta, krot.  Returns the list of outputs [M, N_i] in x's type."""
+    dt = _act(x, "x")
+    _need(x, dt, "x")
     M, K = x.shape
     if out is None:
-        out = [torch.empty((M, m["qweight"].shape[1] * 8), dtype=torch.float16, device=x.device)
-               for m in members]
+        out = [torch.empty((M, m["qweight"].shape[1] * 8), dtype=dt, device=x.device) for m in members]
     arr = _members(x, members, out)
     need = int(paro_w4_linear_group_workspace_size(M, K, len(members), arr, group_size))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
-    check(paro_w4_linear_group(_ptr(x), M, K, len(members), arr, group_size, _ptr(workspace),
-                               workspace.numel(), _stream(stream)), "paro_w4_linear_group")
+    if dt == torch.float16:
+        check(paro_w4_linear_group(_ptr(x), M, K, len(members), arr, group_size, _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "paro_w4_linear_group")
+    else:
+        check(paro_w4_linear_group_dt(_ptr(x), M, K, len(members), arr, group_size, PARO_DTYPE_BF16,
+                                      _ptr(workspace), workspace.numel(), _stream(stream)),
+              "paro_w4_linear_group_dt")
     return out
 
 

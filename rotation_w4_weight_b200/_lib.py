@@ -20,12 +20,16 @@ PARO_ERR_WORKSPACE = 4
 PARO_ERR_CUDA = 5
 PARO_ERR_TIMEOUT = 6
 
+PARO_DTYPE_F16 = 0
+PARO_DTYPE_BF16 = 1
+
 EXPORTED = (
     "paro_status_string", "paro_version", "paro_rotate", "paro_pack_awq", "paro_unpack_awq",
     "paro_w4_linear_workspace_size", "paro_w4_linear", "paro_w4_linear_noalloc",
     "paro_validate_pairs", "paro_device_status", "paro_quantize_w4",
     "paro_w4_linear_group_workspace_size", "paro_w4_linear_group", "paro_w4_linear_group_launches",
-    "paro_selftest_wait_timeout",
+    "paro_selftest_wait_timeout", "paro_rotate_dt", "paro_quantize_w4_dt", "paro_w4_linear_dt",
+    "paro_w4_linear_group_dt", "paro_w4_linear_noalloc_dt",
 )
 
 PARO_MAX_GROUP = 4
@@ -60,6 +64,13 @@ _SIGNATURES = {
     "paro_w4_linear_group": (_int, [_vp, _i64, _i64, _int, _vp, _int, _vp, ctypes.c_size_t, _vp]),
     "paro_w4_linear_group_launches": (_int, [_i64, _i64, _int, _vp, _int]),
     "paro_selftest_wait_timeout": (_int, [ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64), _vp]),
+    "paro_rotate_dt": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _int, _int, _int, _vp]),
+    "paro_quantize_w4_dt": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _int, _vp]),
+    "paro_w4_linear_dt": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _int, _int, _int, _vp, ctypes.c_size_t, _vp]),
+    "paro_w4_linear_group_dt": (_int, [_vp, _i64, _i64, _int, _vp, _int, _int, _vp, ctypes.c_size_t, _vp]),
+    "paro_w4_linear_noalloc_dt": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                         _vp, _int, _int, _int, _vp]),
 }
 
 
@@ -94,6 +105,11 @@ paro_w4_linear_group_workspace_size = lib.paro_w4_linear_group_workspace_size
 paro_w4_linear_group = lib.paro_w4_linear_group
 paro_w4_linear_group_launches = lib.paro_w4_linear_group_launches
 paro_selftest_wait_timeout = lib.paro_selftest_wait_timeout
+paro_rotate_dt = lib.paro_rotate_dt
+paro_quantize_w4_dt = lib.paro_quantize_w4_dt
+paro_w4_linear_dt = lib.paro_w4_linear_dt
+paro_w4_linear_group_dt = lib.paro_w4_linear_group_dt
+paro_w4_linear_noalloc_dt = lib.paro_w4_linear_noalloc_dt
 
 
 class ParoError(RuntimeError):

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -244,6 +245,46 @@ __device__ __forceinline__ void rot_sincos(float t, float* s, float* c) {
   __sincosf(t, s, c);
 }
 
+// ---------------------------------------------------------------- activation type
+// The 16-bit type of a call's activations, scales, bias and output: fp16 or
+// bf16.  Pairs travel as 32-bit words; the weights' 4-bit codes unpack into the
+// same type (the tensor cores take both operands of one MMA in one type).
+template <typename T>
+struct Act;
+
+template <>
+struct Act<__half> {
+  static constexpr bool kBf16 = false;
+  // tcgen05 kind::f16 instruction descriptor, A and B type fields (f16 = 0)
+  static constexpr uint32_t kIdescAB = 0u;
+  static constexpr uint32_t kOnes = 0x3C003C00u;     // pair (1, 1)
+  __device__ static __forceinline__ float2 f2(uint32_t v) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&v));
+  }
+  __device__ static __forceinline__ uint32_t p2(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  __device__ static __forceinline__ float f1(__half v) { return __half2float(v); }
+  __device__ static __forceinline__ __half from(float a) { return __float2half_rn(a); }
+};
+
+template <>
+struct Act<__nv_bfloat16> {
+  static constexpr bool kBf16 = true;
+  static constexpr uint32_t kIdescAB = (1u << 7) | (1u << 10);   // A and B type bf16
+  static constexpr uint32_t kOnes = 0x3F803F80u;
+  __device__ static __forceinline__ float2 f2(uint32_t v) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
+  }
+  __device__ static __forceinline__ uint32_t p2(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  __device__ static __forceinline__ float f1(__nv_bfloat16 v) { return __bfloat162float(v); }
+  __device__ static __forceinline__ __nv_bfloat16 from(float a) { return __float2bfloat16_rn(a); }
+};
+
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
@@ -282,6 +323,36 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
+}
+
+__device__ __forceinline__ uint32_t bsub2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t bmul2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// D = A(16x16, row) * B(16x8, col) + D, bf16 inputs, fp32 accumulate (and with a
+// zero accumulator input).
+__device__ __forceinline__ void mma_16816_bf(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_16816_bf_zc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 // D = A(16x16, row) * B(16x8, col) + D, fp16 inputs, fp32 accumulate.

@@ -39,6 +39,13 @@ inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintp
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// ---------------------------------------------------------------- activation type
+// TMA element type of the activation type (loads and stores copy the bits).
+template <typename TA>
+constexpr CUtensorMapDataType tma_dt() {
+  return Act<TA>::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
+
 // ---------------------------------------------------------------- TMA encode
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -77,15 +84,15 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, size_t esize, const voi
 // X as [K/64 chunks][rows][64] (chunk stride 128 bytes, row stride K*2 bytes):
 // box {64 columns, box_rows rows, box_chunks chunks}, 128-byte swizzle.  One
 // copy brings several groups' activation columns in the layout the GEMV reads.
-bool encode_x_chunks(CUtensorMap* map, const void* x, uint64_t rows, uint64_t K, uint32_t box_rows,
-                     uint32_t box_chunks) {
+bool encode_x_chunks(CUtensorMap* map, CUtensorMapDataType dt, const void* x, uint64_t rows, uint64_t K,
+                     uint32_t box_rows, uint32_t box_chunks) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {64, rows, K / 64};
   cuuint64_t strides[2] = {K * 2, 128};
   cuuint32_t box[3] = {64, box_rows, box_chunks};
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+  return fn(map, dt, 3, const_cast<void*>(x), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -222,28 +229,29 @@ int check_rotation_args(const void* x, const void* xr, int64_t M, int64_t K, con
 
 // Warp-per-row rotation of one x for `count` linears (blockIdx.z), decode sizes
 // (M <= 16, every krot <= kRrMaxKrot; max_krot sizes the tables).
-int launch_rotate_rows(const __half* x, const RrBatch& b, int count, int64_t M, int64_t K, int max_krot,
+template <typename TA>
+int launch_rotate_rows(const TA* x, const RrBatch& b, int count, int64_t M, int64_t K, int max_krot,
                        int gsz, cudaStream_t stream) {
-  // always 8 warps: all of them build the tables, warps past the batch then leave
+  // always kRrWarps warps: all of them build the tables, warps past the batch then leave
   const dim3 grid((unsigned)(K / kGroup), (unsigned)((M + kRrWarps - 1) / kRrWarps), (unsigned)count);
-  if (!allow_smem(rotate_rows_kernel, RrLayout::bytes(kRrMaxKrot))) return PARO_ERR_CUDA;
-  return launch(rotate_rows_kernel, grid, dim3(32 * kRrWarps), RrLayout::bytes(max_krot), stream, true, b, x,
-                (int)M, (int)K, gsz);
+  if (!allow_smem(rotate_rows_kernel<TA>, RrLayout::bytes(kRrMaxKrot))) return PARO_ERR_CUDA;
+  return launch(rotate_rows_kernel<TA>, grid, dim3(32 * kRrWarps), RrLayout::bytes(max_krot), stream, true, b,
+                x, (int)M, (int)K, gsz);
 }
 
 // Tensor-memory rotation kernel (and, with QUANT, the weight quantiser): CTAs
 // stay resident over several 128-row tiles of one group (one wave of at most
 // 2 CTAs per SM: the shared-memory floor of the kernel guarantees no more fit).
-template <bool QUANT>
-int launch_rotate_tmem(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
+template <bool QUANT, typename TA>
+int launch_rotate_tmem(const TA* x, TA* xr, int64_t M, int64_t K, const float* cs,
                        const int16_t* pairs, const float* theta, int krot, int gsz, const RtQuant& qo,
                        cudaStream_t stream) {
   const size_t smem = RtLayout::bytes(krot, QUANT);
   const DeviceInfo& di = device_info();
   if (di.sms == 0) return PARO_ERR_CUDA;
   const bool abs_tables = krot <= kRtAbsMaxKrot;
-  if (abs_tables ? !allow_smem(rotate_tmem_kernel<true, QUANT>, RtLayout::bytes(kRtAbsMaxKrot, QUANT))
-                 : !allow_smem(rotate_tmem_kernel<false, QUANT>, RtLayout::bytes(kMaxKrot, QUANT)))
+  if (abs_tables ? !allow_smem(rotate_tmem_kernel<true, QUANT, TA>, RtLayout::bytes(kRtAbsMaxKrot, QUANT))
+                 : !allow_smem(rotate_tmem_kernel<false, QUANT, TA>, RtLayout::bytes(kMaxKrot, QUANT)))
     return PARO_ERR_CUDA;
   const size_t per_block = smem + di.smem_reserved_per_block;
   int per_sm = (int)(di.smem_per_sm / per_block);
@@ -258,27 +266,27 @@ int launch_rotate_tmem(const __half* x, __half* xr, int64_t M, int64_t K, const 
   gy = (ntiles + per_cta - 1) / per_cta;
   if (gy > 65535) gy = 65535;
   CUtensorMap tmX;
-  if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, kRtRows, 64,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!encode_2d(&tmX, tma_dt<TA>(), 2, x, M, K, kRtRows, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return PARO_ERR_CUDA;
   const dim3 grid((unsigned)groups, (unsigned)gy);
   if (abs_tables)
-    return launch(rotate_tmem_kernel<true, QUANT>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
+    return launch(rotate_tmem_kernel<true, QUANT, TA>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
                   pairs, theta, (int)M, (int)K, krot, gsz, qo);
-  return launch(rotate_tmem_kernel<false, QUANT>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
+  return launch(rotate_tmem_kernel<false, QUANT, TA>, grid, dim3(kRtThreads), smem, stream, true, tmX, xr, cs,
                 pairs, theta, (int)M, (int)K, krot, gsz, qo);
 }
 
-int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float* cs,
+template <typename TA>
+int launch_rotate(const TA* x, TA* xr, int64_t M, int64_t K, const float* cs,
                   const int16_t* pairs, const float* theta, int krot, int gsz, cudaStream_t stream) {
   // Large batches: tensor memory as the permutation network.
-  if (M > 64) return launch_rotate_tmem<false>(x, xr, M, K, cs, pairs, theta, krot, gsz, RtQuant{}, stream);
+  if (M > 64) return launch_rotate_tmem<false, TA>(x, xr, M, K, cs, pairs, theta, krot, gsz, RtQuant{}, stream);
   // Decode batches with few stages: one warp per row, no block barrier per stage.
   if (M <= 16 && krot <= kRrMaxKrot) {
     RrBatch b;
     std::memset(&b, 0, sizeof(b));
     b.op[0] = RrOperand{xr, cs, pairs, theta, krot};
-    return launch_rotate_rows(x, b, 1, M, K, krot, gsz, stream);
+    return launch_rotate_rows<TA>(x, b, 1, M, K, krot, gsz, stream);
   }
   // rows per CTA: 4 for decode-sized batches (more CTAs, shorter latency),
   // 32..64 otherwise (conflict-free 32-row warp accesses)
@@ -290,20 +298,20 @@ int launch_rotate(const __half* x, __half* xr, int64_t M, int64_t K, const float
   // the limit is raised once to what the largest krot needs
   switch (rows) {
     case 4:
-      if (!allow_smem(rotate_kernel<4>, rotate_smem_bytes(4, kMaxKrot))) return PARO_ERR_CUDA;
-      return launch(rotate_kernel<4>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
+      if (!allow_smem(rotate_kernel<4, TA>, rotate_smem_bytes(4, kMaxKrot))) return PARO_ERR_CUDA;
+      return launch(rotate_kernel<4, TA>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
                     (int)M, (int)K, krot, gsz);
     case 32:
-      if (!allow_smem(rotate_kernel<32>, rotate_smem_bytes(32, kMaxKrot))) return PARO_ERR_CUDA;
-      return launch(rotate_kernel<32>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
+      if (!allow_smem(rotate_kernel<32, TA>, rotate_smem_bytes(32, kMaxKrot))) return PARO_ERR_CUDA;
+      return launch(rotate_kernel<32, TA>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
                     (int)M, (int)K, krot, gsz);
     case 64:
-      if (!allow_smem(rotate_kernel<64>, rotate_smem_bytes(64, kMaxKrot))) return PARO_ERR_CUDA;
-      return launch(rotate_kernel<64>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
+      if (!allow_smem(rotate_kernel<64, TA>, rotate_smem_bytes(64, kMaxKrot))) return PARO_ERR_CUDA;
+      return launch(rotate_kernel<64, TA>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
                     (int)M, (int)K, krot, gsz);
     default:
-      if (!allow_smem(rotate_kernel<128>, rotate_smem_bytes(128, kMaxKrot))) return PARO_ERR_CUDA;
-      return launch(rotate_kernel<128>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
+      if (!allow_smem(rotate_kernel<128, TA>, rotate_smem_bytes(128, kMaxKrot))) return PARO_ERR_CUDA;
+      return launch(rotate_kernel<128, TA>, grid, block, smem, stream, true, x, xr, cs, pairs, theta,
                     (int)M, (int)K, krot, gsz);
   }
 }
@@ -316,11 +324,12 @@ struct RotTcMember {
   const int16_t* pairs;
   const float* theta;
   int krot;
-  __half* xr;       // X_r [M, K]
-  __half* rt;       // R' parts [2][K][128]
+  void* xr;         // X_r [M, K]
+  void* rt;         // R' parts [2][K][128]
 };
 
-int launch_rotate_tc(const __half* x, const RotTcMember* mem, int count, int64_t M, int64_t K, int gsz,
+template <typename TA>
+int launch_rotate_tc(const TA* x, const RotTcMember* mem, int count, int64_t M, int64_t K, int gsz,
                      cudaStream_t stream) {
   const DeviceInfo& di = device_info();
   if (di.sms == 0) return PARO_ERR_CUDA;
@@ -334,23 +343,21 @@ int launch_rotate_tc(const __half* x, const RotTcMember* mem, int count, int64_t
   for (int i = 0; i < count; ++i) {
     rb.op[i] = RbOperand{mem[i].cs, mem[i].pairs, mem[i].theta, mem[i].rt, mem[i].krot};
     max_krot = std::max(max_krot, mem[i].krot);
-    if (!encode_2d(&rc.t[i].r, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, mem[i].rt, 2 * K, kGroup, 128, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&rc.t[i].y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, mem[i].xr, M, K, 128, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_2d(&rc.t[i].r, tma_dt<TA>(), 2, mem[i].rt, 2 * K, kGroup, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&rc.t[i].y, tma_dt<TA>(), 2, mem[i].xr, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return PARO_ERR_CUDA;
   }
-  if (!allow_smem(rmat_build_kernel, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
-  if (int st = launch(rmat_build_kernel, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows), (unsigned)count),
+  if (!allow_smem(rmat_build_kernel<TA>, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
+  if (int st = launch(rmat_build_kernel<TA>, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows), (unsigned)count),
                       dim3(kRbThreads), rb_smem_bytes(max_krot), stream, true, rb, (int)K, gsz))
     return st;
   CUtensorMap tmX;
-  if (!encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!encode_2d(&tmX, tma_dt<TA>(), 2, x, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return PARO_ERR_CUDA;
-  if (!allow_smem(rotate_tc_kernel, RcLayout::SMEM)) return PARO_ERR_CUDA;
+  if (!allow_smem(rotate_tc_kernel<TA>, RcLayout::SMEM)) return PARO_ERR_CUDA;
   const int64_t jobs = (int64_t)count * groups * tiles;
   const int64_t ctas = jobs < di.sms ? jobs : di.sms;
-  return launch(rotate_tc_kernel, dim3((unsigned)ctas), dim3(kRcThreads), RcLayout::SMEM, stream, true, tmX,
+  return launch(rotate_tc_kernel<TA>, dim3((unsigned)ctas), dim3(kRcThreads), RcLayout::SMEM, stream, true, tmX,
                 rc, count, (int)K, (int)groups, (int)tiles, (long long)jobs);
 }
 
@@ -447,38 +454,39 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N, int gsz) {
 }
 
 // Prefill (M > 16): tcgen05 GEMM, 256 token rows x 256 output columns per CTA.
-template <int SR>
-int launch_w4_prefill_sr(const __half* xa, __half* y, int64_t M, int64_t K, int64_t N,
-                         const int32_t* qweight, const int32_t* qzeros, const __half* scales,
-                         const __half* bias, int gsz, cudaStream_t s, bool pdl) {
+template <int SR, typename TA>
+int launch_w4_prefill_sr(const TA* xa, TA* y, int64_t M, int64_t K, int64_t N,
+                         const int32_t* qweight, const int32_t* qzeros, const TA* scales,
+                         const TA* bias, int gsz, cudaStream_t s, bool pdl) {
   CUtensorMap tmA, tmW, tmS, tmZ, tmY;
-  bool ok = encode_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xa, M, K, kTcMB * kTcBM, kTcBK,
+  bool ok = encode_2d(&tmA, tma_dt<TA>(), 2, xa, M, K, kTcMB * kTcBM, kTcBK,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, kTcBK, kTcBN / 8,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, scales, K / gsz, N, SR, kTcBN,
+            encode_2d(&tmS, tma_dt<TA>(), 2, scales, K / gsz, N, SR, kTcBN,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / gsz, N / 8, SR, kTcBN / 8,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
-            encode_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, y, M, N, kTcMB * kTcBM, 64,
+            encode_2d(&tmY, tma_dt<TA>(), 2, y, M, N, kTcMB * kTcBM, 64,
                       CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return PARO_ERR_CUDA;
   const dim3 grid((unsigned)((N + kTcBN - 1) / kTcBN), (unsigned)((M + kTcMB * kTcBM - 1) / (kTcMB * kTcBM)), 1);
   if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
   using L = TcLayoutT<SR>;
-  if (!allow_smem(w4_tc_gemm_kernel<SR>, L::SMEM)) return PARO_ERR_CUDA;
-  return launch(w4_tc_gemm_kernel<SR>, grid, dim3(kTcThreads), L::SMEM, s, pdl, tmA, tmW, tmS,
+  if (!allow_smem(w4_tc_gemm_kernel<SR, TA>, L::SMEM)) return PARO_ERR_CUDA;
+  return launch(w4_tc_gemm_kernel<SR, TA>, grid, dim3(kTcThreads), L::SMEM, s, pdl, tmA, tmW, tmS,
                 tmZ, tmY, bias, (int)M, (int)N, (int)K, gsz);
 }
 
-int launch_w4_prefill(const __half* xa, __half* y, int64_t M, int64_t K, int64_t N,
-                      const int32_t* qweight, const int32_t* qzeros, const __half* scales,
-                      const __half* bias, int gsz, cudaStream_t s, bool pdl) {
+template <typename TA>
+int launch_w4_prefill(const TA* xa, TA* y, int64_t M, int64_t K, int64_t N,
+                      const int32_t* qweight, const int32_t* qzeros, const TA* scales,
+                      const TA* bias, int gsz, cudaStream_t s, bool pdl) {
   // scale rows per 64-row k-block: 64 / G groups below G = 64
   switch (gsz) {
-    case 32: return launch_w4_prefill_sr<2>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
-    case 16: return launch_w4_prefill_sr<4>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
-    default: return launch_w4_prefill_sr<1>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
+    case 32: return launch_w4_prefill_sr<2, TA>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
+    case 16: return launch_w4_prefill_sr<4, TA>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
+    default: return launch_w4_prefill_sr<1, TA>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
   }
 }
 
@@ -501,16 +509,16 @@ struct GemvLinearArgs {
   const void* qweight;
   const void* qzeros;
   const void* scales;
-  const __half* x;        // the activations the GEMV reads (X_r, or x itself)
-  const __half* bias;
-  __half* y;
+  const void* x;          // the activations the GEMV reads (X_r, or x itself)
+  const void* bias;
+  void* y;
   int64_t N;
 };
 
 // Decode GEMV launch over `count` (<= NL) linears sharing M and K: grid
 // (column tiles of every linear, splits), one cluster of `splits` CTAs along K
 // per column tile.
-template <int NT, int KP, int NTILE, int STAGES, int NL>
+template <int NT, int KP, int NTILE, int STAGES, int NL, typename TA>
 int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, int64_t M, int64_t K,
                 cudaStream_t s, bool pdl) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
@@ -532,11 +540,12 @@ int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, in
         encode_2d(&o.w, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qweight, K, N / 8, 128, L::WORDS,
                   L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                       : (L::ROW_BYTES == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE)) &&
-        encode_2d(&o.s, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, lin[i].scales, K / plan.gsz, N,
+        encode_2d(&o.s, tma_dt<TA>(), 2, lin[i].scales, K / plan.gsz, N,
                   (uint32_t)(gmax * gq), NTILE, CU_TENSOR_MAP_SWIZZLE_NONE) &&
         encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, K / plan.gsz, N / 8,
                   (uint32_t)(gmax * gq), L::WORDS, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        encode_x_chunks(&o.x, lin[i].x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP, (uint32_t)(2 * gmax));
+        encode_x_chunks(&o.x, tma_dt<TA>(), lin[i].x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP,
+                        (uint32_t)(2 * gmax));
     if (!ok) return PARO_ERR_CUDA;
     o.bias = lin[i].bias;
     o.y = lin[i].y;
@@ -545,7 +554,9 @@ int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, in
     tiles += (N + NTILE - 1) / NTILE;
   }
   if (tiles > INT_MAX / 2) return PARO_ERR_UNSUPPORTED;
-  auto k = w4_gemv_kernel<NT, KP, NTILE, STAGES, NL>;
+  // G = 128 takes the kernel with the group layout fixed at compile time
+  auto k = plan.gsz == kGroup ? w4_gemv_kernel<NT, KP, NTILE, STAGES, NL, TA, 1>
+                              : w4_gemv_kernel<NT, KP, NTILE, STAGES, NL, TA, 0>;
   const dim3 grid((unsigned)tiles, (unsigned)plan.splits, 1);
   const size_t smem = gemv_footprint((size_t)L::smem(gmax, gmax * gq), (int64_t)grid.x * grid.y);
   if (smem == 0 || !allow_smem(k, device_info().smem_optin)) return PARO_ERR_CUDA;
@@ -556,26 +567,63 @@ int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, in
                    (int)K, gmax, gq);
 }
 
-template <int NT, int NL>
+template <int NT, int NL, typename TA>
 int dispatch_gemv_nl(const LinearPlan& plan, const GemvLinearArgs* lin, int count, int64_t M, int64_t K,
                      cudaStream_t s, bool pdl) {
   switch (plan.variant) {
-    case 0: return launch_gemv<NT, 2, 256, 4, NL>(plan, lin, count, M, K, s, pdl);
-    case 2: return launch_gemv<NT, 4, 128, 8, NL>(plan, lin, count, M, K, s, pdl);
-    case 5: return launch_gemv<NT, 4, 64, 8, NL>(plan, lin, count, M, K, s, pdl);
-    default: return launch_gemv<NT, 2, 128, 4, NL>(plan, lin, count, M, K, s, pdl);
+    case 0: return launch_gemv<NT, 2, 256, 4, NL, TA>(plan, lin, count, M, K, s, pdl);
+    case 2: return launch_gemv<NT, 4, 128, 8, NL, TA>(plan, lin, count, M, K, s, pdl);
+    case 5: return launch_gemv<NT, 4, 64, 8, NL, TA>(plan, lin, count, M, K, s, pdl);
+    default: return launch_gemv<NT, 2, 128, 4, NL, TA>(plan, lin, count, M, K, s, pdl);
   }
 }
 
+template <typename TA>
 int dispatch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, int64_t M, int64_t K,
                   cudaStream_t s, bool pdl) {
   if (count == 1)
-    return plan.nt == 1 ? dispatch_gemv_nl<1, 1>(plan, lin, count, M, K, s, pdl)
-                        : dispatch_gemv_nl<2, 1>(plan, lin, count, M, K, s, pdl);
-  return plan.nt == 1 ? dispatch_gemv_nl<1, kGvMaxLinears>(plan, lin, count, M, K, s, pdl)
-                      : dispatch_gemv_nl<2, kGvMaxLinears>(plan, lin, count, M, K, s, pdl);
+    return plan.nt == 1 ? dispatch_gemv_nl<1, 1, TA>(plan, lin, count, M, K, s, pdl)
+                        : dispatch_gemv_nl<2, 1, TA>(plan, lin, count, M, K, s, pdl);
+  return plan.nt == 1 ? dispatch_gemv_nl<1, kGvMaxLinears, TA>(plan, lin, count, M, K, s, pdl)
+                      : dispatch_gemv_nl<2, kGvMaxLinears, TA>(plan, lin, count, M, K, s, pdl);
 }
 
+}  // namespace
+
+// =================================================================== entry bodies
+// The entry points below are these bodies for one activation type: fp16 for
+// the plain names, fp16 or bf16 by `dtype` for the *_dt names.
+namespace {
+template <typename TA>
+int rotate_impl(const void* x, void* x_r, int64_t M, int64_t K, const float* channel_scales,
+                const int16_t* pairs, const float* theta, int group_size, int krot, cudaStream_t s) {
+  if (int st = check_rotation_args(x, x_r, M, K, channel_scales, pairs, theta, group_size, krot))
+    return st;
+  if (M == 0) return PARO_OK;
+  return launch_rotate<TA>(static_cast<const TA*>(x), static_cast<TA*>(x_r), M, K, channel_scales, pairs, theta,
+                           krot, group_of(group_size, K), s);
+}
+
+template <typename TA>
+int quantize_impl(const void* w, const float* channel_scales, const int16_t* pairs, const float* theta,
+                  const void* scales, int32_t* qweight, int32_t* qzeros, int64_t N, int64_t K, int group_size,
+                  int krot, cudaStream_t s) {
+  if (N < 0 || K <= 0 || krot < 0 || N % 8 != 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  if (!supported_group(G, K) || krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
+  if (N == 0) return PARO_OK;   // nothing to touch: NULL data pointers are fine
+  if (w == nullptr || scales == nullptr || qweight == nullptr || qzeros == nullptr) return PARO_ERR_INVALID_ARG;
+  if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
+  if (N * K >= (int64_t(1) << 31)) return PARO_ERR_UNSUPPORTED;
+  if (!aligned(w, 16) || !aligned(scales, 2) || !aligned(qweight, 4) || !aligned(qzeros, 4))
+    return PARO_ERR_ALIGNMENT;
+  if (channel_scales != nullptr && !aligned(channel_scales, 4)) return PARO_ERR_ALIGNMENT;
+  if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
+  const RtQuant qo{scales, qweight, qzeros};
+  return launch_rotate_tmem<true, TA>(static_cast<const TA*>(w), nullptr, N, K, channel_scales, pairs, theta,
+                                      krot, G, qo, s);
+}
 }  // namespace
 
 // =================================================================== C ABI
@@ -599,32 +647,42 @@ const char* paro_version(void) { return "0.1.0"; }
 int paro_rotate(const void* x, void* x_r, int64_t M, int64_t K, const float* channel_scales,
                 const int16_t* pairs, const float* theta, int group_size, int krot,
                 paro_stream_t stream) {
-  if (int st = check_rotation_args(x, x_r, M, K, channel_scales, pairs, theta, group_size, krot))
-    return st;
-  if (M == 0) return PARO_OK;
-  return launch_rotate(static_cast<const __half*>(x), static_cast<__half*>(x_r), M, K,
-                       channel_scales, pairs, theta, krot, group_of(group_size, K),
-                       reinterpret_cast<cudaStream_t>(stream));
+  return paro_rotate_dt(x, x_r, M, K, channel_scales, pairs, theta, group_size, krot, PARO_DTYPE_F16, stream);
+}
+
+int paro_rotate_dt(const void* x, void* x_r, int64_t M, int64_t K, const float* channel_scales,
+                   const int16_t* pairs, const float* theta, int group_size, int krot, int dtype,
+                   paro_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (dtype) {
+    case PARO_DTYPE_F16:
+      return rotate_impl<__half>(x, x_r, M, K, channel_scales, pairs, theta, group_size, krot, s);
+    case PARO_DTYPE_BF16:
+      return rotate_impl<__nv_bfloat16>(x, x_r, M, K, channel_scales, pairs, theta, group_size, krot, s);
+    default: return PARO_ERR_INVALID_ARG;
+  }
 }
 
 int paro_quantize_w4(const void* w, const float* channel_scales, const int16_t* pairs,
                      const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
                      int64_t N, int64_t K, int group_size, int krot, paro_stream_t stream) {
-  if (N < 0 || K <= 0 || krot < 0 || N % 8 != 0) return PARO_ERR_INVALID_ARG;
-  int G = 0;
-  if (int st = normalize_group(group_size, K, &G)) return st;
-  if (!supported_group(G, K) || krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
-  if (N == 0) return PARO_OK;   // nothing to touch: NULL data pointers are fine
-  if (w == nullptr || scales == nullptr || qweight == nullptr || qzeros == nullptr) return PARO_ERR_INVALID_ARG;
-  if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
-  if (N * K >= (int64_t(1) << 31)) return PARO_ERR_UNSUPPORTED;
-  if (!aligned(w, 16) || !aligned(scales, 2) || !aligned(qweight, 4) || !aligned(qzeros, 4))
-    return PARO_ERR_ALIGNMENT;
-  if (channel_scales != nullptr && !aligned(channel_scales, 4)) return PARO_ERR_ALIGNMENT;
-  if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
-  const RtQuant qo{static_cast<const __half*>(scales), qweight, qzeros};
-  return launch_rotate_tmem<true>(static_cast<const __half*>(w), nullptr, N, K, channel_scales, pairs, theta,
-                                  krot, G, qo, reinterpret_cast<cudaStream_t>(stream));
+  return paro_quantize_w4_dt(w, channel_scales, pairs, theta, scales, qweight, qzeros, N, K, group_size, krot,
+                             PARO_DTYPE_F16, stream);
+}
+
+int paro_quantize_w4_dt(const void* w, const float* channel_scales, const int16_t* pairs,
+                        const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
+                        int64_t N, int64_t K, int group_size, int krot, int dtype, paro_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (dtype) {
+    case PARO_DTYPE_F16:
+      return quantize_impl<__half>(w, channel_scales, pairs, theta, scales, qweight, qzeros, N, K, group_size,
+                                   krot, s);
+    case PARO_DTYPE_BF16:
+      return quantize_impl<__nv_bfloat16>(w, channel_scales, pairs, theta, scales, qweight, qzeros, N, K,
+                                          group_size, krot, s);
+    default: return PARO_ERR_INVALID_ARG;
+  }
 }
 
 int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qweight,
@@ -728,6 +786,47 @@ bool group_plan(int64_t M, int64_t K, const paro_linear* lin, int count, int gsz
   *out = p;
   return true;
 }
+
+template <typename TA>
+int linear_impl(const void* x, void* y, int64_t M, int64_t K, int64_t N, const int32_t* qweight,
+                const int32_t* qzeros, const void* scales, const void* bias, const float* channel_scales,
+                const int16_t* pairs, const float* theta, int group_size, int krot, void* workspace,
+                size_t workspace_bytes, cudaStream_t s) {
+  if (int st = check_linear_args(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
+                                 group_size, krot))
+    return st;
+  if (M == 0) return PARO_OK;   // empty batch: nothing to read or write
+
+  const int G = group_of(group_size, K);
+  const LinearPlan plan = make_plan(M, K, N, G);
+
+  const bool rotate = krot > 0 || channel_scales != nullptr;
+  if (rotate && (workspace == nullptr || workspace_bytes < plan.total)) return PARO_ERR_WORKSPACE;
+  if (rotate && !aligned(workspace, 256)) return PARO_ERR_ALIGNMENT;
+  const TA* xa = static_cast<const TA*>(x);
+  // Programmatic dependent launch throughout: the GEMV/GEMM requests weights,
+  // scales and zero points before it waits for the kernel ahead of it (the
+  // rotation, or whatever preceded the call), and reads activations after.
+  const bool pdl = true;
+  if (rotate) {
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    TA* xr = reinterpret_cast<TA*>(ws + plan.off_xr);
+    if (plan.rot_tc) {
+      const RotTcMember one{channel_scales, pairs, theta, krot, xr, ws + plan.off_rt};
+      if (int st = launch_rotate_tc<TA>(xa, &one, 1, M, K, G, s)) return st;
+    } else if (int st = launch_rotate<TA>(xa, xr, M, K, channel_scales, pairs, theta, krot, G, s)) {
+      return st;
+    }
+    xa = xr;
+  }
+
+  if (!plan.decode)
+    return launch_w4_prefill<TA>(xa, static_cast<TA*>(y), M, K, N, qweight, qzeros, static_cast<const TA*>(scales),
+                                 static_cast<const TA*>(bias), G, s, pdl);
+
+  const GemvLinearArgs one{qweight, qzeros, scales, xa, bias, y, N};
+  return dispatch_gemv<TA>(plan, &one, 1, M, K, s, pdl);
+}
 }  // namespace
 
 extern "C" {
@@ -737,43 +836,25 @@ int paro_w4_linear(const void* x, void* y, int64_t M, int64_t K, int64_t N,
                    const void* bias, const float* channel_scales, const int16_t* pairs,
                    const float* theta, int group_size, int krot, void* workspace,
                    size_t workspace_bytes, paro_stream_t stream) {
-  if (int st = check_linear_args(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
-                                 group_size, krot))
-    return st;
-  if (M == 0) return PARO_OK;   // empty batch: nothing to read or write
+  return paro_w4_linear_dt(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta, group_size,
+                           krot, PARO_DTYPE_F16, workspace, workspace_bytes, stream);
+}
 
-  const int G = group_of(group_size, K);
-  const LinearPlan plan = make_plan(M, K, N, G);
-
+int paro_w4_linear_dt(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                      const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                      const void* bias, const float* channel_scales, const int16_t* pairs,
+                      const float* theta, int group_size, int krot, int dtype, void* workspace,
+                      size_t workspace_bytes, paro_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool rotate = krot > 0 || channel_scales != nullptr;
-  if (rotate && (workspace == nullptr || workspace_bytes < plan.total)) return PARO_ERR_WORKSPACE;
-  if (rotate && !aligned(workspace, 256)) return PARO_ERR_ALIGNMENT;
-  const __half* xa = static_cast<const __half*>(x);
-  // Programmatic dependent launch throughout: the GEMV/GEMM requests weights,
-  // scales and zero points before it waits for the kernel ahead of it (the
-  // rotation, or whatever preceded the call), and reads activations after.
-  const bool pdl = true;
-  if (rotate) {
-    unsigned char* ws = static_cast<unsigned char*>(workspace);
-    __half* xr = reinterpret_cast<__half*>(ws + plan.off_xr);
-    if (plan.rot_tc) {
-      const RotTcMember one{channel_scales, pairs, theta, krot, xr, reinterpret_cast<__half*>(ws + plan.off_rt)};
-      if (int st = launch_rotate_tc(xa, &one, 1, M, K, G, s)) return st;
-    } else if (int st = launch_rotate(xa, xr, M, K, channel_scales, pairs, theta, krot, G, s)) {
-      return st;
-    }
-    xa = xr;
+  switch (dtype) {
+    case PARO_DTYPE_F16:
+      return linear_impl<__half>(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
+                                 group_size, krot, workspace, workspace_bytes, s);
+    case PARO_DTYPE_BF16:
+      return linear_impl<__nv_bfloat16>(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs,
+                                        theta, group_size, krot, workspace, workspace_bytes, s);
+    default: return PARO_ERR_INVALID_ARG;
   }
-
-  const __half* b = static_cast<const __half*>(bias);
-  __half* yy = static_cast<__half*>(y);
-  if (!plan.decode)
-    return launch_w4_prefill(xa, yy, M, K, N, qweight, qzeros, static_cast<const __half*>(scales),
-                             b, G, s, pdl);
-
-  const GemvLinearArgs one{qweight, qzeros, scales, xa, b, yy, N};
-  return dispatch_gemv(plan, &one, 1, M, K, s, pdl);
 }
 
 static_assert(PARO_MAX_GROUP == kGvMaxLinears && PARO_MAX_GROUP == kRrMaxLinears && PARO_MAX_GROUP == kRcMaxMembers,
@@ -835,8 +916,12 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
   return (rot > 0 ? (rows_ok ? 1 : rot) : 0) + 1;
 }
 
-int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
-                         int group_size, void* workspace, size_t workspace_bytes, paro_stream_t stream) {
+}  // extern "C"
+
+namespace {
+template <typename TA>
+int group_impl(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears, int group_size,
+               void* workspace, size_t workspace_bytes, cudaStream_t s) {
   if (count < 1 || linears == nullptr) return PARO_ERR_INVALID_ARG;
   if (count > PARO_MAX_GROUP) return PARO_ERR_UNSUPPORTED;
   bool any_rotate = false;
@@ -851,7 +936,6 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
   const size_t need = paro_w4_linear_group_workspace_size(M, K, count, linears, group_size);
   if (any_rotate && (workspace == nullptr || workspace_bytes < need)) return PARO_ERR_WORKSPACE;
   if (any_rotate && !aligned(workspace, 256)) return PARO_ERR_ALIGNMENT;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // member i's X_r lives at workspace + i * per (all members share M and K)
   const int G = group_of(group_size, K);
   const size_t per = make_plan(M, K, linears[0].N, G).total;
@@ -863,25 +947,23 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
     // (x is read once per tile for all of them), then one GEMM per member
     RotTcMember rm[PARO_MAX_GROUP];
     int nrot = 0;
-    const __half* xs[PARO_MAX_GROUP];
+    const TA* xs[PARO_MAX_GROUP];
     for (int i = 0; i < count; ++i) {
       const paro_linear& l = linears[i];
       const int o = rotation_owner(linears, i);
-      xs[i] = static_cast<const __half*>(x);
+      xs[i] = static_cast<const TA*>(x);
       if (o < 0) continue;
-      __half* xr = reinterpret_cast<__half*>(ws + o * per + first.off_xr);
-      if (o == i)
-        rm[nrot++] = RotTcMember{l.channel_scales, l.pairs, l.theta, l.krot, xr,
-                                 reinterpret_cast<__half*>(ws + i * per + first.off_rt)};
+      TA* xr = reinterpret_cast<TA*>(ws + o * per + first.off_xr);
+      if (o == i) rm[nrot++] = RotTcMember{l.channel_scales, l.pairs, l.theta, l.krot, xr, ws + i * per + first.off_rt};
       xs[i] = xr;
     }
     if (nrot > 0)
-      if (int st = launch_rotate_tc(static_cast<const __half*>(x), rm, nrot, M, K, G, s)) return st;
+      if (int st = launch_rotate_tc<TA>(static_cast<const TA*>(x), rm, nrot, M, K, G, s)) return st;
     for (int i = 0; i < count; ++i) {
       const paro_linear& l = linears[i];
-      if (int st = launch_w4_prefill(xs[i], static_cast<__half*>(l.y), M, K, l.N, l.qweight, l.qzeros,
-                                     static_cast<const __half*>(l.scales), static_cast<const __half*>(l.bias), G, s,
-                                     true))
+      if (int st = launch_w4_prefill<TA>(xs[i], static_cast<TA*>(l.y), M, K, l.N, l.qweight, l.qzeros,
+                                         static_cast<const TA*>(l.scales), static_cast<const TA*>(l.bias), G, s,
+                                         true))
         return st;
     }
     return PARO_OK;
@@ -896,18 +978,18 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
       const int o = rotation_owner(linears, i);
       int st;
       if (o >= 0 && o != i)
-        st = paro_w4_linear(ws + o * per + first.off_xr, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias,
-                            nullptr, nullptr, nullptr, group_size, 0, nullptr, 0, stream);
+        st = linear_impl<TA>(ws + o * per + first.off_xr, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias,
+                             nullptr, nullptr, nullptr, group_size, 0, nullptr, 0, s);
       else
-        st = paro_w4_linear(x, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, l.channel_scales, l.pairs,
-                            l.theta, group_size, l.krot, ws ? ws + i * per : nullptr, ws ? per : 0, stream);
+        st = linear_impl<TA>(x, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, l.channel_scales, l.pairs,
+                             l.theta, group_size, l.krot, ws ? ws + i * per : nullptr, ws ? per : 0, s);
       if (st) return st;
     }
     return PARO_OK;
   }
 
   // every member's rotation of x: one warp-per-row launch when all fit it
-  const __half* xa = static_cast<const __half*>(x);
+  const TA* xa = static_cast<const TA*>(x);
   GemvLinearArgs lin[PARO_MAX_GROUP];
   RrBatch rb;
   std::memset(&rb, 0, sizeof(rb));
@@ -916,26 +998,48 @@ int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const p
   for (int i = 0; i < count; ++i) {
     const paro_linear& l = linears[i];
     const int o = rotation_owner(linears, i);
-    __half* xr = o >= 0 ? reinterpret_cast<__half*>(ws + o * per) : nullptr;
+    TA* xr = o >= 0 ? reinterpret_cast<TA*>(ws + o * per) : nullptr;
     if (o == i) {
       rb.op[nrot++] = RrOperand{xr, l.channel_scales, l.pairs, l.theta, l.krot};
       max_krot = std::max(max_krot, l.krot);
       rows_ok = rows_ok && l.krot <= kRrMaxKrot;
     }
-    lin[i] = GemvLinearArgs{l.qweight, l.qzeros, l.scales, o >= 0 ? xr : xa, static_cast<const __half*>(l.bias),
-                            static_cast<__half*>(l.y), l.N};
+    lin[i] = GemvLinearArgs{l.qweight, l.qzeros, l.scales, o >= 0 ? static_cast<const void*>(xr) : xa, l.bias,
+                            l.y, l.N};
   }
   if (nrot > 0) {
     if (rows_ok) {
-      if (int st = launch_rotate_rows(xa, rb, nrot, M, K, max_krot, G, s)) return st;
+      if (int st = launch_rotate_rows<TA>(xa, rb, nrot, M, K, max_krot, G, s)) return st;
     } else {
       for (int r = 0; r < nrot; ++r)
-        if (int st = launch_rotate(xa, rb.op[r].xr, M, K, rb.op[r].cs, rb.op[r].pairs, rb.op[r].theta,
-                                   rb.op[r].krot, G, s))
+        if (int st = launch_rotate<TA>(xa, static_cast<TA*>(rb.op[r].xr), M, K, rb.op[r].cs, rb.op[r].pairs,
+                                       rb.op[r].theta, rb.op[r].krot, G, s))
           return st;
     }
   }
-  return dispatch_gemv(gp, lin, count, M, K, s, true);
+  return dispatch_gemv<TA>(gp, lin, count, M, K, s, true);
+}
+}  // namespace
+
+extern "C" {
+
+int paro_w4_linear_group(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
+                         int group_size, void* workspace, size_t workspace_bytes, paro_stream_t stream) {
+  return paro_w4_linear_group_dt(x, M, K, count, linears, group_size, PARO_DTYPE_F16, workspace, workspace_bytes,
+                                 stream);
+}
+
+int paro_w4_linear_group_dt(const void* x, int64_t M, int64_t K, int count, const paro_linear* linears,
+                            int group_size, int dtype, void* workspace, size_t workspace_bytes,
+                            paro_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (dtype) {
+    case PARO_DTYPE_F16:
+      return group_impl<__half>(x, M, K, count, linears, group_size, workspace, workspace_bytes, s);
+    case PARO_DTYPE_BF16:
+      return group_impl<__nv_bfloat16>(x, M, K, count, linears, group_size, workspace, workspace_bytes, s);
+    default: return PARO_ERR_INVALID_ARG;
+  }
 }
 
 }  // extern "C"
@@ -972,6 +1076,15 @@ int paro_w4_linear_noalloc(const void* x, void* y, int64_t M, int64_t K, int64_t
                            const int32_t* qweight, const int32_t* qzeros, const void* scales,
                            const void* bias, const float* channel_scales, const int16_t* pairs,
                            const float* theta, int group_size, int krot, paro_stream_t stream) {
+  return paro_w4_linear_noalloc_dt(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
+                                   group_size, krot, PARO_DTYPE_F16, stream);
+}
+
+int paro_w4_linear_noalloc_dt(const void* x, void* y, int64_t M, int64_t K, int64_t N,
+                              const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                              const void* bias, const float* channel_scales, const int16_t* pairs,
+                              const float* theta, int group_size, int krot, int dtype, paro_stream_t stream) {
+  if (dtype != PARO_DTYPE_F16 && dtype != PARO_DTYPE_BF16) return PARO_ERR_INVALID_ARG;
   // the same argument checks, in the same order, as paro_w4_linear
   if (int st = check_linear_args(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
                                  group_size, krot))
@@ -980,14 +1093,14 @@ int paro_w4_linear_noalloc(const void* x, void* y, int64_t M, int64_t K, int64_t
   // only a call that rotates (krot > 0 or channel scales) stages anything
   const bool rotate = krot > 0 || channel_scales != nullptr;
   if (!rotate)
-    return paro_w4_linear(x, y, M, K, N, qweight, qzeros, scales, bias, nullptr, pairs, theta, group_size, 0,
-                          nullptr, 0, stream);
+    return paro_w4_linear_dt(x, y, M, K, N, qweight, qzeros, scales, bias, nullptr, pairs, theta, group_size, 0,
+                             dtype, nullptr, 0, stream);
   if (paro_w4_linear_workspace_size(M, K, N, group_size) > (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES)
     return PARO_ERR_WORKSPACE;
   void* scratch = noalloc_scratch_address();
   if (scratch == nullptr) return PARO_ERR_CUDA;
-  return paro_w4_linear(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
-                        group_size, krot, scratch, (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES, stream);
+  return paro_w4_linear_dt(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
+                           group_size, krot, dtype, scratch, (size_t)PARO_W4_LINEAR_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int paro_validate_pairs(const int16_t* pairs_host, int64_t K, int group_size, int krot) {

@@ -72,9 +72,9 @@ struct RotTile {
 
 // grid: (K/128, ceil(M/ROWS)), block 256.  Dynamic smem: krot*64*16 bytes of
 // RotParam + the fp32 tile (rotate_smem_bytes).
-template <int ROWS>
+template <int ROWS, typename TA>
 __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
-    const __half* x, __half* xr, const float* __restrict__ cs,
+    const TA* x, TA* xr, const float* __restrict__ cs,
     const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot, int gsz) {
   using T = RotTile<ROWS>;
   // Programmatic dependent launch: the GEMV that follows may launch at once and
@@ -112,10 +112,10 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
 #pragma unroll
       for (int e = 0; e < 8; ++e) sc[e] = 1.0f;
     }
-    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+    const uint32_t h[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(h[e]);
+      const float2 f = Act<TA>::f2(h[e]);
       xs[(8 * v + 2 * e) * T::PITCH + r] = f.x * sc[2 * e];
       xs[(8 * v + 2 * e + 1) * T::PITCH + r] = f.y * sc[2 * e + 1];
     }
@@ -148,13 +148,11 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(
     const int row = row0 + r;
     if (row >= M) continue;
     const int ch0 = grp * kGroup + 8 * v;
-    uint4 out;
-    __half2* h = reinterpret_cast<__half2*>(&out);
+    uint32_t h[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      h[e] = __floats2half2_rn(xs[(8 * v + 2 * e) * T::PITCH + r],
-                               xs[(8 * v + 2 * e + 1) * T::PITCH + r]);
-    *reinterpret_cast<uint4*>(xr + (size_t)row * K + ch0) = out;
+      h[e] = Act<TA>::p2(xs[(8 * v + 2 * e) * T::PITCH + r], xs[(8 * v + 2 * e + 1) * T::PITCH + r]);
+    *reinterpret_cast<uint4*>(xr + (size_t)row * K + ch0) = make_uint4(h[0], h[1], h[2], h[3]);
   }
 }
 
@@ -183,7 +181,7 @@ struct RrLayout {
 // to kRrMaxLinears linears (blockIdx.z), each with its own tables.
 constexpr int kRrMaxLinears = 4;
 struct RrOperand {
-  __half* xr;
+  void* xr;                // X_r of the activation type
   const float* cs;
   const int16_t* pairs;
   const float* theta;
@@ -193,14 +191,15 @@ struct RrBatch {
   RrOperand op[kRrMaxLinears];
 };
 
-__global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(const RrBatch batch, const __half* x,
+template <typename TA>
+__global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(const RrBatch batch, const TA* x,
                                                                     int M, int K, int gsz) {
   pdl_launch_dependents();                         // the GEMV may start streaming weights
   RrOperand o = batch.op[0];
 #pragma unroll
   for (int i = 1; i < kRrMaxLinears; ++i)
     if ((int)blockIdx.z == i) o = batch.op[i];
-  __half* const xr = o.xr;
+  TA* const xr = static_cast<TA*>(o.xr);
   const float* __restrict__ const cs = o.cs;
   const int16_t* __restrict__ const pairs = o.pairs;
   const float* __restrict__ const theta = o.theta;
@@ -252,8 +251,8 @@ __global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(const RrBatc
   pdl_wait_primary();                              // x may come from the previous kernel
   if (row >= M) return;
   const uint2 raw = *reinterpret_cast<const uint2*>(x + (size_t)row * K + (size_t)grp * kGroup + ch);
-  const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-  const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+  const float2 lo = Act<TA>::f2(raw.x);
+  const float2 hi = Act<TA>::f2(raw.y);
   float v[4] = {lo.x * csv.x, lo.y * csv.y, hi.x * csv.z, hi.y * csv.w};
   const uint32_t rb = smem_u32(smem_raw + RrLayout::row_off(krot) + warp * 512);
 #pragma unroll
@@ -271,10 +270,9 @@ __global__ void __launch_bounds__(32 * kRrWarps) rotate_rows_kernel(const RrBatc
       for (int k = 0; k < 4; ++k) v[k] = fmaf(v[k], c4[k], xp[k] * s4[k]);
     }
   }
-  const __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
   uint2 out;
-  out.x = *reinterpret_cast<const uint32_t*>(&h0);
-  out.y = *reinterpret_cast<const uint32_t*>(&h1);
+  out.x = Act<TA>::p2(v[0], v[1]);
+  out.y = Act<TA>::p2(v[2], v[3]);
   *reinterpret_cast<uint2*>(xr + (size_t)row * K + (size_t)grp * kGroup + ch) = out;
 }
 

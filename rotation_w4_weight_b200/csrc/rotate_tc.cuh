@@ -24,6 +24,10 @@
 // moved (about 2.1 GFLOP per 16 MB) -- less tensor-core time than the bytes
 // take at HBM speed.
 //
+// The activation type (fp16 or bf16) is a template parameter: with bf16
+// activations the parts are bf16 and carry R' to about 2^-16 relative, far
+// below the bf16 rounding of X_r.
+//
 // Layout of the transposed parts in global memory: fp16 [2][K][128]; part 0 is
 // Rhi, part 1 is Rlo; row g*128 + n, column k holds R'_g[k][n], i.e. each
 // 128-row block is the K-major B operand (N = output channel, K = input
@@ -51,7 +55,7 @@ struct RbOperand {
   const float* cs;         // [K] or nullptr
   const int16_t* pairs;    // [krot, K]
   const float* theta;      // [krot, K/2]
-  __half* rt;              // R' parts, fp16 [2][K][128]
+  void* rt;                // R' parts, [2][K][128] of the activation type
   int krot;
 };
 struct RbBatch {
@@ -60,6 +64,7 @@ struct RbBatch {
 
 // grid (K/128, 128/kRbRows, members), block kRbThreads; dynamic shared memory
 // for the largest krot of the batch.
+template <typename TA>
 __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_constant__ RbBatch batch, int K,
                                                                 int gsz) {
   // The rotation that follows waits for this kernel's completion; let it
@@ -69,7 +74,7 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_con
   const float* __restrict__ cs = op.cs;
   const int16_t* __restrict__ pairs = op.pairs;
   const float* __restrict__ theta = op.theta;
-  __half* __restrict__ rt = op.rt;
+  TA* __restrict__ rt = static_cast<TA*>(op.rt);
   const int krot = op.krot;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RotParam* prm = reinterpret_cast<RotParam*>(smem_raw);
@@ -123,14 +128,12 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_con
   for (int e = 0; e < 8; ++e) {
     const float va = lds_f32(vbase + (uint32_t)((16 * h + 2 * e) * kRbPitch + n) * 4u);
     const float vb = lds_f32(vbase + (uint32_t)((16 * h + 2 * e + 1) * kRbPitch + n) * 4u);
-    const __half ah = __float2half_rn(va), bh = __float2half_rn(vb);
-    const __half al = __float2half_rn(va - __half2float(ah));
-    const __half bl = __float2half_rn(vb - __half2float(bh));
-    const __half2 ph = __halves2half2(ah, bh), pl = __halves2half2(al, bl);
-    hi[e] = *reinterpret_cast<const uint32_t*>(&ph);
-    lo[e] = *reinterpret_cast<const uint32_t*>(&pl);
+    // hi part rounded once to the activation type, lo part the remainder
+    const TA ah = Act<TA>::from(va), bh = Act<TA>::from(vb);
+    hi[e] = Act<TA>::p2(Act<TA>::f1(ah), Act<TA>::f1(bh));
+    lo[e] = Act<TA>::p2(va - Act<TA>::f1(ah), vb - Act<TA>::f1(bh));
   }
-  __half* dst = rt + ((size_t)grp * kGroup + n) * kGroup + r0 + 16 * h;
+  TA* dst = rt + ((size_t)grp * kGroup + n) * kGroup + r0 + 16 * h;
   uint4* dh = reinterpret_cast<uint4*>(dst);
   uint4* dl = reinterpret_cast<uint4*>(dst + (size_t)K * kGroup);
   dh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -188,15 +191,16 @@ constexpr uint32_t kRcIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 
 // nearest) in the staging tile: 64-channel box cb / 2, 16-byte chunks
 // 4 (cb % 2) .. +3 of the row, XOR-swizzled by (r & 7) as the 128-byte TMA
 // swizzle expects.
+template <typename TA>
 __device__ __forceinline__ void rc_stage32(uint32_t tile, int r, int cb, const uint32_t (&v)[32]) {
   const uint32_t rowp = tile + (uint32_t)(cb >> 1) * RcLayout::BOX + (uint32_t)r * 128u;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint4 o;
-    __half2* oh = reinterpret_cast<__half2*>(&o);
+    uint32_t* oh = &o.x;
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      oh[e] = __floats2half2_rn(__uint_as_float(v[8 * c + 2 * e]), __uint_as_float(v[8 * c + 2 * e + 1]));
+      oh[e] = Act<TA>::p2(__uint_as_float(v[8 * c + 2 * e]), __uint_as_float(v[8 * c + 2 * e + 1]));
     const uint32_t chunk = (uint32_t)(4 * (cb & 1) + c);
     sts128u(rowp + ((chunk ^ (uint32_t)(r & 7)) << 4), o);
   }
@@ -214,6 +218,7 @@ struct RcBatch {
 
 // grid P <= number of SMs, block kRcThreads.  tmX: x [M, K] fp16, box {64, 128},
 // 128-byte swizzle.  jobs = members * groups * tiles.
+template <typename TA>
 __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ RcBatch batch, int members, int K,
     int groups, int tiles, long long jobs) {
@@ -327,8 +332,8 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
           const uint64_t ad = umma_desc(xs + box + off, 16, 1024, 2);
           const uint64_t bh = umma_desc(base + L::R_OFF + box + off, 16, 1024, 2);
           const uint64_t bl = umma_desc(base + L::R_OFF + 2 * L::BOX + box + off, 16, 1024, 2);
-          umma_f16(d, ad, bh, kRcIdesc, ks > 0 ? 1u : 0u);
-          umma_f16(d, ad, bl, kRcIdesc, 1u);
+          umma_f16(d, ad, bh, kRcIdesc | Act<TA>::kIdescAB, ks > 0 ? 1u : 0u);
+          umma_f16(d, ad, bl, kRcIdesc | Act<TA>::kIdescAB, 1u);
         }
         umma_commit(x_empty0 + 8 * s);    // the x stage and ...
         umma_commit(acc_full0 + 8 * a);   // ... the accumulator, once these MMAs finish
@@ -375,10 +380,10 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
       named_bar_sync(1, 32 * kRcEpiWarps);
       const uint32_t tile = base + L::O_OFF + (uint32_t)(i & 1) * L::O_STAGE;
       if (ok) {
-        rc_stage32(tile, r, 0, v0);
-        rc_stage32(tile, r, 1, v1);
-        rc_stage32(tile, r, 2, v2);
-        rc_stage32(tile, r, 3, v3);
+        rc_stage32<TA>(tile, r, 0, v0);
+        rc_stage32<TA>(tile, r, 1, v1);
+        rc_stage32<TA>(tile, r, 2, v2);
+        rc_stage32<TA>(tile, r, 3, v3);
       }
       fence_proxy_async_smem();            // the tile is read by the TMA (async proxy)
       named_bar_sync(2, 32 * kRcEpiWarps);

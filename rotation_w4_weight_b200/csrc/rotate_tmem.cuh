@@ -74,7 +74,7 @@ constexpr size_t kRtMinSmem = 80 * 1024; // above a third of an SM's shared memo
 
 // Output of the quantising instantiation (rows = N output channels).
 struct RtQuant {
-  const __half* scales;   // [K/G, N] quantiser scales
+  const void* scales;     // [K/G, N] quantiser scales (activation type)
   int32_t* qweight;       // [K, N/8] AWQ words
   int32_t* qzeros;        // [K/G, N/8] AWQ words (all 8)
 };
@@ -136,9 +136,9 @@ __device__ __forceinline__ uint32_t rt_awq_word(uint32_t lo, uint32_t hi) {
 // grid: (K/128, row-tile slots), block 256.  tmX is x as [M, K] fp16 with box
 // {64 channels, 128 rows}, 128-byte swizzle (rows past M read as zeros).
 // QUANT: x is W [N = M, K], xr is unused and qo receives the packed codes.
-template <bool ABS, bool QUANT>
+template <bool ABS, bool QUANT, typename TA>
 __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kernel(
-    const __grid_constant__ CUtensorMap tmX, __half* xr, const float* __restrict__ cs,
+    const __grid_constant__ CUtensorMap tmX, TA* xr, const float* __restrict__ cs,
     const int16_t* __restrict__ pairs, const float* __restrict__ theta, int M, int K, int krot, int gsz,
     const RtQuant qo) {
   using L = RtLayout;
@@ -309,10 +309,10 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
 #pragma unroll
     for (int q = 0; q < SW / 8; ++q) {
       const uint4 raw = *reinterpret_cast<const uint4*>(rowp + ((((uint32_t)(q0 + q)) ^ rsw) << 4));
-      const __half2* hv = reinterpret_cast<const __half2*>(&raw);
+      const uint32_t hv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {                  // the channel scale is the starting factor
-        const float2 f = __half22float2(hv[e]);
+        const float2 f = Act<TA>::f2(hv[e]);
         v[8 * q + 2 * e] = __float_as_uint(f.x);
         v[8 * q + 2 * e + 1] = __float_as_uint(f.y);
       }
@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
 #pragma unroll
       for (int k = 0; k < SW / 16; ++k) {
         const int qg = (grp * kGroup + SW * h + 16 * k) / gsz;
-        float sc = row < M ? __half2float(qo.scales[(size_t)qg * M + row]) : 1.0f;
+        float sc = row < M ? Act<TA>::f1(static_cast<const TA*>(qo.scales)[(size_t)qg * M + row]) : 1.0f;
         sc = fminf(fmaxf(sc, 1e-5f), 1e5f);
         inv[k] = 1.0f / sc;
       }
@@ -445,14 +445,14 @@ __global__ void __launch_bounds__(kRtThreads, kRtMaxCtasPerSm) rotate_tmem_kerne
       }
     } else if (row < M) {
       // ---- fp16 (round to nearest), row r, channels SW*h .. SW*h+SW-1
-      __half* dstp = xr + (size_t)row * K + (size_t)grp * kGroup + SW * h;
+      TA* dstp = xr + (size_t)row * K + (size_t)grp * kGroup + SW * h;
 #pragma unroll
       for (int q = 0; q < SW / 8; ++q) {
         uint4 out;
-        __half2* hv = reinterpret_cast<__half2*>(&out);
+        uint32_t* hv = &out.x;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          hv[e] = __floats2half2_rn(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
+          hv[e] = Act<TA>::p2(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
         *reinterpret_cast<uint4*>(dstp + 8 * q) = out;
       }
     }

@@ -19,6 +19,10 @@
 // Consumer warps are 4 column slices (64 columns each) x KP k-parts; k-part p
 // takes the CTA's groups p, p+KP, ... so every warp works on whole groups.
 //
+// Activations, scales, bias and Y are fp16 or bf16 (template type TA); with
+// bf16 every nibble is unpacked to 128 + q (bf16 has 7 mantissa bits) and the
+// MMA runs on bf16 operands.
+//
 // Quantisation groups of G = 128, 64, 32 or 16 rows: the fold below runs at
 // the end of every G / 16 k-steps with that group's scales and zero words.
 //
@@ -55,7 +59,7 @@ namespace paro {
 constexpr int kGvMaxStages = 8;
 constexpr int kGvMaxGroups = 16;            // 128-row groups of K per CTA
 constexpr uint32_t kGvMagic = 0x64006400u;  // fp16 pair (1024, 1024)
-constexpr uint32_t kGvOnes = 0x3C003C00u;   // fp16 pair (1, 1)
+constexpr uint32_t kGvMagicBf = 0x43004300u;   // bf16 pair (128, 128)
 
 // NTILE output columns per CTA (64 per column-slice warp), KP k-parts, STAGES
 // groups in flight.
@@ -98,8 +102,8 @@ struct alignas(64) GemvOperand {
   CUtensorMap x;          // X_r [M, K] fp16 as [K/64][M][64], box {64, MP, 2 gmax}
   CUtensorMap s;          // scales [K/G, N] fp16, box {NTILE, gmax * 128 / G}
   CUtensorMap z;          // qzeros [K/G, N/8] int32, box {NTILE/8, gmax * 128 / G}
-  const __half* bias;     // [N] or nullptr
-  __half* y;              // [M, N]
+  const void* bias;       // [N] or nullptr (activation type)
+  void* y;                // [M, N] (activation type)
   int n;                  // output columns
   int tile_begin;         // first column tile of this linear in the grid
 };
@@ -109,17 +113,41 @@ struct GemvBatch {
 };
 constexpr int kGvMaxLinears = 4;
 
+// Nibbles j = 0..3 of the two 16-bit halves of m.  fp16: 1024 + q for even j
+// and 1024 + 16 q for odd j (the nibble read in place, 10 mantissa bits);
+// bf16 (7 mantissa bits): every nibble moved to bits 0..3, 128 + q.
+template <typename TA>
 __device__ __forceinline__ void gv_unpack4(uint32_t m, uint32_t (&e)[4]) {
-  const uint32_t m8 = m >> 8;
-  e[0] = and_or(m, 0x000F000Fu, kGvMagic);
-  e[1] = and_or(m, 0x00F000F0u, kGvMagic);
-  e[2] = and_or(m8, 0x000F000Fu, kGvMagic);
-  e[3] = and_or(m8, 0x00F000F0u, kGvMagic);
+  if constexpr (Act<TA>::kBf16) {
+    e[0] = and_or(m, 0x000F000Fu, kGvMagicBf);
+    e[1] = and_or(m >> 4, 0x000F000Fu, kGvMagicBf);
+    e[2] = and_or(m >> 8, 0x000F000Fu, kGvMagicBf);
+    e[3] = and_or(m >> 12, 0x000F000Fu, kGvMagicBf);
+  } else {
+    const uint32_t m8 = m >> 8;
+    e[0] = and_or(m, 0x000F000Fu, kGvMagic);
+    e[1] = and_or(m, 0x00F000F0u, kGvMagic);
+    e[2] = and_or(m8, 0x000F000Fu, kGvMagic);
+    e[3] = and_or(m8, 0x00F000F0u, kGvMagic);
+  }
 }
 
-template <int NT, int KP, int NTILE, int STAGES, int NL>
+template <typename TA>
+__device__ __forceinline__ void gv_mma(bool first, float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (Act<TA>::kBf16) {
+    if (first) mma_16816_bf_zc(d, a, b0, b1);
+    else mma_16816_bf(d, a, b0, b1);
+  } else {
+    if (first) mma_16816_zc(d, a, b0, b1);
+    else mma_16816(d, a, b0, b1);
+  }
+}
+
+// GQ: quantisation groups per 128 rows fixed at compile time (1: G = 128),
+// or 0 to take them from gq_arg (G = 64, 32, 16).
+template <int NT, int KP, int NTILE, int STAGES, int NL, typename TA, int GQ>
 __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kernel(
-    const __grid_constant__ GemvBatch<NL> ops, int M, int K, int gmax, int gq) {
+    const __grid_constant__ GemvBatch<NL> ops, int M, int K, int gmax, int gq_arg) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
   // this CTA's linear (selected by constant offsets into the parameter block)
   const GemvOperand* op = &ops.op[0];
@@ -130,8 +158,8 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const CUtensorMap* const tmX = &op->x;
   const CUtensorMap* const tmS = &op->s;
   const CUtensorMap* const tmZ = &op->z;
-  const __half* const bias = op->bias;
-  __half* const Y = op->y;
+  const TA* const bias = static_cast<const TA*>(op->bias);
+  TA* const Y = static_cast<TA*>(op->y);
   const int N = op->n;
   constexpr int kGvStages = STAGES;
   constexpr int kGvTile = NTILE;
@@ -145,6 +173,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const uint32_t base = smem_u32(sbase);
   // gq = 128 / G quantisation groups per 128-row group (G = 128, 64, 32, 16);
   // spq = G / 16 k-steps of 16 rows each
+  const int gq = GQ > 0 ? GQ : gq_arg;
   const int gr = gmax * gq, spq = 8 / gq;
   const uint32_t full0 = base + L::bar_off(gmax, gr);
   const uint32_t empty0 = full0 + 8 * kGvStages;
@@ -244,7 +273,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
         xo[q][nt][0] = (uint32_t)(tok * 128 + (((c0) ^ (tok & 7)) << 4) + 4 * t);
         xo[q][nt][1] = (uint32_t)(tok * 128 + (((c0 + 1) ^ (tok & 7)) << 4) + 4 * t);
       }
-    const uint32_t ones[4] = {kGvOnes, kGvOnes, kGvOnes, kGvOnes};
+    const uint32_t ones[4] = {Act<TA>::kOnes, Act<TA>::kOnes, Act<TA>::kOnes, Act<TA>::kOnes};
     const uint32_t sq = base + (uint32_t)L::s_off(gmax);   // scales of the range
     const uint32_t zq = base + (uint32_t)L::z_off(gmax, gr);   // zero words of the range
 
@@ -259,6 +288,33 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       if (ready) {
         float cg[4][NT][4];
         float rs[NT][4];
+        // end of the quantisation group that closes at k-step ks: zero-point
+        // correction and group scale, in fp32, with this thread's 8 columns'
+        // constants
+        auto fold = [&](int ks) {
+          const int qrow = i * gq + ks / spq;
+          const uint32_t zw = lds32(zq + (uint32_t)((qrow * L::WORDS + wcol) * 4));
+          const uint4 s8 = lds128(sq + (uint32_t)(qrow * NTILE * 2 + wcol * 16));
+          const uint32_t sw[4] = {s8.x, s8.y, s8.z, s8.w};   // (s[2j], s[2j+1])
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // fp16: 1024 + z (16 z and s / 16 for odd j); bf16: 128 + z
+            const int sh = (!Act<TA>::kBf16 && (j & 1)) ? 4 : 0;
+            const float mg = Act<TA>::kBf16 ? 128.f : 1024.f;
+            const float zl = mg + (float)(((zw >> (4 * j)) & 0xFu) << sh);
+            const float zh = mg + (float)(((zw >> (16 + 4 * j)) & 0xFu) << sh);
+            float2 sf = Act<TA>::f2(sw[j]);
+            if (sh) sf.x *= 0.0625f, sf.y *= 0.0625f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const float r0 = rs[nt][0], r1 = rs[nt][1];   // row sums of tokens 2t, 2t+1
+              acc[j][nt][0] = fmaf(sf.x, fmaf(-zl, r0, cg[j][nt][0]), acc[j][nt][0]);
+              acc[j][nt][1] = fmaf(sf.x, fmaf(-zl, r1, cg[j][nt][1]), acc[j][nt][1]);
+              acc[j][nt][2] = fmaf(sf.y, fmaf(-zh, r0, cg[j][nt][2]), acc[j][nt][2]);
+              acc[j][nt][3] = fmaf(sf.y, fmaf(-zh, r1, cg[j][nt][3]), acc[j][nt][3]);
+            }
+          }
+        };
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t wrow = stq + (uint32_t)(ks * 16 * RB);
@@ -274,54 +330,39 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
             b1[nt] = lds32(xb + xo[ks & 3][nt][1]);
           }
           uint32_t elo01[4], ehi01[4], elo89[4], ehi89[4];
-          gv_unpack4(prmt(w0, w1, 0x5410), elo01);
-          gv_unpack4(prmt(w0, w1, 0x7632), ehi01);
-          gv_unpack4(prmt(w8, w9, 0x5410), elo89);
-          gv_unpack4(prmt(w8, w9, 0x7632), ehi89);
-          // the first k-step of a quantisation group starts its sums at zero
-          const bool first = (ks & (spq - 1)) == 0;
+          gv_unpack4<TA>(prmt(w0, w1, 0x5410), elo01);
+          gv_unpack4<TA>(prmt(w0, w1, 0x7632), ehi01);
+          gv_unpack4<TA>(prmt(w8, w9, 0x5410), elo89);
+          gv_unpack4<TA>(prmt(w8, w9, 0x7632), ehi89);
+          // the first k-step starts the sums at zero (a known constant of the
+          // unrolled loop, so no branch between the two MMA forms)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint32_t a[4] = {elo01[j], ehi01[j], elo89[j], ehi89[j]};
 #pragma unroll
+            for (int nt = 0; nt < NT; ++nt) gv_mma<TA>(ks == 0, cg[j][nt], a, b0[nt], b1[nt]);
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) gv_mma<TA>(ks == 0, rs[nt], ones, b0[nt], b1[nt]);
+          // a quantisation group that closes inside the 128 rows (G < 128):
+          // fold it and restart the sums at zero
+          if (ks != 7 && (ks & (spq - 1)) == spq - 1) {
+            fold(ks);
+#pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              if (first) mma_16816_zc(cg[j][nt], a, b0[nt], b1[nt]);
-              else mma_16816(cg[j][nt], a, b0[nt], b1[nt]);
-            }
-          }
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            if (first) mma_16816_zc(rs[nt], ones, b0[nt], b1[nt]);
-            else mma_16816(rs[nt], ones, b0[nt], b1[nt]);
-          }
-          if ((ks & (spq - 1)) == spq - 1) {
-            // end of a quantisation group: zero-point correction and group
-            // scale, in fp32, with this thread's 8 columns' constants
-            const int qrow = i * gq + ks / spq;
-            const uint32_t zw = lds32(zq + (uint32_t)((qrow * L::WORDS + wcol) * 4));
-            const uint4 s8 = lds128(sq + (uint32_t)(qrow * NTILE * 2 + wcol * 16));
-            const uint32_t sw[4] = {s8.x, s8.y, s8.z, s8.w};   // (s[2j], s[2j+1])
+              for (int e = 0; e < 4; ++e) {
+                rs[nt][e] = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int sh = (j & 1) ? 4 : 0;
-              const float zl = 1024.f + (float)(((zw >> (4 * j)) & 0xFu) << sh);
-              const float zh = 1024.f + (float)(((zw >> (16 + 4 * j)) & 0xFu) << sh);
-              float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sw[j]));
-              if (j & 1) sf.x *= 0.0625f, sf.y *= 0.0625f;
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                const float r0 = rs[nt][0], r1 = rs[nt][1];   // row sums of tokens 2t, 2t+1
-                acc[j][nt][0] = fmaf(sf.x, fmaf(-zl, r0, cg[j][nt][0]), acc[j][nt][0]);
-                acc[j][nt][1] = fmaf(sf.x, fmaf(-zl, r1, cg[j][nt][1]), acc[j][nt][1]);
-                acc[j][nt][2] = fmaf(sf.y, fmaf(-zh, r0, cg[j][nt][2]), acc[j][nt][2]);
-                acc[j][nt][3] = fmaf(sf.y, fmaf(-zh, r1, cg[j][nt][3]), acc[j][nt][3]);
+                for (int j = 0; j < 4; ++j) cg[j][nt][e] = 0.f;
               }
             }
           }
         }
-        // this warp is done reading the stage
+        // this warp is done reading the stage; the last group folds from registers
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
+        fold(7);
       } else {
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);   // keep the producer moving
@@ -376,9 +417,9 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   if (bias != nullptr && tid < nq) {
     const int n = n0 + (int)rank * cols + 4 * (tid % (cols / 4));
     if (n < N) {
-      const __half2 b0 = *reinterpret_cast<const __half2*>(bias + n);
-      const __half2 b1 = *reinterpret_cast<const __half2*>(bias + n + 2);
-      bv = make_float4(__low2float(b0), __high2float(b0), __low2float(b1), __high2float(b1));
+      const float2 b0 = Act<TA>::f2(*reinterpret_cast<const uint32_t*>(bias + n));
+      const float2 b1 = Act<TA>::f2(*reinterpret_cast<const uint32_t*>(bias + n + 2));
+      bv = make_float4(b0.x, b0.y, b1.x, b1.y);
     }
   }
   // this CTA's own partials (CTA barrier) and every peer's (the inbox barrier)
@@ -404,16 +445,15 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     }
     if (bias != nullptr) {
       if (idx != tid) {
-        const __half2 b0 = *reinterpret_cast<const __half2*>(bias + n);
-        const __half2 b1 = *reinterpret_cast<const __half2*>(bias + n + 2);
-        bv = make_float4(__low2float(b0), __high2float(b0), __low2float(b1), __high2float(b1));
+        const float2 b0 = Act<TA>::f2(*reinterpret_cast<const uint32_t*>(bias + n));
+        const float2 b1 = Act<TA>::f2(*reinterpret_cast<const uint32_t*>(bias + n + 2));
+        bv = make_float4(b0.x, b0.y, b1.x, b1.y);
       }
       sum.x += bv.x; sum.y += bv.y; sum.z += bv.z; sum.w += bv.w;
     }
-    const __half2 h0 = __floats2half2_rn(sum.x, sum.y), h1 = __floats2half2_rn(sum.z, sum.w);
     uint2 out;
-    out.x = *reinterpret_cast<const uint32_t*>(&h0);
-    out.y = *reinterpret_cast<const uint32_t*>(&h1);
+    out.x = Act<TA>::p2(sum.x, sum.y);
+    out.y = Act<TA>::p2(sum.z, sum.w);
     *reinterpret_cast<uint2*>(Y + (size_t)tl * N + n) = out;
   }
   if (S > 1) {

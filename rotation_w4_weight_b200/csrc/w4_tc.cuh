@@ -1,6 +1,9 @@
 // Prefill W4 GEMM on the sm_100a tensor cores (tcgen05 / TMEM), M > 16 token rows.
 // Quantisation groups of G = 128, 64, 32 or 16 rows (scales and zero words of
 // the 64-row k-block's max(1, 64 / G) groups come with each TMA stage).
+// Activations, weights as dequantised, scales, bias and Y are fp16 or bf16
+// (template type TA; bf16 unpacks every nibble to 128 + q and runs the MMA
+// with bf16 A and B).
 //
 // What it computes (GPTQModel wiki page "ParoQuant", "Activation and weight
 // transforms" and "Triton plans and tuning"):
@@ -89,11 +92,11 @@ struct TcLayoutT {
 // instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M=128, N=256
 constexpr uint32_t kTcIdesc = (1u << 4) | ((uint32_t)(kTcBN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
 
-template <int SR>
+template <int SR, typename TA>
 __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
-    const __grid_constant__ CUtensorMap tmY, const __half* __restrict__ bias, int M, int N, int K, int gsz) {
+    const __grid_constant__ CUtensorMap tmY, const TA* __restrict__ bias, int M, int N, int K, int gsz) {
   using L = TcLayoutT<SR>;
   constexpr int kTcBBufs = L::BBUFS;
   extern __shared__ unsigned char smem_raw[];
@@ -183,7 +186,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
           for (int mb = 0; mb < kTcMB; ++mb) {
             // A: 128-byte swizzled rows, 8-row groups 1024 B apart; +32 B per 16 k
             const uint64_t ad = umma_desc(a0 + mb * L::A_BLOCK + ks * 32, 16, 1024, 2);
-            umma_f16(tmem_d + (uint32_t)(mb * kTcBN), ad, bd, kTcIdesc, (kb > 0 || ks > 0) ? 1u : 0u);
+            umma_f16(tmem_d + (uint32_t)(mb * kTcBN), ad, bd, kTcIdesc | Act<TA>::kIdescAB,
+                     (kb > 0 || ks > 0) ? 1u : 0u);
           }
         }
         umma_commit(tma_empty0 + 8 * s);   // the TMA stage and ...
@@ -226,15 +230,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
         uint32_t elo[4], ehi[4];
         const uint32_t mlo = prmt(wv[2 * p], wv[2 * p + 1], 0x5410);
         const uint32_t mhi = prmt(wv[2 * p], wv[2 * p + 1], 0x7632);
-        const uint32_t mlo8 = mlo >> 8, mhi8 = mhi >> 8;
-        elo[0] = and_or(mlo, 0x000F000Fu, 0x64006400u);
-        elo[1] = and_or(mlo, 0x00F000F0u, 0x64006400u);
-        elo[2] = and_or(mlo8, 0x000F000Fu, 0x64006400u);
-        elo[3] = and_or(mlo8, 0x00F000F0u, 0x64006400u);
-        ehi[0] = and_or(mhi, 0x000F000Fu, 0x64006400u);
-        ehi[1] = and_or(mhi, 0x00F000F0u, 0x64006400u);
-        ehi[2] = and_or(mhi8, 0x000F000Fu, 0x64006400u);
-        ehi[3] = and_or(mhi8, 0x00F000F0u, 0x64006400u);
+        if constexpr (Act<TA>::kBf16) {
+          // bf16 (7 mantissa bits): every nibble moved to bits 0..3, 128 + q
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            elo[j] = and_or(mlo >> (4 * j), 0x000F000Fu, 0x43004300u);
+            ehi[j] = and_or(mhi >> (4 * j), 0x000F000Fu, 0x43004300u);
+          }
+        } else {
+          const uint32_t mlo8 = mlo >> 8, mhi8 = mhi >> 8;
+          elo[0] = and_or(mlo, 0x000F000Fu, 0x64006400u);
+          elo[1] = and_or(mlo, 0x00F000F0u, 0x64006400u);
+          elo[2] = and_or(mlo8, 0x000F000Fu, 0x64006400u);
+          elo[3] = and_or(mlo8, 0x00F000F0u, 0x64006400u);
+          ehi[0] = and_or(mhi, 0x000F000Fu, 0x64006400u);
+          ehi[1] = and_or(mhi, 0x00F000F0u, 0x64006400u);
+          ehi[2] = and_or(mhi8, 0x000F000Fu, 0x64006400u);
+          ehi[3] = and_or(mhi8, 0x00F000F0u, 0x64006400u);
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           outv[2 * j][p] = elo[j];        // column 2j   (nibble j)
@@ -245,14 +258,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
       for (int col = 0; col < 8; ++col) {
         const int j = col >> 1;
         const int nib = j + 4 * (col & 1);
-        const uint32_t sh = (j & 1) ? 4u : 0u;
-        const uint32_t z = ((zw >> (4 * nib)) & 0xFu) << sh;
-        const uint32_t zz = (z | (z << 16)) | 0x64006400u;
         uint32_t sc = prmt(sw[j], sw[j], (col & 1) ? 0x3232 : 0x1010);   // (s, s)
-        if (j & 1) sc = hmul2_u32(sc, 0x2C002C00u);                      // s / 16
         uint2 o;
-        o.x = hmul2_u32(hsub2_u32(outv[col][0], zz), sc);
-        o.y = hmul2_u32(hsub2_u32(outv[col][1], zz), sc);
+        if constexpr (Act<TA>::kBf16) {
+          const uint32_t z = (zw >> (4 * nib)) & 0xFu;
+          const uint32_t zz = (z | (z << 16)) | 0x43004300u;              // 128 + z
+          o.x = bmul2_u32(bsub2_u32(outv[col][0], zz), sc);
+          o.y = bmul2_u32(bsub2_u32(outv[col][1], zz), sc);
+        } else {
+          const uint32_t sh = (j & 1) ? 4u : 0u;
+          const uint32_t z = ((zw >> (4 * nib)) & 0xFu) << sh;
+          const uint32_t zz = (z | (z << 16)) | 0x64006400u;
+          if (j & 1) sc = hmul2_u32(sc, 0x2C002C00u);                      // s / 16
+          o.x = hmul2_u32(hsub2_u32(outv[col][0], zz), sc);
+          o.y = hmul2_u32(hsub2_u32(outv[col][1], zz), sc);
+        }
         sts64(btile + (uint32_t)(w * kTcBSbo + c * kTcBLbo + col * 16 + h * 8), o);
       }
       fence_proxy_async_smem();         // make the B tile visible to the tensor core
@@ -290,19 +310,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
           float v[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]);
-          if (bias != nullptr && n < N) {   // bias is only 4-byte aligned: half2 loads
-            const __half2* bh = reinterpret_cast<const __half2*>(bias + n + 8 * q);
+          if (bias != nullptr && n < N) {   // bias is only 4-byte aligned: pair loads
+            const uint32_t* bh = reinterpret_cast<const uint32_t*>(bias + n + 8 * q);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 f = __half22float2(bh[e]);
+              const float2 f = Act<TA>::f2(bh[e]);
               v[2 * e] += f.x;
               v[2 * e + 1] += f.y;
             }
           }
           uint4 o;
-          __half2* oh = reinterpret_cast<__half2*>(&o);
+          uint32_t* oh = &o.x;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) oh[e] = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+          for (int e = 0; e < 4; ++e) oh[e] = Act<TA>::p2(v[2 * e], v[2 * e + 1]);
           const uint32_t chunk = (uint32_t)(((col0 & 63) >> 3) + q);
           sts128u(rowp + ((chunk ^ (uint32_t)(row & 7)) << 4), o);
         }

@@ -210,3 +210,34 @@ def test_selftest_wait_limit_is_checked_on_the_host(L):
     assert L.paro_selftest_wait_timeout(0, ctypes.byref(e), None) == L.PARO_ERR_INVALID_ARG
     assert L.paro_selftest_wait_timeout(100_000_001, ctypes.byref(e), None) == L.PARO_ERR_INVALID_ARG
     assert e.value == 7
+
+
+def test_dtype_entry_points_check_the_type_first(L):
+    """The *_dt twins refuse a type other than fp16/bf16 before anything else,
+    and otherwise check their arguments exactly as the fp16 entry points do."""
+    bad = 2
+    assert L.paro_rotate_dt(A16, A16, 4, 256, None, None, None, 128, 0, bad, None) == L.PARO_ERR_INVALID_ARG
+    assert L.paro_quantize_w4_dt(A16, None, None, None, A16, A16, A16, 16, 256, 128, 0, bad,
+                                 None) == L.PARO_ERR_INVALID_ARG
+    assert L.paro_w4_linear_dt(A16, A16, 4, 256, 512, A16, A16, A16, None, None, None, None, 128, 0, -1,
+                               None, 0, None) == L.PARO_ERR_INVALID_ARG
+    assert L.paro_w4_linear_noalloc_dt(A16, A16, 4, 256, 512, A16, A16, A16, None, None, None, None, 128, 0, bad,
+                                       None) == L.PARO_ERR_INVALID_ARG
+    arr = (L.ParoLinear * 1)()
+    arr[0] = L.ParoLinear(512, 0x10000, 0x10000, 0x10000, None, None, None, None, 0, 0x10000)
+    assert L.paro_w4_linear_group_dt(A16, 4, 256, 1, arr, 128, bad, None, 0, None) == L.PARO_ERR_INVALID_ARG
+    bf = L.PARO_DTYPE_BF16
+    # with a valid type, the same statuses as the fp16 calls (no launch is reached)
+    for kw, want in [(dict(M=-1), L.PARO_ERR_INVALID_ARG), (dict(N=40), L.PARO_ERR_UNSUPPORTED),
+                     (dict(G=8), L.PARO_ERR_UNSUPPORTED), (dict(x=MIS), L.PARO_ERR_ALIGNMENT),
+                     (dict(M=0), L.PARO_OK)]:
+        a = dict(x=A16, y=A16, M=4, K=256, N=512, G=128)
+        a.update(kw)
+        got = L.paro_w4_linear_dt(a["x"], a["y"], a["M"], a["K"], a["N"], A16, A16, A16, None, None, None, None,
+                                  a["G"], 0, bf, None, 0, None)
+        assert got == want == lin(L, x=a["x"], M=a["M"], N=a["N"], G=a["G"]), kw
+    assert L.paro_rotate_dt(A16, A16, 4, 256, None, A16, A16, 8, 8, bf, None) == L.PARO_ERR_UNSUPPORTED
+    assert L.paro_quantize_w4_dt(A16, None, A16, A16, A16, A16, A16, 16, 256, 128, 65, bf,
+                                 None) == L.PARO_ERR_UNSUPPORTED
+    assert L.paro_w4_linear_noalloc_dt(A16, A16, 4, 256, 40, A16, A16, A16, None, None, None, None, 128, 0, bf,
+                                       None) == L.PARO_ERR_UNSUPPORTED
