@@ -208,6 +208,9 @@ size_t paro_w4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int group_
  *   on the prefill path; products and sums in fp32 (tensor cores); y rounded
  *   once to fp16 (bf16).
  *   M <= 16 runs the decode GEMV path; larger M the tcgen05 prefill GEMM path.
+ *   A prepared R' (paro_rotation_matrix_prepare, passed as paro_linear.rmat
+ *   through paro_w4_linear_group, also with count == 1) replaces the per-call
+ *   build above 64 rows.
  *   From M >= 65 the rotation itself runs on the tensor cores: each group's
  *   stages with its channel scales are the 128 x 128 matrix
  *   R' = diag(cs) G_0 ... G_{krot-1}, built per call in fp32 (its 128 basis rows
@@ -262,6 +265,12 @@ typedef struct paro_linear {
   const float* theta;              /* [krot, K/2]; NULL only when krot == 0 */
   int krot;
   void* y;                         /* fp16 (or dtype) [M, N] output */
+  /* Optional prepared R' parts of this member (paro_rotation_matrix_prepare
+   * with this member's channel_scales, pairs, theta, K, group_size and krot,
+   * in the call's dtype), 256-byte aligned, or NULL.  Batches above 64 rows
+   * then skip the per-call R' build; nothing else changes (the same build
+   * kernel made them, so results are identical). */
+  const void* rmat;
 } paro_linear;
 
 size_t paro_w4_linear_group_workspace_size(int64_t M, int64_t K, int count, const paro_linear* linears,
@@ -275,6 +284,29 @@ int paro_w4_linear_group_dt(const void* x, int64_t M, int64_t K, int count, cons
  * GEMV/GEMM launches; 0 for an invalid shape or M == 0).  Host-only query. */
 int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_linear* linears,
                                   int group_size);
+
+/*
+ * paro_rotation_matrix_prepare — the R' parts of one layer, built once.
+ * R' = diag(cs) G_0 ... G_{krot-1} per 128-channel tile (the product form of
+ * the page's "Pairwise Givens rotations" with the channel scales of
+ * "Activation and weight transforms") depends only on the stored rotation
+ * (section "Stored tensors": channel_scales, pairs, theta), so a caller may
+ * build it at load time and pass it with every call (paro_linear.rmat);
+ * calls above 64 rows then skip their per-call build.
+ *   channel_scales, pairs, theta, K, group_size, krot: as for paro_rotate
+ *           (NULL pairs/theta only when krot == 0); K < 2^24
+ *   dtype   the activation type of the calls that will use it (the parts are
+ *           stored in that type: R' = Rhi + Rlo)
+ *   rmat    device memory of at least paro_rotation_matrix_size(K) =
+ *           K * 128 * 4 bytes, 256-byte aligned; written on `stream`
+ * The build is the per-call one, so results do not change.  The kernel does
+ * not release its dependents early, so a call right after may use rmat.
+ * paro_rotation_matrix_size returns 0 for a K prepare would reject.
+ */
+size_t paro_rotation_matrix_size(int64_t K);
+int paro_rotation_matrix_prepare(const float* channel_scales, const int16_t* pairs, const float* theta,
+                                 int64_t K, int group_size, int krot, int dtype, void* rmat, size_t rmat_bytes,
+                                 paro_stream_t stream);
 
 /*
  * paro_w4_linear_noalloc — paro_w4_linear for callers that cannot allocate

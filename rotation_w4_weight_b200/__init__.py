@@ -12,6 +12,7 @@ streams) into that ABI.  Functions mirror the C entry points:
     quantize_w4       -> paro_quantize_w4 / paro_quantize_w4_dt
     validate_pairs    -> paro_validate_pairs (host helper)
     device_status     -> paro_device_status
+    rotation_matrix   -> paro_rotation_matrix_prepare (+ paro_rotation_matrix_size)
 
 Activations, scales, bias and outputs are fp16 or bf16 (one type per call,
 taken from x): fp16 calls go to the plain entry points, bf16 calls to the
@@ -32,10 +33,12 @@ from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # n
                    paro_validate_pairs, paro_version, paro_w4_linear, paro_w4_linear_workspace_size,
                    PARO_MAX_GROUP, ParoLinear, paro_w4_linear_group, paro_w4_linear_group_launches,
                    paro_w4_linear_group_workspace_size, PARO_DTYPE_BF16, paro_rotate_dt, paro_quantize_w4_dt,
-                   paro_w4_linear_dt, paro_w4_linear_group_dt)
+                   paro_w4_linear_dt, paro_w4_linear_group_dt, paro_rotation_matrix_size,
+                   paro_rotation_matrix_prepare, PARO_DTYPE_F16)
 
 __all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
-           "w4_linear_group", "w4_linear_group_launches", "quantize_w4", "validate_pairs", "device_status", "ParoError", "LIB_PATH"]
+           "w4_linear_group", "w4_linear_group_launches", "quantize_w4", "validate_pairs", "device_status",
+           "rotation_matrix", "ParoError", "LIB_PATH"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -161,8 +164,17 @@ def w4_linear(x: torch.Tensor, qweight: torch.Tensor, qzeros: torch.Tensor, scal
               pairs: Optional[torch.Tensor], theta: Optional[torch.Tensor],
               group_size: int = 128, krot: Optional[int] = None,
               workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-              stream=None) -> torch.Tensor:
-    """Y = rotate(x * channel_scales) @ dequant(qweight, qzeros, scales) + bias (out in x's type)."""
+              stream=None, rmat: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y = rotate(x * channel_scales) @ dequant(qweight, qzeros, scales) + bias (out in x's type).
+
+    ``rmat``: this layer's prepared R' (``rotation_matrix``); the call then
+    goes through the grouped entry point with one member, which is where the
+    C ABI takes it."""
+    if rmat is not None:
+        m = dict(qweight=qweight, qzeros=qzeros, scales=scales, bias=bias, channel_scales=channel_scales,
+                 pairs=pairs, theta=theta, krot=krot, rmat=rmat)
+        return w4_linear_group(x, [m], group_size, workspace=workspace,
+                               out=None if out is None else [out], stream=stream)[0]
     dt = _act(x, "x")
     _need(x, dt, "x")
     _need(qweight, torch.int32, "qweight")
@@ -222,12 +234,13 @@ def _members(x: torch.Tensor, members, outs):
         if krot is None:
             krot = 0 if m.get("pairs") is None else m["pairs"].shape[0]
         N = m["qweight"].shape[1] * 8
+        _need(m.get("rmat"), torch.uint8, "rmat", True)
         arr[i] = ParoLinear(N, m["qweight"].data_ptr(), m["qzeros"].data_ptr(), m["scales"].data_ptr(),
                             None if m.get("bias") is None else m["bias"].data_ptr(),
                             None if m.get("channel_scales") is None else m["channel_scales"].data_ptr(),
                             None if m.get("pairs") is None else m["pairs"].data_ptr(),
                             None if m.get("theta") is None else m["theta"].data_ptr(), krot,
-                            outs[i].data_ptr())
+                            outs[i].data_ptr(), None if m.get("rmat") is None else m["rmat"].data_ptr())
     return arr
 
 
@@ -235,7 +248,8 @@ def w4_linear_group(x: torch.Tensor, members, group_size: int = 128, workspace: 
                     out=None, stream=None):
     """Several linears over the same x (q/k/v, gate/up): ``members`` is a list of
     dicts with keys qweight, qzeros, scales and optionally bias, channel_scales,
-    pairs, theta, krot.  Returns the list of outputs [M, N_i] in x's type."""
+    pairs, theta, krot and rmat (from ``rotation_matrix``).
+    Returns the list of outputs [M, N_i] in x's type."""
     dt = _act(x, "x")
     _need(x, dt, "x")
     M, K = x.shape
@@ -259,14 +273,40 @@ def w4_linear_group_launches(M: int, K: int, members, group_size: int = 128) -> 
     """Kernel launches one ``w4_linear_group`` call of this shape issues.
 
     ``members``: dicts with N and optionally krot (default 8), channel_scales
-    (bool, default True) and same_rotation_as (index of an earlier member whose
-    rotation tables this member shares).  Only shapes and table identity
-    matter: the descriptors carry placeholder addresses, never dereferenced."""
+    (bool, default True), same_rotation_as (index of an earlier member whose
+    rotation tables this member shares) and rmat (bool: the member carries a
+    prepared R'; default False).  Only shapes and table identity matter: the
+    descriptors carry placeholder addresses, never dereferenced."""
     arr = (ParoLinear * len(members))()
     for i, m in enumerate(members):
         owner = m.get("same_rotation_as", i)
-        tag = 16 * (owner + 1)                   # distinct per rotation, shared by its members
+        tag = 256 * (owner + 1)                  # distinct per rotation, shared by its members
         krot = m.get("krot", 8)
         arr[i] = ParoLinear(m["N"], None, None, None, None, tag if m.get("channel_scales", True) else None,
-                            tag if krot > 0 else None, tag if krot > 0 else None, krot, None)
+                            tag if krot > 0 else None, tag if krot > 0 else None, krot, None,
+                            tag if m.get("rmat", False) else None)
     return int(paro_w4_linear_group_launches(M, K, len(members), arr, group_size))
+
+
+def rotation_matrix(channel_scales: Optional[torch.Tensor], pairs: Optional[torch.Tensor],
+                    theta: Optional[torch.Tensor], K: int, group_size: int = 128, krot: Optional[int] = None,
+                    dtype=torch.float16, stream=None) -> torch.Tensor:
+    """This layer's R' parts, built once (uint8 device tensor of
+    paro_rotation_matrix_size(K) bytes): pass it as ``rmat=`` on the layer's
+    calls.  ``dtype`` is the activation type of those calls."""
+    _need(channel_scales, torch.float32, "channel_scales", True)
+    _need(pairs, torch.int16, "pairs", True)
+    _need(theta, torch.float32, "theta", True)
+    if dtype not in _ACT_TYPES:
+        raise TypeError(f"dtype must be float16 or bfloat16, got {dtype}")
+    if krot is None:
+        krot = 0 if pairs is None else pairs.shape[0]
+    n = int(paro_rotation_matrix_size(K))
+    if n == 0:
+        raise ParoError(PARO_ERR_INVALID_ARG, "paro_rotation_matrix_size")
+    src = [t for t in (channel_scales, pairs, theta) if t is not None]
+    out = torch.empty(n, dtype=torch.uint8, device=src[0].device if src else torch.device("cuda"))
+    code = PARO_DTYPE_F16 if dtype == torch.float16 else PARO_DTYPE_BF16
+    check(paro_rotation_matrix_prepare(_ptr(channel_scales), _ptr(pairs), _ptr(theta), K, group_size, krot, code,
+                                       _ptr(out), n, _stream(stream)), "paro_rotation_matrix_prepare")
+    return out

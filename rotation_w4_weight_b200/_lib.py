@@ -29,7 +29,8 @@ EXPORTED = (
     "paro_validate_pairs", "paro_device_status", "paro_quantize_w4",
     "paro_w4_linear_group_workspace_size", "paro_w4_linear_group", "paro_w4_linear_group_launches",
     "paro_selftest_wait_timeout", "paro_rotate_dt", "paro_quantize_w4_dt", "paro_w4_linear_dt",
-    "paro_w4_linear_group_dt", "paro_w4_linear_noalloc_dt",
+    "paro_w4_linear_group_dt", "paro_w4_linear_noalloc_dt", "paro_rotation_matrix_size",
+    "paro_rotation_matrix_prepare",
 )
 
 PARO_MAX_GROUP = 4
@@ -40,7 +41,7 @@ class ParoLinear(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("qweight", ctypes.c_void_p), ("qzeros", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("channel_scales", ctypes.c_void_p),
                 ("pairs", ctypes.c_void_p), ("theta", ctypes.c_void_p), ("krot", ctypes.c_int),
-                ("y", ctypes.c_void_p)]
+                ("y", ctypes.c_void_p), ("rmat", ctypes.c_void_p)]
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -71,6 +72,8 @@ _SIGNATURES = {
     "paro_w4_linear_group_dt": (_int, [_vp, _i64, _i64, _int, _vp, _int, _int, _vp, ctypes.c_size_t, _vp]),
     "paro_w4_linear_noalloc_dt": (_int, [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                                          _vp, _int, _int, _int, _vp]),
+    "paro_rotation_matrix_size": (ctypes.c_size_t, [_i64]),
+    "paro_rotation_matrix_prepare": (_int, [_vp, _vp, _vp, _i64, _int, _int, _int, _vp, ctypes.c_size_t, _vp]),
 }
 
 
@@ -110,6 +113,8 @@ paro_quantize_w4_dt = lib.paro_quantize_w4_dt
 paro_w4_linear_dt = lib.paro_w4_linear_dt
 paro_w4_linear_group_dt = lib.paro_w4_linear_group_dt
 paro_w4_linear_noalloc_dt = lib.paro_w4_linear_noalloc_dt
+paro_rotation_matrix_size = lib.paro_rotation_matrix_size
+paro_rotation_matrix_prepare = lib.paro_rotation_matrix_prepare
 
 
 class ParoError(RuntimeError):

@@ -326,6 +326,7 @@ struct RotTcMember {
   int krot;
   void* xr;         // X_r [M, K]
   void* rt;         // R' parts [2][K][128]
+  bool prebuilt;    // rt already holds R' (paro_rotation_matrix_prepare): no build
 };
 
 template <typename TA>
@@ -339,18 +340,22 @@ int launch_rotate_tc(const TA* x, const RotTcMember* mem, int count, int64_t M, 
   std::memset(&rb, 0, sizeof(rb));
   RcBatch rc;
   std::memset(&rc, 0, sizeof(rc));
-  int max_krot = 0;
+  int max_krot = 0, nb = 0;
   for (int i = 0; i < count; ++i) {
-    rb.op[i] = RbOperand{mem[i].cs, mem[i].pairs, mem[i].theta, mem[i].rt, mem[i].krot};
-    max_krot = std::max(max_krot, mem[i].krot);
+    if (!mem[i].prebuilt) {      // members without a prepared R' build it now
+      rb.op[nb++] = RbOperand{mem[i].cs, mem[i].pairs, mem[i].theta, mem[i].rt, mem[i].krot};
+      max_krot = std::max(max_krot, mem[i].krot);
+    }
     if (!encode_2d(&rc.t[i].r, tma_dt<TA>(), 2, mem[i].rt, 2 * K, kGroup, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&rc.t[i].y, tma_dt<TA>(), 2, mem[i].xr, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return PARO_ERR_CUDA;
   }
-  if (!allow_smem(rmat_build_kernel<TA>, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
-  if (int st = launch(rmat_build_kernel<TA>, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows), (unsigned)count),
-                      dim3(kRbThreads), rb_smem_bytes(max_krot), stream, true, rb, (int)K, gsz))
-    return st;
+  if (nb > 0) {
+    if (!allow_smem(rmat_build_kernel<TA>, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
+    if (int st = launch(rmat_build_kernel<TA>, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows), (unsigned)nb),
+                        dim3(kRbThreads), rb_smem_bytes(max_krot), stream, true, rb, (int)K, gsz))
+      return st;
+  }
   CUtensorMap tmX;
   if (!encode_2d(&tmX, tma_dt<TA>(), 2, x, M, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return PARO_ERR_CUDA;
@@ -733,6 +738,41 @@ size_t paro_w4_linear_workspace_size(int64_t M, int64_t K, int64_t N, int group_
   return make_plan(M, K, N, group_of(group_size, K)).total;
 }
 
+size_t paro_rotation_matrix_size(int64_t K) {
+  if (K <= 0 || K % kGroup != 0 || K >= (int64_t(1) << 24)) return 0;
+  return (size_t)K * kGroup * 2 * 2;
+}
+
+int paro_rotation_matrix_prepare(const float* channel_scales, const int16_t* pairs, const float* theta,
+                                 int64_t K, int group_size, int krot, int dtype, void* rmat, size_t rmat_bytes,
+                                 paro_stream_t stream) {
+  if (dtype != PARO_DTYPE_F16 && dtype != PARO_DTYPE_BF16) return PARO_ERR_INVALID_ARG;
+  if (K <= 0 || krot < 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  if (!supported_group(G, K) || krot > kMaxKrot || K >= (int64_t(1) << 24)) return PARO_ERR_UNSUPPORTED;
+  if (rmat == nullptr || (krot > 0 && (pairs == nullptr || theta == nullptr))) return PARO_ERR_INVALID_ARG;
+  if (rmat_bytes < paro_rotation_matrix_size(K)) return PARO_ERR_WORKSPACE;
+  if (!aligned(rmat, 256) || (channel_scales != nullptr && !aligned(channel_scales, 4)) ||
+      (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))))
+    return PARO_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  RbBatch rb;
+  std::memset(&rb, 0, sizeof(rb));
+  rb.op[0] = RbOperand{channel_scales, pairs, theta, rmat, krot};
+  const dim3 grid((unsigned)(K / kGroup), (unsigned)(kGroup / kRbRows), 1);
+  // the build kernel that does not release its dependents early: R' is a
+  // layer constant that later calls read before they wait for the kernel ahead
+  if (dtype == PARO_DTYPE_F16) {
+    if (!allow_smem(rmat_build_kernel<__half, false>, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
+    return launch(rmat_build_kernel<__half, false>, grid, dim3(kRbThreads), rb_smem_bytes(krot), s, false, rb,
+                  (int)K, G);
+  }
+  if (!allow_smem(rmat_build_kernel<__nv_bfloat16, false>, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
+  return launch(rmat_build_kernel<__nv_bfloat16, false>, grid, dim3(kRbThreads), rb_smem_bytes(krot), s, false, rb,
+                (int)K, G);
+}
+
 }  // extern "C"
 
 namespace {
@@ -788,13 +828,15 @@ bool group_plan(int64_t M, int64_t K, const paro_linear* lin, int count, int gsz
 }
 
 template <typename TA>
+// rmat: this linear's prepared R' parts (paro_rotation_matrix_prepare) or nullptr.
 int linear_impl(const void* x, void* y, int64_t M, int64_t K, int64_t N, const int32_t* qweight,
                 const int32_t* qzeros, const void* scales, const void* bias, const float* channel_scales,
                 const int16_t* pairs, const float* theta, int group_size, int krot, void* workspace,
-                size_t workspace_bytes, cudaStream_t s) {
+                size_t workspace_bytes, cudaStream_t s, const void* rmat = nullptr) {
   if (int st = check_linear_args(x, y, M, K, N, qweight, qzeros, scales, bias, channel_scales, pairs, theta,
                                  group_size, krot))
     return st;
+  if (rmat != nullptr && !aligned(rmat, 256)) return PARO_ERR_ALIGNMENT;
   if (M == 0) return PARO_OK;   // empty batch: nothing to read or write
 
   const int G = group_of(group_size, K);
@@ -812,7 +854,9 @@ int linear_impl(const void* x, void* y, int64_t M, int64_t K, int64_t N, const i
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     TA* xr = reinterpret_cast<TA*>(ws + plan.off_xr);
     if (plan.rot_tc) {
-      const RotTcMember one{channel_scales, pairs, theta, krot, xr, ws + plan.off_rt};
+      const bool pre = rmat != nullptr;
+      const RotTcMember one{channel_scales, pairs, theta, krot, xr,
+                            pre ? const_cast<void*>(rmat) : static_cast<void*>(ws + plan.off_rt), pre};
       if (int st = launch_rotate_tc<TA>(xa, &one, 1, M, K, G, s)) return st;
     } else if (int st = launch_rotate<TA>(xa, xr, M, K, channel_scales, pairs, theta, krot, G, s)) {
       return st;
@@ -909,7 +953,12 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
   // prefill batches rotating on the tensor cores: one R' build and one X R'
   // launch for all rotating members, then one GEMM each
   const int G = group_of(group_size, K);
-  if (make_plan(M, K, linears[0].N, G).rot_tc) return (rot > 0 ? 2 : 0) + count;
+  if (make_plan(M, K, linears[0].N, G).rot_tc) {
+    // an R' build only for rotations without a prepared R'
+    bool build = false;
+    for (int i = 0; i < count; ++i) build = build || (rotation_owner(linears, i) == i && linears[i].rmat == nullptr);
+    return (rot > 0 ? (build ? 2 : 1) : 0) + count;
+  }
   LinearPlan gp;
   // one after another: each rotating member launches its rotation and its GEMV / GEMM
   if (count == 1 || !group_plan(M, K, linears, count, G, &gp)) return rot + count;
@@ -930,6 +979,7 @@ int group_impl(const void* x, int64_t M, int64_t K, int count, const paro_linear
     if (int st = check_linear_args(x, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, l.channel_scales,
                                    l.pairs, l.theta, group_size, l.krot))
       return st;
+    if (l.rmat != nullptr && !aligned(l.rmat, 256)) return PARO_ERR_ALIGNMENT;
     any_rotate = any_rotate || l.krot > 0 || l.channel_scales != nullptr;
   }
   if (M == 0) return PARO_OK;
@@ -954,7 +1004,12 @@ int group_impl(const void* x, int64_t M, int64_t K, int count, const paro_linear
       xs[i] = static_cast<const TA*>(x);
       if (o < 0) continue;
       TA* xr = reinterpret_cast<TA*>(ws + o * per + first.off_xr);
-      if (o == i) rm[nrot++] = RotTcMember{l.channel_scales, l.pairs, l.theta, l.krot, xr, ws + i * per + first.off_rt};
+      if (o == i) {
+        const bool pre = l.rmat != nullptr;
+        rm[nrot++] = RotTcMember{l.channel_scales, l.pairs, l.theta, l.krot, xr,
+                                 pre ? const_cast<void*>(l.rmat) : static_cast<void*>(ws + i * per + first.off_rt),
+                                 pre};
+      }
       xs[i] = xr;
     }
     if (nrot > 0)
@@ -982,7 +1037,7 @@ int group_impl(const void* x, int64_t M, int64_t K, int count, const paro_linear
                              nullptr, nullptr, nullptr, group_size, 0, nullptr, 0, s);
       else
         st = linear_impl<TA>(x, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, l.channel_scales, l.pairs,
-                             l.theta, group_size, l.krot, ws ? ws + i * per : nullptr, ws ? per : 0, s);
+                             l.theta, group_size, l.krot, ws ? ws + i * per : nullptr, ws ? per : 0, s, l.rmat);
       if (st) return st;
     }
     return PARO_OK;

@@ -64,12 +64,14 @@ struct RbBatch {
 
 // grid (K/128, 128/kRbRows, members), block kRbThreads; dynamic shared memory
 // for the largest krot of the batch.
-template <typename TA>
+// RELEASE: let the kernel that follows launch early (false when the parts are
+// prepared layer constants, which later kernels read before they wait).
+template <typename TA, bool RELEASE = true>
 __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_constant__ RbBatch batch, int K,
                                                                 int gsz) {
   // The rotation that follows waits for this kernel's completion; let it
   // launch and set itself up meanwhile.
-  pdl_launch_dependents();
+  if constexpr (RELEASE) pdl_launch_dependents();
   const RbOperand& op = batch.op[blockIdx.z];
   const float* __restrict__ cs = op.cs;
   const int16_t* __restrict__ pairs = op.pairs;

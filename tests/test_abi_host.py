@@ -192,6 +192,12 @@ def test_group_launch_count_query(L):
     assert pb.w4_linear_group_launches(4096, 4096, qkv) == 5
     assert pb.w4_linear_group_launches(65, 4096, qkv) == 5
     assert pb.w4_linear_group_launches(64, 4096, qkv) == 6
+    # prepared R' parts skip the build (one member without them still builds)
+    qkv_r = [dict(m, rmat=True) for m in qkv]
+    assert pb.w4_linear_group_launches(4096, 4096, qkv_r) == 4
+    assert pb.w4_linear_group_launches(4096, 4096, [qkv_r[0], qkv[1]]) == 4
+    assert pb.w4_linear_group_launches(4096, 4096, [dict(N=4096, rmat=True)]) == 2
+    assert pb.w4_linear_group_launches(1, 4096, qkv_r) in (2, 6)          # decode does not use R'
     assert pb.w4_linear_group_launches(4096, 4096, [dict(N=4096, krot=0, channel_scales=False)] * 2) == 2
     # experts sharing one rotation rotate x once: one rotation (not three) up to
     # 64 rows, and the single-rotation count on the other paths
@@ -202,6 +208,32 @@ def test_group_launch_count_query(L):
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096)]) == 2
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096, krot=0, channel_scales=False)]) == 1
     assert pb.w4_linear_group_launches(1, 4000, qkv) == 0               # invalid K
+
+
+def test_rotation_matrix_size_and_prepare_checks(L):
+    assert L.paro_rotation_matrix_size(4096) == 4096 * 128 * 4
+    for bad in (0, -128, 4000, 1 << 24):
+        assert L.paro_rotation_matrix_size(bad) == 0, bad
+    need = 4096 * 128 * 4
+    prep = lambda cs=None, pr=A16, th=A16, K=4096, G=128, krot=8, dt=0, t=P(0x100000), n=need: \
+        L.paro_rotation_matrix_prepare(cs, pr, th, K, G, krot, dt, t, n, None)  # noqa: E731
+    assert prep(dt=2) == L.PARO_ERR_INVALID_ARG
+    assert prep(K=-128) == L.PARO_ERR_INVALID_ARG
+    assert prep(krot=-1) == L.PARO_ERR_INVALID_ARG
+    assert prep(G=8) == L.PARO_ERR_UNSUPPORTED
+    assert prep(krot=65) == L.PARO_ERR_UNSUPPORTED
+    assert prep(t=None) == L.PARO_ERR_INVALID_ARG
+    assert prep(pr=None) == L.PARO_ERR_INVALID_ARG
+    assert prep(n=need - 1) == L.PARO_ERR_WORKSPACE
+    assert prep(t=P(0x100010)) == L.PARO_ERR_ALIGNMENT
+    assert prep(cs=P(0x10002)) == L.PARO_ERR_ALIGNMENT
+
+
+def test_linear_rejects_misaligned_rmat(L):
+    """The prepared R' pointer is checked before any launch."""
+    arr = (L.ParoLinear * 1)()
+    arr[0] = L.ParoLinear(512, 0x10000, 0x10000, 0x10000, None, None, None, None, 0, 0x10000, 0x100010)
+    assert L.paro_w4_linear_group(A16, 4, 256, 1, arr, 128, A16, 1 << 20, None) == L.PARO_ERR_ALIGNMENT
 
 
 def test_selftest_wait_limit_is_checked_on_the_host(L):
