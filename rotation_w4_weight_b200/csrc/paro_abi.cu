@@ -458,40 +458,70 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N, int gsz) {
   return p;
 }
 
-// Prefill (M > 16): tcgen05 GEMM, 256 token rows x 256 output columns per CTA.
-template <int SR, typename TA>
-int launch_w4_prefill_sr(const TA* xa, TA* y, int64_t M, int64_t K, int64_t N,
-                         const int32_t* qweight, const int32_t* qzeros, const TA* scales,
-                         const TA* bias, int gsz, cudaStream_t s, bool pdl) {
-  CUtensorMap tmA, tmW, tmS, tmZ, tmY;
-  bool ok = encode_2d(&tmA, tma_dt<TA>(), 2, xa, M, K, kTcMB * kTcBM, kTcBK,
-                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, kTcBK, kTcBN / 8,
-                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&tmS, tma_dt<TA>(), 2, scales, K / gsz, N, SR, kTcBN,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
-            encode_2d(&tmZ, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qzeros, K / gsz, N / 8, SR, kTcBN / 8,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
-            encode_2d(&tmY, tma_dt<TA>(), 2, y, M, N, kTcMB * kTcBM, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!ok) return PARO_ERR_CUDA;
-  const dim3 grid((unsigned)((N + kTcBN - 1) / kTcBN), (unsigned)((M + kTcMB * kTcBM - 1) / (kTcMB * kTcBM)), 1);
-  if (grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
+// One linear of a prefill GEMM launch.
+struct PrefillLinear {
+  const void* x;          // the activations the GEMM reads (X_r, or x itself)
+  void* y;
+  int64_t N;
+  const int32_t* qweight;
+  const int32_t* qzeros;
+  const void* scales;
+  const void* bias;
+};
+
+// Prefill (M > 16): tcgen05 GEMM, 256 token rows x 256 output columns per CTA,
+// one launch over the column tiles of `count` (<= NL) linears sharing M and K.
+template <int SR, typename TA, int NL>
+int launch_w4_prefill_nl(const PrefillLinear* lin, int count, int64_t M, int64_t K, int gsz, cudaStream_t s,
+                         bool pdl) {
+  if (count < 1 || count > NL) return PARO_ERR_UNSUPPORTED;
+  TcBatch<NL> b;
+  std::memset(&b, 0, sizeof(b));
+  int64_t tiles = 0;
+  for (int i = 0; i < NL; ++i) {
+    TcOperand& o = b.op[i];
+    if (i >= count) {
+      o.tile_begin = INT_MAX;                   // never selected
+      continue;
+    }
+    const int64_t N = lin[i].N;
+    const bool ok =
+        encode_2d(&o.a, tma_dt<TA>(), 2, lin[i].x, M, K, kTcMB * kTcBM, kTcBK, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        encode_2d(&o.w, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qweight, K, N / 8, kTcBK, kTcBN / 8,
+                  CU_TENSOR_MAP_SWIZZLE_128B) &&
+        encode_2d(&o.s, tma_dt<TA>(), 2, lin[i].scales, K / gsz, N, SR, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, K / gsz, N / 8, SR, kTcBN / 8,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        encode_2d(&o.y, tma_dt<TA>(), 2, lin[i].y, M, N, kTcMB * kTcBM, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return PARO_ERR_CUDA;
+    o.bias = lin[i].bias;
+    o.n = (int)N;
+    o.tile_begin = (int)tiles;
+    tiles += (N + kTcBN - 1) / kTcBN;
+  }
+  const dim3 grid((unsigned)tiles, (unsigned)((M + kTcMB * kTcBM - 1) / (kTcMB * kTcBM)), 1);
+  if (tiles > INT_MAX / 2 || grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
   using L = TcLayoutT<SR>;
-  if (!allow_smem(w4_tc_gemm_kernel<SR, TA>, L::SMEM)) return PARO_ERR_CUDA;
-  return launch(w4_tc_gemm_kernel<SR, TA>, grid, dim3(kTcThreads), L::SMEM, s, pdl, tmA, tmW, tmS,
-                tmZ, tmY, bias, (int)M, (int)N, (int)K, gsz);
+  auto k = w4_tc_gemm_kernel<SR, TA, NL>;
+  if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
+  return launch(k, grid, dim3(kTcThreads), L::SMEM, s, pdl, b, (int)M, (int)K, gsz);
+}
+
+template <int SR, typename TA>
+int launch_w4_prefill_sr(const PrefillLinear* lin, int count, int64_t M, int64_t K, int gsz, cudaStream_t s,
+                         bool pdl) {
+  return count == 1 ? launch_w4_prefill_nl<SR, TA, 1>(lin, count, M, K, gsz, s, pdl)
+                    : launch_w4_prefill_nl<SR, TA, kTcMaxLinears>(lin, count, M, K, gsz, s, pdl);
 }
 
 template <typename TA>
-int launch_w4_prefill(const TA* xa, TA* y, int64_t M, int64_t K, int64_t N,
-                      const int32_t* qweight, const int32_t* qzeros, const TA* scales,
-                      const TA* bias, int gsz, cudaStream_t s, bool pdl) {
+int launch_w4_prefill(const PrefillLinear* lin, int count, int64_t M, int64_t K, int gsz, cudaStream_t s,
+                      bool pdl) {
   // scale rows per 64-row k-block: 64 / G groups below G = 64
   switch (gsz) {
-    case 32: return launch_w4_prefill_sr<2, TA>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
-    case 16: return launch_w4_prefill_sr<4, TA>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
-    default: return launch_w4_prefill_sr<1, TA>(xa, y, M, K, N, qweight, qzeros, scales, bias, gsz, s, pdl);
+    case 32: return launch_w4_prefill_sr<2, TA>(lin, count, M, K, gsz, s, pdl);
+    case 16: return launch_w4_prefill_sr<4, TA>(lin, count, M, K, gsz, s, pdl);
+    default: return launch_w4_prefill_sr<1, TA>(lin, count, M, K, gsz, s, pdl);
   }
 }
 
@@ -864,9 +894,10 @@ int linear_impl(const void* x, void* y, int64_t M, int64_t K, int64_t N, const i
     xa = xr;
   }
 
-  if (!plan.decode)
-    return launch_w4_prefill<TA>(xa, static_cast<TA*>(y), M, K, N, qweight, qzeros, static_cast<const TA*>(scales),
-                                 static_cast<const TA*>(bias), G, s, pdl);
+  if (!plan.decode) {
+    const PrefillLinear one{xa, y, N, qweight, qzeros, scales, bias};
+    return launch_w4_prefill<TA>(&one, 1, M, K, G, s, pdl);
+  }
 
   const GemvLinearArgs one{qweight, qzeros, scales, xa, bias, y, N};
   return dispatch_gemv<TA>(plan, &one, 1, M, K, s, pdl);
@@ -901,7 +932,8 @@ int paro_w4_linear_dt(const void* x, void* y, int64_t M, int64_t K, int64_t N,
   }
 }
 
-static_assert(PARO_MAX_GROUP == kGvMaxLinears && PARO_MAX_GROUP == kRrMaxLinears && PARO_MAX_GROUP == kRcMaxMembers,
+static_assert(PARO_MAX_GROUP == kGvMaxLinears && PARO_MAX_GROUP == kRrMaxLinears && PARO_MAX_GROUP == kRcMaxMembers &&
+                  PARO_MAX_GROUP == kTcMaxLinears,
               "one launch holds every member of a group");
 
 }  // extern "C"
@@ -953,11 +985,15 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
   // prefill batches rotating on the tensor cores: one R' build and one X R'
   // launch for all rotating members, then one GEMM each
   const int G = group_of(group_size, K);
-  if (make_plan(M, K, linears[0].N, G).rot_tc) {
-    // an R' build only for rotations without a prepared R'
+  const LinearPlan first = make_plan(M, K, linears[0].N, G);
+  if (!first.decode) {
+    // prefill: one GEMM launch for the whole group.  Above 64 rows one X R'
+    // launch for all rotating members, after one R' build for those without
+    // a prepared R'; below, a launch per distinct rotation.
+    if (!first.rot_tc) return rot + 1;
     bool build = false;
     for (int i = 0; i < count; ++i) build = build || (rotation_owner(linears, i) == i && linears[i].rmat == nullptr);
-    return (rot > 0 ? (build ? 2 : 1) : 0) + count;
+    return (rot > 0 ? (build ? 2 : 1) : 0) + 1;
   }
   LinearPlan gp;
   // one after another: each rotating member launches its rotation and its GEMV / GEMM
@@ -992,9 +1028,12 @@ int group_impl(const void* x, int64_t M, int64_t K, int count, const paro_linear
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
   const LinearPlan first = make_plan(M, K, linears[0].N, G);
-  if (count > 1 && first.rot_tc) {
-    // prefill: every rotating member's X_r in one R' build + one X R' launch
-    // (x is read once per tile for all of them), then one GEMM per member
+  if (count > 1 && !first.decode) {
+    // prefill: every distinct rotation's X_r, then one GEMM launch over every
+    // member's column tiles.  Above 64 rows the rotating members share one
+    // R' build (members with a prepared R' skip it) and one X R' launch (x
+    // is read once per tile for all of them); below, each distinct rotation
+    // is its own launch.
     RotTcMember rm[PARO_MAX_GROUP];
     int nrot = 0;
     const TA* xs[PARO_MAX_GROUP];
@@ -1005,23 +1044,26 @@ int group_impl(const void* x, int64_t M, int64_t K, int count, const paro_linear
       if (o < 0) continue;
       TA* xr = reinterpret_cast<TA*>(ws + o * per + first.off_xr);
       if (o == i) {
-        const bool pre = l.rmat != nullptr;
-        rm[nrot++] = RotTcMember{l.channel_scales, l.pairs, l.theta, l.krot, xr,
-                                 pre ? const_cast<void*>(l.rmat) : static_cast<void*>(ws + i * per + first.off_rt),
-                                 pre};
+        if (first.rot_tc) {
+          const bool pre = l.rmat != nullptr;
+          rm[nrot++] = RotTcMember{l.channel_scales, l.pairs, l.theta, l.krot, xr,
+                                   pre ? const_cast<void*>(l.rmat) : static_cast<void*>(ws + i * per + first.off_rt),
+                                   pre};
+        } else if (int st = launch_rotate<TA>(static_cast<const TA*>(x), xr, M, K, l.channel_scales, l.pairs,
+                                              l.theta, l.krot, G, s)) {
+          return st;
+        }
       }
       xs[i] = xr;
     }
     if (nrot > 0)
       if (int st = launch_rotate_tc<TA>(static_cast<const TA*>(x), rm, nrot, M, K, G, s)) return st;
+    PrefillLinear pl[PARO_MAX_GROUP];
     for (int i = 0; i < count; ++i) {
       const paro_linear& l = linears[i];
-      if (int st = launch_w4_prefill<TA>(xs[i], static_cast<TA*>(l.y), M, K, l.N, l.qweight, l.qzeros,
-                                         static_cast<const TA*>(l.scales), static_cast<const TA*>(l.bias), G, s,
-                                         true))
-        return st;
+      pl[i] = PrefillLinear{xs[i], l.y, l.N, l.qweight, l.qzeros, l.scales, l.bias};
     }
-    return PARO_OK;
+    return launch_w4_prefill<TA>(pl, count, M, K, G, s, true);
   }
 
   LinearPlan gp;

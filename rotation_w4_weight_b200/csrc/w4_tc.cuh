@@ -92,12 +92,42 @@ struct TcLayoutT {
 // instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M=128, N=256
 constexpr uint32_t kTcIdesc = (1u << 4) | ((uint32_t)(kTcBN >> 3) << 17) | ((uint32_t)(kTcBM >> 4) << 24);
 
-template <int SR, typename TA>
-__global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
-    const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
-    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
-    const __grid_constant__ CUtensorMap tmY, const TA* __restrict__ bias, int M, int N, int K, int gsz) {
+// Operands of one linear of a launch.  A launch covers NL linears that share
+// M and K (a decoder layer's q/k/v, say), each with its own activations (its
+// X_r), weights and output: the column tiles of linear l are blockIdx.x =
+// tile_begin .. tile_begin + ceil(n / 256) - 1.
+struct alignas(64) TcOperand {
+  CUtensorMap a;          // X_r [M, K], box {64, 256}, 128-byte swizzle
+  CUtensorMap w;          // qweight [K, N/8] int32, box {32 words, 64 rows}, 128-byte swizzle
+  CUtensorMap s;          // scales [K/G, N], box {256, SR}
+  CUtensorMap z;          // qzeros [K/G, N/8] int32, box {32, SR}
+  CUtensorMap y;          // Y [M, N], box {64, 256}, 128-byte swizzle
+  const void* bias;       // [N] or nullptr (activation type)
+  int n;                  // output columns
+  int tile_begin;         // first column tile of this linear in the grid
+};
+constexpr int kTcMaxLinears = 4;
+template <int NL>
+struct TcBatch {
+  TcOperand op[NL];
+};
+
+template <int SR, typename TA, int NL>
+__global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(const __grid_constant__ TcBatch<NL> ops,
+                                                                   int M, int K, int gsz) {
   using L = TcLayoutT<SR>;
+  // this CTA's linear (selected by constant offsets into the parameter block)
+  const TcOperand* op = &ops.op[0];
+#pragma unroll
+  for (int i = 1; i < NL; ++i)
+    if ((int)blockIdx.x >= ops.op[i].tile_begin) op = &ops.op[i];
+  const CUtensorMap* const tmA = &op->a;
+  const CUtensorMap* const tmW = &op->w;
+  const CUtensorMap* const tmS = &op->s;
+  const CUtensorMap* const tmZ = &op->z;
+  const CUtensorMap* const tmY = &op->y;
+  const TA* __restrict__ const bias = static_cast<const TA*>(op->bias);
+  const int N = op->n;
   constexpr int kTcBBufs = L::BBUFS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -111,7 +141,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
   volatile int* abort = reinterpret_cast<volatile int*>(sbase + L::MISC_OFF + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * kTcBN;
+  const int n0 = ((int)blockIdx.x - op->tile_begin) * kTcBN;
   const int tok0 = blockIdx.y * (kTcMB * kTcBM);
   const int nk = K / kTcBK;
 
@@ -127,11 +157,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     mbar_init(accum_full, 1);
     *abort = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmW);
-    tma_prefetch_desc(&tmS);
-    tma_prefetch_desc(&tmZ);
-    tma_prefetch_desc(&tmY);
+    tma_prefetch_desc(tmA);
+    tma_prefetch_desc(tmW);
+    tma_prefetch_desc(tmS);
+    tma_prefetch_desc(tmZ);
+    tma_prefetch_desc(tmY);
   }
   if (warp == 1) {                      // the whole warp allocates 2 x 256 TMEM columns
     tmem_alloc(smem_u32(tmem_slot), kTcMB * kTcBN);
@@ -150,22 +180,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
       for (int kb = 0; kb < pre; ++kb) {
         const uint32_t st = base + kb * L::STAGE, bar = tma_full0 + 8 * kb;
         mbar_arrive_expect_tx(bar, L::TX_BYTES);
-        tma_load_2d(st + L::WQ_OFF, &tmW, bar, n0 / 8, kb * kTcBK);
-        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, (kb * kTcBK) / gsz);
-        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::WQ_OFF, tmW, bar, n0 / 8, kb * kTcBK);
+        tma_load_2d(st + L::S_OFF, tmS, bar, n0, (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::Z_OFF, tmZ, bar, n0 / 8, (kb * kTcBK) / gsz);
       }
       pdl_wait_primary();               // X_r is written by the rotation kernel
       for (int kb = 0; kb < pre; ++kb)
-        tma_load_2d(base + kb * L::STAGE + L::A_OFF, &tmA, tma_full0 + 8 * kb, kb * kTcBK, tok0);
+        tma_load_2d(base + kb * L::STAGE + L::A_OFF, tmA, tma_full0 + 8 * kb, kb * kTcBK, tok0);
       for (int kb = pre; kb < nk; ++kb) {
         const int s = kb % kTcStages;
         if (!tc_wait(tma_empty0 + 8 * s, ((kb / kTcStages) - 1) & 1, abort)) break;
         const uint32_t st = base + s * L::STAGE, bar = tma_full0 + 8 * s;
         mbar_arrive_expect_tx(bar, L::TX_BYTES);
-        tma_load_2d(st + L::WQ_OFF, &tmW, bar, n0 / 8, kb * kTcBK);
-        tma_load_2d(st + L::S_OFF, &tmS, bar, n0, (kb * kTcBK) / gsz);
-        tma_load_2d(st + L::Z_OFF, &tmZ, bar, n0 / 8, (kb * kTcBK) / gsz);
-        tma_load_2d(st + L::A_OFF, &tmA, bar, kb * kTcBK, tok0);
+        tma_load_2d(st + L::WQ_OFF, tmW, bar, n0 / 8, kb * kTcBK);
+        tma_load_2d(st + L::S_OFF, tmS, bar, n0, (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::Z_OFF, tmZ, bar, n0 / 8, (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::A_OFF, tmA, bar, kb * kTcBK, tok0);
       }
     }
   } else if (warp == 1) {
@@ -333,7 +363,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(
     if (warp == 2 && lane == 0 && !*abort) {
 #pragma unroll
       for (int b = 0; b < kTcBN / 64; ++b)
-        if (n0 + 64 * b < N) tma_store_2d(&tmY, base + (uint32_t)b * L::O_BOX, n0 + 64 * b, tok0);
+        if (n0 + 64 * b < N) tma_store_2d(tmY, base + (uint32_t)b * L::O_BOX, n0 + 64 * b, tok0);
       bulk_commit_group();
       bulk_wait_group_all();            // written before the kernel completes
     }

@@ -187,23 +187,26 @@ def test_group_launch_count_query(L):
     qkv = [dict(N=4096), dict(N=1024), dict(N=1024)]
     n = pb.w4_linear_group_launches(1, 4096, qkv)
     assert n in (2, 6)                        # shared launches, or one rotation + one GEMV each
-    # prefill above 64 rows: one R' build and one X R' launch for all rotating
-    # members, then one GEMM each; up to 64 rows one rotation + one GEMM per member
-    assert pb.w4_linear_group_launches(4096, 4096, qkv) == 5
-    assert pb.w4_linear_group_launches(65, 4096, qkv) == 5
-    assert pb.w4_linear_group_launches(64, 4096, qkv) == 6
+    # prefill: one GEMM launch for the whole group; above 64 rows one R' build
+    # and one X R' launch for all rotating members, up to 64 rows one rotation
+    # launch per member
+    assert pb.w4_linear_group_launches(4096, 4096, qkv) == 3
+    assert pb.w4_linear_group_launches(65, 4096, qkv) == 3
+    assert pb.w4_linear_group_launches(64, 4096, qkv) == 4
+    assert pb.w4_linear_group_launches(17, 4096, qkv) == 4
     # prepared R' parts skip the build (one member without them still builds)
     qkv_r = [dict(m, rmat=True) for m in qkv]
-    assert pb.w4_linear_group_launches(4096, 4096, qkv_r) == 4
-    assert pb.w4_linear_group_launches(4096, 4096, [qkv_r[0], qkv[1]]) == 4
+    assert pb.w4_linear_group_launches(4096, 4096, qkv_r) == 2
+    assert pb.w4_linear_group_launches(4096, 4096, [qkv_r[0], qkv[1]]) == 3
     assert pb.w4_linear_group_launches(4096, 4096, [dict(N=4096, rmat=True)]) == 2
+    assert pb.w4_linear_group_launches(4096, 4096, [dict(N=4096)]) == 3
     assert pb.w4_linear_group_launches(1, 4096, qkv_r) in (2, 6)          # decode does not use R'
-    assert pb.w4_linear_group_launches(4096, 4096, [dict(N=4096, krot=0, channel_scales=False)] * 2) == 2
+    assert pb.w4_linear_group_launches(4096, 4096, [dict(N=4096, krot=0, channel_scales=False)] * 2) == 1
     # experts sharing one rotation rotate x once: one rotation (not three) up to
     # 64 rows, and the single-rotation count on the other paths
     shared = [dict(N=1024), dict(N=1024, same_rotation_as=0), dict(N=1024, same_rotation_as=0)]
-    assert pb.w4_linear_group_launches(64, 4096, shared) == 1 + 3
-    assert pb.w4_linear_group_launches(4096, 4096, shared) == 2 + 3
+    assert pb.w4_linear_group_launches(64, 4096, shared) == 1 + 1
+    assert pb.w4_linear_group_launches(4096, 4096, shared) == 2 + 1
     assert pb.w4_linear_group_launches(1, 4096, shared) in (2, 4)
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096)]) == 2
     assert pb.w4_linear_group_launches(1, 4096, [dict(N=4096, krot=0, channel_scales=False)]) == 1
