@@ -227,6 +227,40 @@ def w4_linear_columns(x, codes, zero_codes, scales, bias, channel_scales, pairs,
     return Y
 
 
+def moe_linear_from_codes(x, expert_idx, codes, zero_codes, scales, bias, channel_scales, pairs, theta,
+                          group_size, krot):
+    """Stacked experts sharing one rotation (brain.gartu.xyz ParoQuant page,
+    MLX section: the experts' weights are stacked in one tensor and their
+    rotations are shared), float64.
+
+    x [T, K]; expert_idx [T, topk] ints; codes [E, N, K] uint8 (out x in per
+    expert); zero_codes [E, N, K//G]; scales [E, K//G, N]; bias [E, N] or None;
+    one channel_scales / pairs / theta for every expert.  Returns y [T, topk, N]:
+        X_r = rotate(x * channel_scales)                  (once, for all experts)
+        y[t, j] = X_r[t] @ dequant(expert e = expert_idx[t, j]) + bias[e]
+    A slot whose index lies outside 0..E-1 selects no expert: its row is 0
+    (the reading taken for a routing value the pages do not define).
+    """
+    x = np.asarray(x)
+    idx = np.asarray(expert_idx).astype(np.int64)
+    T, K = x.shape
+    E, N = codes.shape[0], codes.shape[1]
+    topk = idx.shape[1]
+    G = normalize_group_size(group_size, K)
+    xr = rotate(x, channel_scales, pairs, theta, G, krot=krot)
+    y = np.zeros((T, topk, N))
+    for e in range(E):
+        t_sel, j_sel = np.nonzero(idx == e)
+        if t_sel.size == 0:
+            continue
+        W = dequant(codes[e], zero_codes[e], scales[e], G)            # [K, N]
+        ye = xr[t_sel] @ W
+        if bias is not None:
+            ye += np.asarray(bias[e], dtype=np.float64).reshape(1, N)
+        y[t_sel, j_sel] = ye
+    return y
+
+
 def transform_weight(W: np.ndarray, channel_scales: Optional[np.ndarray], pairs: Optional[np.ndarray],
                      theta: Optional[np.ndarray], group_size: int, krot: Optional[int] = None) -> np.ndarray:
     """W_r = W D R in float64: row n of W [N, K] (out x in) is multiplied by

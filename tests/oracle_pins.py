@@ -441,6 +441,57 @@ def pin_quantize_weight_packed(impl):
     assert np.array_equal(np.asarray(qw2), qw)
 
 
+def pin_moe_stacked_experts_brute_force(impl):
+    """moe_linear_from_codes against a route that shares none of its steps:
+    X_r = (x * cs) @ R with R the dense product of per-stage Givens matrices
+    built entry by entry (one rotation for every expert), then every output of
+    every slot summed one term at a time with the slot's expert's codes, zero
+    points, scales and bias.  The routing has an expert no token selects, an
+    expert selected twice by one token, ragged per-expert counts and one
+    index outside 0..E-1 (its row must be 0)."""
+    rng = np.random.default_rng(25)
+    T, K, N, G, E, topk, krot = 4, 128, 8, 64, 4, 2, 3
+    pairs, theta = _rand_tables(rng, K, G, krot)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))
+    x = rng.standard_normal((T, K))
+    codes = rng.integers(0, 16, (E, N, K), dtype=np.uint8)
+    zeros = rng.integers(0, 16, (E, N, K // G), dtype=np.uint8)
+    scales = rng.uniform(0.005, 0.02, (E, K // G, N))
+    bias = rng.standard_normal((E, N))
+    idx = np.array([[2, 0], [2, 2], [0, 3], [E, 2]])          # expert 1 empty; (3, 0) invalid
+    xr = (x * cs) @ dense_R(pairs, theta, K, G)
+    ref = np.zeros((T, topk, N))
+    for t in range(T):
+        for j in range(topk):
+            e = int(idx[t, j])
+            if not 0 <= e < E:
+                continue
+            ref[t, j] = _brute_linear(xr[t:t + 1], codes[e], zeros[e], scales[e], bias[e], G)[0]
+    got = np.asarray(impl.moe_linear_from_codes(x, idx, codes, zeros, scales, bias, cs, pairs, theta, G, krot))
+    assert got.shape == (T, topk, N), got.shape
+    assert np.max(np.abs(got - ref)) <= 1e-10 * np.max(np.abs(ref))
+    # no bias: the rows of the invalid slot stay exactly zero as well
+    got0 = np.asarray(impl.moe_linear_from_codes(x, idx, codes, zeros, scales, None, cs, pairs, theta, G, krot))
+    assert np.all(got0[3, 0] == 0.0)
+
+
+def pin_moe_single_expert_is_the_dense_layer(impl):
+    """With one expert and top-1 routing the layer is the dense rotated W4
+    linear (itself pinned above), token for token."""
+    rng = np.random.default_rng(26)
+    T, K, N, G, krot = 5, 256, 16, 128, 4
+    pairs, theta = _rand_tables(rng, K, G, krot)
+    cs = np.exp(rng.uniform(np.log(0.5), np.log(2), K))
+    x = rng.standard_normal((T, K))
+    codes = rng.integers(0, 16, (1, N, K), dtype=np.uint8)
+    zeros = rng.integers(0, 16, (1, N, K // G), dtype=np.uint8)
+    scales = rng.uniform(0.005, 0.02, (1, K // G, N))
+    got = np.asarray(impl.moe_linear_from_codes(x, np.zeros((T, 1), np.int64), codes, zeros, scales, None, cs,
+                                                pairs, theta, G, krot))
+    ref = impl.w4_linear_from_codes(x, codes[0], zeros[0], scales[0], None, cs, pairs, theta, G, krot)
+    assert np.max(np.abs(got[:, 0] - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
 ALL_PINS = [
     pin_single_pair_closed_forms, pin_stage_composition, pin_inverse_restores,
     pin_group_norms_preserved, pin_dense_R_brute_force, pin_golden_g4,
@@ -448,5 +499,6 @@ ALL_PINS = [
     pin_awq_one_hot, pin_awq_round_trip, pin_identity_state_is_plain_w4,
     pin_equivalent_weight_route, pin_dequant_formula,
     pin_weight_transform_identity, pin_sym4_closed_forms, pin_sym4_nearest_level_brute_force,
-    pin_quantized_replay, pin_quantize_weight_packed,
+    pin_quantized_replay, pin_quantize_weight_packed, pin_moe_stacked_experts_brute_force,
+    pin_moe_single_expert_is_the_dense_layer,
 ]

@@ -16,7 +16,8 @@ def make_impl(sign_flip=False, reverse_stages=False, swap_roles=False, no_scale=
               theta_global=False, order=ORDER_OK, no_zero=False, group0_scale=False,
               inverse_forward_order=False, shared_group_base=False, q_half_away=False,
               q_clamp7=False, q_no_offset=False, w_scale_multiplied=False, q_group0_scale=False,
-              q_no_bound=False, w_no_stages=False, qw_no_stages=False, qw_untransposed=False):
+              q_no_bound=False, w_no_stages=False, qw_no_stages=False, qw_untransposed=False,
+              moe_bias0=False, moe_wrap_invalid=False, moe_no_rotation=False, moe_slot_transposed=False):
     def stage_idx(pairs_s, G):
         K = pairs_s.shape[0]
         local = pairs_s.astype(np.int64)
@@ -119,11 +120,29 @@ def make_impl(sign_flip=False, reverse_stages=False, swap_roles=False, no_scale=
             return awq_pack(np.ascontiguousarray(codes.reshape(codes.shape[1], codes.shape[0])), zeros, G)
         return awq_pack(codes, zeros, G)
 
+    def moe_linear_from_codes(x, idx, codes, zeros, scales, bias, cs, pairs, theta, G, krot):
+        idx = np.asarray(idx).astype(np.int64)
+        T, topk = idx.shape
+        E, N = codes.shape[0], codes.shape[1]
+        xr = np.array(x, np.float64) if moe_no_rotation else rotate(x, cs, pairs, theta, G, krot=krot)
+        y = np.zeros((T, topk, N))
+        for t in range(T):
+            for j in range(topk):
+                e = int(idx[j % T, t % topk]) if moe_slot_transposed else int(idx[t, j])
+                if moe_wrap_invalid:
+                    e %= E                         # an index past the experts wraps around
+                elif not 0 <= e < E:
+                    continue
+                y[t, j] = xr[t] @ dequant(codes[e], zeros[e], scales[e], G)
+                if bias is not None:
+                    y[t, j] += np.asarray(bias[0 if moe_bias0 else e], np.float64)
+        return y
+
     return types.SimpleNamespace(rotate=rotate, inverse_rotate=inverse_rotate, awq_pack=awq_pack,
                                  awq_unpack=awq_unpack, dequant=dequant,
                                  w4_linear_from_codes=w4_linear_from_codes,
                                  transform_weight=transform_weight, quantize_sym4=quantize_sym4,
-                                 quantize_weight=quantize_weight)
+                                 quantize_weight=quantize_weight, moe_linear_from_codes=moe_linear_from_codes)
 
 
 def failing_pins(impl):
@@ -160,6 +179,10 @@ MUTATIONS = {
     "weight_stages_skipped": dict(w_no_stages=True),
     "quantize_weight_drops_the_stages": dict(qw_no_stages=True),
     "quantize_weight_packs_untransposed_codes": dict(qw_untransposed=True),
+    "moe_bias_of_the_first_expert": dict(moe_bias0=True),
+    "moe_invalid_index_wraps_around": dict(moe_wrap_invalid=True),
+    "moe_rotation_skipped": dict(moe_no_rotation=True),
+    "moe_slots_read_transposed": dict(moe_slot_transposed=True),
 }
 
 
