@@ -309,6 +309,45 @@ int paro_rotation_matrix_prepare(const float* channel_scales, const int16_t* pai
                                  paro_stream_t stream);
 
 /*
+ * paro_w4_moe_linear — stacked experts that share one rotation: one
+ * projection of a mixture-of-experts block (brain.gartu.xyz ParoQuant page,
+ * MLX section: the experts' weights are stacked in one tensor and their
+ * rotations are shared; each expert is the rotated W4 linear of the page
+ * "ParoQuant", "Activation and weight transforms"):
+ *   X_r = rotate(x * channel_scales)                   once, for every expert
+ *   y[t, j, :] = X_r[t] . dequant(expert e) + bias[e],  e = expert_idx[t, j]
+ *   x            device [T, K] (dtype), T >= 0 tokens (T == 0 is a no-op)
+ *   expert_idx   device int32 [T, topk], 1 <= topk <= 64: the router's choice
+ *                per token (any order; an expert may appear more than once)
+ *   qweight      device int32 [E, K, N/8]; qzeros int32 [E, K/G, N/8];
+ *   scales       [E, K/G, N] (dtype); bias [E, N] (dtype) or NULL;
+ *                1 <= E <= 1024, each expert packed as for paro_w4_linear
+ *   channel_scales, pairs, theta, krot: the one rotation of every expert
+ *   y            device [T, topk, N] (dtype)
+ *   workspace    >= paro_w4_moe_workspace_size(...) bytes, 256-byte aligned
+ *   Shapes as for paro_w4_linear with M = T * topk (< 2^24); E * K < 2^31.
+ * The call rotates x once, sorts the T * topk slots by expert on the device
+ * (a stable counting sort: deterministic), copies each slot's X_r row into
+ * the sorted order, then runs the decode GEMV over segments of at most 8
+ * rows of one expert (T <= 16) or the tcgen05 GEMM over tiles of at most 256
+ * rows of one expert, each writing its rows straight to their slots.  An
+ * expert that no token selects costs nothing.  A slot whose index lies
+ * outside 0..E-1 gets a zero row and is flagged in the device status word
+ * (paro_device_status then reports PARO_ERR_INVALID_ARG).  Arithmetic as for
+ * paro_w4_linear.  paro_w4_moe_launches is a host-only query of the kernel
+ * launches one call issues (rotate != 0: the call rotates), 0 for a rejected
+ * shape.
+ */
+size_t paro_w4_moe_workspace_size(int64_t T, int64_t K, int64_t N, int E, int topk, int group_size);
+int paro_w4_moe_linear(const void* x, void* y, int64_t T, int64_t K, int64_t N, int E, int topk,
+                       const int32_t* expert_idx, const int32_t* qweight, const int32_t* qzeros,
+                       const void* scales, const void* bias, const float* channel_scales,
+                       const int16_t* pairs, const float* theta, int group_size, int krot, int dtype,
+                       void* workspace, size_t workspace_bytes, paro_stream_t stream);
+int paro_w4_moe_launches(int64_t T, int64_t K, int64_t N, int E, int topk, int group_size, int krot,
+                         int rotate);
+
+/*
  * paro_w4_linear_noalloc — paro_w4_linear for callers that cannot allocate
  * device memory.  The paper has no counterpart; this entry point exists for
  * library users, not for the method.
@@ -363,7 +402,8 @@ int paro_validate_pairs(const int16_t* pairs_host, int64_t K, int group_size, in
  * paro_device_status — reads (and, if clear != 0, resets) the device status word
  * of the current device.  Synchronises the device.  Returns PARO_OK,
  * PARO_ERR_TIMEOUT (a bounded wait ran out), PARO_ERR_INVALID_ARG (a pair index
- * outside its group was seen) or PARO_ERR_CUDA (the CUDA query failed).
+ * outside its group, or an expert index outside 0..E-1, was seen) or
+ * PARO_ERR_CUDA (the CUDA query failed).
  */
 int paro_device_status(int clear);
 

@@ -13,6 +13,7 @@ streams) into that ABI.  Functions mirror the C entry points:
     validate_pairs    -> paro_validate_pairs (host helper)
     device_status     -> paro_device_status
     rotation_matrix   -> paro_rotation_matrix_prepare (+ paro_rotation_matrix_size)
+    w4_moe_linear     -> paro_w4_moe_linear (+ paro_w4_moe_workspace_size, paro_w4_moe_launches)
 
 Activations, scales, bias and outputs are fp16 or bf16 (one type per call,
 taken from x): fp16 calls go to the plain entry points, bf16 calls to the
@@ -34,11 +35,12 @@ from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # n
                    PARO_MAX_GROUP, ParoLinear, paro_w4_linear_group, paro_w4_linear_group_launches,
                    paro_w4_linear_group_workspace_size, PARO_DTYPE_BF16, paro_rotate_dt, paro_quantize_w4_dt,
                    paro_w4_linear_dt, paro_w4_linear_group_dt, paro_rotation_matrix_size,
-                   paro_rotation_matrix_prepare, PARO_DTYPE_F16)
+                   paro_rotation_matrix_prepare, PARO_DTYPE_F16, paro_w4_moe_workspace_size,
+                   paro_w4_moe_linear, paro_w4_moe_launches)
 
 __all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
            "w4_linear_group", "w4_linear_group_launches", "quantize_w4", "validate_pairs", "device_status",
-           "rotation_matrix", "ParoError", "LIB_PATH"]
+           "rotation_matrix", "w4_moe_linear", "w4_moe_launches", "ParoError", "LIB_PATH"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -310,3 +312,47 @@ def rotation_matrix(channel_scales: Optional[torch.Tensor], pairs: Optional[torc
     check(paro_rotation_matrix_prepare(_ptr(channel_scales), _ptr(pairs), _ptr(theta), K, group_size, krot, code,
                                        _ptr(out), n, _stream(stream)), "paro_rotation_matrix_prepare")
     return out
+
+
+def w4_moe_linear(x: torch.Tensor, expert_idx: torch.Tensor, qweight: torch.Tensor, qzeros: torch.Tensor,
+                  scales: torch.Tensor, bias: Optional[torch.Tensor], channel_scales: Optional[torch.Tensor],
+                  pairs: Optional[torch.Tensor], theta: Optional[torch.Tensor], group_size: int = 128,
+                  krot: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Stacked experts sharing one rotation: y[t, j] = rotate(x[t]) @ W[expert_idx[t, j]] + b[...].
+
+    x [T, K]; expert_idx int32 [T, topk]; qweight int32 [E, K, N/8]; qzeros
+    int32 [E, K/G, N/8]; scales [E, K/G, N]; bias [E, N] or None.  Returns
+    y [T, topk, N] in x's type."""
+    dt = _act(x, "x")
+    _need(x, dt, "x")
+    _need(expert_idx, torch.int32, "expert_idx")
+    _need(qweight, torch.int32, "qweight")
+    _need(qzeros, torch.int32, "qzeros")
+    _need(scales, dt, "scales")
+    _need(bias, dt, "bias", True)
+    _need(channel_scales, torch.float32, "channel_scales", True)
+    _need(pairs, torch.int16, "pairs", True)
+    _need(theta, torch.float32, "theta", True)
+    if krot is None:
+        krot = 0 if pairs is None else pairs.shape[0]
+    T, K = x.shape
+    topk = expert_idx.shape[1] if expert_idx.dim() == 2 else 1
+    E, N = qweight.shape[0], qweight.shape[2] * 8
+    if out is None:
+        out = torch.empty((T, topk, N), dtype=dt, device=x.device)
+    _need(out, dt, "out")
+    need = int(paro_w4_moe_workspace_size(T, K, N, E, topk, group_size))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    check(paro_w4_moe_linear(_ptr(x), _ptr(out), T, K, N, E, topk, _ptr(expert_idx), _ptr(qweight), _ptr(qzeros),
+                             _ptr(scales), _ptr(bias), _ptr(channel_scales), _ptr(pairs), _ptr(theta), group_size,
+                             krot, PARO_DTYPE_F16 if dt == torch.float16 else PARO_DTYPE_BF16, _ptr(workspace),
+                             workspace.numel(), _stream(stream)), "paro_w4_moe_linear")
+    return out
+
+
+def w4_moe_launches(T: int, K: int, N: int, E: int, topk: int, group_size: int = 128, krot: int = 8,
+                    rotate: bool = True) -> int:
+    """Kernel launches one ``w4_moe_linear`` call of this shape issues (host-only)."""
+    return int(paro_w4_moe_launches(T, K, N, E, topk, group_size, krot, 1 if rotate else 0))

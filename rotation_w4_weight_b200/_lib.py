@@ -30,7 +30,7 @@ EXPORTED = (
     "paro_w4_linear_group_workspace_size", "paro_w4_linear_group", "paro_w4_linear_group_launches",
     "paro_selftest_wait_timeout", "paro_rotate_dt", "paro_quantize_w4_dt", "paro_w4_linear_dt",
     "paro_w4_linear_group_dt", "paro_w4_linear_noalloc_dt", "paro_rotation_matrix_size",
-    "paro_rotation_matrix_prepare",
+    "paro_rotation_matrix_prepare", "paro_w4_moe_workspace_size", "paro_w4_moe_linear", "paro_w4_moe_launches",
 )
 
 PARO_MAX_GROUP = 4
@@ -74,6 +74,10 @@ _SIGNATURES = {
                                          _vp, _int, _int, _int, _vp]),
     "paro_rotation_matrix_size": (ctypes.c_size_t, [_i64]),
     "paro_rotation_matrix_prepare": (_int, [_vp, _vp, _vp, _i64, _int, _int, _int, _vp, ctypes.c_size_t, _vp]),
+    "paro_w4_moe_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _int, _int, _int]),
+    "paro_w4_moe_linear": (_int, [_vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                  _int, _int, _int, _vp, ctypes.c_size_t, _vp]),
+    "paro_w4_moe_launches": (_int, [_i64, _i64, _i64, _int, _int, _int, _int, _int]),
 }
 
 
@@ -115,6 +119,9 @@ paro_w4_linear_group_dt = lib.paro_w4_linear_group_dt
 paro_w4_linear_noalloc_dt = lib.paro_w4_linear_noalloc_dt
 paro_rotation_matrix_size = lib.paro_rotation_matrix_size
 paro_rotation_matrix_prepare = lib.paro_rotation_matrix_prepare
+paro_w4_moe_workspace_size = lib.paro_w4_moe_workspace_size
+paro_w4_moe_linear = lib.paro_w4_moe_linear
+paro_w4_moe_launches = lib.paro_w4_moe_launches
 
 
 class ParoError(RuntimeError):

@@ -15,6 +15,7 @@ namespace paro {
 // Device status word bits (read by paro_device_status).
 constexpr unsigned kErrTimeout = 1u;
 constexpr unsigned kErrPairIndex = 2u;
+constexpr unsigned kErrExpertIndex = 4u;
 
 // The library is one translation unit (no relocatable device code), so the
 // status word is defined here, once.

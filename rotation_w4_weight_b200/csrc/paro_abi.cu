@@ -18,6 +18,7 @@
 #include "rotate.cuh"
 #include "rotate_tmem.cuh"
 #include "rotate_tc.cuh"
+#include "moe.cuh"
 #include "w4_gemv.cuh"
 #include "w4_tc.cuh"
 
@@ -458,6 +459,15 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N, int gsz) {
   return p;
 }
 
+// Routing of a stacked-expert launch (segment variants of the GEMV / GEMM).
+struct SegRouting {
+  const int4* segs;       // {expert, first sorted row, rows}
+  const int* count;       // segments written by the routing (device)
+  const int* perm;        // sorted row -> output row
+  int max_segs;           // grid bound on the segment count
+  int experts;            // E: the weight, scale and zero maps cover E stacked experts
+};
+
 // One linear of a prefill GEMM launch.
 struct PrefillLinear {
   const void* x;          // the activations the GEMM reads (X_r, or x itself)
@@ -471,9 +481,9 @@ struct PrefillLinear {
 
 // Prefill (M > 16): tcgen05 GEMM, 256 token rows x 256 output columns per CTA,
 // one launch over the column tiles of `count` (<= NL) linears sharing M and K.
-template <int SR, typename TA, int NL>
+template <int SR, typename TA, int NL, bool SEG = false>
 int launch_w4_prefill_nl(const PrefillLinear* lin, int count, int64_t M, int64_t K, int gsz, cudaStream_t s,
-                         bool pdl) {
+                         bool pdl, const SegRouting* seg = nullptr) {
   if (count < 1 || count > NL) return PARO_ERR_UNSUPPORTED;
   TcBatch<NL> b;
   std::memset(&b, 0, sizeof(b));
@@ -485,24 +495,32 @@ int launch_w4_prefill_nl(const PrefillLinear* lin, int count, int64_t M, int64_t
       continue;
     }
     const int64_t N = lin[i].N;
+    const int64_t E = SEG ? seg->experts : 1;     // stacked experts along the rows
     const bool ok =
         encode_2d(&o.a, tma_dt<TA>(), 2, lin[i].x, M, K, kTcMB * kTcBM, kTcBK, CU_TENSOR_MAP_SWIZZLE_128B) &&
-        encode_2d(&o.w, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qweight, K, N / 8, kTcBK, kTcBN / 8,
+        encode_2d(&o.w, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qweight, E * K, N / 8, kTcBK, kTcBN / 8,
                   CU_TENSOR_MAP_SWIZZLE_128B) &&
-        encode_2d(&o.s, tma_dt<TA>(), 2, lin[i].scales, K / gsz, N, SR, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, K / gsz, N / 8, SR, kTcBN / 8,
+        encode_2d(&o.s, tma_dt<TA>(), 2, lin[i].scales, E * (K / gsz), N, SR, kTcBN, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, E * (K / gsz), N / 8, SR, kTcBN / 8,
                   CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        encode_2d(&o.y, tma_dt<TA>(), 2, lin[i].y, M, N, kTcMB * kTcBM, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+        (SEG || encode_2d(&o.y, tma_dt<TA>(), 2, lin[i].y, M, N, kTcMB * kTcBM, 64, CU_TENSOR_MAP_SWIZZLE_128B));
     if (!ok) return PARO_ERR_CUDA;
     o.bias = lin[i].bias;
     o.n = (int)N;
     o.tile_begin = (int)tiles;
     tiles += (N + kTcBN - 1) / kTcBN;
+    if (SEG) {
+      o.segs = seg->segs;
+      o.seg_count = seg->count;
+      o.perm = seg->perm;
+      o.yptr = lin[i].y;
+    }
   }
-  const dim3 grid((unsigned)tiles, (unsigned)((M + kTcMB * kTcBM - 1) / (kTcMB * kTcBM)), 1);
+  const dim3 grid((unsigned)tiles, SEG ? (unsigned)seg->max_segs
+                                       : (unsigned)((M + kTcMB * kTcBM - 1) / (kTcMB * kTcBM)), 1);
   if (tiles > INT_MAX / 2 || grid.y > 65535u) return PARO_ERR_UNSUPPORTED;
   using L = TcLayoutT<SR>;
-  auto k = w4_tc_gemm_kernel<SR, TA, NL>;
+  auto k = w4_tc_gemm_kernel<SR, TA, NL, SEG>;
   if (!allow_smem(k, L::SMEM)) return PARO_ERR_CUDA;
   return launch(k, grid, dim3(kTcThreads), L::SMEM, s, pdl, b, (int)M, (int)K, gsz);
 }
@@ -512,6 +530,17 @@ int launch_w4_prefill_sr(const PrefillLinear* lin, int count, int64_t M, int64_t
                          bool pdl) {
   return count == 1 ? launch_w4_prefill_nl<SR, TA, 1>(lin, count, M, K, gsz, s, pdl)
                     : launch_w4_prefill_nl<SR, TA, kTcMaxLinears>(lin, count, M, K, gsz, s, pdl);
+}
+
+// One stacked-expert linear: tiles of the routed rows sorted by expert.
+template <typename TA>
+int launch_w4_prefill_seg(const PrefillLinear& lin, int64_t M, int64_t K, int gsz, cudaStream_t s,
+                          const SegRouting& seg) {
+  switch (gsz) {
+    case 32: return launch_w4_prefill_nl<2, TA, 1, true>(&lin, 1, M, K, gsz, s, true, &seg);
+    case 16: return launch_w4_prefill_nl<4, TA, 1, true>(&lin, 1, M, K, gsz, s, true, &seg);
+    default: return launch_w4_prefill_nl<1, TA, 1, true>(&lin, 1, M, K, gsz, s, true, &seg);
+  }
 }
 
 template <typename TA>
@@ -552,10 +581,11 @@ struct GemvLinearArgs {
 
 // Decode GEMV launch over `count` (<= NL) linears sharing M and K: grid
 // (column tiles of every linear, splits), one cluster of `splits` CTAs along K
-// per column tile.
-template <int NT, int KP, int NTILE, int STAGES, int NL, typename TA>
+// per column tile.  With SEG, one stacked-expert linear: grid (segments x
+// column tiles, splits), x = the routed rows sorted by expert.
+template <int NT, int KP, int NTILE, int STAGES, int NL, typename TA, bool SEG = false>
 int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, int64_t M, int64_t K,
-                cudaStream_t s, bool pdl) {
+                cudaStream_t s, bool pdl, const SegRouting* seg = nullptr) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
   const int groups = (int)(K / kGroup);
   const int gmax = (groups + plan.splits - 1) / plan.splits;   // largest group range of a CTA
@@ -571,13 +601,14 @@ int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, in
       continue;
     }
     const int64_t N = lin[i].N;
+    const int64_t E = SEG ? seg->experts : 1;     // stacked experts along the rows
     const bool ok =
-        encode_2d(&o.w, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qweight, K, N / 8, 128, L::WORDS,
+        encode_2d(&o.w, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qweight, E * K, N / 8, 128, L::WORDS,
                   L::ROW_BYTES == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                       : (L::ROW_BYTES == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE)) &&
-        encode_2d(&o.s, tma_dt<TA>(), 2, lin[i].scales, K / plan.gsz, N,
+        encode_2d(&o.s, tma_dt<TA>(), 2, lin[i].scales, E * (K / plan.gsz), N,
                   (uint32_t)(gmax * gq), NTILE, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, K / plan.gsz, N / 8,
+        encode_2d(&o.z, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, lin[i].qzeros, E * (K / plan.gsz), N / 8,
                   (uint32_t)(gmax * gq), L::WORDS, CU_TENSOR_MAP_SWIZZLE_NONE) &&
         encode_x_chunks(&o.x, tma_dt<TA>(), lin[i].x, (uint64_t)M, (uint64_t)K, (uint32_t)L::MP,
                         (uint32_t)(2 * gmax));
@@ -587,11 +618,18 @@ int launch_gemv(const LinearPlan& plan, const GemvLinearArgs* lin, int count, in
     o.n = (int)N;
     o.tile_begin = (int)tiles;
     tiles += (N + NTILE - 1) / NTILE;
+    if (SEG) {
+      o.segs = seg->segs;
+      o.seg_count = seg->count;
+      o.perm = seg->perm;
+      o.seg_tiles = (int)((N + NTILE - 1) / NTILE);
+    }
   }
+  if (SEG) tiles *= seg->max_segs;
   if (tiles > INT_MAX / 2) return PARO_ERR_UNSUPPORTED;
   // G = 128 takes the kernel with the group layout fixed at compile time
-  auto k = plan.gsz == kGroup ? w4_gemv_kernel<NT, KP, NTILE, STAGES, NL, TA, 1>
-                              : w4_gemv_kernel<NT, KP, NTILE, STAGES, NL, TA, 0>;
+  auto k = plan.gsz == kGroup ? w4_gemv_kernel<NT, KP, NTILE, STAGES, NL, TA, 1, SEG>
+                              : w4_gemv_kernel<NT, KP, NTILE, STAGES, NL, TA, 0, SEG>;
   const dim3 grid((unsigned)tiles, (unsigned)plan.splits, 1);
   const size_t smem = gemv_footprint((size_t)L::smem(gmax, gmax * gq), (int64_t)grid.x * grid.y);
   if (smem == 0 || !allow_smem(k, device_info().smem_optin)) return PARO_ERR_CUDA;
@@ -610,6 +648,19 @@ int dispatch_gemv_nl(const LinearPlan& plan, const GemvLinearArgs* lin, int coun
     case 2: return launch_gemv<NT, 4, 128, 8, NL, TA>(plan, lin, count, M, K, s, pdl);
     case 5: return launch_gemv<NT, 4, 64, 8, NL, TA>(plan, lin, count, M, K, s, pdl);
     default: return launch_gemv<NT, 2, 128, 4, NL, TA>(plan, lin, count, M, K, s, pdl);
+  }
+}
+
+// One stacked-expert linear, segments of one token tile.
+template <typename TA>
+int dispatch_gemv_seg(const LinearPlan& plan, const GemvLinearArgs& lin, int64_t M, int64_t K, cudaStream_t s,
+                      const SegRouting& seg) {
+  if (plan.nt != 1) return PARO_ERR_UNSUPPORTED;
+  switch (plan.variant) {
+    case 0: return launch_gemv<1, 2, 256, 4, 1, TA, true>(plan, &lin, 1, M, K, s, true, &seg);
+    case 2: return launch_gemv<1, 4, 128, 8, 1, TA, true>(plan, &lin, 1, M, K, s, true, &seg);
+    case 5: return launch_gemv<1, 4, 64, 8, 1, TA, true>(plan, &lin, 1, M, K, s, true, &seg);
+    default: return launch_gemv<1, 2, 128, 4, 1, TA, true>(plan, &lin, 1, M, K, s, true, &seg);
   }
 }
 
@@ -1141,6 +1192,129 @@ int paro_w4_linear_group_dt(const void* x, int64_t M, int64_t K, int count, cons
 
 }  // extern "C"
 
+// ------------------------------------------------------------ stacked experts
+namespace {
+constexpr int kMoeMaxTopk = 64;
+constexpr int kMoeDecodeMaxT = kMaxDecodeM;    // tokens up to which the segment GEMV runs
+
+// Workspace of a stacked-expert call: X_r [T, K] (when rotating), the sorted
+// rows Xg [S, K], the routing head, perm [S], decode segments [S] and prefill
+// tiles [S] (each segment or tile has at least one row), 256-byte aligned.
+struct MoePlan {
+  size_t off_xr = 0, off_xg = 0, off_head = 0, off_perm = 0, off_gv = 0, off_tc = 0, total = 0;
+};
+MoePlan moe_plan(int64_t T, int64_t K, int64_t S) {
+  MoePlan p;
+  p.off_xr = 0;
+  p.off_xg = round_up((size_t)T * K * 2, 256);
+  p.off_head = p.off_xg + round_up((size_t)S * K * 2, 256);
+  p.off_perm = p.off_head + 256;
+  p.off_gv = p.off_perm + round_up((size_t)S * 4, 256);
+  p.off_tc = p.off_gv + round_up((size_t)S * 16, 256);
+  p.total = p.off_tc + round_up((size_t)S * 16, 256);
+  return p;
+}
+
+int check_moe_shape(int64_t T, int64_t K, int64_t N, int E, int topk, int group_size) {
+  if (T < 0 || E < 1 || topk < 1) return PARO_ERR_INVALID_ARG;
+  if (E > kMoeMaxExperts || topk > kMoeMaxTopk) return PARO_ERR_UNSUPPORTED;
+  const int64_t S = T * topk;
+  if (int st = check_linear_shape(S, K, N, group_size)) return st;
+  // TMA row coordinates of the stacked weights are 32-bit
+  if ((int64_t)E * K >= (int64_t(1) << 31) || S >= (int64_t(1) << 24)) return PARO_ERR_UNSUPPORTED;
+  return PARO_OK;
+}
+
+template <typename TA>
+int moe_impl(const void* x, void* y, int64_t T, int64_t K, int64_t N, int E, int topk, const int32_t* expert_idx,
+             const int32_t* qweight, const int32_t* qzeros, const void* scales, const void* bias,
+             const float* channel_scales, const int16_t* pairs, const float* theta, int group_size, int krot,
+             void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  if (int st = check_moe_shape(T, K, N, E, topk, group_size)) return st;
+  if (krot < 0) return PARO_ERR_INVALID_ARG;
+  if (krot > kMaxKrot) return PARO_ERR_UNSUPPORTED;
+  if (T == 0) return PARO_OK;
+  if (x == nullptr || y == nullptr || expert_idx == nullptr || qweight == nullptr || qzeros == nullptr ||
+      scales == nullptr || workspace == nullptr)
+    return PARO_ERR_INVALID_ARG;
+  if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(qweight, 16) || !aligned(qzeros, 16) || !aligned(scales, 16) ||
+      !aligned(expert_idx, 4) || (bias != nullptr && !aligned(bias, 4)) || !aligned(workspace, 256))
+    return PARO_ERR_ALIGNMENT;
+  if (channel_scales != nullptr && !aligned(channel_scales, 16)) return PARO_ERR_ALIGNMENT;
+  if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
+  const int64_t S = T * topk;
+  const MoePlan mp = moe_plan(T, K, S);
+  if (workspace_bytes < mp.total) return PARO_ERR_WORKSPACE;
+  const int G = group_of(group_size, K);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const TA* xr = static_cast<const TA*>(x);
+  // the rotation is shared by every expert: once, on the T tokens
+  if (krot > 0 || channel_scales != nullptr) {
+    TA* out = reinterpret_cast<TA*>(ws + mp.off_xr);
+    if (int st = launch_rotate<TA>(static_cast<const TA*>(x), out, T, K, channel_scales, pairs, theta, krot, G, s))
+      return st;
+    xr = out;
+  }
+  MoeHead* head = reinterpret_cast<MoeHead*>(ws + mp.off_head);
+  int* perm = reinterpret_cast<int*>(ws + mp.off_perm);
+  int4* gv = reinterpret_cast<int4*>(ws + mp.off_gv);
+  int4* tc = reinterpret_cast<int4*>(ws + mp.off_tc);
+  TA* xg = reinterpret_cast<TA*>(ws + mp.off_xg);
+  if (int st = launch(moe_route_kernel, dim3(1), dim3(kMoeRouteThreads), 0, s, true, expert_idx, (int)S, E, head,
+                      perm, gv, tc, y, (int)(N * 2)))
+    return st;
+  if (int st = launch(moe_gather_kernel<TA>, dim3((unsigned)((S + 7) / 8)), dim3(256), 0, s, true,
+                      static_cast<const MoeHead*>(head), static_cast<const int*>(perm), xr, xg, (int)K, topk))
+    return st;
+  const int64_t used = std::min<int64_t>(E, S);   // experts that can hold a row
+  if (T <= kMoeDecodeMaxT) {
+    // segments of at most 8 rows: one token tile of the decode GEMV each
+    const LinearPlan plan = make_plan(kMoeGvRows, K, N, G);
+    if (plan.decode) {
+      const SegRouting seg{gv, &head->n_gv, perm, (int)std::min<int64_t>(S, S / kMoeGvRows + used), E};
+      const GemvLinearArgs lin{qweight, qzeros, scales, xg, bias, y, N};
+      return dispatch_gemv_seg<TA>(plan, lin, S, K, s, seg);
+    }
+  }
+  const SegRouting seg{tc, &head->n_tc, perm, (int)std::min<int64_t>(S, S / kMoeTcRows + used), E};
+  const PrefillLinear lin{xg, y, N, qweight, qzeros, scales, bias};
+  return launch_w4_prefill_seg<TA>(lin, S, K, G, s, seg);
+}
+}  // namespace
+
+extern "C" {
+
+size_t paro_w4_moe_workspace_size(int64_t T, int64_t K, int64_t N, int E, int topk, int group_size) {
+  if (check_moe_shape(T, K, N, E, topk, group_size) != PARO_OK) return 0;
+  return moe_plan(T, K, T * topk).total;
+}
+
+int paro_w4_moe_linear(const void* x, void* y, int64_t T, int64_t K, int64_t N, int E, int topk,
+                       const int32_t* expert_idx, const int32_t* qweight, const int32_t* qzeros, const void* scales,
+                       const void* bias, const float* channel_scales, const int16_t* pairs, const float* theta,
+                       int group_size, int krot, int dtype, void* workspace, size_t workspace_bytes,
+                       paro_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (dtype) {
+    case PARO_DTYPE_F16:
+      return moe_impl<__half>(x, y, T, K, N, E, topk, expert_idx, qweight, qzeros, scales, bias, channel_scales,
+                              pairs, theta, group_size, krot, workspace, workspace_bytes, s);
+    case PARO_DTYPE_BF16:
+      return moe_impl<__nv_bfloat16>(x, y, T, K, N, E, topk, expert_idx, qweight, qzeros, scales, bias,
+                                     channel_scales, pairs, theta, group_size, krot, workspace, workspace_bytes, s);
+    default: return PARO_ERR_INVALID_ARG;
+  }
+}
+
+int paro_w4_moe_launches(int64_t T, int64_t K, int64_t N, int E, int topk, int group_size, int krot,
+                         int rotate) {
+  if (check_moe_shape(T, K, N, E, topk, group_size) != PARO_OK || T == 0 || krot < 0 || krot > kMaxKrot) return 0;
+  return (rotate ? 1 : 0) + 3;    // rotation, route, gather, expert GEMV or GEMM
+}
+
+}  // extern "C"
+
 // ------------------------------------------------------------ no-allocation variant
 // Scratch for paro_w4_linear_noalloc: a file-scope device array (every GPU that
 // loads the library holds it until exit).  Host code must not pass the symbol
@@ -1227,7 +1401,7 @@ int paro_device_status(int clear) {
     if (cudaMemcpyToSymbol(paro::g_status, &z, sizeof(z)) != cudaSuccess) return PARO_ERR_CUDA;
   }
   if (v & kErrTimeout) return PARO_ERR_TIMEOUT;
-  if (v & kErrPairIndex) return PARO_ERR_INVALID_ARG;
+  if (v & (kErrPairIndex | kErrExpertIndex)) return PARO_ERR_INVALID_ARG;
   return PARO_OK;
 }
 

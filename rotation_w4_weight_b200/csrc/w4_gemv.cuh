@@ -106,6 +106,15 @@ struct alignas(64) GemvOperand {
   void* y;                // [M, N] (activation type)
   int n;                  // output columns
   int tile_begin;         // first column tile of this linear in the grid
+  // Segment variant (stacked experts): the maps cover all E experts (weights
+  // [E*K, N/8], scales and zero words [E*K/G, ...]; x = the routed rows sorted
+  // by expert), and CTA x = segment * seg_tiles + column tile.  Segment s is
+  // segs[s] = {expert, first sorted row, rows <= 8}; sorted row q is output
+  // row perm[q] of y; bias is [E, N].
+  const int4* segs;
+  const int* seg_count;   // segments written by the routing (device)
+  const int* perm;
+  int seg_tiles;
 };
 template <int NL>
 struct GemvBatch {
@@ -144,8 +153,9 @@ __device__ __forceinline__ void gv_mma(bool first, float (&d)[4], const uint32_t
 }
 
 // GQ: quantisation groups per 128 rows fixed at compile time (1: G = 128),
-// or 0 to take them from gq_arg (G = 64, 32, 16).
-template <int NT, int KP, int NTILE, int STAGES, int NL, typename TA, int GQ>
+// or 0 to take them from gq_arg (G = 64, 32, 16).  SEG: the segment variant
+// (one operand, stacked experts, routing read after the kernel ahead).
+template <int NT, int KP, int NTILE, int STAGES, int NL, typename TA, int GQ, bool SEG = false>
 __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kernel(
     const __grid_constant__ GemvBatch<NL> ops, int M, int K, int gmax, int gq_arg) {
   using L = GemvLayout<NT, KP, NTILE, STAGES>;
@@ -158,7 +168,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const CUtensorMap* const tmX = &op->x;
   const CUtensorMap* const tmS = &op->s;
   const CUtensorMap* const tmZ = &op->z;
-  const TA* const bias = static_cast<const TA*>(op->bias);
+  const TA* bias = static_cast<const TA*>(op->bias);
   TA* const Y = static_cast<TA*>(op->y);
   const int N = op->n;
   constexpr int kGvStages = STAGES;
@@ -166,6 +176,23 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   // The next kernel in the stream may launch now; it waits for our completion
   // before it touches anything we read or write.
   pdl_launch_dependents();
+
+  // Segment variant: this CTA's expert and routed rows are written by the
+  // kernels ahead, so everything (weights included) waits for them.  Every
+  // CTA of a cluster has the same segment, so a cluster leaves as a whole.
+  int ntile = (int)blockIdx.x - op->tile_begin;
+  int expert = 0, row0 = 0, seg_rows = M;
+  if constexpr (SEG) {
+    pdl_wait_primary();
+    const int seg = (int)blockIdx.x / op->seg_tiles;
+    ntile = (int)blockIdx.x - seg * op->seg_tiles;
+    if (seg >= *op->seg_count) return;
+    const int4 sg = op->segs[seg];
+    expert = sg.x;
+    row0 = sg.y;
+    seg_rows = sg.z;
+    if (bias != nullptr) bias += (size_t)expert * N;
+  }
 
   extern __shared__ unsigned char smem_raw[];
   // 1024-byte aligned base, derived on the shared array so every access stays LDS/STS
@@ -181,7 +208,7 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const uint32_t xbar = cbar + 8;                  // X_r
   const uint32_t inbar = xbar + 8;                 // peers' split-K partials landed
 
-  const int ntile = (int)blockIdx.x - op->tile_begin, split = blockIdx.y;
+  const int split = blockIdx.y;
   const int n0 = ntile * kGvTile;
   const int groups = K / 128;
   // 32-bit arithmetic (groups <= 2^16, splits <= 8): no 64-bit division routine
@@ -190,7 +217,9 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
   const int ng = g_end - g_begin;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = gridDim.y;                          // CTAs of the cluster along K
-  const int mrows = min(L::MP, M);
+  const int mrows = min(L::MP, seg_rows);
+  // stacked experts: the expert's first weight row and first scale / zero row
+  const int wrow0 = expert * K, qrow0 = expert * (K / 128) * gq;
 
   if (tid == 0) {
     for (int s = 0; s < kGvStages; ++s) {
@@ -232,22 +261,22 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
       // the tensor maps' boxes hold gmax groups (the largest range of any CTA;
       // rows past this CTA's range are loaded and not used)
       mbar_arrive_expect_tx(cbar, (uint32_t)(gr * (NTILE * 2 + L::WORDS * 4)));
-      tma_load_2d(base + L::s_off(gmax), tmS, cbar, n0, g_begin * gq);
-      tma_load_2d(base + L::z_off(gmax, gr), tmZ, cbar, n0 / 8, g_begin * gq);
+      tma_load_2d(base + L::s_off(gmax), tmS, cbar, n0, qrow0 + g_begin * gq);
+      tma_load_2d(base + L::z_off(gmax, gr), tmZ, cbar, n0 / 8, qrow0 + g_begin * gq);
       for (int i = 0; i < pre; ++i) {
         const uint32_t bar = full0 + 8 * i;
         mbar_arrive_expect_tx(bar, L::W_BYTES);
-        tma_load_2d_hint(base + i * L::STAGE, tmW, bar, n0 / 8, (g_begin + i) * 128, pol);
+        tma_load_2d_hint(base + i * L::STAGE, tmW, bar, n0 / 8, wrow0 + (g_begin + i) * 128, pol);
       }
       pdl_wait_primary();                  // X_r comes from the rotation kernel
       mbar_arrive_expect_tx(xbar, (uint32_t)(gmax * L::XG_BYTES));
-      tma_load_3d(base + L::X_OFF, tmX, xbar, 0, 0, 2 * g_begin);
+      tma_load_3d(base + L::X_OFF, tmX, xbar, 0, row0, 2 * g_begin);
       for (int i = pre; i < ng; ++i) {
         const int s = i % kGvStages;
         if (!mbar_wait_bounded(empty0 + 8 * s, ((i / kGvStages) - 1) & 1)) break;
         const uint32_t bar = full0 + 8 * s;
         mbar_arrive_expect_tx(bar, L::W_BYTES);
-        tma_load_2d_hint(base + s * L::STAGE, tmW, bar, n0 / 8, (g_begin + i) * 128, pol);
+        tma_load_2d_hint(base + s * L::STAGE, tmW, bar, n0 / 8, wrow0 + (g_begin + i) * 128, pol);
       }
     }
   } else {
@@ -454,7 +483,8 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     uint2 out;
     out.x = Act<TA>::p2(sum.x, sum.y);
     out.y = Act<TA>::p2(sum.z, sum.w);
-    *reinterpret_cast<uint2*>(Y + (size_t)tl * N + n) = out;
+    const int yrow = SEG ? op->perm[row0 + tl] : tl;
+    *reinterpret_cast<uint2*>(Y + (size_t)yrow * N + n) = out;
   }
   if (S > 1) {
     // returns once every CTA of the cluster has received all its bytes (each

@@ -105,6 +105,15 @@ struct alignas(64) TcOperand {
   const void* bias;       // [N] or nullptr (activation type)
   int n;                  // output columns
   int tile_begin;         // first column tile of this linear in the grid
+  // Segment variant (stacked experts): the maps cover all E experts (weights
+  // [E*K, N/8], scales and zero words [E*K/G, ...]; a = the routed rows sorted
+  // by expert), and blockIdx.y is the tile: segs[y] = {expert, first sorted
+  // row, rows <= 256}; sorted row q is output row perm[q] of y (written with
+  // plain stores, row by row); bias is [E, N].
+  const int4* segs;
+  const int* seg_count;   // tiles written by the routing (device)
+  const int* perm;
+  void* yptr;             // y [rows of y, N] (activation type)
 };
 constexpr int kTcMaxLinears = 4;
 template <int NL>
@@ -112,7 +121,7 @@ struct TcBatch {
   TcOperand op[NL];
 };
 
-template <int SR, typename TA, int NL>
+template <int SR, typename TA, int NL, bool SEG = false>
 __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(const __grid_constant__ TcBatch<NL> ops,
                                                                    int M, int K, int gsz) {
   using L = TcLayoutT<SR>;
@@ -126,8 +135,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(const __grid_
   const CUtensorMap* const tmS = &op->s;
   const CUtensorMap* const tmZ = &op->z;
   const CUtensorMap* const tmY = &op->y;
-  const TA* __restrict__ const bias = static_cast<const TA*>(op->bias);
+  const TA* __restrict__ bias = static_cast<const TA*>(op->bias);
   const int N = op->n;
+  // Segment variant: the tile's expert and rows are written by the kernels
+  // ahead, so the whole CTA waits for them first (before any setup).
+  int expert = 0, tok0 = blockIdx.y * (kTcMB * kTcBM), tile_rows = 0;
+  if constexpr (SEG) {
+    pdl_wait_primary();
+    if ((int)blockIdx.y >= *op->seg_count) return;
+    const int4 sg = op->segs[blockIdx.y];
+    expert = sg.x;
+    tok0 = sg.y;
+    tile_rows = sg.z;
+    if (bias != nullptr) bias += (size_t)expert * N;
+  }
+  const int wrow0 = expert * K, qrow0 = expert * (K / gsz);   // the expert's weight / scale rows
   constexpr int kTcBBufs = L::BBUFS;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -142,7 +164,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(const __grid_
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = ((int)blockIdx.x - op->tile_begin) * kTcBN;
-  const int tok0 = blockIdx.y * (kTcMB * kTcBM);
   const int nk = K / kTcBK;
 
   if (tid == 0) {
@@ -180,9 +201,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(const __grid_
       for (int kb = 0; kb < pre; ++kb) {
         const uint32_t st = base + kb * L::STAGE, bar = tma_full0 + 8 * kb;
         mbar_arrive_expect_tx(bar, L::TX_BYTES);
-        tma_load_2d(st + L::WQ_OFF, tmW, bar, n0 / 8, kb * kTcBK);
-        tma_load_2d(st + L::S_OFF, tmS, bar, n0, (kb * kTcBK) / gsz);
-        tma_load_2d(st + L::Z_OFF, tmZ, bar, n0 / 8, (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::WQ_OFF, tmW, bar, n0 / 8, wrow0 + kb * kTcBK);
+        tma_load_2d(st + L::S_OFF, tmS, bar, n0, qrow0 + (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::Z_OFF, tmZ, bar, n0 / 8, qrow0 + (kb * kTcBK) / gsz);
       }
       pdl_wait_primary();               // X_r is written by the rotation kernel
       for (int kb = 0; kb < pre; ++kb)
@@ -192,9 +213,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(const __grid_
         if (!tc_wait(tma_empty0 + 8 * s, ((kb / kTcStages) - 1) & 1, abort)) break;
         const uint32_t st = base + s * L::STAGE, bar = tma_full0 + 8 * s;
         mbar_arrive_expect_tx(bar, L::TX_BYTES);
-        tma_load_2d(st + L::WQ_OFF, tmW, bar, n0 / 8, kb * kTcBK);
-        tma_load_2d(st + L::S_OFF, tmS, bar, n0, (kb * kTcBK) / gsz);
-        tma_load_2d(st + L::Z_OFF, tmZ, bar, n0 / 8, (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::WQ_OFF, tmW, bar, n0 / 8, wrow0 + kb * kTcBK);
+        tma_load_2d(st + L::S_OFF, tmS, bar, n0, qrow0 + (kb * kTcBK) / gsz);
+        tma_load_2d(st + L::Z_OFF, tmZ, bar, n0 / 8, qrow0 + (kb * kTcBK) / gsz);
         tma_load_2d(st + L::A_OFF, tmA, bar, kb * kTcBK, tok0);
       }
     }
@@ -360,7 +381,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_gemm_kernel(const __grid_
     }
     fence_proxy_async_smem();           // the staged tile is read by the TMA (async proxy)
     named_bar_sync(1, 32 * kTcDequantWarps);
-    if (warp == 2 && lane == 0 && !*abort) {
+    if constexpr (SEG) {
+      // the tile's rows go to their slots: 16-byte chunks of the staged boxes,
+      // row by row, only the tile's own rows and columns below N
+      if (!*abort) {
+        TA* const Yp = static_cast<TA*>(op->yptr);
+        const int et = tid - 64;                  // epilogue thread 0 .. 511
+        for (int idx = et; idx < tile_rows * (kTcBN / 8); idx += 32 * kTcDequantWarps) {
+          const int r = idx / (kTcBN / 8), ch = idx % (kTcBN / 8);
+          const int n = n0 + 8 * ch;
+          if (n >= N) continue;
+          const uint32_t src = base + (uint32_t)(ch >> 3) * L::O_BOX + (uint32_t)r * 128u +
+                               ((uint32_t)((ch & 7) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(Yp + (size_t)op->perm[tok0 + r] * N + n) = lds128(src);
+        }
+      }
+    } else if (warp == 2 && lane == 0 && !*abort) {
 #pragma unroll
       for (int b = 0; b < kTcBN / 64; ++b)
         if (n0 + 64 * b < N) tma_store_2d(tmY, base + (uint32_t)b * L::O_BOX, n0 + 64 * b, tok0);

@@ -276,3 +276,35 @@ def test_dtype_entry_points_check_the_type_first(L):
                                  None) == L.PARO_ERR_UNSUPPORTED
     assert L.paro_w4_linear_noalloc_dt(A16, A16, 4, 256, 40, A16, A16, A16, None, None, None, None, 128, 0, bf,
                                        None) == L.PARO_ERR_UNSUPPORTED
+
+
+def test_moe_shape_checks_and_queries(L):
+    """Stacked experts: size and launch queries, and argument checks that end
+    before any launch."""
+    assert L.paro_w4_moe_launches(1, 4096, 4096, 64, 8, 128, 8, 1) == 4
+    assert L.paro_w4_moe_launches(4096, 4096, 4096, 64, 8, 128, 0, 0) == 3
+    assert L.paro_w4_moe_launches(1, 4096, 4096, 2048, 8, 128, 8, 1) == 0      # more experts than supported
+    assert L.paro_w4_moe_launches(0, 4096, 4096, 8, 2, 128, 8, 1) == 0
+    need = L.paro_w4_moe_workspace_size(16, 4096, 1024, 8, 2, 128)
+    assert need >= 16 * 4096 * 2 + 32 * 4096 * 2 + 32 * (4 + 16 + 16)
+    assert L.paro_w4_moe_workspace_size(16, 4096, 1024, 0, 2, 128) == 0
+    assert L.paro_w4_moe_workspace_size(16, 4096, 1024, 8, 65, 128) == 0
+    assert L.paro_w4_moe_workspace_size(16, 4000, 1024, 8, 2, 128) == 0
+    moe = lambda x=A16, y=A16, T=16, K=4096, N=1024, E=8, k=2, idx=A16, qw=A16, qz=A16, sc=A16, cs=None, \
+        krot=0, G=128, dt=0, ws=P(0x100000), n=need: L.paro_w4_moe_linear(
+            x, y, T, K, N, E, k, idx, qw, qz, sc, None, cs, None, None, G, krot, dt, ws, n, None)  # noqa: E731
+    assert moe(dt=2) == L.PARO_ERR_INVALID_ARG
+    assert moe(T=-1) == L.PARO_ERR_INVALID_ARG
+    assert moe(E=0) == L.PARO_ERR_INVALID_ARG
+    assert moe(E=1025) == L.PARO_ERR_UNSUPPORTED
+    assert moe(k=65) == L.PARO_ERR_UNSUPPORTED
+    assert moe(G=8) == L.PARO_ERR_UNSUPPORTED
+    assert moe(N=40) == L.PARO_ERR_UNSUPPORTED
+    assert moe(idx=None) == L.PARO_ERR_INVALID_ARG
+    assert moe(krot=8) == L.PARO_ERR_INVALID_ARG                 # pairs / theta missing
+    assert moe(x=MIS) == L.PARO_ERR_ALIGNMENT
+    assert moe(idx=P(0x10002)) == L.PARO_ERR_ALIGNMENT
+    assert moe(ws=P(0x100010)) == L.PARO_ERR_ALIGNMENT
+    assert moe(n=need - 1) == L.PARO_ERR_WORKSPACE
+    assert moe(ws=None) == L.PARO_ERR_INVALID_ARG
+    assert moe(T=0) == L.PARO_OK                                 # no tokens: no work
