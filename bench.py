@@ -61,6 +61,10 @@ WORKLOADS = {
     "quantize_gate_proj": dict(cfg=2, layers=[0], Ms=[], kind="quantize"),
     # both halves of the decoder-layer set in one line
     "layer": dict(cfg=4, kind="pair", halves=["layer_decode", "layer_prefill"]),
+    # stacked experts sharing one rotation: a Mixtral-8x7B-shaped expert gate
+    # projection (8 experts of 4096 -> 14336, top-2 routing), decode and prefill
+    "moe_decode": dict(kind="moe", E=8, topk=2, K=4096, N=14336, T=1),
+    "moe_prefill": dict(kind="moe", E=8, topk=2, K=4096, N=14336, T=4096),
 }
 REPLAYS = 7          # timed replays of the K-step graph; the median is reported
 
@@ -244,6 +248,10 @@ def spread(ms_list, steps):
 def workload_config(workload, world):
     """The workload description shared by both arms' JSON lines."""
     wl = WORKLOADS[workload]
+    if wl["kind"] == "moe":
+        return {"workload": workload, "experts": wl["E"], "topk": wl["topk"], "K": wl["K"], "N": wl["N"],
+                "tokens": wl["T"], "routing": "seeded uniform top-k without repeats, a new draw every call",
+                "group_size": GROUP, "krot": KROT, "accumulate": "f32", "parallelism": f"replicas x{world}"}
     if wl["kind"] == "pair":
         dec, pre = (workload_config(h, world) for h in wl["halves"])
         return {"workload": workload, "layers": dec["layers"], "calls": dec["calls"],
@@ -651,6 +659,160 @@ def run_quantize(args, rank, world, local_rank):
     }
 
 
+def moe_setup(wl, seed=0):
+    """The workload's experts (codes, zero points, scales per expert; no bias)
+    and the shared rotation, drawn once per process."""
+    key = ("moe", wl["E"], wl["K"], wl["N"], seed)
+    if key not in _LAYERS:
+        lays = [synth.make_layer(f"expert{e}", wl["K"], wl["N"], seed=1000 + 17 * e, krot=KROT,
+                                 zero_point=None) for e in range(wl["E"])]
+        _LAYERS[key] = lays
+    return _LAYERS[key]
+
+
+def moe_routing(wl, calls, seed=0):
+    rng = np.random.default_rng(seed)
+    return [np.stack([rng.choice(wl["E"], wl["topk"], replace=False) for _ in range(wl["T"])]).astype(np.int32)
+            for _ in range(calls)]
+
+
+def moe_call_bytes(wl, idx):
+    """Bytes one call must move: x, the distinct selected experts' weights,
+    scales and zero words, and y."""
+    K, N = wl["K"], wl["N"]
+    experts = len(np.unique(idx))
+    return (wl["T"] * K * 2 + experts * (K * N // 2 + (K // GROUP) * N * 2 + (K // GROUP) * N // 2)
+            + idx.size * N * 2)
+
+
+def run_moe(args, rank, world, local_rank):
+    """paro_w4_moe_linear on the workload's experts: one call per step with a
+    fresh routing, experts resident in HBM (8 experts > L2 together)."""
+    import torch
+    import rotation_w4_weight_b200 as pb
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    lays = moe_setup(wl)
+    rot = lays[0]
+
+    def T(a):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    qw, qz = zip(*[pb.pack_awq(T(l.codes), T(l.zero_codes), GROUP) for l in lays])
+    qweight, qzeros = torch.stack(qw).contiguous(), torch.stack(qz).contiguous()
+    del qw, qz
+    scales = T(np.stack([l.scales for l in lays]))
+    cs, pairs, theta = T(rot.channel_scales), T(rot.pairs), T(rot.theta)
+    routes = moe_routing(wl, 64)
+    idx_d = [T(r) for r in routes]
+    xs = [T(synth.make_activations(rot, wl["T"], seed=i)) for i in range(4)]
+    out = torch.empty((wl["T"], wl["topk"], wl["N"]), dtype=torch.float16, device=dev)
+    ws = torch.empty(pb.paro_w4_moe_workspace_size(wl["T"], wl["K"], wl["N"], wl["E"], wl["topk"], GROUP),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    decode = wl["T"] <= 16
+
+    def one_step(i):
+        pb.w4_moe_linear(xs[i % len(xs)], idx_d[i % len(idx_d)], qweight, qzeros, scales, None, cs, pairs, theta,
+                         GROUP, KROT, workspace=ws, out=out, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            one_step(i)
+    torch.cuda.synchronize(dev)
+    assert pb.device_status() == pb.PARO_OK
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(args.steps):
+            one_step(args.warmup + i)
+
+    def replay():
+        with torch.cuda.stream(stream):
+            g.replay()
+
+    replay()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    t_end = time.time() + 0.6
+    while time.time() < t_end:
+        replay()
+        torch.cuda.synchronize(dev)
+    step_ms = timed_replays(replay, stream, world, dev)
+    ms = statistics.median(step_ms)
+    clocks = sampler.stop()
+    assert pb.device_status() == pb.PARO_OK
+    del g
+    bytes_steps = sum(moe_call_bytes(wl, routes[(args.warmup + i) % len(routes)]) for i in range(args.steps))
+    flops_per = 2 * wl["T"] * wl["topk"] * wl["K"] * wl["N"]
+    peaks = load_peaks()
+    step_s = ms * 1e-3 / args.steps
+    if decode:
+        achieved = bytes_steps / args.steps / step_s / 1e9
+        value, unit = job_throughput(world, args.steps, bytes_steps / args.steps, ms) / 1e9, "GB/s"
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm"], 4), "traffic": None,
+                "kernel": "whole call (rotation, routing, gather, expert GEMV segments)",
+                "avg_launch_us": round(step_s * 1e6, 3), "bytes_per_launch": int(bytes_steps / args.steps),
+                "peak_source": peaks["src"]}
+    else:
+        achieved = flops_per / step_s / 1e12
+        value, unit = job_throughput(world, args.steps, flops_per, ms) / 1e12, "TFLOP/s"
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_sus"], 4), "traffic": None,
+                "kernel": "whole call (rotation, routing, gather, expert GEMM tiles)",
+                "avg_launch_us": round(step_s * 1e6, 3), "flops_per_launch": flops_per,
+                "peak_source": "measured bf16 sustained (fp16 runs at the bf16 rate)"}
+    return {
+        "metric": metric_name(args.workload), "value": round(value, 2), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": dict(workload_config(args.workload, world),
+                       l2=f"{wl['E']} experts resident ({wl['E'] * wl['K'] * wl['N'] // 2 / 2**20:.0f} MiB > L2)",
+                       timing=f"median of {REPLAYS} replays of a CUDA graph of the K steps, CUDA events"),
+        "timing": spread(step_ms, args.steps), "roofline": roof,
+        "gpu_launches": pb.w4_moe_launches(wl["T"], wl["K"], wl["N"], wl["E"], wl["topk"], GROUP, KROT) * args.steps,
+        "clocks": clocks,
+    }
+
+
+def moe_oracle_sample(workload, budget_s, max_steps=None):
+    """The float64 oracle's stacked-expert layer on column samples (64 columns
+    of every expert, full rotation per call), until `budget_s` seconds."""
+    import oracle
+    wl = WORKLOADS[workload]
+    lays = moe_setup(wl)
+    rot = lays[0]
+    routes = moe_routing(wl, 4)
+    rng = np.random.default_rng(0)
+    done = t_total = 0.0
+    n = 0
+    ncols = 64
+    while True:
+        cols = np.sort(rng.choice(wl["N"], ncols, replace=False))
+        idx = routes[n % len(routes)]
+        x = synth.make_activations(rot, wl["T"], seed=n)
+        codes = np.stack([l.codes[cols] for l in lays])
+        zeros = np.stack([l.zero_codes[cols] for l in lays])
+        scales = np.stack([l.scales[:, cols] for l in lays])
+        t0 = time.perf_counter()
+        oracle.moe_linear_from_codes(x, idx, codes, zeros, scales, None, rot.channel_scales, rot.pairs,
+                                     rot.theta, GROUP, KROT)
+        t_total += time.perf_counter() - t0
+        frac = ncols / wl["N"]
+        done += (moe_call_bytes(wl, idx) * frac if wl["T"] <= 16 else
+                 2 * wl["T"] * wl["topk"] * wl["K"] * wl["N"] * frac)
+        n += 1
+        if t_total >= budget_s or (max_steps and n >= max_steps):
+            unit = 1e9 if wl["T"] <= 16 else 1e12
+            desc = (f"float64 oracle on {n} calls of {workload} restricted to {ncols} sampled output columns "
+                    f"of every expert (full rotation per call)")
+            return done / t_total / unit, desc, t_total
+
+
 def quantize_oracle_sample(workload, budget_s, max_steps=None):
     """The float64 oracle's weight quantiser on row samples of the workload's
     weight (256 rows per sample), until `budget_s` seconds or max_steps samples."""
@@ -685,6 +847,8 @@ def oracle_sample(workload, budget_s, max_steps=None):
     wl = WORKLOADS[workload]
     if wl["kind"] == "quantize":
         return quantize_oracle_sample(workload, budget_s, max_steps)
+    if wl["kind"] == "moe":
+        return moe_oracle_sample(workload, budget_s, max_steps)
     layers = [cfg_layers(wl["cfg"])[i] for i in wl["layers"]]
     decode = wl["kind"] == "decode"
     rng = np.random.default_rng(0)
@@ -718,6 +882,10 @@ def metric_name(workload):
                 "(value) and prefill TFLOP/s at M=4096 (prefill.value), % of roofline")
     if WORKLOADS[workload]["kind"] == "quantize":
         return f"weight quantiser HBM throughput ({workload})"
+    if WORKLOADS[workload]["kind"] == "moe":
+        return ("stacked-expert rotated W4 linear " +
+                ("decode HBM throughput" if WORKLOADS[workload]["T"] <= 16 else "prefill tensor throughput") +
+                f" ({workload})")
     decode = WORKLOADS[workload]["kind"] == "decode"
     return ("rotated W4 linear decode HBM throughput" if decode else
             "rotated W4 linear prefill tensor throughput") + f" ({workload})"
@@ -726,7 +894,7 @@ def metric_name(workload):
 def reference_half(workload, steps, warmup, world):
     """One workload of the reference arm: the oracle on bounded samples."""
     wl = WORKLOADS[workload]
-    decode = wl["kind"] in ("decode", "quantize")
+    decode = wl["kind"] in ("decode", "quantize") or (wl["kind"] == "moe" and wl["T"] <= 16)
     cores = len(os.sched_getaffinity(0))
     per_step_budget = max(0.2, min(2.0, 150.0 / max(1, steps + warmup)))
     oracle_sample(workload, per_step_budget * warmup, max_steps=warmup)
@@ -797,6 +965,8 @@ def main():
     wl = WORKLOADS[args.workload]
     if wl["kind"] == "quantize":
         out = run_quantize(args, rank, world, local_rank)
+    elif wl["kind"] == "moe":
+        out = run_moe(args, rank, world, local_rank)
     elif wl["kind"] == "pair":
         out = run_pair(args, rank, world, local_rank)
     else:
