@@ -1199,19 +1199,23 @@ constexpr int kMoeDecodeMaxT = kMaxDecodeM;    // tokens up to which the segment
 
 // Workspace of a stacked-expert call: X_r [T, K] (when rotating), the sorted
 // rows Xg [S, K], the routing head, perm [S], decode segments [S] and prefill
-// tiles [S] (each segment or tile has at least one row), 256-byte aligned.
+// tiles [S] (each segment or tile has at least one row), and above 64 tokens
+// the R' parts [2][K][128] of the tensor-core rotation; 256-byte aligned.
 struct MoePlan {
-  size_t off_xr = 0, off_xg = 0, off_head = 0, off_perm = 0, off_gv = 0, off_tc = 0, total = 0;
+  size_t off_xr = 0, off_xg = 0, off_head = 0, off_perm = 0, off_gv = 0, off_tc = 0, off_rt = 0, total = 0;
+  bool rot_tc = false;
 };
 MoePlan moe_plan(int64_t T, int64_t K, int64_t S) {
   MoePlan p;
   p.off_xr = 0;
+  p.rot_tc = T >= kRotTcMinM;
   p.off_xg = round_up((size_t)T * K * 2, 256);
   p.off_head = p.off_xg + round_up((size_t)S * K * 2, 256);
   p.off_perm = p.off_head + 256;
   p.off_gv = p.off_perm + round_up((size_t)S * 4, 256);
   p.off_tc = p.off_gv + round_up((size_t)S * 16, 256);
-  p.total = p.off_tc + round_up((size_t)S * 16, 256);
+  p.off_rt = p.off_tc + round_up((size_t)S * 16, 256);
+  p.total = p.off_rt + (p.rot_tc ? (size_t)K * kGroup * 2 * 2 : 0);
   return p;
 }
 
@@ -1249,11 +1253,17 @@ int moe_impl(const void* x, void* y, int64_t T, int64_t K, int64_t N, int E, int
   const int G = group_of(group_size, K);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   const TA* xr = static_cast<const TA*>(x);
-  // the rotation is shared by every expert: once, on the T tokens
+  // the rotation is shared by every expert: once, on the T tokens (above 64
+  // tokens as X R' on the tensor cores, as paro_w4_linear does)
   if (krot > 0 || channel_scales != nullptr) {
     TA* out = reinterpret_cast<TA*>(ws + mp.off_xr);
-    if (int st = launch_rotate<TA>(static_cast<const TA*>(x), out, T, K, channel_scales, pairs, theta, krot, G, s))
+    if (mp.rot_tc) {
+      const RotTcMember one{channel_scales, pairs, theta, krot, out, ws + mp.off_rt, false};
+      if (int st = launch_rotate_tc<TA>(static_cast<const TA*>(x), &one, 1, T, K, G, s)) return st;
+    } else if (int st = launch_rotate<TA>(static_cast<const TA*>(x), out, T, K, channel_scales, pairs, theta, krot,
+                                          G, s)) {
       return st;
+    }
     xr = out;
   }
   MoeHead* head = reinterpret_cast<MoeHead*>(ws + mp.off_head);
@@ -1310,7 +1320,8 @@ int paro_w4_moe_linear(const void* x, void* y, int64_t T, int64_t K, int64_t N, 
 int paro_w4_moe_launches(int64_t T, int64_t K, int64_t N, int E, int topk, int group_size, int krot,
                          int rotate) {
   if (check_moe_shape(T, K, N, E, topk, group_size) != PARO_OK || T == 0 || krot < 0 || krot > kMaxKrot) return 0;
-  return (rotate ? 1 : 0) + 3;    // rotation, route, gather, expert GEMV or GEMM
+  // rotation (two launches above 64 tokens: R' build and X R'), route, gather, expert GEMV or GEMM
+  return (rotate ? (T >= kRotTcMinM ? 2 : 1) : 0) + 3;
 }
 
 }  // extern "C"

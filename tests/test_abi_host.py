@@ -283,6 +283,8 @@ def test_moe_shape_checks_and_queries(L):
     before any launch."""
     assert L.paro_w4_moe_launches(1, 4096, 4096, 64, 8, 128, 8, 1) == 4
     assert L.paro_w4_moe_launches(4096, 4096, 4096, 64, 8, 128, 0, 0) == 3
+    assert L.paro_w4_moe_launches(4096, 4096, 4096, 64, 8, 128, 8, 1) == 5   # R' build + X R' above 64 tokens
+    assert L.paro_w4_moe_launches(64, 4096, 4096, 64, 8, 128, 8, 1) == 4
     assert L.paro_w4_moe_launches(1, 4096, 4096, 2048, 8, 128, 8, 1) == 0      # more experts than supported
     assert L.paro_w4_moe_launches(0, 4096, 4096, 8, 2, 128, 8, 1) == 0
     need = L.paro_w4_moe_workspace_size(16, 4096, 1024, 8, 2, 128)
