@@ -558,9 +558,11 @@ def run_quantize(args, rank, world, local_rank):
              torch.empty((lay.K // GROUP, lay.N // 8), dtype=torch.int32, device=dev)) for _ in range(2)]
     per_call = quantize_bytes(lay.K, lay.N)
     stream = torch.cuda.Stream(device=dev)
+    qws = torch.empty(pb.paro_quantize_w4_workspace_size(lay.K), dtype=torch.uint8, device=dev)
 
     def one_step(i):
-        pb.quantize_w4(Ws[i % reps], cs, pairs, theta, qsd, GROUP, KROT, out=outs[i % 2], stream=stream)
+        pb.quantize_w4(Ws[i % reps], cs, pairs, theta, qsd, GROUP, KROT, out=outs[i % 2], stream=stream,
+                       method="tensor", workspace=qws)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -606,12 +608,13 @@ def run_quantize(args, rank, world, local_rank):
     assert pb.device_status() == pb.PARO_OK
     del g
 
-    # one kernel per call: the step time is the kernel's launch time
+    # two kernels per call (the R'' build, ~9 us, and the quantising product):
+    # the roofline takes the whole call, so it understates the product kernel
     peaks = load_peaks()
     achieved = per_call * args.steps / (ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm"], 4), "traffic": traffic_for("quantize_gate_proj"),
-            "kernel": "rotate_tmem_kernel<true, true> (weight quantiser)",
+            "kernel": "rotate_tc_kernel<__half, true> (weight quantiser on the tensor cores) + R'' build, per call",
             "avg_launch_us": round(ms * 1e3 / args.steps, 3), "bytes_per_launch": per_call,
             "peak_source": peaks["src"]}
 
@@ -623,7 +626,8 @@ def run_quantize(args, rank, world, local_rank):
 
     def e2e_step():
         Ws[0].copy_(hW, non_blocking=True)
-        pb.quantize_w4(Ws[0], cs, pairs, theta, qsd, GROUP, KROT, out=outs[0], stream=stream)
+        pb.quantize_w4(Ws[0], cs, pairs, theta, qsd, GROUP, KROT, out=outs[0], stream=stream, method="tensor",
+                       workspace=qws)
         hq[0].copy_(outs[0][0], non_blocking=True)
         hq[1].copy_(outs[0][1], non_blocking=True)
 
@@ -652,8 +656,8 @@ def run_quantize(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int(hW.numel() * 2),
                 "d2h_bytes_per_step": int((hq[0].numel() + hq[1].numel()) * 4),
                 "ms_per_step": round(e2e_ms, 4),
-                "how": "pinned host W -> device, paro_quantize_w4, packed words -> pinned host; no graph"},
-        "gpu_launches": args.steps,
+                "how": "pinned host W -> device, paro_quantize_w4_tc, packed words -> pinned host; no graph"},
+        "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "bytes_per_step": per_call,
     }

@@ -174,6 +174,28 @@ int paro_quantize_w4_dt(const void* w, const float* channel_scales, const int16_
                         const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
                         int64_t N, int64_t K, int group_size, int krot, int dtype, paro_stream_t stream);
 
+/*
+ * paro_quantize_w4_tc — paro_quantize_w4 on the tensor cores (fp16 weights).
+ * The weight-side stages with D = 1 / channel_scales are one 128 x 128 map per
+ * group, R'' = diag(D) G_0 ... G_{krot-1} (the product form of the page's
+ * "Pairwise Givens rotations"); the call builds it into the workspace (two
+ * fp16 parts, about 2^-22 relative), computes W_r = W R'' with tensor-core
+ * MMAs into fp32 accumulators, and quantises and packs straight from them
+ * (same quantiser, same words as paro_quantize_w4).
+ *   Arguments as for paro_quantize_w4, plus N % 32 == 0 and a workspace of at
+ *   least paro_quantize_w4_workspace_size(K) = K * 128 * 4 bytes, 256-byte
+ *   aligned (contents need no initialisation).
+ * W_r differs from paro_quantize_w4's fp32 stage-by-stage W_r by summation
+ * order only (within a few units of 2^-22 of the group norm), so a code can
+ * differ between the two only where W_r / s lies that close to a rounding
+ * boundary.  Its last kernel does not release its dependents early.
+ */
+size_t paro_quantize_w4_workspace_size(int64_t K);
+int paro_quantize_w4_tc(const void* w, const float* channel_scales, const int16_t* pairs,
+                        const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
+                        int64_t N, int64_t K, int group_size, int krot, void* workspace,
+                        size_t workspace_bytes, paro_stream_t stream);
+
 /* paro_unpack_awq — exact inverse of paro_pack_awq (same shapes, same rules). */
 int paro_unpack_awq(const int32_t* qweight, const int32_t* qzeros, uint8_t* codes,
                     uint8_t* zero_codes, int64_t N, int64_t K, int group_size,

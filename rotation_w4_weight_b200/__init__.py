@@ -9,7 +9,7 @@ streams) into that ABI.  Functions mirror the C entry points:
     unpack_awq        -> paro_unpack_awq
     w4_linear         -> paro_w4_linear / paro_w4_linear_dt (+ paro_w4_linear_workspace_size)
     w4_linear_group   -> paro_w4_linear_group / paro_w4_linear_group_dt (+ ..._workspace_size)
-    quantize_w4       -> paro_quantize_w4 / paro_quantize_w4_dt
+    quantize_w4       -> paro_quantize_w4_tc (+ its workspace size), or paro_quantize_w4 / paro_quantize_w4_dt
     validate_pairs    -> paro_validate_pairs (host helper)
     device_status     -> paro_device_status
     rotation_matrix   -> paro_rotation_matrix_prepare (+ paro_rotation_matrix_size)
@@ -36,7 +36,8 @@ from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # n
                    paro_w4_linear_group_workspace_size, PARO_DTYPE_BF16, paro_rotate_dt, paro_quantize_w4_dt,
                    paro_w4_linear_dt, paro_w4_linear_group_dt, paro_rotation_matrix_size,
                    paro_rotation_matrix_prepare, PARO_DTYPE_F16, paro_w4_moe_workspace_size,
-                   paro_w4_moe_linear, paro_w4_moe_launches)
+                   paro_w4_moe_linear, paro_w4_moe_launches, paro_quantize_w4_workspace_size,
+                   paro_quantize_w4_tc)
 
 __all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
            "w4_linear_group", "w4_linear_group_launches", "quantize_w4", "validate_pairs", "device_status",
@@ -117,9 +118,15 @@ def pack_awq(codes: torch.Tensor, zero_codes: Optional[torch.Tensor], group_size
 
 def quantize_w4(w: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: Optional[torch.Tensor],
                 theta: Optional[torch.Tensor], scales: torch.Tensor, group_size: int = 128,
-                krot: Optional[int] = None, out=None, stream=None):
+                krot: Optional[int] = None, out=None, stream=None, method: str = "auto",
+                workspace: Optional[torch.Tensor] = None):
     """Float weights w fp16/bf16 [N, K] (out x in) -> (qweight int32 [K, N/8], qzeros int32 [K/G, N/8]):
-    W_r = W D R, four-bit symmetric codes with the quantiser scales [K/G, N] (w's type), AWQ-packed."""
+    W_r = W D R, four-bit symmetric codes with the quantiser scales [K/G, N] (w's type), AWQ-packed.
+
+    ``method``: "tensor" (paro_quantize_w4_tc: the stages as one matrix per
+    group on the tensor cores; fp16 weights, N % 32 == 0), "pairs"
+    (paro_quantize_w4[_dt]: stage by stage), or "auto" (tensor where it
+    applies)."""
     dt = _act(w, "w")
     _need(w, dt, "w")
     _need(channel_scales, torch.float32, "channel_scales", True)
@@ -136,7 +143,16 @@ def quantize_w4(w: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: 
     qweight, qzeros = out
     args = (_ptr(w), _ptr(channel_scales), _ptr(pairs), _ptr(theta), _ptr(scales), _ptr(qweight), _ptr(qzeros),
             N, K, group_size, krot)
-    if dt == torch.float16:
+    if method not in ("auto", "tensor", "pairs"):
+        raise ValueError(f"method must be auto, tensor or pairs, got {method}")
+    tensor = method == "tensor" or (method == "auto" and dt == torch.float16 and N % 32 == 0)
+    if tensor:
+        need = int(paro_quantize_w4_workspace_size(K))
+        if workspace is None:
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=w.device)
+        check(paro_quantize_w4_tc(*args, _ptr(workspace), workspace.numel(), _stream(stream)),
+              "paro_quantize_w4_tc")
+    elif dt == torch.float16:
         check(paro_quantize_w4(*args, _stream(stream)), "paro_quantize_w4")
     else:
         check(paro_quantize_w4_dt(*args, PARO_DTYPE_BF16, _stream(stream)), "paro_quantize_w4_dt")

@@ -364,7 +364,43 @@ int launch_rotate_tc(const TA* x, const RotTcMember* mem, int count, int64_t M, 
   const int64_t jobs = (int64_t)count * groups * tiles;
   const int64_t ctas = jobs < di.sms ? jobs : di.sms;
   return launch(rotate_tc_kernel<TA>, dim3((unsigned)ctas), dim3(kRcThreads), RcLayout::SMEM, stream, true, tmX,
-                rc, count, (int)K, (int)groups, (int)tiles, (long long)jobs);
+                rc, count, (int)K, (int)groups, (int)tiles, (long long)jobs, RcQuant{});
+}
+
+// Weight quantiser on the tensor cores: R'' = diag(1 / cs) G_0 ... G_{krot-1}
+// per group (the build kernel with inverted scales) into the workspace, then
+// W_r = W R'' with the quantising epilogue (codes and AWQ words straight from
+// the fp32 accumulators).  fp16 weights only: R'' in two fp16 parts keeps
+// W_r to about 2^-22 relative, within the fp32 rounding the codes are judged
+// by; bf16 parts would keep only 2^-16.
+int launch_quantize_tc(const __half* w, const float* cs, const int16_t* pairs, const float* theta,
+                       const __half* scales, int32_t* qweight, int32_t* qzeros, int64_t N, int64_t K, int gsz,
+                       int krot, void* rt, cudaStream_t s) {
+  const DeviceInfo& di = device_info();
+  if (di.sms == 0) return PARO_ERR_CUDA;
+  const int64_t groups = K / kGroup, tiles = (N + 127) / 128;
+  RbBatch rb;
+  std::memset(&rb, 0, sizeof(rb));
+  rb.op[0] = RbOperand{cs, pairs, theta, rt, krot};
+  if (!allow_smem(rmat_build_kernel<__half, true, true>, rb_smem_bytes(kMaxKrot))) return PARO_ERR_CUDA;
+  if (int st = launch(rmat_build_kernel<__half, true, true>, dim3((unsigned)groups, (unsigned)(kGroup / kRbRows), 1),
+                      dim3(kRbThreads), rb_smem_bytes(krot), s, true, rb, (int)K, gsz))
+    return st;
+  RcBatch rc;
+  std::memset(&rc, 0, sizeof(rc));
+  CUtensorMap tmX;
+  if (!encode_2d(&rc.t[0].r, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rt, 2 * K, kGroup, 128, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&rc.t[0].y, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 64, 4,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w, N, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return PARO_ERR_CUDA;
+  auto k = rotate_tc_kernel<__half, true>;
+  if (!allow_smem(k, RcLayout::SMEM)) return PARO_ERR_CUDA;
+  const int64_t jobs = groups * tiles;
+  const int64_t ctas = jobs < di.sms ? jobs : di.sms;
+  return launch(k, dim3((unsigned)ctas), dim3(rc_threads<true>()), RcLayout::SMEM, s, true, tmX, rc, 1, (int)K,
+                (int)groups, (int)tiles, (long long)jobs, RcQuant{scales, qzeros, (int)N, gsz});
 }
 
 // ---------------------------------------------------------------- linear plan
@@ -769,6 +805,35 @@ int paro_quantize_w4_dt(const void* w, const float* channel_scales, const int16_
                                           group_size, krot, s);
     default: return PARO_ERR_INVALID_ARG;
   }
+}
+
+size_t paro_quantize_w4_workspace_size(int64_t K) {
+  if (K <= 0 || K % kGroup != 0 || K >= (int64_t(1) << 24)) return 0;
+  return (size_t)K * kGroup * 2 * 2;
+}
+
+int paro_quantize_w4_tc(const void* w, const float* channel_scales, const int16_t* pairs, const float* theta,
+                        const void* scales, int32_t* qweight, int32_t* qzeros, int64_t N, int64_t K,
+                        int group_size, int krot, void* workspace, size_t workspace_bytes, paro_stream_t stream) {
+  if (N < 0 || K <= 0 || krot < 0 || N % 8 != 0) return PARO_ERR_INVALID_ARG;
+  int G = 0;
+  if (int st = normalize_group(group_size, K, &G)) return st;
+  if (!supported_group(G, K) || krot > kMaxKrot || N % 32 != 0 || K >= (int64_t(1) << 24))
+    return PARO_ERR_UNSUPPORTED;
+  if (N == 0) return PARO_OK;   // nothing to touch: NULL data pointers are fine
+  if (w == nullptr || scales == nullptr || qweight == nullptr || qzeros == nullptr || workspace == nullptr)
+    return PARO_ERR_INVALID_ARG;
+  if (krot > 0 && (pairs == nullptr || theta == nullptr)) return PARO_ERR_INVALID_ARG;
+  if (N * K >= (int64_t(1) << 31)) return PARO_ERR_UNSUPPORTED;
+  if (workspace_bytes < paro_quantize_w4_workspace_size(K)) return PARO_ERR_WORKSPACE;
+  if (!aligned(w, 16) || !aligned(scales, 2) || !aligned(qweight, 16) || !aligned(qzeros, 4) ||
+      !aligned(workspace, 256))
+    return PARO_ERR_ALIGNMENT;
+  if (channel_scales != nullptr && !aligned(channel_scales, 4)) return PARO_ERR_ALIGNMENT;
+  if (krot > 0 && (!aligned(pairs, 4) || !aligned(theta, 4))) return PARO_ERR_ALIGNMENT;
+  return launch_quantize_tc(static_cast<const __half*>(w), channel_scales, pairs, theta,
+                            static_cast<const __half*>(scales), qweight, qzeros, N, K, G, krot, workspace,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 int paro_pack_awq(const uint8_t* codes, const uint8_t* zero_codes, int32_t* qweight,

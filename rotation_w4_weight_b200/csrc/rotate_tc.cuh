@@ -66,7 +66,10 @@ struct RbBatch {
 // for the largest krot of the batch.
 // RELEASE: let the kernel that follows launch early (false when the parts are
 // prepared layer constants, which later kernels read before they wait).
-template <typename TA, bool RELEASE = true>
+// INV: the basis rows are scaled by 1 / cs (the weight side, W_r = W D R with
+// D = 1 / channel_scales), the reciprocal taken in fp32 as the weight
+// quantiser takes it.
+template <typename TA, bool RELEASE = true, bool INV = false>
 __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_constant__ RbBatch batch, int K,
                                                                 int gsz) {
   // The rotation that follows waits for this kernel's completion; let it
@@ -91,7 +94,10 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_con
   for (int idx = tid; idx < kRbRows * kGroup; idx += kRbThreads) {
     const int r = idx >> 7, c = idx & (kGroup - 1);
     float val = 0.0f;
-    if (c == r0 + r) val = cs != nullptr ? cs[(size_t)grp * kGroup + c] : 1.0f;
+    if (c == r0 + r) {
+      const float sc = cs != nullptr ? cs[(size_t)grp * kGroup + c] : 1.0f;
+      val = INV ? 1.0f / sc : sc;
+    }
     sts_f32(vbase + (uint32_t)(r * kRbPitch + c) * 4u, val);
   }
   __syncthreads();
@@ -169,6 +175,12 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_con
 constexpr int kRcStages = 3;
 constexpr int kRcEpiWarps = 4;
 constexpr int kRcThreads = 32 * (2 + kRcEpiWarps);
+// The quantising variant has twice the epilogue warps (two per TMEM lane
+// quadrant, 64 columns each): its epilogue does more work per value.
+template <bool QUANT>
+__host__ __device__ constexpr int rc_epi_warps() { return QUANT ? 2 * kRcEpiWarps : kRcEpiWarps; }
+template <bool QUANT>
+__host__ __device__ constexpr int rc_threads() { return 32 * (2 + rc_epi_warps<QUANT>()); }
 constexpr int kRcCols = 256;
 
 struct RcLayout {
@@ -208,6 +220,40 @@ __device__ __forceinline__ void rc_stage32(uint32_t tile, int r, int cb, const u
   }
 }
 
+// The weight quantiser's outputs (QUANT variant): x is W [N, K] (weight rows),
+// the product is W_r = W D R, and each tile is quantised with the quantiser
+// scales [K/G, N] (bounded to [1e-5, 1e5]) into four-bit codes -8..7 + 8 and
+// packed into AWQ words; y is then qweight [K, N/8] int32 with box {4 words,
+// 64 rows} (one epilogue warp's share of a tile), no swizzle, and qzeros
+// [K/G, N/8] is filled with 0x88888888.
+struct RcQuant {
+  const void* scales;
+  int32_t* qzeros;
+  int n;                  // weight rows N
+  int gsz;                // quantisation group size
+};
+
+// 32 fp32 values (channels k0 .. k0+31 of tile row r) -> four-bit codes
+// clamp(rint(v / s), -8, 7) + 8, with inv0 / inv1 the reciprocals of the
+// bounded scales of the two 16-channel chunks; bytes at codes[channel][row]
+// (channel rows `pitch` bytes apart).
+// The bounds are integers, so clamping before rounding gives the same code;
+// rint is one fp32 addition of 1.5 * 2^23 (round to nearest even at unit
+// spacing, exact for |v| <= 8), whose low mantissa bits are then the signed
+// code, offset by 8 in the integer domain.  A NaN quotient gives level 0
+// (code 8), infinities the clamped ends, as the stage-by-stage quantiser does.
+__device__ __forceinline__ void rc_codes32(uint32_t codes, int r, int k0, const uint32_t (&v)[32], float inv0,
+                                           float inv1, uint32_t pitch) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const float x = __uint_as_float(v[e]) * (e < 16 ? inv0 : inv1);
+    const float t = fminf(fmaxf(x == x ? x : 0.0f, -8.0f), 7.0f);   // NaN -> level 0, as rint + clamp gives
+    const uint32_t q = (__float_as_uint(t + 12582912.0f) + 8u) & 0xFu;
+    asm volatile("st.shared.u8 [%0], %1;" ::"r"(codes + (uint32_t)(k0 + e) * pitch + (uint32_t)r), "r"(q)
+                 : "memory");
+  }
+}
+
 // Per member: r = its R' parts as [2K, 128] fp16, y = its X_r [M, K] fp16
 // (stores), both box {64, 128} with the 128-byte swizzle.
 struct alignas(64) RcTarget {
@@ -220,11 +266,12 @@ struct RcBatch {
 
 // grid P <= number of SMs, block kRcThreads.  tmX: x [M, K] fp16, box {64, 128},
 // 128-byte swizzle.  jobs = members * groups * tiles.
-template <typename TA>
-__global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
+template <typename TA, bool QUANT = false>
+__global__ void __launch_bounds__(rc_threads<QUANT>(), 1) rotate_tc_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ RcBatch batch, int members, int K,
-    int groups, int tiles, long long jobs) {
+    int groups, int tiles, long long jobs, const RcQuant qo) {
   using L = RcLayout;
+  constexpr int EPI = rc_epi_warps<QUANT>();
   extern __shared__ unsigned char smem_raw[];
   unsigned char* const sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t base = smem_u32(sbase);
@@ -250,7 +297,7 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(acc_full0 + 8 * a, 1);
-      mbar_init(acc_empty0 + 8 * a, kRcEpiWarps);
+      mbar_init(acc_empty0 + 8 * a, EPI);
     }
     mbar_init(r_full, 1);
     mbar_init(r_free, 1);
@@ -271,8 +318,9 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
   __syncthreads();
   tc_fence_after();
   // tensor memory is held: a dependent kernel may launch now without ever
-  // taking columns this one still needs
-  pdl_launch_dependents();
+  // taking columns this one still needs (not the quantiser: its outputs are
+  // layer constants that the kernels after it read before they wait)
+  if constexpr (!QUANT) pdl_launch_dependents();
   const uint32_t tmem0 = *tmem_slot;
   // R' comes from the build kernel, x from the kernel before it (the build
   // kernel completes only after that one has)
@@ -350,7 +398,9 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
     const int q = warp & 3;                // TMEM lane quadrant of this warp
     const int r = 32 * q + lane;           // tile row of this thread
     const bool leader = warp == 2 && lane == 0;   // issues the TMA stores
-    // All four warps take part in both named barriers of every tile, even
+    // with eight epilogue warps, warps 2..5 take columns 0..63 and 6..9 columns 64..127
+    const int hcol = QUANT ? (warp - 2) >> 2 : 0;
+    // All epilogue warps take part in every named barrier of every tile, even
     // after a wait has given up (the work is skipped, the barriers are not),
     // so no warp can be left at a barrier; a given-up wait returns at once.
     for (int i = 0; i < nj; ++i) {
@@ -358,45 +408,108 @@ __global__ void __launch_bounds__(kRcThreads, 1) rotate_tc_kernel(
       const long long u = j / tiles;
       const int m = (int)(u / groups), g = (int)(u % groups), t = (int)(j % tiles);
       const int a = i & 1;
+      // quantiser scales of this thread's row and 16-channel chunks, requested
+      // before the wait for the accumulator (a chunk lies in one group of G >= 16)
+      float inv[4];                        // chunks 4 hcol .. 4 hcol + 3 of the tile's 8
+      if constexpr (QUANT) {
+        const int n = t * 128 + r;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int qg = (g * kGroup + 64 * hcol + 16 * kk) / qo.gsz;
+          float sc = n < qo.n ? Act<TA>::f1(static_cast<const TA*>(qo.scales)[(size_t)qg * qo.n + n]) : 1.0f;
+          sc = fminf(fmaxf(sc, 1e-5f), 1e5f);
+          inv[kk] = 1.0f / sc;
+        }
+      }
       // warp-uniform (tcgen05.ld is a warp-wide instruction)
       const bool ok = __all_sync(0xffffffffu, tc_wait(acc_full0 + 8 * a, (uint32_t)((i >> 1) & 1), abort));
       uint32_t v0[32], v1[32], v2[32], v3[32];
       if (ok) {
         tc_fence_after();
-        const uint32_t ta = tmem0 + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128);
+        const uint32_t ta = tmem0 + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128 + 64 * hcol);
         tmem_ld32(ta, v0);
         tmem_ld32(ta + 32, v1);
-        tmem_ld32(ta + 64, v2);
-        tmem_ld32(ta + 96, v3);
+        if constexpr (!QUANT) {
+          tmem_ld32(ta + 64, v2);
+          tmem_ld32(ta + 96, v3);
+        }
         tmem_ld_wait_tie(v0);
         tmem_tie(v1);
-        tmem_tie(v2);
-        tmem_tie(v3);
+        if constexpr (!QUANT) {
+          tmem_tie(v2);
+          tmem_tie(v3);
+        }
       }
       // the accumulator may be overwritten once every warp has read it
       tc_fence_before();
       __syncwarp();
       if (lane == 0 && ok) mbar_arrive(acc_empty0 + 8 * a);
-      // staging tile i & 1 is free once the stores of tile i - 2 have read it
-      if (leader) bulk_wait_group_read<1>();
-      named_bar_sync(1, 32 * kRcEpiWarps);
       const uint32_t tile = base + L::O_OFF + (uint32_t)(i & 1) * L::O_STAGE;
-      if (ok) {
-        rc_stage32<TA>(tile, r, 0, v0);
-        rc_stage32<TA>(tile, r, 1, v1);
-        rc_stage32<TA>(tile, r, 2, v2);
-        rc_stage32<TA>(tile, r, 3, v3);
-      }
-      fence_proxy_async_smem();            // the tile is read by the TMA (async proxy)
-      named_bar_sync(2, 32 * kRcEpiWarps);
-      if (leader && !*abort) {
-        tma_store_2d(&batch.t[m].y, tile, g * 128, t * 128);
-        tma_store_2d(&batch.t[m].y, tile + L::BOX, g * 128 + 64, t * 128);
-        bulk_commit_group();
+      if constexpr (QUANT) {
+        // Each warp packs its own 32 rows x 64 channels: codes as bytes
+        // [64 channels][32 rows], then 4 AWQ words per channel [64][4]
+        // (16-byte rows), written by the warp with one TMA store of a
+        // {4 words, 64 rows} box; no CTA-wide barrier.
+        const int ew = warp - 2;                                  // 0 .. 7
+        const uint32_t codes = base + L::O_OFF + (uint32_t)(i & 1) * L::O_STAGE + (uint32_t)ew * 3072u;
+        const uint32_t words = codes + 2048u;
+        if (lane == 0) bulk_wait_group_read<1>();                 // this warp's store of tile i - 2 has read them
+        __syncwarp();
+        if (ok) {
+          rc_codes32(codes, lane, 0, v0, inv[0], inv[1], 32);
+          rc_codes32(codes, lane, 32, v1, inv[2], inv[3], 32);
+        }
+        __syncwarp();
+        if (ok) {
+          // word (k, w): rows 8w .. 8w+7 of channel k, row 8w + i at nibble
+          // (i >> 1) + 4 (i & 1): the even rows' codes fill the low half-word,
+          // the odd rows' the high one
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int idx = lane + 32 * it, k = idx >> 2, w = idx & 3;
+            uint32_t lo, hi;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi)
+                         : "r"(codes + (uint32_t)k * 32u + 8u * (uint32_t)w));
+            const uint32_t ev = prmt(lo, hi, 0x6420), od = prmt(lo, hi, 0x7531);   // bytes of rows 0,2,4,6 / 1,3,5,7
+            const uint32_t e2 = ev | (ev >> 4), o2 = od | (od >> 4);              // two nibbles per even byte
+            sts_f32(words + (uint32_t)k * 16u + 4u * (uint32_t)w, __uint_as_float(prmt(e2, o2, 0x6420)));
+          }
+          if (ew == 0) {
+            // the tile's zero words: rows of its quantisation groups, its 16 word columns
+            const int zrows = kGroup / qo.gsz, zw = qo.n / 8;
+            for (int idx = lane; idx < zrows * 16; idx += 32) {
+              const int wc = t * 16 + (idx & 15);
+              if (wc < zw) qo.qzeros[(size_t)((g * kGroup) / qo.gsz + (idx >> 4)) * zw + wc] = (int32_t)0x88888888u;
+            }
+          }
+        }
+        fence_proxy_async_smem();          // the words are read by the TMA (async proxy)
+        __syncwarp();
+        if (lane == 0 && ok && !*abort) {
+          tma_store_2d(&batch.t[m].y, words, t * 16 + 4 * q, g * 128 + 64 * hcol);
+          bulk_commit_group();
+        }
+      } else {
+        // staging tile i & 1 is free once the stores of tile i - 2 have read it
+        if (leader) bulk_wait_group_read<1>();
+        named_bar_sync(1, 32 * EPI);
+        if (ok) {
+          rc_stage32<TA>(tile, r, 0, v0);
+          rc_stage32<TA>(tile, r, 1, v1);
+          rc_stage32<TA>(tile, r, 2, v2);
+          rc_stage32<TA>(tile, r, 3, v3);
+        }
+        fence_proxy_async_smem();          // the tile is read by the TMA (async proxy)
+        named_bar_sync(2, 32 * EPI);
+        if (leader && !*abort) {
+          tma_store_2d(&batch.t[m].y, tile, g * 128, t * 128);
+          tma_store_2d(&batch.t[m].y, tile + L::BOX, g * 128 + 64, t * 128);
+          bulk_commit_group();
+        }
       }
     }
-    // the stores have written X_r before the kernel completes
-    if (leader) bulk_wait_group_all();
+    // the stores have written X_r (the words) before the kernel completes
+    if (QUANT ? lane == 0 : leader) bulk_wait_group_all();
   }
 
   if (warp == 0 && lane == 0 && *abort) {
