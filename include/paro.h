@@ -131,6 +131,19 @@ int paro_rotate_dt(const void* x, void* x_r, int64_t M, int64_t K, const float* 
                    paro_stream_t stream);
 
 /*
+ * paro_rotate_rmat — X_r = rotate(x * channel_scales) as the product x R' with a
+ * prepared R' (paro_rotation_matrix_prepare, which holds the channel scales,
+ * pairs, theta, group size and krot), on the tensor cores: X R_hi + X R_lo
+ * accumulated in fp32, rounded once to the activation type.  Any M (tiles
+ * of 128 rows); the same result as paro_w4_linear's rotation above 64 rows.
+ *   x, x_r   device [M, K] of `dtype`, 16-byte aligned, not the same buffer
+ *   rmat     the prepared parts for this K and dtype, 256-byte aligned
+ * Faster than paro_rotate for large M (the stages cost no more with krot).
+ */
+int paro_rotate_rmat(const void* x, void* x_r, int64_t M, int64_t K, const void* rmat, int dtype,
+                     paro_stream_t stream);
+
+/*
  * paro_pack_awq — pack 4-bit codes into AWQ int32 words (page "ParoQuant",
  * "Stored tensors": qweight (I, O//8), qzeros (I//G, O//8); packer needs O % 8 == 0).
  *   codes       device uint8 [N, K]    (out x in), values 0..15 (the high nibble is ignored)

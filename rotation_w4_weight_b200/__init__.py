@@ -4,7 +4,7 @@ The compute lives in the CUDA library ``libparo_b200.so`` behind the C ABI of
 ``include/paro.h``; this module only marshals torch tensors (device memory and
 streams) into that ABI.  Functions mirror the C entry points:
 
-    rotate            -> paro_rotate / paro_rotate_dt
+    rotate            -> paro_rotate / paro_rotate_dt, or paro_rotate_rmat with a prepared R'
     pack_awq          -> paro_pack_awq
     unpack_awq        -> paro_unpack_awq
     w4_linear         -> paro_w4_linear / paro_w4_linear_dt (+ paro_w4_linear_workspace_size)
@@ -37,7 +37,7 @@ from ._lib import (PARO_ERR_ALIGNMENT, PARO_ERR_CUDA, PARO_ERR_INVALID_ARG,  # n
                    paro_w4_linear_dt, paro_w4_linear_group_dt, paro_rotation_matrix_size,
                    paro_rotation_matrix_prepare, PARO_DTYPE_F16, paro_w4_moe_workspace_size,
                    paro_w4_moe_linear, paro_w4_moe_launches, paro_quantize_w4_workspace_size,
-                   paro_quantize_w4_tc)
+                   paro_quantize_w4_tc, paro_rotate_rmat)
 
 __all__ = ["rotate", "pack_awq", "unpack_awq", "w4_linear", "w4_linear_workspace_size",
            "w4_linear_group", "w4_linear_group_launches", "quantize_w4", "validate_pairs", "device_status",
@@ -79,10 +79,24 @@ def _need(t: Optional[torch.Tensor], dtype, name: str, allow_none: bool = False)
 
 def rotate(x: torch.Tensor, channel_scales: Optional[torch.Tensor], pairs: Optional[torch.Tensor],
            theta: Optional[torch.Tensor], group_size: int = 128, krot: Optional[int] = None,
-           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """X_r = rotate(x * channel_scales); ``out`` may be ``x`` (in place)."""
+           out: Optional[torch.Tensor] = None, stream=None, rmat: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """X_r = rotate(x * channel_scales); ``out`` may be ``x`` (in place).
+
+    With ``rmat`` (this layer's prepared R', ``rotation_matrix``) the product
+    x R' runs on the tensor cores (channel_scales/pairs/theta are then not
+    read; ``out`` must be another buffer)."""
     dt = _act(x, "x")
     _need(x, dt, "x")
+    if rmat is not None:
+        _need(rmat, torch.uint8, "rmat")
+        if out is None:
+            out = torch.empty_like(x)
+        _need(out, dt, "out")
+        M, K = x.shape
+        check(paro_rotate_rmat(_ptr(x), _ptr(out), M, K, _ptr(rmat),
+                               PARO_DTYPE_F16 if dt == torch.float16 else PARO_DTYPE_BF16, _stream(stream)),
+              "paro_rotate_rmat")
+        return out
     _need(channel_scales, torch.float32, "channel_scales", True)
     _need(pairs, torch.int16, "pairs", True)
     _need(theta, torch.float32, "theta", True)

@@ -31,7 +31,7 @@ EXPORTED = (
     "paro_selftest_wait_timeout", "paro_rotate_dt", "paro_quantize_w4_dt", "paro_w4_linear_dt",
     "paro_w4_linear_group_dt", "paro_w4_linear_noalloc_dt", "paro_rotation_matrix_size",
     "paro_rotation_matrix_prepare", "paro_w4_moe_workspace_size", "paro_w4_moe_linear", "paro_w4_moe_launches",
-    "paro_quantize_w4_workspace_size", "paro_quantize_w4_tc",
+    "paro_quantize_w4_workspace_size", "paro_quantize_w4_tc", "paro_rotate_rmat",
 )
 
 PARO_MAX_GROUP = 4
@@ -80,6 +80,7 @@ _SIGNATURES = {
                                   _int, _int, _int, _vp, ctypes.c_size_t, _vp]),
     "paro_w4_moe_launches": (_int, [_i64, _i64, _i64, _int, _int, _int, _int, _int]),
     "paro_quantize_w4_workspace_size": (ctypes.c_size_t, [_i64]),
+    "paro_rotate_rmat": (_int, [_vp, _vp, _i64, _i64, _vp, _int, _vp]),
     "paro_quantize_w4_tc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp, ctypes.c_size_t,
                                    _vp]),
 }
@@ -128,6 +129,7 @@ paro_w4_moe_linear = lib.paro_w4_moe_linear
 paro_w4_moe_launches = lib.paro_w4_moe_launches
 paro_quantize_w4_workspace_size = lib.paro_quantize_w4_workspace_size
 paro_quantize_w4_tc = lib.paro_quantize_w4_tc
+paro_rotate_rmat = lib.paro_rotate_rmat
 
 
 class ParoError(RuntimeError):

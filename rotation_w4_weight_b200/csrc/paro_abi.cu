@@ -785,6 +785,21 @@ int paro_rotate_dt(const void* x, void* x_r, int64_t M, int64_t K, const float* 
   }
 }
 
+int paro_rotate_rmat(const void* x, void* x_r, int64_t M, int64_t K, const void* rmat, int dtype,
+                     paro_stream_t stream) {
+  if (dtype != PARO_DTYPE_F16 && dtype != PARO_DTYPE_BF16) return PARO_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0) return PARO_ERR_INVALID_ARG;
+  if (K % kGroup != 0 || K >= (int64_t(1) << 24) || M * K >= (int64_t(1) << 31)) return PARO_ERR_UNSUPPORTED;
+  if (M == 0) return PARO_OK;
+  if (x == nullptr || x_r == nullptr || rmat == nullptr) return PARO_ERR_INVALID_ARG;
+  if (x == x_r) return PARO_ERR_INVALID_ARG;      // tiles are read and written by different stages of one pass
+  if (!aligned(x, 16) || !aligned(x_r, 16) || !aligned(rmat, 256)) return PARO_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const RotTcMember one{nullptr, nullptr, nullptr, 0, x_r, const_cast<void*>(rmat), true};
+  if (dtype == PARO_DTYPE_F16) return launch_rotate_tc<__half>(static_cast<const __half*>(x), &one, 1, M, K, kGroup, s);
+  return launch_rotate_tc<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), &one, 1, M, K, kGroup, s);
+}
+
 int paro_quantize_w4(const void* w, const float* channel_scales, const int16_t* pairs,
                      const float* theta, const void* scales, int32_t* qweight, int32_t* qzeros,
                      int64_t N, int64_t K, int group_size, int krot, paro_stream_t stream) {

@@ -310,3 +310,15 @@ def test_moe_shape_checks_and_queries(L):
     assert moe(n=need - 1) == L.PARO_ERR_WORKSPACE
     assert moe(ws=None) == L.PARO_ERR_INVALID_ARG
     assert moe(T=0) == L.PARO_OK                                 # no tokens: no work
+
+
+def test_rotate_rmat_checks(L):
+    r = lambda x=A16, y=P(0x20000), M=4, K=256, rm=P(0x100000), dt=0: L.paro_rotate_rmat(x, y, M, K, rm, dt, None)  # noqa: E731
+    assert r(dt=2) == L.PARO_ERR_INVALID_ARG
+    assert r(M=-1) == L.PARO_ERR_INVALID_ARG
+    assert r(K=200) == L.PARO_ERR_UNSUPPORTED
+    assert r(rm=None) == L.PARO_ERR_INVALID_ARG
+    assert r(y=A16) == L.PARO_ERR_INVALID_ARG          # not in place
+    assert r(x=MIS) == L.PARO_ERR_ALIGNMENT
+    assert r(rm=P(0x100010)) == L.PARO_ERR_ALIGNMENT
+    assert r(M=0) == L.PARO_OK

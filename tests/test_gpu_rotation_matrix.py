@@ -133,3 +133,28 @@ def test_prepare_flags_pair_index_outside_group():
     r = pb.rotation_matrix(d["cs"], dev(bad), d["theta"], K, 128, lay.krot)
     assert r.numel() == K * 128 * 4
     assert pb.device_status(clear=True) == pb.PARO_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("M", [1, 65, 300])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_rotate_with_prepared_rmat(M, dtype):
+    """paro_rotate_rmat: X_r = x R' on the tensor cores, the rotation of a
+    linear call above 64 rows (bit for bit), within the rotation tolerance of
+    the oracle."""
+    K, N = 512, 256
+    lay = synth.make_layer("rr", K, N, seed=M + 3)
+    d = layer_to_device(lay)
+    R = rmat_of(lay, d, dtype)
+    x = torch.from_numpy(synth.make_activations(lay, M).astype(np.float32)).to(dtype).cuda()
+    xr = pb.rotate(x, None, None, None, 128, 0, rmat=R)
+    if M > 64:
+        ws = torch.empty(pb.w4_linear_workspace_size(M, K, N, 128), dtype=torch.uint8, device="cuda")
+        pb.w4_linear(x, d["qweight"], d["qzeros"], d["scales"].to(dtype), None, d["cs"], d["pairs"], d["theta"],
+                     128, lay.krot, workspace=ws, rmat=R)
+        torch.cuda.synchronize()
+        assert torch.equal(xr, ws[: M * K * 2].view(dtype).view(M, K))
+    ref = oracle.rotate(x.float().cpu().numpy().astype(np.float64), lay.channel_scales, lay.pairs, lay.theta, 128)
+    got = xr.float().cpu().numpy().astype(np.float64)
+    rms = np.sqrt(np.mean(ref * ref, axis=1, keepdims=True))
+    tol = 1e-3 if dtype == torch.float16 else 5e-3
+    assert np.max(np.abs(got - ref) / np.maximum(np.abs(ref), rms)) <= tol
