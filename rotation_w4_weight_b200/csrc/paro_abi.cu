@@ -1127,8 +1127,10 @@ int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_li
     return (rot > 0 ? (build ? 2 : 1) : 0) + 1;
   }
   LinearPlan gp;
-  // one after another: each rotating member launches its rotation and its GEMV / GEMM
-  if (count == 1 || !group_plan(M, K, linears, count, G, &gp)) return rot + count;
+  // one GEMV per member: several members still share one warp-per-row
+  // rotation launch when every rotation fits it, else each rotates alone
+  if (count == 1 || !group_plan(M, K, linears, count, G, &gp))
+    return (count > 1 && rows_ok && rot > 0 ? 1 : rot) + count;
   return (rot > 0 ? (rows_ok ? 1 : rot) : 0) + 1;
 }
 
@@ -1199,6 +1201,34 @@ int group_impl(const void* x, int64_t M, int64_t K, int count, const paro_linear
 
   LinearPlan gp;
   if (count == 1 || !group_plan(M, K, linears, count, G, &gp)) {
+    // Decode members that need a GEMV launch each (the group does not fit one
+    // wave) still share one warp-per-row rotation launch for every distinct
+    // rotation; each GEMV then reads its rotation's X_r.
+    if (count > 1 && M <= 16) {
+      RrBatch rb;
+      std::memset(&rb, 0, sizeof(rb));
+      int nrot = 0, max_krot = 0;
+      bool rows_ok = true;
+      for (int i = 0; i < count; ++i) {
+        const paro_linear& l = linears[i];
+        if (rotation_owner(linears, i) != i) continue;
+        rows_ok = rows_ok && l.krot <= kRrMaxKrot;
+        rb.op[nrot++] = RrOperand{ws + i * per + first.off_xr, l.channel_scales, l.pairs, l.theta, l.krot};
+        max_krot = std::max(max_krot, l.krot);
+      }
+      if (rows_ok && nrot > 0) {
+        if (int st = launch_rotate_rows<TA>(static_cast<const TA*>(x), rb, nrot, M, K, max_krot, G, s)) return st;
+        for (int i = 0; i < count; ++i) {
+          const paro_linear& l = linears[i];
+          const int o = rotation_owner(linears, i);
+          const void* src = o >= 0 ? static_cast<const void*>(ws + o * per + first.off_xr) : x;
+          if (int st = linear_impl<TA>(src, l.y, M, K, l.N, l.qweight, l.qzeros, l.scales, l.bias, nullptr, nullptr,
+                                       nullptr, group_size, 0, nullptr, 0, s))
+            return st;
+        }
+        return PARO_OK;
+      }
+    }
     // one call per member, each with its own slice of the workspace; a member
     // that shares an earlier member's rotation reads that member's X_r
     for (int i = 0; i < count; ++i) {
