@@ -391,7 +391,7 @@ int launch_quantize_tc(const __half* w, const float* cs, const int16_t* pairs, c
   CUtensorMap tmX;
   if (!encode_2d(&rc.t[0].r, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, rt, 2 * K, kGroup, 128, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&rc.t[0].y, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, 64, 4,
+      !encode_2d(&rc.t[0].y, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, qweight, K, N / 8, kRcQuantCols, 4,
                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w, N, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return PARO_ERR_CUDA;
@@ -458,14 +458,16 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N, int gsz) {
     p.nt = M <= 8 ? 1 : 2;
     // Configuration by shape class, from sweeps on B200 over the Llama-3-8B
     // decode shapes (column tile, k-parts, stages, split along K):
-    //   wide (N > 4096, e.g. gate/up):      256 columns, 2 k-parts, 4-stage ring, split 2
+    //   wide (N > 4096, e.g. gate/up):      256 columns, 2 k-parts, 4-stage ring, split 4 for
+    //                                        M <= 4 (two CTAs on most SMs: gate 10.2 -> 9.8 us at
+    //                                        M = 1), split 2 above (M = 8: split 4 is 4 % slower)
     //   deep (N <= 4096, K > 4096, down):   128 columns, 2 k-parts, 4-stage ring, split 8
     //   square/narrow (q, o, k, v), M <= 8: 128 columns, 4 k-parts, 8 stages, split 4 (8 if N <= 2048)
     //   square, 8 < M <= 16:                64 columns, 4 k-parts, 8 stages, split 2
     //   narrow (N <= 2048), 8 < M <= 16:    128 columns, 2 k-parts, 4 stages, split 8
     int tile, want;
     if (N > 4096) {
-      tile = 256; p.variant = 0; want = 2;
+      tile = 256; p.variant = 0; want = M <= 4 ? 4 : 2;
     } else if (K > 4096) {
       tile = 128; p.variant = 3; want = 8;
     } else if (M <= 8) {

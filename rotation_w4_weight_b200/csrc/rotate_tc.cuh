@@ -175,10 +175,11 @@ __global__ void __launch_bounds__(kRbThreads) rmat_build_kernel(const __grid_con
 constexpr int kRcStages = 3;
 constexpr int kRcEpiWarps = 4;
 constexpr int kRcThreads = 32 * (2 + kRcEpiWarps);
-// The quantising variant has twice the epilogue warps (two per TMEM lane
-// quadrant, 64 columns each): its epilogue does more work per value.
+// The quantising variant has four times the epilogue warps (four per TMEM
+// lane quadrant, 32 columns each): its epilogue does more work per value.
 template <bool QUANT>
-__host__ __device__ constexpr int rc_epi_warps() { return QUANT ? 2 * kRcEpiWarps : kRcEpiWarps; }
+__host__ __device__ constexpr int rc_epi_warps() { return QUANT ? 4 * kRcEpiWarps : kRcEpiWarps; }
+constexpr int kRcQuantCols = 128 / (4 * kRcEpiWarps / 4);   // columns per quantising epilogue warp
 template <bool QUANT>
 __host__ __device__ constexpr int rc_threads() { return 32 * (2 + rc_epi_warps<QUANT>()); }
 constexpr int kRcCols = 256;
@@ -224,7 +225,7 @@ __device__ __forceinline__ void rc_stage32(uint32_t tile, int r, int cb, const u
 // the product is W_r = W D R, and each tile is quantised with the quantiser
 // scales [K/G, N] (bounded to [1e-5, 1e5]) into four-bit codes -8..7 + 8 and
 // packed into AWQ words; y is then qweight [K, N/8] int32 with box {4 words,
-// 64 rows} (one epilogue warp's share of a tile), no swizzle, and qzeros
+// kRcQuantCols rows} (one epilogue warp's share of a tile), no swizzle, and qzeros
 // [K/G, N/8] is filled with 0x88888888.
 struct RcQuant {
   const void* scales;
@@ -398,8 +399,8 @@ __global__ void __launch_bounds__(rc_threads<QUANT>(), 1) rotate_tc_kernel(
     const int q = warp & 3;                // TMEM lane quadrant of this warp
     const int r = 32 * q + lane;           // tile row of this thread
     const bool leader = warp == 2 && lane == 0;   // issues the TMA stores
-    // with eight epilogue warps, warps 2..5 take columns 0..63 and 6..9 columns 64..127
-    const int hcol = QUANT ? (warp - 2) >> 2 : 0;
+    // quantising: warps 2..5 take columns 0..31, 6..9 columns 32..63, and so on
+    const int c0 = QUANT ? kRcQuantCols * ((warp - 2) >> 2) : 0;
     // All epilogue warps take part in every named barrier of every tile, even
     // after a wait has given up (the work is skipped, the barriers are not),
     // so no warp can be left at a barrier; a given-up wait returns at once.
@@ -410,12 +411,12 @@ __global__ void __launch_bounds__(rc_threads<QUANT>(), 1) rotate_tc_kernel(
       const int a = i & 1;
       // quantiser scales of this thread's row and 16-channel chunks, requested
       // before the wait for the accumulator (a chunk lies in one group of G >= 16)
-      float inv[4];                        // chunks 4 hcol .. 4 hcol + 3 of the tile's 8
+      float inv[kRcQuantCols / 16];        // this warp's 16-channel chunks
       if constexpr (QUANT) {
         const int n = t * 128 + r;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int qg = (g * kGroup + 64 * hcol + 16 * kk) / qo.gsz;
+        for (int kk = 0; kk < kRcQuantCols / 16; ++kk) {
+          const int qg = (g * kGroup + c0 + 16 * kk) / qo.gsz;
           float sc = n < qo.n ? Act<TA>::f1(static_cast<const TA*>(qo.scales)[(size_t)qg * qo.n + n]) : 1.0f;
           sc = fminf(fmaxf(sc, 1e-5f), 1e5f);
           inv[kk] = 1.0f / sc;
@@ -426,16 +427,16 @@ __global__ void __launch_bounds__(rc_threads<QUANT>(), 1) rotate_tc_kernel(
       uint32_t v0[32], v1[32], v2[32], v3[32];
       if (ok) {
         tc_fence_after();
-        const uint32_t ta = tmem0 + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128 + 64 * hcol);
+        const uint32_t ta = tmem0 + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 128 + c0);
         tmem_ld32(ta, v0);
-        tmem_ld32(ta + 32, v1);
         if constexpr (!QUANT) {
+          tmem_ld32(ta + 32, v1);
           tmem_ld32(ta + 64, v2);
           tmem_ld32(ta + 96, v3);
         }
         tmem_ld_wait_tie(v0);
-        tmem_tie(v1);
         if constexpr (!QUANT) {
+          tmem_tie(v1);
           tmem_tie(v2);
           tmem_tie(v3);
         }
@@ -446,26 +447,24 @@ __global__ void __launch_bounds__(rc_threads<QUANT>(), 1) rotate_tc_kernel(
       if (lane == 0 && ok) mbar_arrive(acc_empty0 + 8 * a);
       const uint32_t tile = base + L::O_OFF + (uint32_t)(i & 1) * L::O_STAGE;
       if constexpr (QUANT) {
-        // Each warp packs its own 32 rows x 64 channels: codes as bytes
-        // [64 channels][32 rows], then 4 AWQ words per channel [64][4]
+        // Each warp packs its own 32 rows x 32 channels: codes as bytes
+        // [32 channels][32 rows], then 4 AWQ words per channel [32][4]
         // (16-byte rows), written by the warp with one TMA store of a
-        // {4 words, 64 rows} box; no CTA-wide barrier.
-        const int ew = warp - 2;                                  // 0 .. 7
-        const uint32_t codes = base + L::O_OFF + (uint32_t)(i & 1) * L::O_STAGE + (uint32_t)ew * 3072u;
-        const uint32_t words = codes + 2048u;
+        // {4 words, 32 rows} box; no CTA-wide barrier.
+        const int ew = warp - 2;                                  // 0 .. EPI - 1
+        constexpr uint32_t kCodes = 32u * kRcQuantCols, kWarpArea = kCodes + 16u * kRcQuantCols;
+        const uint32_t codes = base + L::O_OFF + (uint32_t)(i & 1) * L::O_STAGE + (uint32_t)ew * kWarpArea;
+        const uint32_t words = codes + kCodes;
         if (lane == 0) bulk_wait_group_read<1>();                 // this warp's store of tile i - 2 has read them
         __syncwarp();
-        if (ok) {
-          rc_codes32(codes, lane, 0, v0, inv[0], inv[1], 32);
-          rc_codes32(codes, lane, 32, v1, inv[2], inv[3], 32);
-        }
+        if (ok) rc_codes32(codes, lane, 0, v0, inv[0], inv[1], 32);
         __syncwarp();
         if (ok) {
           // word (k, w): rows 8w .. 8w+7 of channel k, row 8w + i at nibble
           // (i >> 1) + 4 (i & 1): the even rows' codes fill the low half-word,
           // the odd rows' the high one
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {
+          for (int it = 0; it < kRcQuantCols * 4 / 32; ++it) {
             const int idx = lane + 32 * it, k = idx >> 2, w = idx & 3;
             uint32_t lo, hi;
             asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo), "=r"(hi)
@@ -486,7 +485,7 @@ __global__ void __launch_bounds__(rc_threads<QUANT>(), 1) rotate_tc_kernel(
         fence_proxy_async_smem();          // the words are read by the TMA (async proxy)
         __syncwarp();
         if (lane == 0 && ok && !*abort) {
-          tma_store_2d(&batch.t[m].y, words, t * 16 + 4 * q, g * 128 + 64 * hcol);
+          tma_store_2d(&batch.t[m].y, words, t * 16 + 4 * q, g * 128 + c0);
           bulk_commit_group();
         }
       } else {
