@@ -433,6 +433,7 @@ size_t gemv_layout_bytes(int variant, int nt, int gmax, int gr) {
   const bool one = nt == 1;
   switch (variant) {
     case 0: return one ? GemvLayout<1, 2, 256, 4>::smem(gmax, gr) : GemvLayout<2, 2, 256, 4>::smem(gmax, gr);
+    case 6: return one ? GemvLayout<1, 2, 256, 2>::smem(gmax, gr) : 0;
     case 2: return one ? GemvLayout<1, 4, 128, 8>::smem(gmax, gr) : GemvLayout<2, 4, 128, 8>::smem(gmax, gr);
     case 5: return one ? GemvLayout<1, 4, 64, 8>::smem(gmax, gr) : GemvLayout<2, 4, 64, 8>::smem(gmax, gr);
     default: return one ? GemvLayout<1, 2, 128, 4>::smem(gmax, gr) : GemvLayout<2, 2, 128, 4>::smem(gmax, gr);
@@ -685,6 +686,9 @@ int dispatch_gemv_nl(const LinearPlan& plan, const GemvLinearArgs* lin, int coun
     case 0: return launch_gemv<NT, 2, 256, 4, NL, TA>(plan, lin, count, M, K, s, pdl);
     case 2: return launch_gemv<NT, 4, 128, 8, NL, TA>(plan, lin, count, M, K, s, pdl);
     case 5: return launch_gemv<NT, 4, 64, 8, NL, TA>(plan, lin, count, M, K, s, pdl);
+    case 6:   // grouped wide members in one wave (group_plan): 2-stage ring
+      if constexpr (NT == 1 && NL > 1) return launch_gemv<NT, 2, 256, 2, NL, TA>(plan, lin, count, M, K, s, pdl);
+      return PARO_ERR_UNSUPPORTED;
     default: return launch_gemv<NT, 2, 128, 4, NL, TA>(plan, lin, count, M, K, s, pdl);
   }
 }
@@ -963,7 +967,7 @@ size_t gemv_smem(const LinearPlan& p, int gmax) {
   return gemv_layout_bytes(p.variant, p.nt, gmax, gmax * (kGroup / p.gsz));
 }
 
-int plan_tile(const LinearPlan& p) { return p.variant == 0 ? 256 : (p.variant == 5 ? 64 : 128); }
+int plan_tile(const LinearPlan& p) { return p.variant == 0 || p.variant == 6 ? 256 : (p.variant == 5 ? 64 : 128); }
 
 // One GEMV launch for a group of decode linears sharing x: the plan of the
 // widest member for all of them, taken only when the whole grid is resident
@@ -974,20 +978,42 @@ bool group_plan(int64_t M, int64_t K, const paro_linear* lin, int count, int gsz
   for (int i = 0; i < count; ++i) widest = std::max(widest, lin[i].N);
   LinearPlan p = make_plan(M, K, widest, gsz);
   if (!p.decode) return false;
-  const int tile = plan_tile(p);
-  int64_t tiles = 0;
-  for (int i = 0; i < count; ++i) tiles += (lin[i].N + tile - 1) / tile;
-  const int64_t ctas = tiles * p.splits;
   const int groups = (int)(K / kGroup);
-  const int gmax = (groups + p.splits - 1) / p.splits;
-  const size_t fp = gemv_footprint(gemv_smem(p, gmax), ctas);
   const DeviceInfo& dev = device_info();
-  if (fp == 0 || dev.sms <= 0) return false;
-  const int64_t per_sm = (int64_t)(dev.smem_per_sm / (fp + dev.smem_reserved_per_block));
-  if (ctas > per_sm * dev.sms) return false;
-  p.n_tiles = (int)tiles;
-  *out = p;
-  return true;
+  if (dev.sms <= 0) return false;
+  auto fits = [&](LinearPlan& q) {
+    const int tile = plan_tile(q);
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) tiles += (lin[i].N + tile - 1) / tile;
+    const int64_t ctas = tiles * q.splits;
+    const int gmax = (groups + q.splits - 1) / q.splits;
+    if (gmax > kGvMaxGroups) return false;
+    const size_t need = gemv_smem(q, gmax);
+    if (need == 0 || need > kSmemPerCta) return false;
+    const size_t fp = gemv_footprint(need, ctas);
+    if (fp == 0) return false;
+    const int64_t per_sm = (int64_t)(dev.smem_per_sm / (fp + dev.smem_reserved_per_block));
+    if (ctas > per_sm * dev.sms) return false;
+    q.n_tiles = (int)tiles;
+    return true;
+  };
+  if (fits(p)) {
+    *out = p;
+    return true;
+  }
+  // wide members (gate and up, say) at up to 8 tokens: half the split and a
+  // 2-stage ring (one stage per k-part) put two CTAs on an SM, so the pair
+  // shares one launch
+  LinearPlan q = p;
+  if (count > 1 && p.variant == 0 && p.nt == 1 && p.splits >= 2) {
+    q.variant = 6;
+    q.splits = p.splits / 2;
+    if (fits(q)) {
+      *out = q;
+      return true;
+    }
+  }
+  return false;
 }
 
 template <typename TA>

@@ -90,6 +90,10 @@ struct GemvLayout {
     return bar_off(gmax, gr) + 8 * (2 * STAGES + 3) + 1024;
   }
   static_assert(STAGES <= kGvMaxStages, "too many stages");
+  // k-part p consumes groups p, p + KP, ...: with STAGES a multiple of KP every
+  // stage (group i sits in stage i % STAGES) belongs to one k-part, so its
+  // mbarrier phases are waited on in order and never aliased by parity
+  static_assert(STAGES % KP == 0, "each stage must belong to one k-part");
   // 128-byte swizzle needs 128-byte rows; 64-byte rows use the 64-byte swizzle
   static constexpr int ROW_BYTES = WORDS * 4;
 };
