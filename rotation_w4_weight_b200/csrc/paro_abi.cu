@@ -973,47 +973,56 @@ int plan_tile(const LinearPlan& p) { return p.variant == 0 || p.variant == 6 ? 2
 // widest member for all of them, taken only when the whole grid is resident
 // at once with that plan's footprint (larger groups gain nothing from sharing
 // a launch: each member already fills the GPU).
+// Whether a decode GEMV grid of `ctas` CTAs with plan p is resident at once
+// (false when the device's limits are unknown).
+bool gemv_one_wave(const LinearPlan& p, int64_t K, int64_t ctas) {
+  const DeviceInfo& dev = device_info();
+  if (dev.sms <= 0) return false;
+  const int groups = (int)(K / kGroup);
+  const int gmax = (groups + p.splits - 1) / p.splits;
+  if (gmax > kGvMaxGroups) return false;
+  const size_t need = gemv_smem(p, gmax);
+  if (need == 0 || need > kSmemPerCta) return false;
+  const size_t fp = gemv_footprint(need, ctas);
+  if (fp == 0) return false;
+  const int64_t per_sm = (int64_t)(dev.smem_per_sm / (fp + dev.smem_reserved_per_block));
+  return ctas <= per_sm * dev.sms;
+}
+
+// A wide plan (256 columns, 4-stage ring) whose grid of `units` x splits CTAs
+// is not resident at once: the 2-stage ring (one stage per k-part) puts two
+// CTAs on an SM, at the same split or at half of it.  Returns whether *p (as
+// possibly changed) fits one wave.
+bool wide_one_wave(LinearPlan* p, int64_t K, int64_t units) {
+  if (gemv_one_wave(*p, K, units * p->splits)) return true;
+  if (p->variant != 0 || p->nt != 1) return false;
+  for (int sp = p->splits; sp >= 1 && 2 * sp >= p->splits; sp /= 2) {
+    LinearPlan q = *p;
+    q.variant = 6;
+    q.splits = sp;
+    if (gemv_one_wave(q, K, units * sp)) {
+      *p = q;
+      return true;
+    }
+  }
+  return false;
+}
+
 bool group_plan(int64_t M, int64_t K, const paro_linear* lin, int count, int gsz, LinearPlan* out) {
   int64_t widest = 0;
   for (int i = 0; i < count; ++i) widest = std::max(widest, lin[i].N);
   LinearPlan p = make_plan(M, K, widest, gsz);
   if (!p.decode) return false;
-  const int groups = (int)(K / kGroup);
-  const DeviceInfo& dev = device_info();
-  if (dev.sms <= 0) return false;
-  auto fits = [&](LinearPlan& q) {
-    const int tile = plan_tile(q);
-    int64_t tiles = 0;
-    for (int i = 0; i < count; ++i) tiles += (lin[i].N + tile - 1) / tile;
-    const int64_t ctas = tiles * q.splits;
-    const int gmax = (groups + q.splits - 1) / q.splits;
-    if (gmax > kGvMaxGroups) return false;
-    const size_t need = gemv_smem(q, gmax);
-    if (need == 0 || need > kSmemPerCta) return false;
-    const size_t fp = gemv_footprint(need, ctas);
-    if (fp == 0) return false;
-    const int64_t per_sm = (int64_t)(dev.smem_per_sm / (fp + dev.smem_reserved_per_block));
-    if (ctas > per_sm * dev.sms) return false;
-    q.n_tiles = (int)tiles;
-    return true;
-  };
-  if (fits(p)) {
-    *out = p;
-    return true;
-  }
-  // wide members (gate and up, say) at up to 8 tokens: half the split and a
-  // 2-stage ring (one stage per k-part) put two CTAs on an SM, so the pair
-  // shares one launch
-  LinearPlan q = p;
-  if (count > 1 && p.variant == 0 && p.nt == 1 && p.splits >= 2) {
-    q.variant = 6;
-    q.splits = p.splits / 2;
-    if (fits(q)) {
-      *out = q;
-      return true;
-    }
-  }
-  return false;
+  // (variant 6 keeps 256-column tiles, so the tile count does not change)
+  const int tile = plan_tile(p);
+  int64_t tiles = 0;
+  for (int i = 0; i < count; ++i) tiles += (lin[i].N + tile - 1) / tile;
+  // wide members (gate and up, say) at up to 8 tokens share one launch on
+  // the 2-stage ring
+  if (!wide_one_wave(&p, K, tiles)) return false;
+  p.n_tiles = (int)tiles;
+  *out = p;
+  return true;
 }
 
 template <typename TA>
@@ -1420,7 +1429,12 @@ int moe_impl(const void* x, void* y, int64_t T, int64_t K, int64_t N, int E, int
     // segments of at most 8 rows: one token tile of the decode GEMV each
     const LinearPlan plan = make_plan(kMoeGvRows, K, N, G);
     if (plan.decode) {
-      const SegRouting seg{gv, &head->n_gv, perm, (int)std::min<int64_t>(S, S / kMoeGvRows + used), E};
+      // (the 2-stage ring that puts a grouped gate/up pair in one wave was
+      // measured slower here: 1707 vs 2047 GB/s for two gate-shaped experts
+      // at one token; the segment GEMV requests no weights before its wait,
+      // so the deeper ring matters more than the second wave)
+      const int max_segs = (int)std::min<int64_t>(S, S / kMoeGvRows + used);
+      const SegRouting seg{gv, &head->n_gv, perm, max_segs, E};
       const GemvLinearArgs lin{qweight, qzeros, scales, xg, bias, y, N};
       return dispatch_gemv_seg<TA>(plan, lin, S, K, s, seg);
     }

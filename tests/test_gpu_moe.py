@@ -167,3 +167,23 @@ def test_moe_large_prefill_sampled_columns():
     rows = np.random.default_rng(1).choice(T, 48, replace=False)
     ref = ref_of(rot, ex, x[rows], idx[rows])
     assert lin_err(y[rows].reshape(-1, N), ref.reshape(-1, N)) <= LIN_TOL
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_moe_decode_wide_experts(T):
+    """Gate-shaped experts (4096 -> 14336, the wide GEMV plan) at one and two
+    tokens, top-2 of 2.  Sampled columns of every slot against the oracle's
+    columns of its expert."""
+    E, K, N, topk = 2, 4096, 14336, 2
+    rot, ex = make_experts(E, K, N, seed=61)
+    x = synth.make_activations(synth.make_layer("xw", K, 32, seed=T), T)
+    idx = route(T, topk, E, seed=T + 4)
+    y = run(rot, ex, x, idx)
+    cols = np.sort(np.random.default_rng(T).choice(N, 96, replace=False))
+    for t in range(T):
+        for j in range(topk):
+            e = int(idx[t, j])
+            ref = oracle.w4_linear_columns(x[t:t + 1], ex["codes"][e], ex["zeros"][e], ex["scales"][e],
+                                           ex["bias"][e], rot.channel_scales, rot.pairs, rot.theta, 128,
+                                           rot.krot, cols)
+            assert lin_err(y[t, j][None, cols], ref) <= LIN_TOL, (t, j)
