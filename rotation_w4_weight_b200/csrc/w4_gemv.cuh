@@ -471,10 +471,17 @@ __global__ void __launch_bounds__(32 * (1 + (NTILE / 64) * KP), 1) w4_gemv_kerne
     const int n = n0 + (int)rank * cols + c;
     if (n >= N) continue;
     float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int q = 0; q < S * KP; ++q) {
-      const uint4 v = lds128(box + (uint32_t)(((q * L::MP + tl) * cols + c) * 4));
-      sum.x += __uint_as_float(v.x); sum.y += __uint_as_float(v.y);
-      sum.z += __uint_as_float(v.z); sum.w += __uint_as_float(v.w);
+    // slots in order (sender rank, k-part); the KP slots of a rank are loaded
+    // together so their latencies overlap
+    for (int r = 0; r < S; ++r) {
+      uint4 v[KP];
+#pragma unroll
+      for (int p = 0; p < KP; ++p) v[p] = lds128(box + (uint32_t)((((r * KP + p) * L::MP + tl) * cols + c) * 4));
+#pragma unroll
+      for (int p = 0; p < KP; ++p) {
+        sum.x += __uint_as_float(v[p].x); sum.y += __uint_as_float(v[p].y);
+        sum.z += __uint_as_float(v[p].z); sum.w += __uint_as_float(v[p].w);
+      }
     }
     if (bias != nullptr) {
       if (idx != tid) {
