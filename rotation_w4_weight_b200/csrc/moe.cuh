@@ -13,8 +13,9 @@
 // decode GEMV's token tile) and tiles of at most 256 rows (the prefill GEMM's
 // tile), and places every valid slot at offset[e] + (its rank among the
 // earlier slots of e): a stable counting sort, so the order is the slots'
-// order and the result is deterministic.  The gather kernel then copies
-// X_r[token(slot)] into the sorted rows.  A slot whose index lies outside
+// order and the result is deterministic.  X_r[token(slot)] is then copied
+// into the sorted rows: by the route kernel itself when they are few (decode),
+// else by the gather kernel.  A slot whose index lies outside
 // 0..E-1 is flagged in the status word and its output row is written as 0.
 #pragma once
 
@@ -26,6 +27,9 @@ constexpr int kMoeRouteThreads = 1024;
 constexpr int kMoeMaxExperts = kMoeRouteThreads;   // one expert per thread in the scans
 constexpr int kMoeGvRows = 8;                       // rows per decode GEMV segment
 constexpr int kMoeTcRows = 256;                     // rows per prefill GEMM tile
+// Routed rows up to this many bytes are gathered by the route kernel (one CTA
+// copies them in a few microseconds at most), saving the gather launch.
+constexpr size_t kMoeRouteGatherBytes = 256 * 1024;
 
 // Routing results, in the caller's workspace.
 struct MoeHead {
@@ -64,11 +68,14 @@ __device__ __forceinline__ int moe_block_scan(int v, int* warp_sums, int* tot) {
 }
 
 // One CTA of kMoeRouteThreads threads.  idx [S] (S = T * topk slots, slot
-// p = t * topk + j); y [S, N] of the activation type, 16-byte aligned.
+// p = t * topk + j); y [S, N] of the activation type, 16-byte aligned.  With
+// `xg` set, sorted row q of xg [S, K] <- row perm[q] / topk of xr [T, K]
+// (rows of x_chunks 16-byte chunks).
 __global__ void __launch_bounds__(kMoeRouteThreads) moe_route_kernel(const int* __restrict__ idx, int S, int E,
                                                                     MoeHead* head, int* __restrict__ perm,
                                                                     int4* __restrict__ gv, int4* __restrict__ tc,
-                                                                    void* y, int row_bytes) {
+                                                                    void* y, int row_bytes, const uint4* xr,
+                                                                    uint4* xg, int x_chunks, int topk) {
   __shared__ int cnt[kMoeMaxExperts];
   __shared__ int off[kMoeMaxExperts];
   __shared__ int warp_sums[32];
@@ -115,6 +122,15 @@ __global__ void __launch_bounds__(kMoeRouteThreads) moe_route_kernel(const int* 
       if (hit) perm[off[e] + run + __popc(m & ((1u << lane) - 1u))] = p;
       run += __popc(m);
     }
+  }
+  if (xg == nullptr) return;
+  // the gather, for few rows: perm is complete (and visible to the CTA) after
+  // the barrier; X_r was written by the kernel ahead (waited for above)
+  __syncthreads();
+  const int64_t chunks = (int64_t)valid * x_chunks;
+  for (int64_t i = tid; i < chunks; i += blockDim.x) {
+    const int q = (int)(i / x_chunks), c = (int)(i - (int64_t)q * x_chunks);
+    xg[i] = xr[(int64_t)(perm[q] / topk) * x_chunks + c];
   }
 }
 

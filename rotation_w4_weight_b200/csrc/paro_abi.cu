@@ -1418,12 +1418,17 @@ int moe_impl(const void* x, void* y, int64_t T, int64_t K, int64_t N, int E, int
   int4* gv = reinterpret_cast<int4*>(ws + mp.off_gv);
   int4* tc = reinterpret_cast<int4*>(ws + mp.off_tc);
   TA* xg = reinterpret_cast<TA*>(ws + mp.off_xg);
+  // few routed rows (decode): the route kernel gathers them itself
+  const bool route_gathers = (size_t)S * K * 2 <= kMoeRouteGatherBytes;
   if (int st = launch(moe_route_kernel, dim3(1), dim3(kMoeRouteThreads), 0, s, true, expert_idx, (int)S, E, head,
-                      perm, gv, tc, y, (int)(N * 2)))
+                      perm, gv, tc, y, (int)(N * 2), reinterpret_cast<const uint4*>(xr),
+                      route_gathers ? reinterpret_cast<uint4*>(xg) : static_cast<uint4*>(nullptr), (int)(K / 8),
+                      topk))
     return st;
-  if (int st = launch(moe_gather_kernel<TA>, dim3((unsigned)((S + 7) / 8)), dim3(256), 0, s, true,
-                      static_cast<const MoeHead*>(head), static_cast<const int*>(perm), xr, xg, (int)K, topk))
-    return st;
+  if (!route_gathers)
+    if (int st = launch(moe_gather_kernel<TA>, dim3((unsigned)((S + 7) / 8)), dim3(256), 0, s, true,
+                        static_cast<const MoeHead*>(head), static_cast<const int*>(perm), xr, xg, (int)K, topk))
+      return st;
   const int64_t used = std::min<int64_t>(E, S);   // experts that can hold a row
   if (T <= kMoeDecodeMaxT) {
     // segments of at most 8 rows: one token tile of the decode GEMV each
@@ -1472,8 +1477,10 @@ int paro_w4_moe_linear(const void* x, void* y, int64_t T, int64_t K, int64_t N, 
 int paro_w4_moe_launches(int64_t T, int64_t K, int64_t N, int E, int topk, int group_size, int krot,
                          int rotate) {
   if (check_moe_shape(T, K, N, E, topk, group_size) != PARO_OK || T == 0 || krot < 0 || krot > kMaxKrot) return 0;
-  // rotation (two launches above 64 tokens: R' build and X R'), route, gather, expert GEMV or GEMM
-  return (rotate ? (T >= kRotTcMinM ? 2 : 1) : 0) + 3;
+  // rotation (two launches above 64 tokens: R' build and X R'), route, gather
+  // (folded into the route for few rows), expert GEMV or GEMM
+  const bool route_gathers = (size_t)(T * topk) * K * 2 <= kMoeRouteGatherBytes;
+  return (rotate ? (T >= kRotTcMinM ? 2 : 1) : 0) + (route_gathers ? 2 : 3);
 }
 
 }  // extern "C"
