@@ -316,7 +316,11 @@ int paro_w4_linear_group_dt(const void* x, int64_t M, int64_t K, int count, cons
                             int group_size, int dtype, void* workspace, size_t workspace_bytes,
                             paro_stream_t stream);
 /* Kernel launches paro_w4_linear_group issues for this group (rotations plus
- * GEMV/GEMM launches; 0 for an invalid shape or M == 0).  Host-only query. */
+ * GEMV/GEMM launches; 0 for an invalid shape or M == 0).  Host-only query; it
+ * reads the current device's SM count and shared memory (cached per
+ * device): whether decode members share one GEMV launch depends on whether
+ * their grid is resident at once.  Without a device it counts one GEMV launch
+ * per decode member. */
 int paro_w4_linear_group_launches(int64_t M, int64_t K, int count, const paro_linear* linears,
                                   int group_size);
 
@@ -363,7 +367,8 @@ int paro_rotation_matrix_prepare(const float* channel_scales, const int16_t* pai
  *   Shapes as for paro_w4_linear with M = T * topk (< 2^24); E * K < 2^31.
  * The call rotates x once, sorts the T * topk slots by expert on the device
  * (a stable counting sort: deterministic), copies each slot's X_r row into
- * the sorted order, then runs the decode GEMV over segments of at most 8
+ * the sorted order (in the sorting kernel itself when the routed rows take at
+ * most 256 KB), then runs the decode GEMV over segments of at most 8
  * rows of one expert (T <= 16) or the tcgen05 GEMM over tiles of at most 256
  * rows of one expert, each writing its rows straight to their slots.  An
  * expert that no token selects costs nothing.  A slot whose index lies
