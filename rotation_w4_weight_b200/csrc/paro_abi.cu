@@ -466,6 +466,8 @@ LinearPlan make_plan(int64_t M, int64_t K, int64_t N, int gsz) {
     //   square/narrow (q, o, k, v), M <= 8: 128 columns, 4 k-parts, 8 stages, split 4 (8 if N <= 2048)
     //   square, 8 < M <= 16:                64 columns, 4 k-parts, 8 stages, split 2
     //   narrow (N <= 2048), 8 < M <= 16:    128 columns, 2 k-parts, 4 stages, split 8
+    // Grouped wide members (gate + up) at M <= 8 take a 2-stage variant of the
+    // wide plan in group_plan, so the pair fits one wave.
     int tile, want;
     if (N > 4096) {
       tile = 256; p.variant = 0; want = M <= 4 ? 4 : 2;
@@ -969,10 +971,6 @@ size_t gemv_smem(const LinearPlan& p, int gmax) {
 
 int plan_tile(const LinearPlan& p) { return p.variant == 0 || p.variant == 6 ? 256 : (p.variant == 5 ? 64 : 128); }
 
-// One GEMV launch for a group of decode linears sharing x: the plan of the
-// widest member for all of them, taken only when the whole grid is resident
-// at once with that plan's footprint (larger groups gain nothing from sharing
-// a launch: each member already fills the GPU).
 // Whether a decode GEMV grid of `ctas` CTAs with plan p is resident at once
 // (false when the device's limits are unknown).
 bool gemv_one_wave(const LinearPlan& p, int64_t K, int64_t ctas) {
@@ -1008,6 +1006,10 @@ bool wide_one_wave(LinearPlan* p, int64_t K, int64_t units) {
   return false;
 }
 
+// One GEMV launch for a group of decode linears sharing x: the plan of the
+// widest member for all of them, taken only when the whole grid is resident
+// at once with that plan's footprint (larger groups gain nothing from sharing
+// a launch: each member already fills the GPU).
 bool group_plan(int64_t M, int64_t K, const paro_linear* lin, int count, int gsz, LinearPlan* out) {
   int64_t widest = 0;
   for (int i = 0; i < count; ++i) widest = std::max(widest, lin[i].N);
