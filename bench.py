@@ -119,6 +119,40 @@ def load_peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
+# B200 data-sheet figures, for context beside the measured denominators:
+# HBM3e 7.7 TB/s (HGX), dense fp16/bf16 tensor 2.25 PFLOP/s
+SPEC_HBM_GBS = 7700.0
+SPEC_F16_TFLOPS = 2250.0
+
+
+def spec_fields(bound, achieved):
+    spec = SPEC_HBM_GBS if bound == "hbm" else SPEC_F16_TFLOPS
+    return {"peak_spec": spec, "frac_of_spec": round(achieved / spec, 4)}
+
+
+def fp16_matmul_tflops(device, n=8192, iters=10):
+    """torch.matmul (cuBLAS) on fp16 n x n x n, timed with CUDA events on the
+    current stream after warm-up: the dense fp16 rate of this GPU in this run,
+    a reference beside the bf16 denominator (not part of any timed step)."""
+    import torch
+    a = torch.randn(n, n, dtype=torch.float16, device=device)
+    b = torch.randn(n, n, dtype=torch.float16, device=device)
+    c = torch.empty(n, n, dtype=torch.float16, device=device)
+    for _ in range(3):
+        torch.matmul(a, b, out=c)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        torch.matmul(a, b, out=c)
+    e1.record()
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1)
+    del a, b, c
+    return round(2.0 * n ** 3 * iters / (ms * 1e-3) / 1e12, 1)
+
+
 def source_digest():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "rotation_w4_weight_b200", "csrc")
@@ -436,7 +470,8 @@ def run_ours(args, rank, world, local_rank, workload=None):
                 "traffic": traffic_for(workload),
                 "kernel": "w4_gemv_kernel (decode GEMV, split-K cluster)",
                 "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
-                "bytes_per_launch": kern_bytes // n_launch, "peak_source": peaks["src"]}
+                "bytes_per_launch": kern_bytes // n_launch, "peak_source": peaks["src"],
+                **spec_fields("hbm", achieved)}
     else:
         # the GEMM graph runs for many milliseconds under the power cap: the
         # sustained dense peak is its denominator (the burst one is for a kernel timed alone)
@@ -447,7 +482,8 @@ def run_ours(args, rank, world, local_rank, workload=None):
                 "kernel": "w4_tc_gemm_kernel (prefill tcgen05 GEMM)", "avg_launch_us": round(kern_ms * 1e3 / n_launch, 3),
                 "flops_per_launch": kern_flops // n_launch,
                 "peak_source": peaks["src"] + " bf16 sustained (fp16 runs at the bf16 rate)",
-                "peak_burst": peaks["bf16"], "frac_of_burst": round(achieved / peaks["bf16"], 4)}
+                "peak_burst": peaks["bf16"], "frac_of_burst": round(achieved / peaks["bf16"], 4),
+                "fp16_matmul_tflops": fp16_matmul_tflops(dev), **spec_fields("tensor", achieved)}
     del g2
 
     # ---- end to end through the public call with host buffers (pinned), per step:
@@ -625,7 +661,7 @@ def run_quantize(args, rank, world, local_rank):
             "frac": round(achieved / peaks["hbm"], 4), "traffic": traffic_for("quantize_gate_proj"),
             "kernel": "rotate_tc_kernel<__half, true> (weight quantiser on the tensor cores) + R'' build, per call",
             "avg_launch_us": round(ms * 1e3 / args.steps, 3), "bytes_per_launch": per_call,
-            "peak_source": peaks["src"]}
+            "peak_source": peaks["src"], **spec_fields("hbm", achieved)}
 
     # end to end through the public call with host buffers: pinned W in, packed words out
     hW = Ws[0].cpu().pin_memory()
@@ -768,9 +804,9 @@ def run_moe(args, rank, world, local_rank):
         value, unit = job_throughput(world, args.steps, bytes_steps / args.steps, ms) / 1e9, "GB/s"
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm"], 4), "traffic": None,
-                "kernel": "whole call (rotation, routing, gather, expert GEMV segments)",
+                "kernel": "whole call (rotation, routing with the gather of the routed rows, expert GEMV segments)",
                 "avg_launch_us": round(step_s * 1e6, 3), "bytes_per_launch": int(bytes_steps / args.steps),
-                "peak_source": peaks["src"]}
+                "peak_source": peaks["src"], **spec_fields("hbm", achieved)}
     else:
         achieved = flops_per / step_s / 1e12
         value, unit = job_throughput(world, args.steps, flops_per, ms) / 1e12, "TFLOP/s"
@@ -778,7 +814,8 @@ def run_moe(args, rank, world, local_rank):
                 "frac": round(achieved / peaks["bf16_sus"], 4), "traffic": None,
                 "kernel": "whole call (rotation, routing, gather, expert GEMM tiles)",
                 "avg_launch_us": round(step_s * 1e6, 3), "flops_per_launch": flops_per,
-                "peak_source": "measured bf16 sustained (fp16 runs at the bf16 rate)"}
+                "peak_source": "measured bf16 sustained (fp16 runs at the bf16 rate)",
+                **spec_fields("tensor", achieved)}
     return {
         "metric": metric_name(args.workload), "value": round(value, 2), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
