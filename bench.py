@@ -889,6 +889,24 @@ def quantize_oracle_sample(workload, budget_s, max_steps=None):
 
 
 # ----------------------------------------------------------------- CPU oracle (baseline / reference)
+def oracle_threads():
+    """Threads the oracle actually uses: its matmuls run on NumPy's BLAS thread
+    pool, everything else on one thread."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(i["num_threads"]) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline_fields(val, unit, desc):
+    return {"value": round(val, 5), "unit": unit, "cores": oracle_threads(),
+            "host_cores": len(os.sched_getaffinity(0)), "kind": "oracle", "sample": desc}
+
+
 def oracle_sample(workload, budget_s, max_steps=None):
     """Times the float64 oracle on column samples of the workload's calls until
     `budget_s` seconds of CPU work (or max_steps samples) are done.  Returns
@@ -945,7 +963,6 @@ def reference_half(workload, steps, warmup, world):
     """One workload of the reference arm: the oracle on bounded samples."""
     wl = WORKLOADS[workload]
     decode = wl["kind"] in ("decode", "quantize") or (wl["kind"] == "moe" and wl["T"] <= 16)
-    cores = len(os.sched_getaffinity(0))
     per_step_budget = max(0.2, min(2.0, 150.0 / max(1, steps + warmup)))
     oracle_sample(workload, per_step_budget * warmup, max_steps=warmup)
     val, desc, secs = oracle_sample(workload, per_step_budget * steps, max_steps=max(1, steps))
@@ -957,8 +974,7 @@ def reference_half(workload, steps, warmup, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": dict(workload_config(workload, world), timing="host wall clock of the oracle"),
-        "cpu_baseline": {"value": round(val, 5), "unit": unit, "cores": cores, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": cpu_baseline_fields(val, unit, desc),
         "e2e": {"value": round(val, 5), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -1025,14 +1041,10 @@ def main():
         if wl["kind"] == "pair":
             for half, obj in zip(wl["halves"], (out, out["prefill"])):
                 val, desc, _ = oracle_sample(half, args.cpu_budget / 2)
-                obj["cpu_baseline"] = {"value": round(val, 5), "unit": obj["unit"],
-                                       "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-                                       "sample": desc}
+                obj["cpu_baseline"] = cpu_baseline_fields(val, obj["unit"], desc)
         else:
             val, desc, _ = oracle_sample(args.workload, args.cpu_budget)
-            out["cpu_baseline"] = {"value": round(val, 5), "unit": out["unit"],
-                                   "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-                                   "sample": desc}
+            out["cpu_baseline"] = cpu_baseline_fields(val, out["unit"], desc)
         print(json.dumps(out), flush=True)
     if world > 1:
         torch.distributed.barrier()
