@@ -37,3 +37,17 @@ def test_quantiser_bytes():
     K, N = 4096, 14336
     expect = N * K * 2 + (K // 128) * N * 2 + K * N // 2 + (K // 128) * N // 2 + 8 * K * 2 + 8 * (K // 2) * 4 + K * 4
     assert bench.quantize_bytes(K, N) == expect
+
+
+def test_spec_fields_and_cpu_baseline_fields():
+    """Data-sheet context beside the measured denominators, and the CPU
+    baseline's thread counts (the oracle's BLAS threads; the host's cores)."""
+    s = bench.spec_fields("hbm", 3850.0)
+    assert s == {"peak_spec": 7700.0, "frac_of_spec": 0.5}
+    t = bench.spec_fields("tensor", 1125.0)
+    assert t == {"peak_spec": 2250.0, "frac_of_spec": 0.5}
+    c = bench.cpu_baseline_fields(0.0312345678, "GB/s", "sample text")
+    assert c["value"] == 0.03123 and c["unit"] == "GB/s" and c["kind"] == "oracle" and c["sample"] == "sample text"
+    assert 1 <= c["cores"] and 1 <= c["host_cores"]
+    assert c["cores"] == bench.oracle_threads()
+
