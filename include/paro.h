@@ -278,9 +278,10 @@ int paro_w4_linear_dt(const void* x, void* y, int64_t M, int64_t K, int64_t N,
  * and one GEMV launch when the combined grid is resident at once (for wide
  * members, gate and up, on a 2-stage ring with two CTAs per SM), else the
  * shared rotation launch is followed by one GEMV launch per member.  Above 16
- * rows one GEMM launch covers every member's column tiles; above 64 rows the
- * rotating members before it share one R' build (skipped for members with a
- * prepared R') and one X R' launch.  Members whose rotation
+ * rows one GEMM launch covers every member's column tiles.  Before it, above
+ * 64 rows the rotating members share one R' build (skipped for members with a
+ * prepared R') and one X R' launch; from 17 to 64 rows each distinct rotation
+ * is one launch.  Members whose rotation
  * is the same — equal krot and the same channel_scales, pairs and theta
  * pointers (experts that share one rotation) — rotate x once: the first of
  * them computes X_r and the others read it.  Results may differ from the
