@@ -148,6 +148,27 @@ def test_group_call_bf16(M):
         assert lin_ok(to64(y), ref) <= 0
 
 
+def test_group_gate_up_decode_bf16():
+    """Gate/up-shaped members at one token: the one-launch plan on the 2-stage
+    ring with bf16 operands; sampled columns against the oracle."""
+    K, N, M = 4096, 14336, 1
+    lays = [synth.make_layer(n, K, N, seed=60 + i, zero_point=None, bias_std=0.01, n_outliers=41)
+            for i, n in enumerate(["gate", "up"])]
+    devs = [device_layer(l) for l in lays]
+    x_t, x_v = bf(synth.make_activations(lays[0], M).astype(np.float32))
+    members = [dict(qweight=d["qweight"], qzeros=d["qzeros"], scales=d["scales"], bias=d["bias"],
+                    channel_scales=d["cs"], pairs=d["pairs"], theta=d["theta"], krot=l.krot)
+               for l, (d, _, _) in zip(lays, devs)]
+    assert pb.w4_linear_group_launches(M, K, [dict(N=N)] * 2) == 2
+    ys = pb.w4_linear_group(x_t, members, 128)
+    cols = np.sort(np.random.default_rng(7).choice(N, 128, replace=False))
+    for l, (_, s_v, b_v), y in zip(lays, devs, ys):
+        assert y.dtype == torch.bfloat16
+        ref = oracle.w4_linear_columns(x_v, l.codes, l.zero_codes, s_v, b_v, l.channel_scales, l.pairs,
+                                       l.theta, 128, l.krot, cols)
+        assert lin_ok(to64(y)[:, cols], ref) <= 0
+
+
 def test_noalloc_bf16_matches_workspace_call():
     K, N, M = 512, 256, 5
     lay = synth.make_layer("nb", K, N, seed=77, zero_point=None)
